@@ -1,0 +1,490 @@
+"""Decode-attention throughput of JSSA on B200 at 128K context (one layer, Llama-3-8B-shaped).
+
+One step = one ``jssa_decode`` call for the whole batch on one layer: store the new token's K/V
+rows and FP8 scoring code, score every cached token, select the top-B per KV head, run the
+gather-free indexed attention. Default workload: 32 query / 8 KV heads, d 128, 131072-token
+contexts in 16-token pages with a random page permutation, r 32, B 2048, batch 16; synthetic
+low-rank keys/queries from the seeded generator; the basis is calibrated on the GPU from 32768
+seeded samples per KV head.
+
+Prints one JSON line (rank 0). ``--impl reference`` times the float64 CPU oracle instead (the
+only reference that exists for this method) on a bounded sample of the same workload.
+Multi-GPU (``torchrun``): every rank runs its own batch of sequences (weak scaling, no
+collective on the data path); times are the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "JSSA decode-attn steps/s & HBM GB/s at 128K ctx vs dense full-KV, 1×B200"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["jssa", "reference"], default="jssa")
+    ap.add_argument("--batch", type=int, default=16)
+    ap.add_argument("--budget", type=int, default=2048)
+    ap.add_argument("--seq-len", type=int, default=131072)
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense baseline timing")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-check", action="store_true", help="skip the sampled oracle check")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks
+# ------------------------------------------------------------------------------------------------
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as fh:
+            for line in fh:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) < 9:
+                    continue
+                try:
+                    sm.append(float(p[1]))
+                    smax.append(float(p[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, p[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------------
+# workload
+# ------------------------------------------------------------------------------------------------
+
+
+def workload(args, rank):
+    from synth import WORKLOADS
+    w = WORKLOADS["llama128k"].replace(batch=args.batch, budget=args.budget, seq_len=args.seq_len)
+    return w.replace(seed=w.seed + 7919 * rank)
+
+
+def setup_gpu(w, dev):
+    import torch
+    import token_level_sparse_fp8_b200 as J
+    from synth import build_paged_kv, layer_factors, sample_calibration, sample_decode_queries
+
+    f = layer_factors(w.seed, 0, w.h_kv, w.d)
+    qc, kc = sample_calibration(f, w.calib_samples, w.group, w.seed, device=dev)
+    cal = J.calibrate(qc, kc, w.rank)
+    del qc, kc
+    kv = build_paged_kv(f, [w.seq_len] * w.batch, w.page_size, w.seed, device=dev)
+    layer = J.PagedLayer(kv["k_cache"], kv["v_cache"], kv["block_table"], kv["seq_lens"], cal["M"],
+                         w.budget)
+    layer.prefill_scores()
+    n_q = 8  # distinct query sets, rotated over the steps
+    qs = [sample_decode_queries(f, w.batch, w.group, w.seed, step=i, device=dev) for i in range(n_q)]
+    # the new token of each step is the last cached position (rewriting it is idempotent)
+    t = w.seq_len - 1
+    bt = kv["block_table"].long()
+    page = bt[:, t // w.page_size]
+    k_new = kv["k_cache"][page, t % w.page_size].contiguous()
+    v_new = kv["v_cache"][page, t % w.page_size].contiguous()
+    torch.cuda.synchronize(dev)
+    return {"layer": layer, "qs": qs, "k_new": k_new, "v_new": v_new, "kv": kv, "factors": f,
+            "cal": cal}
+
+
+def timed(fn, steps, warmup, stream, barrier):
+    """Device time of `steps` calls of fn (CUDA events on `stream`), after `warmup` calls."""
+    import torch
+    for i in range(warmup):
+        fn(i)
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        fn(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    return e0.elapsed_time(e1) / 1e3
+
+
+def algorithmic_bytes(w, dense=False):
+    pages = -(-w.seq_len // w.page_size)
+    if dense:
+        return w.batch * (w.h_kv * w.seq_len * 2 * w.d * 2 + 4 * pages)
+    return w.batch * (w.h_kv * w.seq_len * w.rank + w.h_kv * min(w.budget, w.seq_len) * 2 * w.d * 2
+                      + 4 * pages)
+
+
+def score_bytes(w):
+    pages = -(-w.seq_len // w.page_size)
+    return w.batch * (w.h_kv * w.seq_len * w.rank + 4 * pages)
+
+
+def attend_bytes(w):
+    return w.batch * w.h_kv * min(w.budget, w.seq_len) * 2 * w.d * 2
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle baseline
+# ------------------------------------------------------------------------------------------------
+
+
+def oracle_pair_inputs(state, w, b, h):
+    """Host copies of what the oracle needs for one (sequence, KV head): that sequence's pages of
+    the caches (one head) with an identity page table."""
+    import numpy as np
+    import torch
+    layer = state["layer"]
+    bt = state["kv"]["block_table"][b].long()
+    k = layer.k_cache[bt][:, :, h : h + 1].to(torch.float64).cpu().numpy()
+    v = layer.v_cache[bt][:, :, h : h + 1].to(torch.float64).cpu().numpy()
+    sc = layer.score_cache[bt][:, h : h + 1].cpu().numpy()
+    m = layer.basis[h : h + 1].double().cpu().numpy()
+    return k, v, sc, m, np.arange(bt.numel(), dtype=np.int64)[None]
+
+
+def oracle_step_for_pair(q_b, k, v, sc, m, bt, w):
+    """The oracle's select + attend for one (sequence, KV head); q_b is [G, d] of that head."""
+    import numpy as np
+    from oracle import jssa as O
+    lens = np.array([w.seq_len])
+    idx, count, s = O.select_step(q_b[None], m, sc, bt, lens, w.budget)
+    out = O.indexed_attend_step(q_b[None], k, v, bt, idx, count, 1.0 / math.sqrt(w.d))
+    return idx, count, s, out
+
+
+def cpu_baseline(state, w, seconds):
+    """The oracle, as it stands, on host cores: select + attend for (sequence, KV head) pairs of
+    the timed workload, repeated until about `seconds` of CPU time; scaled to one whole step."""
+    import torch
+    cores = len(os.sched_getaffinity(0))
+    q = state["qs"][0].to(torch.float64).cpu().numpy()
+    g = w.group
+    pairs = [(0, 0), (w.batch - 1, w.h_kv - 1)]
+    inputs = [(q[b, h * g : (h + 1) * g],) + oracle_pair_inputs(state, w, b, h) for b, h in pairs]
+    done, t_total = 0, 0.0
+    while t_total < seconds or done < 2:
+        qb, k, v, sc, m, bt = inputs[done % len(inputs)]
+        t0 = time.perf_counter()
+        oracle_step_for_pair(qb, k, v, sc, m, bt, w)
+        t_total += time.perf_counter() - t0
+        done += 1
+    per_pair = t_total / done
+    steps_per_s = 1.0 / (per_pair * w.batch * w.h_kv)
+    return {"value": steps_per_s, "unit": "steps/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done} oracle calls on 2 (sequence, KV head) pairs of the timed workload "
+                      f"(score+top-B+attend over 131072 tokens, float64 NumPy), {t_total:.1f} s; "
+                      f"steps/s = 1 / (time per pair x {w.batch * w.h_kv} pairs per step)"}
+
+
+def sampled_check(state, w, n_pairs=2):
+    """Oracle agreement on a few (sequence, KV head) pairs of the timed configuration."""
+    import numpy as np
+    import torch
+    layer = state["layer"]
+    q = state["qs"][0]
+    out, idx, count = layer.step(q, state["k_new"], state["v_new"])
+    torch.cuda.synchronize()
+    qn = q.to(torch.float64).cpu().numpy()
+    rng = np.random.default_rng(0)
+    res = []
+    for _ in range(n_pairs):
+        b, h = int(rng.integers(w.batch)), int(rng.integers(w.h_kv))
+        k, v, sc, m, bt = oracle_pair_inputs(state, w, b, h)
+        g = w.group
+        ridx, rcount, s, rout = oracle_step_for_pair(qn[b, h * g : (h + 1) * g], k, v, sc, m, bt, w)
+        gi = idx[b, h].cpu().numpy()
+        sym = np.setxor1d(gi[: int(count[b, h])], ridx[0, 0, : rcount[0, 0]])
+        s = s[(0, 0)]
+        kth = np.sort(s)[::-1][w.budget - 1]
+        ties_ok = bool(np.all(np.abs(s[sym] - kth) <= 1e-4 * np.abs(s).max()))
+        go = out[b, h * g : (h + 1) * g].double().cpu().numpy()
+        err = np.abs(go - rout[0])
+        res.append({"pair": [b, h], "swaps": int(sym.size // 2), "ties_ok": ties_ok,
+                    "max_abs": float(err.max()), "mean_rel": float(err.sum() / np.abs(rout[0]).sum())})
+    ok = all(r["ties_ok"] and r["max_abs"] <= 1e-2 and r["mean_rel"] <= 2e-3 for r in res)
+    return {"ok": ok, "pairs": res}
+
+
+# ------------------------------------------------------------------------------------------------
+# arms
+# ------------------------------------------------------------------------------------------------
+
+
+def run_reference(args):
+    """CPU oracle arm: rank 0 only, bounded sample of the same workload."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+    from oracle import jssa as O
+    from synth import build_paged_kv, layer_factors, sample_decode_queries
+    w = workload(args, 0)
+    cores = len(os.sched_getaffinity(0))
+    f = layer_factors(w.seed, 0, w.h_kv, w.d)
+    # one sequence of the workload, built on the host; the oracle scores one KV head per call
+    kv = build_paged_kv(f, [w.seq_len], w.page_size, w.seed, chunk_pages=1024)
+    q = sample_decode_queries(f, 1, w.group, w.seed).double().numpy()
+    rng = np.random.default_rng(0)
+    m = np.linalg.qr(rng.standard_normal((w.d, w.rank)))[0].T[None]  # an orthonormal basis
+    h = 0
+    k = kv["k_cache"][:, :, h : h + 1].double().numpy()
+    v = kv["v_cache"][:, :, h : h + 1].double().numpy()
+    sc = np.zeros((k.shape[0], 1, w.page_size, w.rank), dtype=np.uint8)
+    sc[:, 0] = O.store_codes(k[:, :, 0].reshape(-1, w.d), m[0]).reshape(k.shape[0], w.page_size, w.rank)
+    bt = kv["block_table"].numpy().astype(np.int64)
+    qb = q[0, 0 : w.group]
+    pairs_per_step = w.batch * w.h_kv
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        oracle_step_for_pair(qb, k, v, sc, m, bt, w)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    per_pair = statistics.mean(times)
+    value = 1.0 / (per_pair * pairs_per_step)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per_pair * pairs_per_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"llama3-8b-layer-128k (h_q {w.h_q}, h_kv {w.h_kv}, d {w.d}, L {w.seq_len}, "
+                               f"ps {w.page_size}, r {w.rank}, B {w.budget}, batch {w.batch})",
+                   "global_batch": w.batch, "seq_len": w.seq_len, "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "steps/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: one (sequence, KV head) pair of the workload "
+                                   f"(score+top-B+attend in float64 NumPy), scaled by "
+                                   f"{pairs_per_step} pairs per step"},
+        "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_jssa(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import token_level_sparse_fp8_b200 as J
+
+    rank, world, local = dist_env()
+    assert torch.cuda.is_available(), "bench needs a CUDA device"
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    w = workload(args, rank)
+    J._lib.load()
+    state = setup_gpu(w, dev)
+    layer = state["layer"]
+    qs, k_new, v_new = state["qs"], state["k_new"], state["v_new"]
+    stream = torch.cuda.current_stream(dev)
+    out = torch.empty_like(qs[0])
+    nq = len(qs)
+
+    def step(i):
+        layer.step(qs[i % nq], k_new, v_new, out)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    t_step = max_over_ranks(timed(step, args.steps, args.warmup, stream, barrier))
+    clocks = sampler.stop()
+    launches_per_step = 3
+
+    # per-kernel device times (same configuration, each kernel launched alone)
+    idx, count = layer.idx, layer.count
+
+    def score_only(i):
+        J.score_topk(qs[i % nq], layer.basis, layer.score_cache, layer.block_table, layer.seq_lens,
+                     w.budget, idx, count)
+
+    def attend_only(i):
+        J.indexed_attend(qs[i % nq], layer.k_cache, layer.v_cache, layer.block_table, idx, count,
+                         layer.scale, out, layer.ws)
+
+    t_score = max_over_ranks(timed(score_only, args.steps, args.warmup, stream, barrier))
+    t_attend = max_over_ranks(timed(attend_only, args.steps, args.warmup, stream, barrier))
+
+    t_dense = None
+    if not args.no_dense:
+        dense_steps = max(3, args.steps // 4)
+        t_dense = max_over_ranks(timed(lambda i: layer.dense(qs[i % nq], out), dense_steps,
+                                       max(3, args.warmup // 2), stream, barrier)) / dense_steps
+
+    # end to end through the public API with host buffers: H2D of the step's inputs, D2H of out
+    q_host = [q.cpu().pin_memory() for q in qs]
+    kn_host, vn_host = k_new.cpu().pin_memory(), v_new.cpu().pin_memory()
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    q_dev, kn_dev, vn_dev = torch.empty_like(qs[0]), torch.empty_like(k_new), torch.empty_like(v_new)
+
+    def e2e_step(i):
+        q_dev.copy_(q_host[i % nq], non_blocking=True)
+        kn_dev.copy_(kn_host, non_blocking=True)
+        vn_dev.copy_(vn_host, non_blocking=True)
+        layer.step(q_dev, kn_dev, vn_dev, out)
+        out_host.copy_(out, non_blocking=True)
+
+    t_e2e = max_over_ranks(timed(e2e_step, args.steps, args.warmup, stream, barrier))
+    h2d = qs[0].numel() * 2 + k_new.numel() * 2 + v_new.numel() * 2
+    d2h = out.numel() * 2
+
+    check = None
+    if rank == 0 and not args.no_check:
+        check = sampled_check(state, w)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(state, w, args.cpu_seconds)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peak, peak_kind = peaks()
+    ms_step = t_step / args.steps * 1e3
+    steps_per_s = world * args.steps / t_step
+    bytes_step = algorithmic_bytes(w)
+    score_launch_s = t_score / args.steps
+    achieved = score_bytes(w) / score_launch_s / 1e9
+    line = {
+        "metric": METRIC,
+        "value": steps_per_s,
+        "unit": "steps/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16 K/V, e4m3 scoring cache, fp32 math",
+        "data": "synthetic",
+        "config": {
+            "workload": f"llama3-8b-layer-128k: h_q {w.h_q}, h_kv {w.h_kv}, d {w.d}, L {w.seq_len}, "
+                        f"page {w.page_size} (permuted), r {w.rank}, B {w.budget}, batch {w.batch} per GPU",
+            "global_batch": w.batch * world,
+            "seq_len": w.seq_len,
+            "budget": w.budget,
+            "parallelism": f"dp{world} (independent sequences per GPU)",
+            "l2": "inputs larger than L2: the 512 MiB scoring cache is streamed every step; 8 query sets rotate",
+        },
+        "hbm_gbs": bytes_step / (ms_step / 1e3) / 1e9,
+        "roofline_step": {"bound": "hbm", "achieved": bytes_step / (ms_step / 1e3) / 1e9, "peak": peak,
+                          "unit": "GB/s", "frac": bytes_step / (ms_step / 1e3) / 1e9 / peak,
+                          "traffic": None, "bytes_per_step": bytes_step, "peak_kind": peak_kind},
+        "roofline": {"bound": "hbm", "kernel": "score_topk", "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "bytes_per_launch": score_bytes(w), "ms_per_launch": score_launch_s * 1e3,
+                     "peak_kind": peak_kind},
+        "kernels_ms": {"score_topk": score_launch_s * 1e3, "indexed_attend": t_attend / args.steps * 1e3,
+                       "attend_gbs": attend_bytes(w) / (t_attend / args.steps) / 1e9},
+        "clocks": clocks,
+        "e2e": {"value": world * args.steps / t_e2e, "unit": "steps/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    if t_dense is not None:
+        dense_bytes = algorithmic_bytes(w, dense=True)
+        line["dense"] = {"steps_per_s": world / t_dense, "ms_per_step": t_dense * 1e3,
+                         "hbm_gbs": dense_bytes / t_dense / 1e9, "frac": dense_bytes / t_dense / 1e9 / peak}
+        line["speedup_vs_dense"] = t_dense / (ms_step / 1e3)
+    if check is not None:
+        line["oracle_check"] = check
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_jssa(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,215 @@
+/*
+ * jssa.h - C ABI of libjssa.so: Joint Subspace Sparse Attention (JSSA) decode and calibration
+ * on NVIDIA B200 (sm_100a).
+ *
+ * Method (JSSA summary, picx.dev, "Theoretical Foundation" and "Methodology" sections 3.1-3.4;
+ * JSSA README, "Paper-to-code map" and section 4): per layer and KV head an orthonormal basis
+ * M (r x d) is calibrated once as the top-r eigenvectors of the sum of the unit-trace second
+ * moments of group-mean queries and of keys (eq. (5)). At each decode step the new key's
+ * projection M k is stored as FP8 E4M3 in a scoring cache (section 3.4), every cached token is
+ * scored with the projected group-mean query (eq. (1), section 3.1 step 2), the top-B tokens are
+ * selected independently per KV head, and attention of every query head runs over its KV head's
+ * selected rows, read in place from the paged KV cache (section 3.3).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers are DEVICE pointers owned by the caller, except where stated. The library never
+ *   allocates or frees memory and never synchronises a stream (jssa_device_error excepted).
+ *   Every call is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy default).
+ * - bf16 tensors are passed as `const jssa_bf16*` (raw 16-bit storage).
+ * - Return value: JSSA_OK (0); a negative JSSA_ERR_* code when the host-side argument check
+ *   fails, in which case nothing was launched; or a positive cudaError_t from the launch.
+ * - Head mapping: query head i belongs to KV head i / G with G = h_q / h_kv.
+ * - Paged KV cache: element (page, slot, head, x) of the K (or V) cache is at
+ *   cache[page*kv_page_stride + slot*kv_slot_stride + head*kv_head_stride + x]; strides are in
+ *   elements, the head dimension is contiguous. Logical position t of sequence b lives in page
+ *   block_table[b*max_pages + t/page_size], slot t%page_size. block_table is int32
+ *   [batch, max_pages], seq_lens int32 [batch].
+ * - Scoring cache: uint8 E4M3 codes laid out [num_pages, h_kv, page_size, r] (one contiguous
+ *   run of page_size*r bytes per page and KV head), same page numbering as the KV cache.
+ * - Basis: float32 [h_kv, r, d], rows orthonormal (output of jssa_compute_basis).
+ * - Index sets: int32 idx [batch, h_kv, budget] holds logical positions in ascending order,
+ *   padded with -1; int32 count [batch, h_kv] = min(budget, seq_len).
+ * - Device-side checks: a page number outside [0, num_pages), a position outside the block
+ *   table, or a seq_len above max_pages*page_size is never dereferenced: the row is skipped and
+ *   a flag is raised in the library's device error word (jssa_device_error). Kernels never trap.
+ * - Supported template shapes: d = 128 with r in {32, 64}; G <= 8 for attention.
+ */
+#ifndef JSSA_H_
+#define JSSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define JSSA_API __attribute__((visibility("default")))
+#else
+#define JSSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t jssa_bf16;   /* bfloat16 storage */
+typedef void* jssa_stream_t;  /* cudaStream_t */
+
+enum jssa_status {
+  JSSA_OK = 0,
+  JSSA_ERR_NULL = -1,         /* a required pointer is NULL */
+  JSSA_ERR_SHAPE = -2,        /* inconsistent or out-of-range sizes */
+  JSSA_ERR_UNSUPPORTED = -3,  /* no kernel instance for (d, r, G) or size beyond the limits */
+  JSSA_ERR_ALIGN = -4,        /* a pointer or stride breaks the 16-byte alignment rule */
+  JSSA_ERR_WORKSPACE = -5,    /* workspace NULL or smaller than jssa_workspace_size */
+  JSSA_ERR_DEVICE = -6        /* no usable CUDA device / device query failed */
+};
+
+/* Device error flags (bitwise OR), read with jssa_device_error. */
+enum jssa_device_flag {
+  JSSA_DEVERR_PAGE = 1,       /* block_table or slot_mapping named a page outside [0, num_pages) */
+  JSSA_DEVERR_INDEX = 2,      /* an index-set entry outside [0, max_pages*page_size) */
+  JSSA_DEVERR_SEQLEN = 4,     /* seq_len < 0 or > max_pages*page_size (clamped) */
+  JSSA_DEVERR_SELECT = 8      /* internal: inconsistent top-B counts (never expected) */
+};
+
+/* Workspace clients for jssa_workspace_size. */
+enum jssa_fn {
+  JSSA_FN_SCORE_TOPK = 1,
+  JSSA_FN_INDEXED_ATTEND = 2,
+  JSSA_FN_DENSE_DECODE = 3,
+  JSSA_FN_DECODE = 4,
+  JSSA_FN_COMPUTE_BASIS = 5
+};
+
+/* Text for a status code (static storage). */
+JSSA_API const char* jssa_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+JSSA_API int jssa_version(void);
+
+/*
+ * Bytes of device workspace the entry point `fn` needs for these sizes (written to *bytes; 0
+ * means none). max_seq_len bounds every seq_len (use max_pages*page_size); budget is ignored
+ * by the dense decode and by the basis. The split-K attention entry points keep a per-(sequence,
+ * KV head) ticket counter in the workspace: a workspace must be cleared once with
+ * jssa_workspace_init before its first use; the kernels leave the counters at zero on exit.
+ * Calls that share one workspace must not overlap on the GPU.
+ */
+JSSA_API int jssa_workspace_size(int fn, int batch, int h_q, int h_kv, int d, int max_seq_len, int budget,
+                        size_t* bytes);
+
+/* Zero `ws_bytes` bytes of workspace on `stream` (cudaMemsetAsync). */
+JSSA_API int jssa_workspace_init(void* ws, size_t ws_bytes, jssa_stream_t stream);
+
+/*
+ * Calibration, step 1: accumulate uncentred second moments of group-mean queries and of keys.
+ * JSSA summary, Theoretical Foundation (the second-moment matrices of eq. (3)) and section 3.2;
+ * JSSA README, section 2 (second moments of post-RoPE queries and keys).
+ *   gram_q[h] += sum_n qbar_n qbar_n^T,  qbar_n = (1/G) sum_g q[n, h*G+g, :]
+ *   gram_k[h] += sum_n k_n k_n^T,        k_n = k[n, h, :]
+ * q: bf16 [n, h_q, d], row n at q + n*q_stride_n (elements, >= h_q*d, multiple of 8).
+ * k: bf16 [n, h_kv, d], row n at k + n*k_stride_n (elements, >= h_kv*d, multiple of 8).
+ * gram_q, gram_k: float64 [h_kv, d, d], accumulated in place (zero them before the first call).
+ * Products of the exact bf16 inputs are summed in fp32 on tensor cores within a tile of samples
+ * and added to the float64 totals. n may be 0 (no-op).
+ */
+JSSA_API int jssa_calibrate_accumulate(const jssa_bf16* q, int64_t q_stride_n, const jssa_bf16* k,
+                              int64_t k_stride_n, int n, int h_q, int h_kv, int d,
+                              double* gram_q, double* gram_k, jssa_stream_t stream);
+
+/*
+ * Calibration, step 2: M = TopEig_r(gram_q/tr(gram_q) + gram_k/tr(gram_k))^T per KV head.
+ * JSSA summary, eq. (5); JSSA README, paper-to-code map (compute_basis) and section 2 (one
+ * eigendecomposition per layer and KV head). Cyclic Jacobi in float64 on the device.
+ * basis: float32 [h_kv, r, d], rows = eigenvectors of the r largest eigenvalues, descending,
+ * each signed so that its largest-magnitude entry is positive (lowest index on ties).
+ * eigvals: float64 [h_kv, d] descending, or NULL. ws: >= jssa_workspace_size(JSSA_FN_COMPUTE_BASIS).
+ */
+JSSA_API int jssa_compute_basis(const double* gram_q, const double* gram_k, int h_kv, int d, int r,
+                       float* basis, double* eigvals, void* ws, size_t ws_bytes,
+                       jssa_stream_t stream);
+
+/*
+ * Store step: scoring code c = e4m3(M_h k) of each given token and KV head.
+ * JSSA summary, section 3.4 (K_proj = K M^T kept as an FP8 scoring-only cache); JSSA README,
+ * section 4 notes (r bytes per token and KV head). The projection is summed in float64 and
+ * rounded once to E4M3 (round to nearest even, saturating to +-448, no scale).
+ * k: bf16 [t, h_kv, d] with row stride k_stride_t elements. slot_mapping: int64 [t], flat slot
+ * page*page_size + offset, negative = skip. score_cache: see conventions.
+ */
+JSSA_API int jssa_store(const jssa_bf16* k, int64_t k_stride_t, const int64_t* slot_mapping, int t,
+               int h_kv, int d, int r, const float* basis, uint8_t* score_cache,
+               int64_t num_pages, int page_size, jssa_stream_t stream);
+
+/*
+ * Score + top-B: for every sequence b and KV head h, p = M_h qbar (qbar the mean of the G query
+ * heads of h), s_t = sum_j dec(c_tj) p_j for every t < seq_len (fp32), and the index set of the
+ * min(budget, seq_len) largest s_t, ties to the lower position, written ascending.
+ * JSSA summary, eq. (1) and section 3.1 steps 1-2; JSSA README, section 4 (jssa_budget).
+ * One thread-block cluster per (sequence, KV head) keeps all scores in shared memory and runs a
+ * radix select over the cluster; nothing but idx/count is written to memory.
+ * q: bf16 [batch, h_q, d] contiguous. ws may be NULL (size 0).
+ */
+JSSA_API int jssa_score_topk(const jssa_bf16* q, const float* basis, const uint8_t* score_cache,
+                    const int32_t* block_table, int max_pages, const int32_t* seq_lens, int batch,
+                    int h_q, int h_kv, int d, int r, int64_t num_pages, int page_size, int budget,
+                    int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
+                    jssa_stream_t stream);
+
+/*
+ * Gather-free indexed attention: out[b, i] = softmax(scale * q_i K_S^T) V_S over the positions
+ * S = idx[b, i/G, 0:count[b, i/G]], with K and V rows read in place from the paged cache (no
+ * staging buffer), split-K over S and an online-softmax merge (last CTA of each (b, h) merges).
+ * JSSA summary, section 3.1 step 3 and section 3.3; JSSA README, paper-to-code map.
+ * q, out: bf16 [batch, h_q, d] contiguous. count = 0 gives a zero output row.
+ */
+JSSA_API int jssa_indexed_attend(const jssa_bf16* q, const jssa_bf16* k_cache, const jssa_bf16* v_cache,
+                        int64_t kv_page_stride, int64_t kv_slot_stride, int64_t kv_head_stride,
+                        const int32_t* block_table, int max_pages, const int32_t* idx,
+                        const int32_t* count, int batch, int h_q, int h_kv, int d, int budget,
+                        int64_t num_pages, int page_size, float softmax_scale, jssa_bf16* out,
+                        void* ws, size_t ws_bytes, jssa_stream_t stream);
+
+/*
+ * Dense paged decode attention (the full-KV baseline): out[b, i] = attention of q_i over every
+ * position [lo, seq_len) with lo = max(0, seq_len - window) when window > 0, else 0.
+ * JSSA README, section 3 (attention microbenchmark against full-KV decode) and section 4 notes
+ * (sliding-window layers keep dense attention). Same kernel body as jssa_indexed_attend.
+ */
+JSSA_API int jssa_dense_decode(const jssa_bf16* q, const jssa_bf16* k_cache, const jssa_bf16* v_cache,
+                      int64_t kv_page_stride, int64_t kv_slot_stride, int64_t kv_head_stride,
+                      const int32_t* block_table, int max_pages, const int32_t* seq_lens,
+                      int batch, int h_q, int h_kv, int d, int64_t num_pages, int page_size,
+                      int window, float softmax_scale, jssa_bf16* out, void* ws,
+                      size_t ws_bytes, jssa_stream_t stream);
+
+/*
+ * One whole decode step for one layer: (1) when k_new and v_new are non-NULL, write the new
+ * token (position seq_len-1 of each sequence) into the K and V caches and its scoring code into
+ * the scoring cache; (2) score + top-B; (3) gather-free indexed attention. The three kernels
+ * are chained on `stream` with programmatic dependent launch and no host synchronisation.
+ * JSSA summary, section 3.1; JSSA README, paper-to-code map (_sparse_decode_forward).
+ * k_new, v_new: bf16 [batch, h_kv, d] contiguous (or both NULL). idx/count: outputs as in
+ * jssa_score_topk. ws: >= jssa_workspace_size(JSSA_FN_DECODE), cleared once by
+ * jssa_workspace_init.
+ */
+JSSA_API int jssa_decode(const jssa_bf16* q, const jssa_bf16* k_new, const jssa_bf16* v_new,
+                jssa_bf16* k_cache, jssa_bf16* v_cache, int64_t kv_page_stride,
+                int64_t kv_slot_stride, int64_t kv_head_stride, uint8_t* score_cache,
+                const float* basis, const int32_t* block_table, int max_pages,
+                const int32_t* seq_lens, int batch, int h_q, int h_kv, int d, int r,
+                int64_t num_pages, int page_size, int budget, float softmax_scale,
+                int32_t* idx, int32_t* count, jssa_bf16* out, void* ws, size_t ws_bytes,
+                jssa_stream_t stream);
+
+/*
+ * Read (and with clear != 0, reset) the device error word of the current device. Synchronises
+ * `stream` first so that the flags of every kernel enqueued on it are visible.
+ */
+JSSA_API int jssa_device_error(uint32_t* flags, int clear, jssa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JSSA_H_ */

@@ -300,6 +300,9 @@ def decode_step(q: np.ndarray, k_new, v_new, k_cache: np.ndarray, v_cache: np.nd
         slots = np.empty(batch, dtype=np.int64)
         for b in range(batch):
             t = int(seq_lens[b]) - 1
+            if t < 0:                      # an empty sequence has no position to store into
+                slots[b] = -1
+                continue
             page = block_table[b, t // ps]
             k_cache[page, t % ps] = k_new[b]
             v_cache[page, t % ps] = v_new[b]

@@ -1,0 +1,92 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point the header declares, and
+its host-side argument checks reject bad calls before anything is launched."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "jssa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from token_level_sparse_fp8_b200 import build, _lib
+    build.build()
+    return _lib.load()
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"JSSA_API\s+[\w\s\*]+?\b(jssa_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared()
+    for n in ["jssa_calibrate_accumulate", "jssa_compute_basis", "jssa_store", "jssa_score_topk",
+              "jssa_indexed_attend", "jssa_decode", "jssa_dense_decode"]:
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from token_level_sparse_fp8_b200 import _lib
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (jssa_\w+)", out))
+    assert set(_declared()) <= exported
+    assert set(_declared()) == set(_lib.SIGNATURES)
+    for n in _declared():
+        assert hasattr(lib, n)
+
+
+def test_built_for_sm100a():
+    from token_level_sparse_fp8_b200 import _lib
+    out = subprocess.run(["cuobjdump", "--list-elf", _lib.LIB_PATH], capture_output=True, text=True)
+    if out.returncode != 0:
+        pytest.skip("cuobjdump unavailable")
+    assert "sm_100a" in out.stdout
+
+
+def test_status_strings_and_version(lib):
+    from token_level_sparse_fp8_b200 import _lib
+    assert lib.jssa_version() >= 100
+    assert _lib.status_string(0) == "ok"
+    for code in range(-6, 0):
+        assert _lib.status_string(code) != "unknown status"
+
+
+def test_workspace_sizes_are_host_only(lib):
+    from token_level_sparse_fp8_b200 import api, _lib
+    assert api.workspace_size(_lib.FN_COMPUTE_BASIS, 0, 1, 8, 128, 0, 0) == 8 * 128 * 128 * 8
+    n = api.workspace_size(_lib.FN_DECODE, 16, 32, 8, 128, 131072, 2048)
+    assert n > 0
+    assert api.workspace_size(_lib.FN_DENSE_DECODE, 16, 32, 8, 128, 131072, 0) > n
+    with pytest.raises(_lib.JSSAError):
+        api.workspace_size(_lib.FN_DECODE, 1, 30, 8, 128, 1024, 64)  # h_q not a multiple of h_kv
+
+
+def test_argument_checks_reject_before_launch(lib):
+    from token_level_sparse_fp8_b200 import _lib
+    # NULL inputs, unsupported shapes and bad alignment are refused on the host
+    st = lib.jssa_score_topk(None, None, None, None, 16, None, 1, 8, 2, 128, 32, 10, 16, 128,
+                             None, None, None, 0, None)
+    assert st == -1
+    st = lib.jssa_score_topk(None, None, None, None, 16, None, 1, 8, 2, 96, 32, 10, 16, 128,
+                             None, None, None, 0, None)
+    assert st == -3  # no d = 96 instance
+    st = lib.jssa_score_topk(None, None, None, None, 16, None, 1, 8, 3, 128, 32, 10, 16, 128,
+                             None, None, None, 0, None)
+    assert st == -2  # 8 query heads over 3 KV heads
+    st = lib.jssa_store(8, 1024, 32, 1, 2, 128, 32, 48, 32, 10, 16, None)
+    assert st == -4  # misaligned key pointer
+    st = lib.jssa_indexed_attend(16, 16, 16, 4096, 256, 128, 16, 8, 16, 16, 1, 64, 2, 128, 128,
+                                 10, 16, ctypes.c_float(0.1), 16, None, 0, None)
+    assert st == -3  # G = 32 query heads per KV head is beyond the m16 tile
+    st = lib.jssa_decode(None, None, None, None, None, 0, 0, 0, None, None, None, 1, None, 0, 8, 2,
+                         128, 32, 1, 16, 128, ctypes.c_float(0.1), None, None, None, None, 0, None)
+    assert st == 0  # batch 0 is a no-op
+    st = lib.jssa_compute_basis(16, 16, 2, 128, 32, 16, None, 16, 100, None)
+    assert st == -5  # workspace too small

@@ -1,0 +1,327 @@
+"""Thin PyTorch binding of libjssa.so.
+
+Argument marshalling only: every step of the method runs in the library's CUDA kernels. PyTorch
+provides device memory (outputs and workspaces are allocated here with torch) and the current
+CUDA stream. There is no CPU path: the functions raise if a tensor is not on a CUDA device or if
+the library is missing.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+from typing import Optional, Tuple
+
+import torch
+
+from . import _lib
+from ._lib import (FN_COMPUTE_BASIS, FN_DECODE, FN_DENSE_DECODE, FN_INDEXED_ATTEND, JSSAError,
+                   call)
+
+__all__ = [
+    "JSSAError", "workspace_size", "Workspace", "calibrate_accumulate", "compute_basis",
+    "calibrate", "store", "score_topk", "indexed_attend", "dense_decode", "decode",
+    "device_error", "kv_strides", "default_rank", "PagedLayer",
+]
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, contiguous: bool = True):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device (there is no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def default_rank(head_dim: int) -> int:
+    """Default subspace rank, head_dim // 4 (JSSA README, section 4: jssa_rank default)."""
+    return head_dim // 4
+
+
+def kv_strides(cache: torch.Tensor) -> Tuple[int, int, int]:
+    """(page, slot, head) element strides of a ``[num_pages, page_size, h_kv, d]`` cache view."""
+    if cache.dim() != 4 or cache.stride(3) != 1:
+        raise ValueError("KV cache must be [num_pages, page_size, h_kv, d] with a contiguous last dim")
+    return cache.stride(0), cache.stride(1), cache.stride(2)
+
+
+def workspace_size(fn: int, batch: int, h_q: int, h_kv: int, d: int, max_seq_len: int,
+                   budget: int) -> int:
+    out = ctypes.c_size_t(0)
+    call("jssa_workspace_size", fn, batch, h_q, h_kv, d, max_seq_len, budget, ctypes.byref(out))
+    return int(out.value)
+
+
+class Workspace:
+    """A zero-initialised device workspace that grows on demand (one per stream of use)."""
+
+    def __init__(self, device=None):
+        self.device = torch.device(device or "cuda")
+        self.buf = None
+
+    def get(self, nbytes: int) -> Tuple[Optional[int], int]:
+        if nbytes == 0:
+            return None, 0
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+            call("jssa_workspace_init", self.buf.data_ptr(), self.buf.numel(), _stream(self.device))
+        return self.buf.data_ptr(), self.buf.numel()
+
+
+_default_ws = {}
+
+
+def _ws(device: torch.device, ws: Optional[Workspace]) -> Workspace:
+    if ws is not None:
+        return ws
+    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    if key not in _default_ws:
+        _default_ws[key] = Workspace(device)
+    return _default_ws[key]
+
+
+# ------------------------------------------------------------------------------------------------
+# Calibration
+# ------------------------------------------------------------------------------------------------
+
+
+def calibrate_accumulate(q: torch.Tensor, k: torch.Tensor, gram_q: torch.Tensor,
+                         gram_k: torch.Tensor) -> None:
+    """Add the second moments of a batch of calibration samples into ``gram_q``/``gram_k``
+    (float64 ``[h_kv, d, d]``). ``q``: bf16 ``[n, h_q, d]``; ``k``: bf16 ``[n, h_kv, d]``."""
+    _need(q, "q", torch.bfloat16, contiguous=False)
+    _need(k, "k", torch.bfloat16, contiguous=False)
+    _need(gram_q, "gram_q", torch.float64)
+    _need(gram_k, "gram_k", torch.float64)
+    n, h_q, d = q.shape
+    h_kv = k.shape[1]
+    if q.stride(2) != 1 or q.stride(1) != d or k.stride(2) != 1 or k.stride(1) != d:
+        raise ValueError("q and k rows must be [heads, d] contiguous")
+    call("jssa_calibrate_accumulate", q.data_ptr(), q.stride(0), k.data_ptr(), k.stride(0), n, h_q,
+         h_kv, d, gram_q.data_ptr(), gram_k.data_ptr(), _stream(q.device))
+
+
+def compute_basis(gram_q: torch.Tensor, gram_k: torch.Tensor, rank: int,
+                  with_eigvals: bool = True):
+    """``M = TopEig_r(G_Q/tr + G_K/tr)^T`` per KV head: float32 ``[h_kv, r, d]`` (and float64
+    eigenvalues ``[h_kv, d]``, descending)."""
+    _need(gram_q, "gram_q", torch.float64)
+    _need(gram_k, "gram_k", torch.float64)
+    h_kv, d, _ = gram_q.shape
+    dev = gram_q.device
+    basis = torch.empty((h_kv, rank, d), dtype=torch.float32, device=dev)
+    eig = torch.empty((h_kv, d), dtype=torch.float64, device=dev) if with_eigvals else None
+    nbytes = workspace_size(FN_COMPUTE_BASIS, 0, 1, h_kv, d, 0, 0)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    call("jssa_compute_basis", gram_q.data_ptr(), gram_k.data_ptr(), h_kv, d, rank, basis.data_ptr(),
+         _ptr(eig), ws.data_ptr(), nbytes, _stream(dev))
+    return basis, eig
+
+
+def calibrate(q: torch.Tensor, k: torch.Tensor, rank: int, batch: int = 8192):
+    """Whole calibration over ``n`` samples, in batches of ``batch`` samples."""
+    n, h_q, d = q.shape
+    h_kv = k.shape[1]
+    gq = torch.zeros((h_kv, d, d), dtype=torch.float64, device=q.device)
+    gk = torch.zeros_like(gq)
+    for s in range(0, n, batch):
+        calibrate_accumulate(q[s:s + batch], k[s:s + batch], gq, gk)
+    basis, eig = compute_basis(gq, gk, rank)
+    return {"M": basis, "eigvals": eig, "gram_q": gq, "gram_k": gk}
+
+
+# ------------------------------------------------------------------------------------------------
+# Decode
+# ------------------------------------------------------------------------------------------------
+
+
+def store(k: torch.Tensor, slot_mapping: torch.Tensor, basis: torch.Tensor,
+          score_cache: torch.Tensor) -> None:
+    """Write ``e4m3(M_h k)`` of each token ``k[t]`` (bf16 ``[t, h_kv, d]``) at flat slot
+    ``slot_mapping[t]`` (int64; negative = skip) of the scoring cache
+    (uint8 ``[num_pages, h_kv, page_size, r]``)."""
+    _need(k, "k", torch.bfloat16, contiguous=False)
+    _need(slot_mapping, "slot_mapping", torch.int64)
+    _need(basis, "basis", torch.float32)
+    _need(score_cache, "score_cache", torch.uint8)
+    t, h_kv, d = k.shape
+    num_pages, _, page_size, r = score_cache.shape
+    if k.stride(2) != 1 or k.stride(1) != d:
+        raise ValueError("k rows must be [h_kv, d] contiguous")
+    call("jssa_store", k.data_ptr(), k.stride(0), slot_mapping.data_ptr(), t, h_kv, d, r,
+         basis.data_ptr(), score_cache.data_ptr(), num_pages, page_size, _stream(k.device))
+
+
+def score_topk(q: torch.Tensor, basis: torch.Tensor, score_cache: torch.Tensor,
+               block_table: torch.Tensor, seq_lens: torch.Tensor, budget: int,
+               idx: Optional[torch.Tensor] = None, count: Optional[torch.Tensor] = None):
+    """Index sets ``idx`` (int32 ``[batch, h_kv, budget]``, ascending, -1 padded) and ``count``."""
+    for t, n, dt in ((q, "q", torch.bfloat16), (basis, "basis", torch.float32),
+                     (score_cache, "score_cache", torch.uint8), (block_table, "block_table", torch.int32),
+                     (seq_lens, "seq_lens", torch.int32)):
+        _need(t, n, dt)
+    batch, h_q, d = q.shape
+    h_kv, r, _ = basis.shape
+    num_pages, _, page_size, _ = score_cache.shape
+    if idx is None:
+        idx = torch.empty((batch, h_kv, budget), dtype=torch.int32, device=q.device)
+    if count is None:
+        count = torch.empty((batch, h_kv), dtype=torch.int32, device=q.device)
+    call("jssa_score_topk", q.data_ptr(), basis.data_ptr(), score_cache.data_ptr(),
+         block_table.data_ptr(), block_table.shape[1], seq_lens.data_ptr(), batch, h_q, h_kv, d, r,
+         num_pages, page_size, budget, idx.data_ptr(), count.data_ptr(), None, 0, _stream(q.device))
+    return idx, count
+
+
+def indexed_attend(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                   block_table: torch.Tensor, idx: torch.Tensor, count: torch.Tensor,
+                   scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                   ws: Optional[Workspace] = None) -> torch.Tensor:
+    """Gather-free attention of every query head over its KV head's index set."""
+    _need(q, "q", torch.bfloat16)
+    _need(k_cache, "k_cache", torch.bfloat16, contiguous=False)
+    _need(v_cache, "v_cache", torch.bfloat16, contiguous=False)
+    _need(block_table, "block_table", torch.int32)
+    _need(idx, "idx", torch.int32)
+    _need(count, "count", torch.int32)
+    batch, h_q, d = q.shape
+    num_pages, page_size, h_kv, _ = k_cache.shape
+    strides = kv_strides(k_cache)
+    if kv_strides(v_cache) != strides:
+        raise ValueError("K and V caches must share one layout")
+    budget = idx.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    out = torch.empty_like(q) if out is None else out
+    w = _ws(q.device, ws)
+    p, n = w.get(workspace_size(FN_INDEXED_ATTEND, batch, h_q, h_kv, d, 0, budget))
+    call("jssa_indexed_attend", q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), *strides,
+         block_table.data_ptr(), block_table.shape[1], idx.data_ptr(), count.data_ptr(), batch, h_q,
+         h_kv, d, budget, num_pages, page_size, scale, out.data_ptr(), p, n, _stream(q.device))
+    return out
+
+
+def dense_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                 block_table: torch.Tensor, seq_lens: torch.Tensor, scale: Optional[float] = None,
+                 window: int = -1, out: Optional[torch.Tensor] = None,
+                 ws: Optional[Workspace] = None) -> torch.Tensor:
+    """Dense paged decode attention over ``[max(0, L - window), L)`` (all when window <= 0)."""
+    _need(q, "q", torch.bfloat16)
+    _need(k_cache, "k_cache", torch.bfloat16, contiguous=False)
+    _need(v_cache, "v_cache", torch.bfloat16, contiguous=False)
+    _need(block_table, "block_table", torch.int32)
+    _need(seq_lens, "seq_lens", torch.int32)
+    batch, h_q, d = q.shape
+    num_pages, page_size, h_kv, _ = k_cache.shape
+    strides = kv_strides(k_cache)
+    if kv_strides(v_cache) != strides:
+        raise ValueError("K and V caches must share one layout")
+    max_pages = block_table.shape[1]
+    span = max_pages * page_size if window <= 0 else min(window, max_pages * page_size)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    out = torch.empty_like(q) if out is None else out
+    w = _ws(q.device, ws)
+    p, n = w.get(workspace_size(FN_DENSE_DECODE, batch, h_q, h_kv, d, span, 0))
+    call("jssa_dense_decode", q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), *strides,
+         block_table.data_ptr(), max_pages, seq_lens.data_ptr(), batch, h_q, h_kv, d, num_pages,
+         page_size, window, scale, out.data_ptr(), p, n, _stream(q.device))
+    return out
+
+
+def decode(q: torch.Tensor, k_new: Optional[torch.Tensor], v_new: Optional[torch.Tensor],
+           k_cache: torch.Tensor, v_cache: torch.Tensor, score_cache: torch.Tensor,
+           basis: torch.Tensor, block_table: torch.Tensor, seq_lens: torch.Tensor, budget: int,
+           scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+           idx: Optional[torch.Tensor] = None, count: Optional[torch.Tensor] = None,
+           ws: Optional[Workspace] = None):
+    """One JSSA decode step for one layer (store new token, score + top-B, indexed attend).
+    Returns ``(out, idx, count)``."""
+    _need(q, "q", torch.bfloat16)
+    if (k_new is None) != (v_new is None):
+        raise ValueError("k_new and v_new go together")
+    if k_new is not None:
+        _need(k_new, "k_new", torch.bfloat16)
+        _need(v_new, "v_new", torch.bfloat16)
+    for t, n, dt in ((basis, "basis", torch.float32), (score_cache, "score_cache", torch.uint8),
+                     (block_table, "block_table", torch.int32), (seq_lens, "seq_lens", torch.int32)):
+        _need(t, n, dt)
+    _need(k_cache, "k_cache", torch.bfloat16, contiguous=False)
+    _need(v_cache, "v_cache", torch.bfloat16, contiguous=False)
+    batch, h_q, d = q.shape
+    num_pages, page_size, h_kv, _ = k_cache.shape
+    r = basis.shape[1]
+    strides = kv_strides(k_cache)
+    if kv_strides(v_cache) != strides:
+        raise ValueError("K and V caches must share one layout")
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    out = torch.empty_like(q) if out is None else out
+    if idx is None:
+        idx = torch.empty((batch, h_kv, budget), dtype=torch.int32, device=q.device)
+    if count is None:
+        count = torch.empty((batch, h_kv), dtype=torch.int32, device=q.device)
+    w = _ws(q.device, ws)
+    p, n = w.get(workspace_size(FN_DECODE, batch, h_q, h_kv, d, 0, budget))
+    call("jssa_decode", q.data_ptr(), _ptr(k_new), _ptr(v_new), k_cache.data_ptr(),
+         v_cache.data_ptr(), *strides, score_cache.data_ptr(), basis.data_ptr(),
+         block_table.data_ptr(), block_table.shape[1], seq_lens.data_ptr(), batch, h_q, h_kv, d, r,
+         num_pages, page_size, budget, scale, idx.data_ptr(), count.data_ptr(), out.data_ptr(), p, n,
+         _stream(q.device))
+    return out, idx, count
+
+
+def device_error(clear: bool = True, device=None) -> int:
+    """Flags raised by the kernels' bounds checks since the last clear (synchronises)."""
+    dev = torch.device(device or "cuda")
+    flags = ctypes.c_uint32(0)
+    call("jssa_device_error", ctypes.byref(flags), int(clear), _stream(dev))
+    return int(flags.value)
+
+
+class PagedLayer:
+    """One attention layer's decode state: paged bf16 K/V caches, the FP8 scoring cache, the
+    basis and the per-step buffers, with ``step`` running one JSSA decode step."""
+
+    def __init__(self, k_cache, v_cache, block_table, seq_lens, basis, budget, scale=None):
+        self.k_cache, self.v_cache = k_cache, v_cache
+        self.block_table, self.seq_lens = block_table, seq_lens
+        self.basis = basis
+        self.budget = budget
+        num_pages, page_size, h_kv, d = k_cache.shape
+        self.page_size = page_size
+        self.scale = 1.0 / math.sqrt(d) if scale is None else scale
+        r = basis.shape[1]
+        self.score_cache = torch.zeros((num_pages, h_kv, page_size, r), dtype=torch.uint8,
+                                       device=k_cache.device)
+        batch = block_table.shape[0]
+        self.idx = torch.empty((batch, h_kv, budget), dtype=torch.int32, device=k_cache.device)
+        self.count = torch.empty((batch, h_kv), dtype=torch.int32, device=k_cache.device)
+        self.ws = Workspace(k_cache.device)
+
+    def prefill_scores(self, chunk_pages: int = 4096) -> None:
+        """Store the scoring code of every cached position (all slots of every page)."""
+        num_pages, page_size, h_kv, d = self.k_cache.shape
+        flat = self.k_cache.view(num_pages * page_size, h_kv, d)
+        for p0 in range(0, num_pages, chunk_pages):
+            p1 = min(num_pages, p0 + chunk_pages)
+            slots = torch.arange(p0 * page_size, p1 * page_size, dtype=torch.int64,
+                                 device=flat.device)
+            store(flat[p0 * page_size:p1 * page_size], slots, self.basis, self.score_cache)
+
+    def step(self, q, k_new=None, v_new=None, out=None):
+        return decode(q, k_new, v_new, self.k_cache, self.v_cache, self.score_cache, self.basis,
+                      self.block_table, self.seq_lens, self.budget, self.scale, out, self.idx,
+                      self.count, self.ws)
+
+    def dense(self, q, out=None, window=-1):
+        return dense_decode(q, self.k_cache, self.v_cache, self.block_table, self.seq_lens,
+                            self.scale, window, out, self.ws)

@@ -1,0 +1,330 @@
+// C ABI of libjssa.so (declared in include/jssa.h): host-side argument checks, workspace sizing
+// and kernel chaining. Nothing here allocates device memory or synchronises (jssa_device_error
+// excepted).
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/jssa.h"
+#include "common.cuh"
+
+namespace jssa {
+
+
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+}  // namespace jssa
+
+namespace {
+
+using jssa::AttendArgs;
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr int64_t kMaxContext = (int64_t)jssa::kMaxClusterCtas * jssa::kScoreChunkMax;
+
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? JSSA_OK : (int)e; }
+inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+inline cudaStream_t as_stream(jssa_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+bool supported_dr(int d, int r) { return d == 128 && (r == 32 || r == 64); }
+
+int check_heads(int h_q, int h_kv) {
+  if (h_q <= 0 || h_kv <= 0 || h_q % h_kv) return JSSA_ERR_SHAPE;
+  return JSSA_OK;
+}
+
+int check_paging(int max_pages, int64_t num_pages, int page_size) {
+  if (max_pages <= 0 || num_pages <= 0 || page_size <= 0) return JSSA_ERR_SHAPE;
+  if ((int64_t)max_pages * page_size > (int64_t)INT32_MAX / 2) return JSSA_ERR_SHAPE;
+  return JSSA_OK;
+}
+
+int check_kv(const void* k_cache, const void* v_cache, int64_t page_stride, int64_t slot_stride,
+             int64_t head_stride, int h_kv, int d, int page_size) {
+  if (!k_cache || !v_cache) return JSSA_ERR_NULL;
+  if (!aligned16(k_cache) || !aligned16(v_cache)) return JSSA_ERR_ALIGN;
+  if (page_stride <= 0 || slot_stride <= 0 || head_stride <= 0) return JSSA_ERR_SHAPE;
+  if ((page_stride | slot_stride | head_stride) & 7) return JSSA_ERR_ALIGN;  // 16-byte rows
+  if (head_stride < d && slot_stride < d) return JSSA_ERR_SHAPE;
+  (void)h_kv;
+  (void)page_size;
+  return JSSA_OK;
+}
+
+size_t score_ws_bytes() { return 0; }
+
+jssa::AttendPlan attend_plan_indexed(int batch, int h_q, int h_kv, int d, int budget) {
+  return jssa::plan_attend(batch * h_kv, budget, h_q / h_kv, d);
+}
+
+jssa::AttendPlan attend_plan_dense(int batch, int h_q, int h_kv, int d, int max_seq_len) {
+  return jssa::plan_attend(batch * h_kv, max_seq_len, h_q / h_kv, d);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* jssa_status_string(int status) {
+  switch (status) {
+    case JSSA_OK: return "ok";
+    case JSSA_ERR_NULL: return "a required pointer is NULL";
+    case JSSA_ERR_SHAPE: return "inconsistent or out-of-range sizes";
+    case JSSA_ERR_UNSUPPORTED: return "no kernel instance for these sizes";
+    case JSSA_ERR_ALIGN: return "pointer or stride not 16-byte aligned";
+    case JSSA_ERR_WORKSPACE: return "workspace missing or too small";
+    case JSSA_ERR_DEVICE: return "no usable CUDA device";
+    default: break;
+  }
+  if (status > 0) return cudaGetErrorString((cudaError_t)status);
+  return "unknown status";
+}
+
+int jssa_version(void) { return kVersion; }
+
+int jssa_workspace_size(int fn, int batch, int h_q, int h_kv, int d, int max_seq_len, int budget,
+                        size_t* bytes) {
+  if (!bytes) return JSSA_ERR_NULL;
+  *bytes = 0;
+  if (batch < 0 || d <= 0 || max_seq_len < 0) return JSSA_ERR_SHAPE;
+  if (fn == JSSA_FN_COMPUTE_BASIS) {
+    if (h_kv <= 0) return JSSA_ERR_SHAPE;
+    *bytes = (size_t)h_kv * d * d * sizeof(double);
+    return JSSA_OK;
+  }
+  int st = check_heads(h_q, h_kv);
+  if (st) return st;
+  switch (fn) {
+    case JSSA_FN_SCORE_TOPK:
+      *bytes = score_ws_bytes();
+      return JSSA_OK;
+    case JSSA_FN_INDEXED_ATTEND:
+    case JSSA_FN_DECODE:
+      if (budget <= 0) return JSSA_ERR_SHAPE;
+      *bytes = attend_plan_indexed(batch, h_q, h_kv, d, budget).ws_bytes;
+      return JSSA_OK;
+    case JSSA_FN_DENSE_DECODE:
+      *bytes = attend_plan_dense(batch, h_q, h_kv, d, max_seq_len).ws_bytes;
+      return JSSA_OK;
+    default:
+      return JSSA_ERR_SHAPE;
+  }
+}
+
+int jssa_workspace_init(void* ws, size_t ws_bytes, jssa_stream_t stream) {
+  if (ws_bytes == 0) return JSSA_OK;
+  if (!ws) return JSSA_ERR_NULL;
+  return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, as_stream(stream)));
+}
+
+int jssa_calibrate_accumulate(const jssa_bf16* q, int64_t q_stride_n, const jssa_bf16* k,
+                              int64_t k_stride_n, int n, int h_q, int h_kv, int d,
+                              double* gram_q, double* gram_k, jssa_stream_t stream) {
+  if (n < 0) return JSSA_ERR_SHAPE;
+  int st = check_heads(h_q, h_kv);
+  if (st) return st;
+  if (d != 128) return JSSA_ERR_UNSUPPORTED;
+  if (h_q / h_kv > 16) return JSSA_ERR_UNSUPPORTED;
+  if (n == 0) return JSSA_OK;
+  if (!q || !k || !gram_q || !gram_k) return JSSA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || (q_stride_n & 7) || (k_stride_n & 7)) return JSSA_ERR_ALIGN;
+  if (q_stride_n < (int64_t)h_q * d || k_stride_n < (int64_t)h_kv * d) return JSSA_ERR_SHAPE;
+  return cuda_status(jssa::launch_gram(q, q_stride_n, k, k_stride_n, n, h_q, h_kv, d, gram_q,
+                                       gram_k, as_stream(stream)));
+}
+
+int jssa_compute_basis(const double* gram_q, const double* gram_k, int h_kv, int d, int r,
+                       float* basis, double* eigvals, void* ws, size_t ws_bytes,
+                       jssa_stream_t stream) {
+  if (h_kv <= 0 || r <= 0 || r > d) return JSSA_ERR_SHAPE;
+  if (d != 128) return JSSA_ERR_UNSUPPORTED;
+  if (!gram_q || !gram_k || !basis) return JSSA_ERR_NULL;
+  const size_t need = (size_t)h_kv * d * d * sizeof(double);
+  if (!ws || ws_bytes < need) return JSSA_ERR_WORKSPACE;
+  if (((uintptr_t)ws & 7u) != 0) return JSSA_ERR_ALIGN;
+  return cuda_status(jssa::launch_basis(gram_q, gram_k, h_kv, d, r, basis, eigvals,
+                                        static_cast<double*>(ws), as_stream(stream)));
+}
+
+int jssa_store(const jssa_bf16* k, int64_t k_stride_t, const int64_t* slot_mapping, int t,
+               int h_kv, int d, int r, const float* basis, uint8_t* score_cache,
+               int64_t num_pages, int page_size, jssa_stream_t stream) {
+  if (t < 0 || h_kv <= 0 || num_pages <= 0 || page_size <= 0) return JSSA_ERR_SHAPE;
+  if (r <= 0 || r > d) return JSSA_ERR_SHAPE;
+  if (!supported_dr(d, r)) return JSSA_ERR_UNSUPPORTED;
+  if (t == 0) return JSSA_OK;
+  if (!k || !slot_mapping || !basis || !score_cache) return JSSA_ERR_NULL;
+  if (!aligned16(k) || (k_stride_t & 7) || !aligned16(score_cache)) return JSSA_ERR_ALIGN;
+  if (k_stride_t < (int64_t)h_kv * d) return JSSA_ERR_SHAPE;
+  return cuda_status(jssa::launch_store(k, k_stride_t, slot_mapping, t, h_kv, d, r, basis,
+                                        score_cache, num_pages, page_size, as_stream(stream)));
+}
+
+static int check_score_args(const jssa_bf16* q, const float* basis, const uint8_t* score_cache,
+                            const int32_t* block_table, int max_pages, const int32_t* seq_lens,
+                            int batch, int h_q, int h_kv, int d, int r, int64_t num_pages,
+                            int page_size, int budget, const int32_t* idx, const int32_t* count) {
+  if (batch < 0 || budget <= 0) return JSSA_ERR_SHAPE;
+  int st = check_heads(h_q, h_kv);
+  if (st) return st;
+  if (r <= 0 || r > d) return JSSA_ERR_SHAPE;
+  if (!supported_dr(d, r)) return JSSA_ERR_UNSUPPORTED;
+  if ((st = check_paging(max_pages, num_pages, page_size))) return st;
+  if ((int64_t)max_pages * page_size > kMaxContext) return JSSA_ERR_UNSUPPORTED;
+  if (batch == 0) return JSSA_OK;
+  if (!q || !basis || !score_cache || !block_table || !seq_lens || !idx || !count)
+    return JSSA_ERR_NULL;
+  if (!aligned16(score_cache) || ((uintptr_t)q & 3u)) return JSSA_ERR_ALIGN;
+  return JSSA_OK;
+}
+
+int jssa_score_topk(const jssa_bf16* q, const float* basis, const uint8_t* score_cache,
+                    const int32_t* block_table, int max_pages, const int32_t* seq_lens, int batch,
+                    int h_q, int h_kv, int d, int r, int64_t num_pages, int page_size, int budget,
+                    int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
+                    jssa_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  int st = check_score_args(q, basis, score_cache, block_table, max_pages, seq_lens, batch, h_q,
+                            h_kv, d, r, num_pages, page_size, budget, idx, count);
+  if (st || batch == 0) return st;
+  return cuda_status(jssa::launch_score_topk(q, basis, score_cache, block_table, max_pages,
+                                             seq_lens, batch, h_q, h_kv, d, r, num_pages,
+                                             page_size, budget, idx, count, false,
+                                             as_stream(stream)));
+}
+
+static int check_attend_common(const jssa_bf16* q, const jssa_bf16* k_cache,
+                               const jssa_bf16* v_cache, int64_t ps, int64_t ss, int64_t hs,
+                               const int32_t* block_table, int max_pages, int batch, int h_q,
+                               int h_kv, int d, int64_t num_pages, int page_size,
+                               const jssa_bf16* out) {
+  if (batch < 0) return JSSA_ERR_SHAPE;
+  int st = check_heads(h_q, h_kv);
+  if (st) return st;
+  if (d != 128) return JSSA_ERR_UNSUPPORTED;
+  if (h_q / h_kv > jssa::kAttendMaxG) return JSSA_ERR_UNSUPPORTED;
+  if ((st = check_paging(max_pages, num_pages, page_size))) return st;
+  if (batch == 0) return JSSA_OK;
+  if (!q || !block_table || !out) return JSSA_ERR_NULL;
+  if ((st = check_kv(k_cache, v_cache, ps, ss, hs, h_kv, d, page_size))) return st;
+  if (((uintptr_t)q & 3u) || ((uintptr_t)out & 1u)) return JSSA_ERR_ALIGN;
+  return JSSA_OK;
+}
+
+int jssa_indexed_attend(const jssa_bf16* q, const jssa_bf16* k_cache, const jssa_bf16* v_cache,
+                        int64_t kv_page_stride, int64_t kv_slot_stride, int64_t kv_head_stride,
+                        const int32_t* block_table, int max_pages, const int32_t* idx,
+                        const int32_t* count, int batch, int h_q, int h_kv, int d, int budget,
+                        int64_t num_pages, int page_size, float softmax_scale, jssa_bf16* out,
+                        void* ws, size_t ws_bytes, jssa_stream_t stream) {
+  if (budget <= 0) return JSSA_ERR_SHAPE;
+  int st = check_attend_common(q, k_cache, v_cache, kv_page_stride, kv_slot_stride,
+                               kv_head_stride, block_table, max_pages, batch, h_q, h_kv, d,
+                               num_pages, page_size, out);
+  if (st || batch == 0) return st;
+  if (!idx || !count) return JSSA_ERR_NULL;
+  const jssa::AttendPlan plan = attend_plan_indexed(batch, h_q, h_kv, d, budget);
+  if (plan.ws_bytes && (!ws || ws_bytes < plan.ws_bytes)) return JSSA_ERR_WORKSPACE;
+  if (plan.ws_bytes && !aligned16(ws)) return JSSA_ERR_ALIGN;
+  AttendArgs a = {};
+  a.q = q; a.k_cache = k_cache; a.v_cache = v_cache;
+  a.page_stride = kv_page_stride; a.slot_stride = kv_slot_stride; a.head_stride = kv_head_stride;
+  a.block_table = block_table; a.max_pages = max_pages; a.idx = idx; a.count = count;
+  a.batch = batch; a.h_q = h_q; a.h_kv = h_kv; a.d = d; a.budget = budget;
+  a.num_pages = num_pages; a.page_size = page_size; a.scale = softmax_scale; a.out = out;
+  a.ws = ws;
+  return cuda_status(jssa::launch_attend(a, true, plan, false, as_stream(stream)));
+}
+
+int jssa_dense_decode(const jssa_bf16* q, const jssa_bf16* k_cache, const jssa_bf16* v_cache,
+                      int64_t kv_page_stride, int64_t kv_slot_stride, int64_t kv_head_stride,
+                      const int32_t* block_table, int max_pages, const int32_t* seq_lens,
+                      int batch, int h_q, int h_kv, int d, int64_t num_pages, int page_size,
+                      int window, float softmax_scale, jssa_bf16* out, void* ws,
+                      size_t ws_bytes, jssa_stream_t stream) {
+  int st = check_attend_common(q, k_cache, v_cache, kv_page_stride, kv_slot_stride,
+                               kv_head_stride, block_table, max_pages, batch, h_q, h_kv, d,
+                               num_pages, page_size, out);
+  if (st || batch == 0) return st;
+  if (!seq_lens) return JSSA_ERR_NULL;
+  int span = max_pages * page_size;
+  if (window > 0 && window < span) span = window;
+  const jssa::AttendPlan plan = jssa::plan_attend(batch * h_kv, span, h_q / h_kv, d);
+  if (plan.ws_bytes && (!ws || ws_bytes < plan.ws_bytes)) return JSSA_ERR_WORKSPACE;
+  if (plan.ws_bytes && !aligned16(ws)) return JSSA_ERR_ALIGN;
+  AttendArgs a = {};
+  a.q = q; a.k_cache = k_cache; a.v_cache = v_cache;
+  a.page_stride = kv_page_stride; a.slot_stride = kv_slot_stride; a.head_stride = kv_head_stride;
+  a.block_table = block_table; a.max_pages = max_pages; a.seq_lens = seq_lens;
+  a.window = window; a.batch = batch; a.h_q = h_q; a.h_kv = h_kv; a.d = d; a.budget = 0;
+  a.num_pages = num_pages; a.page_size = page_size; a.scale = softmax_scale; a.out = out;
+  a.ws = ws;
+  return cuda_status(jssa::launch_attend(a, false, plan, false, as_stream(stream)));
+}
+
+int jssa_decode(const jssa_bf16* q, const jssa_bf16* k_new, const jssa_bf16* v_new,
+                jssa_bf16* k_cache, jssa_bf16* v_cache, int64_t kv_page_stride,
+                int64_t kv_slot_stride, int64_t kv_head_stride, uint8_t* score_cache,
+                const float* basis, const int32_t* block_table, int max_pages,
+                const int32_t* seq_lens, int batch, int h_q, int h_kv, int d, int r,
+                int64_t num_pages, int page_size, int budget, float softmax_scale,
+                int32_t* idx, int32_t* count, jssa_bf16* out, void* ws, size_t ws_bytes,
+                jssa_stream_t stream) {
+  int st = check_score_args(q, basis, score_cache, block_table, max_pages, seq_lens, batch, h_q,
+                            h_kv, d, r, num_pages, page_size, budget, idx, count);
+  if (st) return st;
+  st = check_attend_common(q, k_cache, v_cache, kv_page_stride, kv_slot_stride, kv_head_stride,
+                           block_table, max_pages, batch, h_q, h_kv, d, num_pages, page_size, out);
+  if (st || batch == 0) return st;
+  if ((k_new == nullptr) != (v_new == nullptr)) return JSSA_ERR_NULL;
+  if (k_new && (!aligned16(k_new) || !aligned16(v_new))) return JSSA_ERR_ALIGN;
+  const jssa::AttendPlan plan = attend_plan_indexed(batch, h_q, h_kv, d, budget);
+  if (plan.ws_bytes && (!ws || ws_bytes < plan.ws_bytes)) return JSSA_ERR_WORKSPACE;
+  if (plan.ws_bytes && !aligned16(ws)) return JSSA_ERR_ALIGN;
+  cudaStream_t s = as_stream(stream);
+  bool pdl = false;
+  if (k_new) {
+    cudaError_t e = jssa::launch_store_decode(k_new, v_new, k_cache, v_cache, kv_page_stride,
+                                              kv_slot_stride, kv_head_stride, score_cache, basis,
+                                              block_table, max_pages, seq_lens, batch, h_kv, d, r,
+                                              num_pages, page_size, s);
+    if (e != cudaSuccess) return (int)e;
+    pdl = true;
+  }
+  cudaError_t e = jssa::launch_score_topk(q, basis, score_cache, block_table, max_pages, seq_lens,
+                                          batch, h_q, h_kv, d, r, num_pages, page_size, budget,
+                                          idx, count, pdl, s);
+  if (e != cudaSuccess) return (int)e;
+  AttendArgs a = {};
+  a.q = q; a.k_cache = k_cache; a.v_cache = v_cache;
+  a.page_stride = kv_page_stride; a.slot_stride = kv_slot_stride; a.head_stride = kv_head_stride;
+  a.block_table = block_table; a.max_pages = max_pages; a.idx = idx; a.count = count;
+  a.batch = batch; a.h_q = h_q; a.h_kv = h_kv; a.d = d; a.budget = budget;
+  a.num_pages = num_pages; a.page_size = page_size; a.scale = softmax_scale; a.out = out;
+  a.ws = ws;
+  return cuda_status(jssa::launch_attend(a, true, plan, true, s));
+}
+
+int jssa_device_error(uint32_t* flags, int clear, jssa_stream_t stream) {
+  if (!flags) return JSSA_ERR_NULL;
+  cudaStream_t s = as_stream(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return (int)e;
+  unsigned int v = 0;
+  e = cudaMemcpyFromSymbol(&v, jssa::g_device_error, sizeof(v));
+  if (e != cudaSuccess) return (int)e;
+  *flags = v;
+  if (clear) {
+    const unsigned int zero = 0u;
+    e = cudaMemcpyToSymbol(jssa::g_device_error, &zero, sizeof(zero));
+    if (e != cudaSuccess) return (int)e;
+  }
+  return JSSA_OK;
+}
+
+}  // extern "C"

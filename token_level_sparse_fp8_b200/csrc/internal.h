@@ -1,0 +1,83 @@
+// Internal launch interface between the C ABI (api.cu) and the kernel translation units.
+// Host-side argument checks happen in api.cu; the launchers below assume valid arguments.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace jssa {
+
+constexpr int kMaxClusterCtas = 16;        // non-portable cluster size used by score + top-B
+constexpr int kScoreThreads = 512;
+constexpr int kScoreChunkTarget = 8192;    // tokens of one (sequence, KV head) per CTA
+constexpr int kScoreChunkMax = 40960;      // shared-memory bound on tokens per CTA
+constexpr int kAttendWarps = 4;
+constexpr int kAttendTile = 16;            // tokens per warp-level tile
+constexpr int kAttendMaxG = 8;             // query heads per KV head held in one m16 tile
+
+struct ScorePlan {
+  int cluster;     // CTAs per (sequence, KV head)
+  int chunk;       // tokens per CTA (multiple of the page size and of 64)
+  size_t smem;     // dynamic shared memory per CTA
+};
+
+struct AttendPlan {
+  int splits;      // CTAs per (sequence, KV head)
+  int chunk;       // positions per CTA (multiple of 64)
+  size_t ws_bytes; // tickets + partials
+};
+
+int num_sms();
+
+ScorePlan plan_score(int pairs, int max_seq_len, int page_size);
+AttendPlan plan_attend(int pairs, int positions, int group, int d);
+
+cudaError_t launch_store(const uint16_t* k, int64_t k_stride_t, const int64_t* slot_mapping,
+                         int t, int h_kv, int d, int r, const float* basis, uint8_t* score_cache,
+                         int64_t num_pages, int page_size, cudaStream_t s);
+
+// Decode-time store: token b writes position seq_lens[b]-1 (K/V rows and scoring code).
+cudaError_t launch_store_decode(const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_cache,
+                                uint16_t* v_cache, int64_t ps_stride, int64_t slot_stride,
+                                int64_t head_stride, uint8_t* score_cache, const float* basis,
+                                const int32_t* block_table, int max_pages, const int32_t* seq_lens,
+                                int batch, int h_kv, int d, int r, int64_t num_pages,
+                                int page_size, cudaStream_t s);
+
+cudaError_t launch_score_topk(const uint16_t* q, const float* basis, const uint8_t* score_cache,
+                              const int32_t* block_table, int max_pages, const int32_t* seq_lens,
+                              int batch, int h_q, int h_kv, int d, int r, int64_t num_pages,
+                              int page_size, int budget, int32_t* idx, int32_t* count,
+                              bool pdl, cudaStream_t s);
+
+struct AttendArgs {
+  const uint16_t* q;
+  const uint16_t* k_cache;
+  const uint16_t* v_cache;
+  int64_t page_stride, slot_stride, head_stride;
+  const int32_t* block_table;
+  int max_pages;
+  const int32_t* idx;       // indexed mode
+  const int32_t* count;     // indexed mode
+  const int32_t* seq_lens;  // dense mode
+  int window;               // dense mode
+  int batch, h_q, h_kv, d;
+  int budget;               // indexed mode: index-set capacity
+  int64_t num_pages;
+  int page_size;
+  float scale;
+  uint16_t* out;
+  void* ws;
+};
+
+cudaError_t launch_attend(const AttendArgs& a, bool indexed, const AttendPlan& plan, bool pdl,
+                          cudaStream_t s);
+
+cudaError_t launch_gram(const uint16_t* q, int64_t q_stride, const uint16_t* k, int64_t k_stride,
+                        int n, int h_q, int h_kv, int d, double* gram_q, double* gram_k,
+                        cudaStream_t s);
+
+cudaError_t launch_basis(const double* gram_q, const double* gram_k, int h_kv, int d, int r,
+                         float* basis, double* eigvals, double* ws, cudaStream_t s);
+
+}  // namespace jssa

@@ -1,0 +1,175 @@
+// Store step: FP8 E4M3 projected key c = e4m3(M_h k) for new tokens (JSSA summary, section 3.4
+// "Projected Scoring Cache"; JSSA README, section 4 notes: r bytes per token and KV head).
+//
+// One CTA per (KV head, range of tokens). The basis rows of the head are staged in shared memory
+// once; each warp takes one token at a time, lane j computes output j (and j+32, ...) as a
+// float64 dot product over the d dimensions and rounds it once to E4M3. At decode the same kernel
+// also writes the new token's K and V rows into the paged cache.
+#include "common.cuh"
+
+namespace jssa {
+
+namespace store_detail {
+
+constexpr int kStoreThreads = 256;
+constexpr int kStoreWarps = kStoreThreads / 32;
+
+template <int D, int R, bool DECODE>
+__global__ void __launch_bounds__(kStoreThreads)
+    store_kernel(const uint16_t* __restrict__ k, int64_t k_stride_t,
+                 const int64_t* __restrict__ slot_mapping, int t_count, int h_kv,
+                 const float* __restrict__ basis, uint8_t* __restrict__ score_cache,
+                 int64_t num_pages, int page_size, int tokens_per_block,
+                 // decode-only arguments
+                 const uint16_t* __restrict__ v_new, uint16_t* __restrict__ k_cache,
+                 uint16_t* __restrict__ v_cache, int64_t page_stride, int64_t slot_stride,
+                 int64_t head_stride, const int32_t* __restrict__ block_table, int max_pages,
+                 const int32_t* __restrict__ seq_lens) {
+  extern __shared__ float store_smem[];
+  float* s_m = store_smem;                        // [R][D+1]
+  float* s_k = store_smem + R * (D + 1);            // [warps][D]
+  const int h = blockIdx.x;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const float* m_h = basis + (int64_t)h * R * D;
+  for (int i = threadIdx.x; i < R * D; i += kStoreThreads) s_m[(i / D) * (D + 1) + (i % D)] = m_h[i];
+  __syncthreads();
+
+  const int t0 = blockIdx.y * tokens_per_block;
+  const int t1 = min(t_count, t0 + tokens_per_block);
+  float* kw = s_k + warp * D;
+  for (int t = t0 + warp; t < t1; t += kStoreWarps) {
+    int64_t page, off;
+    if (DECODE) {
+      const int L = seq_lens[t];
+      if (L <= 0 || L > max_pages * page_size) {
+        if (L != 0 && lane == 0) raise_flag(4u);
+        continue;
+      }
+      const int pos = L - 1;
+      page = block_table[(int64_t)t * max_pages + pos / page_size];
+      off = pos % page_size;
+    } else {
+      const int64_t slot = slot_mapping[t];
+      if (slot < 0) continue;
+      page = slot / page_size;
+      off = slot % page_size;
+    }
+    if (page < 0 || page >= num_pages) {
+      if (lane == 0) raise_flag(1u);
+      continue;
+    }
+    const uint16_t* krow = k + (int64_t)t * k_stride_t + (int64_t)h * D;
+    // D/32 consecutive elements per lane (8 bytes for D = 128)
+    constexpr int E = D / 32;
+    static_assert(E == 4 || E == 8, "head dim");
+    uint32_t kw32[E / 2];
+    if (E == 4) {
+      uint2 v = *reinterpret_cast<const uint2*>(krow + lane * 4);
+      kw32[0] = v.x;
+      kw32[1] = v.y;
+    } else {
+      uint4 v = *reinterpret_cast<const uint4*>(krow + lane * 8);
+      kw32[0] = v.x; kw32[1] = v.y; kw32[2] = v.z; kw32[3] = v.w;
+    }
+#pragma unroll
+    for (int e = 0; e < E / 2; ++e) {
+      kw[lane * E + 2 * e] = bf16_lo(kw32[e]);
+      kw[lane * E + 2 * e + 1] = bf16_hi(kw32[e]);
+    }
+    if (DECODE) {
+      const int64_t base = page * page_stride + off * slot_stride + (int64_t)h * head_stride;
+      const uint16_t* vrow = v_new + (int64_t)t * k_stride_t + (int64_t)h * D;
+      if (E == 4) {
+        *reinterpret_cast<uint2*>(k_cache + base + lane * 4) = make_uint2(kw32[0], kw32[1]);
+        *reinterpret_cast<uint2*>(v_cache + base + lane * 4) =
+            *reinterpret_cast<const uint2*>(vrow + lane * 4);
+      } else {
+        *reinterpret_cast<uint4*>(k_cache + base + lane * 8) =
+            make_uint4(kw32[0], kw32[1], kw32[2], kw32[3]);
+        *reinterpret_cast<uint4*>(v_cache + base + lane * 8) =
+            *reinterpret_cast<const uint4*>(vrow + lane * 8);
+      }
+    }
+    __syncwarp();
+    uint8_t* dst = score_cache + ((page * h_kv + h) * page_size + off) * R;
+#pragma unroll
+    for (int j0 = 0; j0 < R; j0 += 32) {
+      const int j = j0 + lane;
+      const float* mrow = s_m + j * (D + 1);
+      double acc = 0.0;
+#pragma unroll 8
+      for (int i = 0; i < D; ++i) acc = fma((double)mrow[i], (double)kw[i], acc);
+      dst[j] = f64_to_e4m3(acc);
+    }
+    __syncwarp();
+  }
+  if (DECODE) pdl_trigger();
+}
+
+template <int D, int R, bool DECODE>
+cudaError_t launch_store_t(dim3 grid, size_t smem, cudaStream_t s, const uint16_t* k,
+                           int64_t k_stride_t, const int64_t* slot_mapping, int t, int h_kv,
+                           const float* basis, uint8_t* score_cache, int64_t num_pages,
+                           int page_size, int tpb, const uint16_t* v_new, uint16_t* k_cache,
+                           uint16_t* v_cache, int64_t page_stride, int64_t slot_stride,
+                           int64_t head_stride, const int32_t* block_table, int max_pages,
+                           const int32_t* seq_lens) {
+  auto kern = store_kernel<D, R, DECODE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kStoreThreads, smem, s>>>(k, k_stride_t, slot_mapping, t, h_kv, basis, score_cache,
+                                         num_pages, page_size, tpb, v_new, k_cache, v_cache,
+                                         page_stride, slot_stride, head_stride, block_table,
+                                         max_pages, seq_lens);
+  return cudaGetLastError();
+}
+
+template <bool DECODE>
+cudaError_t dispatch_store(int d, int r, int t, int h_kv, int tpb, cudaStream_t s,
+                           const uint16_t* k, int64_t k_stride_t, const int64_t* slot_mapping,
+                           const float* basis, uint8_t* score_cache, int64_t num_pages,
+                           int page_size, const uint16_t* v_new, uint16_t* k_cache,
+                           uint16_t* v_cache, int64_t page_stride, int64_t slot_stride,
+                           int64_t head_stride, const int32_t* block_table, int max_pages,
+                           const int32_t* seq_lens) {
+  if (t <= 0) return cudaSuccess;
+  dim3 grid(h_kv, (t + tpb - 1) / tpb);
+  const size_t smem = (size_t)(r * (d + 1) + kStoreWarps * d) * sizeof(float);
+#define JSSA_STORE_CASE(DD, RR)                                                                  \
+  if (d == DD && r == RR)                                                                        \
+    return launch_store_t<DD, RR, DECODE>(grid, smem, s, k, k_stride_t, slot_mapping, t, h_kv,   \
+                                          basis, score_cache, num_pages, page_size, tpb, v_new,  \
+                                          k_cache, v_cache, page_stride, slot_stride,            \
+                                          head_stride, block_table, max_pages, seq_lens);
+  JSSA_STORE_CASE(128, 32)
+  JSSA_STORE_CASE(128, 64)
+#undef JSSA_STORE_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace store_detail
+
+cudaError_t launch_store(const uint16_t* k, int64_t k_stride_t, const int64_t* slot_mapping,
+                         int t, int h_kv, int d, int r, const float* basis, uint8_t* score_cache,
+                         int64_t num_pages, int page_size, cudaStream_t s) {
+  const int tpb = t >= 4096 ? 256 : store_detail::kStoreWarps;
+  return store_detail::dispatch_store<false>(d, r, t, h_kv, tpb, s, k, k_stride_t, slot_mapping, basis,
+                               score_cache, num_pages, page_size, nullptr, nullptr, nullptr, 0, 0,
+                               0, nullptr, 0, nullptr);
+}
+
+cudaError_t launch_store_decode(const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_cache,
+                                uint16_t* v_cache, int64_t page_stride, int64_t slot_stride,
+                                int64_t head_stride, uint8_t* score_cache, const float* basis,
+                                const int32_t* block_table, int max_pages, const int32_t* seq_lens,
+                                int batch, int h_kv, int d, int r, int64_t num_pages,
+                                int page_size, cudaStream_t s) {
+  return store_detail::dispatch_store<true>(d, r, batch, h_kv, store_detail::kStoreWarps, s, k_new, (int64_t)h_kv * d,
+                              nullptr, basis, score_cache, num_pages, page_size, v_new, k_cache,
+                              v_cache, page_stride, slot_stride, head_stride, block_table,
+                              max_pages, seq_lens);
+}
+
+}  // namespace jssa
