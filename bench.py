@@ -34,8 +34,8 @@ METRIC = "JSSA decode-attn steps/s & HBM GB/s at 128K ctx vs dense full-KV, 1×B
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=800)
+    ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", choices=["jssa", "reference"], default="jssa")
     ap.add_argument("--batch", type=int, default=16)
     ap.add_argument("--budget", type=int, default=2048)
@@ -60,53 +60,60 @@ def dist_env():
 
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and throttle reasons sampled with NVML from a thread during a timed region."""
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, cuda_index: int, period_s: float = 0.01):
+        self.cuda_index = cuda_index
+        self.period = period_s
+        self.samples = []
+        self.thread = None
+
+    def _handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        try:
+            idx = torch.cuda._get_nvml_device_index(self.cuda_index)
+        except Exception:
+            idx = self.cuda_index
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(idx)
 
     def start(self):
+        import threading
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
+            self.nvml, self.h = self._handle()
+            self.max_mhz = self.nvml.nvmlDeviceGetMaxClockInfo(self.h, self.nvml.NVML_CLOCK_SM)
         except Exception:
-            self.proc = None
+            self.nvml = None
+            return
+        self.stop_flag = threading.Event()
+
+        def run():
+            while not self.stop_flag.is_set():
+                try:
+                    mhz = self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM)
+                    rs = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    self.samples.append((mhz, rs))
+                except Exception:
+                    pass
+                self.stop_flag.wait(self.period)
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
 
     def stop(self) -> dict:
-        if self.proc is None:
+        if self.nvml is None or self.thread is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.fh.close()
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as fh:
-            for line in fh:
-                p = [x.strip() for x in line.split(",")]
-                if len(p) < 9:
-                    continue
-                try:
-                    sm.append(float(p[1]))
-                    smax.append(float(p[2]))
-                except ValueError:
-                    continue
-                for n, v in zip(names, p[5:9]):
-                    if v.lower().startswith("active"):
-                        reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        self.stop_flag.set()
+        self.thread.join(timeout=2)
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
+        reasons = sorted({name for _, rs in self.samples for bit, name in self.REASONS.items() if rs & bit})
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml"}
 
 
 # ------------------------------------------------------------------------------------------------
@@ -162,6 +169,36 @@ def timed(fn, steps, warmup, stream, barrier):
     torch.cuda.synchronize()
     barrier()
     return e0.elapsed_time(e1) / 1e3
+
+
+class GraphSteps:
+    """`per` consecutive calls fn(0..per-1) captured once in a CUDA graph; stepping replays it.
+    Removes the host launch cost from device timings (the kernels themselves are unchanged)."""
+
+    def __init__(self, fn, per, warmup=2):
+        import torch
+        for i in range(warmup):
+            fn(i)
+        torch.cuda.synchronize()
+        self.per = per
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            for i in range(per):
+                fn(i)
+        torch.cuda.synchronize()
+
+    def __call__(self, i):
+        self.graph.replay()
+
+
+def timed_graph(fn, steps, warmup, stream, barrier, per=8):
+    """Device time of `steps` calls (rounded up to whole graphs of `per` calls) and the count."""
+    g = GraphSteps(fn, per)
+    reps = max(1, -(-steps // per))
+    wreps = max(1, -(-warmup // per))
+    t = timed(g, reps, wreps, stream, barrier)
+    del g
+    return t, reps * per
 
 
 def algorithmic_bytes(w, dense=False):
@@ -367,9 +404,25 @@ def run_jssa(args):
         layer.step(qs[i % nq], k_new, v_new, out)
 
     sampler = ClockSampler(local)
+    # the whole step sequence is replayed from a CUDA graph (as in the pages' decode protocol)
+    g_step = GraphSteps(step, nq)
+    reps = max(1, -(-args.steps // nq))
+    for _ in range(max(1, -(-args.warmup // nq))):
+        g_step(0)
+    barrier()
+    torch.cuda.synchronize()
     sampler.start()
-    t_step = max_over_ranks(timed(step, args.steps, args.warmup, stream, barrier))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        g_step(0)
+    e1.record(stream)
+    torch.cuda.synchronize()
     clocks = sampler.stop()
+    barrier()
+    n_steps = reps * nq
+    t_step = max_over_ranks(e0.elapsed_time(e1) / 1e3)
+    del g_step
     launches_per_step = 3
 
     # per-kernel device times (same configuration, each kernel launched alone)
@@ -383,14 +436,17 @@ def run_jssa(args):
         J.indexed_attend(qs[i % nq], layer.k_cache, layer.v_cache, layer.block_table, idx, count,
                          layer.scale, out, layer.ws)
 
-    t_score = max_over_ranks(timed(score_only, args.steps, args.warmup, stream, barrier))
-    t_attend = max_over_ranks(timed(attend_only, args.steps, args.warmup, stream, barrier))
+    t_score, n_score = timed_graph(score_only, args.steps, args.warmup, stream, barrier, nq)
+    t_score = max_over_ranks(t_score) / n_score
+    t_attend, n_attend = timed_graph(attend_only, args.steps, args.warmup, stream, barrier, nq)
+    t_attend = max_over_ranks(t_attend) / n_attend
 
     t_dense = None
     if not args.no_dense:
-        dense_steps = max(3, args.steps // 4)
-        t_dense = max_over_ranks(timed(lambda i: layer.dense(qs[i % nq], out), dense_steps,
-                                       max(3, args.warmup // 2), stream, barrier)) / dense_steps
+        layer.dense(qs[0], out)  # sizes the shared workspace before capture
+        t_dense, n_dense = timed_graph(lambda i: layer.dense(qs[i % nq], out), max(8, args.steps // 4),
+                                       8, stream, barrier, nq)
+        t_dense = max_over_ranks(t_dense) / n_dense
 
     # end to end through the public API with host buffers: H2D of the step's inputs, D2H of out
     q_host = [q.cpu().pin_memory() for q in qs]
@@ -424,17 +480,17 @@ def run_jssa(args):
         return
 
     peak, peak_kind = peaks()
-    ms_step = t_step / args.steps * 1e3
-    steps_per_s = world * args.steps / t_step
+    ms_step = t_step / n_steps * 1e3
+    steps_per_s = world * n_steps / t_step
     bytes_step = algorithmic_bytes(w)
-    score_launch_s = t_score / args.steps
+    score_launch_s = t_score
     achieved = score_bytes(w) / score_launch_s / 1e9
     line = {
         "metric": METRIC,
         "value": steps_per_s,
         "unit": "steps/s",
         "n_gpus": world,
-        "steps": args.steps,
+        "steps": n_steps,
         "warmup": args.warmup,
         "ms_per_step": ms_step,
         "higher_is_better": True,
@@ -459,12 +515,13 @@ def run_jssa(args):
                      "unit": "GB/s", "frac": achieved / peak, "traffic": None,
                      "bytes_per_launch": score_bytes(w), "ms_per_launch": score_launch_s * 1e3,
                      "peak_kind": peak_kind},
-        "kernels_ms": {"score_topk": score_launch_s * 1e3, "indexed_attend": t_attend / args.steps * 1e3,
-                       "attend_gbs": attend_bytes(w) / (t_attend / args.steps) / 1e9},
+        "kernels_ms": {"score_topk": score_launch_s * 1e3, "indexed_attend": t_attend * 1e3,
+                       "attend_gbs": attend_bytes(w) / t_attend / 1e9},
         "clocks": clocks,
         "e2e": {"value": world * args.steps / t_e2e, "unit": "steps/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": launches_per_step * n_steps,
+        "timing": "CUDA events around replays of a CUDA graph holding 8 consecutive steps",
     }
     if t_dense is not None:
         dense_bytes = algorithmic_bytes(w, dense=True)

@@ -94,7 +94,7 @@ def joint_basis(g_q: np.ndarray, g_k: np.ndarray, r: int) -> tuple:
     w = w[..., ::-1]
     u = u[..., ::-1]
     m = np.swapaxes(u[..., :r], -1, -2)    # TopEig_r(.) as columns, transposed into rows
-    return sign_rows(m), w
+    return np.ascontiguousarray(sign_rows(m)), np.ascontiguousarray(w)
 
 
 def projector(m: np.ndarray) -> np.ndarray:

@@ -138,7 +138,7 @@ def _keys(factors: dict, n: int, gen: torch.Generator, device) -> torch.Tensor:
     mu = torch.as_tensor(factors["mu"], dtype=torch.float32, device=device)
     h_kv, d = mu.shape
     z = torch.randn((n, h_kv, d), generator=gen, device=device, dtype=torch.float32)
-    return (_mix(a_k, z) + mu[None]).to(torch.bfloat16)
+    return (_mix(a_k, z) + mu[None]).to(torch.bfloat16).contiguous()
 
 
 def _queries(factors: dict, n: int, group: int, gen: torch.Generator, device) -> torch.Tensor:
@@ -146,7 +146,7 @@ def _queries(factors: dict, n: int, group: int, gen: torch.Generator, device) ->
     h_kv, d, _ = a_q.shape
     z = torch.randn((n, h_kv * group, d), generator=gen, device=device, dtype=torch.float32)
     a_rep = a_q.repeat_interleave(group, dim=0)  # query head i uses KV head i // group
-    return _mix(a_rep, z).to(torch.bfloat16)
+    return _mix(a_rep, z).to(torch.bfloat16).contiguous()
 
 
 def sample_calibration(factors: dict, n: int, group: int, seed: int, layer: int = 0,

@@ -4,6 +4,10 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <map>
+#include <mutex>
+#include <utility>
+
 #include "../../include/jssa.h"
 #include "common.cuh"
 
@@ -11,10 +15,36 @@ namespace jssa {
 
 
 
+namespace {
+std::mutex g_cfg_mu;
+std::map<std::pair<const void*, int>, int> g_cfg_smem;  // (kernel, device) -> configured bytes
+int g_sms[64] = {0};
+}  // namespace
+
 int num_sms() {
-  int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (g_sms[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    g_sms[dev] = n;
+  }
+  return g_sms[dev];
+}
+
+cudaError_t configure_kernel(const void* fn, int smem_bytes, bool nonportable_cluster) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_cfg_mu);
+  const auto key = std::make_pair(fn, dev);
+  auto it = g_cfg_smem.find(key);
+  if (it != g_cfg_smem.end() && it->second >= smem_bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  if (e == cudaSuccess && nonportable_cluster)
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess) g_cfg_smem[key] = smem_bytes;
+  return e;
 }
 
 }  // namespace jssa

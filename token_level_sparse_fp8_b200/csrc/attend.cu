@@ -301,7 +301,7 @@ template <int D, bool INDEXED>
 cudaError_t launch_t(const AttendArgs& a, const AttendPlan& plan, bool pdl, cudaStream_t s) {
   auto kern = attend_kernel<D, INDEXED>;
   const int smem = Smem<D>::kTotal;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = configure_kernel((const void*)kern, (int)smem, false);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(plan.splits, a.batch * a.h_kv, 1);

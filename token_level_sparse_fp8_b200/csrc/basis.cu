@@ -181,7 +181,7 @@ cudaError_t launch_basis(const double* gram_q, const double* gram_k, int h_kv, i
   if (d != 128) return cudaErrorInvalidValue;
   const size_t smem = (size_t)d * (d + 1) * sizeof(double);
   auto kern = basis_detail::basis_kernel<128>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = configure_kernel((const void*)kern, (int)smem, false);
   if (e != cudaSuccess) return e;
   kern<<<h_kv, basis_detail::kThreads, smem, s>>>(gram_q, gram_k, r, basis, eigvals, ws);
   return cudaGetLastError();

@@ -10,7 +10,8 @@
 // Grid (sample chunks, h_kv, 2 [keys | queries]); 8 warps per CTA tile the full d x d = 128 x 128
 // Gram (warp w: rows 32*(w/2).., cols 64*(w%2)..) with mma.sync m16n8k16. Sample tiles of 32 rows
 // per head are staged in swizzled shared memory with cp.async; both operands are read with
-// ldmatrix.trans (X^T X). Each CTA adds its fp32 chunk sum into the float64 totals.
+// ldmatrix.trans (X^T X). Each CTA adds its chunk sum (fp32, folded per block) into the float64
+// totals.
 #include "common.cuh"
 
 namespace jssa {
@@ -19,7 +20,7 @@ namespace calib_detail {
 
 constexpr int kThreads = 256;
 constexpr int kTileN = 32;        // samples per staged tile
-constexpr int kChunkN = 512;      // samples per CTA
+constexpr int kChunkN = 256;      // samples per CTA
 
 template <int D>
 __global__ void __launch_bounds__(kThreads)
@@ -37,11 +38,16 @@ __global__ void __launch_bounds__(kThreads)
   const int nh = is_q ? G : 1;  // head rows staged per sample
   const int n0 = blockIdx.x * kChunkN, n1 = min(n, n0 + kChunkN);
 
-  float acc[2][8][4];
+  // Tensor-core fp32 accumulation is not round-to-nearest, so the mma accumulators only ever
+  // hold the sum of one (head pair, 32-sample tile) block and are folded into a second set of
+  // fp32 registers with ordinary rounded adds after each block.
+  float acc[2][8][4], tot[2][8][4];
 #pragma unroll
   for (int a = 0; a < 2; ++a)
 #pragma unroll
-    for (int b = 0; b < 8; ++b) acc[a][b][0] = acc[a][b][1] = acc[a][b][2] = acc[a][b][3] = 0.f;
+    for (int b = 0; b < 8; ++b)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[a][b][c] = tot[a][b][c] = 0.f;
 
   const int row0 = 32 * (warp >> 1);   // first Gram row of this warp
   const int col0 = 64 * (warp & 1);    // first Gram column
@@ -91,6 +97,15 @@ __global__ void __launch_bounds__(kThreads)
             }
           }
         }
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+          for (int b = 0; b < 8; ++b)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              tot[a][b][c] += acc[a][b][c];
+              acc[a][b][c] = 0.f;
+            }
       }
     }
     __syncthreads();
@@ -104,10 +119,10 @@ __global__ void __launch_bounds__(kThreads)
     for (int nt = 0; nt < 8; ++nt) {
       const int i = row0 + mt * 16 + (lane >> 2);
       const int j = col0 + nt * 8 + 2 * (lane & 3);
-      atomicAdd(&gram[(int64_t)i * D + j], sc * (double)acc[mt][nt][0]);
-      atomicAdd(&gram[(int64_t)i * D + j + 1], sc * (double)acc[mt][nt][1]);
-      atomicAdd(&gram[(int64_t)(i + 8) * D + j], sc * (double)acc[mt][nt][2]);
-      atomicAdd(&gram[(int64_t)(i + 8) * D + j + 1], sc * (double)acc[mt][nt][3]);
+      atomicAdd(&gram[(int64_t)i * D + j], sc * (double)tot[mt][nt][0]);
+      atomicAdd(&gram[(int64_t)i * D + j + 1], sc * (double)tot[mt][nt][1]);
+      atomicAdd(&gram[(int64_t)(i + 8) * D + j], sc * (double)tot[mt][nt][2]);
+      atomicAdd(&gram[(int64_t)(i + 8) * D + j + 1], sc * (double)tot[mt][nt][3]);
     }
 }
 
@@ -121,7 +136,7 @@ cudaError_t launch_gram(const uint16_t* q, int64_t q_stride, const uint16_t* k, 
   const int G = h_q / h_kv;
   const size_t smem = (size_t)G * calib_detail::kTileN * d * 2;
   auto kern = calib_detail::gram_kernel<128>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = configure_kernel((const void*)kern, (int)smem, false);
   if (e != cudaSuccess) return e;
   dim3 grid((n + calib_detail::kChunkN - 1) / calib_detail::kChunkN, h_kv, 2);
   kern<<<grid, calib_detail::kThreads, smem, s>>>(q, q_stride, k, k_stride, n, h_q, h_kv, gram_q, gram_k);

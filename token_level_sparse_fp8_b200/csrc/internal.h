@@ -29,6 +29,10 @@ struct AttendPlan {
 
 int num_sms();
 
+// Raise a kernel's dynamic shared-memory limit (and allow clusters above 8 CTAs) once per device;
+// later calls are lock-protected lookups, so launches stay cheap and safe under stream capture.
+cudaError_t configure_kernel(const void* fn, int smem_bytes, bool nonportable_cluster);
+
 ScorePlan plan_score(int pairs, int max_seq_len, int page_size);
 AttendPlan plan_attend(int pairs, int positions, int group, int d);
 

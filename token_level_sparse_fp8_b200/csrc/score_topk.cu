@@ -6,14 +6,21 @@
 //   1. p = M_h qbar (qbar = mean of the G query heads of KV head h), fp32, in shared memory;
 //   2. stream the chunk's FP8 scoring rows (page-table indexed, 16-byte non-allocating loads,
 //      8 independent loads per thread in flight) and keep every score as an order-preserving
-//      32-bit key in shared memory -- scores never go to HBM;
-//   3. exact radix select of the budget-th largest key over the whole cluster: three digit
-//      passes (11, 11, 10 bits); each CTA histograms its own keys, the histograms are summed
-//      through distributed shared memory (each CTA reduces one slice of the bins), and every CTA
-//      finds the threshold digit from the slice totals;
+//      32-bit key in shared memory -- scores never go to HBM. The E4M3 codes are widened with
+//      integer operations (sign and the 7 exponent/mantissa bits are moved into an fp32 bit
+//      pattern whose value is the code's value times 2^-120); the power of two is folded into p,
+//      together with a per-head power-of-two scale that keeps every product finite, so each key
+//      orders exactly as the score would. The histogram of the first radix digit is built in the
+//      same loop;
+//   3. exact radix select of the budget-th largest key over the whole cluster: up to three
+//      digit passes (11, 11, 10 bits), stopping early once the threshold bin is taken whole.
+//      Each CTA histograms its own keys, every CTA sums one slice of the bins across the cluster
+//      through distributed shared memory, and every CTA locates the threshold digit from the
+//      slice totals;
 //   4. keys above the threshold are selected, keys equal to it are taken in position order up to
-//      the remaining quota (ties go to the lower position); a cluster-wide prefix of the per-CTA
-//      counts gives each CTA its output offset, so the index set comes out in ascending order.
+//      the remaining quota (ties go to the lower position); warp ballots give each key its rank
+//      inside the CTA and a cluster-wide prefix of the per-CTA counts gives the CTA's offset, so
+//      the index set comes out in ascending order.
 // When seq_len <= budget every position is selected without scoring.
 #include "common.cuh"
 
@@ -26,56 +33,50 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kUnroll = 8;  // 16-byte loads in flight per thread
 constexpr int kBins = 2048;
 
-__device__ __forceinline__ uint32_t warp_sum(uint32_t v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
+template <typename T>
+__device__ __forceinline__ T* remote(T* p, uint32_t rank) {
+  return static_cast<T*>(__cluster_map_shared_rank(p, rank));
 }
 
-// Exclusive prefix sum over the block (in thread order); also returns the block total.
-__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s_warp,
-                                                         uint32_t& total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t x = v;
+// fp32 whose value is (E4M3 code in the top byte of x) * 2^-120: sign stays in bit 31, the
+// exponent and mantissa bits move down by 4 into the low exponent / high mantissa positions.
+__device__ __forceinline__ float e4m3_top_byte_scaled(uint32_t x) {
+  return __uint_as_float((x & 0x80000000u) | ((x & 0x7F000000u) >> 4));
+}
+
+__device__ __forceinline__ float dot16(const uint4& v, const float* p) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc0 = fmaf(e4m3_top_byte_scaled(w[i] << 24), p[4 * i + 0], acc0);
+    acc1 = fmaf(e4m3_top_byte_scaled(w[i] << 16), p[4 * i + 1], acc1);
+    acc0 = fmaf(e4m3_top_byte_scaled(w[i] << 8), p[4 * i + 2], acc0);
+    acc1 = fmaf(e4m3_top_byte_scaled(w[i]), p[4 * i + 3], acc1);
+  }
+  return acc0 + acc1;
+}
+
+__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t x, int lane) {
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
-  if (lane == 31) s_warp[warp] = x;
-  __syncthreads();
-  uint32_t base = 0, tot = 0;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
-    const uint32_t t = s_warp[w];
-    base += (w < warp) ? t : 0u;
-    tot += t;
-  }
-  __syncthreads();
-  total = tot;
-  return base + x - v;
+  return x;
 }
 
 __device__ __forceinline__ uint32_t block_sum(uint32_t v, uint32_t* s_warp) {
-  uint32_t tot;
-  block_exclusive_scan(v, s_warp, tot);
-  return tot;
-}
-
-template <int R>
-__device__ __forceinline__ float dot16(const uint4& v, const float* p) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  float acc = 0.f;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 a = e4m3x2_to_f2((uint16_t)(w[i] & 0xFFFFu));
-    const float2 b = e4m3x2_to_f2((uint16_t)(w[i] >> 16));
-    acc = fmaf(a.x, p[4 * i + 0], acc);
-    acc = fmaf(a.y, p[4 * i + 1], acc);
-    acc = fmaf(b.x, p[4 * i + 2], acc);
-    acc = fmaf(b.y, p[4 * i + 3], acc);
-  }
-  return acc;
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) s_warp[warp] = v;
+  __syncthreads();
+  uint32_t t = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) t += s_warp[w];
+  __syncthreads();
+  return t;
 }
 
 template <int D, int R>
@@ -90,17 +91,19 @@ __global__ void __launch_bounds__(kThreads, 3)
   constexpr int TPG = 32 / PPT;   // tokens covered by one warp-wide load
   static_assert(PPT >= 1 && PPT <= 8, "rank");
 
-  extern __shared__ uint32_t dyn[];
-  uint32_t* s_key = dyn;                                      // [chunk]
-  int32_t* s_page = reinterpret_cast<int32_t*>(dyn + chunk);  // [chunk / page_size + 1]
+  extern __shared__ uint32_t score_dyn[];
+  uint32_t* s_key = score_dyn;                                      // [chunk]
+  int32_t* s_page = reinterpret_cast<int32_t*>(score_dyn + chunk);  // [chunk / page_size + 1]
   __shared__ float s_qbar[D];
   __shared__ float s_p[R];
   __shared__ uint32_t s_hist[kBins];
   __shared__ uint32_t s_red[kBins];
   __shared__ uint32_t s_tot;
-  __shared__ uint32_t s_cnt[2];
+  __shared__ uint32_t s_cnt[2];       // keys above / equal to the threshold in this CTA
   __shared__ uint32_t s_warp[kWarps];
+  __shared__ uint32_t s_wgt[kWarps], s_weq[kWarps];
   __shared__ int32_t s_info[4];
+  __shared__ float s_pmax;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int pair = blockIdx.y;
@@ -128,6 +131,7 @@ __global__ void __launch_bounds__(kThreads, 3)
   }
 
   // ---- 1. projected group-mean query --------------------------------------------------------
+  for (int i = tid; i < kBins; i += kThreads) s_hist[i] = 0u;
   const uint16_t* qh = q + ((int64_t)b * h_q + (int64_t)h * G) * D;
   for (int i = tid; i < D; i += kThreads) {
     float acc = 0.f;
@@ -162,18 +166,32 @@ __global__ void __launch_bounds__(kThreads, 3)
     s_page[i] = pg;
   }
   __syncthreads();
+  if (warp == 0) {
+    float m = 0.f;
+    for (int j = lane; j < R; j += 32) m = fmaxf(m, fabsf(s_p[j]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) s_pmax = m;
+  }
+  __syncthreads();
 
+  // p scaled by 2^(120 - E): the decoded codes carry a factor 2^-120, and E >= 0 keeps
+  // |p'| * 448 * R far below the float range. A power-of-two scale is exact, so the keys order
+  // exactly like the unscaled scores.
   float p_reg[16];
   {
+    const int ex = (int)((__float_as_uint(s_pmax) >> 23) & 0xFF) - 127;  // floor(log2 max|p|)
+    const int E = max(0, ex + 7);
+    const float scale = __uint_as_float((uint32_t)(127 + 120 - E) << 23);
     const int piece = lane % PPT;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) p_reg[e] = s_p[piece * 16 + e];
+    for (int e = 0; e < 16; ++e) p_reg[e] = s_p[piece * 16 + e] * scale;
   }
 
   // The scoring rows of the new token are written by the preceding store kernel.
   pdl_wait();
 
-  // ---- 3. scores -> keys in shared memory ----------------------------------------------------
+  // ---- 3. scores -> keys in shared memory, first-digit histogram -----------------------------
   const int n_groups = (n_local + TPG - 1) / TPG;
   const int64_t head_off = (int64_t)h * page_size * R;
   const int64_t page_bytes = (int64_t)h_kv * page_size * R;
@@ -198,10 +216,14 @@ __global__ void __launch_bounds__(kThreads, 3)
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      float s = dot16<R>(v[u], p_reg);
+      float s = dot16(v[u], p_reg);
 #pragma unroll
       for (int o = 1; o < PPT; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (piece == 0 && tok[u] >= 0) s_key[tok[u]] = score_key(s);
+      if (piece == 0 && tok[u] >= 0) {
+        const uint32_t key = score_key(s);
+        s_key[tok[u]] = key;
+        atomicAdd(&s_hist[key >> 21], 1u);
+      }
     }
   }
   __syncthreads();
@@ -209,26 +231,27 @@ __global__ void __launch_bounds__(kThreads, 3)
   // ---- 4. cluster-wide radix select of the budget-th largest key -----------------------------
   uint32_t prefix = 0, pmask = 0;
   int want = budget;  // rank (1-based, from the top) of the threshold among keys matching prefix
-  const uint32_t hist_addr = smem_u32(s_hist);
-  const uint32_t red_addr = smem_u32(s_red);
-  const uint32_t tot_addr = smem_u32(&s_tot);
+  uint32_t thr = 0;
+  bool resolved = false;
 #pragma unroll 1
-  for (int pass = 0; pass < 3; ++pass) {
+  for (int pass = 0; pass < 3 && !resolved; ++pass) {
     const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
     const int nb = pass == 2 ? 1024 : 2048;
-    for (int i = tid; i < nb; i += kThreads) s_hist[i] = 0u;
-    __syncthreads();
-    for (int i = tid; i < n_local; i += kThreads) {
-      const uint32_t key = s_key[i];
-      if ((key & pmask) == prefix) atomicAdd(&s_hist[(key >> shift) & (nb - 1)], 1u);
+    if (pass > 0) {
+      for (int i = tid; i < nb; i += kThreads) s_hist[i] = 0u;
+      __syncthreads();
+      for (int i = tid; i < n_local; i += kThreads) {
+        const uint32_t key = s_key[i];
+        if ((key & pmask) == prefix) atomicAdd(&s_hist[(key >> shift) & (nb - 1)], 1u);
+      }
     }
     cluster_sync();  // every histogram of the cluster is complete
     const int per = nb / (int)C;
     uint32_t part = 0;
     for (int j = tid; j < per; j += kThreads) {
+      const int bin = (int)crank * per + j;
       uint32_t sum = 0;
-      const uint32_t off = (uint32_t)((int)crank * per + j) * 4u;
-      for (uint32_t r = 0; r < C; ++r) sum += ld_cluster_u32(map_rank(hist_addr + off, r));
+      for (uint32_t r = 0; r < C; ++r) sum += *remote(&s_hist[bin], r);
       s_red[j] = sum;
       part += sum;
     }
@@ -236,113 +259,125 @@ __global__ void __launch_bounds__(kThreads, 3)
     if (tid == 0) s_tot = part;
     cluster_sync();  // every slice sum and slice total is published
     if (warp == 0) {
-      // slice totals, top slice first
+      // slice totals, top slice first; lane i holds slice C-1-i
       const uint32_t r_lane = C - 1 - (uint32_t)lane;
-      uint32_t t = (lane < (int)C) ? ld_cluster_u32(map_rank(tot_addr, r_lane)) : 0u;
-      uint32_t incl = t;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
+      const uint32_t t = (lane < (int)C) ? *remote(&s_tot, r_lane) : 0u;
+      const uint32_t incl = warp_incl_scan(t, lane);
       const uint32_t excl = incl - t;
       const unsigned hit = __ballot_sync(0xffffffffu, lane < (int)C && excl < (uint32_t)want &&
                                                           incl >= (uint32_t)want);
-      // lane index of the slice holding the threshold (always found for consistent counts; the
-      // fallback keeps every cluster address valid if the counts were ever inconsistent)
+      // (always found for consistent counts; the fallback keeps every address in the cluster)
       const int sl = hit ? __ffs(hit) - 1 : 0;
       const uint32_t above_slice = __shfl_sync(0xffffffffu, excl, sl);
       const uint32_t rank_sl = C - 1 - (uint32_t)sl;
+      const uint32_t* red = remote(s_red, rank_sl);
       // bins of that slice, highest first: lane i takes bins [per - (i+1)*bpl, per - i*bpl)
       const int bpl = (per + 31) / 32;
       const int hi = per - lane * bpl;
       const int lo = max(0, hi - bpl);
       uint32_t c = 0;
-      for (int j = lo; j < hi; ++j) c += ld_cluster_u32(map_rank(red_addr + (uint32_t)j * 4u, rank_sl));
-      uint32_t incl2 = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        uint32_t y = __shfl_up_sync(0xffffffffu, incl2, o);
-        if (lane >= o) incl2 += y;
-      }
+      for (int j = lo; j < hi; ++j) c += red[j];
+      const uint32_t incl2 = warp_incl_scan(c, lane);
       const uint32_t excl2 = above_slice + incl2 - c;
       const unsigned hit2 = __ballot_sync(0xffffffffu, hi > lo && excl2 < (uint32_t)want &&
                                                            excl2 + c >= (uint32_t)want);
       const int ln = hit2 ? __ffs(hit2) - 1 : 0;
       if (lane == 0 && (!hit || !hit2)) raise_flag(8u);
       if (lane == ln) {
-        uint32_t run = excl2;
+        uint32_t run = excl2, cnt = 0;
         int bin = lo;
         for (int j = hi - 1; j >= lo; --j) {
-          const uint32_t cj = ld_cluster_u32(map_rank(red_addr + (uint32_t)j * 4u, rank_sl));
-          if (run + cj >= (uint32_t)want) { bin = j; break; }
+          const uint32_t cj = red[j];
+          if (run + cj >= (uint32_t)want) { bin = j; cnt = cj; break; }
           run += cj;
         }
         s_info[0] = (int)rank_sl * per + bin;
         s_info[1] = (int)run;  // keys (matching the prefix) in strictly higher bins
+        s_info[2] = (int)cnt;  // keys in the threshold bin
       }
     }
     __syncthreads();
     const uint32_t digit = (uint32_t)s_info[0];
-    want -= s_info[1];
+    const int above = s_info[1], in_bin = s_info[2];
+    __syncthreads();
+    want -= above;
     prefix |= digit << shift;
     pmask |= (uint32_t)(nb - 1) << shift;
-    __syncthreads();
+    if (want == in_bin) {
+      // the whole threshold bin is selected: select every key >= its lowest key, no quota
+      thr = prefix - 1u;  // prefix > 0: keys of finite scores are >= 0x00800000
+      want = 0;
+      resolved = true;
+    } else if (pass == 2) {
+      thr = prefix;
+      resolved = true;
+    }
   }
-  const uint32_t thr = prefix;  // the budget-th largest key; `want` keys equal to it are taken
 
   // ---- 5. emit the index set in ascending position order -------------------------------------
-  const int kpt = (n_local + kThreads - 1) / kThreads;
-  const int r0 = min(n_local, tid * kpt), r1 = min(n_local, r0 + kpt);
+  // warp w owns positions [w*seg, (w+1)*seg) of the chunk, walked 32 at a time (lane = position)
+  const int seg = ((n_local + kWarps - 1) / kWarps + 31) & ~31;
+  const int w0 = min(n_local, warp * seg), w1 = min(n_local, w0 + seg);
   uint32_t n_gt = 0, n_eq = 0;
-  for (int i = r0; i < r1; ++i) {
-    const uint32_t key = s_key[i];
-    n_gt += key > thr;
-    n_eq += key == thr;
+  for (int i0 = w0; i0 < w1; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t key = i < w1 ? s_key[i] : 0u;
+    n_gt += __popc(__ballot_sync(0xffffffffu, i < w1 && key > thr));
+    n_eq += __popc(__ballot_sync(0xffffffffu, i < w1 && key == thr));
   }
-  uint32_t tot_gt, tot_eq;
-  block_exclusive_scan(n_gt, s_warp, tot_gt);
-  const uint32_t eq_base = block_exclusive_scan(n_eq, s_warp, tot_eq);
-  if (tid == 0) {
-    s_cnt[0] = tot_gt;
-    s_cnt[1] = tot_eq;
-  }
-  cluster_sync();  // per-CTA counts are published
-  if (tid == 0) {
-    const uint32_t cnt_addr = smem_u32(s_cnt);
-    uint32_t rem = (uint32_t)want, offset = 0, my_take = 0;
-    for (uint32_t r = 0; r < C; ++r) {
-      const uint32_t gt = ld_cluster_u32(map_rank(cnt_addr, r));
-      const uint32_t eq = ld_cluster_u32(map_rank(cnt_addr + 4u, r));
-      const uint32_t take = eq < rem ? eq : rem;
-      rem -= take;
-      if (r < crank) offset += gt + take;
-      if (r == crank) my_take = take;
-    }
-    s_info[2] = (int)offset;
-    s_info[3] = (int)my_take;
+  if (lane == 0) {
+    s_wgt[warp] = n_gt;
+    s_weq[warp] = n_eq;
   }
   __syncthreads();
-  const uint32_t offset = (uint32_t)s_info[2], my_take = (uint32_t)s_info[3];
-  uint32_t n_sel = 0;
-  {
-    uint32_t seen = eq_base;
-    for (int i = r0; i < r1; ++i) {
-      const uint32_t key = s_key[i];
-      if (key > thr) ++n_sel;
-      else if (key == thr) { n_sel += seen < my_take; ++seen; }
+  if (tid == 0) {
+    uint32_t g = 0, e = 0;
+    for (int w = 0; w < kWarps; ++w) {
+      g += s_wgt[w];
+      e += s_weq[w];
+    }
+    s_cnt[0] = g;
+    s_cnt[1] = e;
+  }
+  cluster_sync();  // per-CTA counts are published
+  if (warp == 0) {
+    // lane r < C holds CTA r's counts; the tie quota is handed out in rank (= position) order
+    const uint32_t gt = lane < (int)C ? *remote(&s_cnt[0], (uint32_t)lane) : 0u;
+    const uint32_t eq = lane < (int)C ? *remote(&s_cnt[1], (uint32_t)lane) : 0u;
+    const uint32_t eq_before = warp_incl_scan(eq, lane) - eq;
+    const uint32_t rem = (uint32_t)want > eq_before ? (uint32_t)want - eq_before : 0u;
+    const uint32_t take = eq < rem ? eq : rem;
+    const uint32_t sel = gt + take;
+    const uint32_t sel_before = warp_incl_scan(sel, lane) - sel;
+    if (lane == (int)crank) {
+      s_info[2] = (int)sel_before;
+      s_info[3] = (int)take;
     }
   }
-  uint32_t tot_sel;
-  uint32_t pos = offset + block_exclusive_scan(n_sel, s_warp, tot_sel);
-  {
-    uint32_t seen = eq_base;
-    for (int i = r0; i < r1; ++i) {
-      const uint32_t key = s_key[i];
-      bool take = key > thr;
-      if (key == thr) { take = seen < my_take; ++seen; }
-      if (take && pos < (uint32_t)budget) out_idx[pos++] = start + i;
-    }
+  __syncthreads();
+  const uint32_t cta_offset = (uint32_t)s_info[2], cta_take = (uint32_t)s_info[3];
+  // this warp's quota of equal keys and output offset within the CTA
+  uint32_t eq_before = 0, sel_before = 0;
+  for (int w = 0; w < warp; ++w) {
+    const uint32_t rem = cta_take > eq_before ? cta_take - eq_before : 0u;
+    const uint32_t tk = s_weq[w] < rem ? s_weq[w] : rem;
+    sel_before += s_wgt[w] + tk;
+    eq_before += s_weq[w];
+  }
+  uint32_t eq_seen = eq_before;
+  uint32_t pos = cta_offset + sel_before;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int i0 = w0; i0 < w1; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t key = i < w1 ? s_key[i] : 0u;
+    const bool is_eq = i < w1 && key == thr;
+    const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
+    const bool take = (i < w1 && key > thr) || (is_eq && eq_seen + __popc(eqm & lt) < cta_take);
+    const unsigned selm = __ballot_sync(0xffffffffu, take);
+    const uint32_t at = pos + __popc(selm & lt);
+    if (take && at < (uint32_t)budget) out_idx[at] = start + i;
+    pos += __popc(selm);
+    eq_seen += __popc(eqm);
   }
   if (crank == 0 && tid == 0) count[pair] = budget;
   pdl_trigger();
@@ -355,12 +390,8 @@ cudaError_t launch_t(const ScorePlan& plan, int pairs, bool pdl, cudaStream_t s,
                      int max_pages, const int32_t* seq_lens, int h_q, int h_kv, int64_t num_pages,
                      int page_size, int budget, int32_t* idx, int32_t* count) {
   auto kern = score_topk_kernel<D, R>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem);
+  cudaError_t e = configure_kernel((const void*)kern, (int)plan.smem, plan.cluster > 8);
   if (e != cudaSuccess) return e;
-  if (plan.cluster > 8) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(plan.cluster, pairs, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -412,11 +443,13 @@ cudaError_t launch_score_topk(const uint16_t* q, const float* basis, const uint8
   if (pairs == 0) return cudaSuccess;
   const ScorePlan plan = plan_score(pairs, max_pages * page_size, page_size);
   if (d == 128 && r == 32)
-    return score_detail::launch_t<128, 32>(plan, pairs, pdl, s, q, basis, score_cache, block_table, max_pages,
-                             seq_lens, h_q, h_kv, num_pages, page_size, budget, idx, count);
+    return score_detail::launch_t<128, 32>(plan, pairs, pdl, s, q, basis, score_cache, block_table,
+                                           max_pages, seq_lens, h_q, h_kv, num_pages, page_size,
+                                           budget, idx, count);
   if (d == 128 && r == 64)
-    return score_detail::launch_t<128, 64>(plan, pairs, pdl, s, q, basis, score_cache, block_table, max_pages,
-                             seq_lens, h_q, h_kv, num_pages, page_size, budget, idx, count);
+    return score_detail::launch_t<128, 64>(plan, pairs, pdl, s, q, basis, score_cache, block_table,
+                                           max_pages, seq_lens, h_q, h_kv, num_pages, page_size,
+                                           budget, idx, count);
   return cudaErrorInvalidValue;
 }
 

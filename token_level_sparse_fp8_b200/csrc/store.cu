@@ -117,7 +117,7 @@ cudaError_t launch_store_t(dim3 grid, size_t smem, cudaStream_t s, const uint16_
                            int64_t head_stride, const int32_t* block_table, int max_pages,
                            const int32_t* seq_lens) {
   auto kern = store_kernel<D, R, DECODE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = configure_kernel((const void*)kern, (int)smem, false);
   if (e != cudaSuccess) return e;
   kern<<<grid, kStoreThreads, smem, s>>>(k, k_stride_t, slot_mapping, t, h_kv, basis, score_cache,
                                          num_pages, page_size, tpb, v_new, k_cache, v_cache,
