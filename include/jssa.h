@@ -61,7 +61,8 @@ enum jssa_status {
   JSSA_ERR_UNSUPPORTED = -3,  /* no kernel instance for (d, r, G) or size beyond the limits */
   JSSA_ERR_ALIGN = -4,        /* a pointer or stride breaks the 16-byte alignment rule */
   JSSA_ERR_WORKSPACE = -5,    /* workspace NULL or smaller than jssa_workspace_size */
-  JSSA_ERR_DEVICE = -6        /* no usable CUDA device / device query failed */
+  JSSA_ERR_DEVICE = -6,       /* no usable CUDA device / device query failed */
+  JSSA_ERR_SCRATCH_LIMIT = -7 /* sizes need more than the allocation-free entry point's scratch */
 };
 
 /* Device error flags (bitwise OR), read with jssa_device_error. */
@@ -201,6 +202,36 @@ JSSA_API int jssa_decode(const jssa_bf16* q, const jssa_bf16* k_new, const jssa_
                 int64_t num_pages, int page_size, int budget, float softmax_scale,
                 int32_t* idx, int32_t* count, jssa_bf16* out, void* ws, size_t ws_bytes,
                 jssa_stream_t stream);
+
+/* Size of the device scratch array used by jssa_indexed_attend_noalloc (per GPU, bytes). */
+#define JSSA_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/*
+ * Allocation-free indexed attention. The paper has no counterpart to this entry point: it is a
+ * library convenience. It computes exactly what jssa_indexed_attend computes, with the same
+ * arguments except the workspace, for callers that cannot allocate or pass device memory of
+ * their own: an inference runtime that owns all device memory through its own pool and gives
+ * plug-ins no allocator, a latency-critical loop that must avoid cudaMalloc (which synchronises
+ * the device), or a host program that only links this C ABI and has no allocator.
+ * Instead of a workspace, the split-K scratch (ticket counters and fp32 partials) lives in a
+ * fixed device array of JSSA_NOALLOC_SCRATCH_BYTES inside the library; every GPU that loads the
+ * library holds that array until the process exits. Sizes whose scratch would exceed it return
+ * JSSA_ERR_SCRATCH_LIMIT without launching (jssa_workspace_size(JSSA_FN_INDEXED_ATTEND, ...)
+ * gives the requirement). The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that first call before
+ * any stream capture. The call itself allocates nothing (it clears the ticket counters with
+ * cudaMemsetAsync on `stream`, then launches). All calls on a device share the array and it
+ * keeps the last call's contents: calls that overlap on the GPU (different streams or threads
+ * of the same process) race and must be serialised by the caller.
+ */
+JSSA_API int jssa_indexed_attend_noalloc(const jssa_bf16* q, const jssa_bf16* k_cache,
+                                         const jssa_bf16* v_cache, int64_t kv_page_stride,
+                                         int64_t kv_slot_stride, int64_t kv_head_stride,
+                                         const int32_t* block_table, int max_pages,
+                                         const int32_t* idx, const int32_t* count, int batch,
+                                         int h_q, int h_kv, int d, int budget, int64_t num_pages,
+                                         int page_size, float softmax_scale, jssa_bf16* out,
+                                         jssa_stream_t stream);
 
 /*
  * Read (and with clear != 0, reset) the device error word of the current device. Synchronises

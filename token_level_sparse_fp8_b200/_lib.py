@@ -23,6 +23,7 @@ STATUS_NAMES = {
     -4: "JSSA_ERR_ALIGN",
     -5: "JSSA_ERR_WORKSPACE",
     -6: "JSSA_ERR_DEVICE",
+    -7: "JSSA_ERR_SCRATCH_LIMIT",
 }
 FN_SCORE_TOPK, FN_INDEXED_ATTEND, FN_DENSE_DECODE, FN_DECODE, FN_COMPUTE_BASIS = 1, 2, 3, 4, 5
 DEVERR_PAGE, DEVERR_INDEX, DEVERR_SEQLEN = 1, 2, 4
@@ -45,6 +46,8 @@ SIGNATURES = {
     "jssa_decode": (c_int, [P, P, P, P, P, c_int64, c_int64, c_int64, P, P, P, c_int, P, c_int, c_int,
                             c_int, c_int, c_int, c_int64, c_int, c_int, c_float, P, P, P, P, c_size_t,
                             P]),
+    "jssa_indexed_attend_noalloc": (c_int, [P, P, P, c_int64, c_int64, c_int64, P, c_int, P, P, c_int,
+                                            c_int, c_int, c_int, c_int, c_int64, c_int, c_float, P, P]),
     "jssa_device_error": (c_int, [c_uint32_p, c_int, P]),
 }
 

@@ -108,6 +108,7 @@ const char* jssa_status_string(int status) {
     case JSSA_ERR_ALIGN: return "pointer or stride not 16-byte aligned";
     case JSSA_ERR_WORKSPACE: return "workspace missing or too small";
     case JSSA_ERR_DEVICE: return "no usable CUDA device";
+    case JSSA_ERR_SCRATCH_LIMIT: return "sizes exceed the static scratch of the allocation-free entry point";
     default: break;
   }
   if (status > 0) return cudaGetErrorString((cudaError_t)status);

@@ -6,3 +6,4 @@
 #include "attend.cu"
 #include "calib.cu"
 #include "basis.cu"
+#include "noalloc.cu"
