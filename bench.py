@@ -428,13 +428,15 @@ def run_jssa(args):
     # per-kernel device times (same configuration, each kernel launched alone)
     idx, count = layer.idx, layer.count
 
+    ws_score, ws_attend = J.Workspace(dev), J.Workspace(dev)
+
     def score_only(i):
         J.score_topk(qs[i % nq], layer.basis, layer.score_cache, layer.block_table, layer.seq_lens,
-                     w.budget, idx, count)
+                     w.budget, idx, count, ws_score)
 
     def attend_only(i):
         J.indexed_attend(qs[i % nq], layer.k_cache, layer.v_cache, layer.block_table, idx, count,
-                         layer.scale, out, layer.ws)
+                         layer.scale, out, ws_attend)
 
     t_score, n_score = timed_graph(score_only, args.steps, args.warmup, stream, barrier, nq)
     t_score = max_over_ranks(t_score) / n_score

@@ -24,7 +24,7 @@
  *   cache[page*kv_page_stride + slot*kv_slot_stride + head*kv_head_stride + x]; strides are in
  *   elements, the head dimension is contiguous. Logical position t of sequence b lives in page
  *   block_table[b*max_pages + t/page_size], slot t%page_size. block_table is int32
- *   [batch, max_pages], seq_lens int32 [batch].
+ *   [batch, max_pages], seq_lens int32 [batch]. page_size is a power of two.
  * - Scoring cache: uint8 E4M3 codes laid out [num_pages, h_kv, page_size, r] (one contiguous
  *   run of page_size*r bytes per page and KV head), same page numbering as the KV cache.
  * - Basis: float32 [h_kv, r, d], rows orthonormal (output of jssa_compute_basis).
@@ -90,14 +90,19 @@ JSSA_API int jssa_version(void);
 
 /*
  * Bytes of device workspace the entry point `fn` needs for these sizes (written to *bytes; 0
- * means none). max_seq_len bounds every seq_len (use max_pages*page_size); budget is ignored
- * by the dense decode and by the basis. The split-K attention entry points keep a per-(sequence,
- * KV head) ticket counter in the workspace: a workspace must be cleared once with
- * jssa_workspace_init before its first use; the kernels leave the counters at zero on exit.
- * Calls that share one workspace must not overlap on the GPU.
+ * means none). max_pages and page_size are the block-table width and page size the call will
+ * get (every seq_len is at most max_pages*page_size); budget is the token budget B, except for
+ * JSSA_FN_DENSE_DECODE where it carries the call's window (<= 0: full context); the basis
+ * ignores it. Score + top-B keeps its candidate keys and positions in the workspace. The
+ * split-K attention entry points keep a per-(sequence, KV head) ticket counter at the start of
+ * theirs: for jssa_indexed_attend and jssa_dense_decode those counters must be zero when the call
+ * starts -- clear the workspace with jssa_workspace_init before its first use and again after it
+ * served another entry point or a larger batch*h_kv (the kernels leave the counters at zero on
+ * exit). jssa_decode clears its counters itself. Calls that share one workspace must not overlap
+ * on the GPU.
  */
-JSSA_API int jssa_workspace_size(int fn, int batch, int h_q, int h_kv, int d, int max_seq_len, int budget,
-                        size_t* bytes);
+JSSA_API int jssa_workspace_size(int fn, int batch, int h_q, int h_kv, int d, int max_pages,
+                                 int page_size, int budget, size_t* bytes);
 
 /* Zero `ws_bytes` bytes of workspace on `stream` (cudaMemsetAsync). */
 JSSA_API int jssa_workspace_init(void* ws, size_t ws_bytes, jssa_stream_t stream);
@@ -147,9 +152,9 @@ JSSA_API int jssa_store(const jssa_bf16* k, int64_t k_stride_t, const int64_t* s
  * heads of h), s_t = sum_j dec(c_tj) p_j for every t < seq_len (fp32), and the index set of the
  * min(budget, seq_len) largest s_t, ties to the lower position, written ascending.
  * JSSA summary, eq. (1) and section 3.1 steps 1-2; JSSA README, section 4 (jssa_budget).
- * One thread-block cluster per (sequence, KV head) keeps all scores in shared memory and runs a
- * radix select over the cluster; nothing but idx/count is written to memory.
- * q: bf16 [batch, h_q, d] contiguous. ws may be NULL (size 0).
+ * One thread-block cluster per (sequence, KV head) keeps all scores in shared memory; only the
+ * keys that can still be selected (a few per selected token) go through the workspace.
+ * q: bf16 [batch, h_q, d] contiguous. ws: >= jssa_workspace_size(JSSA_FN_SCORE_TOPK).
  */
 JSSA_API int jssa_score_topk(const jssa_bf16* q, const float* basis, const uint8_t* score_cache,
                     const int32_t* block_table, int max_pages, const int32_t* seq_lens, int batch,
@@ -191,8 +196,7 @@ JSSA_API int jssa_dense_decode(const jssa_bf16* q, const jssa_bf16* k_cache, con
  * are chained on `stream` with programmatic dependent launch and no host synchronisation.
  * JSSA summary, section 3.1; JSSA README, paper-to-code map (_sparse_decode_forward).
  * k_new, v_new: bf16 [batch, h_kv, d] contiguous (or both NULL). idx/count: outputs as in
- * jssa_score_topk. ws: >= jssa_workspace_size(JSSA_FN_DECODE), cleared once by
- * jssa_workspace_init.
+ * jssa_score_topk. ws: >= jssa_workspace_size(JSSA_FN_DECODE); no clearing needed.
  */
 JSSA_API int jssa_decode(const jssa_bf16* q, const jssa_bf16* k_new, const jssa_bf16* v_new,
                 jssa_bf16* k_cache, jssa_bf16* v_cache, int64_t kv_page_stride,

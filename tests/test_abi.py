@@ -60,12 +60,17 @@ def test_status_strings_and_version(lib):
 
 def test_workspace_sizes_are_host_only(lib):
     from token_level_sparse_fp8_b200 import api, _lib
-    assert api.workspace_size(_lib.FN_COMPUTE_BASIS, 0, 1, 8, 128, 0, 0) == 8 * 128 * 128 * 8
-    n = api.workspace_size(_lib.FN_DECODE, 16, 32, 8, 128, 131072, 2048)
-    assert n > 0
-    assert api.workspace_size(_lib.FN_DENSE_DECODE, 16, 32, 8, 128, 131072, 0) > n
+    assert api.workspace_size(_lib.FN_COMPUTE_BASIS, 0, 1, 8, 128, 0, 1, 0) == 8 * 128 * 128 * 8
+    n = api.workspace_size(_lib.FN_DECODE, 16, 32, 8, 128, 8192, 16, 2048)
+    n_score = api.workspace_size(_lib.FN_SCORE_TOPK, 16, 32, 8, 128, 8192, 16, 2048)
+    n_attend = api.workspace_size(_lib.FN_INDEXED_ATTEND, 16, 32, 8, 128, 8192, 16, 2048)
+    assert n >= n_score + n_attend > 0
+    assert n_score >= 16 * 8 * 131072 * 8  # candidate keys + positions for every position
+    full = api.workspace_size(_lib.FN_DENSE_DECODE, 16, 32, 8, 128, 8192, 16, 0)
+    windowed = api.workspace_size(_lib.FN_DENSE_DECODE, 16, 32, 8, 128, 8192, 16, 1024)
+    assert full > windowed
     with pytest.raises(_lib.JSSAError):
-        api.workspace_size(_lib.FN_DECODE, 1, 30, 8, 128, 1024, 64)  # h_q not a multiple of h_kv
+        api.workspace_size(_lib.FN_DECODE, 1, 30, 8, 128, 64, 16, 64)  # h_q not a multiple of h_kv
 
 
 def test_argument_checks_reject_before_launch(lib):

@@ -51,7 +51,8 @@ def test_noalloc_matches_regular_entry_point_twice():
     stream = torch.cuda.current_stream(dev).cuda_stream
 
     # the regular entry point with a caller-provided workspace
-    nbytes = api.workspace_size(_lib.FN_INDEXED_ATTEND, batch, h_q, h_kv, d, 0, budget)
+    nbytes = api.workspace_size(_lib.FN_INDEXED_ATTEND, batch, h_q, h_kv, d, bt.shape[1], page_size,
+                                budget)
     assert 0 < nbytes <= 4 << 20
     ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
     out_ref = torch.empty_like(q)

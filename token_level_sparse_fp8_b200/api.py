@@ -15,8 +15,8 @@ from typing import Optional, Tuple
 import torch
 
 from . import _lib
-from ._lib import (FN_COMPUTE_BASIS, FN_DECODE, FN_DENSE_DECODE, FN_INDEXED_ATTEND, JSSAError,
-                   call)
+from ._lib import (FN_COMPUTE_BASIS, FN_DECODE, FN_DENSE_DECODE, FN_INDEXED_ATTEND,
+                   FN_SCORE_TOPK, JSSAError, call)
 
 __all__ = [
     "JSSAError", "workspace_size", "Workspace", "calibrate_accumulate", "compute_basis",
@@ -56,10 +56,11 @@ def kv_strides(cache: torch.Tensor) -> Tuple[int, int, int]:
     return cache.stride(0), cache.stride(1), cache.stride(2)
 
 
-def workspace_size(fn: int, batch: int, h_q: int, h_kv: int, d: int, max_seq_len: int,
-                   budget: int) -> int:
+def workspace_size(fn: int, batch: int, h_q: int, h_kv: int, d: int, max_pages: int,
+                   page_size: int, budget: int) -> int:
     out = ctypes.c_size_t(0)
-    call("jssa_workspace_size", fn, batch, h_q, h_kv, d, max_seq_len, budget, ctypes.byref(out))
+    call("jssa_workspace_size", fn, batch, h_q, h_kv, d, max_pages, page_size, budget,
+         ctypes.byref(out))
     return int(out.value)
 
 
@@ -82,10 +83,12 @@ class Workspace:
 _default_ws = {}
 
 
-def _ws(device: torch.device, ws: Optional[Workspace]) -> Workspace:
+def _ws(device: torch.device, ws: Optional[Workspace], fn: int) -> Workspace:
+    """The caller's workspace, else a default one per (device, stream, entry point): the split-K
+    ticket counters of one entry point must not be overwritten by another's scratch."""
     if ws is not None:
         return ws
-    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    key = (device.index, torch.cuda.current_stream(device).cuda_stream, fn)
     if key not in _default_ws:
         _default_ws[key] = Workspace(device)
     return _default_ws[key]
@@ -122,7 +125,7 @@ def compute_basis(gram_q: torch.Tensor, gram_k: torch.Tensor, rank: int,
     dev = gram_q.device
     basis = torch.empty((h_kv, rank, d), dtype=torch.float32, device=dev)
     eig = torch.empty((h_kv, d), dtype=torch.float64, device=dev) if with_eigvals else None
-    nbytes = workspace_size(FN_COMPUTE_BASIS, 0, 1, h_kv, d, 0, 0)
+    nbytes = workspace_size(FN_COMPUTE_BASIS, 0, 1, h_kv, d, 0, 1, 0)
     ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     call("jssa_compute_basis", gram_q.data_ptr(), gram_k.data_ptr(), h_kv, d, rank, basis.data_ptr(),
          _ptr(eig), ws.data_ptr(), nbytes, _stream(dev))
@@ -165,7 +168,8 @@ def store(k: torch.Tensor, slot_mapping: torch.Tensor, basis: torch.Tensor,
 
 def score_topk(q: torch.Tensor, basis: torch.Tensor, score_cache: torch.Tensor,
                block_table: torch.Tensor, seq_lens: torch.Tensor, budget: int,
-               idx: Optional[torch.Tensor] = None, count: Optional[torch.Tensor] = None):
+               idx: Optional[torch.Tensor] = None, count: Optional[torch.Tensor] = None,
+               ws: Optional[Workspace] = None):
     """Index sets ``idx`` (int32 ``[batch, h_kv, budget]``, ascending, -1 padded) and ``count``."""
     for t, n, dt in ((q, "q", torch.bfloat16), (basis, "basis", torch.float32),
                      (score_cache, "score_cache", torch.uint8), (block_table, "block_table", torch.int32),
@@ -178,9 +182,12 @@ def score_topk(q: torch.Tensor, basis: torch.Tensor, score_cache: torch.Tensor,
         idx = torch.empty((batch, h_kv, budget), dtype=torch.int32, device=q.device)
     if count is None:
         count = torch.empty((batch, h_kv), dtype=torch.int32, device=q.device)
+    max_pages = block_table.shape[1]
+    w = _ws(q.device, ws, FN_SCORE_TOPK)
+    p, n = w.get(workspace_size(FN_SCORE_TOPK, batch, h_q, h_kv, d, max_pages, page_size, budget))
     call("jssa_score_topk", q.data_ptr(), basis.data_ptr(), score_cache.data_ptr(),
-         block_table.data_ptr(), block_table.shape[1], seq_lens.data_ptr(), batch, h_q, h_kv, d, r,
-         num_pages, page_size, budget, idx.data_ptr(), count.data_ptr(), None, 0, _stream(q.device))
+         block_table.data_ptr(), max_pages, seq_lens.data_ptr(), batch, h_q, h_kv, d, r,
+         num_pages, page_size, budget, idx.data_ptr(), count.data_ptr(), p, n, _stream(q.device))
     return idx, count
 
 
@@ -203,8 +210,9 @@ def indexed_attend(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
     budget = idx.shape[2]
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     out = torch.empty_like(q) if out is None else out
-    w = _ws(q.device, ws)
-    p, n = w.get(workspace_size(FN_INDEXED_ATTEND, batch, h_q, h_kv, d, 0, budget))
+    w = _ws(q.device, ws, FN_INDEXED_ATTEND)
+    p, n = w.get(workspace_size(FN_INDEXED_ATTEND, batch, h_q, h_kv, d, block_table.shape[1],
+                                page_size, budget))
     call("jssa_indexed_attend", q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), *strides,
          block_table.data_ptr(), block_table.shape[1], idx.data_ptr(), count.data_ptr(), batch, h_q,
          h_kv, d, budget, num_pages, page_size, scale, out.data_ptr(), p, n, _stream(q.device))
@@ -227,11 +235,10 @@ def dense_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
     if kv_strides(v_cache) != strides:
         raise ValueError("K and V caches must share one layout")
     max_pages = block_table.shape[1]
-    span = max_pages * page_size if window <= 0 else min(window, max_pages * page_size)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     out = torch.empty_like(q) if out is None else out
-    w = _ws(q.device, ws)
-    p, n = w.get(workspace_size(FN_DENSE_DECODE, batch, h_q, h_kv, d, span, 0))
+    w = _ws(q.device, ws, FN_DENSE_DECODE)
+    p, n = w.get(workspace_size(FN_DENSE_DECODE, batch, h_q, h_kv, d, max_pages, page_size, window))
     call("jssa_dense_decode", q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), *strides,
          block_table.data_ptr(), max_pages, seq_lens.data_ptr(), batch, h_q, h_kv, d, num_pages,
          page_size, window, scale, out.data_ptr(), p, n, _stream(q.device))
@@ -269,8 +276,9 @@ def decode(q: torch.Tensor, k_new: Optional[torch.Tensor], v_new: Optional[torch
         idx = torch.empty((batch, h_kv, budget), dtype=torch.int32, device=q.device)
     if count is None:
         count = torch.empty((batch, h_kv), dtype=torch.int32, device=q.device)
-    w = _ws(q.device, ws)
-    p, n = w.get(workspace_size(FN_DECODE, batch, h_q, h_kv, d, 0, budget))
+    w = _ws(q.device, ws, FN_DECODE)
+    p, n = w.get(workspace_size(FN_DECODE, batch, h_q, h_kv, d, block_table.shape[1], page_size,
+                                budget))
     call("jssa_decode", q.data_ptr(), _ptr(k_new), _ptr(v_new), k_cache.data_ptr(),
          v_cache.data_ptr(), *strides, score_cache.data_ptr(), basis.data_ptr(),
          block_table.data_ptr(), block_table.shape[1], seq_lens.data_ptr(), batch, h_q, h_kv, d, r,
@@ -305,7 +313,8 @@ class PagedLayer:
         batch = block_table.shape[0]
         self.idx = torch.empty((batch, h_kv, budget), dtype=torch.int32, device=k_cache.device)
         self.count = torch.empty((batch, h_kv), dtype=torch.int32, device=k_cache.device)
-        self.ws = Workspace(k_cache.device)
+        self.ws = Workspace(k_cache.device)        # decode steps
+        self.ws_dense = Workspace(k_cache.device)  # dense baseline
 
     def prefill_scores(self, chunk_pages: int = 4096) -> None:
         """Store the scoring code of every cached position (all slots of every page)."""
@@ -324,4 +333,4 @@ class PagedLayer:
 
     def dense(self, q, out=None, window=-1):
         return dense_decode(q, self.k_cache, self.v_cache, self.block_table, self.seq_lens,
-                            self.scale, window, out, self.ws)
+                            self.scale, window, out, self.ws_dense)

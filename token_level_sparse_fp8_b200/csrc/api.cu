@@ -69,6 +69,7 @@ int check_heads(int h_q, int h_kv) {
 
 int check_paging(int max_pages, int64_t num_pages, int page_size) {
   if (max_pages <= 0 || num_pages <= 0 || page_size <= 0) return JSSA_ERR_SHAPE;
+  if (page_size & (page_size - 1)) return JSSA_ERR_UNSUPPORTED;  // powers of two only
   if ((int64_t)max_pages * page_size > (int64_t)INT32_MAX / 2) return JSSA_ERR_SHAPE;
   return JSSA_OK;
 }
@@ -85,7 +86,12 @@ int check_kv(const void* k_cache, const void* v_cache, int64_t page_stride, int6
   return JSSA_OK;
 }
 
-size_t score_ws_bytes() { return 0; }
+size_t score_ws_bytes(int batch, int h_kv, int max_seq_len, int page_size) {
+  if (batch * h_kv == 0) return 0;
+  return jssa::plan_score(batch * h_kv, max_seq_len, page_size).ws_bytes;
+}
+
+inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 jssa::AttendPlan attend_plan_indexed(int batch, int h_q, int h_kv, int d, int budget) {
   return jssa::plan_attend(batch * h_kv, budget, h_q / h_kv, d);
@@ -117,11 +123,14 @@ const char* jssa_status_string(int status) {
 
 int jssa_version(void) { return kVersion; }
 
-int jssa_workspace_size(int fn, int batch, int h_q, int h_kv, int d, int max_seq_len, int budget,
-                        size_t* bytes) {
+int jssa_workspace_size(int fn, int batch, int h_q, int h_kv, int d, int max_pages,
+                        int page_size, int budget, size_t* bytes) {
   if (!bytes) return JSSA_ERR_NULL;
   *bytes = 0;
-  if (batch < 0 || d <= 0 || max_seq_len < 0) return JSSA_ERR_SHAPE;
+  if (batch < 0 || d <= 0 || max_pages < 0 || page_size <= 0) return JSSA_ERR_SHAPE;
+  if (page_size & (page_size - 1)) return JSSA_ERR_UNSUPPORTED;
+  if ((int64_t)max_pages * page_size > (int64_t)INT32_MAX / 2) return JSSA_ERR_SHAPE;
+  const int max_seq_len = max_pages * page_size;
   if (fn == JSSA_FN_COMPUTE_BASIS) {
     if (h_kv <= 0) return JSSA_ERR_SHAPE;
     *bytes = (size_t)h_kv * d * d * sizeof(double);
@@ -131,16 +140,22 @@ int jssa_workspace_size(int fn, int batch, int h_q, int h_kv, int d, int max_seq
   if (st) return st;
   switch (fn) {
     case JSSA_FN_SCORE_TOPK:
-      *bytes = score_ws_bytes();
+      *bytes = score_ws_bytes(batch, h_kv, max_seq_len, page_size);
       return JSSA_OK;
     case JSSA_FN_INDEXED_ATTEND:
-    case JSSA_FN_DECODE:
       if (budget <= 0) return JSSA_ERR_SHAPE;
       *bytes = attend_plan_indexed(batch, h_q, h_kv, d, budget).ws_bytes;
       return JSSA_OK;
-    case JSSA_FN_DENSE_DECODE:
-      *bytes = attend_plan_dense(batch, h_q, h_kv, d, max_seq_len).ws_bytes;
+    case JSSA_FN_DECODE:
+      if (budget <= 0) return JSSA_ERR_SHAPE;
+      *bytes = align256(attend_plan_indexed(batch, h_q, h_kv, d, budget).ws_bytes) +
+               score_ws_bytes(batch, h_kv, max_seq_len, page_size);
       return JSSA_OK;
+    case JSSA_FN_DENSE_DECODE: {
+      const int span = (budget > 0 && budget < max_seq_len) ? budget : max_seq_len;
+      *bytes = attend_plan_dense(batch, h_q, h_kv, d, span).ws_bytes;
+      return JSSA_OK;
+    }
     default:
       return JSSA_ERR_SHAPE;
   }
@@ -185,6 +200,7 @@ int jssa_store(const jssa_bf16* k, int64_t k_stride_t, const int64_t* slot_mappi
                int h_kv, int d, int r, const float* basis, uint8_t* score_cache,
                int64_t num_pages, int page_size, jssa_stream_t stream) {
   if (t < 0 || h_kv <= 0 || num_pages <= 0 || page_size <= 0) return JSSA_ERR_SHAPE;
+  if (page_size & (page_size - 1)) return JSSA_ERR_UNSUPPORTED;
   if (r <= 0 || r > d) return JSSA_ERR_SHAPE;
   if (!supported_dr(d, r)) return JSSA_ERR_UNSUPPORTED;
   if (t == 0) return JSSA_OK;
@@ -218,14 +234,15 @@ int jssa_score_topk(const jssa_bf16* q, const float* basis, const uint8_t* score
                     int h_q, int h_kv, int d, int r, int64_t num_pages, int page_size, int budget,
                     int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
                     jssa_stream_t stream) {
-  (void)ws;
-  (void)ws_bytes;
   int st = check_score_args(q, basis, score_cache, block_table, max_pages, seq_lens, batch, h_q,
                             h_kv, d, r, num_pages, page_size, budget, idx, count);
   if (st || batch == 0) return st;
+  const size_t need = score_ws_bytes(batch, h_kv, max_pages * page_size, page_size);
+  if (!ws || ws_bytes < need) return JSSA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return JSSA_ERR_ALIGN;
   return cuda_status(jssa::launch_score_topk(q, basis, score_cache, block_table, max_pages,
                                              seq_lens, batch, h_q, h_kv, d, r, num_pages,
-                                             page_size, budget, idx, count, false,
+                                             page_size, budget, idx, count, ws, nullptr, false,
                                              as_stream(stream)));
 }
 
@@ -315,8 +332,14 @@ int jssa_decode(const jssa_bf16* q, const jssa_bf16* k_new, const jssa_bf16* v_n
   if ((k_new == nullptr) != (v_new == nullptr)) return JSSA_ERR_NULL;
   if (k_new && (!aligned16(k_new) || !aligned16(v_new))) return JSSA_ERR_ALIGN;
   const jssa::AttendPlan plan = attend_plan_indexed(batch, h_q, h_kv, d, budget);
-  if (plan.ws_bytes && (!ws || ws_bytes < plan.ws_bytes)) return JSSA_ERR_WORKSPACE;
-  if (plan.ws_bytes && !aligned16(ws)) return JSSA_ERR_ALIGN;
+  // workspace: [attention tickets + partials | score candidates]; the score kernel clears the
+  // tickets of every (sequence, KV head) before the attention runs, so no prior clearing is needed
+  const size_t score_ws = score_ws_bytes(batch, h_kv, max_pages * page_size, page_size);
+  const size_t attend_bytes = align256(plan.ws_bytes);
+  if (!ws || ws_bytes < attend_bytes + score_ws) return JSSA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return JSSA_ERR_ALIGN;
+  void* attend_ws = ws;
+  void* cand_ws = static_cast<uint8_t*>(ws) + attend_bytes;
   cudaStream_t s = as_stream(stream);
   bool pdl = false;
   if (k_new) {
@@ -329,7 +352,9 @@ int jssa_decode(const jssa_bf16* q, const jssa_bf16* k_new, const jssa_bf16* v_n
   }
   cudaError_t e = jssa::launch_score_topk(q, basis, score_cache, block_table, max_pages, seq_lens,
                                           batch, h_q, h_kv, d, r, num_pages, page_size, budget,
-                                          idx, count, pdl, s);
+                                          idx, count, cand_ws,
+                                          plan.ws_bytes ? static_cast<int*>(attend_ws) : nullptr,
+                                          pdl, s);
   if (e != cudaSuccess) return (int)e;
   AttendArgs a = {};
   a.q = q; a.k_cache = k_cache; a.v_cache = v_cache;
@@ -337,7 +362,7 @@ int jssa_decode(const jssa_bf16* q, const jssa_bf16* k_new, const jssa_bf16* v_n
   a.block_table = block_table; a.max_pages = max_pages; a.idx = idx; a.count = count;
   a.batch = batch; a.h_q = h_q; a.h_kv = h_kv; a.d = d; a.budget = budget;
   a.num_pages = num_pages; a.page_size = page_size; a.scale = softmax_scale; a.out = out;
-  a.ws = ws;
+  a.ws = plan.ws_bytes ? attend_ws : nullptr;
   return cuda_status(jssa::launch_attend(a, true, plan, true, s));
 }
 

@@ -5,15 +5,20 @@
 // of its positions -- a slice of the index set (indexed mode) or of [lo, seq_len) (dense mode).
 //   * Row addresses: the CTA first turns each of its positions into a 64-bit element offset
 //     (page-table lookup, bounds checked) kept in shared memory.
-//   * Each of the 4 warps walks its own 16-token tiles with a 3-stage cp.async pipeline: the K
-//     and V rows (256 B each at d = 128) are copied straight from their paged locations into a
-//     swizzled shared-memory tile -- no staging buffer in global memory.
-//   * The G query heads of the KV head form the rows of an m16 tensor-core tile:
-//     S = Q K^T and O += P V are mma.sync m16n8k16 (bf16 in, fp32 accumulate); P is split into a
-//     bf16 high and low part so the probabilities keep ~16 significant bits.
+//   * Each of the 4 warps walks its own 16-token tiles. A tile's K and V rows (256 B each at
+//     d = 128) are loaded with 16-byte non-allocating loads straight from their paged locations
+//     into registers -- no staging buffer in global or shared memory -- and the next tile's loads
+//     are in flight while the current tile is computed.
+//   * Tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate) with the 16 tokens as the M
+//     rows and the G <= 8 query heads of the KV head as the N columns: S^T = K Q^T, then
+//     O^T += V^T P^T. The head dimension is visited in a fixed permuted order (the same for q and
+//     k, and undone when O is written) so that every lane's fragment elements are contiguous in
+//     the row: a lane reads 64 B of each of its two K rows and 32 B of each of its four V rows.
+//     P^T reaches the B-operand layout with movmatrix, split into a bf16 high and low part so the
+//     probabilities keep ~16 significant bits.
 //   * Online softmax in the log2 domain; warps merge in shared memory; CTAs of one (b, h) merge
-//     through a float partial (m, l, o) in the workspace, the last CTA to take the ticket
-//     combines them, writes the bf16 output and resets the ticket.
+//     through fp32 partials (m, l, o) in the workspace, the last CTA to take the ticket combines
+//     them, writes the bf16 output and resets the ticket.
 #include <float.h>
 
 #include "common.cuh"
@@ -24,48 +29,88 @@ namespace attend_detail {
 
 constexpr int kWarps = kAttendWarps;
 constexpr int kThreads = kWarps * 32;
-constexpr int kStages = 3;
 constexpr int kTile = kAttendTile;
 constexpr int kMaxChunk = 1024;  // positions per CTA (row offsets kept in shared memory)
 
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t r;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+  return r;
+}
+
 template <int D>
-struct Smem {
-  static constexpr int kRowBytes = D * 2;
-  static constexpr int kTileBytes = kTile * kRowBytes;            // one K (or V) tile
-  static constexpr int kStageBytes = 2 * kTileBytes;              // K + V
-  static constexpr int kWarpBytes = kStages * kStageBytes;
-  static constexpr int kPipeBytes = kWarps * kWarpBytes;
-  static constexpr int kOffBytes = kMaxChunk * 8;
-  static constexpr int kTotal = kPipeBytes + kOffBytes;
-  // merge scratch (aliases the pipeline buffers after the main loop)
-  static constexpr int kMergeBytes = kWarps * kAttendMaxG * (D + 2) * 4;
-  static_assert(kMergeBytes <= kPipeBytes, "merge scratch");
+struct TileRegs {
+  uint4 k[2][D / 32];   // rows g, g+8 of the tile: bytes [t * D/2, +D/2)
+  uint4 v[4][D / 64];   // rows 2t, 2t+1, 8+2t, 9+2t: bytes [g * D/4, +D/4)
 };
+
+template <int D>
+__device__ __forceinline__ void load_tile(TileRegs<D>& tr, const uint16_t* __restrict__ kc,
+                                          const uint16_t* __restrict__ vc, const int64_t* s_off,
+                                          int tile, int n_mine, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  const int j0 = tile * kTile;
+  const int krow[2] = {g, g + 8};
+  const int vrow[4] = {2 * t, 2 * t + 1, 8 + 2 * t, 9 + 2 * t};
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int j = j0 + krow[i];
+    const int64_t off = j < n_mine ? s_off[j] : -1;
+    const uint16_t* src = kc + (off >= 0 ? off : 0) + t * (D / 4);
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c)
+      tr.k[i][c] = off >= 0 ? ld_stream_v4(src + c * 8) : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int j = j0 + vrow[i];
+    const int64_t off = j < n_mine ? s_off[j] : -1;
+    const uint16_t* src = vc + (off >= 0 ? off : 0) + g * (D / 8);
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c)
+      tr.v[i][c] = off >= 0 ? ld_stream_v4(src + c * 8) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+__device__ __forceinline__ uint32_t word(const uint4& u, int i) {
+  return i == 0 ? u.x : (i == 1 ? u.y : (i == 2 ? u.z : u.w));
+}
 
 template <int D, bool INDEXED>
 __global__ void __launch_bounds__(kThreads, 2) attend_kernel(AttendArgs a, int chunk, int splits) {
-  using S = Smem<D>;
-  constexpr int CH = D / 8;  // 16-byte chunks per row
-  extern __shared__ __align__(128) uint8_t attend_smem[];
-  int64_t* s_off = reinterpret_cast<int64_t*>(attend_smem + S::kPipeBytes);
+  static_assert(D == 128, "head dim");
+  constexpr int KB = D / 16;  // k-blocks of S^T, m-tiles of O^T
+  __shared__ int64_t s_off[kMaxChunk];
+  __shared__ float s_m[kWarps][kAttendMaxG], s_l[kWarps][kAttendMaxG];
+  __shared__ float s_o[kWarps][kAttendMaxG][D];
   __shared__ int s_last;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
   const int pair = blockIdx.y, split = blockIdx.x;
   const int b = pair / a.h_kv, h = pair % a.h_kv;
   const int G = a.h_q / a.h_kv;
   const int max_len = a.max_pages * a.page_size;
 
-  // Q fragments (rows = the G query heads of this KV head; rows >= G are zero)
-  uint32_t qa0[D / 16], qa2[D / 16];
+  // Q^T fragments (B operand of S^T = K Q^T): column n = head g of this KV head (zero for g >= G);
+  // k-slot 16kb+2t+e <-> physical dim D/4*t + 4kb + e, 16kb+8+2t+e <-> D/4*t + 4kb + 2 + e
+  uint32_t qb0[KB], qb1[KB];
   {
-    const int row = lane >> 2;
-    const uint32_t* qrow =
-        reinterpret_cast<const uint32_t*>(a.q + ((int64_t)b * a.h_q + (int64_t)h * G + row) * D);
+    const uint4* qrow = reinterpret_cast<const uint4*>(
+        a.q + ((int64_t)b * a.h_q + (int64_t)h * G + (g < G ? g : 0)) * D + t * (D / 4));
 #pragma unroll
-    for (int kb = 0; kb < D / 16; ++kb) {
-      qa0[kb] = row < G ? qrow[kb * 8 + (lane & 3)] : 0u;
-      qa2[kb] = row < G ? qrow[kb * 8 + 4 + (lane & 3)] : 0u;
+    for (int c = 0; c < D / 32; ++c) {
+      const uint4 v = g < G ? qrow[c] : make_uint4(0u, 0u, 0u, 0u);
+      qb0[2 * c] = v.x;
+      qb1[2 * c] = v.y;
+      qb0[2 * c + 1] = v.z;
+      qb1[2 * c + 1] = v.w;
     }
   }
 
@@ -89,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(AttendArgs a, int c
   // ---- row offsets of this CTA's positions ---------------------------------------------------
   const int32_t* bt = a.block_table + (int64_t)b * a.max_pages;
   for (int j = tid; j < n_mine; j += kThreads) {
-    int pos = INDEXED ? a.idx[(int64_t)pair * a.budget + j_begin + j] : lo + j_begin + j;
+    const int pos = INDEXED ? a.idx[(int64_t)pair * a.budget + j_begin + j] : lo + j_begin + j;
     int64_t off = -1;
     if (pos < 0 || pos >= max_len) {
       raise_flag(2u);
@@ -104,135 +149,102 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(AttendArgs a, int c
   }
   __syncthreads();
 
-  // ---- per-warp pipelined tiles --------------------------------------------------------------
+  // ---- per-warp tiles, next tile's loads in flight ------------------------------------------
   const int n_tiles = (n_mine + kTile - 1) / kTile;
-  const int my_tiles = n_tiles > warp ? (n_tiles - warp + kWarps - 1) / kWarps : 0;
-  uint8_t* wbase = attend_smem + warp * S::kWarpBytes;
-  const uint32_t wbase_s = smem_u32(wbase);
-
-  auto issue = [&](int i) {
-    if (i < my_tiles) {
-      const int tile = warp + i * kWarps;
-      const int r = lane & 15, half = lane >> 4;
-      const int j = tile * kTile + r;
-      const int64_t off = j < n_mine ? s_off[j] : -1;
-      const uint32_t kdst = wbase_s + (i % kStages) * S::kStageBytes + r * S::kRowBytes;
-      const uint32_t vdst = kdst + S::kTileBytes;
-      const uint16_t* ksrc = off >= 0 ? a.k_cache + off : a.k_cache;
-      const uint16_t* vsrc = off >= 0 ? a.v_cache + off : a.v_cache;
-      const int nbytes = off >= 0 ? 16 : 0;
-#pragma unroll
-      for (int c = half; c < CH; c += 2) {
-        const uint32_t sw = (uint32_t)((c ^ (r & 7)) * 16);
-        cp_async16(kdst + sw, ksrc + c * 8, nbytes);
-        cp_async16(vdst + sw, vsrc + c * 8, nbytes);
-      }
-    }
-    cp_async_commit();
-  };
-
   const float scale_log2 = a.scale * 1.4426950408889634f;
-  float o[D / 8][4];
+  float o[KB][4];
 #pragma unroll
-  for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-  float m_run = -INFINITY, l_run = 0.f;
+  for (int m = 0; m < KB; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};  // heads 2t, 2t+1
 
+  TileRegs<D> cur, nxt;
+  int tile = warp;
+  if (tile < n_tiles) load_tile<D>(cur, a.k_cache, a.v_cache, s_off, tile, n_mine, lane);
+  for (; tile < n_tiles; tile += kWarps) {
+    if (tile + kWarps < n_tiles)
+      load_tile<D>(nxt, a.k_cache, a.v_cache, s_off, tile + kWarps, n_mine, lane);
+
+    // S^T (16 tokens x 8 heads) = K Q^T
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int i = 0; i < kStages - 1; ++i) issue(i);
-
-  for (int i = 0; i < my_tiles; ++i) {
-    issue(i + kStages - 1);
-    cp_async_wait<kStages - 1>();
-    __syncwarp();
-    const int tile = warp + i * kWarps;
-    const uint32_t kbuf = wbase_s + (i % kStages) * S::kStageBytes;
-    const uint32_t vbuf = kbuf + S::kTileBytes;
-
-    // S = Q K^T for 16 tokens (two n8 tiles)
-    float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-    {
-      const int mat = lane >> 3;
-      const int row = (mat >> 1) * 8 + (lane & 7);
-#pragma unroll
-      for (int kb = 0; kb < D / 16; ++kb) {
-        const int c = 2 * kb + (mat & 1);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(kbuf + row * S::kRowBytes + ((c ^ (row & 7)) * 16), b0, b1, b2, b3);
-        mma_bf16(s0, qa0[kb], 0u, qa2[kb], 0u, b0, b1);
-        mma_bf16(s1, qa0[kb], 0u, qa2[kb], 0u, b2, b3);
-      }
+    for (int kb = 0; kb < KB; ++kb) {
+      const int c = kb >> 1, w0 = (kb & 1) * 2;
+      const uint32_t a0 = word(cur.k[0][c], w0), a2 = word(cur.k[0][c], w0 + 1);
+      const uint32_t a1 = word(cur.k[1][c], w0), a3 = word(cur.k[1][c], w0 + 1);
+      mma_bf16(s, a0, a1, a2, a3, qb0[kb], qb1[kb]);
     }
-    // mask positions past the end or with an invalid row
-    const int t0 = tile * kTile + 2 * (lane & 3);
+    // rows: token g (s[0], s[1]) and g+8 (s[2], s[3]); columns: heads 2t, 2t+1
+    const int j0 = tile * kTile;
+    const bool ok0 = j0 + g < n_mine && s_off[j0 + g] >= 0;
+    const bool ok1 = j0 + g + 8 < n_mine && s_off[j0 + g + 8] >= 0;
     float x[4];
-    {
-      const int tt[4] = {t0, t0 + 1, t0 + 8, t0 + 9};
-      const float sv[4] = {s0[0], s0[1], s1[0], s1[1]};
+    x[0] = ok0 ? s[0] * scale_log2 : -INFINITY;
+    x[1] = ok0 ? s[1] * scale_log2 : -INFINITY;
+    x[2] = ok1 ? s[2] * scale_log2 : -INFINITY;
+    x[3] = ok1 ? s[3] * scale_log2 : -INFINITY;
+    float mx0 = fmaxf(x[0], x[2]), mx1 = fmaxf(x[1], x[3]);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const bool ok = tt[e] < n_mine && s_off[tt[e]] >= 0;
-        x[e] = ok ? sv[e] * scale_log2 : -INFINITY;
-      }
+    for (int sh = 4; sh < 32; sh <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, sh));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, sh));
     }
-    float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    const float m_new = fmaxf(m_run, mx);
-    const float m_use = m_new == -INFINITY ? 0.f : m_new;
-    const float corr = fast_exp2(m_run - m_use);
+    const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+    const float mu0 = mn0 == -INFINITY ? 0.f : mn0, mu1 = mn1 == -INFINITY ? 0.f : mn1;
+    const float corr0 = fast_exp2(m_run[0] - mu0), corr1 = fast_exp2(m_run[1] - mu1);
     float p[4];
+    p[0] = fast_exp2(x[0] - mu0);
+    p[1] = fast_exp2(x[1] - mu1);
+    p[2] = fast_exp2(x[2] - mu0);
+    p[3] = fast_exp2(x[3] - mu1);
+    l_run[0] = l_run[0] * corr0 + p[0] + p[2];
+    l_run[1] = l_run[1] * corr1 + p[1] + p[3];
+    m_run[0] = mn0;
+    m_run[1] = mn1;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) p[e] = fast_exp2(x[e] - m_use);
-    l_run = l_run * corr + (p[0] + p[1]) + (p[2] + p[3]);
-    m_run = m_new;
-#pragma unroll
-    for (int n = 0; n < D / 8; ++n) {
-      o[n][0] *= corr;
-      o[n][1] *= corr;
+    for (int m = 0; m < KB; ++m) {
+      o[m][0] *= corr0;
+      o[m][1] *= corr1;
+      o[m][2] *= corr0;
+      o[m][3] *= corr1;
     }
-    // P (16 heads x 16 tokens) as an A operand, split into bf16 high + low parts
-    const uint32_t ph0 = pack_bf16x2(p[0], p[1]);
-    const uint32_t ph2 = pack_bf16x2(p[2], p[3]);
+    // P^T as the B operand (tokens x heads), high and low bf16 parts
+    const uint32_t ph0 = pack_bf16x2(p[0], p[1]);  // token g,   heads 2t, 2t+1
+    const uint32_t ph1 = pack_bf16x2(p[2], p[3]);  // token g+8
     const uint32_t pl0 = pack_bf16x2(p[0] - bf16_lo(ph0), p[1] - bf16_hi(ph0));
-    const uint32_t pl2 = pack_bf16x2(p[2] - bf16_lo(ph2), p[3] - bf16_hi(ph2));
-    {
-      const int mat = lane >> 3;
-      const int row = (mat & 1) * 8 + (lane & 7);
+    const uint32_t pl1 = pack_bf16x2(p[2] - bf16_lo(ph1), p[3] - bf16_hi(ph1));
+    const uint32_t bh0 = movmatrix_t(ph0), bh1 = movmatrix_t(ph1);
+    const uint32_t bl0 = movmatrix_t(pl0), bl1 = movmatrix_t(pl1);
+    // O^T (dims x heads) += V^T P^T; m-tile m: rows g, g+8 = physical dims D/8*g + 2m, +1
 #pragma unroll
-      for (int j = 0; j < D / 16; ++j) {
-        const int c = 2 * j + (mat >> 1);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(vbuf + row * S::kRowBytes + ((c ^ (row & 7)) * 16), b0, b1, b2, b3);
-        mma_bf16(o[2 * j], ph0, 0u, ph2, 0u, b0, b1);
-        mma_bf16(o[2 * j], pl0, 0u, pl2, 0u, b0, b1);
-        mma_bf16(o[2 * j + 1], ph0, 0u, ph2, 0u, b2, b3);
-        mma_bf16(o[2 * j + 1], pl0, 0u, pl2, 0u, b2, b3);
-      }
+    for (int m = 0; m < KB; ++m) {
+      const int c = m >> 2, wi = m & 3;
+      const uint32_t r0 = word(cur.v[0][c], wi), r1 = word(cur.v[1][c], wi);
+      const uint32_t r2 = word(cur.v[2][c], wi), r3 = word(cur.v[3][c], wi);
+      const uint32_t va0 = prmt(r0, r1, 0x5410u), va1 = prmt(r0, r1, 0x7632u);
+      const uint32_t va2 = prmt(r2, r3, 0x5410u), va3 = prmt(r2, r3, 0x7632u);
+      mma_bf16(o[m], va0, va1, va2, va3, bh0, bh1);
+      mma_bf16(o[m], va0, va1, va2, va3, bl0, bl1);
     }
-    __syncwarp();
+    cur = nxt;
   }
-  cp_async_wait<0>();
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
-  __syncthreads();  // pipeline buffers are now reused as merge scratch
+#pragma unroll
+  for (int sh = 4; sh < 32; sh <<= 1) {
+    l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], sh);
+    l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], sh);
+  }
 
   // ---- merge the 4 warps ---------------------------------------------------------------------
-  float* s_m = reinterpret_cast<float*>(attend_smem);          // [warps][8]
-  float* s_l = s_m + kWarps * kAttendMaxG;              // [warps][8]
-  float* s_o = s_l + kWarps * kAttendMaxG;              // [warps][8][D]
   {
-    const int row = lane >> 2;
-    if (row < G) {
-      if ((lane & 3) == 0) {
-        s_m[warp * kAttendMaxG + row] = m_run;
-        s_l[warp * kAttendMaxG + row] = l_run;
-      }
-      float* dst = s_o + (warp * kAttendMaxG + row) * D + 2 * (lane & 3);
+    const int hh0 = 2 * t, hh1 = 2 * t + 1;
+    if (g == 0) {
+      if (hh0 < G) { s_m[warp][hh0] = m_run[0]; s_l[warp][hh0] = l_run[0]; }
+      if (hh1 < G) { s_m[warp][hh1] = m_run[1]; s_l[warp][hh1] = l_run[1]; }
+    }
 #pragma unroll
-      for (int n = 0; n < D / 8; ++n) {
-        dst[8 * n] = o[n][0];
-        dst[8 * n + 1] = o[n][1];
-      }
+    for (int m = 0; m < KB; ++m) {
+      const int d0 = (D / 8) * g + 2 * m;  // physical dims of rows g and g+8 of m-tile m
+      if (hh0 < G) { s_o[warp][hh0][d0] = o[m][0]; s_o[warp][hh0][d0 + 1] = o[m][2]; }
+      if (hh1 < G) { s_o[warp][hh1][d0] = o[m][1]; s_o[warp][hh1][d0 + 1] = o[m][3]; }
     }
   }
   __syncthreads();
@@ -248,14 +260,14 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(AttendArgs a, int c
     const int row = e / D, dim = e % D;
     float mm = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, s_m[w * kAttendMaxG + row]);
+    for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, s_m[w][row]);
     float acc = 0.f, l = 0.f;
     if (mm != -INFINITY) {
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) {
-        const float f = fast_exp2(s_m[w * kAttendMaxG + row] - mm);
-        acc += f * s_o[(w * kAttendMaxG + row) * D + dim];
-        l += f * s_l[w * kAttendMaxG + row];
+        const float f = fast_exp2(s_m[w][row] - mm);
+        acc += f * s_o[w][row][dim];
+        l += f * s_l[w][row];
       }
     }
     if (splits == 1) {
@@ -283,13 +295,13 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(AttendArgs a, int c
     const float* pp = part + ((int64_t)pair * splits * G + row) * (D + 2);
     const int64_t step = (int64_t)G * (D + 2);
     float mm = -INFINITY;
-    for (int s = 0; s < splits; ++s) mm = fmaxf(mm, __ldcg(pp + s * step));
+    for (int s_ = 0; s_ < splits; ++s_) mm = fmaxf(mm, __ldcg(pp + s_ * step));
     float acc = 0.f, l = 0.f;
     if (mm != -INFINITY) {
-      for (int s = 0; s < splits; ++s) {
-        const float f = fast_exp2(__ldcg(pp + s * step) - mm);
-        acc += f * __ldcg(pp + s * step + 2 + dim);
-        l += f * __ldcg(pp + s * step + 1);
+      for (int s_ = 0; s_ < splits; ++s_) {
+        const float f = fast_exp2(__ldcg(pp + s_ * step) - mm);
+        acc += f * __ldcg(pp + s_ * step + 2 + dim);
+        l += f * __ldcg(pp + s_ * step + 1);
       }
     }
     a.out[out_base + (int64_t)row * D + dim] = f_to_bf16(l > 0.f ? acc / l : 0.f);
@@ -300,20 +312,17 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(AttendArgs a, int c
 template <int D, bool INDEXED>
 cudaError_t launch_t(const AttendArgs& a, const AttendPlan& plan, bool pdl, cudaStream_t s) {
   auto kern = attend_kernel<D, INDEXED>;
-  const int smem = Smem<D>::kTotal;
-  cudaError_t e = configure_kernel((const void*)kern, (int)smem, false);
-  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(plan.splits, a.batch * a.h_kv, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  e = cudaLaunchKernelEx(&cfg, kern, a, plan.chunk, plan.splits);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a, plan.chunk, plan.splits);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -325,8 +334,9 @@ AttendPlan plan_attend(int pairs, int positions, int group, int d) {
   const int unit = attend_detail::kWarps * attend_detail::kTile;  // 64 positions
   positions = positions < 1 ? 1 : positions;
   const int max_splits = (positions + unit - 1) / unit;
-  const int want_ctas = 4 * num_sms();
-  int splits = (want_ctas + pairs - 1) / pairs;
+  // about one wave of resident CTAs (2 per SM); more splits only when the pairs are few
+  const int slots = 2 * num_sms();
+  int splits = slots / (pairs > 0 ? pairs : 1);
   if (splits > max_splits) splits = max_splits;
   if (splits < 1) splits = 1;
   int chunk = (positions + splits - 1) / splits;
@@ -344,7 +354,9 @@ AttendPlan plan_attend(int pairs, int positions, int group, int d) {
 cudaError_t launch_attend(const AttendArgs& a, bool indexed, const AttendPlan& plan, bool pdl,
                           cudaStream_t s) {
   if (a.batch * a.h_kv == 0) return cudaSuccess;
-  if (a.d == 128) return indexed ? attend_detail::launch_t<128, true>(a, plan, pdl, s) : attend_detail::launch_t<128, false>(a, plan, pdl, s);
+  if (a.d == 128)
+    return indexed ? attend_detail::launch_t<128, true>(a, plan, pdl, s)
+                   : attend_detail::launch_t<128, false>(a, plan, pdl, s);
   return cudaErrorInvalidValue;
 }
 

@@ -19,6 +19,7 @@ struct ScorePlan {
   int cluster;     // CTAs per (sequence, KV head)
   int chunk;       // tokens per CTA (multiple of the page size and of 64)
   size_t smem;     // dynamic shared memory per CTA
+  size_t ws_bytes; // candidate keys/positions + per-CTA counts
 };
 
 struct AttendPlan {
@@ -52,7 +53,7 @@ cudaError_t launch_score_topk(const uint16_t* q, const float* basis, const uint8
                               const int32_t* block_table, int max_pages, const int32_t* seq_lens,
                               int batch, int h_q, int h_kv, int d, int r, int64_t num_pages,
                               int page_size, int budget, int32_t* idx, int32_t* count,
-                              bool pdl, cudaStream_t s);
+                              void* ws, int* attend_tickets, bool pdl, cudaStream_t s);
 
 struct AttendArgs {
   const uint16_t* q;
