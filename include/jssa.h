@@ -70,7 +70,9 @@ enum jssa_device_flag {
   JSSA_DEVERR_PAGE = 1,       /* block_table or slot_mapping named a page outside [0, num_pages) */
   JSSA_DEVERR_INDEX = 2,      /* an index-set entry outside [0, max_pages*page_size) */
   JSSA_DEVERR_SEQLEN = 4,     /* seq_len < 0 or > max_pages*page_size (clamped) */
-  JSSA_DEVERR_SELECT = 8      /* internal: inconsistent top-B counts (never expected) */
+  JSSA_DEVERR_SELECT = 8,     /* internal: inconsistent top-B counts (never expected) */
+  JSSA_DEVERR_RESCAN = 16     /* information only: a sampled candidate threshold was too high and
+                                 the selection rescanned the sequence (the result is exact) */
 };
 
 /* Workspace clients for jssa_workspace_size. */
@@ -152,9 +154,13 @@ JSSA_API int jssa_store(const jssa_bf16* k, int64_t k_stride_t, const int64_t* s
  * heads of h), s_t = sum_j dec(c_tj) p_j for every t < seq_len (fp32), and the index set of the
  * min(budget, seq_len) largest s_t, ties to the lower position, written ascending.
  * JSSA summary, eq. (1) and section 3.1 steps 1-2; JSSA README, section 4 (jssa_budget).
- * One thread-block cluster per (sequence, KV head) keeps all scores in shared memory; only the
- * keys that can still be selected (a few per selected token) go through the workspace.
+ * Three kernels: a per-(sequence, KV head) prep (query projection, its FP8 digits and a
+ * candidate threshold from a sample of the scores), a streaming scan on the tensor cores that
+ * keeps only keys at or above the threshold, and an exact per-(sequence, KV head) selection
+ * (which rescans when the threshold let through fewer than min(budget, seq_len) keys).
  * q: bf16 [batch, h_q, d] contiguous. ws: >= jssa_workspace_size(JSSA_FN_SCORE_TOPK).
+ * Limits (JSSA_ERR_UNSUPPORTED beyond them): max_pages * page_size <= 4194304 positions and
+ * batch * h_kv <= 65535.
  */
 JSSA_API int jssa_score_topk(const jssa_bf16* q, const float* basis, const uint8_t* score_cache,
                     const int32_t* block_table, int max_pages, const int32_t* seq_lens, int batch,

@@ -1,8 +1,10 @@
 """Parity of the CUDA path (called through the C ABI) with the CPU oracle on seeded inputs.
 
 Sizes: the tiny 2K-context workload (8 query / 2 KV heads, d 128, 16-token pages, r 32, B 128)
-and variations that span several CTAs, clusters of up to 16 CTAs and ragged tails: uneven
-sequence lengths, lengths below/at/above the budget, an empty sequence, r = 64, 32-token pages.
+and variations that span several scan CTAs and ragged tails: uneven sequence lengths, lengths
+below/at/above the budget, an empty sequence, r = 64, 32-token pages, contexts past the point
+where the candidate threshold is sampled, candidate sets too large for shared staging, and an
+adversarial score layout that defeats the sample.
 Criteria are in ``parity.py``.
 """
 
@@ -101,8 +103,8 @@ def test_score_topk_budgets(ragged, budget):
 
 
 @pytest.mark.parametrize("seq_len,batch,budget", [(32768, 2, 2048), (20000, 1, 777), (65536, 1, 4096)])
-def test_score_topk_clusters(seq_len, batch, budget):
-    # contexts that the planner spreads over clusters of 8-16 CTAs
+def test_score_topk_long(seq_len, batch, budget):
+    # contexts with a sampled candidate threshold, over many scan CTAs
     case = Case([seq_len] * batch, seed=1030 + seq_len % 97, calib=2048)
     J = jssa()
     idx, count = J.score_topk(case.gpu(case.q), case.gpu_np(case.m32), case.gpu_np(case.codes),
@@ -140,6 +142,86 @@ def test_score_topk_exact_ties_go_to_lower_position():
     gi = idx.cpu().numpy()
     for h in range(case.h_kv):
         assert np.array_equal(gi[0, h], np.arange(budget))
+
+
+def test_score_topk_long_ties_beyond_staging():
+    # 40000 tied tokens: every key is a candidate (more than the select stage holds in shared
+    # memory), and the set must still be the lowest positions
+    case = Case([40000], seed=1051, calib=2048)
+    codes = case.codes.copy()
+    codes[:] = codes[0, :, :1, :]
+    J = jssa()
+    budget = 2048
+    idx, count = J.score_topk(case.gpu(case.q), case.gpu_np(case.m32), case.gpu_np(codes),
+                              case.gpu(case.block_table), case.gpu(case.seq_lens_t), budget)
+    gi, gc = idx.cpu().numpy(), count.cpu().numpy()
+    for h in range(case.h_kv):
+        assert gc[0, h] == budget
+        assert np.array_equal(gi[0, h], np.arange(budget))
+
+
+def test_score_topk_budget_near_context():
+    # a budget a third of the context: every position is a candidate, beyond shared staging
+    case = Case([24000], seed=1052, calib=2048)
+    J = jssa()
+    budget = 8000
+    idx, count = J.score_topk(case.gpu(case.q), case.gpu_np(case.m32), case.gpu_np(case.codes),
+                              case.gpu(case.block_table), case.gpu(case.seq_lens_t), budget)
+    ref_idx, ref_count, s = _select_oracle(case, budget)
+    gi, gc = idx.cpu().numpy(), count.cpu().numpy()
+    for h in range(case.h_kv):
+        check_selection(gi[0, h], gc[0, h], ref_idx[0, h], ref_count[0, h], s[(0, h)], budget)
+
+
+def _mix32(x):
+    x ^= x >> 16
+    x = (x * 0x7FEB352D) & 0xFFFFFFFF
+    x ^= x >> 15
+    x = (x * 0x846CA68B) & 0xFFFFFFFF
+    x ^= x >> 16
+    return x
+
+
+def _sampled_positions(pair, L, n=2048):
+    # the candidate-threshold sample of the score kernels: one position per stratum of L // n
+    # tokens, at an offset drawn from a 32-bit mix of (stratum, pair), never the last position
+    stratum = L // n
+    out = []
+    for i in range(n):
+        h = _mix32(((i * 0x9E3779B9) & 0xFFFFFFFF) ^ ((pair * 0x85EBCA6B + 1) & 0xFFFFFFFF))
+        out.append(min(i * stratum + h % stratum, L - 2))
+    return np.asarray(out)
+
+
+def test_score_topk_rescan_when_sample_overestimates():
+    # adversarial scores: exactly the sampled positions score high, every other position low, so
+    # the sampled threshold lets through 2048 keys for a budget of 4096; the selection must detect
+    # it, rescan the sequence and still return the exact set (and say so in the device flags)
+    L, budget = 32768, 4096
+    case = Case([L], seed=1053, calib=2048)
+    codes = case.codes.copy()
+    bt = case.np_bt
+    qbar = O.group_mean_query(case.np_q[0], case.h_kv)
+    for h in range(case.h_kv):
+        row = codes[bt[0, 0], h, 0, :].copy()
+        s0 = O.scores(row[None, :], O.projected_query(qbar[h], case.m32[h].astype(np.float64)))[0]
+        assert s0 != 0.0
+        hi, lo = (row, row ^ 0x80) if s0 > 0 else (row ^ 0x80, row)
+        sampled = np.zeros(L, dtype=bool)
+        sampled[_sampled_positions(h, L)] = True
+        for pos in range(L):
+            codes[bt[0, pos // case.ps], h, pos % case.ps, :] = hi if sampled[pos] else lo
+    J = jssa()
+    J.device_error(clear=True)
+    idx, count = J.score_topk(case.gpu(case.q), case.gpu_np(case.m32), case.gpu_np(codes),
+                              case.gpu(case.block_table), case.gpu(case.seq_lens_t), budget)
+    flags = J.device_error(clear=True)
+    ref_idx, ref_count, _ = O.select_step(case.np_q, case.m32.astype(np.float64), codes, bt,
+                                          case.np_lens, budget)
+    gi, gc = idx.cpu().numpy(), count.cpu().numpy()
+    assert np.array_equal(gc, ref_count)
+    assert np.array_equal(gi, ref_idx)
+    assert flags == 16
 
 
 # ------------------------------------------------------------------------------------------------
@@ -229,6 +311,34 @@ def test_decode_step(ragged, budget):
     assert np.array_equal(f64(v_cache), ref["v_cache"])
     gsc = sc.cpu().numpy()
     assert np.array_equal(gsc, ref["score_cache"])
+    gi, gc = idx.cpu().numpy(), count.cpu().numpy()
+    assert np.array_equal(gc, ref["count"])
+    for b in range(len(lens)):
+        for h in range(case.h_kv):
+            check_selection(gi[b, h], gc[b, h], ref["idx"][b, h], ref["count"][b, h],
+                            ref["scores"][(b, h)], budget)
+    check_output(f64(out), ref["out"])
+
+
+def test_decode_step_long_contexts():
+    # contexts past the all-candidates limit: the new token is stored by the same kernel that
+    # draws the threshold sample, and the scan reads its code afterwards
+    case = Case([20000, 17001, 16384], seed=1070, calib=2048)
+    J = jssa()
+    budget = 1024
+    lens = np.asarray(case.seq_lens)
+    rng = np.random.default_rng(7)
+    k_new = torch.from_numpy(rng.standard_normal((len(lens), case.h_kv, case.d))).to(torch.bfloat16)
+    v_new = torch.from_numpy(rng.standard_normal((len(lens), case.h_kv, case.d))).to(torch.bfloat16)
+    k_cache, v_cache = case.gpu(case.k_cache).clone(), case.gpu(case.v_cache).clone()
+    sc = case.gpu_np(case.codes).clone()
+    scale = 1.0 / math.sqrt(case.d)
+    out, idx, count = J.decode(case.gpu(case.q), k_new.cuda(), v_new.cuda(), k_cache, v_cache, sc,
+                               case.gpu_np(case.m32), case.gpu(case.block_table),
+                               case.gpu(case.seq_lens_t), budget, scale)
+    ref = O.decode_step(case.np_q, f64(k_new), f64(v_new), case.np_k, case.np_v, case.codes,
+                        case.np_bt, lens, case.m32.astype(np.float64), budget, scale)
+    assert np.array_equal(sc.cpu().numpy(), ref["score_cache"])
     gi, gc = idx.cpu().numpy(), count.cpu().numpy()
     assert np.array_equal(gc, ref["count"])
     for b in range(len(lens)):

@@ -8,7 +8,7 @@
 #include <mutex>
 #include <utility>
 
-#include "../../include/jssa.h"
+#include "jssa.h"
 #include "common.cuh"
 
 namespace jssa {
@@ -54,7 +54,7 @@ namespace {
 using jssa::AttendArgs;
 
 constexpr int kVersion = 100;  // 0.1.0
-constexpr int64_t kMaxContext = (int64_t)jssa::kMaxClusterCtas * jssa::kScoreChunkMax;
+constexpr int64_t kMaxContext = jssa::kScoreMaxContext;
 
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? JSSA_OK : (int)e; }
 inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
@@ -222,6 +222,7 @@ static int check_score_args(const jssa_bf16* q, const float* basis, const uint8_
   if (!supported_dr(d, r)) return JSSA_ERR_UNSUPPORTED;
   if ((st = check_paging(max_pages, num_pages, page_size))) return st;
   if ((int64_t)max_pages * page_size > kMaxContext) return JSSA_ERR_UNSUPPORTED;
+  if ((int64_t)batch * h_kv > 65535) return JSSA_ERR_UNSUPPORTED;  // one grid row per pair
   if (batch == 0) return JSSA_OK;
   if (!q || !basis || !score_cache || !block_table || !seq_lens || !idx || !count)
     return JSSA_ERR_NULL;
@@ -242,8 +243,8 @@ int jssa_score_topk(const jssa_bf16* q, const float* basis, const uint8_t* score
   if (!aligned16(ws)) return JSSA_ERR_ALIGN;
   return cuda_status(jssa::launch_score_topk(q, basis, score_cache, block_table, max_pages,
                                              seq_lens, batch, h_q, h_kv, d, r, num_pages,
-                                             page_size, budget, idx, count, ws, nullptr, false,
-                                             as_stream(stream)));
+                                             page_size, budget, idx, count, ws, nullptr,
+                                             nullptr, false, as_stream(stream)));
 }
 
 static int check_attend_common(const jssa_bf16* q, const jssa_bf16* k_cache,
@@ -341,20 +342,17 @@ int jssa_decode(const jssa_bf16* q, const jssa_bf16* k_new, const jssa_bf16* v_n
   void* attend_ws = ws;
   void* cand_ws = static_cast<uint8_t*>(ws) + attend_bytes;
   cudaStream_t s = as_stream(stream);
-  bool pdl = false;
+  jssa::StoreNew sn = {};
   if (k_new) {
-    cudaError_t e = jssa::launch_store_decode(k_new, v_new, k_cache, v_cache, kv_page_stride,
-                                              kv_slot_stride, kv_head_stride, score_cache, basis,
-                                              block_table, max_pages, seq_lens, batch, h_kv, d, r,
-                                              num_pages, page_size, s);
-    if (e != cudaSuccess) return (int)e;
-    pdl = true;
+    sn.k_new = k_new; sn.v_new = v_new; sn.k_cache = k_cache; sn.v_cache = v_cache;
+    sn.page_stride = kv_page_stride; sn.slot_stride = kv_slot_stride;
+    sn.head_stride = kv_head_stride; sn.score_cache = score_cache;
   }
   cudaError_t e = jssa::launch_score_topk(q, basis, score_cache, block_table, max_pages, seq_lens,
                                           batch, h_q, h_kv, d, r, num_pages, page_size, budget,
                                           idx, count, cand_ws,
                                           plan.ws_bytes ? static_cast<int*>(attend_ws) : nullptr,
-                                          pdl, s);
+                                          k_new ? &sn : nullptr, false, s);
   if (e != cudaSuccess) return (int)e;
   AttendArgs a = {};
   a.q = q; a.k_cache = k_cache; a.v_cache = v_cache;

@@ -7,19 +7,25 @@
 
 namespace jssa {
 
-constexpr int kMaxClusterCtas = 16;        // non-portable cluster size used by score + top-B
-constexpr int kScoreThreads = 512;
-constexpr int kScoreChunkTarget = 8192;    // tokens of one (sequence, KV head) per CTA
-constexpr int kScoreChunkMax = 40960;      // shared-memory bound on tokens per CTA
+constexpr int64_t kScoreMaxContext = 1 << 22;  // positions per sequence the score kernels plan for
 constexpr int kAttendWarps = 4;
 constexpr int kAttendTile = 16;            // tokens per warp-level tile
 constexpr int kAttendMaxG = 8;             // query heads per KV head held in one m16 tile
 
 struct ScorePlan {
-  int cluster;     // CTAs per (sequence, KV head)
-  int chunk;       // tokens per CTA (multiple of the page size and of 64)
-  size_t smem;     // dynamic shared memory per CTA
-  size_t ws_bytes; // candidate keys/positions + per-CTA counts
+  int chunk;       // positions per scan CTA (power of two, multiple of the page size)
+  int n_chunks;    // scan CTAs per (sequence, KV head)
+  size_t ws_bytes; // prep records + candidate counts + candidate keys/positions
+};
+
+// The new token of a decode step, stored by the score kernels' prep stage.
+struct StoreNew {
+  const uint16_t* k_new;  // bf16 [batch, h_kv, d]
+  const uint16_t* v_new;  // bf16 [batch, h_kv, d]
+  uint16_t* k_cache;
+  uint16_t* v_cache;
+  int64_t page_stride, slot_stride, head_stride;
+  uint8_t* score_cache;
 };
 
 struct AttendPlan {
@@ -53,7 +59,8 @@ cudaError_t launch_score_topk(const uint16_t* q, const float* basis, const uint8
                               const int32_t* block_table, int max_pages, const int32_t* seq_lens,
                               int batch, int h_q, int h_kv, int d, int r, int64_t num_pages,
                               int page_size, int budget, int32_t* idx, int32_t* count,
-                              void* ws, int* attend_tickets, bool pdl, cudaStream_t s);
+                              void* ws, int* attend_tickets, const StoreNew* store, bool pdl,
+                              cudaStream_t s);
 
 struct AttendArgs {
   const uint16_t* q;

@@ -18,7 +18,7 @@
 
 #include <mutex>
 
-#include "../../include/jssa.h"
+#include "jssa.h"
 #include "common.cuh"
 
 namespace jssa {
