@@ -27,7 +27,8 @@
  *   [batch, max_pages], seq_lens int32 [batch]. page_size is a power of two.
  * - Scoring cache: uint8 E4M3 codes laid out [num_pages, h_kv, page_size, r] (one contiguous
  *   run of page_size*r bytes per page and KV head), same page numbering as the KV cache.
- * - Basis: float32 [h_kv, r, d], rows orthonormal (output of jssa_compute_basis).
+ * - Basis: float32 [h_kv, r, d], rows orthonormal (output of jssa_compute_basis); the score
+ *   entry points want it, and the scoring cache, 16-byte aligned (JSSA_ERR_ALIGN otherwise).
  * - Index sets: int32 idx [batch, h_kv, budget] holds logical positions in ascending order,
  *   padded with -1; int32 count [batch, h_kv] = min(budget, seq_len).
  * - Device-side checks: a page number outside [0, num_pages), a position outside the block
@@ -71,8 +72,9 @@ enum jssa_device_flag {
   JSSA_DEVERR_INDEX = 2,      /* an index-set entry outside [0, max_pages*page_size) */
   JSSA_DEVERR_SEQLEN = 4,     /* seq_len < 0 or > max_pages*page_size (clamped) */
   JSSA_DEVERR_SELECT = 8,     /* internal: inconsistent top-B counts (never expected) */
-  JSSA_DEVERR_RESCAN = 16     /* information only: a sampled candidate threshold was too high and
+  JSSA_DEVERR_RESCAN = 16,    /* information only: a sampled candidate threshold was too high and
                                  the selection rescanned the sequence (the result is exact) */
+  JSSA_DEVERR_TIMEOUT = 32    /* a bounded wait inside a kernel ran out (its results are invalid) */
 };
 
 /* Workspace clients for jssa_workspace_size. */
@@ -159,8 +161,9 @@ JSSA_API int jssa_store(const jssa_bf16* k, int64_t k_stride_t, const int64_t* s
  * keeps only keys at or above the threshold, and an exact per-(sequence, KV head) selection
  * (which rescans when the threshold let through fewer than min(budget, seq_len) keys).
  * q: bf16 [batch, h_q, d] contiguous. ws: >= jssa_workspace_size(JSSA_FN_SCORE_TOPK).
- * Limits (JSSA_ERR_UNSUPPORTED beyond them): max_pages * page_size <= 4194304 positions and
- * batch * h_kv <= 65535.
+ * Limits (JSSA_ERR_UNSUPPORTED beyond them): max_pages * page_size <= 4194304 positions,
+ * batch * h_kv <= 65535 and page_size * r >= 128 (the scan copies whole page rows of at least
+ * 128 bytes into shared memory).
  */
 JSSA_API int jssa_score_topk(const jssa_bf16* q, const float* basis, const uint8_t* score_cache,
                     const int32_t* block_table, int max_pages, const int32_t* seq_lens, int batch,

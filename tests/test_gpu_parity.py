@@ -184,12 +184,13 @@ def _mix32(x):
 
 def _sampled_positions(pair, L, n=2048):
     # the candidate-threshold sample of the score kernels: one position per stratum of L // n
-    # tokens, at an offset drawn from a 32-bit mix of (stratum, pair), never the last position
+    # tokens, at an offset drawn from a 32-bit mix of (stratum, pair) scaled to the stratum by a
+    # high multiply, never the last position
     stratum = L // n
     out = []
     for i in range(n):
         h = _mix32(((i * 0x9E3779B9) & 0xFFFFFFFF) ^ ((pair * 0x85EBCA6B + 1) & 0xFFFFFFFF))
-        out.append(min(i * stratum + h % stratum, L - 2))
+        out.append(min(i * stratum + ((h * stratum) >> 32), L - 2))
     return np.asarray(out)
 
 

@@ -26,6 +26,8 @@
 //        than the budget (the sampled threshold was too high -- not expected in practice), the
 //        CTA first rescans the sequence with no threshold, so the result is exact in every case.
 // seq_len <= budget selects every position without scoring.
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 
 namespace jssa {
@@ -36,23 +38,15 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kUnrollBytes = 32;   // bytes of scoring rows per lane per load batch
 constexpr int kBins = 2048;
-constexpr int kDigits = 8;         // FP8 digit columns of p (the n = 8 of the mma)
+constexpr int kDigits = 2;         // f16 digit vectors of p (B columns 2t and 2t + 1 of lane t)
 constexpr int kSample = 2048;      // sampled positions per (sequence, KV head)
 constexpr int kExactMax = 16384;   // up to this context every token is a candidate
 constexpr int kSelectCap = 16384;  // candidates the select kernel stages in shared memory
-constexpr int kMaxRegions = 4096;  // scan regions (chunks x warps) per (sequence, KV head)
+constexpr int kRegionsPerChunk = kWarps;  // candidate regions (one per scan warp) per chunk
+constexpr int kMaxRegions = 4096;  // candidate regions per (sequence, KV head)
 constexpr int kPrepBytes = 1024;   // per (sequence, KV head): digits, scales, threshold, mode
 constexpr int kPrepScale = 512, kPrepThr = 544, kPrepMode = 548;
 constexpr int kModeScan = 0, kModeAll = 1;
-
-__device__ __forceinline__ void mma_e4m3(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t x, int lane) {
 #pragma unroll
@@ -63,83 +57,211 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t x, int lane) {
   return x;
 }
 
-// Bin of a histogram (`nb` bins, read through `at`) holding the want-th largest element counted
-// from the top. Warp-wide; returns (bin, count of elements in strictly higher bins, count in
-// the bin) on every lane.
-template <typename At>
-__device__ __forceinline__ void find_bin(At at, int nb, uint32_t want, int lane, int& bin_out,
-                                         uint32_t& above_out, uint32_t& cnt_out, bool& found) {
-  const int bpl = (nb + 31) / 32;
-  const int hi = nb - lane * bpl;
-  const int lo = max(0, hi - bpl);
+// Block-wide (NT threads): the bin of s_hist[0:nb) that holds the want-th largest element
+// counted from the top bin down, the number of elements in strictly higher bins and the bin's
+// own count, in s_info[0..2] (s_info[3] = 1 when found). Every thread sums nb / NT adjacent
+// bins, then an exclusive scan over the threads (top bins first) finds the one thread whose
+// range holds it.
+template <int NT>
+__device__ void find_bin(const uint32_t* s_hist, int nb, uint32_t want, uint32_t* s_wsum,
+                         int* s_info) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bpt = nb > NT ? nb / NT : 1;
+  const int hi = nb - tid * bpt;
+  const int lo = max(0, hi - bpt);
   uint32_t c = 0;
-  for (int j = lo; j < hi; ++j) c += at(j);
-  const uint32_t incl = warp_incl_scan(c, lane);
-  const uint32_t excl = incl - c;
-  const unsigned hit = __ballot_sync(0xffffffffu, hi > lo && excl < want && excl + c >= want);
-  found = hit != 0;
-  const int ln = hit ? __ffs(hit) - 1 : 0;
-  int bin = 0;
-  uint32_t run = 0, cnt = 0;
-  if (lane == ln) {
-    run = excl;
-    bin = lo;
+  for (int j = lo; j < hi; ++j) c += s_hist[j];
+  const uint32_t incl_w = warp_incl_scan(c, lane);
+  if (lane == 31) s_wsum[warp] = incl_w;
+  if (tid == 0) s_info[3] = 0;
+  __syncthreads();
+  uint32_t before = 0;
+  for (int w = 0; w < warp; ++w) before += s_wsum[w];
+  const uint32_t excl = before + incl_w - c;
+  if (hi > lo && excl < want && excl + c >= want) {
+    uint32_t run = excl;
     for (int j = hi - 1; j >= lo; --j) {
-      const uint32_t cj = at(j);
-      if (run + cj >= want) { bin = j; cnt = cj; break; }
+      const uint32_t cj = s_hist[j];
+      if (run + cj >= want) {
+        s_info[0] = j;
+        s_info[1] = (int)run;
+        s_info[2] = (int)cj;
+        s_info[3] = 1;
+        break;
+      }
       run += cj;
     }
   }
-  bin_out = __shfl_sync(0xffffffffu, bin, ln);
-  above_out = __shfl_sync(0xffffffffu, run, ln);
-  cnt_out = __shfl_sync(0xffffffffu, cnt, ln);
+  __syncthreads();
 }
 
-// Exact radix select over `n` keys read through `key_at(i)`: the threshold key thr and the number
-// `take` of keys equal to thr that belong to the want largest (ties are resolved afterwards by
-// position); every key > thr belongs to them. Block-wide; uses s_hist[kBins] and s_info[3].
-template <typename KeyAt>
-__device__ void radix_select(KeyAt key_at, int n, uint32_t want, uint32_t* s_hist, int* s_info,
-                             uint32_t& thr, uint32_t& take) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  uint32_t prefix = 0, pmask = 0;
+// Block-wide (NT threads) min and max of per-thread values (s_red: 2 * NT / 32 words).
+template <int NT>
+__device__ __forceinline__ void block_min_max(uint32_t& mn, uint32_t& mx, uint32_t* s_red) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  mn = __reduce_min_sync(0xffffffffu, mn);
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  if (lane == 0) {
+    s_red[warp] = mn;
+    s_red[NW + warp] = mx;
+  }
+  __syncthreads();
+  mn = s_red[0];
+  mx = s_red[NW];
+  for (int w = 1; w < NW; ++w) {
+    mn = min(mn, s_red[w]);
+    mx = max(mx, s_red[NW + w]);
+  }
+  __syncthreads();
+}
+
+// Block-wide (NT threads) exclusive prefix of a per-thread 64-bit value; returns the prefix and
+// the total (s_red: NT / 32 words of 64 bits).
+template <int NT>
+__device__ __forceinline__ uint64_t block_excl_scan64(uint64_t v, uint64_t& total, uint64_t* s_red) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint64_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_red[warp] = x;
+  __syncthreads();
+  uint64_t before = 0;
+  total = 0;
+  for (int w = 0; w < NW; ++w) {
+    const uint64_t t = s_red[w];
+    if (w < warp) before += t;
+    total += t;
+  }
+  __syncthreads();
+  return before + x - v;
+}
+
+// Radix select over n keys read through key_at(i), all in [kmin, kmax]: the digits are taken
+// from v = key - kmin, starting at the highest bit of kmax - kmin, at most 11 bits a pass, so
+// the first histogram already spreads the keys over the range they occupy. On return the want
+// largest keys are the keys > thr plus `take` of the keys == thr (exact result), unless
+// max_passes ran out first: then take = 0 and the keys > thr are a superset of them (the lowest
+// key of the bin that holds the want-th largest is thr + 1). Block-wide (NT threads); s_hist:
+// 2048 words, s_wsum: NT / 32 words.
+template <int NT, typename KeyAt>
+__device__ void radix_select(KeyAt key_at, int n, uint32_t want, uint32_t kmin, uint32_t kmax,
+                             int max_passes, uint32_t* s_hist, uint32_t* s_wsum, int* s_info,
+                             int64_t& thr, uint32_t& take) {
+  const int tid = threadIdx.x;
+  int bits = 32 - __clz(kmax - kmin);  // 0 when every key is equal
+  uint32_t prefix = 0;                 // the digits decided so far (bits above `bits`)
+  if (bits == 0 || want == 0) {
+    thr = (int64_t)kmin;
+    take = want;
+    if (want == 0) thr = (int64_t)kmax;
+    return;
+  }
 #pragma unroll 1
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-    const int nb = pass == 2 ? 1024 : 2048;
-    for (int i = tid; i < nb; i += kThreads) s_hist[i] = 0u;
+  for (int pass = 0;; ++pass) {
+    const int dbits = min(11, bits);
+    const int shift = bits - dbits;
+    const int nb = 1 << dbits;
+    for (int i = tid; i < nb; i += NT) s_hist[i] = 0u;
     __syncthreads();
-    for (int i = tid; i < n; i += kThreads) {
-      const uint32_t key = key_at(i);
-      if ((key & pmask) == prefix) atomicAdd(&s_hist[(key >> shift) & (nb - 1)], 1u);
+    for (int i = tid; i < n; i += NT) {
+      const uint32_t v = key_at(i) - kmin;
+      if ((uint32_t)((uint64_t)v >> bits) == prefix)
+        atomicAdd(&s_hist[(v >> shift) & (uint32_t)(nb - 1)], 1u);
     }
     __syncthreads();
-    if (warp == 0) {
-      int bin;
-      uint32_t above, cnt;
-      bool found;
-      find_bin([&](int j) { return s_hist[j]; }, nb, want, lane, bin, above, cnt, found);
-      if (lane == 0) {
-        if (!found) raise_flag(8u);
-        s_info[0] = bin;
-        s_info[1] = (int)above;
-        s_info[2] = (int)cnt;
-      }
-    }
-    __syncthreads();
-    want -= (uint32_t)s_info[1];
-    prefix |= (uint32_t)s_info[0] << shift;
-    pmask |= (uint32_t)(nb - 1) << shift;
-    const uint32_t in_bin = (uint32_t)s_info[2];
-    __syncthreads();
-    if (want == in_bin) {  // the whole bin is taken: everything >= its lowest key
-      thr = prefix - 1u;   // prefix > 0: keys of finite scores are >= 0x00800000
+    find_bin<NT>(s_hist, nb, want, s_wsum, s_info);
+    if (!s_info[3]) {  // fewer keys than want: inconsistent input, select every key
+      if (tid == 0) raise_flag(8u);
+      thr = (int64_t)kmin - 1;
       take = 0;
       return;
     }
+    want -= (uint32_t)s_info[1];
+    prefix = (prefix << dbits) | (uint32_t)s_info[0];
+    bits = shift;
+    const uint32_t in_bin = (uint32_t)s_info[2];
+    __syncthreads();  // s_info and s_hist are reused by the next pass
+    if (want == in_bin || (bits > 0 && pass + 1 == max_passes)) {
+      // the whole bin (or, out of passes, a superset): every key >= its lowest key
+      thr = (int64_t)kmin + ((int64_t)prefix << bits) - 1;
+      take = 0;
+      return;
+    }
+    if (bits == 0) {
+      thr = (int64_t)kmin + prefix;
+      take = want;
+      return;
+    }
   }
-  thr = prefix;
-  take = want;
+}
+
+// Exact threshold for the want largest of n keys in [kmin, kmax] (same contract as
+// radix_select): one 11-bit histogram pass over the key range finds the bin that holds the
+// want-th largest key; a bin taken whole ends it, and a bin of at most 256 keys is resolved by
+// ranking its keys against each other in shared memory; larger bins fall back to radix_select.
+template <int NT, typename KeyAt>
+__device__ void select_threshold(KeyAt key_at, int n, uint32_t want, uint32_t kmin, uint32_t kmax,
+                                 uint32_t* s_hist, uint32_t* s_wsum, int* s_info, int64_t& thr,
+                                 uint32_t& take) {
+  const int tid = threadIdx.x;
+  const int bits = 32 - __clz(kmax - kmin);
+  if (bits <= 11 || want == 0) {
+    radix_select<NT>(key_at, n, want, kmin, kmax, 3, s_hist, s_wsum, s_info, thr, take);
+    return;
+  }
+  const int shift = bits - 11;
+  for (int i = tid; i < kBins; i += NT) s_hist[i] = 0u;
+  __syncthreads();
+  for (int i = tid; i < n; i += NT) atomicAdd(&s_hist[(key_at(i) - kmin) >> shift], 1u);
+  __syncthreads();
+  find_bin<NT>(s_hist, kBins, want, s_wsum, s_info);
+  if (!s_info[3]) {  // fewer keys than want: inconsistent input, select every key
+    if (tid == 0) raise_flag(8u);
+    thr = (int64_t)kmin - 1;
+    take = 0;
+    return;
+  }
+  const uint32_t bin = (uint32_t)s_info[0], m = (uint32_t)s_info[2];
+  const uint32_t w2 = want - (uint32_t)s_info[1];
+  __syncthreads();  // s_info and s_hist are reused below
+  if (w2 == m) {
+    thr = (int64_t)kmin + ((int64_t)bin << shift) - 1;
+    take = 0;
+    return;
+  }
+  if (m > 256) {
+    radix_select<NT>(key_at, n, want, kmin, kmax, 3, s_hist, s_wsum, s_info, thr, take);
+    return;
+  }
+  if (tid == 0) s_info[3] = 0;
+  __syncthreads();
+  for (int i = tid; i < n; i += NT) {
+    const uint32_t key = key_at(i);
+    if (((key - kmin) >> shift) == bin) s_hist[atomicAdd(&s_info[3], 1)] = key;
+  }
+  __syncthreads();
+  if (tid < (int)m) {
+    const uint32_t x = s_hist[tid];
+    uint32_t gt = 0, eq = 0;
+    for (uint32_t j = 0; j < m; ++j) {
+      const uint32_t y = s_hist[j];
+      gt += y > x;
+      eq += y == x;
+    }
+    if (gt < w2 && w2 <= gt + eq) {  // x is the w2-th largest of the bin (equal keys agree)
+      s_info[0] = (int)x;
+      s_info[1] = (int)(w2 - gt);
+    }
+  }
+  __syncthreads();
+  thr = (int64_t)(uint32_t)s_info[0];
+  take = (uint32_t)s_info[1];
+  __syncthreads();
 }
 
 struct Prep {
@@ -147,9 +269,9 @@ struct Prep {
                  // key at kPrepThr, mode at kPrepMode
 };
 struct Cands {
-  uint32_t* key;       // [pairs][n_chunks][kWarps][chunk / kWarps]
+  uint32_t* key;       // [pairs][n_chunks][kRegionsPerChunk][chunk / kRegionsPerChunk]
   int32_t* pos;        // same layout
-  uint32_t* cnt;       // [pairs][n_chunks][kWarps]
+  uint32_t* cnt;       // [pairs][n_chunks][kRegionsPerChunk]
   int* attend_tickets; // [pairs] split-K tickets of the attention that follows, or null
 };
 
@@ -162,56 +284,55 @@ __device__ __forceinline__ uint32_t mix32(uint32_t x) {
   return x;
 }
 
-// Fragment registers of the digit matrix (B operand): column n = digit g; k-block kb, k-slot
-// 4t+j <-> row byte t*LB + 8kb + j and k-slot 16+4t+j <-> byte t*LB + 8kb + 4 + j (the same
-// permutation is applied to the code rows, so the dot products are unchanged).
+// Fragment registers of the digit matrix (B operand of mma m16n8k16, f16). Column n holds digit
+// n & 1 (the two digits repeated four times), so lane (g, t) finds the complete digit-0 and
+// digit-1 sums of its rows in accumulator columns 2t and 2t + 1. K-slots are permuted so that
+// each lane's MMA operands come from its own code bytes: in k-block kb (16 slots), slots
+// 2t, 2t+1, 2t+8, 2t+9 <-> bytes t*LB + 4kb + 0..3 of the row (LB = R / 4 bytes per lane); the
+// same permutation on both operands leaves the dot products unchanged.
 template <int R>
 struct DigitFrags {
-  uint32_t b0[R / 32], b1[R / 32];
+  uint32_t b0[R / 16], b1[R / 16];
   float sc0, sc1;
-  __device__ __forceinline__ void load(const uint8_t* dig, const float* scale, int lane) {
+  // dig: f16 [kDigits][R]; scale: the power-of-two weight of each digit
+  __device__ __forceinline__ void load(const uint16_t* dig, const float* scale, int lane) {
     constexpr int LB = R / 4;
     const int g = lane >> 2, t = lane & 3;
+    const uint16_t* d = dig + (g & 1) * R;
 #pragma unroll
-    for (int kb = 0; kb < R / 32; ++kb) {
-      b0[kb] = 0u;
-      b1[kb] = 0u;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        b0[kb] |= (uint32_t)dig[g * R + t * LB + 8 * kb + j] << (8 * j);
-        b1[kb] |= (uint32_t)dig[g * R + t * LB + 8 * kb + 4 + j] << (8 * j);
-      }
+    for (int kb = 0; kb < R / 16; ++kb) {
+      const int o = t * LB + 4 * kb;
+      b0[kb] = (uint32_t)d[o] | ((uint32_t)d[o + 1] << 16);
+      b1[kb] = (uint32_t)d[o + 2] | ((uint32_t)d[o + 3] << 16);
     }
-    sc0 = scale[2 * t];
-    sc1 = scale[2 * t + 1];
+    sc0 = scale[0];
+    sc1 = scale[1];
   }
 };
 
-// Scores of a 16-token tile: ra / rb are the permuted code rows of tokens g and g+8 held by lane
-// (g, t); on return every lane of the quad has token g's score in s0 and token g+8's in s1.
 template <int R>
-__device__ __forceinline__ void tile_scores(const uint32_t* ra, const uint32_t* rb,
-                                            const DigitFrags<R>& df, float& s0, float& s1) {
-  float c[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int kb = 0; kb < R / 32; ++kb)
-    mma_e4m3(c, ra[2 * kb], rb[2 * kb], ra[2 * kb + 1], rb[2 * kb + 1], df.b0[kb], df.b1[kb]);
-  s0 = c[0] * df.sc0 + c[1] * df.sc1;  // token g   (columns 2t, 2t+1)
-  s1 = c[2] * df.sc0 + c[3] * df.sc1;  // token g+8
-  s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
-  s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
-  s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
-  s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
-}
-
-template <int R>
-__device__ __forceinline__ void load_row(uint32_t* dst, const uint8_t* src, bool ok) {
+__device__ __forceinline__ void load_srow(uint32_t* dst, const uint8_t* src) {
   if (R == 32) {
-    const uint2 v = ok ? ld_stream_v2(src) : make_uint2(0u, 0u);
+    const uint2 v = *reinterpret_cast<const uint2*>(src);
     dst[0] = v.x;
     dst[1] = v.y;
   } else {
-    const uint4 v = ok ? ld_stream_v4(src) : make_uint4(0u, 0u, 0u, 0u);
+    const uint4 v = *reinterpret_cast<const uint4*>(src);
+    dst[0] = v.x;
+    dst[1] = v.y;
+    dst[2] = v.z;
+    dst[3] = v.w;
+  }
+}
+
+template <int R>
+__device__ __forceinline__ void load_row(uint32_t* dst, const uint8_t* src) {
+  if (R == 32) {
+    const uint2 v = ld_stream_v2(src);
+    dst[0] = v.x;
+    dst[1] = v.y;
+  } else {
+    const uint4 v = ld_stream_v4(src);
     dst[0] = v.x;
     dst[1] = v.y;
     dst[2] = v.z;
@@ -248,53 +369,96 @@ struct ChunkGeom {
 
 template <int R>
 struct ScanBuf {
-  static constexpr int kUnroll = kUnrollBytes / (R / 4);
+  static constexpr int kUnroll = kUnrollBytes / (R / 4);  // tiles per batch (even)
   uint32_t ra[kUnroll][R / 16], rb[kUnroll][R / 16];
 };
 
+// Rows of tiles [t0, t0 + kUnroll) (rows g and g+8 of each tile for lane (g, t)). The loads are
+// unconditional: a tile past t_end or the chunk's valid tokens, or on an unusable page, reads
+// page 0 instead (always allocated) and its tokens are never candidates (see scan_emit).
 template <int R>
 __device__ __forceinline__ void scan_load(ScanBuf<R>& buf, const ChunkGeom& cg,
                                           const int32_t* s_page, int t0, int t_end, int lane) {
   constexpr int LB = R / 4;
   const int g = lane >> 2, t = lane & 3;
   const int pmask = (1 << cg.page_shift) - 1;
+  const int lane_off = g * R + t * LB;
+  if (cg.page_shift >= 4) {  // a 16-token tile lies inside one page
 #pragma unroll
-  for (int u = 0; u < ScanBuf<R>::kUnroll; ++u) {
-    const bool live = t0 + u < t_end;
-    const int ta = (t0 + u) * 16 + g, tb = ta + 8;
-    // (a 16-token tile crosses pages only when the page size is below 16)
-    const int pa = live && ta < cg.n_local ? s_page[ta >> cg.page_shift] : -1;
-    const int pb = live && tb < cg.n_local ? s_page[tb >> cg.page_shift] : -1;
-    load_row<R>(buf.ra[u], cg.head_base + (int64_t)pa * cg.page_bytes + (ta & pmask) * R + t * LB,
-                pa >= 0);
-    load_row<R>(buf.rb[u], cg.head_base + (int64_t)pb * cg.page_bytes + (tb & pmask) * R + t * LB,
-                pb >= 0);
+    for (int u = 0; u < ScanBuf<R>::kUnroll; ++u) {
+      const int tok0 = (t0 + u) * 16;
+      const int pg = t0 + u < t_end && tok0 < cg.n_local ? s_page[tok0 >> cg.page_shift] : 0;
+      const uint8_t* row = cg.head_base + (size_t)(uint32_t)max(pg, 0) * cg.page_bytes +
+                           ((tok0 & pmask) * R + lane_off);
+      load_row<R>(buf.ra[u], row);
+      load_row<R>(buf.rb[u], row + 8 * R);
+    }
+  } else {
+#pragma unroll
+    for (int u = 0; u < ScanBuf<R>::kUnroll; ++u) {
+      const bool live = t0 + u < t_end;
+      const int ta = (t0 + u) * 16 + g, tb = ta + 8;
+      const int pa = live && ta < cg.n_local ? s_page[ta >> cg.page_shift] : 0;
+      const int pb = live && tb < cg.n_local ? s_page[tb >> cg.page_shift] : 0;
+      load_row<R>(buf.ra[u], cg.head_base + (size_t)(uint32_t)max(pa, 0) * cg.page_bytes +
+                                 ((ta & pmask) * R + t * LB));
+      load_row<R>(buf.rb[u], cg.head_base + (size_t)(uint32_t)max(pb, 0) * cg.page_bytes +
+                                 ((tb & pmask) * R + t * LB));
+    }
   }
 }
 
-// Keys >= thr of tiles [t0, t0 + kUnroll) appended in position order to this warp's region.
+// Scores of two 16-token tiles, one token per lane: lane (g, t) returns token
+// 16 * (t >> 1) + 8 * (t & 1) + g of the pair. ra / rb hold the lane's code bytes of rows g and
+// g + 8 (R / 4 bytes each); the codes are widened to f16 (exact) and multiplied on the tensor
+// cores with fp32 accumulation, s = 2^e0 C[:, 0] + 2^e1 C[:, 1].
+template <int R>
+__device__ __forceinline__ float pair_scores(const uint32_t* ra0, const uint32_t* rb0,
+                                             const uint32_t* ra1, const uint32_t* rb1,
+                                             const DigitFrags<R>& df, int t) {
+  float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int kb = 0; kb < R / 16; ++kb) {
+    mma_f16(c0, e4m3x2_to_f16x2((uint16_t)ra0[kb]), e4m3x2_to_f16x2((uint16_t)rb0[kb]),
+            e4m3x2_to_f16x2((uint16_t)(ra0[kb] >> 16)), e4m3x2_to_f16x2((uint16_t)(rb0[kb] >> 16)),
+            df.b0[kb], df.b1[kb]);
+    mma_f16(c1, e4m3x2_to_f16x2((uint16_t)ra1[kb]), e4m3x2_to_f16x2((uint16_t)rb1[kb]),
+            e4m3x2_to_f16x2((uint16_t)(ra1[kb] >> 16)), e4m3x2_to_f16x2((uint16_t)(rb1[kb] >> 16)),
+            df.b0[kb], df.b1[kb]);
+  }
+  const bool hi_row = t & 1, tile1 = t & 2;
+  const float x0 = hi_row ? c0[2] : c0[0], y0 = hi_row ? c0[3] : c0[1];
+  const float x1 = hi_row ? c1[2] : c1[0], y1 = hi_row ? c1[3] : c1[1];
+  return (tile1 ? x1 : x0) * df.sc0 + (tile1 ? y1 : y0) * df.sc1;
+}
+
+// Keys >= thr of the tiles [t0, t0 + kUnroll) appended in position order to this warp's region.
 template <int R>
 __device__ __forceinline__ void scan_emit(const ScanBuf<R>& buf, const DigitFrags<R>& df,
-                                          const ChunkGeom& cg, int t0, int t_end, uint32_t thr,
+                                          const ChunkGeom& cg, const int32_t* s_page, int t0,
+                                          int t_end, uint32_t thr,
                                           uint32_t* rkey, int32_t* rpos, uint32_t& run, int lane) {
   const int g = lane >> 2, t = lane & 3;
+  const int tok_in_pair = 16 * (t >> 1) + 8 * (t & 1) + g;
+  // lanes holding earlier tokens of the pair: every lane of a lower t, and lower g for this t
+  const unsigned quad_t = 0x11111111u << t;
+  const unsigned earlier_t = 0x11111111u * ((1u << t) - 1u);
   const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
-  for (int u = 0; u < ScanBuf<R>::kUnroll; ++u) {
-    float s0, s1;
-    tile_scores<R>(buf.ra[u], buf.rb[u], df, s0, s1);
-    const int tok = (t0 + u) * 16 + g + 8 * t;  // lane t = 0 keeps token g, t = 1 token g+8
-    const uint32_t key = score_key(t == 0 ? s0 : s1);
-    const bool c = t < 2 && t0 + u < t_end && tok < cg.n_local && key >= thr;
+  for (int u = 0; u < ScanBuf<R>::kUnroll; u += 2) {
+    const float f = pair_scores<R>(buf.ra[u], buf.rb[u], buf.ra[u + 1], buf.rb[u + 1], df, t);
+    const int tok = (t0 + u) * 16 + tok_in_pair;
+    const bool c = t0 + u < t_end && tok < cg.n_local && score_key(f) >= thr &&
+                   (tok_in_pair < 16 || t0 + u + 1 < t_end) && s_page[tok >> cg.page_shift] >= 0;
     const unsigned m = __ballot_sync(0xffffffffu, c);
-    // position order inside the tile: tokens 0..7 sit on lanes 4g (t = 0), 8..15 on 4g+1
-    const unsigned m0 = m & 0x11111111u, m1 = m & 0x22222222u;
-    if (c) {
-      const uint32_t at = run + (t == 0 ? __popc(m0 & lt) : __popc(m0) + __popc(m1 & lt));
-      rkey[at] = key;
-      rpos[at] = cg.start + tok;
+    if (m) {
+      if (c) {
+        const uint32_t at = run + __popc(m & earlier_t) + __popc(m & quad_t & lt);
+        rkey[at] = score_key(f);
+        rpos[at] = cg.start + tok;
+      }
+      run += __popc(m);
     }
-    run += __popc(m);
   }
 }
 
@@ -310,11 +474,11 @@ __device__ __forceinline__ uint32_t scan_warp(const ChunkGeom& cg, const int32_t
   if (t0 < t_end) scan_load<R>(a, cg, s_page, t0, t_end, lane);
   while (t0 < t_end) {
     if (t0 + kU < t_end) scan_load<R>(b, cg, s_page, t0 + kU, t_end, lane);
-    scan_emit<R>(a, df, cg, t0, t_end, thr, rkey, rpos, run, lane);
+    scan_emit<R>(a, df, cg, s_page, t0, t_end, thr, rkey, rpos, run, lane);
     t0 += kU;
     if (t0 >= t_end) break;
     if (t0 + kU < t_end) scan_load<R>(a, cg, s_page, t0 + kU, t_end, lane);
-    scan_emit<R>(b, df, cg, t0, t_end, thr, rkey, rpos, run, lane);
+    scan_emit<R>(b, df, cg, s_page, t0, t_end, thr, rkey, rpos, run, lane);
     t0 += kU;
   }
   return run;
@@ -323,7 +487,7 @@ __device__ __forceinline__ uint32_t scan_warp(const ChunkGeom& cg, const int32_t
 // Page list of a chunk into shared memory (bounds checked; -1 = unusable page).
 __device__ __forceinline__ void load_pages(int32_t* s_page, const int32_t* bt, int n_pages,
                                            int64_t num_pages) {
-  for (int i = threadIdx.x; i < n_pages; i += kThreads) {
+  for (int i = threadIdx.x; i < n_pages; i += blockDim.x) {
     int32_t pg = bt[i];
     if (pg < 0 || (int64_t)pg >= num_pages) {
       raise_flag(1u);
@@ -341,12 +505,14 @@ __device__ __forceinline__ int clamp_len(int L, int max_len) {
   return L;
 }
 
-// Scan of chunk c of pair `pair` by the calling CTA (page list already in s_page); writes this
-// chunk's kWarps regions and their counts.
+// Scan of chunk c of pair `pair` on the CUDA cores' warp-level MMA, used by the select kernel's
+// rescan (page list already in s_page): warp q < kRegionsPerChunk takes quarter q of the chunk
+// and writes that region and its count.
 template <int R>
 __device__ void scan_chunk(const ScanArgs& a, int pair, int c, int L, uint32_t thr,
                            const DigitFrags<R>& df, const int32_t* s_page) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (warp >= kRegionsPerChunk) return;
   const int h = pair % a.h_kv;
   ChunkGeom cg;
   cg.start = c * a.chunk;
@@ -354,14 +520,14 @@ __device__ void scan_chunk(const ScanArgs& a, int pair, int c, int L, uint32_t t
   cg.page_shift = a.page_shift;
   cg.page_bytes = ((uint32_t)a.h_kv << a.page_shift) * R;
   cg.head_base = a.score_cache + ((int64_t)h << a.page_shift) * R;
-  const int seg = a.chunk / kWarps;
-  const int64_t region = (((int64_t)pair * a.n_chunks + c) * kWarps + warp) * seg;
+  const int seg = a.chunk / kRegionsPerChunk;
+  const int64_t reg = ((int64_t)pair * a.n_chunks + c) * kRegionsPerChunk + warp;
   const int n_tiles = (cg.n_local + 15) >> 4;
-  const int tpw = seg / 16;  // tiles per warp (one region)
+  const int tpw = seg / 16;
   const int t_begin = min(n_tiles, warp * tpw), t_end = min(n_tiles, t_begin + tpw);
-  const uint32_t n = scan_warp<R>(cg, s_page, df, thr, t_begin, t_end, a.cands.key + region,
-                                  a.cands.pos + region, lane);
-  if (lane == 0) a.cands.cnt[((int64_t)pair * a.n_chunks + c) * kWarps + warp] = n;
+  const uint32_t n = scan_warp<R>(cg, s_page, df, thr, t_begin, t_end, a.cands.key + reg * seg,
+                                  a.cands.pos + reg * seg, lane);
+  if (lane == 0) a.cands.cnt[reg] = n;
 }
 
 template <int D, int R>
@@ -380,13 +546,14 @@ __global__ void __launch_bounds__(kThreads, 3) scan_kernel(ScanArgs a) {
   const uint8_t* rec = a.prep.rec + (int64_t)pair * kPrepBytes;
   const int mode = *reinterpret_cast<const int*>(rec + kPrepMode);
   if (mode == kModeAll || n_local == 0) {
-    if ((threadIdx.x & 31) == 0)
-      a.cands.cnt[((int64_t)pair * a.n_chunks + c) * kWarps + (threadIdx.x >> 5)] = 0u;
+    if ((threadIdx.x & 31) == 0 && (threadIdx.x >> 5) < kRegionsPerChunk)
+      a.cands.cnt[((int64_t)pair * a.n_chunks + c) * kRegionsPerChunk + (threadIdx.x >> 5)] = 0u;
     pdl_trigger();
     return;
   }
   DigitFrags<R> df;
-  df.load(rec, reinterpret_cast<const float*>(rec + kPrepScale), threadIdx.x & 31);
+  df.load(reinterpret_cast<const uint16_t*>(rec), reinterpret_cast<const float*>(rec + kPrepScale),
+          threadIdx.x & 31);
   const uint32_t thr = *reinterpret_cast<const uint32_t*>(rec + kPrepThr);
   scan_chunk<R>(a, pair, c, L, thr, df, scan_pages);
   pdl_trigger();
@@ -411,170 +578,236 @@ struct PrepArgs {
   StoreNew store;  // decode: the new token (position seq_len - 1)
 };
 
+// Sampled position i of (pair, L): one per stratum of L / kSample tokens at an offset drawn from
+// a 32-bit mix of (i, pair) (scaled to the stratum by a high multiply), never the last position
+// (the token a decode step stores right now).
+__device__ __forceinline__ int sample_pos(int i, int pair, int L) {
+  const int stratum = L / kSample;
+  const uint32_t hsh = mix32((uint32_t)i * 0x9E3779B9u ^ ((uint32_t)pair * 0x85EBCA6Bu + 1u));
+  return min(i * stratum + (int)__umulhi(hsh, (uint32_t)stratum), L - 2);
+}
+
+constexpr int kQGroups = kThreads / 16;  // query rows loaded per pass (16 threads x 8 dims a row)
+
+// Dynamic shared memory of the prep kernel.
+template <int D, int R>
+struct PrepSmem {
+  uint8_t rows[kSample * R];     // code rows of the sampled positions
+  float m[R * D];                // M_h, row-major [R][D]
+  float qpart[kQGroups][D];      // partial sums of the group's query rows
+  uint32_t skey[kSample];        // sampled keys
+  uint32_t hist[kBins];
+  uint8_t valid[kSample];        // sampled position on a usable page
+};
+
 template <int D, int R, bool STORE>
 __global__ void __launch_bounds__(kThreads) prep_kernel(PrepArgs a) {
   constexpr int LB = R / 4;
+  constexpr int kTilesPerWarp = kSample / 16 / kWarps;  // 16
+  extern __shared__ __align__(16) uint8_t prep_dyn[];
+  PrepSmem<D, R>& sm = *reinterpret_cast<PrepSmem<D, R>*>(prep_dyn);
   __shared__ float s_qbar[D];
-  __shared__ float s_p[R];
   __shared__ float s_k[D];
-  __shared__ __align__(16) uint8_t s_dig[kDigits * R];
+  __shared__ float s_p[R];
+  __shared__ __align__(16) uint16_t s_dig[kDigits * R];  // f16 digits
   __shared__ float s_scale[kDigits];
-  __shared__ uint32_t s_skey[kSample];
-  __shared__ int64_t s_srow[kSample];
-  __shared__ uint32_t s_hist[kBins];
+  __shared__ uint32_t s_wsum[2 * kWarps];
   __shared__ int s_info[4];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
   const int pair = blockIdx.x;
   const int b = pair / a.h_kv, h = pair % a.h_kv;
   const int G = a.h_q / a.h_kv;
   const int page_size = 1 << a.page_shift;
-  const int L = clamp_len(a.seq_lens[b], a.max_pages << a.page_shift);
   const int32_t* bt = a.block_table + (int64_t)b * a.max_pages;
   const float* m_h = a.basis + (int64_t)h * R * D;
 
-  // ---- decode: store the new token (K/V rows and scoring code) ---------------------------------
-  if (STORE && L > 0) {
+  // ---- independent loads first: M_h into shared memory (async), L, qbar, the sample's pages ----
+  for (int i = tid; i < R * D / 4; i += kThreads) cp_async16(smem_u32(sm.m + 4 * i), m_h + 4 * i, 16);
+  cp_async_commit();
+  const int L = clamp_len(a.seq_lens[b], a.max_pages << a.page_shift);
+  {
+    // the G query rows of this KV head: 16 threads x 8 dims per row, kQGroups rows at a time
+    static_assert(D == 128, "query row split");
+    const uint16_t* qh = a.q + ((int64_t)b * a.h_q + (int64_t)h * G) * D;
+    const int rg = tid / 16, d8 = (tid % 16) * 8;
+    float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int r = rg; r < G; r += kQGroups) {
+      const uint4 v = *reinterpret_cast<const uint4*>(qh + (int64_t)r * D + d8);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        part[2 * e] += bf16_lo(w[e]);
+        part[2 * e + 1] += bf16_hi(w[e]);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sm.qpart[rg][d8 + e] = part[e];
+  }
+  int mode = kModeScan;
+  int k = 0;  // sampled keys to reach (0: no sampling, every key is a candidate)
+  if (L <= a.budget) {
+    mode = kModeAll;
+  } else if (L > kExactMax) {
+    const double expect = (double)a.budget * kSample / (double)L;
+    k = (int)ceil(expect + 4.0 * sqrt(expect) + 8.0);
+    if (k >= kSample / 2) k = 0;
+  }
+  if (k) {
+    // the sampled code rows go straight to shared memory (asynchronous 16-byte copies issued as
+    // soon as each page number arrives; a row on an unusable page is zero-filled)
+    constexpr int kPer = kSample / kThreads;
+    int pos[kPer], pg[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      pos[u] = sample_pos(tid + u * kThreads, pair, L);
+      pg[u] = bt[pos[u] >> a.page_shift];
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = tid + u * kThreads;
+      const bool ok = pg[u] >= 0 && (int64_t)pg[u] < a.num_pages;
+      sm.valid[i] = ok;
+      const uint8_t* src = a.score_cache +
+          ((((int64_t)(ok ? pg[u] : 0) * a.h_kv + h) << a.page_shift) + (pos[u] & (page_size - 1))) * R;
+#pragma unroll
+      for (int c = 0; c < R / 16; ++c)
+        cp_async16(smem_u32(sm.rows + i * R + c * 16), src + c * 16, ok ? 16 : 0);
+    }
+    cp_async_commit();
+  }
+  const bool store = STORE && L > 0;
+  int32_t st_page = -1;
+  if (store) {  // decode: copy the new token's K and V rows into the cache
     const StoreNew& st = a.store;
     const int pos = L - 1;
-    const int32_t page = bt[pos >> a.page_shift];
-    const int off = pos & (page_size - 1);
-    const bool ok = page >= 0 && (int64_t)page < a.num_pages;
-    if (!ok && tid == 0) raise_flag(1u);
+    st_page = bt[pos >> a.page_shift];
+    if (st_page < 0 || (int64_t)st_page >= a.num_pages) {
+      if (tid == 0) raise_flag(1u);
+      st_page = -1;
+    }
     const uint16_t* krow = st.k_new + ((int64_t)b * a.h_kv + h) * D;
     const uint16_t* vrow = st.v_new + ((int64_t)b * a.h_kv + h) * D;
-    for (int i = tid; i < D; i += kThreads) s_k[i] = bf16_to_f(krow[i]);
-    if (ok) {
-      const int64_t base = (int64_t)page * st.page_stride + (int64_t)off * st.slot_stride +
-                           (int64_t)h * st.head_stride;
-      for (int i = tid; i < D; i += kThreads) {
-        st.k_cache[base + i] = krow[i];
-        st.v_cache[base + i] = vrow[i];
-      }
-    }
-    __syncthreads();
-    if (ok) {
-      uint8_t* dst = st.score_cache + (((int64_t)page * a.h_kv + h) * page_size + off) * R;
-      for (int j = tid; j < R; j += kThreads) {
-        const float* mrow = m_h + (int64_t)j * D;
-        double acc = 0.0;
-        for (int i = 0; i < D; ++i) acc = fma((double)mrow[i], (double)s_k[i], acc);
-        dst[j] = f64_to_e4m3(acc);
+    for (int i = tid; i < D; i += kThreads) {
+      const uint16_t kv = krow[i], vv = vrow[i];
+      s_k[i] = bf16_to_f(kv);
+      if (st_page >= 0) {
+        const int64_t base = (int64_t)st_page * st.page_stride +
+                             (int64_t)(pos & (page_size - 1)) * st.slot_stride +
+                             (int64_t)h * st.head_stride;
+        st.k_cache[base + i] = kv;
+        st.v_cache[base + i] = vv;
       }
     }
   }
-
-  // ---- projected group-mean query and its FP8 digits -------------------------------------------
-  const uint16_t* qh = a.q + ((int64_t)b * a.h_q + (int64_t)h * G) * D;
+  if (k) cp_async_wait<1>();  // M_h landed; the sample rows may still be in flight
+  else cp_async_wait<0>();
+  __syncthreads();
   for (int i = tid; i < D; i += kThreads) {
     float acc = 0.f;
-    for (int gg = 0; gg < G; ++gg) acc += bf16_to_f(qh[(int64_t)gg * D + i]);
+    for (int r = 0; r < min(G, kQGroups); ++r) acc += sm.qpart[r][i];
     s_qbar[i] = acc / (float)G;
   }
-  __syncthreads();
+
+  __syncthreads();  // qbar
+
+  // ---- p = M_h qbar and, at decode, the new token's code e4m3(M_h k) ---------------------------
   {
     constexpr int TPJ = kThreads / R;  // threads per output
     constexpr int DPT = D / TPJ;
     static_assert(TPJ >= 1 && TPJ <= 32 && D % TPJ == 0, "projection split");
     const int j = tid / TPJ, sub = tid % TPJ;
-    const float* mrow = m_h + (int64_t)j * D + sub * DPT;
+    const float* mrow = sm.m + j * D + sub * DPT;
     float acc = 0.f;
+    double acc_k = 0.0;
 #pragma unroll
-    for (int i = 0; i < DPT; ++i) acc = fmaf(mrow[i], s_qbar[sub * DPT + i], acc);
+    for (int i = 0; i < DPT; ++i) {
+      acc = fmaf(mrow[i], s_qbar[sub * DPT + i], acc);
+      if (store) acc_k = fma((double)mrow[i], (double)s_k[sub * DPT + i], acc_k);
+    }
 #pragma unroll
-    for (int o = TPJ / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (sub == 0) s_p[j] = acc;
+    for (int o = TPJ / 2; o > 0; o >>= 1) {
+      acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (store) acc_k += __shfl_xor_sync(0xffffffffu, acc_k, o);
+    }
+    if (sub == 0) {
+      s_p[j] = acc;
+      if (store && st_page >= 0) {
+        const int pos = L - 1;
+        a.store.score_cache[(((int64_t)st_page * a.h_kv + h) * page_size + (pos & (page_size - 1))) * R + j] =
+            f64_to_e4m3(acc_k);
+      }
+    }
   }
   __syncthreads();
   if (warp == 0) {
-    // digit c: the scale 2^e_c puts the largest remaining component in [128, 256), inside the
-    // E4M3 range, and D_c = e4m3(remainder / 2^e_c); the remainder update is exact
+    // p = 2^-e0 D0 + 2^-e1 D1 with f16 digit vectors: D0 = f16(p 2^e0), e0 chosen so that the
+    // largest |component| lands in [2^14, 2^15) (inside the f16 range), and D1 = f16(r 2^e1) for
+    // the remainder r = p 2^e0 - D0 (exact in fp32), scaled the same way; about 22 significant
+    // bits of every component relative to the largest one.
     float rem[R / 32];
 #pragma unroll
     for (int i = 0; i < R / 32; ++i) rem[i] = s_p[lane + 32 * i];
+    float weight = 1.f;  // 2^-(e0 + ... + e_c): the value of one unit of the current remainder
     for (int c = 0; c < kDigits; ++c) {
       float mx = 0.f;
 #pragma unroll
       for (int i = 0; i < R / 32; ++i) mx = fmaxf(mx, fabsf(rem[i]));
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      float sc = 0.f, inv = 0.f;
-      if (mx > 0.f) {
-        const int ex = (int)((__float_as_uint(mx) >> 23) & 0xFF) - 127 - 7;
-        sc = ldexpf(1.0f, ex);
-        inv = ldexpf(1.0f, -ex);
-      }
+      int ex = 0;
+      if (mx > 0.f) ex = min(100, 14 - ((int)((__float_as_uint(mx) >> 23) & 0xFF) - 127));
+      const float up = ldexpf(1.0f, ex);
+      weight = ldexpf(weight, -ex);
 #pragma unroll
       for (int i = 0; i < R / 32; ++i) {
-        uint8_t code = 0;
-        if (mx > 0.f) {
-          uint16_t pk;
-          asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %1;" : "=h"(pk) : "f"(rem[i] * inv));
-          code = (uint8_t)(pk & 0xFF);
-          rem[i] -= e4m3x2_to_f2((uint16_t)code).x * sc;
-        }
-        s_dig[c * R + lane + 32 * i] = code;
+        const float v = rem[i] * up;
+        const __half dh = __float2half_rn(v);
+        s_dig[c * R + lane + 32 * i] = __half_as_ushort(dh);
+        rem[i] = v - __half2float(dh);
       }
-      if (lane == 0) s_scale[c] = sc;
+      if (lane == 0) s_scale[c] = weight;
     }
   }
   __syncthreads();
   uint8_t* rec = a.prep.rec + (int64_t)pair * kPrepBytes;
-  for (int i = tid; i < kDigits * R; i += kThreads) rec[i] = s_dig[i];
+  for (int i = tid; i < kDigits * R; i += kThreads) reinterpret_cast<uint16_t*>(rec)[i] = s_dig[i];
   if (tid < kDigits) reinterpret_cast<float*>(rec + kPrepScale)[tid] = s_scale[tid];
 
-  // ---- candidate threshold --------------------------------------------------------------------
-  int mode = kModeScan;
+  // ---- candidate threshold from the sample ----------------------------------------------------
   uint32_t thr = 0u;  // every key of a finite score is above 0
-  if (L <= a.budget) {
-    mode = kModeAll;
-  } else if (L > kExactMax) {
-    const double expect = (double)a.budget * kSample / (double)L;
-    const int k = (int)ceil(2.0 * expect + 4.0 * sqrt(expect) + 8.0);
-    if (k < kSample / 2) {
-      // stratified sample: one position per stratum of L / kSample tokens (never the new
-      // token, whose code this kernel may have just written)
-      const int stratum = L / kSample;
-      for (int i = tid; i < kSample; i += kThreads) {
-        const uint32_t hsh = mix32((uint32_t)i * 0x9E3779B9u ^ ((uint32_t)pair * 0x85EBCA6Bu + 1u));
-        int pos = i * stratum + (int)(hsh % (uint32_t)stratum);
-        if (pos >= L - 1) pos = L - 2;
-        const int32_t pg = bt[pos >> a.page_shift];
-        s_srow[i] = (pg < 0 || (int64_t)pg >= a.num_pages)
-                        ? (int64_t)-1
-                        : (((int64_t)pg * a.h_kv + h) << a.page_shift) + (pos & (page_size - 1));
-      }
-      __syncthreads();
-      DigitFrags<R> df;
-      df.load(s_dig, s_scale, lane);
-      const int g = lane >> 2, t = lane & 3;
-      // 128 tiles of 16 samples, 16 per warp in two batches of 8; loads issued before the math
-      constexpr int kBatch = 8;
-      for (int bt0 = 0; bt0 < kSample / 16 / kWarps; bt0 += kBatch) {
-        uint32_t ra[kBatch][R / 16], rb[kBatch][R / 16];
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-          const int tile = warp * (kSample / 16 / kWarps) + bt0 + u;
-          const int64_t sa = s_srow[tile * 16 + g], sb = s_srow[tile * 16 + g + 8];
-          load_row<R>(ra[u], a.score_cache + (sa < 0 ? 0 : sa) * R + t * LB, sa >= 0);
-          load_row<R>(rb[u], a.score_cache + (sb < 0 ? 0 : sb) * R + t * LB, sb >= 0);
-        }
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-          float s0, s1;
-          tile_scores<R>(ra[u], rb[u], df, s0, s1);
-          const int tile = warp * (kSample / 16 / kWarps) + bt0 + u;
-          if (t < 2) s_skey[tile * 16 + g + 8 * t] = score_key(t == 0 ? s0 : s1);
-        }
-      }
-      __syncthreads();
-      uint32_t take;
-      radix_select([&](int i) { return s_skey[i]; }, kSample, (uint32_t)k, s_hist, s_info, thr,
-                   take);
-      // candidates: keys >= the k-th largest sampled key (radix_select returns that key itself,
-      // or one below the lowest key of a bin taken whole)
-      if (take == 0u) thr += 1u;
+  if (k) {
+    cp_async_wait<0>();
+    __syncthreads();  // every thread's sample rows
+    DigitFrags<R> df;
+    df.load(s_dig, s_scale, lane);
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+#pragma unroll 4
+    for (int u = 0; u < kTilesPerWarp; u += 2) {
+      const int i0 = (warp * kTilesPerWarp + u) * 16;
+      uint32_t ra0[R / 16], rb0[R / 16], ra1[R / 16], rb1[R / 16];
+      load_srow<R>(ra0, sm.rows + (i0 + g) * R + t * LB);
+      load_srow<R>(rb0, sm.rows + (i0 + g + 8) * R + t * LB);
+      load_srow<R>(ra1, sm.rows + (i0 + 16 + g) * R + t * LB);
+      load_srow<R>(rb1, sm.rows + (i0 + 24 + g) * R + t * LB);
+      const float f = pair_scores<R>(ra0, rb0, ra1, rb1, df, t);
+      // lane t holds sample 16 * (t >> 1) + 8 * (t & 1) + g of the two tiles
+      const int i = i0 + 16 * (t >> 1) + 8 * (t & 1) + g;
+      // a sample on an unusable page (flagged by the scan) counts as the lowest key
+      const uint32_t key = sm.valid[i] ? score_key(f) : 0u;
+      kmin = min(kmin, key);
+      kmax = max(kmax, key);
+      sm.skey[i] = key;
     }
+    block_min_max<kThreads>(kmin, kmax, s_wsum);  // (its barrier also publishes the keys)
+    // one radix pass of 11 bits over the sample's own key range: the lowest key of the bin that
+    // holds the k-th largest sampled key (or that key itself when the range is narrow)
+    int64_t t64;
+    uint32_t take;
+    radix_select<kThreads>([&](int i) { return sm.skey[i]; }, kSample, (uint32_t)k, kmin, kmax, 1,
+                           sm.hist, s_wsum, s_info, t64, take);
+    thr = (uint32_t)(take ? t64 : t64 + 1);  // candidates: keys >= thr
   }
   if (tid == 0) {
     *reinterpret_cast<uint32_t*>(rec + kPrepThr) = thr;
@@ -595,29 +828,32 @@ struct SelectArgs {
   int32_t* count;
 };
 
+constexpr int kSelThreads = 512;
+constexpr int kSelWarps = kSelThreads / 32;
+
 template <int D, int R>
-__global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs s) {
+__global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
   extern __shared__ uint32_t sel_dyn[];  // keys [kSelectCap] then positions [kSelectCap]
   uint32_t* s_ckey = sel_dyn;
   int32_t* s_cpos = reinterpret_cast<int32_t*>(sel_dyn + kSelectCap);
   __shared__ uint32_t s_hist[kBins];
   __shared__ int s_info[4];
   __shared__ uint32_t s_roff[kMaxRegions + 1];
-  __shared__ uint32_t s_wa[kWarps], s_wb[kWarps];
+  __shared__ uint32_t s_wsum[2 * kSelWarps];
+  __shared__ uint64_t s_red64[kSelWarps];
 
   const ScanArgs& a = s.scan;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, lane = tid & 31;
   const int pair = blockIdx.x;
   const int b = pair / a.h_kv;
   const int L = clamp_len(a.seq_lens[b], a.max_pages << a.page_shift);
   const int budget = a.budget;
   int32_t* out_idx = s.idx + (int64_t)pair * budget;
-  const unsigned lt = (1u << lane) - 1u;
   pdl_wait();  // the scan's candidates
   const uint8_t* rec = a.prep.rec + (int64_t)pair * kPrepBytes;
   const int mode = *reinterpret_cast<const int*>(rec + kPrepMode);
   if (mode == kModeAll) {
-    for (int j = tid; j < budget; j += kThreads) out_idx[j] = j < L ? j : -1;
+    for (int j = tid; j < budget; j += kSelThreads) out_idx[j] = j < L ? j : -1;
     if (tid == 0) {
       s.count[pair] = L;
       if (a.cands.attend_tickets) a.cands.attend_tickets[pair] = 0;
@@ -625,26 +861,34 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs s) {
     pdl_trigger();
     return;
   }
-  const int n_reg = a.n_chunks * kWarps;
-  const int seg = a.chunk / kWarps;
+  const int n_reg = a.n_chunks * kRegionsPerChunk;
+  const int seg = a.chunk / kRegionsPerChunk;
   const uint32_t* ck = a.cands.key + (int64_t)pair * n_reg * seg;
   const int32_t* cp = a.cands.pos + (int64_t)pair * n_reg * seg;
   const uint32_t* cc = a.cands.cnt + (int64_t)pair * n_reg;
   const uint32_t want = (uint32_t)min(budget, L);
 
-  // region offsets: exclusive prefix of the counts, in position order
+  // region offsets: exclusive prefix of the counts, in position order (each thread loads and
+  // sums a run of adjacent regions, then a block-wide scan)
   auto offsets = [&]() {
-    if (warp == 0) {
-      uint32_t run = 0;
-      for (int r0 = 0; r0 < n_reg; r0 += 32) {
-        const int r = r0 + lane;
-        const uint32_t v = r < n_reg ? cc[r] : 0u;
-        const uint32_t incl = warp_incl_scan(v, lane);
-        if (r < n_reg) s_roff[r] = run + incl - v;
-        run += __shfl_sync(0xffffffffu, incl, 31);
-      }
-      if (lane == 0) s_roff[n_reg] = run;
+    constexpr int kPer = kMaxRegions / kSelThreads;
+    const int per = (n_reg + kSelThreads - 1) / kSelThreads;  // <= kPer
+    const int r0 = min(n_reg, tid * per), r1 = min(n_reg, r0 + per);
+    uint32_t v[kPer];
+    uint32_t sum = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      v[i] = r0 + i < r1 ? cc[r0 + i] : 0u;
+      sum += v[i];
     }
+    uint64_t total;
+    uint32_t run = (uint32_t)block_excl_scan64<kSelThreads>(sum, total, s_red64);
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      if (r0 + i < r1) s_roff[r0 + i] = run;
+      run += v[i];
+    }
+    if (tid == 0) s_roff[n_reg] = (uint32_t)total;
     __syncthreads();
   };
   offsets();
@@ -653,7 +897,8 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs s) {
     // no threshold (all keys become candidates), then select exactly as usual
     if (tid == 0) raise_flag(16u);
     DigitFrags<R> df;
-    df.load(rec, reinterpret_cast<const float*>(rec + kPrepScale), lane);
+    df.load(reinterpret_cast<const uint16_t*>(rec), reinterpret_cast<const float*>(rec + kPrepScale),
+            lane);
     int32_t* s_page = reinterpret_cast<int32_t*>(s_ckey);  // free until the staging below
     for (int c = 0; c < a.n_chunks; ++c) {
       const int start = c * a.chunk;
@@ -670,18 +915,7 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs s) {
   }
   const uint32_t n = s_roff[n_reg];
   const bool staged = n <= (uint32_t)kSelectCap;
-  if (staged) {
-    // flatten the regions into shared memory (keys and positions, position order)
-    for (int r = warp; r < n_reg; r += kWarps) {
-      const uint32_t cnt = s_roff[r + 1] - s_roff[r], off = s_roff[r];
-      for (uint32_t i = lane; i < cnt; i += 32) {
-        s_ckey[off + i] = ck[(int64_t)r * seg + i];
-        s_cpos[off + i] = cp[(int64_t)r * seg + i];
-      }
-    }
-    __syncthreads();
-  }
-  // flattened candidate j -> region (the last r with s_roff[r] <= j) when not staged
+  // flattened candidate j -> region (the last r with s_roff[r] <= j)
   auto region_of = [&](int j) {
     int lo = 0, hi = n_reg - 1;
     while (lo < hi) {
@@ -690,65 +924,101 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs s) {
     }
     return lo;
   };
-  auto key_at = [&](int j) -> uint32_t {
-    if (staged) return s_ckey[j];
+  auto src_of = [&](int j) -> int64_t {
     const int r = region_of(j);
-    return ck[(int64_t)r * seg + (j - (int)s_roff[r])];
+    return (int64_t)r * seg + (j - (int)s_roff[r]);
   };
-  auto pos_at = [&](int j) -> int32_t {
-    if (staged) return s_cpos[j];
-    const int r = region_of(j);
-    return cp[(int64_t)r * seg + (j - (int)s_roff[r])];
-  };
-  uint32_t thr, take;
-  radix_select(key_at, (int)n, want, s_hist, s_info, thr, take);
-  // ordered emission: keys > thr, and the first `take` keys == thr in position order
-  constexpr int kBlk = kThreads * 8;  // candidates per block, 256 per warp
-  uint32_t written = 0, eq_seen = 0;
-  for (uint32_t b0 = 0; b0 < n; b0 += kBlk) {
-    const uint32_t w0 = min(n, b0 + (uint32_t)warp * 256u), w1 = min(n, w0 + 256u);
-    uint32_t n_gt = 0, n_eq = 0;
-    for (uint32_t i0 = w0; i0 < w1; i0 += 32) {
-      const uint32_t i = i0 + lane;
-      const uint32_t key = i < w1 ? key_at((int)i) : 0u;
-      n_gt += __popc(__ballot_sync(0xffffffffu, i < w1 && key > thr));
-      n_eq += __popc(__ballot_sync(0xffffffffu, i < w1 && key == thr));
-    }
-    if (lane == 0) {
-      s_wa[warp] = n_gt;
-      s_wb[warp] = n_eq;
-    }
-    __syncthreads();
-    uint32_t eq_before = eq_seen, sel_before = written, blk_sel = 0, blk_eq = 0;
-    for (int w = 0; w < kWarps; ++w) {
-      const uint32_t e_before = eq_seen + blk_eq;
-      const uint32_t rem = take > e_before ? take - e_before : 0u;
-      const uint32_t tk = s_wb[w] < rem ? s_wb[w] : rem;
-      if (w < warp) {
-        sel_before += s_wa[w] + tk;
-        eq_before += s_wb[w];
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  if (staged) {
+    // flatten the regions (keys and positions, position order) into shared memory: each warp
+    // copies 8 regions at a time, the first 64 candidates of each with all loads issued before
+    // any store (one round trip), the rare rest of a longer region afterwards; key range on
+    // the way
+    constexpr int kRB = 8;
+    for (int rb = (threadIdx.x >> 5) * kRB; rb < n_reg; rb += kSelWarps * kRB) {
+      uint32_t kk[kRB][2];
+      int32_t pp[kRB][2];
+#pragma unroll
+      for (int u = 0; u < kRB; ++u) {
+        const int r = rb + u;
+        const uint32_t cnt = r < n_reg ? s_roff[r + 1] - s_roff[r] : 0u;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const uint32_t i = lane + 32 * e;
+          kk[u][e] = i < cnt ? ck[(int64_t)r * seg + i] : 0u;
+          pp[u][e] = i < cnt ? cp[(int64_t)r * seg + i] : 0;
+        }
       }
-      blk_sel += s_wa[w] + tk;
-      blk_eq += s_wb[w];
+#pragma unroll
+      for (int u = 0; u < kRB; ++u) {
+        const int r = rb + u;
+        const uint32_t cnt = r < n_reg ? s_roff[r + 1] - s_roff[r] : 0u;
+        const uint32_t off = r < n_reg ? s_roff[r] : 0u;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const uint32_t i = lane + 32 * e;
+          if (i < cnt) {
+            s_ckey[off + i] = kk[u][e];
+            s_cpos[off + i] = pp[u][e];
+            kmin = min(kmin, kk[u][e]);
+            kmax = max(kmax, kk[u][e]);
+          }
+        }
+        for (uint32_t i = 64 + lane; i < cnt; i += 32) {
+          const uint32_t key = ck[(int64_t)r * seg + i];
+          s_ckey[off + i] = key;
+          s_cpos[off + i] = cp[(int64_t)r * seg + i];
+          kmin = min(kmin, key);
+          kmax = max(kmax, key);
+        }
+      }
     }
-    uint32_t pos = sel_before, eqs = eq_before;
-    for (uint32_t i0 = w0; i0 < w1; i0 += 32) {
-      const uint32_t i = i0 + lane;
-      const uint32_t key = i < w1 ? key_at((int)i) : 0u;
-      const bool is_eq = i < w1 && key == thr;
-      const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
-      const bool tk = (i < w1 && key > thr) || (is_eq && eqs + __popc(eqm & lt) < take);
-      const unsigned selm = __ballot_sync(0xffffffffu, tk);
-      const uint32_t at = pos + __popc(selm & lt);
-      if (tk && at < (uint32_t)budget) out_idx[at] = pos_at((int)i);
-      pos += __popc(selm);
-      eqs += __popc(eqm);
+  } else {
+    for (int j = tid; j < (int)n; j += kSelThreads) {
+      const uint32_t key = ck[src_of(j)];
+      kmin = min(kmin, key);
+      kmax = max(kmax, key);
     }
-    written += blk_sel;
-    eq_seen += blk_eq;
-    __syncthreads();
   }
-  for (int j = (int)want + tid; j < budget; j += kThreads) out_idx[j] = -1;
+  block_min_max<kSelThreads>(kmin, kmax, s_wsum);  // (its barrier also publishes the candidates)
+  auto key_at = [&](int j) -> uint32_t { return staged ? s_ckey[j] : ck[src_of(j)]; };
+  auto pos_at = [&](int j) -> int32_t { return staged ? s_cpos[j] : cp[src_of(j)]; };
+  int64_t thr;
+  uint32_t take;
+  select_threshold<kSelThreads>(key_at, (int)n, want, kmin, kmax, s_hist, s_wsum, s_info, thr,
+                                take);
+  // ordered emission: the selected candidates are the keys > thr and the first `take` keys == thr
+  // in position order, written in candidate (= position) order. Each thread owns a contiguous run
+  // of candidates; one block scan of (count > thr, count == thr) gives every candidate's slot:
+  // (keys > thr before it) + min(keys == thr before it, take).
+  const int per = ((int)n + kSelThreads - 1) / kSelThreads;
+  const int j0 = min((int)n, tid * per), j1 = min((int)n, j0 + per);
+  uint32_t n_gt = 0, n_eq = 0;
+  for (int j = j0; j < j1; ++j) {
+    const int64_t key = (int64_t)key_at(j);
+    n_gt += key > thr;
+    n_eq += key == thr;
+  }
+  uint64_t total;
+  const uint64_t before =
+      block_excl_scan64<kSelThreads>(((uint64_t)n_eq << 32) | n_gt, total, s_red64);
+  uint32_t gt_b = (uint32_t)before, eq_b = (uint32_t)(before >> 32);
+  for (int j = j0; j < j1; ++j) {
+    const int64_t key = (int64_t)key_at(j);
+    if (key > thr) {
+      const uint32_t at = gt_b + min(eq_b, take);
+      if (at < (uint32_t)budget) out_idx[at] = pos_at(j);
+      ++gt_b;
+    } else if (key == thr) {
+      if (eq_b < take) {
+        const uint32_t at = gt_b + eq_b;
+        if (at < (uint32_t)budget) out_idx[at] = pos_at(j);
+      }
+      ++eq_b;
+    }
+  }
+  const uint32_t written = (uint32_t)total + min((uint32_t)(total >> 32), take);
+  for (int j = (int)want + tid; j < budget; j += kSelThreads) out_idx[j] = -1;
   if (tid == 0) {
     if (written != want) raise_flag(8u);
     s.count[pair] = (int)want;
@@ -758,11 +1028,12 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs s) {
   pdl_trigger();
 }
 
-template <typename Kern, typename Arg>
-cudaError_t launch_k(Kern kern, dim3 grid, size_t smem, bool pdl, cudaStream_t s, const Arg& arg) {
+template <typename Kern, typename... Args>
+cudaError_t launch_k(Kern kern, dim3 grid, int threads, size_t smem, bool pdl, cudaStream_t s,
+                     const Args&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -770,7 +1041,7 @@ cudaError_t launch_k(Kern kern, dim3 grid, size_t smem, bool pdl, cudaStream_t s
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, arg);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -779,18 +1050,26 @@ template <int D, int R>
 cudaError_t launch_t(const ScorePlan& plan, int pairs, const PrepArgs& pa, const ScanArgs& sa,
                      const SelectArgs& sel, bool store, bool pdl, cudaStream_t s) {
   cudaError_t e;
-  if (store) e = launch_k(prep_kernel<D, R, true>, dim3(pairs), 0, pdl, s, pa);
-  else e = launch_k(prep_kernel<D, R, false>, dim3(pairs), 0, pdl, s, pa);
+  const size_t prep_smem = sizeof(PrepSmem<D, R>);
+  if (store) {
+    e = configure_kernel((const void*)prep_kernel<D, R, true>, (int)prep_smem, false);
+    if (e == cudaSuccess)
+      e = launch_k(prep_kernel<D, R, true>, dim3(pairs), kThreads, prep_smem, pdl, s, pa);
+  } else {
+    e = configure_kernel((const void*)prep_kernel<D, R, false>, (int)prep_smem, false);
+    if (e == cudaSuccess)
+      e = launch_k(prep_kernel<D, R, false>, dim3(pairs), kThreads, prep_smem, pdl, s, pa);
+  }
   if (e != cudaSuccess) return e;
   const size_t scan_smem = (size_t)(plan.chunk / (1 << sa.page_shift) + 1) * 4;
   e = configure_kernel((const void*)scan_kernel<D, R>, (int)scan_smem, false);
   if (e != cudaSuccess) return e;
-  e = launch_k(scan_kernel<D, R>, dim3(plan.n_chunks, pairs), scan_smem, true, s, sa);
+  e = launch_k(scan_kernel<D, R>, dim3(plan.n_chunks, pairs), kThreads, scan_smem, true, s, sa);
   if (e != cudaSuccess) return e;
   const size_t sel_smem = (size_t)kSelectCap * 8;
   e = configure_kernel((const void*)select_kernel<D, R>, (int)sel_smem, false);
   if (e != cudaSuccess) return e;
-  return launch_k(select_kernel<D, R>, dim3(pairs), sel_smem, true, s, sel);
+  return launch_k(select_kernel<D, R>, dim3(pairs), kSelThreads, sel_smem, true, s, sel);
 }
 
 }  // namespace score_detail
@@ -804,12 +1083,12 @@ ScorePlan plan_score(int pairs, int max_seq_len, int page_size) {
   while (chunk > 2048 && (long long)pairs * ((max_seq_len + chunk - 1) / chunk) < 6LL * num_sms())
     chunk >>= 1;
   while (chunk % page_size) chunk <<= 1;
-  while ((long long)((max_seq_len + chunk - 1) / chunk) * kWarps > kMaxRegions) chunk <<= 1;
+  while ((long long)((max_seq_len + chunk - 1) / chunk) * kRegionsPerChunk > kMaxRegions) chunk <<= 1;
   p.chunk = chunk;
   p.n_chunks = (max_seq_len + chunk - 1) / chunk;
   if (p.n_chunks < 1) p.n_chunks = 1;
   const size_t prep = (size_t)pairs * kPrepBytes;
-  const size_t counts = ((size_t)pairs * p.n_chunks * kWarps * 4 + 255) / 256 * 256;
+  const size_t counts = ((size_t)pairs * p.n_chunks * kRegionsPerChunk * 4 + 255) / 256 * 256;
   const size_t entries = (size_t)pairs * p.n_chunks * chunk;
   p.ws_bytes = prep + counts + entries * 8;
   return p;
@@ -829,7 +1108,7 @@ cudaError_t launch_score_topk(const uint16_t* q, const float* basis, const uint8
   while ((1 << shift) < page_size) ++shift;
   uint8_t* w = static_cast<uint8_t*>(ws);
   const Prep prep{w};
-  const size_t counts = ((size_t)pairs * plan.n_chunks * kWarps * 4 + 255) / 256 * 256;
+  const size_t counts = ((size_t)pairs * plan.n_chunks * kRegionsPerChunk * 4 + 255) / 256 * 256;
   const size_t entries = (size_t)pairs * plan.n_chunks * plan.chunk;
   Cands cands;
   cands.cnt = reinterpret_cast<uint32_t*>(w + (size_t)pairs * kPrepBytes);
