@@ -156,14 +156,15 @@ JSSA_API int jssa_store(const jssa_bf16* k, int64_t k_stride_t, const int64_t* s
  * heads of h), s_t = sum_j dec(c_tj) p_j for every t < seq_len (fp32), and the index set of the
  * min(budget, seq_len) largest s_t, ties to the lower position, written ascending.
  * JSSA summary, eq. (1) and section 3.1 steps 1-2; JSSA README, section 4 (jssa_budget).
- * Three kernels: a per-(sequence, KV head) prep (query projection, its FP8 digits and a
- * candidate threshold from a sample of the scores), a streaming scan on the tensor cores that
- * keeps only keys at or above the threshold, and an exact per-(sequence, KV head) selection
- * (which rescans when the threshold let through fewer than min(budget, seq_len) keys).
+ * Three kernels: a per-(sequence, KV head) prep (query projection, p split into two f16 digit
+ * vectors with power-of-two weights, and a candidate threshold from a sample of the scores), a
+ * streaming scan (codes widened exactly to f16 and multiplied on the tensor cores, fp32
+ * accumulation) that keeps only keys at or above the threshold, and an exact per-(sequence,
+ * KV head) selection (which rescans when the threshold let through fewer than
+ * min(budget, seq_len) keys).
  * q: bf16 [batch, h_q, d] contiguous. ws: >= jssa_workspace_size(JSSA_FN_SCORE_TOPK).
- * Limits (JSSA_ERR_UNSUPPORTED beyond them): max_pages * page_size <= 4194304 positions,
- * batch * h_kv <= 65535 and page_size * r >= 128 (the scan copies whole page rows of at least
- * 128 bytes into shared memory).
+ * Limits (JSSA_ERR_UNSUPPORTED beyond them): max_pages * page_size <= 4194304 positions and
+ * batch * h_kv <= 65535.
  */
 JSSA_API int jssa_score_topk(const jssa_bf16* q, const float* basis, const uint8_t* score_cache,
                     const int32_t* block_table, int max_pages, const int32_t* seq_lens, int batch,

@@ -129,6 +129,20 @@ def test_score_topk_rank64_and_page32():
             check_selection(gi[b, h], gc[b, h], ref_idx[b, h], ref_count[b, h], s[(b, h)], budget)
 
 
+@pytest.mark.parametrize("page_size,lens,budget", [(4, [3000, 777], 200), (8, [20000], 512)])
+def test_score_topk_small_pages(page_size, lens, budget):
+    # pages shorter than a 16-token scan tile (rows of one tile come from several pages)
+    case = Case(lens, page_size=page_size, seed=1045 + page_size, calib=2048)
+    J = jssa()
+    idx, count = J.score_topk(case.gpu(case.q), case.gpu_np(case.m32), case.gpu_np(case.codes),
+                              case.gpu(case.block_table), case.gpu(case.seq_lens_t), budget)
+    ref_idx, ref_count, s = _select_oracle(case, budget)
+    gi, gc = idx.cpu().numpy(), count.cpu().numpy()
+    for b in range(len(lens)):
+        for h in range(case.h_kv):
+            check_selection(gi[b, h], gc[b, h], ref_idx[b, h], ref_count[b, h], s[(b, h)], budget)
+
+
 def test_score_topk_exact_ties_go_to_lower_position():
     # every token of a sequence gets the same code row -> all scores tie; the set must be the
     # lowest positions 0..B-1 on both sides
@@ -182,15 +196,17 @@ def _mix32(x):
     return x
 
 
-def _sampled_positions(pair, L, n=2048):
-    # the candidate-threshold sample of the score kernels: one position per stratum of L // n
-    # tokens, at an offset drawn from a 32-bit mix of (stratum, pair) scaled to the stratum by a
-    # high multiply, never the last position
-    stratum = L // n
+def _sampled_positions(pair, L, groups=512, run=4):
+    # the candidate-threshold sample of the score kernels: one run of 4 consecutive positions per
+    # stratum of L // 512 tokens, starting at a 4-aligned offset drawn from a 32-bit mix of
+    # (stratum, pair) scaled to the stratum by a high multiply
+    stratum = L // groups
     out = []
-    for i in range(n):
-        h = _mix32(((i * 0x9E3779B9) & 0xFFFFFFFF) ^ ((pair * 0x85EBCA6B + 1) & 0xFFFFFFFF))
-        out.append(min(i * stratum + ((h * stratum) >> 32), L - 2))
+    for g in range(groups):
+        h = _mix32(((g * 0x9E3779B9) & 0xFFFFFFFF) ^ ((pair * 0x85EBCA6B + 1) & 0xFFFFFFFF))
+        first = (g * stratum + run - 1) // run
+        p0 = run * (first + ((h * (stratum // run - 1)) >> 32))
+        out.extend(range(p0, p0 + run))
     return np.asarray(out)
 
 

@@ -223,7 +223,6 @@ static int check_score_args(const jssa_bf16* q, const float* basis, const uint8_
   if ((st = check_paging(max_pages, num_pages, page_size))) return st;
   if ((int64_t)max_pages * page_size > kMaxContext) return JSSA_ERR_UNSUPPORTED;
   if ((int64_t)batch * h_kv > 65535) return JSSA_ERR_UNSUPPORTED;  // one grid row per pair
-  if (page_size * r < 128) return JSSA_ERR_UNSUPPORTED;  // tensor-copy tiles of >= 128 bytes
   if (batch == 0) return JSSA_OK;
   if (!q || !basis || !score_cache || !block_table || !seq_lens || !idx || !count)
     return JSSA_ERR_NULL;

@@ -371,29 +371,34 @@ template <int R>
 struct ScanBuf {
   static constexpr int kUnroll = kUnrollBytes / (R / 4);  // tiles per batch (even)
   uint32_t ra[kUnroll][R / 16], rb[kUnroll][R / 16];
+  uint32_t ok;  // bit u: tile u is inside the run and the chunk and its page is usable
 };
 
 // Rows of tiles [t0, t0 + kUnroll) (rows g and g+8 of each tile for lane (g, t)). The loads are
 // unconditional: a tile past t_end or the chunk's valid tokens, or on an unusable page, reads
 // page 0 instead (always allocated) and its tokens are never candidates (see scan_emit).
-template <int R>
+// BIG: pages of at least 16 tokens, so a tile lies inside one page.
+template <int R, bool BIG>
 __device__ __forceinline__ void scan_load(ScanBuf<R>& buf, const ChunkGeom& cg,
                                           const int32_t* s_page, int t0, int t_end, int lane) {
   constexpr int LB = R / 4;
   const int g = lane >> 2, t = lane & 3;
   const int pmask = (1 << cg.page_shift) - 1;
-  const int lane_off = g * R + t * LB;
-  if (cg.page_shift >= 4) {  // a 16-token tile lies inside one page
+  if (BIG) {
+    const int lane_off = g * R + t * LB;
+    buf.ok = 0u;
 #pragma unroll
     for (int u = 0; u < ScanBuf<R>::kUnroll; ++u) {
       const int tok0 = (t0 + u) * 16;
-      const int pg = t0 + u < t_end && tok0 < cg.n_local ? s_page[tok0 >> cg.page_shift] : 0;
+      const int pg = t0 + u < t_end && tok0 < cg.n_local ? s_page[tok0 >> cg.page_shift] : -1;
+      buf.ok |= (uint32_t)(pg >= 0) << u;
       const uint8_t* row = cg.head_base + (size_t)(uint32_t)max(pg, 0) * cg.page_bytes +
                            ((tok0 & pmask) * R + lane_off);
       load_row<R>(buf.ra[u], row);
       load_row<R>(buf.rb[u], row + 8 * R);
     }
   } else {
+    buf.ok = ~0u;  // token validity is checked per token at emission
 #pragma unroll
     for (int u = 0; u < ScanBuf<R>::kUnroll; ++u) {
       const bool live = t0 + u < t_end;
@@ -432,12 +437,20 @@ __device__ __forceinline__ float pair_scores(const uint32_t* ra0, const uint32_t
   return (tile1 ? x1 : x0) * df.sc0 + (tile1 ? y1 : y0) * df.sc1;
 }
 
+// The smallest float whose key is >= thr (keys of non-NaN floats are >= thr exactly when the
+// float is >= it); -inf when every key qualifies.
+__device__ __forceinline__ float key_floor(uint32_t thr) {
+  if (thr <= 0x007FFFFFu) return -INFINITY;  // at or below the key of -inf
+  const uint32_t u = (thr & 0x80000000u) ? (thr & 0x7FFFFFFFu) : ~thr;
+  return __uint_as_float(u);
+}
+
 // Keys >= thr of the tiles [t0, t0 + kUnroll) appended in position order to this warp's region.
-template <int R>
+template <int R, bool BIG>
 __device__ __forceinline__ void scan_emit(const ScanBuf<R>& buf, const DigitFrags<R>& df,
                                           const ChunkGeom& cg, const int32_t* s_page, int t0,
-                                          int t_end, uint32_t thr,
-                                          uint32_t* rkey, int32_t* rpos, uint32_t& run, int lane) {
+                                          int t_end, float thr_f, uint32_t* rkey, int32_t* rpos,
+                                          uint32_t& run, int lane) {
   const int g = lane >> 2, t = lane & 3;
   const int tok_in_pair = 16 * (t >> 1) + 8 * (t & 1) + g;
   // lanes holding earlier tokens of the pair: every lane of a lower t, and lower g for this t
@@ -448,8 +461,13 @@ __device__ __forceinline__ void scan_emit(const ScanBuf<R>& buf, const DigitFrag
   for (int u = 0; u < ScanBuf<R>::kUnroll; u += 2) {
     const float f = pair_scores<R>(buf.ra[u], buf.rb[u], buf.ra[u + 1], buf.rb[u + 1], df, t);
     const int tok = (t0 + u) * 16 + tok_in_pair;
-    const bool c = t0 + u < t_end && tok < cg.n_local && score_key(f) >= thr &&
-                   (tok_in_pair < 16 || t0 + u + 1 < t_end) && s_page[tok >> cg.page_shift] >= 0;
+    bool c = f >= thr_f && tok < cg.n_local;
+    if (BIG) {
+      c = c && ((buf.ok >> (u + (t >> 1))) & 1u);
+    } else {
+      c = c && t0 + u < t_end && (tok_in_pair < 16 || t0 + u + 1 < t_end) &&
+          s_page[tok >> cg.page_shift] >= 0;
+    }
     const unsigned m = __ballot_sync(0xffffffffu, c);
     if (m) {
       if (c) {
@@ -463,22 +481,22 @@ __device__ __forceinline__ void scan_emit(const ScanBuf<R>& buf, const DigitFrag
 }
 
 // One warp's contiguous run of tiles [t_begin, t_end), register double-buffered.
-template <int R>
+template <int R, bool BIG>
 __device__ __forceinline__ uint32_t scan_warp(const ChunkGeom& cg, const int32_t* s_page,
-                                              const DigitFrags<R>& df, uint32_t thr, int t_begin,
+                                              const DigitFrags<R>& df, float thr_f, int t_begin,
                                               int t_end, uint32_t* rkey, int32_t* rpos, int lane) {
   constexpr int kU = ScanBuf<R>::kUnroll;
   uint32_t run = 0;
   ScanBuf<R> a, b;
   int t0 = t_begin;
-  if (t0 < t_end) scan_load<R>(a, cg, s_page, t0, t_end, lane);
+  if (t0 < t_end) scan_load<R, BIG>(a, cg, s_page, t0, t_end, lane);
   while (t0 < t_end) {
-    if (t0 + kU < t_end) scan_load<R>(b, cg, s_page, t0 + kU, t_end, lane);
-    scan_emit<R>(a, df, cg, s_page, t0, t_end, thr, rkey, rpos, run, lane);
+    if (t0 + kU < t_end) scan_load<R, BIG>(b, cg, s_page, t0 + kU, t_end, lane);
+    scan_emit<R, BIG>(a, df, cg, s_page, t0, t_end, thr_f, rkey, rpos, run, lane);
     t0 += kU;
     if (t0 >= t_end) break;
-    if (t0 + kU < t_end) scan_load<R>(a, cg, s_page, t0 + kU, t_end, lane);
-    scan_emit<R>(b, df, cg, s_page, t0, t_end, thr, rkey, rpos, run, lane);
+    if (t0 + kU < t_end) scan_load<R, BIG>(a, cg, s_page, t0 + kU, t_end, lane);
+    scan_emit<R, BIG>(b, df, cg, s_page, t0, t_end, thr_f, rkey, rpos, run, lane);
     t0 += kU;
   }
   return run;
@@ -525,8 +543,13 @@ __device__ void scan_chunk(const ScanArgs& a, int pair, int c, int L, uint32_t t
   const int n_tiles = (cg.n_local + 15) >> 4;
   const int tpw = seg / 16;
   const int t_begin = min(n_tiles, warp * tpw), t_end = min(n_tiles, t_begin + tpw);
-  const uint32_t n = scan_warp<R>(cg, s_page, df, thr, t_begin, t_end, a.cands.key + reg * seg,
-                                  a.cands.pos + reg * seg, lane);
+  const float thr_f = key_floor(thr);
+  const uint32_t n =
+      cg.page_shift >= 4
+          ? scan_warp<R, true>(cg, s_page, df, thr_f, t_begin, t_end, a.cands.key + reg * seg,
+                               a.cands.pos + reg * seg, lane)
+          : scan_warp<R, false>(cg, s_page, df, thr_f, t_begin, t_end, a.cands.key + reg * seg,
+                                a.cands.pos + reg * seg, lane);
   if (lane == 0) a.cands.cnt[reg] = n;
 }
 
@@ -578,13 +601,17 @@ struct PrepArgs {
   StoreNew store;  // decode: the new token (position seq_len - 1)
 };
 
-// Sampled position i of (pair, L): one per stratum of L / kSample tokens at an offset drawn from
-// a 32-bit mix of (i, pair) (scaled to the stratum by a high multiply), never the last position
-// (the token a decode step stores right now).
-__device__ __forceinline__ int sample_pos(int i, int pair, int L) {
-  const int stratum = L / kSample;
-  const uint32_t hsh = mix32((uint32_t)i * 0x9E3779B9u ^ ((uint32_t)pair * 0x85EBCA6Bu + 1u));
-  return min(i * stratum + (int)__umulhi(hsh, (uint32_t)stratum), L - 2);
+// The sample: kSampleGroups strata of L / kSampleGroups tokens, in each a run of kGroup
+// consecutive positions (one 128-byte line of codes at r = 32) starting at a kGroup-aligned
+// offset drawn from a 32-bit mix of (stratum, pair), scaled to the stratum by a high multiply;
+// never the last position (the token a decode step stores right now).
+constexpr int kGroup = 4;
+constexpr int kSampleGroups = kSample / kGroup;
+__device__ __forceinline__ int sample_group_start(int grp, int pair, int L) {
+  const int stratum = L / kSampleGroups;  // >= 32 whenever the sample is drawn
+  const uint32_t hsh = mix32((uint32_t)grp * 0x9E3779B9u ^ ((uint32_t)pair * 0x85EBCA6Bu + 1u));
+  const int first = (grp * stratum + kGroup - 1) / kGroup;  // first aligned slot of the stratum
+  return kGroup * (first + (int)__umulhi(hsh, (uint32_t)(stratum / kGroup - 1)));
 }
 
 constexpr int kQGroups = kThreads / 16;  // query rows loaded per pass (16 threads x 8 dims a row)
@@ -655,28 +682,36 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(PrepArgs a) {
     if (k >= kSample / 2) k = 0;
   }
   if (k) {
-    // the sampled code rows go straight to shared memory (asynchronous 16-byte copies issued as
-    // soon as each page number arrives; a row on an unusable page is zero-filled)
-    constexpr int kPer = kSample / kThreads;
-    int pos[kPer], pg[kPer];
+    // the sampled code rows go straight to shared memory: each thread looks up the pages of its
+    // groups and copies their rows with asynchronous 16-byte copies (a group is one contiguous
+    // run of kGroup rows in one page when pages hold at least kGroup tokens; otherwise each
+    // position is looked up); a row on an unusable page is zero-filled and marked invalid
+    constexpr int kPer = kSampleGroups / kThreads;
+    constexpr int kPieces = R / 16;
+    int p0[kPer], pg0[kPer];
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
-      pos[u] = sample_pos(tid + u * kThreads, pair, L);
-      pg[u] = bt[pos[u] >> a.page_shift];
+      p0[u] = sample_group_start(tid + u * kThreads, pair, L);
+      pg0[u] = bt[p0[u] >> a.page_shift];
     }
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
-      const int i = tid + u * kThreads;
-      const bool ok = pg[u] >= 0 && (int64_t)pg[u] < a.num_pages;
-      sm.valid[i] = ok;
-      const uint8_t* src = a.score_cache +
-          ((((int64_t)(ok ? pg[u] : 0) * a.h_kv + h) << a.page_shift) + (pos[u] & (page_size - 1))) * R;
+      const int grp = tid + u * kThreads;
 #pragma unroll
-      for (int c = 0; c < R / 16; ++c)
-        cp_async16(smem_u32(sm.rows + i * R + c * 16), src + c * 16, ok ? 16 : 0);
+      for (int j = 0; j < kGroup; ++j) {
+        const int pos = p0[u] + j, i = grp * kGroup + j;
+        int32_t pg = page_size >= kGroup ? pg0[u] : bt[pos >> a.page_shift];
+        if (pg < 0 || (int64_t)pg >= a.num_pages) pg = -1;
+        sm.valid[i] = pg >= 0;
+        const uint8_t* src = a.score_cache +
+            ((((int64_t)max(pg, 0) * a.h_kv + h) << a.page_shift) + (pos & (page_size - 1))) * R;
+#pragma unroll
+        for (int c = 0; c < kPieces; ++c)
+          cp_async16(smem_u32(sm.rows + i * R + c * 16), src + c * 16, pg >= 0 ? 16 : 0);
+      }
     }
-    cp_async_commit();
   }
+  cp_async_commit();  // (group: the sample rows; M_h is the group before)
   const bool store = STORE && L > 0;
   int32_t st_page = -1;
   if (store) {  // decode: copy the new token's K and V rows into the cache
@@ -701,8 +736,7 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(PrepArgs a) {
       }
     }
   }
-  if (k) cp_async_wait<1>();  // M_h landed; the sample rows may still be in flight
-  else cp_async_wait<0>();
+  cp_async_wait<1>();  // M_h landed; the sample rows may still be in flight
   __syncthreads();
   for (int i = tid; i < D; i += kThreads) {
     float acc = 0.f;
