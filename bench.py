@@ -54,6 +54,45 @@ def dist_env():
     return rank, world, local
 
 
+class RankGroup:
+    """One process per GPU (torchrun environment): barriers and the max over ranks of a time.
+    Every rank takes the same collective steps in the same order; with one rank nothing is
+    initialised. backend: "nccl" on GPUs, "gloo" for the CPU tests of this plumbing."""
+
+    def __init__(self, backend="nccl", device=None, timeout_s=300):
+        import torch.distributed as dist
+        from datetime import timedelta
+        self.rank, self.world, self.local = dist_env()
+        self.device = device
+        self.dist = dist
+        if self.world > 1:
+            kw = {"device_id": device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=timedelta(seconds=timeout_s), **kw)
+
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
+
+    def max_over_ranks(self, x):
+        if self.world == 1:
+            return x
+        import torch
+        t = torch.tensor([float(x)], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.world > 1:
+            self.dist.barrier()
+            self.dist.destroy_process_group()
+
+
+def whole_job_rate(world, steps_per_rank, t_max_s):
+    """Weak scaling: every rank runs steps_per_rank steps on its own batch; the job's rate is the
+    steps all ranks processed over the slowest rank's time."""
+    return world * steps_per_rank / t_max_s
+
+
 # ------------------------------------------------------------------------------------------------
 # clocks
 # ------------------------------------------------------------------------------------------------
@@ -207,6 +246,22 @@ def algorithmic_bytes(w, dense=False):
         return w.batch * (w.h_kv * w.seq_len * 2 * w.d * 2 + 4 * pages)
     return w.batch * (w.h_kv * w.seq_len * w.rank + w.h_kv * min(w.budget, w.seq_len) * 2 * w.d * 2
                       + 4 * pages)
+
+
+def recorded_traffic(kernel, w):
+    """DRAM bytes per launch from the committed ncu capture of this workload, or None when the
+    workload differs or a kernel source changed since the counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic_llama128k_b16.json")
+    if not (w.batch == 16 and w.seq_len == 131072 and w.budget == 2048 and os.path.exists(path)):
+        return None
+    rec = json.load(open(path))
+    csrc = os.path.join(ROOT, "token_level_sparse_fp8_b200", "csrc")
+    for name, digest in rec["sources_sha256_16"].items():
+        with open(os.path.join(csrc, name), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest()[:16] != digest:
+                return None
+    return rec["bytes_per_launch"].get(kernel)
 
 
 def score_bytes(w):
@@ -369,27 +424,14 @@ def run_reference(args):
 def run_jssa(args):
     import numpy as np
     import torch
-    import torch.distributed as dist
     import token_level_sparse_fp8_b200 as J
 
     rank, world, local = dist_env()
     assert torch.cuda.is_available(), "bench needs a CUDA device"
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    group = RankGroup("nccl", dev)
+    barrier, max_over_ranks = group.barrier, group.max_over_ranks
 
     w = workload(args, rank)
     J._lib.load()
@@ -475,15 +517,13 @@ def run_jssa(args):
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline(state, w, args.cpu_seconds)
 
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    group.close()
     if rank != 0:
         return
 
     peak, peak_kind = peaks()
     ms_step = t_step / n_steps * 1e3
-    steps_per_s = world * n_steps / t_step
+    steps_per_s = whole_job_rate(world, n_steps, t_step)
     bytes_step = algorithmic_bytes(w)
     score_launch_s = t_score
     achieved = score_bytes(w) / score_launch_s / 1e9
@@ -514,13 +554,14 @@ def run_jssa(args):
                           "unit": "GB/s", "frac": bytes_step / (ms_step / 1e3) / 1e9 / peak,
                           "traffic": None, "bytes_per_step": bytes_step, "peak_kind": peak_kind},
         "roofline": {"bound": "hbm", "kernel": "score_topk", "achieved": achieved, "peak": peak,
-                     "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": recorded_traffic("score_topk", w),
                      "bytes_per_launch": score_bytes(w), "ms_per_launch": score_launch_s * 1e3,
                      "peak_kind": peak_kind},
         "kernels_ms": {"score_topk": score_launch_s * 1e3, "indexed_attend": t_attend * 1e3,
                        "attend_gbs": attend_bytes(w) / t_attend / 1e9},
         "clocks": clocks,
-        "e2e": {"value": world * args.steps / t_e2e, "unit": "steps/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": whole_job_rate(world, args.steps, t_e2e), "unit": "steps/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * n_steps,
         "timing": "CUDA events around replays of a CUDA graph holding 8 consecutive steps",

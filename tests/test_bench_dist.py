@@ -1,0 +1,63 @@
+"""The multi-rank plumbing of bench.py (one process per GPU under torchrun), exercised on CPU with
+the gloo backend and two ranks: the barrier, the max over ranks of a time, distinct per-rank
+workload seeds, the weak-scaling aggregate, and a clean shutdown."""
+
+import multiprocessing as mp
+import os
+import socket
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    os.environ.update({"RANK": str(rank), "WORLD_SIZE": str(world), "LOCAL_RANK": str(rank),
+                       "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    sys.path.insert(0, ROOT)
+    import bench
+
+    class Args:
+        batch, budget, seq_len = 16, 2048, 131072
+
+    group = bench.RankGroup("gloo", timeout_s=60)
+    group.barrier()
+    t_max = group.max_over_ranks(1.5 + rank)  # ranks report different times
+    seed = bench.workload(Args, group.rank).seed
+    rate = bench.whole_job_rate(group.world, 800, t_max)
+    group.close()
+    out.put((rank, group.world, t_max, seed, rate))
+
+
+def test_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(out.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (r0, w0, t0, s0, v0), (r1, w1, t1, s1, v1) = res
+    assert (r0, r1) == (0, 1) and w0 == w1 == 2
+    assert t0 == t1 == 2.5              # max over ranks, seen by every rank
+    assert s0 != s1                     # each rank draws its own sequences
+    assert v0 == v1 == 2 * 800 / 2.5    # steps of all ranks over the slowest rank's time
+
+
+def test_single_rank_has_no_process_group(monkeypatch):
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    sys.path.insert(0, ROOT)
+    import bench
+    g = bench.RankGroup("gloo")
+    assert g.world == 1 and g.max_over_ranks(3.0) == 3.0
+    g.barrier()
+    g.close()
