@@ -6,16 +6,16 @@
 //   * Row addresses: the CTA first turns each of its positions into a 64-bit element offset
 //     (page-table lookup, bounds checked) kept in shared memory.
 //   * Each of the 4 warps walks its own 16-token tiles. A tile's K and V rows (256 B each at
-//     d = 128) are loaded with 16-byte non-allocating loads straight from their paged locations
-//     into registers -- no staging buffer in global or shared memory -- and the next tile's loads
-//     are in flight while the current tile is computed.
+//     d = 128) are copied straight from their paged locations into the warp's ring of kStages
+//     shared-memory stages with 16-byte cp.async (rows past the slice or on unusable pages are
+//     zero-filled) -- no staging buffer in global memory -- so kStages - 1 tiles are in flight
+//     while one is computed. Inside a stage a row's 16-byte chunk c sits at chunk c ^ (row & 7),
+//     which makes the ldmatrix reads below conflict-free.
 //   * Tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate) with the 16 tokens as the M
-//     rows and the G <= 8 query heads of the KV head as the N columns: S^T = K Q^T, then
-//     O^T += V^T P^T. The head dimension is visited in a fixed permuted order (the same for q and
-//     k, and undone when O is written) so that every lane's fragment elements are contiguous in
-//     the row: a lane reads 64 B of each of its two K rows and 32 B of each of its four V rows.
-//     P^T reaches the B-operand layout with movmatrix, split into a bf16 high and low part so the
-//     probabilities keep ~16 significant bits.
+//     rows and the G <= 8 query heads of the KV head as the N columns: S^T = K Q^T (K fragments
+//     by ldmatrix), then O^T += V^T P^T (V^T fragments by ldmatrix.trans). P^T reaches the
+//     B-operand layout with movmatrix, split into a bf16 high and low part so the probabilities
+//     keep ~16 significant bits.
 //   * Online softmax in the log2 domain; warps merge in shared memory; CTAs of one (b, h) merge
 //     through fp32 partials (m, l, o) in the workspace, the last CTA to take the ticket combines
 //     them, writes the bf16 output and resets the ticket.
@@ -31,12 +31,10 @@ constexpr int kWarps = kAttendWarps;
 constexpr int kThreads = kWarps * 32;
 constexpr int kTile = kAttendTile;
 constexpr int kMaxChunk = 1024;  // positions per CTA (row offsets kept in shared memory)
-
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t r;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
-  return r;
-}
+constexpr int kStages = 3;       // tiles per warp ring (kStages - 1 in flight)
+constexpr int kTileBytes = kTile * 128 * 2;   // K (or V) rows of one tile at d = 128
+constexpr int kStageBytes = 2 * kTileBytes;   // K then V
+constexpr int kRingBytes = kWarps * kStages * kStageBytes;  // dynamic shared memory per CTA
 
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
   uint32_t r;
@@ -44,52 +42,15 @@ __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
   return r;
 }
 
-template <int D>
-struct TileRegs {
-  uint4 k[2][D / 32];   // rows g, g+8 of the tile: bytes [t * D/2, +D/2)
-  uint4 v[4][D / 64];   // rows 2t, 2t+1, 8+2t, 9+2t: bytes [g * D/4, +D/4)
-};
-
-template <int D>
-__device__ __forceinline__ void load_tile(TileRegs<D>& tr, const uint16_t* __restrict__ kc,
-                                          const uint16_t* __restrict__ vc, const int64_t* s_off,
-                                          int tile, int n_mine, int lane) {
-  const int g = lane >> 2, t = lane & 3;
-  const int j0 = tile * kTile;
-  const int krow[2] = {g, g + 8};
-  const int vrow[4] = {2 * t, 2 * t + 1, 8 + 2 * t, 9 + 2 * t};
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int j = j0 + krow[i];
-    const int64_t off = j < n_mine ? s_off[j] : -1;
-    const uint16_t* src = kc + (off >= 0 ? off : 0) + t * (D / 4);
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c)
-      tr.k[i][c] = off >= 0 ? ld_stream_v4(src + c * 8) : make_uint4(0u, 0u, 0u, 0u);
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int j = j0 + vrow[i];
-    const int64_t off = j < n_mine ? s_off[j] : -1;
-    const uint16_t* src = vc + (off >= 0 ? off : 0) + g * (D / 8);
-#pragma unroll
-    for (int c = 0; c < D / 64; ++c)
-      tr.v[i][c] = off >= 0 ? ld_stream_v4(src + c * 8) : make_uint4(0u, 0u, 0u, 0u);
-  }
-}
-
-__device__ __forceinline__ uint32_t word(const uint4& u, int i) {
-  return i == 0 ? u.x : (i == 1 ? u.y : (i == 2 ? u.z : u.w));
-}
-
 template <int D, bool INDEXED>
 __global__ void __launch_bounds__(kThreads, 2) attend_kernel(AttendArgs a, int chunk, int splits) {
   static_assert(D == 128, "head dim");
   constexpr int KB = D / 16;  // k-blocks of S^T, m-tiles of O^T
+  extern __shared__ __align__(128) uint8_t att_ring[];  // warp rings; the warp merge reuses it
   __shared__ int64_t s_off[kMaxChunk];
   __shared__ float s_m[kWarps][kAttendMaxG], s_l[kWarps][kAttendMaxG];
-  __shared__ float s_o[kWarps][kAttendMaxG][D];
   __shared__ int s_last;
+  float(*s_o)[kAttendMaxG][D] = reinterpret_cast<float(*)[kAttendMaxG][D]>(att_ring);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
@@ -99,18 +60,15 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(AttendArgs a, int c
   const int max_len = a.max_pages * a.page_size;
 
   // Q^T fragments (B operand of S^T = K Q^T): column n = head g of this KV head (zero for g >= G);
-  // k-slot 16kb+2t+e <-> physical dim D/4*t + 4kb + e, 16kb+8+2t+e <-> D/4*t + 4kb + 2 + e
+  // k-block kb: dims 16kb + 2t, +1 (b0) and 16kb + 8 + 2t, +1 (b1)
   uint32_t qb0[KB], qb1[KB];
   {
-    const uint4* qrow = reinterpret_cast<const uint4*>(
-        a.q + ((int64_t)b * a.h_q + (int64_t)h * G + (g < G ? g : 0)) * D + t * (D / 4));
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+        a.q + ((int64_t)b * a.h_q + (int64_t)h * G + (g < G ? g : 0)) * D);
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      const uint4 v = g < G ? qrow[c] : make_uint4(0u, 0u, 0u, 0u);
-      qb0[2 * c] = v.x;
-      qb1[2 * c] = v.y;
-      qb0[2 * c + 1] = v.z;
-      qb1[2 * c + 1] = v.w;
+    for (int kb = 0; kb < KB; ++kb) {
+      qb0[kb] = g < G ? qrow[8 * kb + t] : 0u;
+      qb1[kb] = g < G ? qrow[8 * kb + 4 + t] : 0u;
     }
   }
 
@@ -131,46 +89,88 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(AttendArgs a, int c
   const int j_begin = split * chunk;
   const int n_mine = max(0, min(chunk, n_total - j_begin));
 
-  // ---- row offsets of this CTA's positions ---------------------------------------------------
-  const int32_t* bt = a.block_table + (int64_t)b * a.max_pages;
-  for (int j = tid; j < n_mine; j += kThreads) {
-    const int pos = INDEXED ? a.idx[(int64_t)pair * a.budget + j_begin + j] : lo + j_begin + j;
-    int64_t off = -1;
-    if (pos < 0 || pos >= max_len) {
-      raise_flag(2u);
-    } else {
-      const int32_t pg = bt[pos / a.page_size];
-      if (pg < 0 || (int64_t)pg >= a.num_pages) raise_flag(1u);
-      else
-        off = (int64_t)pg * a.page_stride + (int64_t)(pos % a.page_size) * a.slot_stride +
-              (int64_t)h * a.head_stride;
+  // ---- row offsets of this CTA's positions: all index loads, then all page-table loads -------
+  {
+    constexpr int kPer = kMaxChunk / kThreads;
+    const int32_t* bt = a.block_table + (int64_t)b * a.max_pages;
+    int pos[kPer], pg[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int j = tid + u * kThreads;
+      pos[u] = -1;
+      if (j < n_mine)
+        pos[u] = INDEXED ? a.idx[(int64_t)pair * a.budget + j_begin + j] : lo + j_begin + j;
     }
-    s_off[j] = off;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const bool in = pos[u] >= 0 && pos[u] < max_len;
+      pg[u] = in ? bt[pos[u] / a.page_size] : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int j = tid + u * kThreads;
+      if (j >= n_mine) continue;
+      int64_t off = -1;
+      if (pos[u] < 0 || pos[u] >= max_len) raise_flag(2u);
+      else if (pg[u] < 0 || (int64_t)pg[u] >= a.num_pages) raise_flag(1u);
+      else
+        off = (int64_t)pg[u] * a.page_stride + (int64_t)(pos[u] % a.page_size) * a.slot_stride +
+              (int64_t)h * a.head_stride;
+      s_off[j] = off;
+    }
   }
   __syncthreads();
 
-  // ---- per-warp tiles, next tile's loads in flight ------------------------------------------
+  // ---- per-warp tiles through a ring of shared-memory stages --------------------------------
   const int n_tiles = (n_mine + kTile - 1) / kTile;
+  const int n_warp_tiles = warp < n_tiles ? (n_tiles - warp + kWarps - 1) / kWarps : 0;
   const float scale_log2 = a.scale * 1.4426950408889634f;
   float o[KB][4];
 #pragma unroll
   for (int m = 0; m < KB; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
   float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};  // heads 2t, 2t+1
 
-  TileRegs<D> cur, nxt;
-  int tile = warp;
-  if (tile < n_tiles) load_tile<D>(cur, a.k_cache, a.v_cache, s_off, tile, n_mine, lane);
-  for (; tile < n_tiles; tile += kWarps) {
-    if (tile + kWarps < n_tiles)
-      load_tile<D>(nxt, a.k_cache, a.v_cache, s_off, tile + kWarps, n_mine, lane);
+  const uint32_t ring = smem_u32(att_ring) + warp * kStages * kStageBytes;
+  // copies of tile `tl` into stage `st`: piece p = 32 it + lane is row p / 16, chunk p % 16
+  auto issue = [&](int tl, int st) {
+    const int j0 = tl * kTile;
+#pragma unroll
+    for (int it = 0; it < kTile * 16 / 32; ++it) {
+      const int p = 32 * it + lane;
+      const int row = p >> 4, c = p & 15;
+      const int j = j0 + row;
+      const int64_t off = j < n_mine ? s_off[j] : -1;
+      const int64_t src = (off >= 0 ? off : 0) + c * 8;
+      const uint32_t dst = ring + st * kStageBytes + row * 256 + ((c ^ (row & 7)) << 4);
+      cp_async16(dst, a.k_cache + src, off >= 0 ? 16 : 0);
+      cp_async16(dst + kTileBytes, a.v_cache + src, off >= 0 ? 16 : 0);
+    }
+  };
+#pragma unroll
+  for (int i = 0; i < kStages - 1; ++i) {
+    if (i < n_warp_tiles) issue(warp + kWarps * i, i);
+    cp_async_commit();
+  }
+  // ldmatrix row addresses (lane -> matrix lane / 8, row lane % 8)
+  const int mat = lane >> 3, mr = lane & 7;
+  const int k_row = (mat & 1) * 8 + mr, k_half = mat >> 1;  // K: rows 0-7 / 8-15, k lo / hi
+  const int v_row = (mat >> 1) * 8 + mr, v_half = mat & 1;  // V: tokens 0-7 / 8-15, dims lo / hi
+  for (int i = 0; i < n_warp_tiles; ++i) {
+    if (i + kStages - 1 < n_warp_tiles)
+      issue(warp + kWarps * (i + kStages - 1), (i + kStages - 1) % kStages);
+    cp_async_commit();
+    cp_async_wait<kStages - 1>();
+    __syncwarp();
+    const int tile = warp + kWarps * i;
+    const uint32_t st = ring + (i % kStages) * kStageBytes;
 
     // S^T (16 tokens x 8 heads) = K Q^T
     float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int kb = 0; kb < KB; ++kb) {
-      const int c = kb >> 1, w0 = (kb & 1) * 2;
-      const uint32_t a0 = word(cur.k[0][c], w0), a2 = word(cur.k[0][c], w0 + 1);
-      const uint32_t a1 = word(cur.k[1][c], w0), a3 = word(cur.k[1][c], w0 + 1);
+      const int c = 2 * kb + k_half;
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(st + k_row * 256 + ((c ^ (k_row & 7)) << 4), a0, a1, a2, a3);
       mma_bf16(s, a0, a1, a2, a3, qb0[kb], qb1[kb]);
     }
     // rows: token g (s[0], s[1]) and g+8 (s[2], s[3]); columns: heads 2t, 2t+1
@@ -214,26 +214,26 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(AttendArgs a, int c
     const uint32_t pl1 = pack_bf16x2(p[2] - bf16_lo(ph1), p[3] - bf16_hi(ph1));
     const uint32_t bh0 = movmatrix_t(ph0), bh1 = movmatrix_t(ph1);
     const uint32_t bl0 = movmatrix_t(pl0), bl1 = movmatrix_t(pl1);
-    // O^T (dims x heads) += V^T P^T; m-tile m: rows g, g+8 = physical dims D/8*g + 2m, +1
+    // O^T (dims x heads) += V^T P^T; m-tile m: rows = dims 16m + g and 16m + g + 8
 #pragma unroll
     for (int m = 0; m < KB; ++m) {
-      const int c = m >> 2, wi = m & 3;
-      const uint32_t r0 = word(cur.v[0][c], wi), r1 = word(cur.v[1][c], wi);
-      const uint32_t r2 = word(cur.v[2][c], wi), r3 = word(cur.v[3][c], wi);
-      const uint32_t va0 = prmt(r0, r1, 0x5410u), va1 = prmt(r0, r1, 0x7632u);
-      const uint32_t va2 = prmt(r2, r3, 0x5410u), va3 = prmt(r2, r3, 0x7632u);
+      const int c = 2 * m + v_half;
+      uint32_t va0, va1, va2, va3;
+      ldsm_x4_t(st + kTileBytes + v_row * 256 + ((c ^ (v_row & 7)) << 4), va0, va1, va2, va3);
       mma_bf16(o[m], va0, va1, va2, va3, bh0, bh1);
       mma_bf16(o[m], va0, va1, va2, va3, bl0, bl1);
     }
-    cur = nxt;
+    __syncwarp();  // the stage is refilled by the next iteration's copies
   }
+  cp_async_wait<0>();
 #pragma unroll
   for (int sh = 4; sh < 32; sh <<= 1) {
     l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], sh);
     l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], sh);
   }
 
-  // ---- merge the 4 warps ---------------------------------------------------------------------
+  // ---- merge the 4 warps (their rings are done: the shared memory is reused) ------------------
+  __syncthreads();
   {
     const int hh0 = 2 * t, hh1 = 2 * t + 1;
     if (g == 0) {
@@ -242,9 +242,9 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(AttendArgs a, int c
     }
 #pragma unroll
     for (int m = 0; m < KB; ++m) {
-      const int d0 = (D / 8) * g + 2 * m;  // physical dims of rows g and g+8 of m-tile m
-      if (hh0 < G) { s_o[warp][hh0][d0] = o[m][0]; s_o[warp][hh0][d0 + 1] = o[m][2]; }
-      if (hh1 < G) { s_o[warp][hh1][d0] = o[m][1]; s_o[warp][hh1][d0 + 1] = o[m][3]; }
+      const int d0 = 16 * m + g;  // dims of rows g and g+8 of m-tile m
+      if (hh0 < G) { s_o[warp][hh0][d0] = o[m][0]; s_o[warp][hh0][d0 + 8] = o[m][2]; }
+      if (hh1 < G) { s_o[warp][hh1][d0] = o[m][1]; s_o[warp][hh1][d0 + 8] = o[m][3]; }
     }
   }
   __syncthreads();
@@ -312,10 +312,13 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(AttendArgs a, int c
 template <int D, bool INDEXED>
 cudaError_t launch_t(const AttendArgs& a, const AttendPlan& plan, bool pdl, cudaStream_t s) {
   auto kern = attend_kernel<D, INDEXED>;
+  static_assert(kRingBytes >= kWarps * kAttendMaxG * 128 * (int)sizeof(float), "merge buffer");
+  cudaError_t ce = configure_kernel((const void*)kern, kRingBytes, false);
+  if (ce != cudaSuccess) return ce;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(plan.splits, a.batch * a.h_kv, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = kRingBytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

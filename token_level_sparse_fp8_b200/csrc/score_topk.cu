@@ -502,16 +502,27 @@ __device__ __forceinline__ uint32_t scan_warp(const ChunkGeom& cg, const int32_t
   return run;
 }
 
-// Page list of a chunk into shared memory (bounds checked; -1 = unusable page).
+// Page list of a chunk into shared memory (bounds checked; -1 = unusable page); four loads per
+// thread in flight at a time.
 __device__ __forceinline__ void load_pages(int32_t* s_page, const int32_t* bt, int n_pages,
                                            int64_t num_pages) {
-  for (int i = threadIdx.x; i < n_pages; i += blockDim.x) {
-    int32_t pg = bt[i];
-    if (pg < 0 || (int64_t)pg >= num_pages) {
-      raise_flag(1u);
-      pg = -1;
+  for (int i0 = threadIdx.x; i0 < n_pages; i0 += 4 * blockDim.x) {
+    int32_t pg[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * blockDim.x;
+      pg[u] = i < n_pages ? bt[i] : 0;
     }
-    s_page[i] = pg;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i >= n_pages) continue;
+      if (pg[u] < 0 || (int64_t)pg[u] >= num_pages) {
+        raise_flag(1u);
+        pg[u] = -1;
+      }
+      s_page[i] = pg[u];
+    }
   }
 }
 
