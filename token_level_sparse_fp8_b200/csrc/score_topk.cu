@@ -693,33 +693,33 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(PrepArgs a) {
     if (k >= kSample / 2) k = 0;
   }
   if (k) {
-    // the sampled code rows go straight to shared memory: each thread looks up the pages of its
-    // groups and copies their rows with asynchronous 16-byte copies (a group is one contiguous
-    // run of kGroup rows in one page when pages hold at least kGroup tokens; otherwise each
-    // position is looked up); a row on an unusable page is zero-filled and marked invalid
-    constexpr int kPer = kSampleGroups / kThreads;
-    constexpr int kPieces = R / 16;
-    int p0[kPer], pg0[kPer];
+    // the sampled code rows go straight to shared memory with asynchronous 16-byte copies; a
+    // warp instruction covers whole groups (kGroup rows of r bytes, one contiguous run when the
+    // page holds at least kGroup tokens), so its lanes coalesce into a few line requests. A row
+    // on an unusable page is zero-filled and marked invalid.
+    constexpr int kPieces = R / 16;                       // 16-byte pieces per row
+    constexpr int kLanesPerGroup = kGroup * kPieces;      // 8 (r = 32) or 16 (r = 64)
+    constexpr int kGroupsPerIssue = 32 / kLanesPerGroup;  // groups per warp instruction
+    constexpr int kWarpGroups = kSampleGroups / kWarps;   // 64 groups per warp
+    constexpr int kIssues = kWarpGroups / kGroupsPerIssue;
+    const int gl = lane / kLanesPerGroup, piece = lane % kLanesPerGroup;
+    const int j = piece / kPieces, part = piece % kPieces;
+    int p0[kIssues], pg0[kIssues];
 #pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      p0[u] = sample_group_start(tid + u * kThreads, pair, L);
-      pg0[u] = bt[p0[u] >> a.page_shift];
+    for (int u = 0; u < kIssues; ++u) {
+      const int grp = warp * kWarpGroups + u * kGroupsPerIssue + gl;
+      p0[u] = sample_group_start(grp, pair, L);
+      pg0[u] = bt[(p0[u] + (page_size >= kGroup ? 0 : j)) >> a.page_shift];
     }
 #pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int grp = tid + u * kThreads;
-#pragma unroll
-      for (int j = 0; j < kGroup; ++j) {
-        const int pos = p0[u] + j, i = grp * kGroup + j;
-        int32_t pg = page_size >= kGroup ? pg0[u] : bt[pos >> a.page_shift];
-        if (pg < 0 || (int64_t)pg >= a.num_pages) pg = -1;
-        sm.valid[i] = pg >= 0;
-        const uint8_t* src = a.score_cache +
-            ((((int64_t)max(pg, 0) * a.h_kv + h) << a.page_shift) + (pos & (page_size - 1))) * R;
-#pragma unroll
-        for (int c = 0; c < kPieces; ++c)
-          cp_async16(smem_u32(sm.rows + i * R + c * 16), src + c * 16, pg >= 0 ? 16 : 0);
-      }
+    for (int u = 0; u < kIssues; ++u) {
+      const int grp = warp * kWarpGroups + u * kGroupsPerIssue + gl;
+      const int pos = p0[u] + j, i = grp * kGroup + j;
+      const int32_t pg = (pg0[u] < 0 || (int64_t)pg0[u] >= a.num_pages) ? -1 : pg0[u];
+      if (part == 0) sm.valid[i] = pg >= 0;
+      const uint8_t* src = a.score_cache +
+          ((((int64_t)max(pg, 0) * a.h_kv + h) << a.page_shift) + (pos & (page_size - 1))) * R;
+      cp_async16(smem_u32(sm.rows + i * R + part * 16), src + part * 16, pg >= 0 ? 16 : 0);
     }
   }
   cp_async_commit();  // (group: the sample rows; M_h is the group before)
