@@ -476,12 +476,23 @@ def run_jssa(args):
         J.score_topk(qs[i % nq], layer.basis, layer.score_cache, layer.block_table, layer.seq_lens,
                      w.budget, idx, count, ws_score)
 
-    def attend_only(i):
-        J.indexed_attend(qs[i % nq], layer.k_cache, layer.v_cache, layer.block_table, idx, count,
-                         layer.scale, out, ws_attend)
-
     t_score, n_score = timed_graph(score_only, args.steps, args.warmup, stream, barrier, nq)
     t_score = max_over_ranks(t_score) / n_score
+
+    # the attention alone, on the index set of each rotating query set (so its K/V rows change
+    # from launch to launch as in the step, instead of repeating one set out of L2)
+    sets = []
+    for i in range(nq):
+        ii, cc = torch.empty_like(idx), torch.empty_like(count)
+        J.score_topk(qs[i], layer.basis, layer.score_cache, layer.block_table, layer.seq_lens,
+                     w.budget, ii, cc, ws_score)
+        sets.append((ii, cc))
+
+    def attend_only(i):
+        ii, cc = sets[i % nq]
+        J.indexed_attend(qs[i % nq], layer.k_cache, layer.v_cache, layer.block_table, ii, cc,
+                         layer.scale, out, ws_attend)
+
     t_attend, n_attend = timed_graph(attend_only, args.steps, args.warmup, stream, barrier, nq)
     t_attend = max_over_ranks(t_attend) / n_attend
 

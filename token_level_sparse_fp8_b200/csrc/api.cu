@@ -244,7 +244,7 @@ int jssa_score_topk(const jssa_bf16* q, const float* basis, const uint8_t* score
   return cuda_status(jssa::launch_score_topk(q, basis, score_cache, block_table, max_pages,
                                              seq_lens, batch, h_q, h_kv, d, r, num_pages,
                                              page_size, budget, idx, count, ws, nullptr,
-                                             nullptr, false, as_stream(stream)));
+                                             nullptr, true, as_stream(stream)));
 }
 
 static int check_attend_common(const jssa_bf16* q, const jssa_bf16* k_cache,
@@ -352,7 +352,7 @@ int jssa_decode(const jssa_bf16* q, const jssa_bf16* k_new, const jssa_bf16* v_n
                                           batch, h_q, h_kv, d, r, num_pages, page_size, budget,
                                           idx, count, cand_ws,
                                           plan.ws_bytes ? static_cast<int*>(attend_ws) : nullptr,
-                                          k_new ? &sn : nullptr, false, s);
+                                          k_new ? &sn : nullptr, true, s);
   if (e != cudaSuccess) return (int)e;
   AttendArgs a = {};
   a.q = q; a.k_cache = k_cache; a.v_cache = v_cache;

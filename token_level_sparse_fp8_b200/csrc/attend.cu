@@ -120,6 +120,9 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(AttendArgs a, int c
     }
   }
   __syncthreads();
+  // a kernel launched next may be scheduled now; it waits for this grid to complete before
+  // reading anything (the decode step's first kernel does)
+  pdl_trigger();
 
   // ---- per-warp tiles through a ring of shared-memory stages --------------------------------
   const int n_tiles = (n_mine + kTile - 1) / kTile;

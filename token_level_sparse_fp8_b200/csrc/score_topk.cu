@@ -577,12 +577,12 @@ __global__ void __launch_bounds__(kThreads, 3) scan_kernel(ScanArgs a) {
              n_pages, a.num_pages);
   __syncthreads();
   pdl_wait();  // digits, threshold and the new token's code come from the prep kernel
+  pdl_trigger();  // the select may be scheduled; it waits for this grid to complete
   const uint8_t* rec = a.prep.rec + (int64_t)pair * kPrepBytes;
   const int mode = *reinterpret_cast<const int*>(rec + kPrepMode);
   if (mode == kModeAll || n_local == 0) {
     if ((threadIdx.x & 31) == 0 && (threadIdx.x >> 5) < kRegionsPerChunk)
       a.cands.cnt[((int64_t)pair * a.n_chunks + c) * kRegionsPerChunk + (threadIdx.x >> 5)] = 0u;
-    pdl_trigger();
     return;
   }
   DigitFrags<R> df;
@@ -590,7 +590,6 @@ __global__ void __launch_bounds__(kThreads, 3) scan_kernel(ScanArgs a) {
           threadIdx.x & 31);
   const uint32_t thr = *reinterpret_cast<const uint32_t*>(rec + kPrepThr);
   scan_chunk<R>(a, pair, c, L, thr, df, scan_pages);
-  pdl_trigger();
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -660,6 +659,12 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(PrepArgs a) {
   const int page_size = 1 << a.page_shift;
   const int32_t* bt = a.block_table + (int64_t)b * a.max_pages;
   const float* m_h = a.basis + (int64_t)h * R * D;
+
+  // launched as a programmatic dependent of whatever precedes it on the stream: nothing is read
+  // before that kernel has completed. The scan may be scheduled at once (it waits for this grid
+  // before reading what it writes).
+  pdl_wait();
+  pdl_trigger();
 
   // ---- independent loads first: M_h into shared memory (async), L, qbar, the sample's pages ----
   for (int i = tid; i < R * D / 4; i += kThreads) cp_async16(smem_u32(sm.m + 4 * i), m_h + 4 * i, 16);
@@ -858,9 +863,6 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(PrepArgs a) {
     *reinterpret_cast<uint32_t*>(rec + kPrepThr) = thr;
     *reinterpret_cast<int*>(rec + kPrepMode) = mode;
   }
-  // complete only after the kernel before this one: the scan reads what both wrote
-  pdl_wait();
-  pdl_trigger();
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -895,6 +897,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
   const int budget = a.budget;
   int32_t* out_idx = s.idx + (int64_t)pair * budget;
   pdl_wait();  // the scan's candidates
+  pdl_trigger();  // the attention may be scheduled; it waits for this grid to complete
   const uint8_t* rec = a.prep.rec + (int64_t)pair * kPrepBytes;
   const int mode = *reinterpret_cast<const int*>(rec + kPrepMode);
   if (mode == kModeAll) {
@@ -903,7 +906,6 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
       s.count[pair] = L;
       if (a.cands.attend_tickets) a.cands.attend_tickets[pair] = 0;
     }
-    pdl_trigger();
     return;
   }
   const int n_reg = a.n_chunks * kRegionsPerChunk;
@@ -1070,7 +1072,6 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
     // the attention launched next merges its splits through these counters
     if (a.cands.attend_tickets) a.cands.attend_tickets[pair] = 0;
   }
-  pdl_trigger();
 }
 
 template <typename Kern, typename... Args>
