@@ -45,7 +45,7 @@ constexpr int kSelectCap = 16384;  // candidates the select kernel stages in sha
 constexpr int kRegionsPerChunk = kWarps;  // candidate regions (one per scan warp) per chunk
 constexpr int kMaxRegions = 4096;  // candidate regions per (sequence, KV head)
 constexpr int kPrepBytes = 1024;   // per (sequence, KV head): digits, scales, threshold, mode
-constexpr int kPrepScale = 512, kPrepThr = 544, kPrepMode = 548;
+constexpr int kPrepScale = 512, kPrepThr = 544, kPrepMode = 548, kPrepKmax = 552;
 constexpr int kModeScan = 0, kModeAll = 1;
 
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t x, int lane) {
@@ -262,6 +262,54 @@ __device__ void select_threshold(KeyAt key_at, int n, uint32_t want, uint32_t km
   thr = (int64_t)(uint32_t)s_info[0];
   take = (uint32_t)s_info[1];
   __syncthreads();
+}
+
+// Exact threshold (contract of radix_select) from a histogram of the n keys built beforehand
+// with bin(key) = min(2047, (key - base) >> shift), every key >= base: the bin of the want-th
+// largest key, taken whole or resolved by ranking its keys (at most 256) against each other.
+// Returns false, leaving thr / take unset, when that bin is the top one (it also holds every key
+// above the range) or holds more keys: the caller then runs a general selection.
+template <int NT, typename KeyAt>
+__device__ bool threshold_from_hist(KeyAt key_at, int n, uint32_t want, uint32_t base, int shift,
+                                    uint32_t* s_hist, uint32_t* s_wsum, int* s_info, int64_t& thr,
+                                    uint32_t& take) {
+  const int tid = threadIdx.x;
+  find_bin<NT>(s_hist, kBins, want, s_wsum, s_info);
+  const bool found = s_info[3] != 0;
+  const uint32_t bin = (uint32_t)s_info[0], m = (uint32_t)s_info[2];
+  const uint32_t w2 = want - (uint32_t)s_info[1];
+  __syncthreads();  // s_info and s_hist are reused below
+  if (!found || bin == kBins - 1 || (w2 != m && m > 256)) return false;
+  if (w2 == m) {
+    thr = (int64_t)base + ((int64_t)bin << shift) - 1;
+    take = 0;
+    return true;
+  }
+  if (tid == 0) s_info[3] = 0;
+  __syncthreads();
+  for (int i = tid; i < n; i += NT) {
+    const uint32_t key = key_at(i);
+    if (((key - base) >> shift) == bin) s_hist[atomicAdd(&s_info[3], 1)] = key;
+  }
+  __syncthreads();
+  if (tid < (int)m) {
+    const uint32_t x = s_hist[tid];
+    uint32_t gt = 0, eq = 0;
+    for (uint32_t j = 0; j < m; ++j) {
+      const uint32_t y = s_hist[j];
+      gt += y > x;
+      eq += y == x;
+    }
+    if (gt < w2 && w2 <= gt + eq) {  // x is the w2-th largest of the bin (equal keys agree)
+      s_info[0] = (int)x;
+      s_info[1] = (int)(w2 - gt);
+    }
+  }
+  __syncthreads();
+  thr = (int64_t)(uint32_t)s_info[0];
+  take = (uint32_t)s_info[1];
+  __syncthreads();
+  return true;
 }
 
 struct Prep {
@@ -768,13 +816,16 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(PrepArgs a) {
     constexpr int DPT = D / TPJ;
     static_assert(TPJ >= 1 && TPJ <= 32 && D % TPJ == 0, "projection split");
     const int j = tid / TPJ, sub = tid % TPJ;
-    const float* mrow = sm.m + j * D + sub * DPT;
+    const float* mrow = sm.m + j * D;
     float acc = 0.f;
     double acc_k = 0.0;
+    // thread sub takes dims sub, sub + TPJ, ... (interleaved: neighbouring threads read
+    // neighbouring words)
 #pragma unroll
     for (int i = 0; i < DPT; ++i) {
-      acc = fmaf(mrow[i], s_qbar[sub * DPT + i], acc);
-      if (store) acc_k = fma((double)mrow[i], (double)s_k[sub * DPT + i], acc_k);
+      const int e = i * TPJ + sub;
+      acc = fmaf(mrow[e], s_qbar[e], acc);
+      if (store) acc_k = fma((double)mrow[e], (double)s_k[e], acc_k);
     }
 #pragma unroll
     for (int o = TPJ / 2; o > 0; o >>= 1) {
@@ -826,7 +877,8 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(PrepArgs a) {
   if (tid < kDigits) reinterpret_cast<float*>(rec + kPrepScale)[tid] = s_scale[tid];
 
   // ---- candidate threshold from the sample ----------------------------------------------------
-  uint32_t thr = 0u;  // every key of a finite score is above 0
+  uint32_t thr = 0u;       // every key of a finite score is above 0
+  uint32_t sample_max = 0u;  // largest sampled key (0: no sample)
   if (k) {
     cp_async_wait<0>();
     __syncthreads();  // every thread's sample rows
@@ -851,17 +903,20 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(PrepArgs a) {
       sm.skey[i] = key;
     }
     block_min_max<kThreads>(kmin, kmax, s_wsum);  // (its barrier also publishes the keys)
-    // one radix pass of 11 bits over the sample's own key range: the lowest key of the bin that
-    // holds the k-th largest sampled key (or that key itself when the range is narrow)
+    sample_max = kmax;
+    // two radix passes of 11 bits over the sample's own key range: the k-th largest sampled key
+    // itself, or the lowest key of a second-pass bin that holds it (a much narrower bin than one
+    // pass leaves, so few more tokens than the margin asks for become candidates)
     int64_t t64;
     uint32_t take;
-    radix_select<kThreads>([&](int i) { return sm.skey[i]; }, kSample, (uint32_t)k, kmin, kmax, 1,
+    radix_select<kThreads>([&](int i) { return sm.skey[i]; }, kSample, (uint32_t)k, kmin, kmax, 2,
                            sm.hist, s_wsum, s_info, t64, take);
     thr = (uint32_t)(take ? t64 : t64 + 1);  // candidates: keys >= thr
   }
   if (tid == 0) {
     *reinterpret_cast<uint32_t*>(rec + kPrepThr) = thr;
     *reinterpret_cast<int*>(rec + kPrepMode) = mode;
+    *reinterpret_cast<uint32_t*>(rec + kPrepKmax) = sample_max;
   }
 }
 
@@ -914,6 +969,13 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
   const int32_t* cp = a.cands.pos + (int64_t)pair * n_reg * seg;
   const uint32_t* cc = a.cands.cnt + (int64_t)pair * n_reg;
   const uint32_t want = (uint32_t)min(budget, L);
+  // histogram of the candidate keys, built while they are staged, over [the prep's threshold,
+  // the largest sampled key] (keys above it fall into the top bin)
+  const uint32_t base = *reinterpret_cast<const uint32_t*>(rec + kPrepThr);
+  const uint32_t sample_max = *reinterpret_cast<const uint32_t*>(rec + kPrepKmax);
+  bool use_hist = base > 0u && sample_max > base;
+  const int hshift = use_hist ? max(0, (32 - __clz(sample_max - base)) - 11) : 0;
+  for (int i = tid; i < kBins; i += kSelThreads) s_hist[i] = 0u;
 
   // region offsets: exclusive prefix of the counts, in position order (each thread loads and
   // sums a run of adjacent regions, then a block-wide scan)
@@ -943,6 +1005,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
     // rescue: the sampled threshold was too high; score every token of the sequence again with
     // no threshold (all keys become candidates), then select exactly as usual
     if (tid == 0) raise_flag(16u);
+    use_hist = false;
     DigitFrags<R> df;
     df.load(reinterpret_cast<const uint16_t*>(rec), reinterpret_cast<const float*>(rec + kPrepScale),
             lane);
@@ -1009,6 +1072,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
             s_cpos[off + i] = pp[u][e];
             kmin = min(kmin, kk[u][e]);
             kmax = max(kmax, kk[u][e]);
+            if (use_hist) atomicAdd(&s_hist[min(kBins - 1u, (kk[u][e] - base) >> hshift)], 1u);
           }
         }
         for (uint32_t i = 64 + lane; i < cnt; i += 32) {
@@ -1017,6 +1081,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
           s_cpos[off + i] = cp[(int64_t)r * seg + i];
           kmin = min(kmin, key);
           kmax = max(kmax, key);
+          if (use_hist) atomicAdd(&s_hist[min(kBins - 1u, (key - base) >> hshift)], 1u);
         }
       }
     }
@@ -1027,44 +1092,65 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
       kmax = max(kmax, key);
     }
   }
-  block_min_max<kSelThreads>(kmin, kmax, s_wsum);  // (its barrier also publishes the candidates)
+  __syncthreads();  // the staged candidates and their histogram
   auto key_at = [&](int j) -> uint32_t { return staged ? s_ckey[j] : ck[src_of(j)]; };
   auto pos_at = [&](int j) -> int32_t { return staged ? s_cpos[j] : cp[src_of(j)]; };
   int64_t thr;
   uint32_t take;
-  select_threshold<kSelThreads>(key_at, (int)n, want, kmin, kmax, s_hist, s_wsum, s_info, thr,
-                                take);
+  const bool done = use_hist && staged &&
+                    threshold_from_hist<kSelThreads>(key_at, (int)n, want, base, hshift, s_hist,
+                                                     s_wsum, s_info, thr, take);
+  if (!done) {
+    block_min_max<kSelThreads>(kmin, kmax, s_wsum);
+    select_threshold<kSelThreads>(key_at, (int)n, want, kmin, kmax, s_hist, s_wsum, s_info, thr,
+                                  take);
+  }
   // ordered emission: the selected candidates are the keys > thr and the first `take` keys == thr
-  // in position order, written in candidate (= position) order. Each thread owns a contiguous run
-  // of candidates; one block scan of (count > thr, count == thr) gives every candidate's slot:
-  // (keys > thr before it) + min(keys == thr before it, take).
-  const int per = ((int)n + kSelThreads - 1) / kSelThreads;
-  const int j0 = min((int)n, tid * per), j1 = min((int)n, j0 + per);
+  // in position order, written in candidate (= position) order at slot
+  // (keys > thr before it) + min(keys == thr before it, take). Warp w owns a contiguous span of
+  // candidates, read 32 at a time (consecutive lanes, consecutive words: no bank conflicts); the
+  // spans' counts are combined across warps in shared memory.
+  const unsigned lt = (1u << lane) - 1u;
+  const int warp_id = tid >> 5;
+  const int span = (((int)n + kSelWarps - 1) / kSelWarps + 31) & ~31;
+  const int lo = min((int)n, warp_id * span), hi = min((int)n, lo + span);
   uint32_t n_gt = 0, n_eq = 0;
-  for (int j = j0; j < j1; ++j) {
-    const int64_t key = (int64_t)key_at(j);
-    n_gt += key > thr;
-    n_eq += key == thr;
+  for (int i0 = lo; i0 < hi; i0 += 32) {
+    const int i = i0 + lane;
+    const int64_t key = i < hi ? (int64_t)key_at(i) : -1;
+    n_gt += __popc(__ballot_sync(0xffffffffu, key > thr));
+    n_eq += __popc(__ballot_sync(0xffffffffu, key == thr));
   }
-  uint64_t total;
-  const uint64_t before =
-      block_excl_scan64<kSelThreads>(((uint64_t)n_eq << 32) | n_gt, total, s_red64);
-  uint32_t gt_b = (uint32_t)before, eq_b = (uint32_t)(before >> 32);
-  for (int j = j0; j < j1; ++j) {
-    const int64_t key = (int64_t)key_at(j);
-    if (key > thr) {
-      const uint32_t at = gt_b + min(eq_b, take);
-      if (at < (uint32_t)budget) out_idx[at] = pos_at(j);
-      ++gt_b;
-    } else if (key == thr) {
-      if (eq_b < take) {
-        const uint32_t at = gt_b + eq_b;
-        if (at < (uint32_t)budget) out_idx[at] = pos_at(j);
-      }
-      ++eq_b;
+  if (lane == 0) {
+    s_wsum[warp_id] = n_gt;
+    s_wsum[kSelWarps + warp_id] = n_eq;
+  }
+  __syncthreads();
+  uint32_t gt_b = 0, eq_b = 0, total_gt = 0, total_eq = 0;
+  for (int w = 0; w < kSelWarps; ++w) {
+    const uint32_t a_ = s_wsum[w], e_ = s_wsum[kSelWarps + w];
+    if (w < warp_id) {
+      gt_b += a_;
+      eq_b += e_;
     }
+    total_gt += a_;
+    total_eq += e_;
   }
-  const uint32_t written = (uint32_t)total + min((uint32_t)(total >> 32), take);
+  for (int i0 = lo; i0 < hi; i0 += 32) {
+    const int i = i0 + lane;
+    const int64_t key = i < hi ? (int64_t)key_at(i) : -1;
+    const bool is_gt = key > thr, is_eq = key == thr;
+    const unsigned gtm = __ballot_sync(0xffffffffu, is_gt);
+    const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
+    const uint32_t g_before = gt_b + __popc(gtm & lt), e_before = eq_b + __popc(eqm & lt);
+    if (is_gt || (is_eq && e_before < take)) {
+      const uint32_t at = g_before + min(e_before, take);
+      if (at < (uint32_t)budget) out_idx[at] = pos_at(i);
+    }
+    gt_b += __popc(gtm);
+    eq_b += __popc(eqm);
+  }
+  const uint32_t written = total_gt + min(total_eq, take);
   for (int j = (int)want + tid; j < budget; j += kSelThreads) out_idx[j] = -1;
   if (tid == 0) {
     if (written != want) raise_flag(8u);
