@@ -312,6 +312,68 @@ __device__ bool threshold_from_hist(KeyAt key_at, int n, uint32_t want, uint32_t
   return true;
 }
 
+// The k-th largest of the sampled keys, NK of them in each thread's registers and all in
+// [kmin, kmax]: radix passes of 11 bits over the range the keys occupy (the first pass spreads
+// them over [kmin, kmax]) until the bin that holds the k-th largest key is one key value or holds
+// at most 256 keys, which are then ranked against each other. s_hist (kBins words) is zero on
+// entry; s_list holds 256 keys; *s_nlist is zero on entry. Every thread returns the same value.
+// Block-wide (NT threads).
+template <int NT, int NK>
+__device__ uint32_t sample_threshold(const uint32_t (&key)[NK], uint32_t k, uint32_t kmin,
+                                     uint32_t kmax, uint32_t* s_hist, uint32_t* s_list,
+                                     int* s_nlist, uint32_t* s_wsum, int* s_info) {
+  const int tid = threadIdx.x;
+  if (kmax == kmin) return kmin;
+  uint32_t lo = kmin;                   // lowest key of the current bin
+  int bits = 32 - __clz(kmax - kmin);   // the current bin is [lo, lo + 2^bits)
+  uint32_t want = k;                    // rank of the wanted key inside the current bin
+#pragma unroll 1
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = max(0, bits - 11);
+    if (pass > 0) {
+      for (int i = tid; i < kBins; i += NT) s_hist[i] = 0u;
+      __syncthreads();
+    }
+#pragma unroll
+    for (int j = 0; j < NK; ++j) {
+      const uint64_t v = (uint64_t)key[j] - lo;  // huge when key < lo
+      if ((v >> bits) == 0) atomicAdd(&s_hist[(uint32_t)v >> shift], 1u);
+    }
+    __syncthreads();
+    find_bin<NT>(s_hist, kBins, want, s_wsum, s_info);
+    if (!s_info[3]) {  // fewer keys than wanted: inconsistent input, every key qualifies
+      if (tid == 0) raise_flag(8u);
+      return kmin;
+    }
+    want -= (uint32_t)s_info[1];
+    const uint32_t m = (uint32_t)s_info[2];
+    lo += (uint32_t)s_info[0] << shift;
+    bits = shift;
+    if (bits == 0) return lo;
+    if (m <= 256) {
+      // rank the bin's keys: the want-th largest of them (equal keys agree)
+#pragma unroll
+      for (int j = 0; j < NK; ++j)
+        if ((((uint64_t)key[j] - lo) >> bits) == 0) s_list[atomicAdd(s_nlist, 1)] = key[j];
+      __syncthreads();
+      if (tid < (int)m) {
+        const uint32_t x = s_list[tid];
+        uint32_t gt = 0, eq = 0;
+        for (uint32_t i = 0; i < m; ++i) {
+          const uint32_t y = s_list[i];
+          gt += y > x;
+          eq += y == x;
+        }
+        if (gt < want && want <= gt + eq) s_info[0] = (int)x;
+      }
+      __syncthreads();
+      return (uint32_t)s_info[0];
+    }
+    __syncthreads();  // s_hist and s_info are reused by the next pass
+  }
+  return lo;  // not reached: three passes resolve 33 bits
+}
+
 struct Prep {
   uint8_t* rec;  // [pairs][kPrepBytes]: digits [8][R] at 0, scales at kPrepScale, threshold
                  // key at kPrepThr, mode at kPrepMode
@@ -680,13 +742,13 @@ struct PrepSmem {
   uint8_t rows[kSample * R];     // code rows of the sampled positions
   float m[R * D];                // M_h, row-major [R][D]
   float qpart[kQGroups][D];      // partial sums of the group's query rows
-  uint32_t skey[kSample];        // sampled keys
+  uint32_t list[256];            // keys of the bin that holds the threshold
   uint32_t hist[kBins];
   uint8_t valid[kSample];        // sampled position on a usable page
 };
 
 template <int D, int R, bool STORE>
-__global__ void __launch_bounds__(kThreads) prep_kernel(PrepArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
   constexpr int LB = R / 4;
   constexpr int kTilesPerWarp = kSample / 16 / kWarps;  // 16
   extern __shared__ __align__(16) uint8_t prep_dyn[];
@@ -698,6 +760,7 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(PrepArgs a) {
   __shared__ float s_scale[kDigits];
   __shared__ uint32_t s_wsum[2 * kWarps];
   __shared__ int s_info[4];
+  __shared__ int s_nlist;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
@@ -714,28 +777,26 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(PrepArgs a) {
   pdl_wait();
   pdl_trigger();
 
-  // ---- independent loads first: M_h into shared memory (async), L, qbar, the sample's pages ----
+  // ---- independent loads first: M_h into shared memory (async); L, the group's query rows and
+  // the new token's K and V rows into registers ----
   for (int i = tid; i < R * D / 4; i += kThreads) cp_async16(smem_u32(sm.m + 4 * i), m_h + 4 * i, 16);
   cp_async_commit();
   const int L = clamp_len(a.seq_lens[b], a.max_pages << a.page_shift);
-  {
-    // the G query rows of this KV head: 16 threads x 8 dims per row, kQGroups rows at a time
-    static_assert(D == 128, "query row split");
-    const uint16_t* qh = a.q + ((int64_t)b * a.h_q + (int64_t)h * G) * D;
-    const int rg = tid / 16, d8 = (tid % 16) * 8;
-    float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int r = rg; r < G; r += kQGroups) {
-      const uint4 v = *reinterpret_cast<const uint4*>(qh + (int64_t)r * D + d8);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        part[2 * e] += bf16_lo(w[e]);
-        part[2 * e + 1] += bf16_hi(w[e]);
-      }
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) sm.qpart[rg][d8 + e] = part[e];
+  // the G query rows of this KV head: 16 threads x 8 dims per row, kQGroups rows at a time
+  static_assert(D == 128, "query row split");
+  const uint16_t* qh = a.q + ((int64_t)b * a.h_q + (int64_t)h * G) * D;
+  const int rg = tid / 16, d8 = (tid % 16) * 8;
+  uint4 qv = make_uint4(0u, 0u, 0u, 0u);
+  if (rg < G) qv = *reinterpret_cast<const uint4*>(qh + (int64_t)rg * D + d8);
+  const bool store = STORE && L > 0;
+  uint16_t k_el = 0, v_el = 0;  // element tid of the new token's K and V rows (tid < D)
+  if (STORE && tid < D) {
+    k_el = a.store.k_new[((int64_t)b * a.h_kv + h) * D + tid];
+    v_el = a.store.v_new[((int64_t)b * a.h_kv + h) * D + tid];
   }
+  for (int i = tid; i < kBins; i += kThreads) sm.hist[i] = 0u;
+  if (tid == 0) s_nlist = 0;
+
   int mode = kModeScan;
   int k = 0;  // sampled keys to reach (0: no sampling, every key is a candidate)
   if (L <= a.budget) {
@@ -745,6 +806,9 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(PrepArgs a) {
     k = (int)ceil(expect + 4.0 * sqrt(expect) + 8.0);
     if (k >= kSample / 2) k = 0;
   }
+  // decode: the page of the new token (position L - 1), read with the sample's pages
+  int32_t st_page = -1;
+  if (store) st_page = bt[(L - 1) >> a.page_shift];
   if (k) {
     // the sampled code rows go straight to shared memory with asynchronous 16-byte copies; a
     // warp instruction covers whole groups (kGroup rows of r bytes, one contiguous run when the
@@ -776,27 +840,41 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(PrepArgs a) {
     }
   }
   cp_async_commit();  // (group: the sample rows; M_h is the group before)
-  const bool store = STORE && L > 0;
-  int32_t st_page = -1;
+  {
+    float part[8];
+    const uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      part[2 * e] = bf16_lo(w[e]);
+      part[2 * e + 1] = bf16_hi(w[e]);
+    }
+    for (int r = rg + kQGroups; r < G; r += kQGroups) {  // more than kQGroups rows per group
+      const uint4 v = *reinterpret_cast<const uint4*>(qh + (int64_t)r * D + d8);
+      const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        part[2 * e] += bf16_lo(x[e]);
+        part[2 * e + 1] += bf16_hi(x[e]);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sm.qpart[rg][d8 + e] = part[e];
+  }
   if (store) {  // decode: copy the new token's K and V rows into the cache
-    const StoreNew& st = a.store;
-    const int pos = L - 1;
-    st_page = bt[pos >> a.page_shift];
     if (st_page < 0 || (int64_t)st_page >= a.num_pages) {
       if (tid == 0) raise_flag(1u);
       st_page = -1;
     }
-    const uint16_t* krow = st.k_new + ((int64_t)b * a.h_kv + h) * D;
-    const uint16_t* vrow = st.v_new + ((int64_t)b * a.h_kv + h) * D;
-    for (int i = tid; i < D; i += kThreads) {
-      const uint16_t kv = krow[i], vv = vrow[i];
-      s_k[i] = bf16_to_f(kv);
+    const StoreNew& st = a.store;
+    const int pos = L - 1;
+    if (tid < D) {
+      s_k[tid] = bf16_to_f(k_el);
       if (st_page >= 0) {
         const int64_t base = (int64_t)st_page * st.page_stride +
                              (int64_t)(pos & (page_size - 1)) * st.slot_stride +
                              (int64_t)h * st.head_stride;
-        st.k_cache[base + i] = kv;
-        st.v_cache[base + i] = vv;
+        st.k_cache[base + tid] = k_el;
+        st.v_cache[base + tid] = v_el;
       }
     }
   }
@@ -885,7 +963,8 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(PrepArgs a) {
     DigitFrags<R> df;
     df.load(s_dig, s_scale, lane);
     uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-#pragma unroll 4
+    uint32_t key[kTilesPerWarp / 2];  // this lane's sampled keys
+#pragma unroll
     for (int u = 0; u < kTilesPerWarp; u += 2) {
       const int i0 = (warp * kTilesPerWarp + u) * 16;
       uint32_t ra0[R / 16], rb0[R / 16], ra1[R / 16], rb1[R / 16];
@@ -897,21 +976,15 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(PrepArgs a) {
       // lane t holds sample 16 * (t >> 1) + 8 * (t & 1) + g of the two tiles
       const int i = i0 + 16 * (t >> 1) + 8 * (t & 1) + g;
       // a sample on an unusable page (flagged by the scan) counts as the lowest key
-      const uint32_t key = sm.valid[i] ? score_key(f) : 0u;
-      kmin = min(kmin, key);
-      kmax = max(kmax, key);
-      sm.skey[i] = key;
+      key[u / 2] = sm.valid[i] ? score_key(f) : 0u;
+      kmin = min(kmin, key[u / 2]);
+      kmax = max(kmax, key[u / 2]);
     }
-    block_min_max<kThreads>(kmin, kmax, s_wsum);  // (its barrier also publishes the keys)
+    block_min_max<kThreads>(kmin, kmax, s_wsum);
     sample_max = kmax;
-    // two radix passes of 11 bits over the sample's own key range: the k-th largest sampled key
-    // itself, or the lowest key of a second-pass bin that holds it (a much narrower bin than one
-    // pass leaves, so few more tokens than the margin asks for become candidates)
-    int64_t t64;
-    uint32_t take;
-    radix_select<kThreads>([&](int i) { return sm.skey[i]; }, kSample, (uint32_t)k, kmin, kmax, 2,
-                           sm.hist, s_wsum, s_info, t64, take);
-    thr = (uint32_t)(take ? t64 : t64 + 1);  // candidates: keys >= thr
+    // the k-th largest sampled key: the tokens whose keys reach it become candidates
+    thr = sample_threshold<kThreads>(key, (uint32_t)k, kmin, kmax, sm.hist, sm.list, &s_nlist,
+                                     s_wsum, s_info);
   }
   if (tid == 0) {
     *reinterpret_cast<uint32_t*>(rec + kPrepThr) = thr;
