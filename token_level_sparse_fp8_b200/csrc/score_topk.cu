@@ -312,49 +312,71 @@ __device__ bool threshold_from_hist(KeyAt key_at, int n, uint32_t want, uint32_t
   return true;
 }
 
-// The k-th largest of the sampled keys, NK of them in each thread's registers and all in
-// [kmin, kmax]: radix passes of 11 bits over the range the keys occupy (the first pass spreads
-// them over [kmin, kmax]) until the bin that holds the k-th largest key is one key value or holds
-// at most 256 keys, which are then ranked against each other. s_hist (kBins words) is zero on
-// entry; s_list holds 256 keys; *s_nlist is zero on entry. Every thread returns the same value.
-// Block-wide (NT threads).
-template <int NT, int NK>
+// The score a key was made from (score_key inverted); keys below the key of the lowest finite
+// score (unusable samples) give -inf.
+__device__ __forceinline__ float key_value(uint32_t key) {
+  if (key < 0x00800000u) return -INFINITY;
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// The k-th largest of the sampled keys, NK of them in each thread's registers; [kmin, kmax] is
+// the range of the keys of finite scores. Each pass histograms the keys still in play (all at
+// first, then those of the bin picked last) into NB bins spaced evenly in score over their range
+// (score keys are not linear in the score: one bin range in key space spans every binade of the
+// small scores near zero), finds the bin that holds the wanted key, and stops when that bin holds
+// at most 256 keys, which are then ranked against each other. Keys below kmin fall into the
+// lowest bin. s_hist (NB words) is zero on entry; s_list holds 256 keys; *s_nlist is zero on
+// entry. Every thread returns the same value. Block-wide (NT threads).
+template <int NT, int NB, int NK>
 __device__ uint32_t sample_threshold(const uint32_t (&key)[NK], uint32_t k, uint32_t kmin,
                                      uint32_t kmax, uint32_t* s_hist, uint32_t* s_list,
                                      int* s_nlist, uint32_t* s_wsum, int* s_info) {
+  static_assert(NB <= NT * 8 && (NB & (NB - 1)) == 0, "histogram size");
+  constexpr int kLog = NB == 256 ? 8 : NB == 512 ? 9 : NB == 1024 ? 10 : 11;
   const int tid = threadIdx.x;
-  if (kmax == kmin) return kmin;
-  uint32_t lo = kmin;                   // lowest key of the current bin
-  int bits = 32 - __clz(kmax - kmin);   // the current bin is [lo, lo + 2^bits)
-  uint32_t want = k;                    // rank of the wanted key inside the current bin
+  uint32_t live = (1u << NK) - 1u;  // bit j: key[j] is in the bin being refined
+  uint32_t lo = kmin, hi = kmax;    // key range of the live keys (of finite scores)
+  uint32_t want = k;                // rank of the wanted key among the live keys
 #pragma unroll 1
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = max(0, bits - 11);
+  for (int pass = 0; pass < 4; ++pass) {
+    if (hi <= lo) return hi;  // one key value left (or no finite score at all)
+    const float vlo = key_value(lo), vhi = key_value(hi);
+    const float scale = (float)NB / (vhi - vlo);
+    // bins evenly spaced in score; in key space when the score range is not representable
+    const bool linear = isfinite(vhi - vlo) && isfinite(scale) && scale > 0.f;
+    const int kshift = max(0, 32 - kLog - __clz(hi - lo));  // key space: at most NB bins
+    int kb[NK];
+#pragma unroll
+    for (int j = 0; j < NK; ++j) {
+      if (linear)
+        kb[j] = min(NB - 1, (int)fmaxf(0.f, (key_value(key[j]) - vlo) * scale));
+      else
+        kb[j] = key[j] < lo ? 0 : min(NB - 1, (int)((key[j] - lo) >> kshift));
+    }
     if (pass > 0) {
-      for (int i = tid; i < kBins; i += NT) s_hist[i] = 0u;
+      for (int i = tid; i < NB; i += NT) s_hist[i] = 0u;
       __syncthreads();
     }
 #pragma unroll
-    for (int j = 0; j < NK; ++j) {
-      const uint64_t v = (uint64_t)key[j] - lo;  // huge when key < lo
-      if ((v >> bits) == 0) atomicAdd(&s_hist[(uint32_t)v >> shift], 1u);
-    }
+    for (int j = 0; j < NK; ++j)
+      if (live >> j & 1u) atomicAdd(&s_hist[kb[j]], 1u);
     __syncthreads();
-    find_bin<NT>(s_hist, kBins, want, s_wsum, s_info);
+    find_bin<NT>(s_hist, NB, want, s_wsum, s_info);
     if (!s_info[3]) {  // fewer keys than wanted: inconsistent input, every key qualifies
       if (tid == 0) raise_flag(8u);
-      return kmin;
+      return 0u;
     }
+    const int bin = s_info[0];
     want -= (uint32_t)s_info[1];
     const uint32_t m = (uint32_t)s_info[2];
-    lo += (uint32_t)s_info[0] << shift;
-    bits = shift;
-    if (bits == 0) return lo;
+#pragma unroll
+    for (int j = 0; j < NK; ++j)
+      if (kb[j] != bin) live &= ~(1u << j);
     if (m <= 256) {
       // rank the bin's keys: the want-th largest of them (equal keys agree)
 #pragma unroll
       for (int j = 0; j < NK; ++j)
-        if ((((uint64_t)key[j] - lo) >> bits) == 0) s_list[atomicAdd(s_nlist, 1)] = key[j];
+        if (live >> j & 1u) s_list[atomicAdd(s_nlist, 1)] = key[j];
       __syncthreads();
       if (tid < (int)m) {
         const uint32_t x = s_list[tid];
@@ -369,9 +391,19 @@ __device__ uint32_t sample_threshold(const uint32_t (&key)[NK], uint32_t k, uint
       __syncthreads();
       return (uint32_t)s_info[0];
     }
-    __syncthreads();  // s_hist and s_info are reused by the next pass
+    // the next pass spreads the picked bin's keys over the whole histogram
+    uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+#pragma unroll
+    for (int j = 0; j < NK; ++j)
+      if (live >> j & 1u) {
+        mn = min(mn, key[j]);
+        mx = max(mx, key[j]);
+      }
+    block_min_max<NT>(mn, mx, s_wsum);  // (its barriers also retire s_hist and s_info)
+    lo = mn;
+    hi = mx;
   }
-  return lo;  // not reached: three passes resolve 33 bits
+  return lo;  // still more than 256 keys in play: the lowest of them (a superset threshold)
 }
 
 struct Prep {
@@ -735,6 +767,7 @@ __device__ __forceinline__ int sample_group_start(int grp, int pair, int L) {
 }
 
 constexpr int kQGroups = kThreads / 16;  // query rows loaded per pass (16 threads x 8 dims a row)
+constexpr int kSampleBins = 256;          // histogram bins of the sampled scores
 
 // Dynamic shared memory of the prep kernel.
 template <int D, int R>
@@ -743,7 +776,7 @@ struct PrepSmem {
   float m[R * D];                // M_h, row-major [R][D]
   float qpart[kQGroups][D];      // partial sums of the group's query rows
   uint32_t list[256];            // keys of the bin that holds the threshold
-  uint32_t hist[kBins];
+  uint32_t hist[kSampleBins];
   uint8_t valid[kSample];        // sampled position on a usable page
 };
 
@@ -794,7 +827,7 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
     k_el = a.store.k_new[((int64_t)b * a.h_kv + h) * D + tid];
     v_el = a.store.v_new[((int64_t)b * a.h_kv + h) * D + tid];
   }
-  for (int i = tid; i < kBins; i += kThreads) sm.hist[i] = 0u;
+  for (int i = tid; i < kSampleBins; i += kThreads) sm.hist[i] = 0u;
   if (tid == 0) s_nlist = 0;
 
   int mode = kModeScan;
@@ -977,14 +1010,14 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
       const int i = i0 + 16 * (t >> 1) + 8 * (t & 1) + g;
       // a sample on an unusable page (flagged by the scan) counts as the lowest key
       key[u / 2] = sm.valid[i] ? score_key(f) : 0u;
-      kmin = min(kmin, key[u / 2]);
+      if (key[u / 2] >= 0x00800000u) kmin = min(kmin, key[u / 2]);
       kmax = max(kmax, key[u / 2]);
     }
     block_min_max<kThreads>(kmin, kmax, s_wsum);
     sample_max = kmax;
     // the k-th largest sampled key: the tokens whose keys reach it become candidates
-    thr = sample_threshold<kThreads>(key, (uint32_t)k, kmin, kmax, sm.hist, sm.list, &s_nlist,
-                                     s_wsum, s_info);
+    thr = sample_threshold<kThreads, kSampleBins>(key, (uint32_t)k, kmin, kmax, sm.hist, sm.list,
+                                                  &s_nlist, s_wsum, s_info);
   }
   if (tid == 0) {
     *reinterpret_cast<uint32_t*>(rec + kPrepThr) = thr;
