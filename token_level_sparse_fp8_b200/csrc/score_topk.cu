@@ -467,6 +467,22 @@ __device__ __forceinline__ void load_srow(uint32_t* dst, const uint8_t* src) {
   }
 }
 
+// A lane's R / 4 code bytes of one row from shared memory (shared-window address).
+template <int R>
+__device__ __forceinline__ void lds_row(uint32_t* dst, uint32_t saddr) {
+  if (R == 32) {
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
+                 : "=r"(dst[0]), "=r"(dst[1])
+                 : "r"(saddr)
+                 : "memory");
+  } else {
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(dst[0]), "=r"(dst[1]), "=r"(dst[2]), "=r"(dst[3])
+                 : "r"(saddr)
+                 : "memory");
+  }
+}
+
 template <int R>
 __device__ __forceinline__ void load_row(uint32_t* dst, const uint8_t* src) {
   if (R == 32) {
@@ -644,6 +660,105 @@ __device__ __forceinline__ uint32_t scan_warp(const ChunkGeom& cg, const int32_t
   return run;
 }
 
+// The scan kernel's warps stream their tiles through a ring of kScanStages shared-memory stages
+// (kUnroll tiles each) filled by asynchronous 16-byte copies, kScanStages - 1 stages ahead of the
+// one being scored: deeper than a register double buffer without holding the rows in registers.
+constexpr int kScanStages = 4;
+constexpr int kScanStageBytes = 2048;  // kUnroll tiles of 16 rows of r bytes
+constexpr int kScanRingBytes = kWarps * kScanStages * kScanStageBytes;
+
+// Copies of tiles [t0, t0 + kUnroll) into the stage at shared address `dst`; returns the tiles'
+// ok bits (as scan_load). A tile past t_end or the chunk's valid tokens, or a row on an unusable
+// page, is zero-filled (its tokens are never candidates, see scan_emit).
+template <int R, bool BIG>
+__device__ __forceinline__ uint32_t scan_issue(uint32_t dst, const ChunkGeom& cg,
+                                               const int32_t* s_page, int t0, int t_end, int lane) {
+  constexpr int kU = ScanBuf<R>::kUnroll;
+  constexpr int kTileBytes = 16 * R;
+  constexpr int kPieces = kTileBytes / 512;  // 16-byte copies per lane per tile
+  static_assert(kU * kTileBytes == kScanStageBytes, "stage size");
+  const int pmask = (1 << cg.page_shift) - 1;
+  uint32_t ok = BIG ? 0u : ~0u;
+#pragma unroll
+  for (int u = 0; u < kU; ++u) {
+    const int tok0 = (t0 + u) * 16;
+    const bool live = t0 + u < t_end && tok0 < cg.n_local;
+    if (BIG) {
+      const int pg = live ? s_page[tok0 >> cg.page_shift] : -1;
+      ok |= (uint32_t)(pg >= 0) << u;
+      const uint8_t* tile = cg.head_base + (size_t)(uint32_t)max(pg, 0) * cg.page_bytes +
+                            (tok0 & pmask) * R;
+#pragma unroll
+      for (int p = 0; p < kPieces; ++p) {
+        const int o = (p * 32 + lane) * 16;
+        cp_async16(dst + u * kTileBytes + o, tile + o, pg >= 0 ? 16 : 0);
+      }
+    } else {
+#pragma unroll
+      for (int p = 0; p < kPieces; ++p) {
+        const int o = (p * 32 + lane) * 16;
+        const int tok = tok0 + o / R;
+        const int pg = live && tok < cg.n_local ? s_page[tok >> cg.page_shift] : -1;
+        const uint8_t* src = cg.head_base + (size_t)(uint32_t)max(pg, 0) * cg.page_bytes +
+                             ((tok & pmask) * R + o % R);
+        cp_async16(dst + u * kTileBytes + o, src, pg >= 0 ? 16 : 0);
+      }
+    }
+  }
+  return ok;
+}
+
+// One warp's contiguous run of tiles [t_begin, t_end) through its ring (`ring`: this warp's
+// kScanStages stages in shared memory).
+template <int R, bool BIG>
+__device__ __forceinline__ uint32_t scan_warp_ring(const ChunkGeom& cg, const int32_t* s_page,
+                                                   const DigitFrags<R>& df, float thr_f,
+                                                   int t_begin, int t_end, uint32_t* rkey,
+                                                   int32_t* rpos, uint8_t* ring, int lane) {
+  constexpr int kU = ScanBuf<R>::kUnroll;
+  constexpr int S = kScanStages;
+  constexpr uint32_t kMask = (1u << kU) - 1u;
+  constexpr int LB = R / 4;
+  static_assert(S * kU <= 32, "ok bits");
+  const int g = lane >> 2, t = lane & 3;
+  const uint32_t ring_s = smem_u32(ring);
+  const int n_batch = (t_end - t_begin + kU - 1) / kU;
+  uint32_t ok_ring = 0u;  // stage s: bits [s * kU, s * kU + kU)
+#pragma unroll
+  for (int i = 0; i < S - 1; ++i) {
+    if (i < n_batch)
+      ok_ring |= scan_issue<R, BIG>(ring_s + i * kScanStageBytes, cg, s_page, t_begin + i * kU,
+                                    t_end, lane) << (i * kU);
+    cp_async_commit();
+  }
+  uint32_t run = 0;
+  for (int i = 0; i < n_batch; ++i) {
+    const int nx = i + S - 1;
+    if (nx < n_batch) {
+      const int sx = nx % S;
+      const uint32_t okx = scan_issue<R, BIG>(ring_s + sx * kScanStageBytes, cg, s_page,
+                                              t_begin + nx * kU, t_end, lane);
+      ok_ring = (ok_ring & ~(kMask << (sx * kU))) | ((okx & kMask) << (sx * kU));
+    }
+    cp_async_commit();
+    cp_async_wait<S - 1>();
+    __syncwarp();
+    const int st = i % S;
+    const uint32_t stage = ring_s + st * kScanStageBytes;
+    ScanBuf<R> buf;
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      lds_row<R>(buf.ra[u], stage + u * 16 * R + g * R + t * LB);
+      lds_row<R>(buf.rb[u], stage + u * 16 * R + (g + 8) * R + t * LB);
+    }
+    buf.ok = BIG ? (ok_ring >> (st * kU)) & kMask : ~0u;
+    __syncwarp();  // the stage is refilled by the next iteration's copies
+    scan_emit<R, BIG>(buf, df, cg, s_page, t_begin + i * kU, t_end, thr_f, rkey, rpos, run, lane);
+  }
+  cp_async_wait<0>();
+  return run;
+}
+
 // Page list of a chunk into shared memory (bounds checked; -1 = unusable page); four loads per
 // thread in flight at a time.
 __device__ __forceinline__ void load_pages(int32_t* s_page, const int32_t* bt, int n_pages,
@@ -676,12 +791,13 @@ __device__ __forceinline__ int clamp_len(int L, int max_len) {
   return L;
 }
 
-// Scan of chunk c of pair `pair` on the CUDA cores' warp-level MMA, used by the select kernel's
-// rescan (page list already in s_page): warp q < kRegionsPerChunk takes quarter q of the chunk
-// and writes that region and its count.
-template <int R>
+// Scan of chunk c of pair `pair` on the warp-level MMA (page list already in s_page): warp
+// q < kRegionsPerChunk takes the q-th eighth of the chunk and writes that region and its count.
+// RING: the scan kernel's shared-memory tile rings (`ring`); otherwise register double buffers
+// (the select kernel's rescan).
+template <int R, bool RING>
 __device__ void scan_chunk(const ScanArgs& a, int pair, int c, int L, uint32_t thr,
-                           const DigitFrags<R>& df, const int32_t* s_page) {
+                           const DigitFrags<R>& df, const int32_t* s_page, uint8_t* ring) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (warp >= kRegionsPerChunk) return;
   const int h = pair % a.h_kv;
@@ -697,18 +813,28 @@ __device__ void scan_chunk(const ScanArgs& a, int pair, int c, int L, uint32_t t
   const int tpw = seg / 16;
   const int t_begin = min(n_tiles, warp * tpw), t_end = min(n_tiles, t_begin + tpw);
   const float thr_f = key_floor(thr);
-  const uint32_t n =
-      cg.page_shift >= 4
-          ? scan_warp<R, true>(cg, s_page, df, thr_f, t_begin, t_end, a.cands.key + reg * seg,
-                               a.cands.pos + reg * seg, lane)
-          : scan_warp<R, false>(cg, s_page, df, thr_f, t_begin, t_end, a.cands.key + reg * seg,
-                                a.cands.pos + reg * seg, lane);
+  uint32_t n;
+  if (RING) {
+    uint8_t* wr = ring + warp * kScanStages * kScanStageBytes;
+    n = cg.page_shift >= 4
+            ? scan_warp_ring<R, true>(cg, s_page, df, thr_f, t_begin, t_end,
+                                      a.cands.key + reg * seg, a.cands.pos + reg * seg, wr, lane)
+            : scan_warp_ring<R, false>(cg, s_page, df, thr_f, t_begin, t_end,
+                                       a.cands.key + reg * seg, a.cands.pos + reg * seg, wr, lane);
+  } else {
+    n = cg.page_shift >= 4
+            ? scan_warp<R, true>(cg, s_page, df, thr_f, t_begin, t_end, a.cands.key + reg * seg,
+                                 a.cands.pos + reg * seg, lane)
+            : scan_warp<R, false>(cg, s_page, df, thr_f, t_begin, t_end, a.cands.key + reg * seg,
+                                  a.cands.pos + reg * seg, lane);
+  }
   if (lane == 0) a.cands.cnt[reg] = n;
 }
 
 template <int D, int R>
 __global__ void __launch_bounds__(kThreads, 3) scan_kernel(ScanArgs a) {
-  extern __shared__ int32_t scan_pages[];  // chunk / page_size + 1 entries
+  extern __shared__ __align__(16) uint8_t scan_dyn[];  // tile ring, then the page list
+  int32_t* scan_pages = reinterpret_cast<int32_t*>(scan_dyn + kScanRingBytes);
   const int c = blockIdx.x, pair = blockIdx.y;
   const int b = pair / a.h_kv;
   const int L = clamp_len(a.seq_lens[b], a.max_pages << a.page_shift);
@@ -731,7 +857,7 @@ __global__ void __launch_bounds__(kThreads, 3) scan_kernel(ScanArgs a) {
   df.load(reinterpret_cast<const uint16_t*>(rec), reinterpret_cast<const float*>(rec + kPrepScale),
           threadIdx.x & 31);
   const uint32_t thr = *reinterpret_cast<const uint32_t*>(rec + kPrepThr);
-  scan_chunk<R>(a, pair, c, L, thr, df, scan_pages);
+  scan_chunk<R, true>(a, pair, c, L, thr, df, scan_pages, scan_dyn);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -1124,7 +1250,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
       load_pages(s_page, a.block_table + (int64_t)b * a.max_pages + (start >> a.page_shift),
                  n_pages, a.num_pages);
       __syncthreads();
-      scan_chunk<R>(a, pair, c, L, 0u, df, s_page);
+      scan_chunk<R, false>(a, pair, c, L, 0u, df, s_page, nullptr);
     }
     __syncthreads();
     offsets();
@@ -1299,7 +1425,8 @@ cudaError_t launch_t(const ScorePlan& plan, int pairs, const PrepArgs& pa, const
       e = launch_k(prep_kernel<D, R, false>, dim3(pairs), kThreads, prep_smem, pdl, s, pa);
   }
   if (e != cudaSuccess) return e;
-  const size_t scan_smem = (size_t)(plan.chunk / (1 << sa.page_shift) + 1) * 4;
+  const size_t scan_smem =
+      (size_t)kScanRingBytes + (size_t)(plan.chunk / (1 << sa.page_shift) + 1) * 4;
   e = configure_kernel((const void*)scan_kernel<D, R>, (int)scan_smem, false);
   if (e != cudaSuccess) return e;
   e = launch_k(scan_kernel<D, R>, dim3(plan.n_chunks, pairs), kThreads, scan_smem, true, s, sa);
