@@ -660,12 +660,17 @@ __device__ __forceinline__ uint32_t scan_warp(const ChunkGeom& cg, const int32_t
   return run;
 }
 
-// The scan kernel's warps stream their tiles through a ring of kScanStages shared-memory stages
-// (kUnroll tiles each) filled by asynchronous 16-byte copies, kScanStages - 1 stages ahead of the
-// one being scored: deeper than a register double buffer without holding the rows in registers.
-constexpr int kScanStages = 4;
+// The scan kernel's warps stream their tiles through a ring of scan_stages<R>() shared-memory
+// stages (kUnroll tiles each) filled by asynchronous 16-byte copies, all but one stage ahead of
+// the one being scored: deeper than a register double buffer without holding the rows in
+// registers. At r = 32, three stages and four CTAs per SM; at r = 64, four stages and three.
 constexpr int kScanStageBytes = 2048;  // kUnroll tiles of 16 rows of r bytes
-constexpr int kScanRingBytes = kWarps * kScanStages * kScanStageBytes;
+template <int R>
+constexpr int scan_stages() { return R == 32 ? 3 : 4; }
+template <int R>
+constexpr int scan_ctas_per_sm() { return R == 32 ? 4 : 3; }
+template <int R>
+constexpr int scan_ring_bytes() { return kWarps * scan_stages<R>() * kScanStageBytes; }
 
 // Copies of tiles [t0, t0 + kUnroll) into the stage at shared address `dst`; returns the tiles'
 // ok bits (as scan_load). A tile past t_end or the chunk's valid tokens, or a row on an unusable
@@ -709,14 +714,14 @@ __device__ __forceinline__ uint32_t scan_issue(uint32_t dst, const ChunkGeom& cg
 }
 
 // One warp's contiguous run of tiles [t_begin, t_end) through its ring (`ring`: this warp's
-// kScanStages stages in shared memory).
+// scan_stages<R>() stages in shared memory).
 template <int R, bool BIG>
 __device__ __forceinline__ uint32_t scan_warp_ring(const ChunkGeom& cg, const int32_t* s_page,
                                                    const DigitFrags<R>& df, float thr_f,
                                                    int t_begin, int t_end, uint32_t* rkey,
                                                    int32_t* rpos, uint8_t* ring, int lane) {
   constexpr int kU = ScanBuf<R>::kUnroll;
-  constexpr int S = kScanStages;
+  constexpr int S = scan_stages<R>();
   constexpr uint32_t kMask = (1u << kU) - 1u;
   constexpr int LB = R / 4;
   static_assert(S * kU <= 32, "ok bits");
@@ -815,7 +820,7 @@ __device__ void scan_chunk(const ScanArgs& a, int pair, int c, int L, uint32_t t
   const float thr_f = key_floor(thr);
   uint32_t n;
   if (RING) {
-    uint8_t* wr = ring + warp * kScanStages * kScanStageBytes;
+    uint8_t* wr = ring + warp * scan_stages<R>() * kScanStageBytes;
     n = cg.page_shift >= 4
             ? scan_warp_ring<R, true>(cg, s_page, df, thr_f, t_begin, t_end,
                                       a.cands.key + reg * seg, a.cands.pos + reg * seg, wr, lane)
@@ -832,9 +837,9 @@ __device__ void scan_chunk(const ScanArgs& a, int pair, int c, int L, uint32_t t
 }
 
 template <int D, int R>
-__global__ void __launch_bounds__(kThreads, 3) scan_kernel(ScanArgs a) {
+__global__ void __launch_bounds__(kThreads, scan_ctas_per_sm<R>()) scan_kernel(ScanArgs a) {
   extern __shared__ __align__(16) uint8_t scan_dyn[];  // tile ring, then the page list
-  int32_t* scan_pages = reinterpret_cast<int32_t*>(scan_dyn + kScanRingBytes);
+  int32_t* scan_pages = reinterpret_cast<int32_t*>(scan_dyn + scan_ring_bytes<R>());
   const int c = blockIdx.x, pair = blockIdx.y;
   const int b = pair / a.h_kv;
   const int L = clamp_len(a.seq_lens[b], a.max_pages << a.page_shift);
@@ -1426,7 +1431,7 @@ cudaError_t launch_t(const ScorePlan& plan, int pairs, const PrepArgs& pa, const
   }
   if (e != cudaSuccess) return e;
   const size_t scan_smem =
-      (size_t)kScanRingBytes + (size_t)(plan.chunk / (1 << sa.page_shift) + 1) * 4;
+      (size_t)scan_ring_bytes<R>() + (size_t)(plan.chunk / (1 << sa.page_shift) + 1) * 4;
   e = configure_kernel((const void*)scan_kernel<D, R>, (int)scan_smem, false);
   if (e != cudaSuccess) return e;
   e = launch_k(scan_kernel<D, R>, dim3(plan.n_chunks, pairs), kThreads, scan_smem, true, s, sa);
