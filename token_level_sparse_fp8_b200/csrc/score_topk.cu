@@ -265,21 +265,21 @@ __device__ void select_threshold(KeyAt key_at, int n, uint32_t want, uint32_t km
 }
 
 // Exact threshold (contract of radix_select) from a histogram of the n keys built beforehand
-// with bin(key) = min(2047, (key - base) >> shift), every key >= base: the bin of the want-th
+// with bin(key) = min(NB - 1, (key - base) >> shift), every key >= base: the bin of the want-th
 // largest key, taken whole or resolved by ranking its keys (at most 256) against each other.
 // Returns false, leaving thr / take unset, when that bin is the top one (it also holds every key
 // above the range) or holds more keys: the caller then runs a general selection.
-template <int NT, typename KeyAt>
+template <int NT, int NB, typename KeyAt>
 __device__ bool threshold_from_hist(KeyAt key_at, int n, uint32_t want, uint32_t base, int shift,
                                     uint32_t* s_hist, uint32_t* s_wsum, int* s_info, int64_t& thr,
                                     uint32_t& take) {
   const int tid = threadIdx.x;
-  find_bin<NT>(s_hist, kBins, want, s_wsum, s_info);
+  find_bin<NT>(s_hist, NB, want, s_wsum, s_info);
   const bool found = s_info[3] != 0;
   const uint32_t bin = (uint32_t)s_info[0], m = (uint32_t)s_info[2];
   const uint32_t w2 = want - (uint32_t)s_info[1];
   __syncthreads();  // s_info and s_hist are reused below
-  if (!found || bin == kBins - 1 || (w2 != m && m > 256)) return false;
+  if (!found || bin == NB - 1 || (w2 != m && m > 256)) return false;
   if (w2 == m) {
     thr = (int64_t)base + ((int64_t)bin << shift) - 1;
     take = 0;
@@ -1169,6 +1169,138 @@ struct SelectArgs {
 
 constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kSelBinBits = 9;  // histogram of the staged candidate keys: 512 bins
+constexpr int kSelBins = 1 << kSelBinBits;
+
+constexpr int kSelRun = 12;  // candidates per lane on the register path
+
+// Selection for one (sequence, KV head) with the candidates (flattened position order) held in
+// registers, read straight from the regions: warp w owns a contiguous span of 32 kSelRun
+// candidates at most, lane l the candidates span + 32 u + l (coalesced loads). Histogram of the
+// keys over [base, ...) in kSelBins bins of 2^hshift keys (the top bin also takes every larger
+// key), the bin of the want-th largest key, the exact key by ranking that bin's keys against
+// each other, then the ordered emission (keys > thr and the first `take` keys == thr, each at
+// slot (keys > thr before it) + min(keys == thr before it, take)). Returns false, having written
+// nothing, when that bin is the top one or holds more than 256 keys. s_hist is zero on entry;
+// s_list holds 256 keys; s_wsum 2 kSelWarps words.
+template <typename RegionOf>
+__device__ bool select_in_registers(const SelectArgs& s, int pair, int n_reg, int seg,
+                                    uint32_t want, uint32_t base, int hshift, RegionOf region_of,
+                                    const uint32_t* s_roff, uint32_t* s_hist, uint32_t* s_list,
+                                    uint32_t* s_wsum, int* s_info) {
+  const ScanArgs& a = s.scan;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int budget = a.budget;
+  const int n = (int)s_roff[n_reg];
+  const uint32_t* ck = a.cands.key + (int64_t)pair * n_reg * seg;
+  const int32_t* cp = a.cands.pos + (int64_t)pair * n_reg * seg;
+  const int span = ((n + kSelWarps - 1) / kSelWarps + 31) & ~31;  // <= 32 kSelRun
+  const int lo = min(n, warp * span), hi = min(n, lo + span);
+  uint32_t key[kSelRun];
+  int32_t pos[kSelRun];
+  int r = lo + lane < hi ? region_of(lo + lane) : 0;
+#pragma unroll
+  for (int u = 0; u < kSelRun; ++u) {
+    const int j = lo + 32 * u + lane;
+    key[u] = 0u;
+    pos[u] = 0;
+    if (j < hi) {
+      while (s_roff[r + 1] <= (uint32_t)j) ++r;
+      const int64_t src = (int64_t)r * seg + (j - (int)s_roff[r]);
+      key[u] = ck[src];
+      pos[u] = cp[src];
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kSelRun; ++u)
+    if (lo + 32 * u + lane < hi)
+      atomicAdd(&s_hist[min((uint32_t)kSelBins - 1u, (key[u] - base) >> hshift)], 1u);
+  __syncthreads();
+  find_bin<kSelThreads>(s_hist, kSelBins, want, s_wsum, s_info);
+  const bool found = s_info[3] != 0;
+  const uint32_t bin = (uint32_t)s_info[0], m = (uint32_t)s_info[2];
+  const uint32_t w2 = want - (uint32_t)s_info[1];
+  __syncthreads();  // s_info and s_wsum are rewritten below
+  if (!found || bin == kSelBins - 1 || (w2 != m && m > 256)) return false;
+  int64_t thr;
+  uint32_t take;
+  if (w2 == m) {  // the whole bin: every key from its lowest one
+    thr = (int64_t)base + ((int64_t)bin << hshift) - 1;
+    take = 0;
+  } else {
+    if (tid == 0) s_info[3] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kSelRun; ++u)
+      if (lo + 32 * u + lane < hi && ((key[u] - base) >> hshift) == bin)
+        s_list[atomicAdd(&s_info[3], 1)] = key[u];
+    __syncthreads();
+    if (tid < (int)m) {
+      const uint32_t x = s_list[tid];
+      uint32_t gt = 0, eq = 0;
+      for (uint32_t i = 0; i < m; ++i) {
+        const uint32_t y = s_list[i];
+        gt += y > x;
+        eq += y == x;
+      }
+      if (gt < w2 && w2 <= gt + eq) {  // x is the w2-th largest of the bin (equal keys agree)
+        s_info[0] = (int)x;
+        s_info[1] = (int)(w2 - gt);
+      }
+    }
+    __syncthreads();
+    thr = (int64_t)(uint32_t)s_info[0];
+    take = (uint32_t)s_info[1];
+  }
+  // per-warp counts, then each warp's offsets from the warps before it
+  unsigned gtm[kSelRun], eqm[kSelRun];
+  uint32_t n_gt = 0, n_eq = 0;
+#pragma unroll
+  for (int u = 0; u < kSelRun; ++u) {
+    const bool in = lo + 32 * u + lane < hi;
+    gtm[u] = __ballot_sync(0xffffffffu, in && (int64_t)key[u] > thr);
+    eqm[u] = __ballot_sync(0xffffffffu, in && (int64_t)key[u] == thr);
+    n_gt += __popc(gtm[u]);
+    n_eq += __popc(eqm[u]);
+  }
+  if (lane == 0) {
+    s_wsum[warp] = n_gt;
+    s_wsum[kSelWarps + warp] = n_eq;
+  }
+  __syncthreads();
+  uint32_t gt_b = 0, eq_b = 0, total_gt = 0, total_eq = 0;
+#pragma unroll
+  for (int w = 0; w < kSelWarps; ++w) {
+    const uint32_t g_ = s_wsum[w], e_ = s_wsum[kSelWarps + w];
+    gt_b += w < warp ? g_ : 0u;
+    eq_b += w < warp ? e_ : 0u;
+    total_gt += g_;
+    total_eq += e_;
+  }
+  const unsigned lt = (1u << lane) - 1u;
+  int32_t* out_idx = s.idx + (int64_t)pair * budget;
+#pragma unroll
+  for (int u = 0; u < kSelRun; ++u) {
+    const uint32_t g_before = gt_b + __popc(gtm[u] & lt), e_before = eq_b + __popc(eqm[u] & lt);
+    if ((gtm[u] >> lane) & 1u) {
+      const uint32_t at = g_before + min(e_before, take);
+      if (at < (uint32_t)budget) out_idx[at] = pos[u];
+    } else if (((eqm[u] >> lane) & 1u) && e_before < take && g_before + e_before < (uint32_t)budget) {
+      out_idx[g_before + e_before] = pos[u];
+    }
+    gt_b += __popc(gtm[u]);
+    eq_b += __popc(eqm[u]);
+  }
+  const uint32_t written = total_gt + min(total_eq, take);
+  for (int j = (int)want + tid; j < budget; j += kSelThreads) out_idx[j] = -1;
+  if (tid == 0) {
+    if (written != want) raise_flag(8u);
+    s.count[pair] = (int)want;
+    // the attention launched next merges its splits through these counters
+    if (a.cands.attend_tickets) a.cands.attend_tickets[pair] = 0;
+  }
+  return true;
+}
 
 template <int D, int R>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
@@ -1211,8 +1343,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
   const uint32_t base = *reinterpret_cast<const uint32_t*>(rec + kPrepThr);
   const uint32_t sample_max = *reinterpret_cast<const uint32_t*>(rec + kPrepKmax);
   bool use_hist = base > 0u && sample_max > base;
-  const int hshift = use_hist ? max(0, (32 - __clz(sample_max - base)) - 11) : 0;
-  for (int i = tid; i < kBins; i += kSelThreads) s_hist[i] = 0u;
+  const int hshift = use_hist ? max(0, (32 - __clz(sample_max - base)) - kSelBinBits) : 0;
+  for (int i = tid; i < kSelBins; i += kSelThreads) s_hist[i] = 0u;
 
   // region offsets: exclusive prefix of the counts, in position order (each thread loads and
   // sums a run of adjacent regions, then a block-wide scan)
@@ -1238,6 +1370,22 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
     __syncthreads();
   };
   offsets();
+  // flattened candidate j -> region (the last r with s_roff[r] <= j)
+  auto region_of = [&](int j) {
+    int lo = 0, hi = n_reg - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_roff[mid] <= (uint32_t)j) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+  };
+  if (use_hist && s_roff[n_reg] >= want && s_roff[n_reg] <= (uint32_t)(kSelThreads * kSelRun)) {
+    if (select_in_registers(s, pair, n_reg, seg, want, base, hshift, region_of, s_roff, s_hist,
+                            s_ckey, s_wsum, s_info))
+      return;
+    for (int i = tid; i < kSelBins; i += kSelThreads) s_hist[i] = 0u;  // (general path below)
+    __syncthreads();
+  }
   if (s_roff[n_reg] < want) {
     // rescue: the sampled threshold was too high; score every token of the sequence again with
     // no threshold (all keys become candidates), then select exactly as usual
@@ -1262,15 +1410,6 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
   }
   const uint32_t n = s_roff[n_reg];
   const bool staged = n <= (uint32_t)kSelectCap;
-  // flattened candidate j -> region (the last r with s_roff[r] <= j)
-  auto region_of = [&](int j) {
-    int lo = 0, hi = n_reg - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s_roff[mid] <= (uint32_t)j) lo = mid; else hi = mid - 1;
-    }
-    return lo;
-  };
   auto src_of = [&](int j) -> int64_t {
     const int r = region_of(j);
     return (int64_t)r * seg + (j - (int)s_roff[r]);
@@ -1279,10 +1418,17 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
   if (staged) {
     // flatten the regions (keys and positions, position order) into shared memory: each warp
     // copies 8 regions at a time, the first 64 candidates of each with all loads issued before
-    // any store (one round trip), the rare rest of a longer region afterwards; key range on
-    // the way
+    // any store (one round trip), the rare rest of a longer region afterwards; key range and
+    // histogram on the way
+    auto put = [&](uint32_t at, uint32_t key, int32_t pos) {
+      s_ckey[at] = key;
+      s_cpos[at] = pos;
+      kmin = min(kmin, key);
+      kmax = max(kmax, key);
+      if (use_hist) atomicAdd(&s_hist[min((uint32_t)kSelBins - 1u, (key - base) >> hshift)], 1u);
+    };
     constexpr int kRB = 8;
-    for (int rb = (threadIdx.x >> 5) * kRB; rb < n_reg; rb += kSelWarps * kRB) {
+    for (int rb = (tid >> 5) * kRB; rb < n_reg; rb += kSelWarps * kRB) {
       uint32_t kk[kRB][2];
       int32_t pp[kRB][2];
 #pragma unroll
@@ -1304,22 +1450,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const uint32_t i = lane + 32 * e;
-          if (i < cnt) {
-            s_ckey[off + i] = kk[u][e];
-            s_cpos[off + i] = pp[u][e];
-            kmin = min(kmin, kk[u][e]);
-            kmax = max(kmax, kk[u][e]);
-            if (use_hist) atomicAdd(&s_hist[min(kBins - 1u, (kk[u][e] - base) >> hshift)], 1u);
-          }
+          if (i < cnt) put(off + i, kk[u][e], pp[u][e]);
         }
-        for (uint32_t i = 64 + lane; i < cnt; i += 32) {
-          const uint32_t key = ck[(int64_t)r * seg + i];
-          s_ckey[off + i] = key;
-          s_cpos[off + i] = cp[(int64_t)r * seg + i];
-          kmin = min(kmin, key);
-          kmax = max(kmax, key);
-          if (use_hist) atomicAdd(&s_hist[min(kBins - 1u, (key - base) >> hshift)], 1u);
-        }
+        for (uint32_t i = 64 + lane; i < cnt; i += 32)
+          put(off + i, ck[(int64_t)r * seg + i], cp[(int64_t)r * seg + i]);
       }
     }
   } else {
@@ -1335,57 +1469,63 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
   int64_t thr;
   uint32_t take;
   const bool done = use_hist && staged &&
-                    threshold_from_hist<kSelThreads>(key_at, (int)n, want, base, hshift, s_hist,
-                                                     s_wsum, s_info, thr, take);
+                    threshold_from_hist<kSelThreads, kSelBins>(key_at, (int)n, want, base, hshift,
+                                                               s_hist, s_wsum, s_info, thr, take);
   if (!done) {
     block_min_max<kSelThreads>(kmin, kmax, s_wsum);
     select_threshold<kSelThreads>(key_at, (int)n, want, kmin, kmax, s_hist, s_wsum, s_info, thr,
                                   take);
   }
   // ordered emission: the selected candidates are the keys > thr and the first `take` keys == thr
-  // in position order, written in candidate (= position) order at slot
-  // (keys > thr before it) + min(keys == thr before it, take). Warp w owns a contiguous span of
-  // candidates, read 32 at a time (consecutive lanes, consecutive words: no bank conflicts); the
-  // spans' counts are combined across warps in shared memory.
-  const unsigned lt = (1u << lane) - 1u;
-  const int warp_id = tid >> 5;
-  const int span = (((int)n + kSelWarps - 1) / kSelWarps + 31) & ~31;
-  const int lo = min((int)n, warp_id * span), hi = min((int)n, lo + span);
+  // in position order; candidate j goes to slot (keys > thr before it) + min(keys == thr before
+  // it, take). Thread i owns the contiguous run [i q, i q + q) of candidates (q a multiple of 4:
+  // 16-byte shared loads when staged); one block-wide scan of its two counts gives its offsets.
+  const int q = (((int)n + kSelThreads - 1) / kSelThreads + 3) & ~3;
+  const int lo = min((int)n, tid * q), hi = min((int)n, lo + q);
   uint32_t n_gt = 0, n_eq = 0;
-  for (int i0 = lo; i0 < hi; i0 += 32) {
-    const int i = i0 + lane;
-    const int64_t key = i < hi ? (int64_t)key_at(i) : -1;
-    n_gt += __popc(__ballot_sync(0xffffffffu, key > thr));
-    n_eq += __popc(__ballot_sync(0xffffffffu, key == thr));
-  }
-  if (lane == 0) {
-    s_wsum[warp_id] = n_gt;
-    s_wsum[kSelWarps + warp_id] = n_eq;
-  }
-  __syncthreads();
-  uint32_t gt_b = 0, eq_b = 0, total_gt = 0, total_eq = 0;
-  for (int w = 0; w < kSelWarps; ++w) {
-    const uint32_t a_ = s_wsum[w], e_ = s_wsum[kSelWarps + w];
-    if (w < warp_id) {
-      gt_b += a_;
-      eq_b += e_;
+  if (staged) {
+    for (int j0 = lo; j0 < hi; j0 += 4) {
+      const uint4 k4 = *reinterpret_cast<const uint4*>(s_ckey + j0);
+      const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool in = j0 + e < hi;
+        n_gt += in && (int64_t)kv[e] > thr;
+        n_eq += in && (int64_t)kv[e] == thr;
+      }
     }
-    total_gt += a_;
-    total_eq += e_;
-  }
-  for (int i0 = lo; i0 < hi; i0 += 32) {
-    const int i = i0 + lane;
-    const int64_t key = i < hi ? (int64_t)key_at(i) : -1;
-    const bool is_gt = key > thr, is_eq = key == thr;
-    const unsigned gtm = __ballot_sync(0xffffffffu, is_gt);
-    const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
-    const uint32_t g_before = gt_b + __popc(gtm & lt), e_before = eq_b + __popc(eqm & lt);
-    if (is_gt || (is_eq && e_before < take)) {
-      const uint32_t at = g_before + min(e_before, take);
-      if (at < (uint32_t)budget) out_idx[at] = pos_at(i);
+  } else {
+    for (int j = lo; j < hi; ++j) {
+      const int64_t key = key_at(j);
+      n_gt += key > thr;
+      n_eq += key == thr;
     }
-    gt_b += __popc(gtm);
-    eq_b += __popc(eqm);
+  }
+  uint64_t totals;
+  const uint64_t before =
+      block_excl_scan64<kSelThreads>(((uint64_t)n_gt << 32) | n_eq, totals, s_red64);
+  const uint32_t total_gt = (uint32_t)(totals >> 32), total_eq = (uint32_t)totals;
+  uint32_t gt_b = (uint32_t)(before >> 32), eq_b = (uint32_t)before;
+  auto emit = [&](int64_t key, int j) {
+    if (key > thr) {
+      const uint32_t at = gt_b + min(eq_b, take);
+      if (at < (uint32_t)budget) out_idx[at] = pos_at(j);
+      ++gt_b;
+    } else if (key == thr) {
+      if (eq_b < take && gt_b + eq_b < (uint32_t)budget) out_idx[gt_b + eq_b] = pos_at(j);
+      ++eq_b;
+    }
+  };
+  if (staged) {
+    for (int j0 = lo; j0 < hi; j0 += 4) {
+      const uint4 k4 = *reinterpret_cast<const uint4*>(s_ckey + j0);
+      const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (j0 + e < hi) emit((int64_t)kv[e], j0 + e);
+    }
+  } else {
+    for (int j = lo; j < hi; ++j) emit((int64_t)key_at(j), j);
   }
   const uint32_t written = total_gt + min(total_eq, take);
   for (int j = (int)want + tid; j < budget; j += kSelThreads) out_idx[j] = -1;
