@@ -1172,25 +1172,209 @@ constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelBinBits = 9;  // histogram of the staged candidate keys: 512 bins
 constexpr int kSelBins = 1 << kSelBinBits;
 
-constexpr int kSelRun = 12;  // candidates per lane on the register path
+constexpr int kSelRun = 12;         // candidates per lane on the flattened register path
+constexpr int kSelRegsPerWarp = 8;  // regions per warp on the region-major register path
+constexpr int kSelPerRegion = 64;   // entries per region held in registers (two per lane)
 
-// Selection for one (sequence, KV head) with the candidates (flattened position order) held in
-// registers, read straight from the regions: warp w owns a contiguous span of 32 kSelRun
-// candidates at most, lane l the candidates span + 32 u + l (coalesced loads). Histogram of the
-// keys over [base, ...) in kSelBins bins of 2^hshift keys (the top bin also takes every larger
-// key), the bin of the want-th largest key, the exact key by ranking that bin's keys against
-// each other, then the ordered emission (keys > thr and the first `take` keys == thr, each at
-// slot (keys > thr before it) + min(keys == thr before it, take)). Returns false, having written
-// nothing, when that bin is the top one or holds more than 256 keys. s_hist is zero on entry;
-// s_list holds 256 keys; s_wsum 2 kSelWarps words.
+// Threshold of the want largest candidate keys held in registers (each(f) calls f(key) for
+// every key this thread holds), every key >= base: a histogram in kSelBins bins of 2^hshift
+// keys (the top bin also takes every larger key), the bin of the want-th largest key, then the
+// exact key by ranking that bin's keys against each other. On return the want largest keys are
+// the keys > thr plus the first `take` keys == thr. Returns false when that bin is the top one
+// or holds more than 256 keys. s_hist is zero on entry; s_list holds 256 keys.
+template <typename EachKey>
+__device__ bool threshold_in_registers(EachKey each, uint32_t want, uint32_t base, int hshift,
+                                       uint32_t* s_hist, uint32_t* s_list, uint32_t* s_wsum,
+                                       int* s_info, int64_t& thr, uint32_t& take) {
+  const int tid = threadIdx.x;
+  each([&](uint32_t k) {
+    atomicAdd(&s_hist[min((uint32_t)kSelBins - 1u, (k - base) >> hshift)], 1u);
+  });
+  __syncthreads();
+  find_bin<kSelThreads>(s_hist, kSelBins, want, s_wsum, s_info);
+  const bool found = s_info[3] != 0;
+  const uint32_t bin = (uint32_t)s_info[0], m = (uint32_t)s_info[2];
+  const uint32_t w2 = want - (uint32_t)s_info[1];
+  __syncthreads();  // s_info and s_wsum are rewritten below
+  if (!found || bin == kSelBins - 1 || (w2 != m && m > 256)) return false;
+  if (w2 == m) {  // the whole bin: every key from its lowest one
+    thr = (int64_t)base + ((int64_t)bin << hshift) - 1;
+    take = 0;
+    return true;
+  }
+  if (tid == 0) s_info[3] = 0;
+  __syncthreads();
+  each([&](uint32_t k) {
+    if (((k - base) >> hshift) == bin) s_list[atomicAdd(&s_info[3], 1)] = k;
+  });
+  __syncthreads();
+  if (tid < (int)m) {
+    const uint32_t x = s_list[tid];
+    uint32_t gt = 0, eq = 0;
+    for (uint32_t i = 0; i < m; ++i) {
+      const uint32_t y = s_list[i];
+      gt += y > x;
+      eq += y == x;
+    }
+    if (gt < w2 && w2 <= gt + eq) {  // x is the w2-th largest of the bin (equal keys agree)
+      s_info[0] = (int)x;
+      s_info[1] = (int)(w2 - gt);
+    }
+  }
+  __syncthreads();
+  thr = (int64_t)(uint32_t)s_info[0];
+  take = (uint32_t)s_info[1];
+  return true;
+}
+
+// Warp offsets of the ordered emission: this warp's selected keys come after gt_b keys > thr
+// and eq_b keys == thr of the warps before it (s_cnt: 2 kSelWarps words).
+__device__ __forceinline__ void warp_offsets(uint32_t n_gt, uint32_t n_eq, uint32_t* s_cnt,
+                                             uint32_t& gt_b, uint32_t& eq_b, uint32_t& total_gt,
+                                             uint32_t& total_eq) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) {
+    s_cnt[warp] = n_gt;
+    s_cnt[kSelWarps + warp] = n_eq;
+  }
+  __syncthreads();
+  gt_b = eq_b = total_gt = total_eq = 0u;
+#pragma unroll
+  for (int w = 0; w < kSelWarps; ++w) {
+    const uint32_t g_ = s_cnt[w], e_ = s_cnt[kSelWarps + w];
+    gt_b += w < warp ? g_ : 0u;
+    eq_b += w < warp ? e_ : 0u;
+    total_gt += g_;
+    total_eq += e_;
+  }
+}
+
+// One ballot group of the ordered emission (32 consecutive candidates, lane order = position
+// order): keys > thr, and keys == thr while fewer than `take` came before, go to slot
+// (keys > thr before) + min(keys == thr before, take).
+__device__ __forceinline__ void emit_group(bool in, int64_t key, int32_t pos, int64_t thr,
+                                           uint32_t take, int budget, int32_t* out_idx,
+                                           uint32_t& gt_b, uint32_t& eq_b) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  const bool is_gt = in && key > thr, is_eq = in && key == thr;
+  const unsigned gtm = __ballot_sync(0xffffffffu, is_gt);
+  const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
+  const uint32_t g_before = gt_b + __popc(gtm & lt), e_before = eq_b + __popc(eqm & lt);
+  if (is_gt || (is_eq && e_before < take)) {
+    const uint32_t at = g_before + min(e_before, take);
+    if (at < (uint32_t)budget) out_idx[at] = pos;
+  }
+  gt_b += __popc(gtm);
+  eq_b += __popc(eqm);
+}
+
+__device__ __forceinline__ void select_finish(const SelectArgs& s, int pair, uint32_t want,
+                                              uint32_t written, int32_t* out_idx) {
+  const int tid = threadIdx.x;
+  for (int j = (int)want + tid; j < s.scan.budget; j += kSelThreads) out_idx[j] = -1;
+  if (tid == 0) {
+    if (written != want) raise_flag(8u);
+    s.count[pair] = (int)want;
+    // the attention launched next merges its splits through these counters
+    if (s.scan.cands.attend_tickets) s.scan.cands.attend_tickets[pair] = 0;
+  }
+}
+
+// Region-major register path (at most kSelWarps * kSelRegsPerWarp regions): warp w holds
+// regions [w kSelRegsPerWarp, (w + 1) kSelRegsPerWarp), lane l entries l and l + 32 of each,
+// loaded together with the region counts (one round trip, no offsets needed: the warp's
+// candidates are in position order). Returns false, having written nothing, when a region holds
+// more than kSelPerRegion candidates, there are fewer candidates than wanted, or the threshold
+// bin cannot be resolved (s_hist is then dirty).
+__device__ bool select_region_major(const SelectArgs& s, int pair, int n_reg, int seg,
+                                    uint32_t want, uint32_t base, int hshift, uint32_t* s_hist,
+                                    uint32_t* s_list, uint32_t* s_wsum, uint32_t* s_cnt,
+                                    int* s_info) {
+  constexpr int RW = kSelRegsPerWarp, E = kSelPerRegion / 32;
+  const ScanArgs& a = s.scan;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t* ck = a.cands.key + (int64_t)pair * n_reg * seg;
+  const int32_t* cp = a.cands.pos + (int64_t)pair * n_reg * seg;
+  const uint32_t* cc = a.cands.cnt + (int64_t)pair * n_reg;
+  uint32_t cnt[RW], key[RW][E];
+  int32_t pos[RW][E];
+#pragma unroll
+  for (int u = 0; u < RW; ++u) {
+    const int r = warp * RW + u;
+    cnt[u] = r < n_reg ? cc[r] : 0u;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      key[u][e] = r < n_reg ? ck[(int64_t)r * seg + lane + 32 * e] : 0u;
+      pos[u][e] = r < n_reg ? cp[(int64_t)r * seg + lane + 32 * e] : 0;
+    }
+  }
+  uint32_t wn = 0, over = 0;
+#pragma unroll
+  for (int u = 0; u < RW; ++u) {
+    wn += cnt[u];
+    over |= cnt[u] > (uint32_t)kSelPerRegion;
+  }
+  if (lane == 0) {
+    s_cnt[warp] = wn;
+    s_cnt[kSelWarps + warp] = over;
+  }
+  __syncthreads();
+  uint32_t n = 0;
+  over = 0;
+#pragma unroll
+  for (int w = 0; w < kSelWarps; ++w) {
+    n += s_cnt[w];
+    over |= s_cnt[kSelWarps + w];
+  }
+  __syncthreads();  // s_cnt is rewritten below
+  if (over || n < want) return false;
+  auto each = [&](auto&& f) {
+#pragma unroll
+    for (int u = 0; u < RW; ++u)
+#pragma unroll
+      for (int e = 0; e < E; ++e)
+        if ((uint32_t)(lane + 32 * e) < cnt[u]) f(key[u][e]);
+  };
+  int64_t thr;
+  uint32_t take;
+  if (!threshold_in_registers(each, want, base, hshift, s_hist, s_list, s_wsum, s_info, thr, take))
+    return false;
+  uint32_t n_gt = 0, n_eq = 0;
+  each([&](uint32_t k) {
+    n_gt += (int64_t)k > thr;
+    n_eq += (int64_t)k == thr;
+  });
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    n_gt += __shfl_xor_sync(0xffffffffu, n_gt, o);
+    n_eq += __shfl_xor_sync(0xffffffffu, n_eq, o);
+  }
+  uint32_t gt_b, eq_b, total_gt, total_eq;
+  warp_offsets(n_gt, n_eq, s_cnt, gt_b, eq_b, total_gt, total_eq);
+  int32_t* out_idx = s.idx + (int64_t)pair * a.budget;
+#pragma unroll
+  for (int u = 0; u < RW; ++u)
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+      if (32 * e < (int)cnt[u])  // (warp-uniform)
+        emit_group((uint32_t)(lane + 32 * e) < cnt[u], key[u][e], pos[u][e], thr, take, a.budget,
+                   out_idx, gt_b, eq_b);
+  select_finish(s, pair, want, total_gt + min(total_eq, take), out_idx);
+  return true;
+}
+
+// Flattened register path (at most kSelThreads * kSelRun candidates, any region count, offsets
+// s_roff known): warp w owns a contiguous span of 32 kSelRun candidates at most, lane l the
+// candidates span + 32 u + l (coalesced loads straight from the regions). Returns false, having
+// written nothing, when the threshold bin cannot be resolved (s_hist is then dirty).
 template <typename RegionOf>
 __device__ bool select_in_registers(const SelectArgs& s, int pair, int n_reg, int seg,
                                     uint32_t want, uint32_t base, int hshift, RegionOf region_of,
                                     const uint32_t* s_roff, uint32_t* s_hist, uint32_t* s_list,
-                                    uint32_t* s_wsum, int* s_info) {
+                                    uint32_t* s_wsum, uint32_t* s_cnt, int* s_info) {
   const ScanArgs& a = s.scan;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int budget = a.budget;
   const int n = (int)s_roff[n_reg];
   const uint32_t* ck = a.cands.key + (int64_t)pair * n_reg * seg;
   const int32_t* cp = a.cands.pos + (int64_t)pair * n_reg * seg;
@@ -1211,94 +1395,34 @@ __device__ bool select_in_registers(const SelectArgs& s, int pair, int n_reg, in
       pos[u] = cp[src];
     }
   }
-#pragma unroll
-  for (int u = 0; u < kSelRun; ++u)
-    if (lo + 32 * u + lane < hi)
-      atomicAdd(&s_hist[min((uint32_t)kSelBins - 1u, (key[u] - base) >> hshift)], 1u);
-  __syncthreads();
-  find_bin<kSelThreads>(s_hist, kSelBins, want, s_wsum, s_info);
-  const bool found = s_info[3] != 0;
-  const uint32_t bin = (uint32_t)s_info[0], m = (uint32_t)s_info[2];
-  const uint32_t w2 = want - (uint32_t)s_info[1];
-  __syncthreads();  // s_info and s_wsum are rewritten below
-  if (!found || bin == kSelBins - 1 || (w2 != m && m > 256)) return false;
-  int64_t thr;
-  uint32_t take;
-  if (w2 == m) {  // the whole bin: every key from its lowest one
-    thr = (int64_t)base + ((int64_t)bin << hshift) - 1;
-    take = 0;
-  } else {
-    if (tid == 0) s_info[3] = 0;
-    __syncthreads();
+  auto each = [&](auto&& f) {
 #pragma unroll
     for (int u = 0; u < kSelRun; ++u)
-      if (lo + 32 * u + lane < hi && ((key[u] - base) >> hshift) == bin)
-        s_list[atomicAdd(&s_info[3], 1)] = key[u];
-    __syncthreads();
-    if (tid < (int)m) {
-      const uint32_t x = s_list[tid];
-      uint32_t gt = 0, eq = 0;
-      for (uint32_t i = 0; i < m; ++i) {
-        const uint32_t y = s_list[i];
-        gt += y > x;
-        eq += y == x;
-      }
-      if (gt < w2 && w2 <= gt + eq) {  // x is the w2-th largest of the bin (equal keys agree)
-        s_info[0] = (int)x;
-        s_info[1] = (int)(w2 - gt);
-      }
-    }
-    __syncthreads();
-    thr = (int64_t)(uint32_t)s_info[0];
-    take = (uint32_t)s_info[1];
-  }
-  // per-warp counts, then each warp's offsets from the warps before it
-  unsigned gtm[kSelRun], eqm[kSelRun];
+      if (lo + 32 * u + lane < hi) f(key[u]);
+  };
+  int64_t thr;
+  uint32_t take;
+  if (!threshold_in_registers(each, want, base, hshift, s_hist, s_list, s_wsum, s_info, thr, take))
+    return false;
   uint32_t n_gt = 0, n_eq = 0;
+  each([&](uint32_t k) {
+    n_gt += (int64_t)k > thr;
+    n_eq += (int64_t)k == thr;
+  });
 #pragma unroll
-  for (int u = 0; u < kSelRun; ++u) {
-    const bool in = lo + 32 * u + lane < hi;
-    gtm[u] = __ballot_sync(0xffffffffu, in && (int64_t)key[u] > thr);
-    eqm[u] = __ballot_sync(0xffffffffu, in && (int64_t)key[u] == thr);
-    n_gt += __popc(gtm[u]);
-    n_eq += __popc(eqm[u]);
+  for (int o = 16; o > 0; o >>= 1) {
+    n_gt += __shfl_xor_sync(0xffffffffu, n_gt, o);
+    n_eq += __shfl_xor_sync(0xffffffffu, n_eq, o);
   }
-  if (lane == 0) {
-    s_wsum[warp] = n_gt;
-    s_wsum[kSelWarps + warp] = n_eq;
-  }
-  __syncthreads();
-  uint32_t gt_b = 0, eq_b = 0, total_gt = 0, total_eq = 0;
+  uint32_t gt_b, eq_b, total_gt, total_eq;
+  warp_offsets(n_gt, n_eq, s_cnt, gt_b, eq_b, total_gt, total_eq);
+  int32_t* out_idx = s.idx + (int64_t)pair * a.budget;
 #pragma unroll
-  for (int w = 0; w < kSelWarps; ++w) {
-    const uint32_t g_ = s_wsum[w], e_ = s_wsum[kSelWarps + w];
-    gt_b += w < warp ? g_ : 0u;
-    eq_b += w < warp ? e_ : 0u;
-    total_gt += g_;
-    total_eq += e_;
-  }
-  const unsigned lt = (1u << lane) - 1u;
-  int32_t* out_idx = s.idx + (int64_t)pair * budget;
-#pragma unroll
-  for (int u = 0; u < kSelRun; ++u) {
-    const uint32_t g_before = gt_b + __popc(gtm[u] & lt), e_before = eq_b + __popc(eqm[u] & lt);
-    if ((gtm[u] >> lane) & 1u) {
-      const uint32_t at = g_before + min(e_before, take);
-      if (at < (uint32_t)budget) out_idx[at] = pos[u];
-    } else if (((eqm[u] >> lane) & 1u) && e_before < take && g_before + e_before < (uint32_t)budget) {
-      out_idx[g_before + e_before] = pos[u];
-    }
-    gt_b += __popc(gtm[u]);
-    eq_b += __popc(eqm[u]);
-  }
-  const uint32_t written = total_gt + min(total_eq, take);
-  for (int j = (int)want + tid; j < budget; j += kSelThreads) out_idx[j] = -1;
-  if (tid == 0) {
-    if (written != want) raise_flag(8u);
-    s.count[pair] = (int)want;
-    // the attention launched next merges its splits through these counters
-    if (a.cands.attend_tickets) a.cands.attend_tickets[pair] = 0;
-  }
+  for (int u = 0; u < kSelRun; ++u)
+    if (lo + 32 * u < hi)  // (warp-uniform)
+      emit_group(lo + 32 * u + lane < hi, key[u], pos[u], thr, take, a.budget, out_idx, gt_b,
+                 eq_b);
+  select_finish(s, pair, want, total_gt + min(total_eq, take), out_idx);
   return true;
 }
 
@@ -1320,10 +1444,15 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
   const int L = clamp_len(a.seq_lens[b], a.max_pages << a.page_shift);
   const int budget = a.budget;
   int32_t* out_idx = s.idx + (int64_t)pair * budget;
+  // the prep's record: the prep grid completed before any scan CTA passed its own wait, and
+  // this grid starts only once every scan CTA has passed it, so the record may be read before
+  // waiting for the scan (from L2: no stale L1 line)
+  const uint8_t* rec = a.prep.rec + (int64_t)pair * kPrepBytes;
+  const int mode = __ldcg(reinterpret_cast<const int*>(rec + kPrepMode));
+  const uint32_t base = __ldcg(reinterpret_cast<const unsigned int*>(rec + kPrepThr));
+  const uint32_t sample_max = __ldcg(reinterpret_cast<const unsigned int*>(rec + kPrepKmax));
   pdl_wait();  // the scan's candidates
   pdl_trigger();  // the attention may be scheduled; it waits for this grid to complete
-  const uint8_t* rec = a.prep.rec + (int64_t)pair * kPrepBytes;
-  const int mode = *reinterpret_cast<const int*>(rec + kPrepMode);
   if (mode == kModeAll) {
     for (int j = tid; j < budget; j += kSelThreads) out_idx[j] = j < L ? j : -1;
     if (tid == 0) {
@@ -1338,13 +1467,19 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
   const int32_t* cp = a.cands.pos + (int64_t)pair * n_reg * seg;
   const uint32_t* cc = a.cands.cnt + (int64_t)pair * n_reg;
   const uint32_t want = (uint32_t)min(budget, L);
-  // histogram of the candidate keys, built while they are staged, over [the prep's threshold,
-  // the largest sampled key] (keys above it fall into the top bin)
-  const uint32_t base = *reinterpret_cast<const uint32_t*>(rec + kPrepThr);
-  const uint32_t sample_max = *reinterpret_cast<const uint32_t*>(rec + kPrepKmax);
+  // histogram of the candidate keys over [the prep's threshold, the largest sampled key] (keys
+  // above it fall into the top bin)
   bool use_hist = base > 0u && sample_max > base;
   const int hshift = use_hist ? max(0, (32 - __clz(sample_max - base)) - kSelBinBits) : 0;
   for (int i = tid; i < kSelBins; i += kSelThreads) s_hist[i] = 0u;
+  uint32_t* s_cnt = reinterpret_cast<uint32_t*>(s_red64);  // 2 kSelWarps words
+  if (use_hist && n_reg <= kSelWarps * kSelRegsPerWarp) {
+    if (select_region_major(s, pair, n_reg, seg, want, base, hshift, s_hist, s_ckey, s_wsum,
+                            s_cnt, s_info))
+      return;
+    __syncthreads();
+    for (int i = tid; i < kSelBins; i += kSelThreads) s_hist[i] = 0u;  // (paths below)
+  }
 
   // region offsets: exclusive prefix of the counts, in position order (each thread loads and
   // sums a run of adjacent regions, then a block-wide scan)
@@ -1381,7 +1516,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
   };
   if (use_hist && s_roff[n_reg] >= want && s_roff[n_reg] <= (uint32_t)(kSelThreads * kSelRun)) {
     if (select_in_registers(s, pair, n_reg, seg, want, base, hshift, region_of, s_roff, s_hist,
-                            s_ckey, s_wsum, s_info))
+                            s_ckey, s_wsum, s_cnt, s_info))
       return;
     for (int i = tid; i < kSelBins; i += kSelThreads) s_hist[i] = 0u;  // (general path below)
     __syncthreads();
