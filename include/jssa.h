@@ -34,7 +34,9 @@
  * - Device-side checks: a page number outside [0, num_pages), a position outside the block
  *   table, or a seq_len above max_pages*page_size is never dereferenced: the row is skipped and
  *   a flag is raised in the library's device error word (jssa_device_error). Kernels never trap.
- * - Supported template shapes: d = 128 with r in {32, 64}; G <= 8 for attention.
+ * - Supported template shapes: d = 128 with r in {32, 64}, and d = 256 with r = 64 (the
+ *   global layer of a hybrid sliding-window / global stack); G <= 8 for attention; calibration
+ *   needs G * d <= 2048.
  */
 #ifndef JSSA_H_
 #define JSSA_H_
@@ -133,7 +135,8 @@ JSSA_API int jssa_calibrate_accumulate(const jssa_bf16* q, int64_t q_stride_n, c
  * eigendecomposition per layer and KV head). Cyclic Jacobi in float64 on the device.
  * basis: float32 [h_kv, r, d], rows = eigenvectors of the r largest eigenvalues, descending,
  * each signed so that its largest-magnitude entry is positive (lowest index on ties).
- * eigvals: float64 [h_kv, d] descending, or NULL. ws: >= jssa_workspace_size(JSSA_FN_COMPUTE_BASIS).
+ * eigvals: float64 [h_kv, d] descending, or NULL. ws: >= jssa_workspace_size(JSSA_FN_COMPUTE_BASIS)
+ * (h_kv d^2 doubles for the eigenvectors, plus h_kv d (d + 1) for the matrices at d = 256).
  */
 JSSA_API int jssa_compute_basis(const double* gram_q, const double* gram_k, int h_kv, int d, int r,
                        float* basis, double* eigvals, void* ws, size_t ws_bytes,

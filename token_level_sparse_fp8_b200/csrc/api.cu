@@ -60,7 +60,10 @@ inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? JSSA_OK : (int
 inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 inline cudaStream_t as_stream(jssa_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
-bool supported_dr(int d, int r) { return d == 128 && (r == 32 || r == 64); }
+bool supported_dr(int d, int r) {
+  return (d == 128 && (r == 32 || r == 64)) || (d == 256 && r == 64);
+}
+bool supported_d(int d) { return d == 128 || d == 256; }
 
 int check_heads(int h_q, int h_kv) {
   if (h_q <= 0 || h_kv <= 0 || h_q % h_kv) return JSSA_ERR_SHAPE;
@@ -84,6 +87,14 @@ int check_kv(const void* k_cache, const void* v_cache, int64_t page_stride, int6
   (void)h_kv;
   (void)page_size;
   return JSSA_OK;
+}
+
+// eigenvectors [h_kv][d][d] float64; at d = 256 also the matrices [h_kv][d][d + 1] (they do not
+// fit in shared memory)
+size_t basis_ws_bytes(int h_kv, int d) {
+  size_t n = (size_t)h_kv * d * d;
+  if (d > 128) n += (size_t)h_kv * d * (d + 1);
+  return n * sizeof(double);
 }
 
 size_t score_ws_bytes(int batch, int h_kv, int max_seq_len, int page_size) {
@@ -133,7 +144,7 @@ int jssa_workspace_size(int fn, int batch, int h_q, int h_kv, int d, int max_pag
   const int max_seq_len = max_pages * page_size;
   if (fn == JSSA_FN_COMPUTE_BASIS) {
     if (h_kv <= 0) return JSSA_ERR_SHAPE;
-    *bytes = (size_t)h_kv * d * d * sizeof(double);
+    *bytes = basis_ws_bytes(h_kv, d);
     return JSSA_OK;
   }
   int st = check_heads(h_q, h_kv);
@@ -173,8 +184,8 @@ int jssa_calibrate_accumulate(const jssa_bf16* q, int64_t q_stride_n, const jssa
   if (n < 0) return JSSA_ERR_SHAPE;
   int st = check_heads(h_q, h_kv);
   if (st) return st;
-  if (d != 128) return JSSA_ERR_UNSUPPORTED;
-  if (h_q / h_kv > 16) return JSSA_ERR_UNSUPPORTED;
+  if (!supported_d(d)) return JSSA_ERR_UNSUPPORTED;
+  if (h_q / h_kv > 16 || (h_q / h_kv) * d > 2048) return JSSA_ERR_UNSUPPORTED;
   if (n == 0) return JSSA_OK;
   if (!q || !k || !gram_q || !gram_k) return JSSA_ERR_NULL;
   if (!aligned16(q) || !aligned16(k) || (q_stride_n & 7) || (k_stride_n & 7)) return JSSA_ERR_ALIGN;
@@ -187,9 +198,9 @@ int jssa_compute_basis(const double* gram_q, const double* gram_k, int h_kv, int
                        float* basis, double* eigvals, void* ws, size_t ws_bytes,
                        jssa_stream_t stream) {
   if (h_kv <= 0 || r <= 0 || r > d) return JSSA_ERR_SHAPE;
-  if (d != 128) return JSSA_ERR_UNSUPPORTED;
+  if (!supported_d(d)) return JSSA_ERR_UNSUPPORTED;
   if (!gram_q || !gram_k || !basis) return JSSA_ERR_NULL;
-  const size_t need = (size_t)h_kv * d * d * sizeof(double);
+  const size_t need = basis_ws_bytes(h_kv, d);
   if (!ws || ws_bytes < need) return JSSA_ERR_WORKSPACE;
   if (((uintptr_t)ws & 7u) != 0) return JSSA_ERR_ALIGN;
   return cuda_status(jssa::launch_basis(gram_q, gram_k, h_kv, d, r, basis, eigvals,
@@ -255,7 +266,7 @@ static int check_attend_common(const jssa_bf16* q, const jssa_bf16* k_cache,
   if (batch < 0) return JSSA_ERR_SHAPE;
   int st = check_heads(h_q, h_kv);
   if (st) return st;
-  if (d != 128) return JSSA_ERR_UNSUPPORTED;
+  if (!supported_d(d)) return JSSA_ERR_UNSUPPORTED;
   if (h_q / h_kv > jssa::kAttendMaxG) return JSSA_ERR_UNSUPPORTED;
   if ((st = check_paging(max_pages, num_pages, page_size))) return st;
   if (batch == 0) return JSSA_OK;

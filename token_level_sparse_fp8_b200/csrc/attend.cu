@@ -5,8 +5,8 @@
 // of its positions -- a slice of the index set (indexed mode) or of [lo, seq_len) (dense mode).
 //   * Row addresses: the CTA first turns each of its positions into a 64-bit element offset
 //     (page-table lookup, bounds checked) kept in shared memory.
-//   * Each of the 4 warps walks its own 16-token tiles. A tile's K and V rows (256 B each at
-//     d = 128) are copied straight from their paged locations into the warp's ring of kStages
+//   * Each of the 4 warps walks its own 16-token tiles. A tile's K and V rows (2d bytes each:
+//     256 B at d = 128, 512 B at d = 256) are copied straight from their paged locations into the warp's ring of kStages
 //     shared-memory stages with 16-byte cp.async (rows past the slice or on unusable pages are
 //     zero-filled) -- no staging buffer in global memory -- so kStages - 1 tiles are in flight
 //     while one is computed. Inside a stage a row's 16-byte chunk c sits at chunk c ^ (row & 7),
@@ -32,9 +32,17 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kTile = kAttendTile;
 constexpr int kMaxChunk = 1024;  // positions per CTA (row offsets kept in shared memory)
 constexpr int kStages = 3;       // tiles per warp ring (kStages - 1 in flight)
-constexpr int kTileBytes = kTile * 128 * 2;   // K (or V) rows of one tile at d = 128
-constexpr int kStageBytes = 2 * kTileBytes;   // K then V
-constexpr int kRingBytes = kWarps * kStages * kStageBytes;  // dynamic shared memory per CTA
+// Shared-memory ring geometry for head dim D: K (or V) rows of one tile, a stage (K then V), the
+// dynamic shared memory of a CTA; CTAs per SM (d = 128: two; d = 256: one, its ring is 192 KB).
+template <int D>
+struct Ring {
+  static constexpr int kRowBytes = D * 2;
+  static constexpr int kChunks = kRowBytes / 16;  // 16-byte chunks per row
+  static constexpr int kTileBytes = kTile * kRowBytes;
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kBytes = kWarps * kStages * kStageBytes;
+  static constexpr int kCtasPerSm = D == 128 ? 2 : 1;
+};
 
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
   uint32_t r;
@@ -43,9 +51,12 @@ __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
 }
 
 template <int D, bool INDEXED>
-__global__ void __launch_bounds__(kThreads, 2) attend_kernel(AttendArgs a, int chunk, int splits) {
-  static_assert(D == 128, "head dim");
+__global__ void __launch_bounds__(kThreads, Ring<D>::kCtasPerSm)
+    attend_kernel(AttendArgs a, int chunk, int splits) {
+  static_assert(D == 128 || D == 256, "head dim");
   constexpr int KB = D / 16;  // k-blocks of S^T, m-tiles of O^T
+  constexpr int kRowBytes = Ring<D>::kRowBytes, kChunks = Ring<D>::kChunks;
+  constexpr int kTileBytes = Ring<D>::kTileBytes, kStageBytes = Ring<D>::kStageBytes;
   extern __shared__ __align__(128) uint8_t att_ring[];  // warp rings; the warp merge reuses it
   __shared__ int64_t s_off[kMaxChunk];
   __shared__ float s_m[kWarps][kAttendMaxG], s_l[kWarps][kAttendMaxG];
@@ -134,17 +145,18 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(AttendArgs a, int c
   float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};  // heads 2t, 2t+1
 
   const uint32_t ring = smem_u32(att_ring) + warp * kStages * kStageBytes;
-  // copies of tile `tl` into stage `st`: piece p = 32 it + lane is row p / 16, chunk p % 16
+  // copies of tile `tl` into stage `st`: piece p = 32 it + lane is row p / kChunks, chunk
+  // p % kChunks
   auto issue = [&](int tl, int st) {
     const int j0 = tl * kTile;
 #pragma unroll
-    for (int it = 0; it < kTile * 16 / 32; ++it) {
+    for (int it = 0; it < kTile * kChunks / 32; ++it) {
       const int p = 32 * it + lane;
-      const int row = p >> 4, c = p & 15;
+      const int row = p / kChunks, c = p % kChunks;
       const int j = j0 + row;
       const int64_t off = j < n_mine ? s_off[j] : -1;
       const int64_t src = (off >= 0 ? off : 0) + c * 8;
-      const uint32_t dst = ring + st * kStageBytes + row * 256 + ((c ^ (row & 7)) << 4);
+      const uint32_t dst = ring + st * kStageBytes + row * kRowBytes + ((c ^ (row & 7)) << 4);
       cp_async16(dst, a.k_cache + src, off >= 0 ? 16 : 0);
       cp_async16(dst + kTileBytes, a.v_cache + src, off >= 0 ? 16 : 0);
     }
@@ -173,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(AttendArgs a, int c
     for (int kb = 0; kb < KB; ++kb) {
       const int c = 2 * kb + k_half;
       uint32_t a0, a1, a2, a3;
-      ldsm_x4(st + k_row * 256 + ((c ^ (k_row & 7)) << 4), a0, a1, a2, a3);
+      ldsm_x4(st + k_row * kRowBytes + ((c ^ (k_row & 7)) << 4), a0, a1, a2, a3);
       mma_bf16(s, a0, a1, a2, a3, qb0[kb], qb1[kb]);
     }
     // rows: token g (s[0], s[1]) and g+8 (s[2], s[3]); columns: heads 2t, 2t+1
@@ -222,7 +234,8 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(AttendArgs a, int c
     for (int m = 0; m < KB; ++m) {
       const int c = 2 * m + v_half;
       uint32_t va0, va1, va2, va3;
-      ldsm_x4_t(st + kTileBytes + v_row * 256 + ((c ^ (v_row & 7)) << 4), va0, va1, va2, va3);
+      ldsm_x4_t(st + kTileBytes + v_row * kRowBytes + ((c ^ (v_row & 7)) << 4), va0, va1, va2,
+                va3);
       mma_bf16(o[m], va0, va1, va2, va3, bh0, bh1);
       mma_bf16(o[m], va0, va1, va2, va3, bl0, bl1);
     }
@@ -315,7 +328,8 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(AttendArgs a, int c
 template <int D, bool INDEXED>
 cudaError_t launch_t(const AttendArgs& a, const AttendPlan& plan, bool pdl, cudaStream_t s) {
   auto kern = attend_kernel<D, INDEXED>;
-  static_assert(kRingBytes >= kWarps * kAttendMaxG * 128 * (int)sizeof(float), "merge buffer");
+  constexpr int kRingBytes = Ring<D>::kBytes;
+  static_assert(kRingBytes >= kWarps * kAttendMaxG * D * (int)sizeof(float), "merge buffer");
   cudaError_t ce = configure_kernel((const void*)kern, kRingBytes, false);
   if (ce != cudaSuccess) return ce;
   cudaLaunchConfig_t cfg = {};
@@ -340,8 +354,9 @@ AttendPlan plan_attend(int pairs, int positions, int group, int d) {
   const int unit = attend_detail::kWarps * attend_detail::kTile;  // 64 positions
   positions = positions < 1 ? 1 : positions;
   const int max_splits = (positions + unit - 1) / unit;
-  // about one wave of resident CTAs (2 per SM); more splits only when the pairs are few
-  const int slots = 2 * num_sms();
+  // about one wave of resident CTAs (2 per SM at d = 128, 1 at d = 256); more splits only when
+  // the pairs are few
+  const int slots = (d == 128 ? 2 : 1) * num_sms();
   int splits = slots / (pairs > 0 ? pairs : 1);
   if (splits > max_splits) splits = max_splits;
   if (splits < 1) splits = 1;
@@ -363,6 +378,9 @@ cudaError_t launch_attend(const AttendArgs& a, bool indexed, const AttendPlan& p
   if (a.d == 128)
     return indexed ? attend_detail::launch_t<128, true>(a, plan, pdl, s)
                    : attend_detail::launch_t<128, false>(a, plan, pdl, s);
+  if (a.d == 256)
+    return indexed ? attend_detail::launch_t<256, true>(a, plan, pdl, s)
+                   : attend_detail::launch_t<256, false>(a, plan, pdl, s);
   return cudaErrorInvalidValue;
 }
 

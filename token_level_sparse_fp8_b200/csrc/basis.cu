@@ -3,8 +3,9 @@
 // eigendecomposition per layer and KV head).
 //
 // One CTA per KV head runs a parallel cyclic Jacobi eigensolver in float64: the d x d matrix
-// lives in shared memory (rows padded by one element), the eigenvectors are accumulated as the
-// rows of V^T in the workspace. Each sweep is d-1 rounds of the round-robin ("circle") pairing,
+// lives in shared memory at d = 128 (rows padded by one element) and in the workspace at
+// d = 256 (512 KB: too large for shared memory; it stays in L2), the eigenvectors are
+// accumulated as the rows of V^T in the workspace. Each sweep is d-1 rounds of the round-robin ("circle") pairing,
 // so the d/2 rotations of a round touch disjoint index pairs and run in parallel: rotation
 // parameters, then the row update (A <- J^T A, V^T <- J^T V^T), then the column update
 // (A <- A J). Sweeps stop when the off-diagonal Frobenius norm is below 1e-14 of the total, or
@@ -46,7 +47,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     basis_kernel(const double* __restrict__ gram_q, const double* __restrict__ gram_k, int r,
                  float* __restrict__ basis, double* __restrict__ eigvals, double* __restrict__ ws) {
   constexpr int LD = D + 1;
-  extern __shared__ __align__(16) double sA[];  // [D][LD]
+  constexpr bool kGlobalA = D > 128;
+  extern __shared__ __align__(16) double s_a[];  // [D][LD] (D = 128)
   __shared__ double s_c[D / 2], s_s[D / 2];
   __shared__ int s_p[D / 2], s_q[D / 2];
   __shared__ double s_red[kThreads / 32];
@@ -58,6 +60,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const double* gq = gram_q + (int64_t)h * D * D;
   const double* gk = gram_k + (int64_t)h * D * D;
   double* vt = ws + (int64_t)h * D * D;  // rows are eigenvectors
+  double* sA = kGlobalA ? ws + (int64_t)gridDim.x * D * D + (int64_t)h * D * LD : s_a;
 
   double tq = 0.0, tk = 0.0;
   for (int i = tid; i < D; i += kThreads) {
@@ -178,9 +181,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 cudaError_t launch_basis(const double* gram_q, const double* gram_k, int h_kv, int d, int r,
                          float* basis, double* eigvals, double* ws, cudaStream_t s) {
   if (h_kv <= 0) return cudaSuccess;
-  if (d != 128) return cudaErrorInvalidValue;
-  const size_t smem = (size_t)d * (d + 1) * sizeof(double);
-  auto kern = basis_detail::basis_kernel<128>;
+  if (d != 128 && d != 256) return cudaErrorInvalidValue;
+  const size_t smem = d == 128 ? (size_t)d * (d + 1) * sizeof(double) : 0;
+  auto kern = d == 128 ? basis_detail::basis_kernel<128> : basis_detail::basis_kernel<256>;
   cudaError_t e = configure_kernel((const void*)kern, (int)smem, false);
   if (e != cudaSuccess) return e;
   kern<<<h_kv, basis_detail::kThreads, smem, s>>>(gram_q, gram_k, r, basis, eigvals, ws);

@@ -7,8 +7,9 @@
 // The second form keeps the tensor-core inputs exact: every q_{n,g} is a bf16 value, so the
 // G^2 products per sample are exact in the fp32 accumulators (qbar itself is not bf16).
 //
-// Grid (sample chunks, h_kv, 2 [keys | queries]); 8 warps per CTA tile the full d x d = 128 x 128
-// Gram (warp w: rows 32*(w/2).., cols 64*(w%2)..) with mma.sync m16n8k16. Sample tiles of 32 rows
+// Grid (sample chunks, h_kv, 2 [keys | queries] x (d / 128)^2 tiles); 8 warps per CTA tile one
+// 128 x 128 block of the d x d Gram (warp w: rows 32*(w/2).., cols 64*(w%2).. of the block) with
+// mma.sync m16n8k16. Sample tiles of 32 rows
 // per head are staged in swizzled shared memory with cp.async; both operands are read with
 // ldmatrix.trans (X^T X). Each CTA adds its chunk sum (fp32, folded per block) into the float64
 // totals.
@@ -27,13 +28,15 @@ __global__ void __launch_bounds__(kThreads)
     gram_kernel(const uint16_t* __restrict__ q, int64_t q_stride, const uint16_t* __restrict__ k,
                 int64_t k_stride, int n, int h_q, int h_kv, double* __restrict__ gram_q,
                 double* __restrict__ gram_k) {
-  static_assert(D == 128, "one CTA tiles a 128 x 128 Gram");
+  static_assert(D == 128 || D == 256, "one CTA tiles a 128 x 128 block of the Gram");
   constexpr int RB = D * 2;  // row bytes
+  constexpr int T = D / 128;  // blocks per Gram row
   extern __shared__ __align__(128) uint8_t calib_smem[];
   const uint32_t sbase = smem_u32(calib_smem);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h = blockIdx.y;
-  const bool is_q = blockIdx.z == 1;
+  const bool is_q = (blockIdx.z & 1) == 1;
+  const int blk = blockIdx.z >> 1;  // Gram block (blk / T, blk % T)
   const int G = h_q / h_kv;
   const int nh = is_q ? G : 1;  // head rows staged per sample
   const int n0 = blockIdx.x * kChunkN, n1 = min(n, n0 + kChunkN);
@@ -49,8 +52,8 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
       for (int c = 0; c < 4; ++c) acc[a][b][c] = tot[a][b][c] = 0.f;
 
-  const int row0 = 32 * (warp >> 1);   // first Gram row of this warp
-  const int col0 = 64 * (warp & 1);    // first Gram column
+  const int row0 = 128 * (blk / T) + 32 * (warp >> 1);  // first Gram row of this warp
+  const int col0 = 128 * (blk % T) + 64 * (warp & 1);   // first Gram column
 
   for (int t0 = n0; t0 < n1; t0 += kTileN) {
     // stage [nh][kTileN][D] (row r of head gl at ((gl*kTileN + r) * RB), chunks swizzled by r)
@@ -132,13 +135,14 @@ cudaError_t launch_gram(const uint16_t* q, int64_t q_stride, const uint16_t* k, 
                         int n, int h_q, int h_kv, int d, double* gram_q, double* gram_k,
                         cudaStream_t s) {
   if (n <= 0 || h_kv <= 0) return cudaSuccess;
-  if (d != 128) return cudaErrorInvalidValue;
+  if (d != 128 && d != 256) return cudaErrorInvalidValue;
   const int G = h_q / h_kv;
   const size_t smem = (size_t)G * calib_detail::kTileN * d * 2;
-  auto kern = calib_detail::gram_kernel<128>;
+  auto kern = d == 128 ? calib_detail::gram_kernel<128> : calib_detail::gram_kernel<256>;
   cudaError_t e = configure_kernel((const void*)kern, (int)smem, false);
   if (e != cudaSuccess) return e;
-  dim3 grid((n + calib_detail::kChunkN - 1) / calib_detail::kChunkN, h_kv, 2);
+  const int blocks = (d / 128) * (d / 128);
+  dim3 grid((n + calib_detail::kChunkN - 1) / calib_detail::kChunkN, h_kv, 2 * blocks);
   kern<<<grid, calib_detail::kThreads, smem, s>>>(q, q_stride, k, k_stride, n, h_q, h_kv, gram_q, gram_k);
   return cudaGetLastError();
 }

@@ -897,7 +897,9 @@ __device__ __forceinline__ int sample_group_start(int grp, int pair, int L) {
   return kGroup * (first + (int)__umulhi(hsh, (uint32_t)(stratum / kGroup - 1)));
 }
 
-constexpr int kQGroups = kThreads / 16;  // query rows loaded per pass (16 threads x 8 dims a row)
+// query rows loaded per pass: D / 8 threads x 8 dims a row
+template <int D>
+constexpr int q_groups() { return kThreads / (D / 8); }
 constexpr int kSampleBins = 256;          // histogram bins of the sampled scores
 
 // Dynamic shared memory of the prep kernel.
@@ -905,7 +907,7 @@ template <int D, int R>
 struct PrepSmem {
   uint8_t rows[kSample * R];     // code rows of the sampled positions
   float m[R * D];                // M_h, row-major [R][D]
-  float qpart[kQGroups][D];      // partial sums of the group's query rows
+  float qpart[q_groups<D>()][D]; // partial sums of the group's query rows
   uint32_t list[256];            // keys of the bin that holds the threshold
   uint32_t hist[kSampleBins];
   uint8_t valid[kSample];        // sampled position on a usable page
@@ -946,10 +948,11 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
   for (int i = tid; i < R * D / 4; i += kThreads) cp_async16(smem_u32(sm.m + 4 * i), m_h + 4 * i, 16);
   cp_async_commit();
   const int L = clamp_len(a.seq_lens[b], a.max_pages << a.page_shift);
-  // the G query rows of this KV head: 16 threads x 8 dims per row, kQGroups rows at a time
-  static_assert(D == 128, "query row split");
+  // the G query rows of this KV head: D / 8 threads x 8 dims per row, kQGroups rows at a time
+  static_assert(D == 128 || D == 256, "query row split");
+  constexpr int kQGroups = q_groups<D>();
   const uint16_t* qh = a.q + ((int64_t)b * a.h_q + (int64_t)h * G) * D;
-  const int rg = tid / 16, d8 = (tid % 16) * 8;
+  const int rg = tid / (D / 8), d8 = (tid % (D / 8)) * 8;
   uint4 qv = make_uint4(0u, 0u, 0u, 0u);
   if (rg < G) qv = *reinterpret_cast<const uint4*>(qh + (int64_t)rg * D + d8);
   const bool store = STORE && L > 0;
@@ -1777,6 +1780,8 @@ cudaError_t launch_score_topk(const uint16_t* q, const float* basis, const uint8
     return score_detail::launch_t<128, 32>(plan, pairs, pa, sa, sel, store != nullptr, pdl, s);
   if (d == 128 && r == 64)
     return score_detail::launch_t<128, 64>(plan, pairs, pa, sa, sel, store != nullptr, pdl, s);
+  if (d == 256 && r == 64)
+    return score_detail::launch_t<256, 64>(plan, pairs, pa, sa, sel, store != nullptr, pdl, s);
   return cudaErrorInvalidValue;
 }
 

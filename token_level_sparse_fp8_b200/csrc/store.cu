@@ -145,6 +145,7 @@ cudaError_t dispatch_store(int d, int r, int t, int h_kv, int tpb, cudaStream_t 
                                           head_stride, block_table, max_pages, seq_lens);
   JSSA_STORE_CASE(128, 32)
   JSSA_STORE_CASE(128, 64)
+  JSSA_STORE_CASE(256, 64)
 #undef JSSA_STORE_CASE
   return cudaErrorInvalidValue;
 }
