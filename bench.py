@@ -37,6 +37,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=800)
     ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", choices=["jssa", "reference"], default="jssa")
+    ap.add_argument("--workload", choices=["llama128k", "hybrid"], default="llama128k",
+                    help="llama128k: one 128K-context GQA layer (the headline); hybrid: a stack of "
+                         "5 sliding-window layers (dense over the last 1024 positions) and 1 global "
+                         "JSSA layer, head dim 256, 64K context")
     ap.add_argument("--batch", type=int, default=16)
     ap.add_argument("--budget", type=int, default=2048)
     ap.add_argument("--seq-len", type=int, default=131072)
@@ -589,10 +593,135 @@ def run_jssa(args):
     print(json.dumps(line), flush=True)
 
 
+def hybrid_bytes(w, dense=False):
+    """Algorithmic bytes of one stack step: the global layer (JSSA, or dense over the whole
+    context) plus the local layers' K/V rows of the window."""
+    pages = -(-w.seq_len // w.page_size)
+    local = (w.layers - 1) * w.batch * w.h_kv * w.window * 2 * w.d * 2
+    if dense:
+        glob = w.batch * (w.h_kv * w.seq_len * 2 * w.d * 2 + 4 * pages)
+    else:
+        glob = w.batch * (w.h_kv * w.seq_len * w.rank + w.h_kv * min(w.budget, w.seq_len) * 2 * w.d * 2
+                          + 4 * pages)
+    return glob + local
+
+
+def run_hybrid(args):
+    """One stack step of a hybrid model: (layers - 1) sliding-window layers, each dense paged
+    decode over the last `window` positions of its own KV cache, and one global layer, a full JSSA
+    decode step (store + score + top-B + indexed attend) over the whole context."""
+    import torch
+    import token_level_sparse_fp8_b200 as J
+    from synth import WORKLOADS, build_paged_kv, layer_factors
+
+    rank, world, local = dist_env()
+    assert torch.cuda.is_available(), "bench needs a CUDA device"
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    group = RankGroup("nccl", dev)
+    barrier, max_over_ranks = group.barrier, group.max_over_ranks
+    w = WORKLOADS["hybrid"]
+    w = w.replace(seed=w.seed + 7919 * rank)
+    J._lib.load()
+    state = setup_gpu(w, dev)
+    layer = state["layer"]
+    qs, k_new, v_new = state["qs"], state["k_new"], state["v_new"]
+    nq = len(qs)
+    locals_ = []
+    for li in range(1, w.layers):
+        f = layer_factors(w.seed, li, w.h_kv, w.d)
+        kv = build_paged_kv(f, [w.window] * w.batch, w.page_size, w.seed, layer=li, device=dev)
+        locals_.append(kv)
+    scale = 1.0 / math.sqrt(w.d)
+    out = torch.empty_like(qs[0])
+    outs = [torch.empty_like(qs[0]) for _ in locals_]
+    stream = torch.cuda.current_stream(dev)
+    ws_local = J.Workspace(dev)
+
+    def local_layers(i):
+        for kv, o in zip(locals_, outs):
+            J.dense_decode(qs[i % nq], kv["k_cache"], kv["v_cache"], kv["block_table"],
+                           kv["seq_lens"], scale, w.window, o, ws_local)
+
+    def step(i):
+        local_layers(i)
+        layer.step(qs[i % nq], k_new, v_new, out)
+
+    def dense_step(i):
+        local_layers(i)
+        layer.dense(qs[i % nq], out)
+
+    sampler = ClockSampler(local)
+    step(0)
+    dense_step(0)  # sizes the workspaces before capture
+    torch.cuda.synchronize()
+    barrier()
+    sampler.start()
+    t_step, n_steps = timed_graph(step, args.steps, args.warmup, stream, barrier, nq)
+    clocks = sampler.stop()
+    t_step = max_over_ranks(t_step)
+    t_dense = None
+    if not args.no_dense:
+        t_dense, n_dense = timed_graph(dense_step, max(8, args.steps // 4), 8, stream, barrier, nq)
+        t_dense = max_over_ranks(t_dense) / n_dense
+    check = None
+    if rank == 0 and not args.no_check:
+        check = sampled_check(state, w)
+    group.close()
+    if rank != 0:
+        return
+    peak, peak_kind = peaks()
+    ms_step = t_step / n_steps * 1e3
+    bytes_step = hybrid_bytes(w)
+    achieved = bytes_step / (ms_step / 1e3) / 1e9
+    line = {
+        "metric": "hybrid local/global stack decode steps/s (5 sliding-window + 1 global JSSA layer), 1xB200",
+        "value": whole_job_rate(world, n_steps, t_step),
+        "unit": "steps/s",
+        "n_gpus": world,
+        "steps": n_steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16 K/V, e4m3 scoring cache, fp32 math",
+        "data": "synthetic",
+        "config": {
+            "workload": f"hybrid stack: {w.layers - 1} sliding-window layers (dense over the last "
+                        f"{w.window} positions) + 1 global JSSA layer; h_q {w.h_q}, h_kv {w.h_kv}, "
+                        f"d {w.d}, L {w.seq_len}, page {w.page_size} (permuted), r {w.rank}, "
+                        f"B {w.budget}, batch {w.batch} per GPU",
+            "global_batch": w.batch * world,
+            "seq_len": w.seq_len,
+            "budget": w.budget,
+            "parallelism": f"dp{world} (independent sequences per GPU)",
+            "l2": "inputs larger than L2: the global layer's 256 MiB scoring cache is streamed every step",
+        },
+        "hbm_gbs": achieved,
+        "roofline_step": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                          "frac": achieved / peak, "traffic": None, "bytes_per_step": bytes_step,
+                          "peak_kind": peak_kind},
+        "clocks": clocks,
+        "gpu_launches": (w.layers - 1 + 3) * n_steps,
+        "timing": "CUDA events around replays of a CUDA graph holding 8 consecutive stack steps",
+    }
+    if t_dense is not None:
+        dense_bytes = hybrid_bytes(w, dense=True)
+        line["dense"] = {"steps_per_s": world / t_dense, "ms_per_step": t_dense * 1e3,
+                         "hbm_gbs": dense_bytes / t_dense / 1e9, "frac": dense_bytes / t_dense / 1e9 / peak}
+        line["speedup_vs_dense"] = t_dense / (ms_step / 1e3)
+    if check is not None:
+        line["oracle_check"] = check
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "hybrid":
+        run_hybrid(args)
     else:
         run_jssa(args)
 
