@@ -500,6 +500,19 @@ def run_jssa(args):
     t_attend, n_attend = timed_graph(attend_only, args.steps, args.warmup, stream, barrier, nq)
     t_attend = max_over_ranks(t_attend) / n_attend
 
+    # the ablation: gather the same index sets into staging buffers, then dense attention there
+    ws_gta = J.Workspace(dev)
+    bufs = J.gather_kv(layer.k_cache, layer.v_cache, layer.block_table, sets[0][0], sets[0][1])
+
+    def gather_then_attend(i):
+        ii, cc = sets[i % nq]
+        J.gather_then_attend(qs[i % nq], layer.k_cache, layer.v_cache, layer.block_table, ii, cc,
+                             layer.scale, out, ws_gta, bufs)
+
+    gather_then_attend(0)  # sizes the workspace before capture
+    t_gta, n_gta = timed_graph(gather_then_attend, args.steps, args.warmup, stream, barrier, nq)
+    t_gta = max_over_ranks(t_gta) / n_gta
+
     t_dense = None
     if not args.no_dense:
         layer.dense(qs[0], out)  # sizes the shared workspace before capture
@@ -586,6 +599,14 @@ def run_jssa(args):
         line["dense"] = {"steps_per_s": world / t_dense, "ms_per_step": t_dense * 1e3,
                          "hbm_gbs": dense_bytes / t_dense / 1e9, "frac": dense_bytes / t_dense / 1e9 / peak}
         line["speedup_vs_dense"] = t_dense / (ms_step / 1e3)
+    line["ablation_gather"] = {
+        "gather_free_attend_ms": t_attend * 1e3,
+        "gather_then_attend_ms": t_gta * 1e3,
+        "gather_free_over_gather": t_gta / t_attend,
+    }
+    if t_dense is not None:
+        line["ablation_gather"]["attend_speedup_vs_dense"] = {
+            "gather_free": t_dense / t_attend, "gather_then_attend": t_dense / t_gta}
     if check is not None:
         line["oracle_check"] = check
     if cpu is not None:

@@ -203,6 +203,27 @@ JSSA_API int jssa_dense_decode(const jssa_bf16* q, const jssa_bf16* k_cache, con
                       size_t ws_bytes, jssa_stream_t stream);
 
 /*
+ * Gather-then-attend ablation, step 1: copy the selected K and V rows of every (sequence, KV
+ * head), in index order, into contiguous staging buffers (JSSA README, "Highlights" and section
+ * 3: the gather-free attention is measured against gathering the selected rows first; JSSA
+ * summary, section 3.3). Step 2 is jssa_dense_decode over the staging buffers viewed as a paged
+ * cache of 16-token pages: page_stride 16*h_kv*d, slot_stride h_kv*d, head_stride d, sequence b
+ * on pages b*budget_pad/16 ... (b+1)*budget_pad/16 - 1, seq_lens = lens_out.
+ * idx, count: as produced by jssa_score_topk (count clamped to [0, budget]).
+ * k_out, v_out: bf16 [batch, budget_pad, h_kv, d], budget_pad = budget rounded up to a multiple
+ * of 16, 16-byte aligned, owned by the caller; slots at or past count are left untouched.
+ * lens_out: int32 [batch] = count[b, 0] (every head of a sequence has the same count).
+ * A position outside the block table or an unusable page is skipped (its staged row is
+ * written as zeros) and flagged in the device error word.
+ */
+JSSA_API int jssa_gather_kv(const jssa_bf16* k_cache, const jssa_bf16* v_cache,
+                            int64_t kv_page_stride, int64_t kv_slot_stride, int64_t kv_head_stride,
+                            const int32_t* block_table, int max_pages, const int32_t* idx,
+                            const int32_t* count, int batch, int h_kv, int d, int budget,
+                            int64_t num_pages, int page_size, jssa_bf16* k_out, jssa_bf16* v_out,
+                            int32_t* lens_out, jssa_stream_t stream);
+
+/*
  * One whole decode step for one layer: (1) when k_new and v_new are non-NULL, write the new
  * token (position seq_len-1 of each sequence) into the K and V caches and its scoring code into
  * the scoring cache; (2) score + top-B; (3) gather-free indexed attention. The three kernels

@@ -426,3 +426,45 @@ def test_calibration(tiny, n):
         assert np.max(np.abs(lam[h] - res["eigvals"][h])) <= 1e-5 * lam[h, 0]
         # rows agree with the oracle's rows up to the shared sign rule
         assert np.max(np.abs(m[h] - res["M"][h])) <= 5e-3
+
+
+# ------------------------------------------------------------------------------------------------
+# gather-then-attend (the ablation the gather-free attention is compared with)
+# ------------------------------------------------------------------------------------------------
+
+
+def test_gather_kv_is_an_exact_copy(ragged):
+    J = jssa()
+    budget = 128
+    ref_idx, ref_count, _ = _select_oracle(ragged, budget)
+    k, v, lens = J.gather_kv(ragged.gpu(ragged.k_cache), ragged.gpu(ragged.v_cache),
+                             ragged.gpu(ragged.block_table), ragged.gpu_np(ref_idx),
+                             ragged.gpu_np(ref_count))
+    assert lens.cpu().numpy().tolist() == ref_count[:, 0].tolist()
+    kc, vc = ragged.k_cache.view(torch.int16).numpy(), ragged.v_cache.view(torch.int16).numpy()
+    gk, gv = k.cpu().view(torch.int16).numpy(), v.cpu().view(torch.int16).numpy()
+    ps = ragged.ps
+    for b in range(len(ragged.seq_lens)):
+        for h in range(ragged.h_kv):
+            for j in range(ref_count[b, h]):
+                t = ref_idx[b, h, j]
+                page = ragged.np_bt[b, t // ps]
+                assert np.array_equal(gk[b, j, h], kc[page, t % ps, h])
+                assert np.array_equal(gv[b, j, h], vc[page, t % ps, h])
+
+
+@pytest.mark.parametrize("budget", [128, 1000])
+def test_gather_then_attend(ragged, budget):
+    J = jssa()
+    ref_idx, ref_count, _ = _select_oracle(ragged, budget)
+    scale = 1.0 / math.sqrt(ragged.d)
+    out = J.gather_then_attend(ragged.gpu(ragged.q), ragged.gpu(ragged.k_cache),
+                               ragged.gpu(ragged.v_cache), ragged.gpu(ragged.block_table),
+                               ragged.gpu_np(ref_idx), ragged.gpu_np(ref_count), scale)
+    ref = O.indexed_attend_step(ragged.np_q, ragged.np_k, ragged.np_v, ragged.np_bt, ref_idx,
+                                ref_count, scale)
+    check_output(f64(out), ref)
+    gf = J.indexed_attend(ragged.gpu(ragged.q), ragged.gpu(ragged.k_cache),
+                          ragged.gpu(ragged.v_cache), ragged.gpu(ragged.block_table),
+                          ragged.gpu_np(ref_idx), ragged.gpu_np(ref_count), scale)
+    check_output(f64(gf), ref)

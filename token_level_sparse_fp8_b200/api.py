@@ -19,6 +19,7 @@ from ._lib import (FN_COMPUTE_BASIS, FN_DECODE, FN_DENSE_DECODE, FN_INDEXED_ATTE
                    FN_SCORE_TOPK, JSSAError, call)
 
 __all__ = [
+    "gather_kv", "staged_pages", "gather_then_attend",
     "JSSAError", "workspace_size", "Workspace", "calibrate_accumulate", "compute_basis",
     "calibrate", "store", "score_topk", "indexed_attend", "dense_decode", "decode",
     "device_error", "kv_strides", "default_rank", "PagedLayer",
@@ -217,6 +218,59 @@ def indexed_attend(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
          block_table.data_ptr(), block_table.shape[1], idx.data_ptr(), count.data_ptr(), batch, h_q,
          h_kv, d, budget, num_pages, page_size, scale, out.data_ptr(), p, n, _stream(q.device))
     return out
+
+
+def gather_kv(k_cache: torch.Tensor, v_cache: torch.Tensor, block_table: torch.Tensor,
+              idx: torch.Tensor, count: torch.Tensor, bufs=None):
+    """Copies of the selected K and V rows in index order (the gather step of the
+    gather-then-attend ablation): ``k, v`` bf16 ``[batch, budget_pad, h_kv, d]`` and
+    ``lens`` int32 ``[batch]`` (= count[:, 0]); ``bufs`` = (k, v, lens) to reuse."""
+    _need(k_cache, "k_cache", torch.bfloat16, contiguous=False)
+    _need(v_cache, "v_cache", torch.bfloat16, contiguous=False)
+    _need(block_table, "block_table", torch.int32)
+    _need(idx, "idx", torch.int32)
+    _need(count, "count", torch.int32)
+    num_pages, page_size, h_kv, d = k_cache.shape
+    strides = kv_strides(k_cache)
+    if kv_strides(v_cache) != strides:
+        raise ValueError("K and V caches must share one layout")
+    batch, _, budget = idx.shape
+    budget_pad = -(-budget // 16) * 16
+    if bufs is None:
+        k = torch.empty((batch, budget_pad, h_kv, d), dtype=torch.bfloat16, device=k_cache.device)
+        bufs = (k, torch.empty_like(k), torch.empty((batch,), dtype=torch.int32, device=k_cache.device))
+    k, v, lens = bufs
+    if k.shape != (batch, budget_pad, h_kv, d) or v.shape != k.shape or lens.shape != (batch,):
+        raise ValueError("staging buffers of the wrong shape")
+    _need(k, "k", torch.bfloat16)
+    _need(v, "v", torch.bfloat16)
+    _need(lens, "lens", torch.int32)
+    call("jssa_gather_kv", k_cache.data_ptr(), v_cache.data_ptr(), *strides, block_table.data_ptr(),
+         block_table.shape[1], idx.data_ptr(), count.data_ptr(), batch, h_kv, d, budget, num_pages,
+         page_size, k.data_ptr(), v.data_ptr(), lens.data_ptr(), _stream(k_cache.device))
+    return k, v, lens
+
+
+def staged_pages(k: torch.Tensor, v: torch.Tensor):
+    """The staging buffers of :func:`gather_kv` viewed as a paged cache of 16-token pages, with
+    its block table (sequence b on its own consecutive pages)."""
+    batch, budget_pad, h_kv, d = k.shape
+    pages = budget_pad // 16
+    kc = k.view(batch * pages, 16, h_kv, d)
+    vc = v.view(batch * pages, 16, h_kv, d)
+    bt = torch.arange(batch * pages, dtype=torch.int32, device=k.device).view(batch, pages)
+    return kc, vc, bt
+
+
+def gather_then_attend(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                       block_table: torch.Tensor, idx: torch.Tensor, count: torch.Tensor,
+                       scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                       ws: Optional[Workspace] = None, bufs=None) -> torch.Tensor:
+    """The gather-then-attend ablation: copy the selected rows into staging buffers, then run
+    the dense paged decode over them (same result as :func:`indexed_attend`)."""
+    k, v, lens = gather_kv(k_cache, v_cache, block_table, idx, count, bufs)
+    kc, vc, bt = staged_pages(k, v)
+    return dense_decode(q, kc, vc, bt, lens, scale, -1, out, ws)
 
 
 def dense_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,

@@ -327,6 +327,27 @@ int jssa_dense_decode(const jssa_bf16* q, const jssa_bf16* k_cache, const jssa_b
   return cuda_status(jssa::launch_attend(a, false, plan, false, as_stream(stream)));
 }
 
+int jssa_gather_kv(const jssa_bf16* k_cache, const jssa_bf16* v_cache, int64_t kv_page_stride,
+                   int64_t kv_slot_stride, int64_t kv_head_stride, const int32_t* block_table,
+                   int max_pages, const int32_t* idx, const int32_t* count, int batch, int h_kv,
+                   int d, int budget, int64_t num_pages, int page_size, jssa_bf16* k_out,
+                   jssa_bf16* v_out, int32_t* lens_out, jssa_stream_t stream) {
+  if (batch < 0 || h_kv <= 0 || budget <= 0) return JSSA_ERR_SHAPE;
+  if (!supported_d(d)) return JSSA_ERR_UNSUPPORTED;
+  int st = check_paging(max_pages, num_pages, page_size);
+  if (st) return st;
+  if (batch == 0) return JSSA_OK;
+  if (!block_table || !idx || !count || !k_out || !v_out || !lens_out) return JSSA_ERR_NULL;
+  if ((st = check_kv(k_cache, v_cache, kv_page_stride, kv_slot_stride, kv_head_stride, h_kv, d,
+                     page_size)))
+    return st;
+  if (!aligned16(k_out) || !aligned16(v_out)) return JSSA_ERR_ALIGN;
+  return cuda_status(jssa::launch_gather(k_cache, v_cache, kv_page_stride, kv_slot_stride,
+                                         kv_head_stride, block_table, max_pages, idx, count, batch,
+                                         h_kv, d, budget, num_pages, page_size, k_out, v_out,
+                                         lens_out, as_stream(stream)));
+}
+
 int jssa_decode(const jssa_bf16* q, const jssa_bf16* k_new, const jssa_bf16* v_new,
                 jssa_bf16* k_cache, jssa_bf16* v_cache, int64_t kv_page_stride,
                 int64_t kv_slot_stride, int64_t kv_head_stride, uint8_t* score_cache,

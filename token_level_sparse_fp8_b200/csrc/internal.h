@@ -85,6 +85,12 @@ struct AttendArgs {
 cudaError_t launch_attend(const AttendArgs& a, bool indexed, const AttendPlan& plan, bool pdl,
                           cudaStream_t s);
 
+cudaError_t launch_gather(const uint16_t* k_cache, const uint16_t* v_cache, int64_t page_stride,
+                          int64_t slot_stride, int64_t head_stride, const int32_t* block_table,
+                          int max_pages, const int32_t* idx, const int32_t* count, int batch,
+                          int h_kv, int d, int budget, int64_t num_pages, int page_size,
+                          uint16_t* k_out, uint16_t* v_out, int32_t* lens_out, cudaStream_t s);
+
 cudaError_t launch_gram(const uint16_t* q, int64_t q_stride, const uint16_t* k, int64_t k_stride,
                         int n, int h_q, int h_kv, int d, double* gram_q, double* gram_k,
                         cudaStream_t s);

@@ -4,6 +4,7 @@
 #include "store.cu"
 #include "score_topk.cu"
 #include "attend.cu"
+#include "gather.cu"
 #include "calib.cu"
 #include "basis.cu"
 #include "noalloc.cu"
