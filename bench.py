@@ -500,6 +500,26 @@ def run_jssa(args):
     t_attend, n_attend = timed_graph(attend_only, args.steps, args.warmup, stream, barrier, nq)
     t_attend = max_over_ranks(t_attend) / n_attend
 
+    # the scoring-cache ablation: the same scores from a bf16 cache (twice the bytes)
+    t_score_bf16 = None
+    if w.rank == 32 and w.d == 128:
+        num_pages, page_size = layer.k_cache.shape[0], layer.k_cache.shape[1]
+        sc16 = torch.empty((num_pages, w.h_kv, page_size, w.rank), dtype=torch.bfloat16, device=dev)
+        flat = layer.k_cache.view(num_pages * page_size, w.h_kv, w.d)
+        for p0 in range(0, num_pages, 4096):
+            p1 = min(num_pages, p0 + 4096)
+            slots = torch.arange(p0 * page_size, p1 * page_size, dtype=torch.int64, device=dev)
+            J.store(flat[p0 * page_size:p1 * page_size], slots, layer.basis, sc16)
+        idx16, count16 = torch.empty_like(idx), torch.empty_like(count)
+
+        def score_bf16(i):
+            J.score_topk(qs[i % nq], layer.basis, sc16, layer.block_table, layer.seq_lens, w.budget,
+                         idx16, count16, ws_score)
+
+        t_score_bf16, n16 = timed_graph(score_bf16, args.steps, args.warmup, stream, barrier, nq)
+        t_score_bf16 = max_over_ranks(t_score_bf16) / n16
+        del sc16
+
     # the ablation: gather the same index sets into staging buffers, then dense attention there
     ws_gta = J.Workspace(dev)
     bufs = J.gather_kv(layer.k_cache, layer.v_cache, layer.block_table, sets[0][0], sets[0][1])
@@ -599,6 +619,14 @@ def run_jssa(args):
         line["dense"] = {"steps_per_s": world / t_dense, "ms_per_step": t_dense * 1e3,
                          "hbm_gbs": dense_bytes / t_dense / 1e9, "frac": dense_bytes / t_dense / 1e9 / peak}
         line["speedup_vs_dense"] = t_dense / (ms_step / 1e3)
+    if t_score_bf16 is not None:
+        bytes16 = score_bytes(w) + w.batch * w.h_kv * w.seq_len * w.rank  # codes twice as wide
+        line["ablation_bf16_cache"] = {
+            "score_topk_ms_fp8": score_launch_s * 1e3, "score_topk_ms_bf16": t_score_bf16 * 1e3,
+            "bf16_over_fp8_time": t_score_bf16 / score_launch_s,
+            "bytes_fp8": score_bytes(w), "bytes_bf16": bytes16,
+            "bf16_gbs": bytes16 / t_score_bf16 / 1e9,
+        }
     line["ablation_gather"] = {
         "gather_free_attend_ms": t_attend * 1e3,
         "gather_then_attend_ms": t_gta * 1e3,

@@ -203,6 +203,26 @@ JSSA_API int jssa_dense_decode(const jssa_bf16* q, const jssa_bf16* k_cache, con
                       size_t ws_bytes, jssa_stream_t stream);
 
 /*
+ * BF16 scoring-cache ablation (JSSA README, section 4 notes, and JSSA summary, section 3.4: the
+ * method keeps the projected keys in FP8; these two entry points keep them in bf16, two bytes per
+ * dimension, to measure that choice). jssa_store_bf16 is jssa_store writing bf16(M_h k) (float64
+ * dot product, one correct rounding) into score_cache bf16 [num_pages, h_kv, page_size, r];
+ * jssa_score_topk_bf16 is jssa_score_topk reading that cache (the scores multiply the bf16 codes
+ * by four bf16 digits of p). Only d = 128, r = 32 (JSSA_ERR_UNSUPPORTED otherwise). Same
+ * arguments, layouts, workspace and errors as the FP8 entry points.
+ */
+JSSA_API int jssa_store_bf16(const jssa_bf16* k, int64_t k_stride_t, const int64_t* slot_mapping,
+                             int t, int h_kv, int d, int r, const float* basis,
+                             jssa_bf16* score_cache, int64_t num_pages, int page_size,
+                             jssa_stream_t stream);
+JSSA_API int jssa_score_topk_bf16(const jssa_bf16* q, const float* basis,
+                                  const jssa_bf16* score_cache, const int32_t* block_table,
+                                  int max_pages, const int32_t* seq_lens, int batch, int h_q,
+                                  int h_kv, int d, int r, int64_t num_pages, int page_size,
+                                  int budget, int32_t* idx, int32_t* count, void* ws,
+                                  size_t ws_bytes, jssa_stream_t stream);
+
+/*
  * Gather-then-attend ablation, step 1: copy the selected K and V rows of every (sequence, KV
  * head), in index order, into contiguous staging buffers (JSSA README, "Highlights" and section
  * 3: the gather-free attention is measured against gathering the selected rows first; JSSA

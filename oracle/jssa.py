@@ -27,6 +27,7 @@ from __future__ import annotations
 
 import numpy as np
 
+from .bf16 import bf16_decode, bf16_encode
 from .fp8 import e4m3_decode, e4m3_encode
 
 # ---------------------------------------------------------------------------------------------
@@ -136,6 +137,19 @@ def store_codes(k: np.ndarray, m: np.ndarray) -> np.ndarray:
     return e4m3_encode(y)
 
 
+def store_codes_bf16(k: np.ndarray, m: np.ndarray) -> np.ndarray:
+    """The scoring-cache ablation: ``bf16(M k)`` (float64 product, one rounding) instead of the
+    E4M3 code of :func:`store_codes`. ``k``: ``[T, d]``, ``m``: ``[r, d]`` -> ``uint16 [T, r]``
+    bit patterns."""
+    y = np.asarray(k, dtype=np.float64) @ np.asarray(m, dtype=np.float64).T
+    return bf16_encode(y)
+
+
+def scores_bf16(codes: np.ndarray, p: np.ndarray) -> np.ndarray:
+    """:func:`scores` over a bf16 scoring cache: ``s_t = sum_j bf16(c_tj) p_j``."""
+    return bf16_decode(codes) @ np.asarray(p, dtype=np.float64)
+
+
 def projected_query(qbar: np.ndarray, m: np.ndarray) -> np.ndarray:
     """``p = M q_bar`` (JSSA summary, eq. (1): ``s_hat = q_bar^T P k = (M q_bar) . (M k)``)."""
     return np.asarray(m, dtype=np.float64) @ np.asarray(qbar, dtype=np.float64)
@@ -222,7 +236,9 @@ def select_step(q: np.ndarray, m: np.ndarray, score_cache: np.ndarray, block_tab
                 seq_lens: np.ndarray, budget: int) -> tuple:
     """Per-(sequence, KV head) index sets for one decode step: group-mean query, projection,
     scores over every cached token, top-B. Returns ``idx int32 [batch, h_kv, budget]`` (ascending,
-    -1 padded), ``count int32 [batch, h_kv]`` and the float64 scores per (b, h) as a dict."""
+    -1 padded), ``count int32 [batch, h_kv]`` and the float64 scores per (b, h) as a dict.
+    A ``uint16`` scoring cache holds bf16 codes (the ablation), a ``uint8`` one E4M3 codes."""
+    score = scores_bf16 if np.asarray(score_cache).dtype == np.uint16 else scores
     batch = q.shape[0]
     h_kv = m.shape[0]
     idx = np.full((batch, h_kv, budget), -1, dtype=np.int32)
@@ -232,8 +248,8 @@ def select_step(q: np.ndarray, m: np.ndarray, score_cache: np.ndarray, block_tab
     for b in range(batch):
         L = int(seq_lens[b])
         for h in range(h_kv):
-            s = scores(scoring_rows(score_cache, block_table, b, h, L),
-                       projected_query(qbar[b, h], m[h]))
+            s = score(scoring_rows(score_cache, block_table, b, h, L),
+                      projected_query(qbar[b, h], m[h]))
             sel = select_top_b(s, budget)
             idx[b, h, : sel.shape[0]] = sel
             count[b, h] = sel.shape[0]

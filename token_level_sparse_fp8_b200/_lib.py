@@ -43,6 +43,9 @@ SIGNATURES = {
                                     c_int, c_int, c_int, c_int64, c_int, c_float, P, P, c_size_t, P]),
     "jssa_dense_decode": (c_int, [P, P, P, c_int64, c_int64, c_int64, P, c_int, P, c_int, c_int, c_int,
                                   c_int, c_int64, c_int, c_int, c_float, P, P, c_size_t, P]),
+    "jssa_store_bf16": (c_int, [P, c_int64, P, c_int, c_int, c_int, c_int, P, P, c_int64, c_int, P]),
+    "jssa_score_topk_bf16": (c_int, [P, P, P, P, c_int, P, c_int, c_int, c_int, c_int, c_int,
+                                     c_int64, c_int, c_int, P, P, P, c_size_t, P]),
     "jssa_gather_kv": (c_int, [P, P, c_int64, c_int64, c_int64, P, c_int, P, P, c_int, c_int, c_int,
                                c_int, c_int64, c_int, P, P, P, P]),
     "jssa_decode": (c_int, [P, P, P, P, P, c_int64, c_int64, c_int64, P, P, P, c_int, P, c_int, c_int,

@@ -154,27 +154,32 @@ def store(k: torch.Tensor, slot_mapping: torch.Tensor, basis: torch.Tensor,
           score_cache: torch.Tensor) -> None:
     """Write ``e4m3(M_h k)`` of each token ``k[t]`` (bf16 ``[t, h_kv, d]``) at flat slot
     ``slot_mapping[t]`` (int64; negative = skip) of the scoring cache
-    (uint8 ``[num_pages, h_kv, page_size, r]``)."""
+    (uint8 ``[num_pages, h_kv, page_size, r]``; a bfloat16 cache of that shape holds
+    ``bf16(M_h k)`` instead, the scoring-cache ablation)."""
     _need(k, "k", torch.bfloat16, contiguous=False)
     _need(slot_mapping, "slot_mapping", torch.int64)
     _need(basis, "basis", torch.float32)
-    _need(score_cache, "score_cache", torch.uint8)
+    bf16 = score_cache.dtype == torch.bfloat16
+    _need(score_cache, "score_cache", torch.bfloat16 if bf16 else torch.uint8)
     t, h_kv, d = k.shape
     num_pages, _, page_size, r = score_cache.shape
     if k.stride(2) != 1 or k.stride(1) != d:
         raise ValueError("k rows must be [h_kv, d] contiguous")
-    call("jssa_store", k.data_ptr(), k.stride(0), slot_mapping.data_ptr(), t, h_kv, d, r,
-         basis.data_ptr(), score_cache.data_ptr(), num_pages, page_size, _stream(k.device))
+    call("jssa_store_bf16" if bf16 else "jssa_store", k.data_ptr(), k.stride(0),
+         slot_mapping.data_ptr(), t, h_kv, d, r, basis.data_ptr(), score_cache.data_ptr(),
+         num_pages, page_size, _stream(k.device))
 
 
 def score_topk(q: torch.Tensor, basis: torch.Tensor, score_cache: torch.Tensor,
                block_table: torch.Tensor, seq_lens: torch.Tensor, budget: int,
                idx: Optional[torch.Tensor] = None, count: Optional[torch.Tensor] = None,
                ws: Optional[Workspace] = None):
-    """Index sets ``idx`` (int32 ``[batch, h_kv, budget]``, ascending, -1 padded) and ``count``."""
+    """Index sets ``idx`` (int32 ``[batch, h_kv, budget]``, ascending, -1 padded) and ``count``.
+    A bfloat16 ``score_cache`` selects the bf16 scoring-cache ablation."""
+    bf16 = score_cache.dtype == torch.bfloat16
     for t, n, dt in ((q, "q", torch.bfloat16), (basis, "basis", torch.float32),
-                     (score_cache, "score_cache", torch.uint8), (block_table, "block_table", torch.int32),
-                     (seq_lens, "seq_lens", torch.int32)):
+                     (score_cache, "score_cache", torch.bfloat16 if bf16 else torch.uint8),
+                     (block_table, "block_table", torch.int32), (seq_lens, "seq_lens", torch.int32)):
         _need(t, n, dt)
     batch, h_q, d = q.shape
     h_kv, r, _ = basis.shape
@@ -186,7 +191,8 @@ def score_topk(q: torch.Tensor, basis: torch.Tensor, score_cache: torch.Tensor,
     max_pages = block_table.shape[1]
     w = _ws(q.device, ws, FN_SCORE_TOPK)
     p, n = w.get(workspace_size(FN_SCORE_TOPK, batch, h_q, h_kv, d, max_pages, page_size, budget))
-    call("jssa_score_topk", q.data_ptr(), basis.data_ptr(), score_cache.data_ptr(),
+    call("jssa_score_topk_bf16" if bf16 else "jssa_score_topk", q.data_ptr(), basis.data_ptr(),
+         score_cache.data_ptr(),
          block_table.data_ptr(), max_pages, seq_lens.data_ptr(), batch, h_q, h_kv, d, r,
          num_pages, page_size, budget, idx.data_ptr(), count.data_ptr(), p, n, _stream(q.device))
     return idx, count

@@ -207,19 +207,34 @@ int jssa_compute_basis(const double* gram_q, const double* gram_k, int h_kv, int
                                         static_cast<double*>(ws), as_stream(stream)));
 }
 
-int jssa_store(const jssa_bf16* k, int64_t k_stride_t, const int64_t* slot_mapping, int t,
-               int h_kv, int d, int r, const float* basis, uint8_t* score_cache,
-               int64_t num_pages, int page_size, jssa_stream_t stream) {
+static int store_codes(const jssa_bf16* k, int64_t k_stride_t, const int64_t* slot_mapping, int t,
+                       int h_kv, int d, int r, const float* basis, void* score_cache,
+                       int64_t num_pages, int page_size, jssa_stream_t stream, bool bf16) {
   if (t < 0 || h_kv <= 0 || num_pages <= 0 || page_size <= 0) return JSSA_ERR_SHAPE;
   if (page_size & (page_size - 1)) return JSSA_ERR_UNSUPPORTED;
   if (r <= 0 || r > d) return JSSA_ERR_SHAPE;
-  if (!supported_dr(d, r)) return JSSA_ERR_UNSUPPORTED;
+  if (bf16 ? !(d == 128 && r == 32) : !supported_dr(d, r)) return JSSA_ERR_UNSUPPORTED;
   if (t == 0) return JSSA_OK;
   if (!k || !slot_mapping || !basis || !score_cache) return JSSA_ERR_NULL;
   if (!aligned16(k) || (k_stride_t & 7) || !aligned16(score_cache)) return JSSA_ERR_ALIGN;
   if (k_stride_t < (int64_t)h_kv * d) return JSSA_ERR_SHAPE;
   return cuda_status(jssa::launch_store(k, k_stride_t, slot_mapping, t, h_kv, d, r, basis,
-                                        score_cache, num_pages, page_size, as_stream(stream)));
+                                        static_cast<uint8_t*>(score_cache), num_pages, page_size,
+                                        as_stream(stream), bf16));
+}
+
+int jssa_store(const jssa_bf16* k, int64_t k_stride_t, const int64_t* slot_mapping, int t,
+               int h_kv, int d, int r, const float* basis, uint8_t* score_cache,
+               int64_t num_pages, int page_size, jssa_stream_t stream) {
+  return store_codes(k, k_stride_t, slot_mapping, t, h_kv, d, r, basis, score_cache, num_pages,
+                     page_size, stream, false);
+}
+
+int jssa_store_bf16(const jssa_bf16* k, int64_t k_stride_t, const int64_t* slot_mapping, int t,
+                    int h_kv, int d, int r, const float* basis, jssa_bf16* score_cache,
+                    int64_t num_pages, int page_size, jssa_stream_t stream) {
+  return store_codes(k, k_stride_t, slot_mapping, t, h_kv, d, r, basis, score_cache, num_pages,
+                     page_size, stream, true);
 }
 
 static int check_score_args(const jssa_bf16* q, const float* basis, const uint8_t* score_cache,
@@ -256,6 +271,25 @@ int jssa_score_topk(const jssa_bf16* q, const float* basis, const uint8_t* score
                                              seq_lens, batch, h_q, h_kv, d, r, num_pages,
                                              page_size, budget, idx, count, ws, nullptr,
                                              nullptr, true, as_stream(stream)));
+}
+
+int jssa_score_topk_bf16(const jssa_bf16* q, const float* basis, const jssa_bf16* score_cache,
+                         const int32_t* block_table, int max_pages, const int32_t* seq_lens,
+                         int batch, int h_q, int h_kv, int d, int r, int64_t num_pages,
+                         int page_size, int budget, int32_t* idx, int32_t* count, void* ws,
+                         size_t ws_bytes, jssa_stream_t stream) {
+  const uint8_t* sc = reinterpret_cast<const uint8_t*>(score_cache);
+  int st = check_score_args(q, basis, sc, block_table, max_pages, seq_lens, batch, h_q, h_kv, d,
+                            r, num_pages, page_size, budget, idx, count);
+  if (st || batch == 0) return st;
+  if (!(d == 128 && r == 32)) return JSSA_ERR_UNSUPPORTED;
+  const size_t need = score_ws_bytes(batch, h_kv, max_pages * page_size, page_size);
+  if (!ws || ws_bytes < need) return JSSA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return JSSA_ERR_ALIGN;
+  return cuda_status(jssa::launch_score_topk(q, basis, sc, block_table, max_pages, seq_lens,
+                                             batch, h_q, h_kv, d, r, num_pages, page_size, budget,
+                                             idx, count, ws, nullptr, nullptr, true,
+                                             as_stream(stream), true));
 }
 
 static int check_attend_common(const jssa_bf16* q, const jssa_bf16* k_cache,

@@ -97,6 +97,13 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
+// float64 -> bf16 bits with a single correct rounding (nearest, ties to even), by the same
+// round-to-odd narrowing to float first (float keeps 16 more bits than bf16).
+__device__ __forceinline__ uint16_t f64_to_bf16(double y) {
+  float f = __double2float_rz(y);
+  if ((double)f != y) f = __uint_as_float(__float_as_uint(f) | 1u);
+  return f_to_bf16(f);
+}
 
 // ---------------------------------------------------------------------------------------------
 // Warp-level tensor core fragments (bf16 in, fp32 accumulate)

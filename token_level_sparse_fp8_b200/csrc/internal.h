@@ -45,7 +45,8 @@ AttendPlan plan_attend(int pairs, int positions, int group, int d);
 
 cudaError_t launch_store(const uint16_t* k, int64_t k_stride_t, const int64_t* slot_mapping,
                          int t, int h_kv, int d, int r, const float* basis, uint8_t* score_cache,
-                         int64_t num_pages, int page_size, cudaStream_t s);
+                         int64_t num_pages, int page_size, cudaStream_t s,
+                         bool bf16_codes = false);
 
 // Decode-time store: token b writes position seq_lens[b]-1 (K/V rows and scoring code).
 cudaError_t launch_store_decode(const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_cache,
@@ -60,7 +61,7 @@ cudaError_t launch_score_topk(const uint16_t* q, const float* basis, const uint8
                               int batch, int h_q, int h_kv, int d, int r, int64_t num_pages,
                               int page_size, int budget, int32_t* idx, int32_t* count,
                               void* ws, int* attend_tickets, const StoreNew* store, bool pdl,
-                              cudaStream_t s);
+                              cudaStream_t s, bool bf16_codes = false);
 
 struct AttendArgs {
   const uint16_t* q;

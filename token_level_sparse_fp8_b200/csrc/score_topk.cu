@@ -38,7 +38,6 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kUnrollBytes = 32;   // bytes of scoring rows per lane per load batch
 constexpr int kBins = 2048;
-constexpr int kDigits = 2;         // f16 digit vectors of p (B columns 2t and 2t + 1 of lane t)
 constexpr int kSample = 2048;      // sampled positions per (sequence, KV head)
 constexpr int kExactMax = 16384;   // up to this context every token is a candidate
 constexpr int kSelectCap = 16384;  // candidates the select kernel stages in shared memory
@@ -47,6 +46,19 @@ constexpr int kMaxRegions = 4096;  // candidate regions per (sequence, KV head)
 constexpr int kPrepBytes = 1024;   // per (sequence, KV head): digits, scales, threshold, mode
 constexpr int kPrepScale = 512, kPrepThr = 544, kPrepMode = 548, kPrepKmax = 552;
 constexpr int kModeScan = 0, kModeAll = 1;
+
+// Scoring-cache code format: E4M3, one byte per projected dimension (the method's cache), or
+// BF16, two bytes (the ablation the FP8 choice is compared with; JSSA README, section 4 notes,
+// and JSSA summary, section 3.4). A row of R codes is split over the 4 lanes of a quad.
+template <int R_, bool BF16_>
+struct Codes {
+  static constexpr int R = R_;
+  static constexpr bool kBF16 = BF16_;
+  static constexpr int kBytes = BF16_ ? 2 * R_ : R_;  // per token
+  static constexpr int kLaneBytes = kBytes / 4;        // one lane's share of a row
+  static constexpr int kRegs = kLaneBytes / 4;         // 32-bit registers per row per lane
+  static constexpr int kDigits = BF16_ ? 4 : 2;        // digit vectors of p
+};
 
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t x, int lane) {
 #pragma unroll
@@ -426,75 +438,93 @@ __device__ __forceinline__ uint32_t mix32(uint32_t x) {
   return x;
 }
 
-// Fragment registers of the digit matrix (B operand of mma m16n8k16, f16). Column n holds digit
-// n & 1 (the two digits repeated four times), so lane (g, t) finds the complete digit-0 and
-// digit-1 sums of its rows in accumulator columns 2t and 2t + 1. K-slots are permuted so that
-// each lane's MMA operands come from its own code bytes: in k-block kb (16 slots), slots
-// 2t, 2t+1, 2t+8, 2t+9 <-> bytes t*LB + 4kb + 0..3 of the row (LB = R / 4 bytes per lane); the
-// same permutation on both operands leaves the dot products unchanged.
-template <int R>
+// Fragment registers of the digit matrix (B operand of mma m16n8k16: f16 digits for E4M3 codes,
+// bf16 digits for BF16 codes). Column n holds digit n & 1 (the two digits repeated four times;
+// BF16 codes use a second set for digits 2 and 3), so lane (g, t) finds the complete digit sums
+// of its rows in accumulator columns 2t and 2t + 1. K-slots are permuted so that each lane's MMA
+// operands come from its own code bytes: in k-block kb (16 slots), slots 2t, 2t+1, 2t+8, 2t+9
+// <-> dimensions t*R/4 + 4kb + 0..3 of the row; the same permutation on both operands leaves the
+// dot products unchanged.
+template <class C>
 struct DigitFrags {
-  uint32_t b0[R / 16], b1[R / 16];
-  float sc0, sc1;
-  // dig: f16 [kDigits][R]; scale: the power-of-two weight of each digit
+  static constexpr int R = C::R, KB = R / 16;
+  uint32_t b0[KB], b1[KB];                              // digits 0 and 1
+  uint32_t b2[C::kBF16 ? KB : 1], b3[C::kBF16 ? KB : 1];  // digits 2 and 3 (BF16 codes)
+  float sc[C::kDigits];
+  // dig: 16-bit digits [kDigits][R]; scale: the power-of-two weight of each digit
   __device__ __forceinline__ void load(const uint16_t* dig, const float* scale, int lane) {
-    constexpr int LB = R / 4;
+    constexpr int LD = R / 4;  // dimensions per lane
     const int g = lane >> 2, t = lane & 3;
     const uint16_t* d = dig + (g & 1) * R;
 #pragma unroll
-    for (int kb = 0; kb < R / 16; ++kb) {
-      const int o = t * LB + 4 * kb;
+    for (int kb = 0; kb < KB; ++kb) {
+      const int o = t * LD + 4 * kb;
       b0[kb] = (uint32_t)d[o] | ((uint32_t)d[o + 1] << 16);
       b1[kb] = (uint32_t)d[o + 2] | ((uint32_t)d[o + 3] << 16);
+      if (C::kBF16) {
+        const uint16_t* d2 = d + 2 * R;
+        b2[kb] = (uint32_t)d2[o] | ((uint32_t)d2[o + 1] << 16);
+        b3[kb] = (uint32_t)d2[o + 2] | ((uint32_t)d2[o + 3] << 16);
+      }
     }
-    sc0 = scale[0];
-    sc1 = scale[1];
+#pragma unroll
+    for (int c = 0; c < C::kDigits; ++c) sc[c] = scale[c];
   }
 };
 
-template <int R>
+// A lane's LB code bytes of one row: from shared memory through a generic pointer, from shared
+// memory by shared-window address, and from global memory (streamed, no L1 allocation).
+template <int LB>
 __device__ __forceinline__ void load_srow(uint32_t* dst, const uint8_t* src) {
-  if (R == 32) {
+  if (LB == 8) {
     const uint2 v = *reinterpret_cast<const uint2*>(src);
     dst[0] = v.x;
     dst[1] = v.y;
   } else {
-    const uint4 v = *reinterpret_cast<const uint4*>(src);
-    dst[0] = v.x;
-    dst[1] = v.y;
-    dst[2] = v.z;
-    dst[3] = v.w;
+#pragma unroll
+    for (int i = 0; i < LB / 16; ++i) {
+      const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * i);
+      dst[4 * i] = v.x;
+      dst[4 * i + 1] = v.y;
+      dst[4 * i + 2] = v.z;
+      dst[4 * i + 3] = v.w;
+    }
   }
 }
 
-// A lane's R / 4 code bytes of one row from shared memory (shared-window address).
-template <int R>
+template <int LB>
 __device__ __forceinline__ void lds_row(uint32_t* dst, uint32_t saddr) {
-  if (R == 32) {
+  if (LB == 8) {
     asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
                  : "=r"(dst[0]), "=r"(dst[1])
                  : "r"(saddr)
                  : "memory");
   } else {
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(dst[0]), "=r"(dst[1]), "=r"(dst[2]), "=r"(dst[3])
-                 : "r"(saddr)
-                 : "memory");
+#pragma unroll
+    for (int i = 0; i < LB / 16; ++i)
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(dst[4 * i]), "=r"(dst[4 * i + 1]), "=r"(dst[4 * i + 2]),
+                     "=r"(dst[4 * i + 3])
+                   : "r"(saddr + 16 * i)
+                   : "memory");
   }
 }
 
-template <int R>
+template <int LB>
 __device__ __forceinline__ void load_row(uint32_t* dst, const uint8_t* src) {
-  if (R == 32) {
+  if (LB == 8) {
     const uint2 v = ld_stream_v2(src);
     dst[0] = v.x;
     dst[1] = v.y;
   } else {
-    const uint4 v = ld_stream_v4(src);
-    dst[0] = v.x;
-    dst[1] = v.y;
-    dst[2] = v.z;
-    dst[3] = v.w;
+#pragma unroll
+    for (int i = 0; i < LB / 16; ++i) {
+      const uint4 v = ld_stream_v4(src + 16 * i);
+      dst[4 * i] = v.x;
+      dst[4 * i + 1] = v.y;
+      dst[4 * i + 2] = v.z;
+      dst[4 * i + 3] = v.w;
+    }
   }
 }
 
@@ -525,10 +555,11 @@ struct ChunkGeom {
   int start;                 // first position of the chunk
 };
 
-template <int R>
+template <class C>
 struct ScanBuf {
-  static constexpr int kUnroll = kUnrollBytes / (R / 4);  // tiles per batch (even)
-  uint32_t ra[kUnroll][R / 16], rb[kUnroll][R / 16];
+  // tiles per batch (even)
+  static constexpr int kUnroll = kUnrollBytes / C::kLaneBytes > 2 ? kUnrollBytes / C::kLaneBytes : 2;
+  uint32_t ra[kUnroll][C::kRegs], rb[kUnroll][C::kRegs];
   uint32_t ok;  // bit u: tile u is inside the run and the chunk and its page is usable
 };
 
@@ -536,63 +567,79 @@ struct ScanBuf {
 // unconditional: a tile past t_end or the chunk's valid tokens, or on an unusable page, reads
 // page 0 instead (always allocated) and its tokens are never candidates (see scan_emit).
 // BIG: pages of at least 16 tokens, so a tile lies inside one page.
-template <int R, bool BIG>
-__device__ __forceinline__ void scan_load(ScanBuf<R>& buf, const ChunkGeom& cg,
+template <class C, bool BIG>
+__device__ __forceinline__ void scan_load(ScanBuf<C>& buf, const ChunkGeom& cg,
                                           const int32_t* s_page, int t0, int t_end, int lane) {
-  constexpr int LB = R / 4;
+  constexpr int LB = C::kLaneBytes, RB = C::kBytes;
   const int g = lane >> 2, t = lane & 3;
   const int pmask = (1 << cg.page_shift) - 1;
   if (BIG) {
-    const int lane_off = g * R + t * LB;
+    const int lane_off = g * RB + t * LB;
     buf.ok = 0u;
 #pragma unroll
-    for (int u = 0; u < ScanBuf<R>::kUnroll; ++u) {
+    for (int u = 0; u < ScanBuf<C>::kUnroll; ++u) {
       const int tok0 = (t0 + u) * 16;
       const int pg = t0 + u < t_end && tok0 < cg.n_local ? s_page[tok0 >> cg.page_shift] : -1;
       buf.ok |= (uint32_t)(pg >= 0) << u;
       const uint8_t* row = cg.head_base + (size_t)(uint32_t)max(pg, 0) * cg.page_bytes +
-                           ((tok0 & pmask) * R + lane_off);
-      load_row<R>(buf.ra[u], row);
-      load_row<R>(buf.rb[u], row + 8 * R);
+                           ((tok0 & pmask) * RB + lane_off);
+      load_row<LB>(buf.ra[u], row);
+      load_row<LB>(buf.rb[u], row + 8 * RB);
     }
   } else {
     buf.ok = ~0u;  // token validity is checked per token at emission
 #pragma unroll
-    for (int u = 0; u < ScanBuf<R>::kUnroll; ++u) {
+    for (int u = 0; u < ScanBuf<C>::kUnroll; ++u) {
       const bool live = t0 + u < t_end;
       const int ta = (t0 + u) * 16 + g, tb = ta + 8;
       const int pa = live && ta < cg.n_local ? s_page[ta >> cg.page_shift] : 0;
       const int pb = live && tb < cg.n_local ? s_page[tb >> cg.page_shift] : 0;
-      load_row<R>(buf.ra[u], cg.head_base + (size_t)(uint32_t)max(pa, 0) * cg.page_bytes +
-                                 ((ta & pmask) * R + t * LB));
-      load_row<R>(buf.rb[u], cg.head_base + (size_t)(uint32_t)max(pb, 0) * cg.page_bytes +
-                                 ((tb & pmask) * R + t * LB));
+      load_row<LB>(buf.ra[u], cg.head_base + (size_t)(uint32_t)max(pa, 0) * cg.page_bytes +
+                                  ((ta & pmask) * RB + t * LB));
+      load_row<LB>(buf.rb[u], cg.head_base + (size_t)(uint32_t)max(pb, 0) * cg.page_bytes +
+                                  ((tb & pmask) * RB + t * LB));
     }
   }
 }
 
 // Scores of two 16-token tiles, one token per lane: lane (g, t) returns token
 // 16 * (t >> 1) + 8 * (t & 1) + g of the pair. ra / rb hold the lane's code bytes of rows g and
-// g + 8 (R / 4 bytes each); the codes are widened to f16 (exact) and multiplied on the tensor
-// cores with fp32 accumulation, s = 2^e0 C[:, 0] + 2^e1 C[:, 1].
-template <int R>
+// g + 8 (a quarter of a row each). E4M3 codes are widened to f16 (exact) and multiplied by the
+// f16 digits, BF16 codes are multiplied as they are by the bf16 digits, on the tensor cores with
+// fp32 accumulation: s = sum_c 2^-e_c C_c (c over the digits).
+template <class C>
 __device__ __forceinline__ float pair_scores(const uint32_t* ra0, const uint32_t* rb0,
                                              const uint32_t* ra1, const uint32_t* rb1,
-                                             const DigitFrags<R>& df, int t) {
+                                             const DigitFrags<C>& df, int t) {
+  constexpr int KB = C::R / 16;
   float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+  float e0[4] = {0.f, 0.f, 0.f, 0.f}, e1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int kb = 0; kb < R / 16; ++kb) {
-    mma_f16(c0, e4m3x2_to_f16x2((uint16_t)ra0[kb]), e4m3x2_to_f16x2((uint16_t)rb0[kb]),
-            e4m3x2_to_f16x2((uint16_t)(ra0[kb] >> 16)), e4m3x2_to_f16x2((uint16_t)(rb0[kb] >> 16)),
-            df.b0[kb], df.b1[kb]);
-    mma_f16(c1, e4m3x2_to_f16x2((uint16_t)ra1[kb]), e4m3x2_to_f16x2((uint16_t)rb1[kb]),
-            e4m3x2_to_f16x2((uint16_t)(ra1[kb] >> 16)), e4m3x2_to_f16x2((uint16_t)(rb1[kb] >> 16)),
-            df.b0[kb], df.b1[kb]);
+  for (int kb = 0; kb < KB; ++kb) {
+    if (C::kBF16) {
+      mma_bf16(c0, ra0[2 * kb], rb0[2 * kb], ra0[2 * kb + 1], rb0[2 * kb + 1], df.b0[kb], df.b1[kb]);
+      mma_bf16(c1, ra1[2 * kb], rb1[2 * kb], ra1[2 * kb + 1], rb1[2 * kb + 1], df.b0[kb], df.b1[kb]);
+      mma_bf16(e0, ra0[2 * kb], rb0[2 * kb], ra0[2 * kb + 1], rb0[2 * kb + 1], df.b2[kb], df.b3[kb]);
+      mma_bf16(e1, ra1[2 * kb], rb1[2 * kb], ra1[2 * kb + 1], rb1[2 * kb + 1], df.b2[kb], df.b3[kb]);
+    } else {
+      mma_f16(c0, e4m3x2_to_f16x2((uint16_t)ra0[kb]), e4m3x2_to_f16x2((uint16_t)rb0[kb]),
+              e4m3x2_to_f16x2((uint16_t)(ra0[kb] >> 16)), e4m3x2_to_f16x2((uint16_t)(rb0[kb] >> 16)),
+              df.b0[kb], df.b1[kb]);
+      mma_f16(c1, e4m3x2_to_f16x2((uint16_t)ra1[kb]), e4m3x2_to_f16x2((uint16_t)rb1[kb]),
+              e4m3x2_to_f16x2((uint16_t)(ra1[kb] >> 16)), e4m3x2_to_f16x2((uint16_t)(rb1[kb] >> 16)),
+              df.b0[kb], df.b1[kb]);
+    }
   }
   const bool hi_row = t & 1, tile1 = t & 2;
   const float x0 = hi_row ? c0[2] : c0[0], y0 = hi_row ? c0[3] : c0[1];
   const float x1 = hi_row ? c1[2] : c1[0], y1 = hi_row ? c1[3] : c1[1];
-  return (tile1 ? x1 : x0) * df.sc0 + (tile1 ? y1 : y0) * df.sc1;
+  float f = (tile1 ? x1 : x0) * df.sc[0] + (tile1 ? y1 : y0) * df.sc[1];
+  if (C::kBF16) {
+    const float u0 = hi_row ? e0[2] : e0[0], v0 = hi_row ? e0[3] : e0[1];
+    const float u1 = hi_row ? e1[2] : e1[0], v1 = hi_row ? e1[3] : e1[1];
+    f += (tile1 ? u1 : u0) * df.sc[C::kDigits - 2] + (tile1 ? v1 : v0) * df.sc[C::kDigits - 1];
+  }
+  return f;
 }
 
 // The smallest float whose key is >= thr (keys of non-NaN floats are >= thr exactly when the
@@ -604,8 +651,8 @@ __device__ __forceinline__ float key_floor(uint32_t thr) {
 }
 
 // Keys >= thr of the tiles [t0, t0 + kUnroll) appended in position order to this warp's region.
-template <int R, bool BIG>
-__device__ __forceinline__ void scan_emit(const ScanBuf<R>& buf, const DigitFrags<R>& df,
+template <class C, bool BIG>
+__device__ __forceinline__ void scan_emit(const ScanBuf<C>& buf, const DigitFrags<C>& df,
                                           const ChunkGeom& cg, const int32_t* s_page, int t0,
                                           int t_end, float thr_f, uint32_t* rkey, int32_t* rpos,
                                           uint32_t& run, int lane) {
@@ -616,8 +663,8 @@ __device__ __forceinline__ void scan_emit(const ScanBuf<R>& buf, const DigitFrag
   const unsigned earlier_t = 0x11111111u * ((1u << t) - 1u);
   const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
-  for (int u = 0; u < ScanBuf<R>::kUnroll; u += 2) {
-    const float f = pair_scores<R>(buf.ra[u], buf.rb[u], buf.ra[u + 1], buf.rb[u + 1], df, t);
+  for (int u = 0; u < ScanBuf<C>::kUnroll; u += 2) {
+    const float f = pair_scores<C>(buf.ra[u], buf.rb[u], buf.ra[u + 1], buf.rb[u + 1], df, t);
     const int tok = (t0 + u) * 16 + tok_in_pair;
     bool c = f >= thr_f && tok < cg.n_local;
     if (BIG) {
@@ -639,49 +686,51 @@ __device__ __forceinline__ void scan_emit(const ScanBuf<R>& buf, const DigitFrag
 }
 
 // One warp's contiguous run of tiles [t_begin, t_end), register double-buffered.
-template <int R, bool BIG>
+template <class C, bool BIG>
 __device__ __forceinline__ uint32_t scan_warp(const ChunkGeom& cg, const int32_t* s_page,
-                                              const DigitFrags<R>& df, float thr_f, int t_begin,
+                                              const DigitFrags<C>& df, float thr_f, int t_begin,
                                               int t_end, uint32_t* rkey, int32_t* rpos, int lane) {
-  constexpr int kU = ScanBuf<R>::kUnroll;
+  constexpr int kU = ScanBuf<C>::kUnroll;
   uint32_t run = 0;
-  ScanBuf<R> a, b;
+  ScanBuf<C> a, b;
   int t0 = t_begin;
-  if (t0 < t_end) scan_load<R, BIG>(a, cg, s_page, t0, t_end, lane);
+  if (t0 < t_end) scan_load<C, BIG>(a, cg, s_page, t0, t_end, lane);
   while (t0 < t_end) {
-    if (t0 + kU < t_end) scan_load<R, BIG>(b, cg, s_page, t0 + kU, t_end, lane);
-    scan_emit<R, BIG>(a, df, cg, s_page, t0, t_end, thr_f, rkey, rpos, run, lane);
+    if (t0 + kU < t_end) scan_load<C, BIG>(b, cg, s_page, t0 + kU, t_end, lane);
+    scan_emit<C, BIG>(a, df, cg, s_page, t0, t_end, thr_f, rkey, rpos, run, lane);
     t0 += kU;
     if (t0 >= t_end) break;
-    if (t0 + kU < t_end) scan_load<R, BIG>(a, cg, s_page, t0 + kU, t_end, lane);
-    scan_emit<R, BIG>(b, df, cg, s_page, t0, t_end, thr_f, rkey, rpos, run, lane);
+    if (t0 + kU < t_end) scan_load<C, BIG>(a, cg, s_page, t0 + kU, t_end, lane);
+    scan_emit<C, BIG>(b, df, cg, s_page, t0, t_end, thr_f, rkey, rpos, run, lane);
     t0 += kU;
   }
   return run;
 }
 
-// The scan kernel's warps stream their tiles through a ring of scan_stages<R>() shared-memory
+// The scan kernel's warps stream their tiles through a ring of scan_stages<C>() shared-memory
 // stages (kUnroll tiles each) filled by asynchronous 16-byte copies, all but one stage ahead of
 // the one being scored: deeper than a register double buffer without holding the rows in
-// registers. At r = 32, three stages and four CTAs per SM; at r = 64, four stages and three.
-constexpr int kScanStageBytes = 2048;  // kUnroll tiles of 16 rows of r bytes
-template <int R>
-constexpr int scan_stages() { return R == 32 ? 3 : 4; }
-template <int R>
-constexpr int scan_ctas_per_sm() { return R == 32 ? 4 : 3; }
-template <int R>
-constexpr int scan_ring_bytes() { return kWarps * scan_stages<R>() * kScanStageBytes; }
+// registers. E4M3 at r = 32: three stages and four CTAs per SM; otherwise four stages and three.
+template <class C>
+constexpr int scan_stage_bytes() { return ScanBuf<C>::kUnroll * 16 * C::kBytes; }
+template <class C>
+constexpr int scan_stages() { return C::kBytes == 32 ? 3 : 4; }
+template <class C>
+constexpr int scan_ctas_per_sm() { return C::kBytes == 32 ? 4 : 3; }
+template <class C>
+constexpr int scan_ring_bytes() { return kWarps * scan_stages<C>() * scan_stage_bytes<C>(); }
 
 // Copies of tiles [t0, t0 + kUnroll) into the stage at shared address `dst`; returns the tiles'
 // ok bits (as scan_load). A tile past t_end or the chunk's valid tokens, or a row on an unusable
 // page, is zero-filled (its tokens are never candidates, see scan_emit).
-template <int R, bool BIG>
+template <class C, bool BIG>
 __device__ __forceinline__ uint32_t scan_issue(uint32_t dst, const ChunkGeom& cg,
                                                const int32_t* s_page, int t0, int t_end, int lane) {
-  constexpr int kU = ScanBuf<R>::kUnroll;
-  constexpr int kTileBytes = 16 * R;
+  constexpr int kU = ScanBuf<C>::kUnroll;
+  constexpr int RB = C::kBytes;
+  constexpr int kTileBytes = 16 * RB;
   constexpr int kPieces = kTileBytes / 512;  // 16-byte copies per lane per tile
-  static_assert(kU * kTileBytes == kScanStageBytes, "stage size");
+  static_assert(kU * kTileBytes == scan_stage_bytes<C>(), "stage size");
   const int pmask = (1 << cg.page_shift) - 1;
   uint32_t ok = BIG ? 0u : ~0u;
 #pragma unroll
@@ -692,7 +741,7 @@ __device__ __forceinline__ uint32_t scan_issue(uint32_t dst, const ChunkGeom& cg
       const int pg = live ? s_page[tok0 >> cg.page_shift] : -1;
       ok |= (uint32_t)(pg >= 0) << u;
       const uint8_t* tile = cg.head_base + (size_t)(uint32_t)max(pg, 0) * cg.page_bytes +
-                            (tok0 & pmask) * R;
+                            (tok0 & pmask) * RB;
 #pragma unroll
       for (int p = 0; p < kPieces; ++p) {
         const int o = (p * 32 + lane) * 16;
@@ -702,10 +751,10 @@ __device__ __forceinline__ uint32_t scan_issue(uint32_t dst, const ChunkGeom& cg
 #pragma unroll
       for (int p = 0; p < kPieces; ++p) {
         const int o = (p * 32 + lane) * 16;
-        const int tok = tok0 + o / R;
+        const int tok = tok0 + o / RB;
         const int pg = live && tok < cg.n_local ? s_page[tok >> cg.page_shift] : -1;
         const uint8_t* src = cg.head_base + (size_t)(uint32_t)max(pg, 0) * cg.page_bytes +
-                             ((tok & pmask) * R + o % R);
+                             ((tok & pmask) * RB + o % RB);
         cp_async16(dst + u * kTileBytes + o, src, pg >= 0 ? 16 : 0);
       }
     }
@@ -714,16 +763,17 @@ __device__ __forceinline__ uint32_t scan_issue(uint32_t dst, const ChunkGeom& cg
 }
 
 // One warp's contiguous run of tiles [t_begin, t_end) through its ring (`ring`: this warp's
-// scan_stages<R>() stages in shared memory).
-template <int R, bool BIG>
+// scan_stages<C>() stages in shared memory).
+template <class C, bool BIG>
 __device__ __forceinline__ uint32_t scan_warp_ring(const ChunkGeom& cg, const int32_t* s_page,
-                                                   const DigitFrags<R>& df, float thr_f,
+                                                   const DigitFrags<C>& df, float thr_f,
                                                    int t_begin, int t_end, uint32_t* rkey,
                                                    int32_t* rpos, uint8_t* ring, int lane) {
-  constexpr int kU = ScanBuf<R>::kUnroll;
-  constexpr int S = scan_stages<R>();
+  constexpr int kU = ScanBuf<C>::kUnroll;
+  constexpr int S = scan_stages<C>();
+  constexpr int kStageBytes = scan_stage_bytes<C>();
   constexpr uint32_t kMask = (1u << kU) - 1u;
-  constexpr int LB = R / 4;
+  constexpr int LB = C::kLaneBytes, RB = C::kBytes;
   static_assert(S * kU <= 32, "ok bits");
   const int g = lane >> 2, t = lane & 3;
   const uint32_t ring_s = smem_u32(ring);
@@ -732,7 +782,7 @@ __device__ __forceinline__ uint32_t scan_warp_ring(const ChunkGeom& cg, const in
 #pragma unroll
   for (int i = 0; i < S - 1; ++i) {
     if (i < n_batch)
-      ok_ring |= scan_issue<R, BIG>(ring_s + i * kScanStageBytes, cg, s_page, t_begin + i * kU,
+      ok_ring |= scan_issue<C, BIG>(ring_s + i * kStageBytes, cg, s_page, t_begin + i * kU,
                                     t_end, lane) << (i * kU);
     cp_async_commit();
   }
@@ -741,7 +791,7 @@ __device__ __forceinline__ uint32_t scan_warp_ring(const ChunkGeom& cg, const in
     const int nx = i + S - 1;
     if (nx < n_batch) {
       const int sx = nx % S;
-      const uint32_t okx = scan_issue<R, BIG>(ring_s + sx * kScanStageBytes, cg, s_page,
+      const uint32_t okx = scan_issue<C, BIG>(ring_s + sx * kStageBytes, cg, s_page,
                                               t_begin + nx * kU, t_end, lane);
       ok_ring = (ok_ring & ~(kMask << (sx * kU))) | ((okx & kMask) << (sx * kU));
     }
@@ -749,16 +799,16 @@ __device__ __forceinline__ uint32_t scan_warp_ring(const ChunkGeom& cg, const in
     cp_async_wait<S - 1>();
     __syncwarp();
     const int st = i % S;
-    const uint32_t stage = ring_s + st * kScanStageBytes;
-    ScanBuf<R> buf;
+    const uint32_t stage = ring_s + st * kStageBytes;
+    ScanBuf<C> buf;
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
-      lds_row<R>(buf.ra[u], stage + u * 16 * R + g * R + t * LB);
-      lds_row<R>(buf.rb[u], stage + u * 16 * R + (g + 8) * R + t * LB);
+      lds_row<LB>(buf.ra[u], stage + u * 16 * RB + g * RB + t * LB);
+      lds_row<LB>(buf.rb[u], stage + u * 16 * RB + (g + 8) * RB + t * LB);
     }
     buf.ok = BIG ? (ok_ring >> (st * kU)) & kMask : ~0u;
     __syncwarp();  // the stage is refilled by the next iteration's copies
-    scan_emit<R, BIG>(buf, df, cg, s_page, t_begin + i * kU, t_end, thr_f, rkey, rpos, run, lane);
+    scan_emit<C, BIG>(buf, df, cg, s_page, t_begin + i * kU, t_end, thr_f, rkey, rpos, run, lane);
   }
   cp_async_wait<0>();
   return run;
@@ -800,9 +850,9 @@ __device__ __forceinline__ int clamp_len(int L, int max_len) {
 // q < kRegionsPerChunk takes the q-th eighth of the chunk and writes that region and its count.
 // RING: the scan kernel's shared-memory tile rings (`ring`); otherwise register double buffers
 // (the select kernel's rescan).
-template <int R, bool RING>
+template <class C, bool RING>
 __device__ void scan_chunk(const ScanArgs& a, int pair, int c, int L, uint32_t thr,
-                           const DigitFrags<R>& df, const int32_t* s_page, uint8_t* ring) {
+                           const DigitFrags<C>& df, const int32_t* s_page, uint8_t* ring) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (warp >= kRegionsPerChunk) return;
   const int h = pair % a.h_kv;
@@ -810,8 +860,8 @@ __device__ void scan_chunk(const ScanArgs& a, int pair, int c, int L, uint32_t t
   cg.start = c * a.chunk;
   cg.n_local = max(0, min(a.chunk, L - cg.start));
   cg.page_shift = a.page_shift;
-  cg.page_bytes = ((uint32_t)a.h_kv << a.page_shift) * R;
-  cg.head_base = a.score_cache + ((int64_t)h << a.page_shift) * R;
+  cg.page_bytes = ((uint32_t)a.h_kv << a.page_shift) * C::kBytes;
+  cg.head_base = a.score_cache + ((int64_t)h << a.page_shift) * C::kBytes;
   const int seg = a.chunk / kRegionsPerChunk;
   const int64_t reg = ((int64_t)pair * a.n_chunks + c) * kRegionsPerChunk + warp;
   const int n_tiles = (cg.n_local + 15) >> 4;
@@ -820,26 +870,26 @@ __device__ void scan_chunk(const ScanArgs& a, int pair, int c, int L, uint32_t t
   const float thr_f = key_floor(thr);
   uint32_t n;
   if (RING) {
-    uint8_t* wr = ring + warp * scan_stages<R>() * kScanStageBytes;
+    uint8_t* wr = ring + warp * scan_stages<C>() * scan_stage_bytes<C>();
     n = cg.page_shift >= 4
-            ? scan_warp_ring<R, true>(cg, s_page, df, thr_f, t_begin, t_end,
+            ? scan_warp_ring<C, true>(cg, s_page, df, thr_f, t_begin, t_end,
                                       a.cands.key + reg * seg, a.cands.pos + reg * seg, wr, lane)
-            : scan_warp_ring<R, false>(cg, s_page, df, thr_f, t_begin, t_end,
+            : scan_warp_ring<C, false>(cg, s_page, df, thr_f, t_begin, t_end,
                                        a.cands.key + reg * seg, a.cands.pos + reg * seg, wr, lane);
   } else {
     n = cg.page_shift >= 4
-            ? scan_warp<R, true>(cg, s_page, df, thr_f, t_begin, t_end, a.cands.key + reg * seg,
+            ? scan_warp<C, true>(cg, s_page, df, thr_f, t_begin, t_end, a.cands.key + reg * seg,
                                  a.cands.pos + reg * seg, lane)
-            : scan_warp<R, false>(cg, s_page, df, thr_f, t_begin, t_end, a.cands.key + reg * seg,
+            : scan_warp<C, false>(cg, s_page, df, thr_f, t_begin, t_end, a.cands.key + reg * seg,
                                   a.cands.pos + reg * seg, lane);
   }
   if (lane == 0) a.cands.cnt[reg] = n;
 }
 
-template <int D, int R>
-__global__ void __launch_bounds__(kThreads, scan_ctas_per_sm<R>()) scan_kernel(ScanArgs a) {
+template <int D, class C>
+__global__ void __launch_bounds__(kThreads, scan_ctas_per_sm<C>()) scan_kernel(ScanArgs a) {
   extern __shared__ __align__(16) uint8_t scan_dyn[];  // tile ring, then the page list
-  int32_t* scan_pages = reinterpret_cast<int32_t*>(scan_dyn + scan_ring_bytes<R>());
+  int32_t* scan_pages = reinterpret_cast<int32_t*>(scan_dyn + scan_ring_bytes<C>());
   const int c = blockIdx.x, pair = blockIdx.y;
   const int b = pair / a.h_kv;
   const int L = clamp_len(a.seq_lens[b], a.max_pages << a.page_shift);
@@ -858,11 +908,11 @@ __global__ void __launch_bounds__(kThreads, scan_ctas_per_sm<R>()) scan_kernel(S
       a.cands.cnt[((int64_t)pair * a.n_chunks + c) * kRegionsPerChunk + (threadIdx.x >> 5)] = 0u;
     return;
   }
-  DigitFrags<R> df;
+  DigitFrags<C> df;
   df.load(reinterpret_cast<const uint16_t*>(rec), reinterpret_cast<const float*>(rec + kPrepScale),
           threadIdx.x & 31);
   const uint32_t thr = *reinterpret_cast<const uint32_t*>(rec + kPrepThr);
-  scan_chunk<R, true>(a, pair, c, L, thr, df, scan_pages, scan_dyn);
+  scan_chunk<C, true>(a, pair, c, L, thr, df, scan_pages, scan_dyn);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -903,26 +953,27 @@ constexpr int q_groups() { return kThreads / (D / 8); }
 constexpr int kSampleBins = 256;          // histogram bins of the sampled scores
 
 // Dynamic shared memory of the prep kernel.
-template <int D, int R>
+template <int D, class C>
 struct PrepSmem {
-  uint8_t rows[kSample * R];     // code rows of the sampled positions
-  float m[R * D];                // M_h, row-major [R][D]
+  uint8_t rows[kSample * C::kBytes];  // code rows of the sampled positions
+  float m[C::R * D];                  // M_h, row-major [R][D]
   float qpart[q_groups<D>()][D]; // partial sums of the group's query rows
   uint32_t list[256];            // keys of the bin that holds the threshold
   uint32_t hist[kSampleBins];
   uint8_t valid[kSample];        // sampled position on a usable page
 };
 
-template <int D, int R, bool STORE>
+template <int D, class C, bool STORE>
 __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
-  constexpr int LB = R / 4;
+  constexpr int R = C::R, LB = C::kLaneBytes, RB = C::kBytes;
+  constexpr int kDigits = C::kDigits;
   constexpr int kTilesPerWarp = kSample / 16 / kWarps;  // 16
   extern __shared__ __align__(16) uint8_t prep_dyn[];
-  PrepSmem<D, R>& sm = *reinterpret_cast<PrepSmem<D, R>*>(prep_dyn);
+  PrepSmem<D, C>& sm = *reinterpret_cast<PrepSmem<D, C>*>(prep_dyn);
   __shared__ float s_qbar[D];
   __shared__ float s_k[D];
   __shared__ float s_p[R];
-  __shared__ __align__(16) uint16_t s_dig[kDigits * R];  // f16 digits
+  __shared__ __align__(16) uint16_t s_dig[kDigits * R];  // f16 (E4M3 codes) or bf16 digits
   __shared__ float s_scale[kDigits];
   __shared__ uint32_t s_wsum[2 * kWarps];
   __shared__ int s_info[4];
@@ -981,8 +1032,8 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
     // warp instruction covers whole groups (kGroup rows of r bytes, one contiguous run when the
     // page holds at least kGroup tokens), so its lanes coalesce into a few line requests. A row
     // on an unusable page is zero-filled and marked invalid.
-    constexpr int kPieces = R / 16;                       // 16-byte pieces per row
-    constexpr int kLanesPerGroup = kGroup * kPieces;      // 8 (r = 32) or 16 (r = 64)
+    constexpr int kPieces = RB / 16;                      // 16-byte pieces per row
+    constexpr int kLanesPerGroup = kGroup * kPieces;      // 8 (32-byte rows) or 16 (64-byte)
     constexpr int kGroupsPerIssue = 32 / kLanesPerGroup;  // groups per warp instruction
     constexpr int kWarpGroups = kSampleGroups / kWarps;   // 64 groups per warp
     constexpr int kIssues = kWarpGroups / kGroupsPerIssue;
@@ -1002,8 +1053,8 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
       const int32_t pg = (pg0[u] < 0 || (int64_t)pg0[u] >= a.num_pages) ? -1 : pg0[u];
       if (part == 0) sm.valid[i] = pg >= 0;
       const uint8_t* src = a.score_cache +
-          ((((int64_t)max(pg, 0) * a.h_kv + h) << a.page_shift) + (pos & (page_size - 1))) * R;
-      cp_async16(smem_u32(sm.rows + i * R + part * 16), src + part * 16, pg >= 0 ? 16 : 0);
+          ((((int64_t)max(pg, 0) * a.h_kv + h) << a.page_shift) + (pos & (page_size - 1))) * RB;
+      cp_async16(smem_u32(sm.rows + i * RB + part * 16), src + part * 16, pg >= 0 ? 16 : 0);
     }
   }
   cp_async_commit();  // (group: the sample rows; M_h is the group before)
@@ -1055,7 +1106,7 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
 
   __syncthreads();  // qbar
 
-  // ---- p = M_h qbar and, at decode, the new token's code e4m3(M_h k) ---------------------------
+  // ---- p = M_h qbar and, at decode, the new token's code e4m3(M_h k) (or bf16(M_h k)) ----------
   {
     constexpr int TPJ = kThreads / R;  // threads per output
     constexpr int DPT = D / TPJ;
@@ -1081,17 +1132,20 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
       s_p[j] = acc;
       if (store && st_page >= 0) {
         const int pos = L - 1;
-        a.store.score_cache[(((int64_t)st_page * a.h_kv + h) * page_size + (pos & (page_size - 1))) * R + j] =
-            f64_to_e4m3(acc_k);
+        uint8_t* row = a.store.score_cache +
+            (((int64_t)st_page * a.h_kv + h) * page_size + (pos & (page_size - 1))) * RB;
+        if (C::kBF16) reinterpret_cast<uint16_t*>(row)[j] = f64_to_bf16(acc_k);
+        else row[j] = f64_to_e4m3(acc_k);
       }
     }
   }
   __syncthreads();
   if (warp == 0) {
-    // p = 2^-e0 D0 + 2^-e1 D1 with f16 digit vectors: D0 = f16(p 2^e0), e0 chosen so that the
-    // largest |component| lands in [2^14, 2^15) (inside the f16 range), and D1 = f16(r 2^e1) for
-    // the remainder r = p 2^e0 - D0 (exact in fp32), scaled the same way; about 22 significant
-    // bits of every component relative to the largest one.
+    // p = 2^-e0 D0 + 2^-e1 D1 (+ ...) with 16-bit digit vectors: D0 = f16(p 2^e0), e0 chosen so
+    // that the largest |component| lands in [2^14, 2^15) (inside the f16 range), and D1 =
+    // f16(r 2^e1) for the remainder r = p 2^e0 - D0 (exact in fp32), scaled the same way; about
+    // 22 significant bits of every component relative to the largest one. BF16 codes multiply
+    // bf16 digits (8 significant bits each), four of them for about 24 bits.
     float rem[R / 32];
 #pragma unroll
     for (int i = 0; i < R / 32; ++i) rem[i] = s_p[lane + 32 * i];
@@ -1109,9 +1163,15 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
 #pragma unroll
       for (int i = 0; i < R / 32; ++i) {
         const float v = rem[i] * up;
-        const __half dh = __float2half_rn(v);
-        s_dig[c * R + lane + 32 * i] = __half_as_ushort(dh);
-        rem[i] = v - __half2float(dh);
+        if (C::kBF16) {
+          const uint16_t db = f_to_bf16(v);
+          s_dig[c * R + lane + 32 * i] = db;
+          rem[i] = v - bf16_to_f(db);
+        } else {
+          const __half dh = __float2half_rn(v);
+          s_dig[c * R + lane + 32 * i] = __half_as_ushort(dh);
+          rem[i] = v - __half2float(dh);
+        }
       }
       if (lane == 0) s_scale[c] = weight;
     }
@@ -1127,19 +1187,19 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
   if (k) {
     cp_async_wait<0>();
     __syncthreads();  // every thread's sample rows
-    DigitFrags<R> df;
+    DigitFrags<C> df;
     df.load(s_dig, s_scale, lane);
     uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
     uint32_t key[kTilesPerWarp / 2];  // this lane's sampled keys
 #pragma unroll
     for (int u = 0; u < kTilesPerWarp; u += 2) {
       const int i0 = (warp * kTilesPerWarp + u) * 16;
-      uint32_t ra0[R / 16], rb0[R / 16], ra1[R / 16], rb1[R / 16];
-      load_srow<R>(ra0, sm.rows + (i0 + g) * R + t * LB);
-      load_srow<R>(rb0, sm.rows + (i0 + g + 8) * R + t * LB);
-      load_srow<R>(ra1, sm.rows + (i0 + 16 + g) * R + t * LB);
-      load_srow<R>(rb1, sm.rows + (i0 + 24 + g) * R + t * LB);
-      const float f = pair_scores<R>(ra0, rb0, ra1, rb1, df, t);
+      uint32_t ra0[C::kRegs], rb0[C::kRegs], ra1[C::kRegs], rb1[C::kRegs];
+      load_srow<LB>(ra0, sm.rows + (i0 + g) * RB + t * LB);
+      load_srow<LB>(rb0, sm.rows + (i0 + g + 8) * RB + t * LB);
+      load_srow<LB>(ra1, sm.rows + (i0 + 16 + g) * RB + t * LB);
+      load_srow<LB>(rb1, sm.rows + (i0 + 24 + g) * RB + t * LB);
+      const float f = pair_scores<C>(ra0, rb0, ra1, rb1, df, t);
       // lane t holds sample 16 * (t >> 1) + 8 * (t & 1) + g of the two tiles
       const int i = i0 + 16 * (t >> 1) + 8 * (t & 1) + g;
       // a sample on an unusable page (flagged by the scan) counts as the lowest key
@@ -1429,7 +1489,7 @@ __device__ bool select_in_registers(const SelectArgs& s, int pair, int n_reg, in
   return true;
 }
 
-template <int D, int R>
+template <int D, class C>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
   extern __shared__ uint32_t sel_dyn[];  // keys [kSelectCap] then positions [kSelectCap]
   uint32_t* s_ckey = sel_dyn;
@@ -1529,7 +1589,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
     // no threshold (all keys become candidates), then select exactly as usual
     if (tid == 0) raise_flag(16u);
     use_hist = false;
-    DigitFrags<R> df;
+    DigitFrags<C> df;
     df.load(reinterpret_cast<const uint16_t*>(rec), reinterpret_cast<const float*>(rec + kPrepScale),
             lane);
     int32_t* s_page = reinterpret_cast<int32_t*>(s_ckey);  // free until the staging below
@@ -1541,7 +1601,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
       load_pages(s_page, a.block_table + (int64_t)b * a.max_pages + (start >> a.page_shift),
                  n_pages, a.num_pages);
       __syncthreads();
-      scan_chunk<R, false>(a, pair, c, L, 0u, df, s_page, nullptr);
+      scan_chunk<C, false>(a, pair, c, L, 0u, df, s_page, nullptr);
     }
     __syncthreads();
     offsets();
@@ -1693,31 +1753,31 @@ cudaError_t launch_k(Kern kern, dim3 grid, int threads, size_t smem, bool pdl, c
   return cudaGetLastError();
 }
 
-template <int D, int R>
+template <int D, class C>
 cudaError_t launch_t(const ScorePlan& plan, int pairs, const PrepArgs& pa, const ScanArgs& sa,
                      const SelectArgs& sel, bool store, bool pdl, cudaStream_t s) {
   cudaError_t e;
-  const size_t prep_smem = sizeof(PrepSmem<D, R>);
+  const size_t prep_smem = sizeof(PrepSmem<D, C>);
   if (store) {
-    e = configure_kernel((const void*)prep_kernel<D, R, true>, (int)prep_smem, false);
+    e = configure_kernel((const void*)prep_kernel<D, C, true>, (int)prep_smem, false);
     if (e == cudaSuccess)
-      e = launch_k(prep_kernel<D, R, true>, dim3(pairs), kThreads, prep_smem, pdl, s, pa);
+      e = launch_k(prep_kernel<D, C, true>, dim3(pairs), kThreads, prep_smem, pdl, s, pa);
   } else {
-    e = configure_kernel((const void*)prep_kernel<D, R, false>, (int)prep_smem, false);
+    e = configure_kernel((const void*)prep_kernel<D, C, false>, (int)prep_smem, false);
     if (e == cudaSuccess)
-      e = launch_k(prep_kernel<D, R, false>, dim3(pairs), kThreads, prep_smem, pdl, s, pa);
+      e = launch_k(prep_kernel<D, C, false>, dim3(pairs), kThreads, prep_smem, pdl, s, pa);
   }
   if (e != cudaSuccess) return e;
   const size_t scan_smem =
-      (size_t)scan_ring_bytes<R>() + (size_t)(plan.chunk / (1 << sa.page_shift) + 1) * 4;
-  e = configure_kernel((const void*)scan_kernel<D, R>, (int)scan_smem, false);
+      (size_t)scan_ring_bytes<C>() + (size_t)(plan.chunk / (1 << sa.page_shift) + 1) * 4;
+  e = configure_kernel((const void*)scan_kernel<D, C>, (int)scan_smem, false);
   if (e != cudaSuccess) return e;
-  e = launch_k(scan_kernel<D, R>, dim3(plan.n_chunks, pairs), kThreads, scan_smem, true, s, sa);
+  e = launch_k(scan_kernel<D, C>, dim3(plan.n_chunks, pairs), kThreads, scan_smem, true, s, sa);
   if (e != cudaSuccess) return e;
   const size_t sel_smem = (size_t)kSelectCap * 8;
-  e = configure_kernel((const void*)select_kernel<D, R>, (int)sel_smem, false);
+  e = configure_kernel((const void*)select_kernel<D, C>, (int)sel_smem, false);
   if (e != cudaSuccess) return e;
-  return launch_k(select_kernel<D, R>, dim3(pairs), kSelThreads, sel_smem, true, s, sel);
+  return launch_k(select_kernel<D, C>, dim3(pairs), kSelThreads, sel_smem, true, s, sel);
 }
 
 }  // namespace score_detail
@@ -1747,7 +1807,7 @@ cudaError_t launch_score_topk(const uint16_t* q, const float* basis, const uint8
                               int batch, int h_q, int h_kv, int d, int r, int64_t num_pages,
                               int page_size, int budget, int32_t* idx, int32_t* count, void* ws,
                               int* attend_tickets, const StoreNew* store, bool pdl,
-                              cudaStream_t s) {
+                              cudaStream_t s, bool bf16_codes) {
   using namespace score_detail;
   const int pairs = batch * h_kv;
   if (pairs == 0) return cudaSuccess;
@@ -1776,12 +1836,15 @@ cudaError_t launch_score_topk(const uint16_t* q, const float* basis, const uint8
   sa.chunk = plan.chunk; sa.n_chunks = plan.n_chunks; sa.budget = budget; sa.prep = prep;
   sa.cands = cands;
   const SelectArgs sel = {sa, idx, count};
-  if (d == 128 && r == 32)
-    return score_detail::launch_t<128, 32>(plan, pairs, pa, sa, sel, store != nullptr, pdl, s);
-  if (d == 128 && r == 64)
-    return score_detail::launch_t<128, 64>(plan, pairs, pa, sa, sel, store != nullptr, pdl, s);
-  if (d == 256 && r == 64)
-    return score_detail::launch_t<256, 64>(plan, pairs, pa, sa, sel, store != nullptr, pdl, s);
+  const bool st = store != nullptr;
+  if (bf16_codes) {
+    if (d == 128 && r == 32)
+      return launch_t<128, Codes<32, true>>(plan, pairs, pa, sa, sel, st, pdl, s);
+    return cudaErrorInvalidValue;
+  }
+  if (d == 128 && r == 32) return launch_t<128, Codes<32, false>>(plan, pairs, pa, sa, sel, st, pdl, s);
+  if (d == 128 && r == 64) return launch_t<128, Codes<64, false>>(plan, pairs, pa, sa, sel, st, pdl, s);
+  if (d == 256 && r == 64) return launch_t<256, Codes<64, false>>(plan, pairs, pa, sa, sel, st, pdl, s);
   return cudaErrorInvalidValue;
 }
 

@@ -1,6 +1,8 @@
 // Store step: FP8 E4M3 projected key c = e4m3(M_h k) for new tokens (JSSA summary, section 3.4
 // "Projected Scoring Cache"; JSSA README, section 4 notes: r bytes per token and KV head).
 //
+// BF16 = true stores bf16(M_h k) instead (two bytes per dimension: the scoring-cache ablation).
+//
 // One CTA per (KV head, range of tokens). The basis rows of the head are staged in shared memory
 // once; each warp takes one token at a time, lane j computes output j (and j+32, ...) as a
 // float64 dot product over the d dimensions and rounds it once to E4M3. At decode the same kernel
@@ -14,7 +16,7 @@ namespace store_detail {
 constexpr int kStoreThreads = 256;
 constexpr int kStoreWarps = kStoreThreads / 32;
 
-template <int D, int R, bool DECODE>
+template <int D, int R, bool DECODE, bool BF16>
 __global__ void __launch_bounds__(kStoreThreads)
     store_kernel(const uint16_t* __restrict__ k, int64_t k_stride_t,
                  const int64_t* __restrict__ slot_mapping, int t_count, int h_kv,
@@ -93,7 +95,8 @@ __global__ void __launch_bounds__(kStoreThreads)
       }
     }
     __syncwarp();
-    uint8_t* dst = score_cache + ((page * h_kv + h) * page_size + off) * R;
+    constexpr int RB = BF16 ? 2 * R : R;  // code bytes per token
+    uint8_t* dst = score_cache + ((page * h_kv + h) * page_size + off) * RB;
 #pragma unroll
     for (int j0 = 0; j0 < R; j0 += 32) {
       const int j = j0 + lane;
@@ -101,14 +104,15 @@ __global__ void __launch_bounds__(kStoreThreads)
       double acc = 0.0;
 #pragma unroll 8
       for (int i = 0; i < D; ++i) acc = fma((double)mrow[i], (double)kw[i], acc);
-      dst[j] = f64_to_e4m3(acc);
+      if (BF16) reinterpret_cast<uint16_t*>(dst)[j] = f64_to_bf16(acc);
+      else dst[j] = f64_to_e4m3(acc);
     }
     __syncwarp();
   }
   if (DECODE) pdl_trigger();
 }
 
-template <int D, int R, bool DECODE>
+template <int D, int R, bool DECODE, bool BF16>
 cudaError_t launch_store_t(dim3 grid, size_t smem, cudaStream_t s, const uint16_t* k,
                            int64_t k_stride_t, const int64_t* slot_mapping, int t, int h_kv,
                            const float* basis, uint8_t* score_cache, int64_t num_pages,
@@ -116,7 +120,7 @@ cudaError_t launch_store_t(dim3 grid, size_t smem, cudaStream_t s, const uint16_
                            uint16_t* v_cache, int64_t page_stride, int64_t slot_stride,
                            int64_t head_stride, const int32_t* block_table, int max_pages,
                            const int32_t* seq_lens) {
-  auto kern = store_kernel<D, R, DECODE>;
+  auto kern = store_kernel<D, R, DECODE, BF16>;
   cudaError_t e = configure_kernel((const void*)kern, (int)smem, false);
   if (e != cudaSuccess) return e;
   kern<<<grid, kStoreThreads, smem, s>>>(k, k_stride_t, slot_mapping, t, h_kv, basis, score_cache,
@@ -126,7 +130,7 @@ cudaError_t launch_store_t(dim3 grid, size_t smem, cudaStream_t s, const uint16_
   return cudaGetLastError();
 }
 
-template <bool DECODE>
+template <bool DECODE, bool BF16 = false>
 cudaError_t dispatch_store(int d, int r, int t, int h_kv, int tpb, cudaStream_t s,
                            const uint16_t* k, int64_t k_stride_t, const int64_t* slot_mapping,
                            const float* basis, uint8_t* score_cache, int64_t num_pages,
@@ -139,10 +143,15 @@ cudaError_t dispatch_store(int d, int r, int t, int h_kv, int tpb, cudaStream_t 
   const size_t smem = (size_t)(r * (d + 1) + kStoreWarps * d) * sizeof(float);
 #define JSSA_STORE_CASE(DD, RR)                                                                  \
   if (d == DD && r == RR)                                                                        \
-    return launch_store_t<DD, RR, DECODE>(grid, smem, s, k, k_stride_t, slot_mapping, t, h_kv,   \
+    return launch_store_t<DD, RR, DECODE, BF16>(grid, smem, s, k, k_stride_t, slot_mapping, t,   \
+                                          h_kv,                                                  \
                                           basis, score_cache, num_pages, page_size, tpb, v_new,  \
                                           k_cache, v_cache, page_stride, slot_stride,            \
                                           head_stride, block_table, max_pages, seq_lens);
+  if (BF16) {
+    JSSA_STORE_CASE(128, 32)
+    return cudaErrorInvalidValue;
+  }
   JSSA_STORE_CASE(128, 32)
   JSSA_STORE_CASE(128, 64)
   JSSA_STORE_CASE(256, 64)
@@ -154,8 +163,12 @@ cudaError_t dispatch_store(int d, int r, int t, int h_kv, int tpb, cudaStream_t 
 
 cudaError_t launch_store(const uint16_t* k, int64_t k_stride_t, const int64_t* slot_mapping,
                          int t, int h_kv, int d, int r, const float* basis, uint8_t* score_cache,
-                         int64_t num_pages, int page_size, cudaStream_t s) {
+                         int64_t num_pages, int page_size, cudaStream_t s, bool bf16_codes) {
   const int tpb = t >= 4096 ? 256 : store_detail::kStoreWarps;
+  if (bf16_codes)
+    return store_detail::dispatch_store<false, true>(d, r, t, h_kv, tpb, s, k, k_stride_t,
+                               slot_mapping, basis, score_cache, num_pages, page_size, nullptr,
+                               nullptr, nullptr, 0, 0, 0, nullptr, 0, nullptr);
   return store_detail::dispatch_store<false>(d, r, t, h_kv, tpb, s, k, k_stride_t, slot_mapping, basis,
                                score_cache, num_pages, page_size, nullptr, nullptr, nullptr, 0, 0,
                                0, nullptr, 0, nullptr);
