@@ -306,21 +306,56 @@ __global__ void __launch_bounds__(kThreads, Ring<D>::kCtasPerSm)
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  for (int e = tid; e < G * D; e += kThreads) {
-    const int row = e / D, dim = e % D;
-    const float* pp = part + ((int64_t)pair * splits * G + row) * (D + 2);
-    const int64_t step = (int64_t)G * (D + 2);
-    float mm = -INFINITY;
-    for (int s_ = 0; s_ < splits; ++s_) mm = fmaxf(mm, __ldcg(pp + s_ * step));
-    float acc = 0.f, l = 0.f;
-    if (mm != -INFINITY) {
-      for (int s_ = 0; s_ < splits; ++s_) {
-        const float f = fast_exp2(__ldcg(pp + s_ * step) - mm);
-        acc += f * __ldcg(pp + s_ * step + 2 + dim);
-        l += f * __ldcg(pp + s_ * step + 1);
-      }
+  const float* pbase = part + (int64_t)pair * splits * G * (D + 2);
+  const int64_t step = (int64_t)G * (D + 2);  // floats per split
+  if (splits * G * 3 * (int)sizeof(float) <= Ring<D>::kBytes) {
+    // every split's (m, l) of every row into shared memory at once (the ring is free now), one
+    // weight per (split, row) w = 2^(m - M) / L with M the rows' maximum and L the merged sum,
+    // then each output element is one weighted sum of independent loads
+    float* s_pm = reinterpret_cast<float*>(att_ring);
+    float* s_pl = s_pm + splits * G;
+    float* s_w = s_pl + splits * G;
+    for (int i = tid; i < splits * G; i += kThreads) {
+      const int sp = i / G, row = i % G;
+      s_pm[i] = __ldcg(pbase + sp * step + (int64_t)row * (D + 2));
+      s_pl[i] = __ldcg(pbase + sp * step + (int64_t)row * (D + 2) + 1);
     }
-    a.out[out_base + (int64_t)row * D + dim] = f_to_bf16(l > 0.f ? acc / l : 0.f);
+    __syncthreads();
+    if (tid < G) {
+      float mm = -INFINITY;
+      for (int sp = 0; sp < splits; ++sp) mm = fmaxf(mm, s_pm[sp * G + tid]);
+      float l = 0.f;
+      if (mm != -INFINITY)
+        for (int sp = 0; sp < splits; ++sp) l += fast_exp2(s_pm[sp * G + tid] - mm) * s_pl[sp * G + tid];
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      for (int sp = 0; sp < splits; ++sp)
+        s_w[sp * G + tid] = mm != -INFINITY ? fast_exp2(s_pm[sp * G + tid] - mm) * inv : 0.f;
+    }
+    __syncthreads();
+    for (int e = tid; e < G * D; e += kThreads) {
+      const int row = e / D, dim = e % D;
+      const float* pp = pbase + (int64_t)row * (D + 2) + 2 + dim;
+      float acc = 0.f;
+#pragma unroll 8
+      for (int sp = 0; sp < splits; ++sp) acc += s_w[sp * G + row] * __ldcg(pp + sp * step);
+      a.out[out_base + (int64_t)row * D + dim] = f_to_bf16(acc);
+    }
+  } else {
+    for (int e = tid; e < G * D; e += kThreads) {
+      const int row = e / D, dim = e % D;
+      const float* pp = pbase + (int64_t)row * (D + 2);
+      float mm = -INFINITY;
+      for (int s_ = 0; s_ < splits; ++s_) mm = fmaxf(mm, __ldcg(pp + s_ * step));
+      float acc = 0.f, l = 0.f;
+      if (mm != -INFINITY) {
+        for (int s_ = 0; s_ < splits; ++s_) {
+          const float f = fast_exp2(__ldcg(pp + s_ * step) - mm);
+          acc += f * __ldcg(pp + s_ * step + 2 + dim);
+          l += f * __ldcg(pp + s_ * step + 1);
+        }
+      }
+      a.out[out_base + (int64_t)row * D + dim] = f_to_bf16(l > 0.f ? acc / l : 0.f);
+    }
   }
   if (tid == 0) tickets[pair] = 0;
 }
@@ -362,6 +397,7 @@ AttendPlan plan_attend(int pairs, int positions, int group, int d) {
   if (splits < 1) splits = 1;
   int chunk = (positions + splits - 1) / splits;
   chunk = (chunk + unit - 1) / unit * unit;
+  if (chunk < 4 * unit) chunk = 4 * unit;  // at least 4 tiles per warp (fill the ring)
   if (chunk > attend_detail::kMaxChunk) chunk = attend_detail::kMaxChunk;
   splits = (positions + chunk - 1) / chunk;
   p.splits = splits;
