@@ -85,7 +85,8 @@ enum jssa_fn {
   JSSA_FN_INDEXED_ATTEND = 2,
   JSSA_FN_DENSE_DECODE = 3,
   JSSA_FN_DECODE = 4,
-  JSSA_FN_COMPUTE_BASIS = 5
+  JSSA_FN_COMPUTE_BASIS = 5,
+  JSSA_FN_MLA_ATTEND = 6
 };
 
 /* Text for a status code (static storage). */
@@ -221,6 +222,27 @@ JSSA_API int jssa_score_topk_bf16(const jssa_bf16* q, const float* basis,
                                   int h_kv, int d, int r, int64_t num_pages, int page_size,
                                   int budget, int32_t* idx, int32_t* count, void* ws,
                                   size_t ws_bytes, jssa_stream_t stream);
+
+/*
+ * Multi-head latent attention over selected positions, absorbed form (JSSA summary, section 3.3;
+ * JSSA README, paper-to-code map and section 4 notes: one latent row per token, 512 latent + 64
+ * rotary dimensions, attended in place):
+ *   out[b, i, :] = sum_j softmax_j(softmax_scale * q[b, i] . kv[j]) kv[j, 0:512]
+ * over j in the index set of sequence b, i.e. jssa_score_topk run with h_kv = 1, d = 576 and
+ * r = 128 on the latent scoring cache (basis rows: the projected 512 latent dimensions, then the
+ * 64 rotary dimensions passed through).
+ * q: bf16 [batch, h_q, 576] absorbed queries (h_q a multiple of 16). kv_cache: bf16 latent cache,
+ * row (page p, slot s) at p*kv_page_stride + s*kv_slot_stride elements (576 contiguous, 16-byte
+ * aligned). idx/count: int32 [batch, 1, budget] / [batch, 1] (count clamped to [0, budget]).
+ * out: bf16 [batch, h_q, 512]. ws: >= jssa_workspace_size(JSSA_FN_MLA_ATTEND, batch, h_q, 1,
+ * 576, ...); its split counters must be zero when the call starts (jssa_workspace_init once) and
+ * are zero again when it ends. Out-of-range positions and pages are skipped and flagged.
+ */
+JSSA_API int jssa_mla_attend(const jssa_bf16* q, const jssa_bf16* kv_cache, int64_t kv_page_stride,
+                             int64_t kv_slot_stride, const int32_t* block_table, int max_pages,
+                             const int32_t* idx, const int32_t* count, int batch, int h_q,
+                             int budget, int64_t num_pages, int page_size, float softmax_scale,
+                             jssa_bf16* out, void* ws, size_t ws_bytes, jssa_stream_t stream);
 
 /*
  * Gather-then-attend ablation, step 1: copy the selected K and V rows of every (sequence, KV

@@ -150,6 +150,20 @@ def scores_bf16(codes: np.ndarray, p: np.ndarray) -> np.ndarray:
     return bf16_decode(codes) @ np.asarray(p, dtype=np.float64)
 
 
+def mla_scoring_basis(m_lat: np.ndarray, rope_dims: int = 64) -> np.ndarray:
+    """Latent scoring projection of multi-head latent attention: the rank-r basis acts on the
+    latent dimensions only and the rotary dimensions pass through unprojected, so a token's
+    scoring row is ``[M_lat c ; k_rope]`` (r + rope_dims codes). JSSA README, section 4 notes
+    (the MLA basis is [1, r, kv_lora_rank]; the rotary part is kept) and JSSA summary, section 3.4.
+    ``m_lat``: ``[r, latent]`` -> ``[r + rope_dims, latent + rope_dims]``."""
+    m_lat = np.asarray(m_lat, dtype=np.float64)
+    r, lat = m_lat.shape
+    out = np.zeros((r + rope_dims, lat + rope_dims))
+    out[:r, :lat] = m_lat
+    out[r:, lat:] = np.eye(rope_dims)
+    return out
+
+
 def projected_query(qbar: np.ndarray, m: np.ndarray) -> np.ndarray:
     """``p = M q_bar`` (JSSA summary, eq. (1): ``s_hat = q_bar^T P k = (M q_bar) . (M k)``)."""
     return np.asarray(m, dtype=np.float64) @ np.asarray(qbar, dtype=np.float64)

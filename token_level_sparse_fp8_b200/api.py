@@ -15,11 +15,11 @@ from typing import Optional, Tuple
 import torch
 
 from . import _lib
-from ._lib import (FN_COMPUTE_BASIS, FN_DECODE, FN_DENSE_DECODE, FN_INDEXED_ATTEND,
+from ._lib import (FN_COMPUTE_BASIS, FN_DECODE, FN_DENSE_DECODE, FN_INDEXED_ATTEND, FN_MLA_ATTEND,
                    FN_SCORE_TOPK, JSSAError, call)
 
 __all__ = [
-    "gather_kv", "staged_pages", "gather_then_attend",
+    "gather_kv", "staged_pages", "gather_then_attend", "mla_scoring_basis", "mla_attend",
     "JSSAError", "workspace_size", "Workspace", "calibrate_accumulate", "compute_basis",
     "calibrate", "store", "score_topk", "indexed_attend", "dense_decode", "decode",
     "device_error", "kv_strides", "default_rank", "PagedLayer",
@@ -223,6 +223,43 @@ def indexed_attend(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
     call("jssa_indexed_attend", q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), *strides,
          block_table.data_ptr(), block_table.shape[1], idx.data_ptr(), count.data_ptr(), batch, h_q,
          h_kv, d, budget, num_pages, page_size, scale, out.data_ptr(), p, n, _stream(q.device))
+    return out
+
+
+def mla_scoring_basis(m_lat: torch.Tensor, rope_dims: int = 64) -> torch.Tensor:
+    """Rows of the latent scoring projection of multi-head latent attention: the rank-r basis of
+    the latent dimensions, then the rotary dimensions passed through (float32
+    ``[1, r + rope_dims, latent + rope_dims]`` from ``m_lat`` ``[1, r, latent]``)."""
+    _, r, lat = m_lat.shape
+    out = torch.zeros((1, r + rope_dims, lat + rope_dims), dtype=torch.float32, device=m_lat.device)
+    out[0, :r, :lat] = m_lat[0]
+    out[0, r:, lat:] = torch.eye(rope_dims, dtype=torch.float32, device=m_lat.device)
+    return out
+
+
+def mla_attend(q: torch.Tensor, kv_cache: torch.Tensor, block_table: torch.Tensor,
+               idx: torch.Tensor, count: torch.Tensor, scale: float,
+               out: Optional[torch.Tensor] = None, ws: Optional[Workspace] = None) -> torch.Tensor:
+    """Multi-head latent attention (absorbed queries ``q`` bf16 ``[batch, h_q, 576]``) over the
+    selected rows of the latent cache ``kv_cache`` bf16 ``[num_pages, page_size, 576]``; values
+    are the first 512 dimensions of each row. Returns bf16 ``[batch, h_q, 512]``."""
+    _need(q, "q", torch.bfloat16)
+    _need(kv_cache, "kv_cache", torch.bfloat16, contiguous=False)
+    _need(block_table, "block_table", torch.int32)
+    _need(idx, "idx", torch.int32)
+    _need(count, "count", torch.int32)
+    batch, h_q, dk = q.shape
+    num_pages, page_size, dkc = kv_cache.shape
+    if dk != 576 or dkc != 576 or kv_cache.stride(2) != 1:
+        raise ValueError("latent rows must be 576 contiguous bf16")
+    budget = idx.shape[2]
+    out = torch.empty((batch, h_q, 512), dtype=torch.bfloat16, device=q.device) if out is None else out
+    w = _ws(q.device, ws, FN_MLA_ATTEND)
+    p, n = w.get(workspace_size(FN_MLA_ATTEND, batch, h_q, 1, 576, block_table.shape[1], page_size,
+                                budget))
+    call("jssa_mla_attend", q.data_ptr(), kv_cache.data_ptr(), kv_cache.stride(0), kv_cache.stride(1),
+         block_table.data_ptr(), block_table.shape[1], idx.data_ptr(), count.data_ptr(), batch, h_q,
+         budget, num_pages, page_size, scale, out.data_ptr(), p, n, _stream(q.device))
     return out
 
 

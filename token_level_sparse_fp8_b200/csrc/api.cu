@@ -61,7 +61,7 @@ inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 inline cudaStream_t as_stream(jssa_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
 bool supported_dr(int d, int r) {
-  return (d == 128 && (r == 32 || r == 64)) || (d == 256 && r == 64);
+  return (d == 128 && (r == 32 || r == 64)) || (d == 256 && r == 64) || (d == 576 && r == 128);
 }
 bool supported_d(int d) { return d == 128 || d == 256; }
 
@@ -161,6 +161,10 @@ int jssa_workspace_size(int fn, int batch, int h_q, int h_kv, int d, int max_pag
       if (budget <= 0) return JSSA_ERR_SHAPE;
       *bytes = align256(attend_plan_indexed(batch, h_q, h_kv, d, budget).ws_bytes) +
                score_ws_bytes(batch, h_kv, max_seq_len, page_size);
+      return JSSA_OK;
+    case JSSA_FN_MLA_ATTEND:
+      if (budget <= 0 || h_kv != 1 || d != 576 || h_q % 16) return JSSA_ERR_SHAPE;
+      *bytes = jssa::plan_mla(batch, h_q, budget).ws_bytes;
       return JSSA_OK;
     case JSSA_FN_DENSE_DECODE: {
       const int span = (budget > 0 && budget < max_seq_len) ? budget : max_seq_len;
@@ -359,6 +363,30 @@ int jssa_dense_decode(const jssa_bf16* q, const jssa_bf16* k_cache, const jssa_b
   a.num_pages = num_pages; a.page_size = page_size; a.scale = softmax_scale; a.out = out;
   a.ws = ws;
   return cuda_status(jssa::launch_attend(a, false, plan, false, as_stream(stream)));
+}
+
+int jssa_mla_attend(const jssa_bf16* q, const jssa_bf16* kv_cache, int64_t kv_page_stride,
+                    int64_t kv_slot_stride, const int32_t* block_table, int max_pages,
+                    const int32_t* idx, const int32_t* count, int batch, int h_q, int budget,
+                    int64_t num_pages, int page_size, float softmax_scale, jssa_bf16* out,
+                    void* ws, size_t ws_bytes, jssa_stream_t stream) {
+  if (batch < 0 || h_q <= 0 || budget <= 0) return JSSA_ERR_SHAPE;
+  if (h_q % 16 || budget > 256 * 1024) return JSSA_ERR_UNSUPPORTED;
+  int st = check_paging(max_pages, num_pages, page_size);
+  if (st) return st;
+  if (batch == 0) return JSSA_OK;
+  if (!q || !kv_cache || !block_table || !idx || !count || !out) return JSSA_ERR_NULL;
+  if (kv_page_stride <= 0 || kv_slot_stride < 576) return JSSA_ERR_SHAPE;
+  if (!aligned16(kv_cache) || !aligned16(q) || ((kv_page_stride | kv_slot_stride) & 7) ||
+      ((uintptr_t)out & 3u))
+    return JSSA_ERR_ALIGN;
+  const jssa::MlaPlan plan = jssa::plan_mla(batch, h_q, budget);
+  if (plan.ws_bytes && (!ws || ws_bytes < plan.ws_bytes)) return JSSA_ERR_WORKSPACE;
+  if (plan.ws_bytes && !aligned16(ws)) return JSSA_ERR_ALIGN;
+  return cuda_status(jssa::launch_mla(q, kv_cache, kv_page_stride, kv_slot_stride, block_table,
+                                      max_pages, idx, count, batch, h_q, budget, num_pages,
+                                      page_size, softmax_scale, out, ws, plan, true,
+                                      as_stream(stream)));
 }
 
 int jssa_gather_kv(const jssa_bf16* k_cache, const jssa_bf16* v_cache, int64_t kv_page_stride,

@@ -92,6 +92,20 @@ cudaError_t launch_gather(const uint16_t* k_cache, const uint16_t* v_cache, int6
                           int h_kv, int d, int budget, int64_t num_pages, int page_size,
                           uint16_t* k_out, uint16_t* v_out, int32_t* lens_out, cudaStream_t s);
 
+// Multi-head latent attention over selected positions (absorbed form, 576-dim key rows,
+// 512-dim values, 16 query heads per CTA): split-K plan and launch.
+struct MlaPlan {
+  int splits;
+  int chunk;
+  size_t ws_bytes;
+};
+MlaPlan plan_mla(int batch, int h_q, int budget);
+cudaError_t launch_mla(const uint16_t* q, const uint16_t* kv, int64_t page_stride,
+                       int64_t slot_stride, const int32_t* block_table, int max_pages,
+                       const int32_t* idx, const int32_t* count, int batch, int h_q, int budget,
+                       int64_t num_pages, int page_size, float scale, uint16_t* out, void* ws,
+                       const MlaPlan& plan, bool pdl, cudaStream_t s);
+
 cudaError_t launch_gram(const uint16_t* q, int64_t q_stride, const uint16_t* k, int64_t k_stride,
                         int n, int h_q, int h_kv, int d, double* gram_q, double* gram_k,
                         cudaStream_t s);

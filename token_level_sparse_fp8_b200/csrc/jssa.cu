@@ -5,6 +5,7 @@
 #include "score_topk.cu"
 #include "attend.cu"
 #include "gather.cu"
+#include "mla.cu"
 #include "calib.cu"
 #include "basis.cu"
 #include "noalloc.cu"

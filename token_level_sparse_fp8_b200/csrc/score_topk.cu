@@ -38,7 +38,7 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kUnrollBytes = 32;   // bytes of scoring rows per lane per load batch
 constexpr int kBins = 2048;
-constexpr int kSample = 2048;      // sampled positions per (sequence, KV head)
+constexpr int kSample = 2048;      // sampled positions per (sequence, KV head), up to 64-byte rows
 constexpr int kExactMax = 16384;   // up to this context every token is a candidate
 constexpr int kSelectCap = 16384;  // candidates the select kernel stages in shared memory
 constexpr int kRegionsPerChunk = kWarps;  // candidate regions (one per scan warp) per chunk
@@ -710,11 +710,12 @@ __device__ __forceinline__ uint32_t scan_warp(const ChunkGeom& cg, const int32_t
 // The scan kernel's warps stream their tiles through a ring of scan_stages<C>() shared-memory
 // stages (kUnroll tiles each) filled by asynchronous 16-byte copies, all but one stage ahead of
 // the one being scored: deeper than a register double buffer without holding the rows in
-// registers. E4M3 at r = 32: three stages and four CTAs per SM; otherwise four stages and three.
+// registers. 32-byte rows: three stages and four CTAs per SM; 64-byte rows: four stages and
+// three; 128-byte rows (the latent scoring of multi-head latent attention): two stages and three.
 template <class C>
 constexpr int scan_stage_bytes() { return ScanBuf<C>::kUnroll * 16 * C::kBytes; }
 template <class C>
-constexpr int scan_stages() { return C::kBytes == 32 ? 3 : 4; }
+constexpr int scan_stages() { return C::kBytes == 32 ? 3 : C::kBytes == 64 ? 4 : 2; }
 template <class C>
 constexpr int scan_ctas_per_sm() { return C::kBytes == 32 ? 4 : 3; }
 template <class C>
@@ -934,14 +935,16 @@ struct PrepArgs {
   StoreNew store;  // decode: the new token (position seq_len - 1)
 };
 
-// The sample: kSampleGroups strata of L / kSampleGroups tokens, in each a run of kGroup
-// consecutive positions (one 128-byte line of codes at r = 32) starting at a kGroup-aligned
-// offset drawn from a 32-bit mix of (stratum, pair), scaled to the stratum by a high multiply;
-// never the last position (the token a decode step stores right now).
+// The sample: n_groups strata of L / n_groups tokens, in each a run of kGroup consecutive
+// positions (one 128-byte line of codes at r = 32) starting at a kGroup-aligned offset drawn
+// from a 32-bit mix of (stratum, pair), scaled to the stratum by a high multiply; never the last
+// position (the token a decode step stores right now). 2048 positions for rows of up to 64
+// bytes, 1024 for 128-byte rows (the sampled rows are staged in shared memory).
 constexpr int kGroup = 4;
-constexpr int kSampleGroups = kSample / kGroup;
-__device__ __forceinline__ int sample_group_start(int grp, int pair, int L) {
-  const int stratum = L / kSampleGroups;  // >= 32 whenever the sample is drawn
+template <class C>
+constexpr int sample_size() { return C::kBytes > 64 ? kSample / 2 : kSample; }
+__device__ __forceinline__ int sample_group_start(int grp, int pair, int L, int n_groups) {
+  const int stratum = L / n_groups;  // >= 32 whenever the sample is drawn
   const uint32_t hsh = mix32((uint32_t)grp * 0x9E3779B9u ^ ((uint32_t)pair * 0x85EBCA6Bu + 1u));
   const int first = (grp * stratum + kGroup - 1) / kGroup;  // first aligned slot of the stratum
   return kGroup * (first + (int)__umulhi(hsh, (uint32_t)(stratum / kGroup - 1)));
@@ -952,22 +955,28 @@ template <int D>
 constexpr int q_groups() { return kThreads / (D / 8); }
 constexpr int kSampleBins = 256;          // histogram bins of the sampled scores
 
+// M_h is staged in shared memory when it takes at most 64 KB; otherwise (d 576, r 128: the
+// latent scoring of multi-head latent attention) the projection reads it from global memory.
+template <int D, class C>
+constexpr bool prep_m_in_smem() { return C::R * D * 4 <= 64 * 1024; }
+
 // Dynamic shared memory of the prep kernel.
 template <int D, class C>
 struct PrepSmem {
-  uint8_t rows[kSample * C::kBytes];  // code rows of the sampled positions
-  float m[C::R * D];                  // M_h, row-major [R][D]
+  uint8_t rows[sample_size<C>() * C::kBytes];  // code rows of the sampled positions
+  float m[prep_m_in_smem<D, C>() ? C::R * D : 1];  // M_h, row-major [R][D] (when it fits)
   float qpart[q_groups<D>()][D]; // partial sums of the group's query rows
   uint32_t list[256];            // keys of the bin that holds the threshold
   uint32_t hist[kSampleBins];
-  uint8_t valid[kSample];        // sampled position on a usable page
+  uint8_t valid[sample_size<C>()];  // sampled position on a usable page
 };
 
 template <int D, class C, bool STORE>
 __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
   constexpr int R = C::R, LB = C::kLaneBytes, RB = C::kBytes;
   constexpr int kDigits = C::kDigits;
-  constexpr int kTilesPerWarp = kSample / 16 / kWarps;  // 16
+  constexpr int kS = sample_size<C>(), kSampleGroups = kS / kGroup;
+  constexpr int kTilesPerWarp = kS / 16 / kWarps;  // 16 (8 for 128-byte rows)
   extern __shared__ __align__(16) uint8_t prep_dyn[];
   PrepSmem<D, C>& sm = *reinterpret_cast<PrepSmem<D, C>*>(prep_dyn);
   __shared__ float s_qbar[D];
@@ -996,21 +1005,29 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
 
   // ---- independent loads first: M_h into shared memory (async); L, the group's query rows and
   // the new token's K and V rows into registers ----
-  for (int i = tid; i < R * D / 4; i += kThreads) cp_async16(smem_u32(sm.m + 4 * i), m_h + 4 * i, 16);
+  constexpr bool kMSmem = prep_m_in_smem<D, C>();
+  if (kMSmem)
+    for (int i = tid; i < R * D / 4; i += kThreads) cp_async16(smem_u32(sm.m + 4 * i), m_h + 4 * i, 16);
   cp_async_commit();
   const int L = clamp_len(a.seq_lens[b], a.max_pages << a.page_shift);
   // the G query rows of this KV head: D / 8 threads x 8 dims per row, kQGroups rows at a time
-  static_assert(D == 128 || D == 256, "query row split");
+  static_assert(D % 8 == 0 && D / 8 <= kThreads, "query row split");
   constexpr int kQGroups = q_groups<D>();
   const uint16_t* qh = a.q + ((int64_t)b * a.h_q + (int64_t)h * G) * D;
   const int rg = tid / (D / 8), d8 = (tid % (D / 8)) * 8;
   uint4 qv = make_uint4(0u, 0u, 0u, 0u);
-  if (rg < G) qv = *reinterpret_cast<const uint4*>(qh + (int64_t)rg * D + d8);
+  if (rg < kQGroups && rg < G) qv = *reinterpret_cast<const uint4*>(qh + (int64_t)rg * D + d8);
   const bool store = STORE && L > 0;
-  uint16_t k_el = 0, v_el = 0;  // element tid of the new token's K and V rows (tid < D)
-  if (STORE && tid < D) {
-    k_el = a.store.k_new[((int64_t)b * a.h_kv + h) * D + tid];
-    v_el = a.store.v_new[((int64_t)b * a.h_kv + h) * D + tid];
+  constexpr int KE = (D + kThreads - 1) / kThreads;  // elements of the new K / V rows per thread
+  uint16_t k_el[KE], v_el[KE];                        // elements tid, tid + kThreads, ...
+#pragma unroll
+  for (int u = 0; u < KE; ++u) {
+    const int i = tid + u * kThreads;
+    k_el[u] = v_el[u] = 0;
+    if (STORE && i < D) {
+      k_el[u] = a.store.k_new[((int64_t)b * a.h_kv + h) * D + i];
+      v_el[u] = a.store.v_new[((int64_t)b * a.h_kv + h) * D + i];
+    }
   }
   for (int i = tid; i < kSampleBins; i += kThreads) sm.hist[i] = 0u;
   if (tid == 0) s_nlist = 0;
@@ -1020,9 +1037,9 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
   if (L <= a.budget) {
     mode = kModeAll;
   } else if (L > kExactMax) {
-    const double expect = (double)a.budget * kSample / (double)L;
+    const double expect = (double)a.budget * kS / (double)L;
     k = (int)ceil(expect + 4.0 * sqrt(expect) + 8.0);
-    if (k >= kSample / 2) k = 0;
+    if (k >= kS / 2) k = 0;
   }
   // decode: the page of the new token (position L - 1), read with the sample's pages
   int32_t st_page = -1;
@@ -1043,7 +1060,7 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
 #pragma unroll
     for (int u = 0; u < kIssues; ++u) {
       const int grp = warp * kWarpGroups + u * kGroupsPerIssue + gl;
-      p0[u] = sample_group_start(grp, pair, L);
+      p0[u] = sample_group_start(grp, pair, L, kSampleGroups);
       pg0[u] = bt[(p0[u] + (page_size >= kGroup ? 0 : j)) >> a.page_shift];
     }
 #pragma unroll
@@ -1066,7 +1083,7 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
       part[2 * e] = bf16_lo(w[e]);
       part[2 * e + 1] = bf16_hi(w[e]);
     }
-    for (int r = rg + kQGroups; r < G; r += kQGroups) {  // more than kQGroups rows per group
+    for (int r = rg + kQGroups; rg < kQGroups && r < G; r += kQGroups) {  // G > kQGroups
       const uint4 v = *reinterpret_cast<const uint4*>(qh + (int64_t)r * D + d8);
       const uint32_t x[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -1076,7 +1093,8 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
       }
     }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) sm.qpart[rg][d8 + e] = part[e];
+    for (int e = 0; e < 8; ++e)
+      if (rg < kQGroups) sm.qpart[rg][d8 + e] = part[e];
   }
   if (store) {  // decode: copy the new token's K and V rows into the cache
     if (st_page < 0 || (int64_t)st_page >= a.num_pages) {
@@ -1085,14 +1103,17 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
     }
     const StoreNew& st = a.store;
     const int pos = L - 1;
-    if (tid < D) {
-      s_k[tid] = bf16_to_f(k_el);
+#pragma unroll
+    for (int u = 0; u < KE; ++u) {
+      const int i = tid + u * kThreads;
+      if (i >= D) continue;
+      s_k[i] = bf16_to_f(k_el[u]);
       if (st_page >= 0) {
         const int64_t base = (int64_t)st_page * st.page_stride +
                              (int64_t)(pos & (page_size - 1)) * st.slot_stride +
                              (int64_t)h * st.head_stride;
-        st.k_cache[base + tid] = k_el;
-        st.v_cache[base + tid] = v_el;
+        st.k_cache[base + i] = k_el[u];
+        st.v_cache[base + i] = v_el[u];
       }
     }
   }
@@ -1112,7 +1133,7 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
     constexpr int DPT = D / TPJ;
     static_assert(TPJ >= 1 && TPJ <= 32 && D % TPJ == 0, "projection split");
     const int j = tid / TPJ, sub = tid % TPJ;
-    const float* mrow = sm.m + j * D;
+    const float* mrow = kMSmem ? sm.m + j * D : m_h + j * D;
     float acc = 0.f;
     double acc_k = 0.0;
     // thread sub takes dims sub, sub + TPJ, ... (interleaved: neighbouring threads read
@@ -1845,6 +1866,7 @@ cudaError_t launch_score_topk(const uint16_t* q, const float* basis, const uint8
   if (d == 128 && r == 32) return launch_t<128, Codes<32, false>>(plan, pairs, pa, sa, sel, st, pdl, s);
   if (d == 128 && r == 64) return launch_t<128, Codes<64, false>>(plan, pairs, pa, sa, sel, st, pdl, s);
   if (d == 256 && r == 64) return launch_t<256, Codes<64, false>>(plan, pairs, pa, sa, sel, st, pdl, s);
+  if (d == 576 && r == 128) return launch_t<576, Codes<128, false>>(plan, pairs, pa, sa, sel, st, pdl, s);
   return cudaErrorInvalidValue;
 }
 

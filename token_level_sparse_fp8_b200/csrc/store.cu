@@ -3,9 +3,10 @@
 //
 // BF16 = true stores bf16(M_h k) instead (two bytes per dimension: the scoring-cache ablation).
 //
-// One CTA per (KV head, range of tokens). The basis rows of the head are staged in shared memory
-// once; each warp takes one token at a time, lane j computes output j (and j+32, ...) as a
-// float64 dot product over the d dimensions and rounds it once to E4M3. At decode the same kernel
+// One CTA per (KV head, slice of basis rows, range of tokens). The slice of the head's basis rows
+// (all r rows up to r = 64; 32 rows at r = 128, where the whole basis would not fit) is staged in
+// shared memory once; each warp takes one token at a time, lane j computes output j (and j+32,
+// ...) of the slice as a float64 dot product over the d dimensions and rounds it once. At decode the same kernel
 // also writes the new token's K and V rows into the paged cache.
 #include "common.cuh"
 
@@ -15,6 +16,7 @@ namespace store_detail {
 
 constexpr int kStoreThreads = 256;
 constexpr int kStoreWarps = kStoreThreads / 32;
+constexpr int store_rows_per_cta(int r) { return r > 64 ? 32 : r; }
 
 template <int D, int R, bool DECODE, bool BF16>
 __global__ void __launch_bounds__(kStoreThreads)
@@ -27,15 +29,16 @@ __global__ void __launch_bounds__(kStoreThreads)
                  uint16_t* __restrict__ v_cache, int64_t page_stride, int64_t slot_stride,
                  int64_t head_stride, const int32_t* __restrict__ block_table, int max_pages,
                  const int32_t* __restrict__ seq_lens) {
+  constexpr int RS = store_rows_per_cta(R);
   extern __shared__ float store_smem[];
-  float* s_m = store_smem;                        // [R][D+1]
-  float* s_k = store_smem + R * (D + 1);            // [warps][D]
-  const int h = blockIdx.x;
+  float* s_m = store_smem;                        // [RS][D+1]
+  float* s_k = store_smem + RS * (D + 1);           // [warps][D]
+  const int h = blockIdx.x / (R / RS), r0 = (blockIdx.x % (R / RS)) * RS;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const float* m_h = basis + (int64_t)h * R * D;
-  for (int i = threadIdx.x; i < R * D; i += kStoreThreads) s_m[(i / D) * (D + 1) + (i % D)] = m_h[i];
+  const float* m_h = basis + ((int64_t)h * R + r0) * D;
+  for (int i = threadIdx.x; i < RS * D; i += kStoreThreads) s_m[(i / D) * (D + 1) + (i % D)] = m_h[i];
   __syncthreads();
 
   const int t0 = blockIdx.y * tokens_per_block;
@@ -63,42 +66,60 @@ __global__ void __launch_bounds__(kStoreThreads)
       continue;
     }
     const uint16_t* krow = k + (int64_t)t * k_stride_t + (int64_t)h * D;
-    // D/32 consecutive elements per lane (8 bytes for D = 128)
-    constexpr int E = D / 32;
-    static_assert(E == 4 || E == 8, "head dim");
-    uint32_t kw32[E / 2];
-    if (E == 4) {
-      uint2 v = *reinterpret_cast<const uint2*>(krow + lane * 4);
-      kw32[0] = v.x;
-      kw32[1] = v.y;
-    } else {
-      uint4 v = *reinterpret_cast<const uint4*>(krow + lane * 8);
-      kw32[0] = v.x; kw32[1] = v.y; kw32[2] = v.z; kw32[3] = v.w;
+    if (D != 128 && D != 256) {  // any even D: 32-bit words, lane-strided
+      static_assert(D % 2 == 0, "head dim");
+      const uint32_t* k32 = reinterpret_cast<const uint32_t*>(krow);
+      for (int w = lane; w < D / 2; w += 32) {
+        const uint32_t v = k32[w];
+        kw[2 * w] = bf16_lo(v);
+        kw[2 * w + 1] = bf16_hi(v);
+      }
+      if (DECODE) {
+        const int64_t base = page * page_stride + off * slot_stride + (int64_t)h * head_stride;
+        const uint32_t* v32 = reinterpret_cast<const uint32_t*>(v_new + (int64_t)t * k_stride_t + (int64_t)h * D);
+        for (int w = lane; w < D / 2; w += 32) {
+          reinterpret_cast<uint32_t*>(k_cache + base)[w] = k32[w];
+          reinterpret_cast<uint32_t*>(v_cache + base)[w] = v32[w];
+        }
+      }
     }
-#pragma unroll
-    for (int e = 0; e < E / 2; ++e) {
-      kw[lane * E + 2 * e] = bf16_lo(kw32[e]);
-      kw[lane * E + 2 * e + 1] = bf16_hi(kw32[e]);
-    }
-    if (DECODE) {
-      const int64_t base = page * page_stride + off * slot_stride + (int64_t)h * head_stride;
-      const uint16_t* vrow = v_new + (int64_t)t * k_stride_t + (int64_t)h * D;
+    if (D == 128 || D == 256) {
+      // D/32 consecutive elements per lane (8 bytes for D = 128)
+      constexpr int E = D / 32;
+      uint32_t kw32[E / 2];
       if (E == 4) {
-        *reinterpret_cast<uint2*>(k_cache + base + lane * 4) = make_uint2(kw32[0], kw32[1]);
-        *reinterpret_cast<uint2*>(v_cache + base + lane * 4) =
-            *reinterpret_cast<const uint2*>(vrow + lane * 4);
+        uint2 v = *reinterpret_cast<const uint2*>(krow + lane * 4);
+        kw32[0] = v.x;
+        kw32[1] = v.y;
       } else {
-        *reinterpret_cast<uint4*>(k_cache + base + lane * 8) =
-            make_uint4(kw32[0], kw32[1], kw32[2], kw32[3]);
-        *reinterpret_cast<uint4*>(v_cache + base + lane * 8) =
-            *reinterpret_cast<const uint4*>(vrow + lane * 8);
+        uint4 v = *reinterpret_cast<const uint4*>(krow + lane * 8);
+        kw32[0] = v.x; kw32[1] = v.y; kw32[2] = v.z; kw32[3] = v.w;
+      }
+#pragma unroll
+      for (int e = 0; e < E / 2; ++e) {
+        kw[lane * E + 2 * e] = bf16_lo(kw32[e]);
+        kw[lane * E + 2 * e + 1] = bf16_hi(kw32[e]);
+      }
+      if (DECODE) {
+        const int64_t base = page * page_stride + off * slot_stride + (int64_t)h * head_stride;
+        const uint16_t* vrow = v_new + (int64_t)t * k_stride_t + (int64_t)h * D;
+        if (E == 4) {
+          *reinterpret_cast<uint2*>(k_cache + base + lane * 4) = make_uint2(kw32[0], kw32[1]);
+          *reinterpret_cast<uint2*>(v_cache + base + lane * 4) =
+              *reinterpret_cast<const uint2*>(vrow + lane * 4);
+        } else {
+          *reinterpret_cast<uint4*>(k_cache + base + lane * 8) =
+              make_uint4(kw32[0], kw32[1], kw32[2], kw32[3]);
+          *reinterpret_cast<uint4*>(v_cache + base + lane * 8) =
+              *reinterpret_cast<const uint4*>(vrow + lane * 8);
+        }
       }
     }
     __syncwarp();
     constexpr int RB = BF16 ? 2 * R : R;  // code bytes per token
-    uint8_t* dst = score_cache + ((page * h_kv + h) * page_size + off) * RB;
+    uint8_t* dst = score_cache + ((page * h_kv + h) * page_size + off) * RB + r0 * (RB / R);
 #pragma unroll
-    for (int j0 = 0; j0 < R; j0 += 32) {
+    for (int j0 = 0; j0 < RS; j0 += 32) {
       const int j = j0 + lane;
       const float* mrow = s_m + j * (D + 1);
       double acc = 0.0;
@@ -139,8 +160,9 @@ cudaError_t dispatch_store(int d, int r, int t, int h_kv, int tpb, cudaStream_t 
                            int64_t head_stride, const int32_t* block_table, int max_pages,
                            const int32_t* seq_lens) {
   if (t <= 0) return cudaSuccess;
-  dim3 grid(h_kv, (t + tpb - 1) / tpb);
-  const size_t smem = (size_t)(r * (d + 1) + kStoreWarps * d) * sizeof(float);
+  const int rs = store_rows_per_cta(r);
+  dim3 grid(h_kv * (r / rs), (t + tpb - 1) / tpb);
+  const size_t smem = (size_t)(rs * (d + 1) + kStoreWarps * d) * sizeof(float);
 #define JSSA_STORE_CASE(DD, RR)                                                                  \
   if (d == DD && r == RR)                                                                        \
     return launch_store_t<DD, RR, DECODE, BF16>(grid, smem, s, k, k_stride_t, slot_mapping, t,   \
@@ -155,6 +177,9 @@ cudaError_t dispatch_store(int d, int r, int t, int h_kv, int tpb, cudaStream_t 
   JSSA_STORE_CASE(128, 32)
   JSSA_STORE_CASE(128, 64)
   JSSA_STORE_CASE(256, 64)
+  if (!DECODE) {
+    JSSA_STORE_CASE(576, 128)
+  }
 #undef JSSA_STORE_CASE
   return cudaErrorInvalidValue;
 }
