@@ -37,10 +37,11 @@ def parse():
     ap.add_argument("--steps", type=int, default=800)
     ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", choices=["jssa", "reference"], default="jssa")
-    ap.add_argument("--workload", choices=["llama128k", "hybrid"], default="llama128k",
+    ap.add_argument("--workload", choices=["llama128k", "hybrid", "mla"], default="llama128k",
                     help="llama128k: one 128K-context GQA layer (the headline); hybrid: a stack of "
                          "5 sliding-window layers (dense over the last 1024 positions) and 1 global "
-                         "JSSA layer, head dim 256, 64K context")
+                         "JSSA layer, head dim 256, 64K context; mla: one multi-head latent "
+                         "attention layer, 128 heads, 576-dim latent rows, 128K context")
     ap.add_argument("--batch", type=int, default=16)
     ap.add_argument("--budget", type=int, default=2048)
     ap.add_argument("--seq-len", type=int, default=131072)
@@ -765,12 +766,193 @@ def run_hybrid(args):
     print(json.dumps(line), flush=True)
 
 
+def mla_bytes(batch, seq_len, budget, page_size, dense=False):
+    """Algorithmic bytes of one MLA decode step: 128-byte scoring rows + the selected 1152-byte
+    latent rows + page table (dense: every latent row)."""
+    pages = -(-seq_len // page_size)
+    if dense:
+        return batch * (seq_len * 1152 + 4 * pages)
+    return batch * (seq_len * 128 + min(budget, seq_len) * 1152 + 4 * pages)
+
+
+def run_mla(args):
+    """One decode step of a multi-head latent attention layer (128 query heads, one latent head of
+    512 + 64 dims, 64-token pages): store of the new token's scoring row, score + top-B on the
+    latent scoring cache, absorbed latent attention over the selected rows."""
+    import torch
+    import token_level_sparse_fp8_b200 as J
+    from synth import build_paged_kv, layer_factors, sample_calibration, sample_decode_queries
+
+    rank, world, local = dist_env()
+    assert torch.cuda.is_available(), "bench needs a CUDA device"
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    group = RankGroup("nccl", dev)
+    barrier, max_over_ranks = group.barrier, group.max_over_ranks
+    batch, h_q, L, ps, B, r_lat = 16, 128, args.seq_len, 64, args.budget, 64
+    seed = 1004 + 7919 * rank
+    J._lib.load()
+    f = layer_factors(seed, 0, 1, 576)
+    # latent basis: second moments of the head-mean latent queries and of the latent rows, then
+    # the top-64 eigenvectors (the library's Jacobi solver)
+    qc, kc = sample_calibration(f, 4096, h_q, seed, device=dev)
+    qbar = qc[..., :512].double().mean(dim=1)
+    lat = kc[:, 0, :512].double()
+    gram_q = (qbar.T @ qbar)[None].contiguous()
+    gram_k = (lat.T @ lat)[None].contiguous()
+    del qc, kc, qbar, lat
+    m_lat, _ = J.compute_basis(gram_q, gram_k, r_lat)
+    m_big = J.mla_scoring_basis(m_lat)
+    kv = build_paged_kv(f, [L] * batch, ps, seed, device=dev)
+    latent = kv["k_cache"].view(kv["k_cache"].shape[0], ps, 576)
+    del kv["v_cache"]
+    bt, lens = kv["block_table"], kv["seq_lens"]
+    num_pages = latent.shape[0]
+    sc = torch.zeros((num_pages, 1, ps, 128), dtype=torch.uint8, device=dev)
+    flat = latent.view(num_pages * ps, 1, 576)
+    for p0 in range(0, num_pages, 4096):
+        p1 = min(num_pages, p0 + 4096)
+        slots = torch.arange(p0 * ps, p1 * ps, dtype=torch.int64, device=dev)
+        J.store(flat[p0 * ps:p1 * ps], slots, m_big, sc)
+    nq = 8
+    qs = [sample_decode_queries(f, batch, h_q, seed, step=i, device=dev) for i in range(nq)]
+    # the new token of each step is the last cached position (rewriting its code is idempotent)
+    t = L - 1
+    new_slots = (bt[:, t // ps].long() * ps + t % ps).contiguous()
+    k_new = flat[new_slots].contiguous()
+    idx = torch.empty((batch, 1, B), dtype=torch.int32, device=dev)
+    count = torch.empty((batch, 1), dtype=torch.int32, device=dev)
+    out = torch.empty((batch, h_q, 512), dtype=torch.bfloat16, device=dev)
+    ws_s, ws_a = J.Workspace(dev), J.Workspace(dev)
+    scale = 1.0 / math.sqrt(576.0)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        J.store(k_new, new_slots, m_big, sc)
+        J.score_topk(qs[i % nq], m_big, sc, bt, lens, B, idx, count, ws_s)
+        J.mla_attend(qs[i % nq], latent, bt, idx, count, scale, out, ws_a)
+
+    sampler = ClockSampler(local)
+    step(0)
+    torch.cuda.synchronize()
+    barrier()
+    sampler.start()
+    t_step, n_steps = timed_graph(step, args.steps, args.warmup, stream, barrier, nq)
+    clocks = sampler.stop()
+    t_step = max_over_ranks(t_step)
+
+    def attend_only(i):
+        J.mla_attend(qs[i % nq], latent, bt, idx, count, scale, out, ws_a)
+
+    t_att, n_att = timed_graph(attend_only, args.steps, args.warmup, stream, barrier, nq)
+    t_att = max_over_ranks(t_att) / n_att
+    t_dense = None
+    if not args.no_dense:
+        idx_full = torch.arange(L, dtype=torch.int32, device=dev).repeat(batch, 1).view(batch, 1, L)
+        count_full = torch.full((batch, 1), L, dtype=torch.int32, device=dev)
+        ws_d = J.Workspace(dev)
+
+        def dense(i):
+            J.mla_attend(qs[i % nq], latent, bt, idx_full, count_full, scale, out, ws_d)
+
+        dense(0)
+        t_dense, n_dense = timed_graph(dense, max(8, args.steps // 8), 8, stream, barrier, nq)
+        t_dense = max_over_ranks(t_dense) / n_dense
+    check = None
+    if rank == 0 and not args.no_check:
+        check = mla_check(qs[0], latent, bt, lens, m_big, sc, idx, count, out, B, scale, step)
+    group.close()
+    if rank != 0:
+        return
+    peak, peak_kind = peaks()
+    ms_step = t_step / n_steps * 1e3
+    bytes_step = mla_bytes(batch, L, B, ps)
+    achieved = bytes_step / (ms_step / 1e3) / 1e9
+    flops_att = 2.0 * batch * h_q * min(B, L) * (576 + 512)
+    line = {
+        "metric": "MLA decode steps/s (128 heads, 576-dim latent rows) at 128K ctx, 1xB200",
+        "value": whole_job_rate(world, n_steps, t_step),
+        "unit": "steps/s",
+        "n_gpus": world,
+        "steps": n_steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16 latent rows, e4m3 scoring cache, fp32 math",
+        "data": "synthetic",
+        "config": {
+            "workload": f"MLA layer: h_q {h_q}, latent 512 + rotary 64 (1152 B per token), scoring "
+                        f"64 latent + 64 rotary FP8 codes (128 B per token), L {L}, page {ps} "
+                        f"(permuted), B {B}, batch {batch} per GPU",
+            "global_batch": batch * world,
+            "seq_len": L,
+            "budget": B,
+            "parallelism": f"dp{world} (independent sequences per GPU)",
+            "l2": "inputs larger than L2: the 256 MiB scoring cache is streamed every step",
+        },
+        "hbm_gbs": achieved,
+        "roofline_step": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                          "frac": achieved / peak, "traffic": None, "bytes_per_step": bytes_step,
+                          "peak_kind": peak_kind},
+        "mla_attend": {"ms": t_att * 1e3, "tflops_algorithmic": flops_att / t_att / 1e12,
+                       "hbm_gbs": batch * min(B, L) * 1152 / t_att / 1e9},
+        "clocks": clocks,
+        "gpu_launches": 4 * n_steps,
+        "timing": "CUDA events around replays of a CUDA graph holding 8 consecutive steps",
+    }
+    if t_dense is not None:
+        dense_bytes = mla_bytes(batch, L, B, ps, dense=True)
+        line["dense"] = {"steps_per_s": world / t_dense, "ms_per_step": t_dense * 1e3,
+                         "hbm_gbs": dense_bytes / t_dense / 1e9, "frac": dense_bytes / t_dense / 1e9 / peak,
+                         "kind": "the same latent attention kernel over every position"}
+        line["speedup_vs_dense"] = t_dense / (ms_step / 1e3)
+    if check is not None:
+        line["oracle_check"] = check
+    print(json.dumps(line), flush=True)
+
+
+def mla_check(q, latent, bt, lens, m_big, sc, idx, count, out, budget, scale, step):
+    """Oracle agreement of the MLA step on one sequence (selection within the tie tolerance,
+    attention output within the output tolerances)."""
+    import numpy as np
+    import torch
+    from oracle import jssa as O
+    step(0)
+    torch.cuda.synchronize()
+    b = 0
+    L = int(lens[b])
+    pages = bt[b].long()
+    kv = latent[pages].double().cpu().numpy()[:, :, None]          # [pages, ps, 1, 576]
+    codes = sc[pages].cpu().numpy()
+    ident = np.arange(pages.numel(), dtype=np.int64)[None]
+    qn = q[b:b + 1].double().cpu().numpy()
+    ridx, rcount, s = O.select_step(qn, m_big.double().cpu().numpy(), codes, ident,
+                                    np.array([L]), budget)
+    rout = O.indexed_attend_step(qn, kv, kv[..., :512], ident, ridx, rcount, scale)
+    gi = idx[b, 0].cpu().numpy()
+    sym = np.setxor1d(gi[: int(count[b, 0])], ridx[0, 0, : rcount[0, 0]])
+    s = s[(0, 0)]
+    kth = np.sort(s)[::-1][budget - 1]
+    ties_ok = bool(np.all(np.abs(s[sym] - kth) <= 1e-4 * np.abs(s).max()))
+    # the GPU attended to its own index set: compare with the oracle on that same set
+    gout = O.indexed_attend_step(qn, kv, kv[..., :512], ident, idx[b:b + 1].cpu().numpy(),
+                                 count[b:b + 1].cpu().numpy(), scale)
+    err = np.abs(out[b].double().cpu().numpy() - gout[0])
+    ok = ties_ok and err.max() <= 1e-2 and err.sum() / np.abs(gout[0]).sum() <= 2e-3
+    return {"ok": bool(ok), "swaps": int(sym.size // 2), "ties_ok": ties_ok,
+            "max_abs": float(err.max()), "mean_rel": float(err.sum() / np.abs(gout[0]).sum())}
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
     elif args.workload == "hybrid":
         run_hybrid(args)
+    elif args.workload == "mla":
+        run_mla(args)
     else:
         run_jssa(args)
 

@@ -202,7 +202,7 @@ int jssa_compute_basis(const double* gram_q, const double* gram_k, int h_kv, int
                        float* basis, double* eigvals, void* ws, size_t ws_bytes,
                        jssa_stream_t stream) {
   if (h_kv <= 0 || r <= 0 || r > d) return JSSA_ERR_SHAPE;
-  if (!supported_d(d)) return JSSA_ERR_UNSUPPORTED;
+  if (!supported_d(d) && d != 512) return JSSA_ERR_UNSUPPORTED;
   if (!gram_q || !gram_k || !basis) return JSSA_ERR_NULL;
   const size_t need = basis_ws_bytes(h_kv, d);
   if (!ws || ws_bytes < need) return JSSA_ERR_WORKSPACE;

@@ -4,7 +4,8 @@
 //
 // One CTA per KV head runs a parallel cyclic Jacobi eigensolver in float64: the d x d matrix
 // lives in shared memory at d = 128 (rows padded by one element) and in the workspace at
-// d = 256 (512 KB: too large for shared memory; it stays in L2), the eigenvectors are
+// d = 256 and 512 (the latent basis of multi-head latent attention; too large for shared
+// memory, it stays in L2), the eigenvectors are
 // accumulated as the rows of V^T in the workspace. Each sweep is d-1 rounds of the round-robin ("circle") pairing,
 // so the d/2 rotations of a round touch disjoint index pairs and run in parallel: rotation
 // parameters, then the row update (A <- J^T A, V^T <- J^T V^T), then the column update
@@ -181,9 +182,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 cudaError_t launch_basis(const double* gram_q, const double* gram_k, int h_kv, int d, int r,
                          float* basis, double* eigvals, double* ws, cudaStream_t s) {
   if (h_kv <= 0) return cudaSuccess;
-  if (d != 128 && d != 256) return cudaErrorInvalidValue;
+  if (d != 128 && d != 256 && d != 512) return cudaErrorInvalidValue;
   const size_t smem = d == 128 ? (size_t)d * (d + 1) * sizeof(double) : 0;
-  auto kern = d == 128 ? basis_detail::basis_kernel<128> : basis_detail::basis_kernel<256>;
+  auto kern = d == 128 ? basis_detail::basis_kernel<128>
+                       : d == 256 ? basis_detail::basis_kernel<256> : basis_detail::basis_kernel<512>;
   cudaError_t e = configure_kernel((const void*)kern, (int)smem, false);
   if (e != cudaSuccess) return e;
   kern<<<h_kv, basis_detail::kThreads, smem, s>>>(gram_q, gram_k, r, basis, eigvals, ws);

@@ -9,13 +9,16 @@
 // token, one "KV head") and the index set of score_topk run with h_kv = 1 on the latent scoring
 // cache.
 //
-// Grid (splits, batch, h_q / 16). A CTA owns 16 query heads of one sequence and one contiguous
-// slice of its index set. Its 4 warps share every 16-token tile of latent rows (a CTA-wide ring
+// Grid (h_q / 16, splits, batch): a CTA owns 16 query heads of one sequence and one contiguous
+// slice of its index set; the head blocks of one slice are neighbours in launch order, so the
+// rows they all read come from L2 after the first. Its 4 warps share every 16-token tile of latent rows (a CTA-wide ring
 // of kStages shared-memory stages filled by 16-byte cp.async, chunk c of a row at
-// (c & ~7) | ((c ^ row) & 7) so that ldmatrix reads are conflict-free). Each warp computes the
-// scores S = Q K^T of the 16 heads x 16 tokens on the tensor cores (mma.sync m16n8k16 bf16,
-// fp32 accumulate; the 16 heads are the M rows) and keeps its own online softmax, then adds
-// P V into its quarter (128 dims) of the output (P split into bf16 high and low parts). Splits
+// (c & ~7) | ((c ^ row) & 7) so that ldmatrix reads are conflict-free). The scores S = Q K^T of
+// the 16 heads x 16 tokens are computed on the tensor cores (mma.sync m16n8k16 bf16, fp32
+// accumulate; the 16 heads are the M rows) with the 576 dimensions split over the 4 warps (9
+// k-blocks each) and the partial sums added through shared memory; every warp then keeps the
+// same online softmax and adds P V into its quarter (128 dims) of the output (P split into bf16
+// high and low parts). Splits
 // of one (sequence, head block) merge through fp32 partials and a ticket, as the GQA attention.
 #include "common.cuh"
 
@@ -62,11 +65,12 @@ __device__ __forceinline__ uint32_t swz(int row, int c) {
 __global__ void __launch_bounds__(kThreads, 2) mla_kernel(Args a, int chunk, int splits) {
   extern __shared__ __align__(128) uint8_t mla_smem[];
   __shared__ int64_t s_off[kMaxChunk];
+  __shared__ float s_part[kWarps][32][8];  // each warp's partial S, in fragment order
   __shared__ int s_last;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
-  const int split = blockIdx.x, b = blockIdx.y, hb = blockIdx.z;
-  const int n_hb = gridDim.z;
+  const int hb = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
+  const int n_hb = gridDim.x;
   const int max_len = a.max_pages * a.page_size;
   const uint32_t s_q = smem_u32(mla_smem);
   const uint32_t ring = s_q + kQBytes;
@@ -147,15 +151,27 @@ __global__ void __launch_bounds__(kThreads, 2) mla_kernel(Args a, int chunk, int
     __syncthreads();
     const uint32_t st = ring + (i % kStages) * kTileBytes;
 
-    // S (16 heads x 16 tokens) = Q K^T over the 576 dimensions
+    // S (16 heads x 16 tokens) = Q K^T over the 576 dimensions: this warp's 9 k-blocks, then
+    // the four partial sums through shared memory (the same fragment order in every warp)
     float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-    for (int kb = 0; kb < kDK / 16; ++kb) {
+    constexpr int kKB = kDK / 16 / kWarps;  // 9
+#pragma unroll
+    for (int u = 0; u < kKB; ++u) {
+      const int kb = warp * kKB + u;
       uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
       ldsm_x4(s_q + swz(qa_row, 2 * kb + qa_half), a0, a1, a2, a3);
       ldsm_x4(st + swz(kb_row, 2 * kb + kb_half), b0, b1, b2, b3);
       mma_bf16(s0, a0, a1, a2, a3, b0, b1);
       mma_bf16(s1, a0, a1, a2, a3, b2, b3);
+    }
+    *reinterpret_cast<float4*>(&s_part[warp][lane][0]) = make_float4(s0[0], s0[1], s0[2], s0[3]);
+    *reinterpret_cast<float4*>(&s_part[warp][lane][4]) = make_float4(s1[0], s1[1], s1[2], s1[3]);
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      s0[e] = s_part[0][lane][e] + s_part[1][lane][e] + s_part[2][lane][e] + s_part[3][lane][e];
+      s1[e] = s_part[0][lane][4 + e] + s_part[1][lane][4 + e] + s_part[2][lane][4 + e] +
+              s_part[3][lane][4 + e];
     }
     // rows g (s[0], s[1]) and g + 8 (s[2], s[3]); columns: tokens 2t, 2t + 1 (+ 8 in s1)
     const int j0 = i * kTile;
@@ -337,7 +353,7 @@ cudaError_t launch_mla(const uint16_t* q, const uint16_t* kv, int64_t page_strid
   Args a = {q, kv, page_stride, slot_stride, block_table, max_pages, idx, count, batch, h_q,
             budget, num_pages, page_size, scale, out, ws};
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(plan.splits, batch, h_q / kHeads);
+  cfg.gridDim = dim3(h_q / kHeads, plan.splits, batch);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = s;
