@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-check", action="store_true", help="skip the sampled oracle check")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--mla-batch", type=int, default=16, help="sequences of the mla workload")
     return ap.parse_args()
 
 
@@ -789,7 +790,7 @@ def run_mla(args):
     dev = torch.device("cuda", local)
     group = RankGroup("nccl", dev)
     barrier, max_over_ranks = group.barrier, group.max_over_ranks
-    batch, h_q, L, ps, B, r_lat = 16, 128, args.seq_len, 64, args.budget, 64
+    batch, h_q, L, ps, B, r_lat = args.mla_batch, 128, args.seq_len, 64, args.budget, 64
     seed = 1004 + 7919 * rank
     J._lib.load()
     f = layer_factors(seed, 0, 1, 576)

@@ -118,14 +118,19 @@ __global__ void __launch_bounds__(kThreads, 2) mla_kernel(Args a, int chunk, int
   pdl_trigger();
 
   const int n_tiles = (n_mine + kTile - 1) / kTile;
+  // copies of a tile: 8 threads per row, thread q of a row takes chunks q, q + 8, ..., q + 64 (a
+  // warp instruction covers 128 contiguous bytes of each of its 4 rows); the swizzle only flips
+  // the low 3 bits of the chunk index, so a thread's destinations are 128 bytes apart
+  static_assert(kThreads == kTile * 8 && kChunks % 8 == 0, "copy split");
+  const int cp_row = tid >> 3, cp_q = tid & 7;
+  const uint32_t cp_dst = (uint32_t)(cp_row * kRowBytes + ((cp_q ^ (cp_row & 7)) << 4));
   auto issue = [&](int tl, int st) {
-    for (int i = tid; i < kTile * kChunks; i += kThreads) {
-      const int row = i / kChunks, c = i % kChunks;
-      const int j = tl * kTile + row;
-      const int64_t off = j < n_mine ? s_off[j] : -1;
-      cp_async16(ring + st * kTileBytes + swz(row, c), a.kv + (off >= 0 ? off : 0) + c * 8,
-                 off >= 0 ? 16 : 0);
-    }
+    const int j = tl * kTile + cp_row;
+    const int64_t off = j < n_mine ? s_off[j] : -1;
+    const uint16_t* src = a.kv + (off >= 0 ? off : 0) + cp_q * 8;
+    const uint32_t dst = ring + st * kTileBytes + cp_dst;
+#pragma unroll
+    for (int k = 0; k < kChunks / 8; ++k) cp_async16(dst + 128 * k, src + 64 * k, off >= 0 ? 16 : 0);
   };
 #pragma unroll
   for (int i = 0; i < kStages - 1; ++i) {
