@@ -847,6 +847,12 @@ def run_mla(args):
 
     t_att, n_att = timed_graph(attend_only, args.steps, args.warmup, stream, barrier, nq)
     t_att = max_over_ranks(t_att) / n_att
+
+    def score_only(i):
+        J.score_topk(qs[i % nq], m_big, sc, bt, lens, B, idx, count, ws_s)
+
+    t_sc, n_sc = timed_graph(score_only, args.steps, args.warmup, stream, barrier, nq)
+    t_sc = max_over_ranks(t_sc) / n_sc
     t_dense = None
     if not args.no_dense:
         idx_full = torch.arange(L, dtype=torch.int32, device=dev).repeat(batch, 1).view(batch, 1, L)
@@ -899,6 +905,7 @@ def run_mla(args):
                           "peak_kind": peak_kind},
         "mla_attend": {"ms": t_att * 1e3, "tflops_algorithmic": flops_att / t_att / 1e12,
                        "hbm_gbs": batch * min(B, L) * 1152 / t_att / 1e9},
+        "score_topk": {"ms": t_sc * 1e3, "hbm_gbs": batch * (L * 128 + 4 * (-(-L // ps))) / t_sc / 1e9},
         "clocks": clocks,
         "gpu_launches": 4 * n_steps,
         "timing": "CUDA events around replays of a CUDA graph holding 8 consecutive steps",

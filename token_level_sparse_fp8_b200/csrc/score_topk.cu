@@ -1083,6 +1083,7 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
       part[2 * e] = bf16_lo(w[e]);
       part[2 * e + 1] = bf16_hi(w[e]);
     }
+#pragma unroll 4
     for (int r = rg + kQGroups; rg < kQGroups && r < G; r += kQGroups) {  // G > kQGroups
       const uint4 v = *reinterpret_cast<const uint4*>(qh + (int64_t)r * D + d8);
       const uint32_t x[4] = {v.x, v.y, v.z, v.w};
@@ -1128,12 +1129,58 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
   __syncthreads();  // qbar
 
   // ---- p = M_h qbar and, at decode, the new token's code e4m3(M_h k) (or bf16(M_h k)) ----------
-  {
+  if (!kMSmem) {
+    // M_h from global memory: each warp owns R / kWarps output rows and reads them together,
+    // lanes striding over the dimensions (coalesced 128-byte reads, R / kWarps independent loads
+    // per step), then one warp reduction per row
+    constexpr int kRW = R / kWarps;
+    static_assert(D % 32 == 0 && R % kWarps == 0, "projection split");
+    float acc[kRW];
+    double acc_k[kRW];
+#pragma unroll
+    for (int jj = 0; jj < kRW; ++jj) {
+      acc[jj] = 0.f;
+      acc_k[jj] = 0.0;
+    }
+    const float* mbase = m_h + (int64_t)(warp * kRW) * D;
+#pragma unroll 2
+    for (int e = lane; e < D; e += 32) {
+      const float qv = s_qbar[e];
+      const double kv = store ? (double)s_k[e] : 0.0;
+#pragma unroll
+      for (int jj = 0; jj < kRW; ++jj) {
+        const float mv = __ldg(mbase + jj * D + e);
+        acc[jj] = fmaf(mv, qv, acc[jj]);
+        if (store) acc_k[jj] = fma((double)mv, kv, acc_k[jj]);
+      }
+    }
+#pragma unroll
+    for (int jj = 0; jj < kRW; ++jj) {
+      float v = acc[jj];
+      double vk = acc_k[jj];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (store) vk += __shfl_xor_sync(0xffffffffu, vk, o);
+      }
+      if (lane == 0) {
+        const int j = warp * kRW + jj;
+        s_p[j] = v;
+        if (store && st_page >= 0) {
+          const int pos = L - 1;
+          uint8_t* row = a.store.score_cache +
+              (((int64_t)st_page * a.h_kv + h) * page_size + (pos & (page_size - 1))) * RB;
+          if (C::kBF16) reinterpret_cast<uint16_t*>(row)[j] = f64_to_bf16(vk);
+          else row[j] = f64_to_e4m3(vk);
+        }
+      }
+    }
+  } else {
     constexpr int TPJ = kThreads / R;  // threads per output
     constexpr int DPT = D / TPJ;
     static_assert(TPJ >= 1 && TPJ <= 32 && D % TPJ == 0, "projection split");
     const int j = tid / TPJ, sub = tid % TPJ;
-    const float* mrow = kMSmem ? sm.m + j * D : m_h + j * D;
+    const float* mrow = sm.m + j * D;
     float acc = 0.f;
     double acc_k = 0.0;
     // thread sub takes dims sub, sub + TPJ, ... (interleaved: neighbouring threads read
