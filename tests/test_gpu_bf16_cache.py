@@ -77,3 +77,19 @@ def test_bf16_score_topk(case, budget):
     for b in range(len(case.seq_lens)):
         for h in range(case.h_kv):
             check_selection(gi[b, h], gc[b, h], ref_idx[b, h], ref_count[b, h], s[(b, h)], budget)
+
+
+def test_bf16_score_topk_small_pages_and_short():
+    J = jssa()
+    c = Case([17000, 200, 0], page_size=4, seed=1410, calib=1024, extra_pages=3)
+    codes, _ = bf16_cache(c)
+    budget = 256
+    sc = torch.from_numpy(codes.view(np.int16)).view(torch.bfloat16).cuda()
+    idx, count = J.score_topk(c.gpu(c.q), c.gpu_np(c.m32), sc, c.gpu(c.block_table),
+                              c.gpu(c.seq_lens_t), budget)
+    ref_idx, ref_count, s = O.select_step(c.np_q, c.m32.astype(np.float64), codes, c.np_bt,
+                                          c.np_lens, budget)
+    gi, gc = idx.cpu().numpy(), count.cpu().numpy()
+    for b in range(len(c.seq_lens)):
+        for h in range(c.h_kv):
+            check_selection(gi[b, h], gc[b, h], ref_idx[b, h], ref_count[b, h], s[(b, h)], budget)

@@ -153,3 +153,17 @@ def test_hybrid_calibration():
         # and its objective may fall on either side of the float64 optimum by a few 1e-9
         assert abs(O.l_marg(p_gpu, a_q, a_k) - opt) <= 1e-7
         assert np.max(np.abs(lam[h] - res["eigvals"][h])) <= 1e-5 * lam[h, 0]
+
+
+def test_hybrid_small_pages_score_topk():
+    # 8-token pages: tiles span two pages (the per-token page path of the scan and the sample)
+    case = Case([18000, 999], page_size=8, seed=1330, calib=1024, extra_pages=4, **HYBRID)
+    J = jssa()
+    budget = 600
+    idx, count = J.score_topk(case.gpu(case.q), case.gpu_np(case.m32), case.gpu_np(case.codes),
+                              case.gpu(case.block_table), case.gpu(case.seq_lens_t), budget)
+    ref_idx, ref_count, s = _select_oracle(case, budget)
+    gi, gc = idx.cpu().numpy(), count.cpu().numpy()
+    for b in range(len(case.seq_lens)):
+        for h in range(case.h_kv):
+            check_selection(gi[b, h], gc[b, h], ref_idx[b, h], ref_count[b, h], s[(b, h)], budget)

@@ -92,3 +92,24 @@ def test_mla_attend(case, budget):
     ref = O.indexed_attend_step(f64(case.q), case.np_kv, case.np_kv[..., :512], case.np_bt, ref_idx,
                                 ref_count, scale)
     check_output(f64(out), ref)
+
+
+def test_mla_short_empty_and_exact_budget():
+    # an empty sequence (zeros out), one below the budget (every position), one exactly at it
+    J = jssa()
+    c = MlaCase([0, 100, 512], seed=1510)
+    budget = 512
+    idx, count = J.score_topk(c.q.cuda(), torch.from_numpy(c.m_big).cuda(),
+                              torch.from_numpy(c.codes).cuda(), c.bt.cuda(), c.lens_t.cuda(), budget)
+    assert count.cpu().numpy().ravel().tolist() == [0, 100, 512]
+    gi = idx.cpu().numpy()
+    assert np.all(gi[0, 0] == -1)
+    assert np.array_equal(gi[1, 0, :100], np.arange(100)) and np.all(gi[1, 0, 100:] == -1)
+    assert np.array_equal(gi[2, 0], np.arange(512))
+    scale = 1.0 / math.sqrt(D)
+    kv = c.kv.cuda().view(c.kv.shape[0], PS, D)
+    out = J.mla_attend(c.q.cuda(), kv, c.bt.cuda(), idx, count, scale)
+    ref = O.indexed_attend_step(f64(c.q), c.np_kv, c.np_kv[..., :512], c.np_bt, gi,
+                                count.cpu().numpy(), scale)
+    check_output(f64(out), ref)
+    assert torch.count_nonzero(out[0]).item() == 0
