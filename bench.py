@@ -471,7 +471,7 @@ def run_jssa(args):
     n_steps = reps * nq
     t_step = max_over_ranks(e0.elapsed_time(e1) / 1e3)
     del g_step
-    launches_per_step = 3
+    launches_per_step = 4  # prep, scan, select, attention
 
     # per-kernel device times (same configuration, each kernel launched alone)
     idx, count = layer.idx, layer.count
@@ -754,7 +754,7 @@ def run_hybrid(args):
                           "frac": achieved / peak, "traffic": None, "bytes_per_step": bytes_step,
                           "peak_kind": peak_kind},
         "clocks": clocks,
-        "gpu_launches": (w.layers - 1 + 3) * n_steps,
+        "gpu_launches": (w.layers - 1 + 4) * n_steps,  # a dense kernel per local layer + 4
         "timing": "CUDA events around replays of a CUDA graph holding 8 consecutive stack steps",
     }
     if t_dense is not None:
@@ -907,7 +907,7 @@ def run_mla(args):
                        "hbm_gbs": batch * min(B, L) * 1152 / t_att / 1e9},
         "score_topk": {"ms": t_sc * 1e3, "hbm_gbs": batch * (L * 128 + 4 * (-(-L // ps))) / t_sc / 1e9},
         "clocks": clocks,
-        "gpu_launches": 4 * n_steps,
+        "gpu_launches": 5 * n_steps,  # store, prep, scan, select, latent attention
         "timing": "CUDA events around replays of a CUDA graph holding 8 consecutive steps",
     }
     if t_dense is not None:
