@@ -47,7 +47,7 @@ def parse():
     ap.add_argument("--seq-len", type=int, default=131072)
     ap.add_argument("--no-dense", action="store_true", help="skip the dense baseline timing")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--no-check", action="store_true", help="skip the sampled oracle check")
+    ap.add_argument("--no-check", action="store_true", help="skip the oracle agreement in the CPU baseline leg")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--mla-batch", type=int, default=16, help="sequences of the mla workload")
     return ap.parse_args()
@@ -318,57 +318,143 @@ def oracle_step_for_pair(q_b, k, v, sc, m, bt, w):
     return idx, count, s, out
 
 
-def cpu_baseline(state, w, seconds):
+def pair_agreement(s, sym, budget, go, rout):
+    """Oracle agreement of one (sequence, KV head): the index sets may differ only at near-ties,
+    the outputs within the parity tolerances."""
+    import numpy as np
+    kth = np.sort(s)[::-1][min(budget, s.shape[0]) - 1]
+    ties_ok = bool(np.all(np.abs(s[sym] - kth) <= 1e-4 * np.abs(s).max()))
+    err = np.abs(go - rout)
+    rel = float(err.sum() / max(np.abs(rout).sum(), 1e-300))
+    return {"swaps": int(sym.size // 2), "ties_ok": ties_ok, "max_abs": float(err.max()),
+            "mean_rel": rel, "ok": ties_ok and float(err.max()) <= 1e-2 and rel <= 2e-3}
+
+
+def cpu_baseline(state, w, seconds, check=True):
     """The oracle, as it stands, on host cores: select + attend for (sequence, KV head) pairs of
-    the timed workload, repeated until about `seconds` of CPU time; scaled to one whole step."""
+    the timed workload, repeated until about `seconds` of CPU time; scaled to one whole step.
+    The first oracle result of each pair is also compared with the GPU step's (agreement)."""
+    import numpy as np
     import torch
     cores = len(os.sched_getaffinity(0))
-    q = state["qs"][0].to(torch.float64).cpu().numpy()
+    layer = state["layer"]
+    q0 = state["qs"][0]
+    gout, gidx, gcount = layer.step(q0, state["k_new"], state["v_new"])
+    torch.cuda.synchronize()
+    q = q0.to(torch.float64).cpu().numpy()
     g = w.group
     pairs = [(0, 0), (w.batch - 1, w.h_kv - 1)]
     inputs = [(q[b, h * g : (h + 1) * g],) + oracle_pair_inputs(state, w, b, h) for b, h in pairs]
+    agreement = []
     done, t_total = 0, 0.0
     while t_total < seconds or done < 2:
         qb, k, v, sc, m, bt = inputs[done % len(inputs)]
         t0 = time.perf_counter()
-        oracle_step_for_pair(qb, k, v, sc, m, bt, w)
+        ridx, rcount, s, rout = oracle_step_for_pair(qb, k, v, sc, m, bt, w)
         t_total += time.perf_counter() - t0
+        if check and done < len(pairs):
+            b, h = pairs[done]
+            gi = gidx[b, h].cpu().numpy()
+            sym = np.setxor1d(gi[: int(gcount[b, h])], ridx[0, 0, : rcount[0, 0]])
+            go = gout[b, h * g : (h + 1) * g].double().cpu().numpy()
+            agreement.append(dict(pair=[b, h], **pair_agreement(s[(0, 0)], sym, w.budget, go, rout[0])))
         done += 1
     per_pair = t_total / done
     steps_per_s = 1.0 / (per_pair * w.batch * w.h_kv)
-    return {"value": steps_per_s, "unit": "steps/s", "cores": cores, "kind": "oracle",
-            "sample": f"{done} oracle calls on 2 (sequence, KV head) pairs of the timed workload "
-                      f"(score+top-B+attend over 131072 tokens, float64 NumPy), {t_total:.1f} s; "
-                      f"steps/s = 1 / (time per pair x {w.batch * w.h_kv} pairs per step)"}
+    res = {"value": steps_per_s, "unit": "steps/s", "cores": cores, "kind": "oracle",
+           "sample": f"{done} oracle calls on 2 (sequence, KV head) pairs of the timed workload "
+                     f"(score+top-B+attend over {w.seq_len} tokens, float64 NumPy), {t_total:.1f} s; "
+                     f"steps/s = 1 / (time per pair x {w.batch * w.h_kv} pairs per step)"}
+    if check:
+        res["agreement"] = {"ok": all(a["ok"] for a in agreement), "pairs": agreement}
+    return res
 
 
-def sampled_check(state, w, n_pairs=2):
-    """Oracle agreement on a few (sequence, KV head) pairs of the timed configuration."""
+def cpu_baseline_hybrid(state, w, seconds, local_kv, q0, scale, check=True):
+    """The oracle on host cores for the hybrid stack: the global layer's select + attend on
+    (sequence, KV head) pairs (as for the single-layer workload) and one sliding-window layer's
+    dense attention on a (sequence, KV head) pair; one stack step = pairs x (global + local
+    layers x window)."""
     import numpy as np
     import torch
-    layer = state["layer"]
-    q = state["qs"][0]
-    out, idx, count = layer.step(q, state["k_new"], state["v_new"])
+    import token_level_sparse_fp8_b200 as J
+    from oracle import jssa as O
+    glob = cpu_baseline(state, w, seconds / 2, check)
+    t_glob = 1.0 / (glob["value"] * w.batch * w.h_kv)
+    gout = J.dense_decode(q0, local_kv["k_cache"], local_kv["v_cache"], local_kv["block_table"],
+                          local_kv["seq_lens"], scale, w.window)
     torch.cuda.synchronize()
-    qn = q.to(torch.float64).cpu().numpy()
-    rng = np.random.default_rng(0)
-    res = []
-    for _ in range(n_pairs):
-        b, h = int(rng.integers(w.batch)), int(rng.integers(w.h_kv))
-        k, v, sc, m, bt = oracle_pair_inputs(state, w, b, h)
-        g = w.group
-        ridx, rcount, s, rout = oracle_step_for_pair(qn[b, h * g : (h + 1) * g], k, v, sc, m, bt, w)
-        gi = idx[b, h].cpu().numpy()
-        sym = np.setxor1d(gi[: int(count[b, h])], ridx[0, 0, : rcount[0, 0]])
-        s = s[(0, 0)]
-        kth = np.sort(s)[::-1][w.budget - 1]
-        ties_ok = bool(np.all(np.abs(s[sym] - kth) <= 1e-4 * np.abs(s).max()))
-        go = out[b, h * g : (h + 1) * g].double().cpu().numpy()
+    b, h, g = 0, 0, w.group
+    bt = local_kv["block_table"][b].long()
+    k = local_kv["k_cache"][bt][:, :, h : h + 1].double().cpu().numpy()
+    v = local_kv["v_cache"][bt][:, :, h : h + 1].double().cpu().numpy()
+    ident = np.arange(bt.numel(), dtype=np.int64)[None]
+    qb = q0[b : b + 1, h * g : (h + 1) * g].double().cpu().numpy()
+    lens = np.array([int(local_kv["seq_lens"][b])])
+    done, t_total, rout = 0, 0.0, None
+    while t_total < seconds / 2 or done < 2:
+        t0 = time.perf_counter()
+        rout = O.dense_step(qb, k, v, ident, lens, scale, w.window)
+        t_total += time.perf_counter() - t0
+        done += 1
+    t_local = t_total / done
+    per_step = w.batch * w.h_kv * (t_glob + (w.layers - 1) * t_local)
+    res = {"value": 1.0 / per_step, "unit": "steps/s", "cores": glob["cores"], "kind": "oracle",
+           "sample": f"global layer: {glob['sample']}; sliding-window layer: {done} oracle dense "
+                     f"calls over {w.window} positions of one (sequence, KV head), {t_total:.1f} s; "
+                     f"steps/s = 1 / ({w.batch * w.h_kv} pairs x (global + {w.layers - 1} x local))"}
+    if check:
+        go = gout[b, h * g : (h + 1) * g].double().cpu().numpy()
         err = np.abs(go - rout[0])
-        res.append({"pair": [b, h], "swaps": int(sym.size // 2), "ties_ok": ties_ok,
-                    "max_abs": float(err.max()), "mean_rel": float(err.sum() / np.abs(rout[0]).sum())})
-    ok = all(r["ties_ok"] and r["max_abs"] <= 1e-2 and r["mean_rel"] <= 2e-3 for r in res)
-    return {"ok": ok, "pairs": res}
+        rel = float(err.sum() / max(np.abs(rout[0]).sum(), 1e-300))
+        local = {"pair": [b, h], "max_abs": float(err.max()), "mean_rel": rel,
+                 "ok": float(err.max()) <= 1e-2 and rel <= 2e-3}
+        res["agreement"] = {"ok": glob["agreement"]["ok"] and local["ok"],
+                            "global": glob["agreement"]["pairs"], "sliding_window": local}
+    return res
+
+
+def cpu_baseline_mla(q, latent, bt, lens, m_big, sc, idx, count, out, budget, scale, step,
+                     seconds, check=True):
+    """The oracle on host cores for the MLA step on one sequence (select over the latent scoring
+    cache + latent attention over the selected rows), repeated for about `seconds`; the first
+    result is also compared with the GPU step's (selection within the tie tolerance, output within
+    the output tolerances on the GPU's own index set)."""
+    import numpy as np
+    import torch
+    from oracle import jssa as O
+    cores = len(os.sched_getaffinity(0))
+    step(0)
+    torch.cuda.synchronize()
+    batch = q.shape[0]
+    b = 0
+    L = int(lens[b])
+    pages = bt[b].long()
+    kv = latent[pages].double().cpu().numpy()[:, :, None]          # [pages, ps, 1, 576]
+    codes = sc[pages].cpu().numpy()
+    ident = np.arange(pages.numel(), dtype=np.int64)[None]
+    qn = q[b:b + 1].double().cpu().numpy()
+    mn = m_big.double().cpu().numpy()
+    done, t_total = 0, 0.0
+    while t_total < seconds or done < 1:
+        t0 = time.perf_counter()
+        ridx, rcount, s = O.select_step(qn, mn, codes, ident, np.array([L]), budget)
+        O.indexed_attend_step(qn, kv, kv[..., :512], ident, ridx, rcount, scale)
+        t_total += time.perf_counter() - t0
+        done += 1
+    res = {"value": 1.0 / (t_total / done * batch), "unit": "steps/s", "cores": cores,
+           "kind": "oracle",
+           "sample": f"{done} oracle calls (select over {L} latent scoring rows + latent attention "
+                     f"over the top {budget}) on one sequence of the timed workload, float64 NumPy, "
+                     f"{t_total:.1f} s; steps/s = 1 / (time per sequence x {batch} sequences)"}
+    if check:
+        gi = idx[b, 0].cpu().numpy()
+        sym = np.setxor1d(gi[: int(count[b, 0])], ridx[0, 0, : rcount[0, 0]])
+        gout = O.indexed_attend_step(qn, kv, kv[..., :512], ident, idx[b:b + 1].cpu().numpy(),
+                                     count[b:b + 1].cpu().numpy(), scale)
+        res["agreement"] = pair_agreement(s[(0, 0)], sym, budget, out[b].double().cpu().numpy(),
+                                          gout[0])
+    return res
 
 
 # ------------------------------------------------------------------------------------------------
@@ -559,13 +645,9 @@ def run_jssa(args):
     h2d = qs[0].numel() * 2 + k_new.numel() * 2 + v_new.numel() * 2
     d2h = out.numel() * 2
 
-    check = None
-    if rank == 0 and not args.no_check:
-        check = sampled_check(state, w)
-
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        cpu = cpu_baseline(state, w, args.cpu_seconds)
+        cpu = cpu_baseline(state, w, args.cpu_seconds, check=not args.no_check)
 
     group.close()
     if rank != 0:
@@ -637,8 +719,6 @@ def run_jssa(args):
     if t_dense is not None:
         line["ablation_gather"]["attend_speedup_vs_dense"] = {
             "gather_free": t_dense / t_attend, "gather_then_attend": t_dense / t_gta}
-    if check is not None:
-        line["oracle_check"] = check
     if cpu is not None:
         line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)
@@ -715,9 +795,10 @@ def run_hybrid(args):
     if not args.no_dense:
         t_dense, n_dense = timed_graph(dense_step, max(8, args.steps // 4), 8, stream, barrier, nq)
         t_dense = max_over_ranks(t_dense) / n_dense
-    check = None
-    if rank == 0 and not args.no_check:
-        check = sampled_check(state, w)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline_hybrid(state, w, args.cpu_seconds, locals_[0], qs[0], scale,
+                                  check=not args.no_check)
     group.close()
     if rank != 0:
         return
@@ -762,8 +843,8 @@ def run_hybrid(args):
         line["dense"] = {"steps_per_s": world / t_dense, "ms_per_step": t_dense * 1e3,
                          "hbm_gbs": dense_bytes / t_dense / 1e9, "frac": dense_bytes / t_dense / 1e9 / peak}
         line["speedup_vs_dense"] = t_dense / (ms_step / 1e3)
-    if check is not None:
-        line["oracle_check"] = check
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)
 
 
@@ -865,9 +946,10 @@ def run_mla(args):
         dense(0)
         t_dense, n_dense = timed_graph(dense, max(8, args.steps // 8), 8, stream, barrier, nq)
         t_dense = max_over_ranks(t_dense) / n_dense
-    check = None
-    if rank == 0 and not args.no_check:
-        check = mla_check(qs[0], latent, bt, lens, m_big, sc, idx, count, out, B, scale, step)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline_mla(qs[0], latent, bt, lens, m_big, sc, idx, count, out, B, scale, step,
+                               args.cpu_seconds, check=not args.no_check)
     group.close()
     if rank != 0:
         return
@@ -916,41 +998,9 @@ def run_mla(args):
                          "hbm_gbs": dense_bytes / t_dense / 1e9, "frac": dense_bytes / t_dense / 1e9 / peak,
                          "kind": "the same latent attention kernel over every position"}
         line["speedup_vs_dense"] = t_dense / (ms_step / 1e3)
-    if check is not None:
-        line["oracle_check"] = check
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)
-
-
-def mla_check(q, latent, bt, lens, m_big, sc, idx, count, out, budget, scale, step):
-    """Oracle agreement of the MLA step on one sequence (selection within the tie tolerance,
-    attention output within the output tolerances)."""
-    import numpy as np
-    import torch
-    from oracle import jssa as O
-    step(0)
-    torch.cuda.synchronize()
-    b = 0
-    L = int(lens[b])
-    pages = bt[b].long()
-    kv = latent[pages].double().cpu().numpy()[:, :, None]          # [pages, ps, 1, 576]
-    codes = sc[pages].cpu().numpy()
-    ident = np.arange(pages.numel(), dtype=np.int64)[None]
-    qn = q[b:b + 1].double().cpu().numpy()
-    ridx, rcount, s = O.select_step(qn, m_big.double().cpu().numpy(), codes, ident,
-                                    np.array([L]), budget)
-    rout = O.indexed_attend_step(qn, kv, kv[..., :512], ident, ridx, rcount, scale)
-    gi = idx[b, 0].cpu().numpy()
-    sym = np.setxor1d(gi[: int(count[b, 0])], ridx[0, 0, : rcount[0, 0]])
-    s = s[(0, 0)]
-    kth = np.sort(s)[::-1][budget - 1]
-    ties_ok = bool(np.all(np.abs(s[sym] - kth) <= 1e-4 * np.abs(s).max()))
-    # the GPU attended to its own index set: compare with the oracle on that same set
-    gout = O.indexed_attend_step(qn, kv, kv[..., :512], ident, idx[b:b + 1].cpu().numpy(),
-                                 count[b:b + 1].cpu().numpy(), scale)
-    err = np.abs(out[b].double().cpu().numpy() - gout[0])
-    ok = ties_ok and err.max() <= 1e-2 and err.sum() / np.abs(gout[0]).sum() <= 2e-3
-    return {"ok": bool(ok), "swaps": int(sym.size // 2), "ties_ok": ties_ok,
-            "max_abs": float(err.max()), "mean_rel": float(err.sum() / np.abs(gout[0]).sum())}
 
 
 def main():
