@@ -27,8 +27,9 @@
  *   [batch, max_pages], seq_lens int32 [batch]. page_size is a power of two.
  * - Scoring cache: uint8 E4M3 codes laid out [num_pages, h_kv, page_size, r] (one contiguous
  *   run of page_size*r bytes per page and KV head), same page numbering as the KV cache.
- * - Basis: float32 [h_kv, r, d], rows orthonormal (output of jssa_compute_basis); the score
- *   entry points want it, and the scoring cache, 16-byte aligned (JSSA_ERR_ALIGN otherwise).
+ * - Basis: float32 [h_kv, r, d], rows orthonormal (output of jssa_compute_basis); the store
+ *   and score entry points want it, the scoring cache and the queries q 16-byte aligned
+ *   (JSSA_ERR_ALIGN otherwise).
  * - Index sets: int32 idx [batch, h_kv, budget] holds logical positions in ascending order,
  *   padded with -1; int32 count [batch, h_kv] = min(budget, seq_len).
  * - Device-side checks: a page number outside [0, num_pages), a position outside the block
@@ -231,12 +232,15 @@ JSSA_API int jssa_score_topk_bf16(const jssa_bf16* q, const float* basis,
  * over j in the index set of sequence b, i.e. jssa_score_topk run with h_kv = 1, d = 576 and
  * r = 128 on the latent scoring cache (basis rows: the projected 512 latent dimensions, then the
  * 64 rotary dimensions passed through).
- * q: bf16 [batch, h_q, 576] absorbed queries (h_q a multiple of 16). kv_cache: bf16 latent cache,
+ * q: bf16 [batch, h_q, 576] absorbed queries (h_q a multiple of 16; budget <= 98304,
+ * JSSA_ERR_UNSUPPORTED otherwise). kv_cache: bf16 latent cache,
  * row (page p, slot s) at p*kv_page_stride + s*kv_slot_stride elements (576 contiguous, 16-byte
  * aligned). idx/count: int32 [batch, 1, budget] / [batch, 1] (count clamped to [0, budget]).
- * out: bf16 [batch, h_q, 512]. ws: >= jssa_workspace_size(JSSA_FN_MLA_ATTEND, batch, h_q, 1,
- * 576, ...); its split counters must be zero when the call starts (jssa_workspace_init once) and
- * are zero again when it ends. Out-of-range positions and pages are skipped and flagged.
+ * out: bf16 [batch, h_q, 512], 16-byte aligned. ws: >= jssa_workspace_size(JSSA_FN_MLA_ATTEND,
+ * batch, h_q, 1, 576, ...); its split counters must be zero when the call starts
+ * (jssa_workspace_init once) and are zero again when it ends. Out-of-range positions and pages
+ * are skipped and flagged; a bounded wait on the tensor cores that runs out raises
+ * JSSA_DEVERR_TIMEOUT (the output is then invalid).
  */
 JSSA_API int jssa_mla_attend(const jssa_bf16* q, const jssa_bf16* kv_cache, int64_t kv_page_stride,
                              int64_t kv_slot_stride, const int32_t* block_table, int max_pages,

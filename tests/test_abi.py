@@ -87,6 +87,10 @@ def test_argument_checks_reject_before_launch(lib):
     assert st == -2  # 8 query heads over 3 KV heads
     st = lib.jssa_store(8, 1024, 32, 1, 2, 128, 32, 48, 32, 10, 16, None)
     assert st == -4  # misaligned key pointer
+    # queries 4- but not 16-byte aligned (the prep reads query rows with 16-byte loads)
+    st = lib.jssa_score_topk(0x1004, 0x2000, 0x3000, 0x4000, 16, 0x5000, 1, 8, 2, 128, 32, 10, 16,
+                             128, 0x6000, 0x7000, 0x8000, 1 << 30, None)
+    assert st == -4
     st = lib.jssa_indexed_attend(16, 16, 16, 4096, 256, 128, 16, 8, 16, 16, 1, 64, 2, 128, 128,
                                  10, 16, ctypes.c_float(0.1), 16, None, 0, None)
     assert st == -3  # G = 32 query heads per KV head is beyond the m16 tile

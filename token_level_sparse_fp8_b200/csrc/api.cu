@@ -164,6 +164,7 @@ int jssa_workspace_size(int fn, int batch, int h_q, int h_kv, int d, int max_pag
       return JSSA_OK;
     case JSSA_FN_MLA_ATTEND:
       if (budget <= 0 || h_kv != 1 || d != 576 || h_q % 16) return JSSA_ERR_SHAPE;
+      if (jssa::plan_mla(batch, h_q, budget).splits == 0) return JSSA_ERR_UNSUPPORTED;
       *bytes = jssa::plan_mla(batch, h_q, budget).ws_bytes;
       return JSSA_OK;
     case JSSA_FN_DENSE_DECODE: {
@@ -220,7 +221,8 @@ static int store_codes(const jssa_bf16* k, int64_t k_stride_t, const int64_t* sl
   if (bf16 ? !(d == 128 && r == 32) : !supported_dr(d, r)) return JSSA_ERR_UNSUPPORTED;
   if (t == 0) return JSSA_OK;
   if (!k || !slot_mapping || !basis || !score_cache) return JSSA_ERR_NULL;
-  if (!aligned16(k) || (k_stride_t & 7) || !aligned16(score_cache)) return JSSA_ERR_ALIGN;
+  if (!aligned16(k) || (k_stride_t & 7) || !aligned16(score_cache) || !aligned16(basis))
+    return JSSA_ERR_ALIGN;
   if (k_stride_t < (int64_t)h_kv * d) return JSSA_ERR_SHAPE;
   return cuda_status(jssa::launch_store(k, k_stride_t, slot_mapping, t, h_kv, d, r, basis,
                                         static_cast<uint8_t*>(score_cache), num_pages, page_size,
@@ -256,7 +258,8 @@ static int check_score_args(const jssa_bf16* q, const float* basis, const uint8_
   if (batch == 0) return JSSA_OK;
   if (!q || !basis || !score_cache || !block_table || !seq_lens || !idx || !count)
     return JSSA_ERR_NULL;
-  if (!aligned16(score_cache) || !aligned16(basis) || ((uintptr_t)q & 3u)) return JSSA_ERR_ALIGN;
+  // (the prep reads each query row with 16-byte loads)
+  if (!aligned16(score_cache) || !aligned16(basis) || !aligned16(q)) return JSSA_ERR_ALIGN;
   return JSSA_OK;
 }
 
@@ -371,16 +374,17 @@ int jssa_mla_attend(const jssa_bf16* q, const jssa_bf16* kv_cache, int64_t kv_pa
                     int64_t num_pages, int page_size, float softmax_scale, jssa_bf16* out,
                     void* ws, size_t ws_bytes, jssa_stream_t stream) {
   if (batch < 0 || h_q <= 0 || budget <= 0) return JSSA_ERR_SHAPE;
-  if (h_q % 16 || budget > 256 * 1024) return JSSA_ERR_UNSUPPORTED;
+  if (h_q % 16 || budget > 96 * 1024) return JSSA_ERR_UNSUPPORTED;
   int st = check_paging(max_pages, num_pages, page_size);
   if (st) return st;
   if (batch == 0) return JSSA_OK;
   if (!q || !kv_cache || !block_table || !idx || !count || !out) return JSSA_ERR_NULL;
   if (kv_page_stride <= 0 || kv_slot_stride < 576) return JSSA_ERR_SHAPE;
   if (!aligned16(kv_cache) || !aligned16(q) || ((kv_page_stride | kv_slot_stride) & 7) ||
-      ((uintptr_t)out & 3u))
+      !aligned16(out))
     return JSSA_ERR_ALIGN;
   const jssa::MlaPlan plan = jssa::plan_mla(batch, h_q, budget);
+  if (plan.splits == 0) return JSSA_ERR_UNSUPPORTED;
   if (plan.ws_bytes && (!ws || ws_bytes < plan.ws_bytes)) return JSSA_ERR_WORKSPACE;
   if (plan.ws_bytes && !aligned16(ws)) return JSSA_ERR_ALIGN;
   return cuda_status(jssa::launch_mla(q, kv_cache, kv_page_stride, kv_slot_stride, block_table,

@@ -93,9 +93,10 @@ cudaError_t launch_gather(const uint16_t* k_cache, const uint16_t* v_cache, int6
                           uint16_t* k_out, uint16_t* v_out, int32_t* lens_out, cudaStream_t s);
 
 // Multi-head latent attention over selected positions (absorbed form, 576-dim key rows,
-// 512-dim values, 16 query heads per CTA): split-K plan and launch.
+// 512-dim values, 128 query heads x 128 value dimensions per CTA on the 5th-generation tensor
+// cores): split-K plan and launch.
 struct MlaPlan {
-  int splits;
+  int splits;  // 0: the budget is beyond what the split merge holds (unsupported)
   int chunk;
   size_t ws_bytes;
 };

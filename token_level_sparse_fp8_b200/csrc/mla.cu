@@ -9,18 +9,27 @@
 // token, one "KV head") and the index set of score_topk run with h_kv = 1 on the latent scoring
 // cache.
 //
-// Grid (h_q / 16, splits, batch): a CTA owns 16 query heads of one sequence and one contiguous
-// slice of its index set; the head blocks of one slice are neighbours in launch order, so the
-// rows they all read come from L2 after the first. Its 4 warps share every 16-token tile of latent rows (a CTA-wide ring
-// of kStages shared-memory stages filled by 16-byte cp.async, chunk c of a row at
-// (c & ~7) | ((c ^ row) & 7) so that ldmatrix reads are conflict-free). The scores S = Q K^T of
-// the 16 heads x 16 tokens are computed on the tensor cores (mma.sync m16n8k16 bf16, fp32
-// accumulate; the 16 heads are the M rows) with the 576 dimensions split over the 4 warps (9
-// k-blocks each) and the partial sums added through shared memory; every warp then keeps the
-// same online softmax and adds P V into its quarter (128 dims) of the output (P split into bf16
-// high and low parts). Splits
-// of one (sequence, head block) merge through fp32 partials and a ticket, as the GQA attention.
+// On the 5th-generation tensor cores, with every operand that is reused held in tensor memory.
+// Grid (head blocks x 4, splits, batch): a CTA owns 128 query heads of one sequence (the M = 128
+// rows of every MMA; a smaller h_q pads the block with zero queries), one quarter (128 of the
+// 512) of the value dimensions and one contiguous slice of the index set. Tensor memory (512
+// columns x 128 lanes, lane = head):
+//   columns   0-287  Q, the A operand of S = Q K^T (576 bf16 per row, written once)
+//   columns 288-351  S (64 tokens, fp32), then in place P = softmax weights as two bf16 parts
+//                    (high 288-319, low 320-351: P V is two MMAs and the weights keep ~16 bits)
+//   columns 384-511  O, this CTA's 128 value dimensions (fp32 accumulator)
+// Latent rows arrive by 16-byte cp.async, 64 tokens per tile, in a 2-stage ring. A tile is kept
+// as 9 column blocks of 64 dimensions (128 bytes per token, 128-byte swizzle), the layout that
+// serves both as the K-major B operand of S (N = 64 tokens) and as the MN-major B operand of P V
+// (N = 128 value dimensions, K = 64 tokens), so each row is read from L2 once per CTA. One
+// thread issues the MMAs; the 4 warps read S (one head per thread: the softmax needs no
+// shuffles), keep the online softmax with a lazy rescale (O is rescaled through tensor memory
+// only when a row's maximum grows by more than 2^8), and write P back. Every wait on the tensor
+// cores is bounded (a timeout raises JSSA_DEVERR_TIMEOUT and the CTA still releases its tensor
+// memory). Splits of one (sequence, head block, quarter) merge through fp32 partials and a
+// ticket.
 #include "common.cuh"
+#include "tcgen05.cuh"
 
 namespace jssa {
 
@@ -28,19 +37,25 @@ namespace mla_detail {
 
 constexpr int kDK = 576;             // latent + rotary dimensions of a key row
 constexpr int kDV = 512;             // latent dimensions (the value row)
-constexpr int kHeads = 16;           // query heads per CTA (the MMA's M rows)
-constexpr int kWarps = 4;            // each owns kDV / kWarps output dimensions
-constexpr int kThreads = kWarps * 32;
-constexpr int kTile = 16;            // tokens per tile
-constexpr int kStages = 3;
-constexpr int kRowBytes = kDK * 2;   // 1152
-constexpr int kChunks = kRowBytes / 16;  // 72
-constexpr int kTileBytes = kTile * kRowBytes;
-constexpr int kQBytes = kHeads * kRowBytes;
-constexpr int kMaxChunk = 1024;      // positions per CTA
-constexpr int kSmem = kQBytes + kStages * kTileBytes;
-constexpr int kDimsPerWarp = kDV / kWarps;  // 128
-constexpr int kMaxMergeSplits = kStages * kTileBytes / (kHeads * 3 * 4);  // 288
+constexpr int kM = 128;              // query heads per CTA (the MMA's M rows)
+constexpr int kQuarters = 4;         // value-dimension quarters (one per CTA)
+constexpr int kDQ = kDV / kQuarters; // 128 value dimensions per CTA
+constexpr int kThreads = 128;        // thread t <-> head t <-> tensor-memory lane t
+constexpr int kTT = 64;              // tokens per tile
+constexpr int kStages = 2;
+constexpr int kBlocks = kDK / 64;                // 9 column blocks of 64 dimensions
+constexpr int kBlockBytes = kTT * 128;           // 8 KB
+constexpr int kTileBytes = kBlocks * kBlockBytes;  // 72 KB
+constexpr int kSmem = 1024 + kStages * kTileBytes;  // (+ the 1024-byte alignment of the ring)
+constexpr int kMaxChunk = 1024;                  // positions per CTA
+constexpr uint32_t kCols = 512;
+constexpr uint32_t kQCol = 0, kSCol = 288, kOCol = 384;
+constexpr int kMaxMergeSplits = kStages * kTileBytes / (kM * 3 * 4);  // 96
+constexpr float kRescaleSlack = 8.f;             // log2 units
+constexpr int kPRow = kDQ + 4;                   // partial row: m, l, 2 pad, o[128] (16-byte aligned)
+
+static_assert(kQCol + kDK / 2 <= kSCol && kSCol + kTT <= kOCol && kOCol + kDQ <= kCols, "tmem");
+static_assert(kTT == 64 && kThreads == kM, "one head per thread, 64-bit token masks");
 
 struct Args {
   const uint16_t* q;
@@ -58,32 +73,33 @@ struct Args {
   void* ws;
 };
 
-__device__ __forceinline__ uint32_t swz(int row, int c) {
-  return (uint32_t)(row * kRowBytes + (((c & ~7) | ((c ^ row) & 7)) << 4));
-}
-
-__global__ void __launch_bounds__(kThreads, 2) mla_kernel(Args a, int chunk, int splits) {
-  extern __shared__ __align__(128) uint8_t mla_smem[];
+__global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int splits) {
+  extern __shared__ __align__(1024) uint8_t mla_smem[];
   __shared__ int64_t s_off[kMaxChunk];
-  __shared__ float s_part[kWarps][32][8];  // each warp's partial S, in fragment order
+  __shared__ uint32_t s_valid[kMaxChunk / 32];  // bit j: position j of the slice is usable
+  __shared__ __align__(8) uint64_t s_bar[3];     // S ready, P V done, drain
+  __shared__ uint32_t s_tmem;
   __shared__ int s_last;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int g = lane >> 2, t = lane & 3;
-  const int hb = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
-  const int n_hb = gridDim.x;
+  const int hb = blockIdx.x / kQuarters, dq = blockIdx.x % kQuarters;
+  const int split = blockIdx.y, b = blockIdx.z;
+  const int n_hb = gridDim.x / kQuarters;
   const int max_len = a.max_pages * a.page_size;
-  const uint32_t s_q = smem_u32(mla_smem);
-  const uint32_t ring = s_q + kQBytes;
+  const uint32_t ring = (smem_u32(mla_smem) + 1023u) & ~1023u;
+  const uint32_t bar_s = smem_u32(&s_bar[0]), bar_o = smem_u32(&s_bar[1]);
+  const uint32_t bar_d = smem_u32(&s_bar[2]);
 
-  // the 16 heads' absorbed queries (inputs of the step, complete before it) -> shared memory
-  {
-    const uint16_t* qb = a.q + ((int64_t)b * a.h_q + (int64_t)hb * kHeads) * kDK;
-    for (int i = tid; i < kHeads * kChunks; i += kThreads) {
-      const int row = i / kChunks, c = i % kChunks;
-      cp_async16(s_q + swz(row, c), qb + (int64_t)row * kDK + c * 8, 16);
-    }
-    cp_async_commit();
+  if (tid == 0) {
+    tc::mbar_init(bar_s, 1);
+    tc::mbar_init(bar_o, 1);
+    tc::mbar_init(bar_d, 1);
+    tc::fence_mbar_init();
   }
+  if (warp == 0) {
+    tc::tmem_alloc(smem_u32(&s_tmem), kCols);
+    tc::tmem_relinquish();
+  }
+
   pdl_wait();  // index sets come from the preceding score + top-B kernel
   int n_total = a.count[b];
   n_total = n_total < 0 ? 0 : (n_total > a.budget ? a.budget : n_total);
@@ -106,179 +122,253 @@ __global__ void __launch_bounds__(kThreads, 2) mla_kernel(Args a, int chunk, int
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
       const int j = tid + u * kThreads;
-      if (j >= n_mine) continue;
       int64_t off = -1;
-      if (pos[u] < 0 || pos[u] >= max_len) raise_flag(2u);
-      else if (pg[u] < 0 || (int64_t)pg[u] >= a.num_pages) raise_flag(1u);
-      else off = (int64_t)pg[u] * a.page_stride + (int64_t)(pos[u] % a.page_size) * a.slot_stride;
+      if (j < n_mine) {
+        if (pos[u] < 0 || pos[u] >= max_len) raise_flag(2u);
+        else if (pg[u] < 0 || (int64_t)pg[u] >= a.num_pages) raise_flag(1u);
+        else off = (int64_t)pg[u] * a.page_stride + (int64_t)(pos[u] % a.page_size) * a.slot_stride;
+      }
       s_off[j] = off;
+      const unsigned m = __ballot_sync(0xffffffffu, off >= 0);
+      if (lane == 0) s_valid[j >> 5] = m;
     }
   }
+  tc::fence_before_sync();
   __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = s_tmem;
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+
+  // this thread's query row -> tensor-memory lane tid, columns [0, 288)
+  {
+    const int head = hb * kM + tid;
+    const bool hv = head < a.h_q;
+    const uint4* qrow = reinterpret_cast<const uint4*>(a.q + ((int64_t)b * a.h_q + (hv ? head : 0)) * kDK);
+    // three groups of 32 columns per round: 24 independent 16-byte loads in flight
+#pragma unroll 1
+    for (int r0 = 0; r0 < kDK / 64; r0 += 3) {
+      uint4 x[24];
+#pragma unroll
+      for (int u = 0; u < 24; ++u) x[u] = hv ? __ldg(qrow + r0 * 8 + u) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int g3 = 0; g3 < 3; ++g3) {
+        uint32_t v[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          v[4 * u] = x[8 * g3 + u].x;
+          v[4 * u + 1] = x[8 * g3 + u].y;
+          v[4 * u + 2] = x[8 * g3 + u].z;
+          v[4 * u + 3] = x[8 * g3 + u].w;
+        }
+        tc::tmem_st32(tmem + lane_base + kQCol + 32 * (r0 + g3), v);
+      }
+    }
+    tc::tmem_wait_st();
+  }
   pdl_trigger();
 
-  const int n_tiles = (n_mine + kTile - 1) / kTile;
-  // copies of a tile: 8 threads per row, thread q of a row takes chunks q, q + 8, ..., q + 64 (a
-  // warp instruction covers 128 contiguous bytes of each of its 4 rows); the swizzle only flips
-  // the low 3 bits of the chunk index, so a thread's destinations are 128 bytes apart
-  static_assert(kThreads == kTile * 8 && kChunks % 8 == 0, "copy split");
+  // copies of a tile: 8 threads per row, thread q of a row takes the q-th 16-byte chunk of each
+  // 128-byte column block (a warp instruction covers 128 contiguous bytes of each of its 4 rows)
+  const int n_tiles = (n_mine + kTT - 1) / kTT;
   const int cp_row = tid >> 3, cp_q = tid & 7;
-  const uint32_t cp_dst = (uint32_t)(cp_row * kRowBytes + ((cp_q ^ (cp_row & 7)) << 4));
   auto issue = [&](int tl, int st) {
-    const int j = tl * kTile + cp_row;
-    const int64_t off = j < n_mine ? s_off[j] : -1;
-    const uint16_t* src = a.kv + (off >= 0 ? off : 0) + cp_q * 8;
-    const uint32_t dst = ring + st * kTileBytes + cp_dst;
+    const uint32_t stage = ring + st * kTileBytes;
 #pragma unroll
-    for (int k = 0; k < kChunks / 8; ++k) cp_async16(dst + 128 * k, src + 64 * k, off >= 0 ? 16 : 0);
+    for (int p = 0; p < kTT / 16; ++p) {
+      const int row = p * 16 + cp_row;
+      const int j = tl * kTT + row;
+      const int64_t off = j < n_mine ? s_off[j] : -1;
+      const uint16_t* src = a.kv + (off >= 0 ? off : 0) + cp_q * 8;
+      const uint32_t dst = stage + row * 128 + ((cp_q ^ (row & 7)) << 4);
+#pragma unroll
+      for (int blk = 0; blk < kBlocks; ++blk)
+        cp_async16(dst + blk * kBlockBytes, src + blk * 64, off >= 0 ? 16 : 0);
+    }
   };
 #pragma unroll
   for (int i = 0; i < kStages - 1; ++i) {
     if (i < n_tiles) issue(i, i);
     cp_async_commit();
   }
+  tc::fence_before_sync();
+  __syncthreads();  // Q in tensor memory before the first MMA
+  tc::fence_after_sync();
 
   const float scale_log2 = a.scale * 1.4426950408889634f;
-  float o[kDimsPerWarp / 8][4];
-#pragma unroll
-  for (int n = 0; n < kDimsPerWarp / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};  // rows g, g + 8
-  // ldmatrix lane roles
-  const int mat = lane >> 3, mr = lane & 7;
-  const int qa_row = mr + (mat & 1) * 8, qa_half = mat >> 1;   // Q (A): heads 0-7 / 8-15, k lo / hi
-  const int kb_row = mr + (mat >> 1) * 8, kb_half = mat & 1;   // K (B): tokens 0-7 / 8-15, k lo / hi
-  const int vb_row = mr + (mat & 1) * 8, vb_next = mat >> 1;   // V (B, trans): tokens lo / hi, n-tile
-
+  constexpr uint32_t kIdescS = tc::idesc_bf16(kM, kTT, false);
+  constexpr uint32_t kIdescO = tc::idesc_bf16(kM, kDQ, true);
+  float m_ref = -INFINITY, l_run = 0.f;
+  bool ok = true;
   for (int i = 0; i < n_tiles; ++i) {
+    if (i > 0) {  // P V of the previous tile done: its stage, S / P and O are free
+      const bool w = tc::mbar_wait(bar_o, (i - 1) & 1);
+      if (__syncthreads_or(!w)) {
+        ok = false;
+        break;
+      }
+      tc::fence_after_sync();
+    }
     if (i + kStages - 1 < n_tiles) issue(i + kStages - 1, (i + kStages - 1) % kStages);
     cp_async_commit();
     cp_async_wait<kStages - 1>();
+    tc::fence_proxy_async_smem();
     __syncthreads();
-    const uint32_t st = ring + (i % kStages) * kTileBytes;
-
-    // S (16 heads x 16 tokens) = Q K^T over the 576 dimensions: this warp's 9 k-blocks, then
-    // the four partial sums through shared memory (the same fragment order in every warp)
-    float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-    constexpr int kKB = kDK / 16 / kWarps;  // 9
-#pragma unroll
-    for (int u = 0; u < kKB; ++u) {
-      const int kb = warp * kKB + u;
-      uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
-      ldsm_x4(s_q + swz(qa_row, 2 * kb + qa_half), a0, a1, a2, a3);
-      ldsm_x4(st + swz(kb_row, 2 * kb + kb_half), b0, b1, b2, b3);
-      mma_bf16(s0, a0, a1, a2, a3, b0, b1);
-      mma_bf16(s1, a0, a1, a2, a3, b2, b3);
+    const uint32_t stage = ring + (i % kStages) * kTileBytes;
+    if (tid == 0) {
+      tc::fence_after_sync();
+      // S = Q K^T: 36 steps of 16 dimensions; step kk reads 32 bytes at (kk % 4) * 32 of the
+      // 128-byte rows of column block kk / 4
+#pragma unroll 4
+      for (int kk = 0; kk < kDK / 16; ++kk) {
+        const uint64_t bd = tc::sw128_desc(stage + (kk >> 2) * kBlockBytes + (kk & 3) * 32, 16, 1024);
+        tc::mma_ts(tmem + kSCol, tmem + kQCol + kk * 8, bd, kIdescS, kk > 0);
+      }
+      tc::mma_commit(bar_s);
     }
-    *reinterpret_cast<float4*>(&s_part[warp][lane][0]) = make_float4(s0[0], s0[1], s0[2], s0[3]);
-    *reinterpret_cast<float4*>(&s_part[warp][lane][4]) = make_float4(s1[0], s1[1], s1[2], s1[3]);
+    {
+      const bool w = tc::mbar_wait(bar_s, i & 1);
+      if (__syncthreads_or(!w)) {
+        ok = false;
+        break;
+      }
+    }
+    tc::fence_after_sync();
+    uint32_t sr[2][32];
+    tc::tmem_ld32(tmem + lane_base + kSCol, sr[0]);
+    tc::tmem_ld32(tmem + lane_base + kSCol + 32, sr[1]);
+    tc::tmem_wait_ld();
+    const uint32_t v0 = s_valid[2 * i], v1 = s_valid[2 * i + 1];
+    float x[kTT];
+    float mt = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < kTT; ++c) {
+      const bool v = ((c < 32 ? v0 >> c : v1 >> (c - 32)) & 1u) != 0;
+      x[c] = v ? __uint_as_float(sr[c >> 5][c & 31]) * scale_log2 : -INFINITY;
+      mt = fmaxf(mt, x[c]);
+    }
+    // lazy rescale: the weights are taken relative to m_ref, which moves only when a row's
+    // maximum exceeds it by more than the slack (weights stay <= 2^8)
+    const bool first = m_ref == -INFINITY;
+    const bool grow = mt > m_ref + kRescaleSlack;
+    const bool resc = grow && !first;  // O holds earlier weights relative to the old m_ref
+    const float m_new = grow ? mt : m_ref;
+    const float corr = resc ? fast_exp2(m_ref - m_new) : 1.f;
+    if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll 1
+      for (int c = 0; c < kDQ / 32; ++c) {
+        uint32_t o[32];
+        tc::tmem_ld32(tmem + lane_base + kOCol + 32 * c, o);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
+        tc::tmem_st32(tmem + lane_base + kOCol + 32 * c, o);
+      }
+    }
+    l_run *= corr;
+    m_ref = m_new;
+    uint32_t ph[32], pl[32];
+    float lsum = 0.f;
+#pragma unroll
+    for (int e = 0; e < kTT / 2; ++e) {
+      const float p0 = x[2 * e] == -INFINITY ? 0.f : fast_exp2(x[2 * e] - m_ref);
+      const float p1 = x[2 * e + 1] == -INFINITY ? 0.f : fast_exp2(x[2 * e + 1] - m_ref);
+      lsum += p0 + p1;
+      const uint32_t h = pack_bf16x2(p0, p1);
+      ph[e] = h;
+      pl[e] = pack_bf16x2(p0 - bf16_lo(h), p1 - bf16_hi(h));
+    }
+    l_run += lsum;
+    tc::tmem_st32(tmem + lane_base + kSCol, ph);
+    tc::tmem_st32(tmem + lane_base + kSCol + 32, pl);
+    tc::tmem_wait_st();
+    tc::fence_before_sync();
     __syncthreads();
+    if (tid == 0) {
+      tc::fence_after_sync();
+      // O += P V: K = 16 tokens per step; B = rows 16 kk.. of the quarter's two column blocks
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      s0[e] = s_part[0][lane][e] + s_part[1][lane][e] + s_part[2][lane][e] + s_part[3][lane][e];
-      s1[e] = s_part[0][lane][4 + e] + s_part[1][lane][4 + e] + s_part[2][lane][4 + e] +
-              s_part[3][lane][4 + e];
-    }
-    // rows g (s[0], s[1]) and g + 8 (s[2], s[3]); columns: tokens 2t, 2t + 1 (+ 8 in s1)
-    const int j0 = i * kTile;
-    const bool v00 = j0 + 2 * t < n_mine && s_off[j0 + 2 * t] >= 0;
-    const bool v01 = j0 + 2 * t + 1 < n_mine && s_off[j0 + 2 * t + 1] >= 0;
-    const bool v10 = j0 + 8 + 2 * t < n_mine && s_off[j0 + 8 + 2 * t] >= 0;
-    const bool v11 = j0 + 9 + 2 * t < n_mine && s_off[j0 + 9 + 2 * t] >= 0;
-    float x[8];
-    x[0] = v00 ? s0[0] * scale_log2 : -INFINITY;  // row g
-    x[1] = v01 ? s0[1] * scale_log2 : -INFINITY;
-    x[2] = v10 ? s1[0] * scale_log2 : -INFINITY;
-    x[3] = v11 ? s1[1] * scale_log2 : -INFINITY;
-    x[4] = v00 ? s0[2] * scale_log2 : -INFINITY;  // row g + 8
-    x[5] = v01 ? s0[3] * scale_log2 : -INFINITY;
-    x[6] = v10 ? s1[2] * scale_log2 : -INFINITY;
-    x[7] = v11 ? s1[3] * scale_log2 : -INFINITY;
-    float mx0 = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-    float mx1 = fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7]));
+      for (int part = 0; part < 2; ++part)
 #pragma unroll
-    for (int sh = 1; sh < 4; sh <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, sh));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, sh));
+        for (int kk = 0; kk < kTT / 16; ++kk) {
+          const uint64_t bd = tc::sw128_desc(stage + 2 * dq * kBlockBytes + kk * 16 * 128,
+                                             kBlockBytes, 1024);
+          tc::mma_ts(tmem + kOCol, tmem + kSCol + 32 * part + kk * 8, bd, kIdescO,
+                     i > 0 || part > 0 || kk > 0);
+        }
+      tc::mma_commit(bar_o);
     }
-    const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
-    const float mu0 = mn0 == -INFINITY ? 0.f : mn0, mu1 = mn1 == -INFINITY ? 0.f : mn1;
-    const float corr0 = fast_exp2(m_run[0] - mu0), corr1 = fast_exp2(m_run[1] - mu1);
-    float p[8];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      p[e] = fast_exp2(x[e] - mu0);
-      p[4 + e] = fast_exp2(x[4 + e] - mu1);
-    }
-    l_run[0] = l_run[0] * corr0 + (p[0] + p[1] + p[2] + p[3]);
-    l_run[1] = l_run[1] * corr1 + (p[4] + p[5] + p[6] + p[7]);
-    m_run[0] = mn0;
-    m_run[1] = mn1;
-#pragma unroll
-    for (int n = 0; n < kDimsPerWarp / 8; ++n) {
-      o[n][0] *= corr0;
-      o[n][1] *= corr0;
-      o[n][2] *= corr1;
-      o[n][3] *= corr1;
-    }
-    // P as the A operand (16 heads x 16 tokens), high and low bf16 parts
-    const uint32_t h0 = pack_bf16x2(p[0], p[1]), h1 = pack_bf16x2(p[4], p[5]);
-    const uint32_t h2 = pack_bf16x2(p[2], p[3]), h3 = pack_bf16x2(p[6], p[7]);
-    const uint32_t l0 = pack_bf16x2(p[0] - bf16_lo(h0), p[1] - bf16_hi(h0));
-    const uint32_t l1 = pack_bf16x2(p[4] - bf16_lo(h1), p[5] - bf16_hi(h1));
-    const uint32_t l2 = pack_bf16x2(p[2] - bf16_lo(h2), p[3] - bf16_hi(h2));
-    const uint32_t l3 = pack_bf16x2(p[6] - bf16_lo(h3), p[7] - bf16_hi(h3));
-    // O (16 heads x this warp's 128 dims) += P V
-#pragma unroll
-    for (int n = 0; n < kDimsPerWarp / 8; n += 2) {
-      const int c = (warp * kDimsPerWarp + n * 8) / 8 + vb_next;
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4_t(st + swz(vb_row, c), b0, b1, b2, b3);
-      mma_bf16(o[n], h0, h1, h2, h3, b0, b1);
-      mma_bf16(o[n], l0, l1, l2, l3, b0, b1);
-      mma_bf16(o[n + 1], h0, h1, h2, h3, b2, b3);
-      mma_bf16(o[n + 1], l0, l1, l2, l3, b2, b3);
-    }
-    __syncthreads();  // the stage is refilled by the next iteration's copies
+  }
+  if (ok && n_tiles > 0) {
+    const bool w = tc::mbar_wait(bar_o, (n_tiles - 1) & 1);
+    if (__syncthreads_or(!w)) ok = false;
+    tc::fence_after_sync();
   }
   cp_async_wait<0>();
-#pragma unroll
-  for (int sh = 1; sh < 4; sh <<= 1) {
-    l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], sh);
-    l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], sh);
-  }
+  // every MMA issued has completed before the tensor memory is read for the last time and freed
+  if (tid == 0) tc::mma_commit(bar_d);
+  if (__syncthreads_or(!tc::mbar_wait(bar_d, 0))) ok = false;
+  tc::fence_after_sync();
+  if (!ok && tid == 0) raise_flag(JSSA_DEVERR_TIMEOUT);
 
-  const int head0 = hb * kHeads;
-  const int64_t out_row0 = (int64_t)b * a.h_q + head0;
-  if (splits == 1) {
-#pragma unroll
-    for (int n = 0; n < kDimsPerWarp / 8; ++n) {
-      const int d0 = warp * kDimsPerWarp + n * 8 + 2 * t;
-      const float i0 = l_run[0] > 0.f ? 1.f / l_run[0] : 0.f, i1 = l_run[1] > 0.f ? 1.f / l_run[1] : 0.f;
-      *reinterpret_cast<uint32_t*>(a.out + (out_row0 + g) * kDV + d0) = pack_bf16x2(o[n][0] * i0, o[n][1] * i0);
-      *reinterpret_cast<uint32_t*>(a.out + (out_row0 + g + 8) * kDV + d0) = pack_bf16x2(o[n][2] * i1, o[n][3] * i1);
-    }
-    return;
-  }
-  // partials [batch][head block][split][16 heads][2 + 512] (m in log2 units, l, o) and tickets
-  const int64_t n_blocks = (int64_t)a.batch * n_hb;
+  const int head = hb * kM + tid;
+  const bool hv = head < a.h_q && ok;
+  const bool have_o = n_tiles > 0 && ok;
+  uint16_t* orow = a.out + ((int64_t)b * a.h_q + head) * kDV + dq * kDQ;
+  const int64_t blk = ((int64_t)b * n_hb + hb) * kQuarters + dq;
+  const int64_t n_blocks = (int64_t)a.batch * n_hb * kQuarters;
   int* tickets = reinterpret_cast<int*>(a.ws);
-  float* part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(a.ws) + ((n_blocks * 4 + 255) / 256) * 256);
-  const int64_t blk = (int64_t)b * n_hb + hb;
-  float* pb = part + (blk * splits + split) * kHeads * (kDV + 2);
-  if (warp == 0 && t == 0) {
-    __stcg(pb + g * (kDV + 2), m_run[0]);
-    __stcg(pb + g * (kDV + 2) + 1, l_run[0]);
-    __stcg(pb + (g + 8) * (kDV + 2), m_run[1]);
-    __stcg(pb + (g + 8) * (kDV + 2) + 1, l_run[1]);
-  }
+  float* part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(a.ws) +
+                                         ((n_blocks * 4 + 255) / 256) * 256);
+  float* prow = part + ((blk * splits + split) * kM + tid) * kPRow;
+  if (splits == 1) {
+    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll 1
+    for (int c = 0; c < kDQ / 32; ++c) {
+      uint32_t o[32];
+      if (have_o) {
+        tc::tmem_ld32(tmem + lane_base + kOCol + 32 * c, o);
+        tc::tmem_wait_ld();
+      } else {
 #pragma unroll
-  for (int n = 0; n < kDimsPerWarp / 8; ++n) {
-    const int d0 = warp * kDimsPerWarp + n * 8 + 2 * t;
-    __stcg(pb + g * (kDV + 2) + 2 + d0, o[n][0]);
-    __stcg(pb + g * (kDV + 2) + 3 + d0, o[n][1]);
-    __stcg(pb + (g + 8) * (kDV + 2) + 2 + d0, o[n][2]);
-    __stcg(pb + (g + 8) * (kDV + 2) + 3 + d0, o[n][3]);
+        for (int e = 0; e < 32; ++e) o[e] = 0u;
+      }
+      uint32_t w[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+      if (hv)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          reinterpret_cast<uint4*>(orow + 32 * c)[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+    }
+  } else {
+    // partial [m (log2 units), l, -, -, o[128]] of this split (16-byte stores), then a ticket
+    float4* p4 = reinterpret_cast<float4*>(prow);
+    __stcg(p4, make_float4(m_ref, l_run, 0.f, 0.f));
+#pragma unroll 1
+    for (int c = 0; c < kDQ / 32; ++c) {
+      uint32_t o[32];
+      if (have_o) {
+        tc::tmem_ld32(tmem + lane_base + kOCol + 32 * c, o);
+        tc::tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = 0u;
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        __stcg(p4 + 1 + 8 * c + e, make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                                               __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3])));
+    }
   }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kCols);
+  }
+  if (splits == 1) return;
+
   __threadfence();
   __syncthreads();
   if (tid == 0) s_last = atomicAdd(&tickets[blk], 1) == splits - 1;
@@ -287,35 +377,63 @@ __global__ void __launch_bounds__(kThreads, 2) mla_kernel(Args a, int chunk, int
   __threadfence();
   // merge: weights w = 2^(m - M) / L per (split, head) in shared memory (the ring is free), then
   // one weighted sum of independent loads per output element
-  const float* p0 = part + blk * splits * kHeads * (kDV + 2);
-  const int64_t step = (int64_t)kHeads * (kDV + 2);
-  float* s_pm = reinterpret_cast<float*>(mla_smem + kQBytes);
-  float* s_pl = s_pm + splits * kHeads;
-  float* s_w = s_pl + splits * kHeads;
-  for (int i = tid; i < splits * kHeads; i += kThreads) {
-    const int sp = i / kHeads, row = i % kHeads;
-    s_pm[i] = __ldcg(p0 + sp * step + (int64_t)row * (kDV + 2));
-    s_pl[i] = __ldcg(p0 + sp * step + (int64_t)row * (kDV + 2) + 1);
+  const float* p0 = part + blk * splits * kM * kPRow;
+  const int64_t step = (int64_t)kM * kPRow;
+  float* s_pm = reinterpret_cast<float*>(mla_smem + (ring - smem_u32(mla_smem)));
+  float* s_pl = s_pm + splits * kM;
+  float* s_w = s_pl + splits * kM;
+  for (int i = tid; i < splits * kM; i += kThreads) {
+    const int sp = i / kM, row = i % kM;
+    const float2 ml = __ldcg(reinterpret_cast<const float2*>(p0 + sp * step + (int64_t)row * kPRow));
+    s_pm[i] = ml.x;
+    s_pl[i] = ml.y;
   }
   __syncthreads();
-  if (tid < kHeads) {
+  {
     float mm = -INFINITY;
-    for (int sp = 0; sp < splits; ++sp) mm = fmaxf(mm, s_pm[sp * kHeads + tid]);
+    for (int sp = 0; sp < splits; ++sp) mm = fmaxf(mm, s_pm[sp * kM + tid]);
     float l = 0.f;
     if (mm != -INFINITY)
-      for (int sp = 0; sp < splits; ++sp) l += fast_exp2(s_pm[sp * kHeads + tid] - mm) * s_pl[sp * kHeads + tid];
+      for (int sp = 0; sp < splits; ++sp) l += fast_exp2(s_pm[sp * kM + tid] - mm) * s_pl[sp * kM + tid];
     const float inv = l > 0.f ? 1.f / l : 0.f;
     for (int sp = 0; sp < splits; ++sp)
-      s_w[sp * kHeads + tid] = mm != -INFINITY ? fast_exp2(s_pm[sp * kHeads + tid] - mm) * inv : 0.f;
+      s_w[sp * kM + tid] = mm != -INFINITY ? fast_exp2(s_pm[sp * kM + tid] - mm) * inv : 0.f;
   }
   __syncthreads();
-  for (int e = tid; e < kHeads * kDV; e += kThreads) {
-    const int row = e / kDV, dim = e % kDV;
-    const float* pp = p0 + (int64_t)row * (kDV + 2) + 2 + dim;
-    float acc = 0.f;
-#pragma unroll 8
-    for (int sp = 0; sp < splits; ++sp) acc += s_w[sp * kHeads + row] * __ldcg(pp + sp * step);
-    a.out[(out_row0 + row) * kDV + dim] = f_to_bf16(acc);
+  // 4 consecutive dimensions per task, consecutive threads on consecutive 16-byte pieces of a
+  // row; 8 tasks unrolled so that their loads are in flight together
+  constexpr int kTasks = kM * kDQ / 4;
+#pragma unroll 1
+  for (int e0 = 0; e0 < kTasks; e0 += 8 * kThreads) {
+    float4 acc[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+    for (int sp = 0; sp < splits; ++sp) {
+      float4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int e = e0 + u * kThreads + tid, row = e / (kDQ / 4), d4 = e % (kDQ / 4);
+        v[u] = __ldcg(reinterpret_cast<const float4*>(p0 + sp * step + (int64_t)row * kPRow + 4) + d4);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int e = e0 + u * kThreads + tid, row = e / (kDQ / 4);
+        const float w = s_w[sp * kM + row];
+        acc[u].x += w * v[u].x;
+        acc[u].y += w * v[u].y;
+        acc[u].z += w * v[u].z;
+        acc[u].w += w * v[u].w;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = e0 + u * kThreads + tid, row = e / (kDQ / 4), d4 = e % (kDQ / 4);
+      const int h = hb * kM + row;
+      if (h < a.h_q)
+        *reinterpret_cast<uint2*>(a.out + ((int64_t)b * a.h_q + h) * kDV + dq * kDQ + 4 * d4) =
+            make_uint2(pack_bf16x2(acc[u].x, acc[u].y), pack_bf16x2(acc[u].z, acc[u].w));
+    }
   }
   if (tid == 0) tickets[blk] = 0;
 }
@@ -325,22 +443,22 @@ __global__ void __launch_bounds__(kThreads, 2) mla_kernel(Args a, int chunk, int
 MlaPlan plan_mla(int batch, int h_q, int budget) {
   using namespace mla_detail;
   MlaPlan p;
-  const int blocks = batch * (h_q / kHeads);
-  const int unit = 4 * kTile;  // at least 4 tiles per CTA
-  int splits = (2 * num_sms()) / (blocks > 0 ? blocks : 1);
-  const int max_splits = (budget + unit - 1) / unit;
+  const int blocks = batch * ((h_q + kM - 1) / kM) * kQuarters;
+  int splits = num_sms() / (blocks > 0 ? blocks : 1);  // one CTA per SM
+  const int max_splits = (budget + kTT - 1) / kTT;
   if (splits > max_splits) splits = max_splits;
   if (splits < 1) splits = 1;
   int chunk = (budget + splits - 1) / splits;
-  chunk = (chunk + unit - 1) / unit * unit;
+  chunk = (chunk + kTT - 1) / kTT * kTT;
   const int min_chunk = (budget + kMaxMergeSplits - 1) / kMaxMergeSplits;  // the merge buffer
-  if (chunk < min_chunk) chunk = (min_chunk + unit - 1) / unit * unit;
+  if (chunk < min_chunk) chunk = (min_chunk + kTT - 1) / kTT * kTT;
   if (chunk > kMaxChunk) chunk = kMaxChunk;
   splits = (budget + chunk - 1) / chunk;
+  if (splits > kMaxMergeSplits) splits = 0;  // budget above kMaxMergeSplits * kMaxChunk: refused
   p.splits = splits;
   p.chunk = chunk;
   p.ws_bytes = splits > 1 ? (((size_t)blocks * 4 + 255) / 256) * 256 +
-                                (size_t)blocks * splits * kHeads * (kDV + 2) * sizeof(float)
+                                (size_t)blocks * splits * kM * kPRow * sizeof(float)
                           : 0;
   return p;
 }
@@ -352,13 +470,13 @@ cudaError_t launch_mla(const uint16_t* q, const uint16_t* kv, int64_t page_strid
                        const MlaPlan& plan, bool pdl, cudaStream_t s) {
   using namespace mla_detail;
   if (batch == 0) return cudaSuccess;
-  static_assert(kSmem >= kStages * kTileBytes, "merge buffer");
+  static_assert(kSmem - 1024 >= kMaxMergeSplits * kM * 12, "merge buffer");
   cudaError_t e = configure_kernel((const void*)mla_kernel, kSmem, false);
   if (e != cudaSuccess) return e;
   Args a = {q, kv, page_stride, slot_stride, block_table, max_pages, idx, count, batch, h_q,
             budget, num_pages, page_size, scale, out, ws};
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(h_q / kHeads, plan.splits, batch);
+  cfg.gridDim = dim3(((h_q + kM - 1) / kM) * kQuarters, plan.splits, batch);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = s;

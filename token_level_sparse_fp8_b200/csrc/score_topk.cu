@@ -1006,13 +1006,28 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
   // ---- independent loads first: M_h into shared memory (async); L, the group's query rows and
   // the new token's K and V rows into registers ----
   constexpr bool kMSmem = prep_m_in_smem<D, C>();
+  constexpr int kQGroups = q_groups<D>();
+  {
+    // a group of many query heads (the 128 heads of a latent layer) is summed over many rounds
+    // of loads, and a basis too large for shared memory is read row by row: both are prefetched
+    // into L2 in 4 KB pieces first, so that those rounds wait on L2 and not on HBM
+    constexpr int kPiece = 4096;
+    const int q_bytes = G > kQGroups ? G * D * 2 : 0;
+    const int m_bytes = kMSmem ? 0 : R * D * 4;
+    const int q_pieces = (q_bytes + kPiece - 1) / kPiece, m_pieces = (m_bytes + kPiece - 1) / kPiece;
+    const uint8_t* q_src = reinterpret_cast<const uint8_t*>(a.q + ((int64_t)b * a.h_q + (int64_t)h * G) * D);
+    const uint8_t* m_src = reinterpret_cast<const uint8_t*>(m_h);
+    for (int i = tid; i < q_pieces + m_pieces; i += kThreads) {
+      if (i < q_pieces) prefetch_l2_bulk(q_src + i * kPiece, min(kPiece, q_bytes - i * kPiece));
+      else prefetch_l2_bulk(m_src + (i - q_pieces) * kPiece, min(kPiece, m_bytes - (i - q_pieces) * kPiece));
+    }
+  }
   if (kMSmem)
     for (int i = tid; i < R * D / 4; i += kThreads) cp_async16(smem_u32(sm.m + 4 * i), m_h + 4 * i, 16);
   cp_async_commit();
   const int L = clamp_len(a.seq_lens[b], a.max_pages << a.page_shift);
   // the G query rows of this KV head: D / 8 threads x 8 dims per row, kQGroups rows at a time
   static_assert(D % 8 == 0 && D / 8 <= kThreads, "query row split");
-  constexpr int kQGroups = q_groups<D>();
   const uint16_t* qh = a.q + ((int64_t)b * a.h_q + (int64_t)h * G) * D;
   const int rg = tid / (D / 8), d8 = (tid % (D / 8)) * 8;
   uint4 qv = make_uint4(0u, 0u, 0u, 0u);

@@ -4,10 +4,11 @@
 // BF16 = true stores bf16(M_h k) instead (two bytes per dimension: the scoring-cache ablation).
 //
 // One CTA per (KV head, slice of basis rows, range of tokens). The slice of the head's basis rows
-// (all r rows up to r = 64; 32 rows at r = 128, where the whole basis would not fit) is staged in
-// shared memory once; each warp takes one token at a time, lane j computes output j (and j+32,
-// ...) of the slice as a float64 dot product over the d dimensions and rounds it once. At decode the same kernel
-// also writes the new token's K and V rows into the paged cache.
+// (all r rows up to r = 64; 32 rows at r = 128, where the whole basis would not fit) is staged
+// in shared memory once, widened to float64; each warp takes one token at a time, lane j
+// computes output j (and j+32, ...) of the slice as a float64 dot product over the d dimensions
+// and rounds it once. At decode the same kernel also writes the new token's K and V rows into
+// the paged cache.
 #include "common.cuh"
 
 namespace jssa {
@@ -30,20 +31,32 @@ __global__ void __launch_bounds__(kStoreThreads)
                  int64_t head_stride, const int32_t* __restrict__ block_table, int max_pages,
                  const int32_t* __restrict__ seq_lens) {
   constexpr int RS = store_rows_per_cta(R);
-  extern __shared__ float store_smem[];
-  float* s_m = store_smem;                        // [RS][D+1]
-  float* s_k = store_smem + RS * (D + 1);           // [warps][D]
+  // both operands of the float64 products are widened once, when staged: the slice of basis
+  // rows per CTA and each warp's key row per token
+  extern __shared__ double store_smem[];
+  double* s_m = store_smem;                        // [RS][D+1]
+  double* s_k = store_smem + RS * (D + 1);         // [warps][D]
   const int h = blockIdx.x / (R / RS), r0 = (blockIdx.x % (R / RS)) * RS;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const float* m_h = basis + ((int64_t)h * R + r0) * D;
-  for (int i = threadIdx.x; i < RS * D; i += kStoreThreads) s_m[(i / D) * (D + 1) + (i % D)] = m_h[i];
+  // the slice of basis rows, 16-byte loads (several in flight per thread) into the padded layout
+  static_assert(D % 4 == 0, "basis rows in 16-byte pieces");
+  const float4* m_h = reinterpret_cast<const float4*>(basis + ((int64_t)h * R + r0) * D);
+#pragma unroll 6
+  for (int i = threadIdx.x; i < RS * D / 4; i += kStoreThreads) {
+    const float4 v = m_h[i];
+    double* dst = s_m + (4 * i / D) * (D + 1) + (4 * i) % D;
+    dst[0] = v.x;
+    dst[1] = v.y;
+    dst[2] = v.z;
+    dst[3] = v.w;
+  }
   __syncthreads();
 
   const int t0 = blockIdx.y * tokens_per_block;
   const int t1 = min(t_count, t0 + tokens_per_block);
-  float* kw = s_k + warp * D;
+  double* kw = s_k + warp * D;
   for (int t = t0 + warp; t < t1; t += kStoreWarps) {
     int64_t page, off;
     if (DECODE) {
@@ -121,10 +134,18 @@ __global__ void __launch_bounds__(kStoreThreads)
 #pragma unroll
     for (int j0 = 0; j0 < RS; j0 += 32) {
       const int j = j0 + lane;
-      const float* mrow = s_m + j * (D + 1);
-      double acc = 0.0;
-#pragma unroll 8
-      for (int i = 0; i < D; ++i) acc = fma((double)mrow[i], (double)kw[i], acc);
+      const double* mrow = s_m + j * (D + 1);
+      // float64 dot product in four interleaved partial sums (short dependency chains), one
+      // rounding at the end
+      double acc0 = 0.0, acc1 = 0.0, acc2 = 0.0, acc3 = 0.0;
+#pragma unroll 4
+      for (int i = 0; i < D; i += 4) {
+        acc0 = fma(mrow[i], kw[i], acc0);
+        acc1 = fma(mrow[i + 1], kw[i + 1], acc1);
+        acc2 = fma(mrow[i + 2], kw[i + 2], acc2);
+        acc3 = fma(mrow[i + 3], kw[i + 3], acc3);
+      }
+      const double acc = (acc0 + acc1) + (acc2 + acc3);
       if (BF16) reinterpret_cast<uint16_t*>(dst)[j] = f64_to_bf16(acc);
       else dst[j] = f64_to_e4m3(acc);
     }
@@ -162,7 +183,7 @@ cudaError_t dispatch_store(int d, int r, int t, int h_kv, int tpb, cudaStream_t 
   if (t <= 0) return cudaSuccess;
   const int rs = store_rows_per_cta(r);
   dim3 grid(h_kv * (r / rs), (t + tpb - 1) / tpb);
-  const size_t smem = (size_t)(rs * (d + 1) + kStoreWarps * d) * sizeof(float);
+  const size_t smem = (size_t)(rs * (d + 1) + kStoreWarps * d) * sizeof(double);
 #define JSSA_STORE_CASE(DD, RR)                                                                  \
   if (d == DD && r == RR)                                                                        \
     return launch_store_t<DD, RR, DECODE, BF16>(grid, smem, s, k, k_stride_t, slot_mapping, t,   \
