@@ -40,7 +40,7 @@ constexpr int kDV = 512;             // latent dimensions (the value row)
 constexpr int kM = 128;              // query heads per CTA (the MMA's M rows)
 constexpr int kQuarters = 4;         // value-dimension quarters (one per CTA)
 constexpr int kDQ = kDV / kQuarters; // 128 value dimensions per CTA
-constexpr int kThreads = 128;        // thread t <-> head t <-> tensor-memory lane t
+constexpr int kThreads = 256;        // thread t <-> head t % 128 (tensor-memory lane), half t / 128
 constexpr int kTT = 64;              // tokens per tile
 constexpr int kStages = 2;
 constexpr int kBlocks = kDK / 64;                // 9 column blocks of 64 dimensions
@@ -55,7 +55,7 @@ constexpr float kRescaleSlack = 8.f;             // log2 units
 constexpr int kPRow = kDQ + 4;                   // partial row: m, l, 2 pad, o[128] (16-byte aligned)
 
 static_assert(kQCol + kDK / 2 <= kSCol && kSCol + kTT <= kOCol && kOCol + kDQ <= kCols, "tmem");
-static_assert(kTT == 64 && kThreads == kM, "one head per thread, 64-bit token masks");
+static_assert(kTT == 64 && kThreads == 2 * kM, "two threads per head, 32 tokens each");
 
 struct Args {
   const uint16_t* q;
@@ -78,9 +78,13 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int
   __shared__ int64_t s_off[kMaxChunk];
   __shared__ uint32_t s_valid[kMaxChunk / 32];  // bit j: position j of the slice is usable
   __shared__ __align__(8) uint64_t s_bar[3];     // S ready, P V done, drain
+  __shared__ float s_half[2][kM];  // per-row exchange between the two halves (max, then l)
   __shared__ uint32_t s_tmem;
   __shared__ int s_last;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // warps w and w + 4 share tensor-memory lanes 32 (w % 4) .. +31 (heads); half 0 takes tokens
+  // 0-31 of a tile, the low half of the value dimensions and columns 0-159 of Q, half 1 the rest
+  const int row = tid & (kM - 1), half = tid >> 7;
   const int hb = blockIdx.x / kQuarters, dq = blockIdx.x % kQuarters;
   const int split = blockIdx.y, b = blockIdx.z;
   const int n_hb = gridDim.x / kQuarters;
@@ -137,35 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = s_tmem;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-
-  // this thread's query row -> tensor-memory lane tid, columns [0, 288)
-  {
-    const int head = hb * kM + tid;
-    const bool hv = head < a.h_q;
-    const uint4* qrow = reinterpret_cast<const uint4*>(a.q + ((int64_t)b * a.h_q + (hv ? head : 0)) * kDK);
-    // three groups of 32 columns per round: 24 independent 16-byte loads in flight
-#pragma unroll 1
-    for (int r0 = 0; r0 < kDK / 64; r0 += 3) {
-      uint4 x[24];
-#pragma unroll
-      for (int u = 0; u < 24; ++u) x[u] = hv ? __ldg(qrow + r0 * 8 + u) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-      for (int g3 = 0; g3 < 3; ++g3) {
-        uint32_t v[32];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          v[4 * u] = x[8 * g3 + u].x;
-          v[4 * u + 1] = x[8 * g3 + u].y;
-          v[4 * u + 2] = x[8 * g3 + u].z;
-          v[4 * u + 3] = x[8 * g3 + u].w;
-        }
-        tc::tmem_st32(tmem + lane_base + kQCol + 32 * (r0 + g3), v);
-      }
-    }
-    tc::tmem_wait_st();
-  }
-  pdl_trigger();
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
 
   // copies of a tile: 8 threads per row, thread q of a row takes the q-th 16-byte chunk of each
   // 128-byte column block (a warp instruction covers 128 contiguous bytes of each of its 4 rows)
@@ -174,8 +150,8 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int
   auto issue = [&](int tl, int st) {
     const uint32_t stage = ring + st * kTileBytes;
 #pragma unroll
-    for (int p = 0; p < kTT / 16; ++p) {
-      const int row = p * 16 + cp_row;
+    for (int p = 0; p < kTT / 32; ++p) {
+      const int row = p * 32 + cp_row;
       const int j = tl * kTT + row;
       const int64_t off = j < n_mine ? s_off[j] : -1;
       const uint16_t* src = a.kv + (off >= 0 ? off : 0) + cp_q * 8;
@@ -190,6 +166,38 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int
     if (i < n_tiles) issue(i, i);
     cp_async_commit();
   }
+
+  // the query row of head `row` -> its tensor-memory lane, columns [0, 288): half 0 writes the
+  // column groups 0-4, half 1 the groups 5-8 (24 independent 16-byte loads per round)
+  {
+    const int head = hb * kM + row;
+    const bool hv = head < a.h_q;
+    const uint4* qrow = reinterpret_cast<const uint4*>(a.q + ((int64_t)b * a.h_q + (hv ? head : 0)) * kDK);
+    const int g_begin = half ? 5 : 0, g_end = half ? kDK / 64 : 5;
+#pragma unroll 1
+    for (int g0 = g_begin; g0 < g_end; g0 += 3) {
+      const int n = min(3, g_end - g0);  // (uniform over a warp)
+      uint4 x[24];
+#pragma unroll
+      for (int u = 0; u < 24; ++u)
+        x[u] = (hv && u < 8 * n) ? __ldg(qrow + g0 * 8 + u) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int g3 = 0; g3 < 3; ++g3) {
+        if (g3 >= n) break;
+        uint32_t v[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          v[4 * u] = x[8 * g3 + u].x;
+          v[4 * u + 1] = x[8 * g3 + u].y;
+          v[4 * u + 2] = x[8 * g3 + u].z;
+          v[4 * u + 3] = x[8 * g3 + u].w;
+        }
+        tc::tmem_st32(tmem + lane_base + kQCol + 32 * (g0 + g3), v);
+      }
+    }
+    tc::tmem_wait_st();
+  }
+  pdl_trigger();
   tc::fence_before_sync();
   __syncthreads();  // Q in tensor memory before the first MMA
   tc::fence_after_sync();
@@ -233,19 +241,23 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int
       }
     }
     tc::fence_after_sync();
-    uint32_t sr[2][32];
-    tc::tmem_ld32(tmem + lane_base + kSCol, sr[0]);
-    tc::tmem_ld32(tmem + lane_base + kSCol + 32, sr[1]);
+    uint32_t sr[32];
+    tc::tmem_ld32(tmem + lane_base + kSCol + 32 * half, sr);
     tc::tmem_wait_ld();
-    const uint32_t v0 = s_valid[2 * i], v1 = s_valid[2 * i + 1];
-    float x[kTT];
+    const uint32_t vm = s_valid[2 * i + half];
+    float x[32];
     float mt = -INFINITY;
 #pragma unroll
-    for (int c = 0; c < kTT; ++c) {
-      const bool v = ((c < 32 ? v0 >> c : v1 >> (c - 32)) & 1u) != 0;
-      x[c] = v ? __uint_as_float(sr[c >> 5][c & 31]) * scale_log2 : -INFINITY;
+    for (int c = 0; c < 32; ++c) {
+      x[c] = ((vm >> c) & 1u) ? __uint_as_float(sr[c]) * scale_log2 : -INFINITY;
       mt = fmaxf(mt, x[c]);
     }
+    // the row maximum over both halves; every S read is complete before P overwrites it
+    s_half[half][row] = mt;
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    mt = fmaxf(s_half[0][row], s_half[1][row]);
     // lazy rescale: the weights are taken relative to m_ref, which moves only when a row's
     // maximum exceeds it by more than the slack (weights stay <= 2^8)
     const bool first = m_ref == -INFINITY;
@@ -253,23 +265,24 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int
     const bool resc = grow && !first;  // O holds earlier weights relative to the old m_ref
     const float m_new = grow ? mt : m_ref;
     const float corr = resc ? fast_exp2(m_ref - m_new) : 1.f;
-    if (__any_sync(0xffffffffu, resc)) {
+    if (__any_sync(0xffffffffu, resc)) {  // this half's 64 columns of O
 #pragma unroll 1
-      for (int c = 0; c < kDQ / 32; ++c) {
+      for (int c = 0; c < kDQ / 64; ++c) {
         uint32_t o[32];
-        tc::tmem_ld32(tmem + lane_base + kOCol + 32 * c, o);
+        const uint32_t col = kOCol + 64 * half + 32 * c;
+        tc::tmem_ld32(tmem + lane_base + col, o);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
-        tc::tmem_st32(tmem + lane_base + kOCol + 32 * c, o);
+        tc::tmem_st32(tmem + lane_base + col, o);
       }
     }
-    l_run *= corr;
+    l_run *= corr;  // (this half's share of the row sum)
     m_ref = m_new;
-    uint32_t ph[32], pl[32];
+    uint32_t ph[16], pl[16];
     float lsum = 0.f;
 #pragma unroll
-    for (int e = 0; e < kTT / 2; ++e) {
+    for (int e = 0; e < 16; ++e) {
       const float p0 = x[2 * e] == -INFINITY ? 0.f : fast_exp2(x[2 * e] - m_ref);
       const float p1 = x[2 * e + 1] == -INFINITY ? 0.f : fast_exp2(x[2 * e + 1] - m_ref);
       lsum += p0 + p1;
@@ -278,8 +291,8 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int
       pl[e] = pack_bf16x2(p0 - bf16_lo(h), p1 - bf16_hi(h));
     }
     l_run += lsum;
-    tc::tmem_st32(tmem + lane_base + kSCol, ph);
-    tc::tmem_st32(tmem + lane_base + kSCol + 32, pl);
+    tc::tmem_st16(tmem + lane_base + kSCol + 16 * half, ph);
+    tc::tmem_st16(tmem + lane_base + kSCol + 32 + 16 * half, pl);
     tc::tmem_wait_st();
     tc::fence_before_sync();
     __syncthreads();
@@ -310,7 +323,11 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int
   tc::fence_after_sync();
   if (!ok && tid == 0) raise_flag(JSSA_DEVERR_TIMEOUT);
 
-  const int head = hb * kM + tid;
+  // row sum over both halves
+  s_half[half][row] = l_run;
+  __syncthreads();
+  const float l_tot = s_half[0][row] + s_half[1][row];
+  const int head = hb * kM + row;
   const bool hv = head < a.h_q && ok;
   const bool have_o = n_tiles > 0 && ok;
   uint16_t* orow = a.out + ((int64_t)b * a.h_q + head) * kDV + dq * kDQ;
@@ -319,11 +336,11 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int
   int* tickets = reinterpret_cast<int*>(a.ws);
   float* part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(a.ws) +
                                          ((n_blocks * 4 + 255) / 256) * 256);
-  float* prow = part + ((blk * splits + split) * kM + tid) * kPRow;
+  float* prow = part + ((blk * splits + split) * kM + row) * kPRow;
   if (splits == 1) {
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+    const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
 #pragma unroll 1
-    for (int c = 0; c < kDQ / 32; ++c) {
+    for (int c = 2 * half; c < 2 * half + 2; ++c) {  // this half's 64 value dimensions
       uint32_t o[32];
       if (have_o) {
         tc::tmem_ld32(tmem + lane_base + kOCol + 32 * c, o);
@@ -344,9 +361,9 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int
   } else {
     // partial [m (log2 units), l, -, -, o[128]] of this split (16-byte stores), then a ticket
     float4* p4 = reinterpret_cast<float4*>(prow);
-    __stcg(p4, make_float4(m_ref, l_run, 0.f, 0.f));
+    if (half == 0) __stcg(p4, make_float4(m_ref, l_tot, 0.f, 0.f));
 #pragma unroll 1
-    for (int c = 0; c < kDQ / 32; ++c) {
+    for (int c = 2 * half; c < 2 * half + 2; ++c) {
       uint32_t o[32];
       if (have_o) {
         tc::tmem_ld32(tmem + lane_base + kOCol + 32 * c, o);
@@ -389,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int
     s_pl[i] = ml.y;
   }
   __syncthreads();
-  {
+  if (tid < kM) {
     float mm = -INFINITY;
     for (int sp = 0; sp < splits; ++sp) mm = fmaxf(mm, s_pm[sp * kM + tid]);
     float l = 0.f;

@@ -1098,14 +1098,26 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
       part[2 * e] = bf16_lo(w[e]);
       part[2 * e + 1] = bf16_hi(w[e]);
     }
-#pragma unroll 4
-    for (int r = rg + kQGroups; rg < kQGroups && r < G; r += kQGroups) {  // G > kQGroups
-      const uint4 v = *reinterpret_cast<const uint4*>(qh + (int64_t)r * D + d8);
-      const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+    // G > kQGroups (the many heads of a latent layer): batches of kQB rows, their loads issued
+    // together, then added in row order
+    constexpr int kQB = 16;
+#pragma unroll 1
+    for (int r0 = rg + kQGroups; rg < kQGroups && r0 < G; r0 += kQB * kQGroups) {
+      uint4 v[kQB];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        part[2 * e] += bf16_lo(x[e]);
-        part[2 * e + 1] += bf16_hi(x[e]);
+      for (int u = 0; u < kQB; ++u) {
+        const int r = r0 + u * kQGroups;
+        v[u] = r < G ? *reinterpret_cast<const uint4*>(qh + (int64_t)r * D + d8) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kQB; ++u) {
+        if (r0 + u * kQGroups >= G) break;
+        const uint32_t x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          part[2 * e] += bf16_lo(x[e]);
+          part[2 * e + 1] += bf16_hi(x[e]);
+        }
       }
     }
 #pragma unroll
@@ -1158,7 +1170,7 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
       acc_k[jj] = 0.0;
     }
     const float* mbase = m_h + (int64_t)(warp * kRW) * D;
-#pragma unroll 2
+#pragma unroll 3
     for (int e = lane; e < D; e += 32) {
       const float qv = s_qbar[e];
       const double kv = store ? (double)s_k[e] : 0.0;
@@ -1842,9 +1854,14 @@ cudaError_t launch_t(const ScorePlan& plan, int pairs, const PrepArgs& pa, const
   cudaError_t e;
   const size_t prep_smem = sizeof(PrepSmem<D, C>);
   if (store) {
-    e = configure_kernel((const void*)prep_kernel<D, C, true>, (int)prep_smem, false);
-    if (e == cudaSuccess)
-      e = launch_k(prep_kernel<D, C, true>, dim3(pairs), kThreads, prep_smem, pdl, s, pa);
+    // (the fused decode store exists for the head dimensions that have decode attention)
+    if constexpr (D == 128 || D == 256) {
+      e = configure_kernel((const void*)prep_kernel<D, C, true>, (int)prep_smem, false);
+      if (e == cudaSuccess)
+        e = launch_k(prep_kernel<D, C, true>, dim3(pairs), kThreads, prep_smem, pdl, s, pa);
+    } else {
+      e = cudaErrorInvalidValue;
+    }
   } else {
     e = configure_kernel((const void*)prep_kernel<D, C, false>, (int)prep_smem, false);
     if (e == cudaSuccess)
