@@ -232,7 +232,7 @@ JSSA_API int jssa_score_topk_bf16(const jssa_bf16* q, const float* basis,
  * over j in the index set of sequence b, i.e. jssa_score_topk run with h_kv = 1, d = 576 and
  * r = 128 on the latent scoring cache (basis rows: the projected 512 latent dimensions, then the
  * 64 rotary dimensions passed through).
- * q: bf16 [batch, h_q, 576] absorbed queries (h_q a multiple of 16; budget <= 98304,
+ * q: bf16 [batch, h_q, 576] absorbed queries (h_q a multiple of 16; budget <= 262144,
  * JSSA_ERR_UNSUPPORTED otherwise). kv_cache: bf16 latent cache,
  * row (page p, slot s) at p*kv_page_stride + s*kv_slot_stride elements (576 contiguous, 16-byte
  * aligned). idx/count: int32 [batch, 1, budget] / [batch, 1] (count clamped to [0, budget]).

@@ -374,7 +374,7 @@ int jssa_mla_attend(const jssa_bf16* q, const jssa_bf16* kv_cache, int64_t kv_pa
                     int64_t num_pages, int page_size, float softmax_scale, jssa_bf16* out,
                     void* ws, size_t ws_bytes, jssa_stream_t stream) {
   if (batch < 0 || h_q <= 0 || budget <= 0) return JSSA_ERR_SHAPE;
-  if (h_q % 16 || budget > 96 * 1024) return JSSA_ERR_UNSUPPORTED;
+  if (h_q % 16 || budget > 256 * 1024) return JSSA_ERR_UNSUPPORTED;
   int st = check_paging(max_pages, num_pages, page_size);
   if (st) return st;
   if (batch == 0) return JSSA_OK;

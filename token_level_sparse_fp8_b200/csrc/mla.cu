@@ -50,7 +50,7 @@ constexpr int kSmem = 1024 + kStages * kTileBytes;  // (+ the 1024-byte alignmen
 constexpr int kMaxChunk = 1024;                  // positions per CTA
 constexpr uint32_t kCols = 512;
 constexpr uint32_t kQCol = 0, kSCol = 288, kOCol = 384;
-constexpr int kMaxMergeSplits = kStages * kTileBytes / (kM * 3 * 4);  // 96
+constexpr int kMaxMergeSplits = kStages * kTileBytes / (kM * 4);  // 288 (merge weights)
 constexpr float kRescaleSlack = 8.f;             // log2 units
 constexpr int kPRow = kDQ + 4;                   // partial row: m, l, 2 pad, o[128] (16-byte aligned)
 
@@ -396,25 +396,37 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int
   // one weighted sum of independent loads per output element
   const float* p0 = part + blk * splits * kM * kPRow;
   const int64_t step = (int64_t)kM * kPRow;
-  float* s_pm = reinterpret_cast<float*>(mla_smem + (ring - smem_u32(mla_smem)));
-  float* s_pl = s_pm + splits * kM;
-  float* s_w = s_pl + splits * kM;
-  for (int i = tid; i < splits * kM; i += kThreads) {
-    const int sp = i / kM, row = i % kM;
-    const float2 ml = __ldcg(reinterpret_cast<const float2*>(p0 + sp * step + (int64_t)row * kPRow));
-    s_pm[i] = ml.x;
-    s_pl[i] = ml.y;
-  }
-  __syncthreads();
-  if (tid < kM) {
-    float mm = -INFINITY;
-    for (int sp = 0; sp < splits; ++sp) mm = fmaxf(mm, s_pm[sp * kM + tid]);
-    float l = 0.f;
-    if (mm != -INFINITY)
-      for (int sp = 0; sp < splits; ++sp) l += fast_exp2(s_pm[sp * kM + tid] - mm) * s_pl[sp * kM + tid];
+  float* s_w = reinterpret_cast<float*>(mla_smem + (ring - smem_u32(mla_smem)));
+  if (tid < kM) {  // row tid: the splits' (m, l) in batches of 8 independent loads, twice
+    const float2* ml = reinterpret_cast<const float2*>(p0 + (int64_t)tid * kPRow);
+    const int64_t st2 = step / 2;
+    float mm = -INFINITY, l = 0.f;  // running maximum and the sum relative to it
+    for (int sp0 = 0; sp0 < splits; sp0 += 8) {
+      float2 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        v[u] = sp0 + u < splits ? __ldcg(ml + (sp0 + u) * st2) : make_float2(-INFINITY, 0.f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (v[u].x == -INFINITY) continue;
+        if (v[u].x > mm) {
+          l = l * fast_exp2(mm - v[u].x) + v[u].y;
+          mm = v[u].x;
+        } else {
+          l += fast_exp2(v[u].x - mm) * v[u].y;
+        }
+      }
+    }
     const float inv = l > 0.f ? 1.f / l : 0.f;
-    for (int sp = 0; sp < splits; ++sp)
-      s_w[sp * kM + tid] = mm != -INFINITY ? fast_exp2(s_pm[sp * kM + tid] - mm) * inv : 0.f;
+    for (int sp0 = 0; sp0 < splits; sp0 += 8) {
+      float m8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) m8[u] = sp0 + u < splits ? __ldcg(ml + (sp0 + u) * st2).x : -INFINITY;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (sp0 + u < splits)
+          s_w[(sp0 + u) * kM + tid] = m8[u] != -INFINITY ? fast_exp2(m8[u] - mm) * inv : 0.f;
+    }
   }
   __syncthreads();
   // 4 consecutive dimensions per task, consecutive threads on consecutive 16-byte pieces of a
@@ -471,7 +483,7 @@ MlaPlan plan_mla(int batch, int h_q, int budget) {
   if (chunk < min_chunk) chunk = (min_chunk + kTT - 1) / kTT * kTT;
   if (chunk > kMaxChunk) chunk = kMaxChunk;
   splits = (budget + chunk - 1) / chunk;
-  if (splits > kMaxMergeSplits) splits = 0;  // budget above kMaxMergeSplits * kMaxChunk: refused
+  if (splits > kMaxMergeSplits) splits = 0;  // budget above kMaxMergeSplits * kMaxChunk
   p.splits = splits;
   p.chunk = chunk;
   p.ws_bytes = splits > 1 ? (((size_t)blocks * 4 + 255) / 256) * 256 +
@@ -487,7 +499,7 @@ cudaError_t launch_mla(const uint16_t* q, const uint16_t* kv, int64_t page_strid
                        const MlaPlan& plan, bool pdl, cudaStream_t s) {
   using namespace mla_detail;
   if (batch == 0) return cudaSuccess;
-  static_assert(kSmem - 1024 >= kMaxMergeSplits * kM * 12, "merge buffer");
+  static_assert(kSmem - 1024 >= kMaxMergeSplits * kM * 4, "merge buffer");
   cudaError_t e = configure_kernel((const void*)mla_kernel, kSmem, false);
   if (e != cudaSuccess) return e;
   Args a = {q, kv, page_stride, slot_stride, block_table, max_pages, idx, count, batch, h_q,

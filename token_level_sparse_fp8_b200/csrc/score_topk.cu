@@ -1886,9 +1886,14 @@ ScorePlan plan_score(int pairs, int max_seq_len, int page_size) {
   using namespace score_detail;
   ScorePlan p;
   // positions per scan CTA: a power of two in [2048, 8192] and a multiple of the page size,
-  // smaller while the grid would not cover every SM several times over
+  // smaller while the grid would not cover every SM several times over, as long as a pair's
+  // candidate regions stay within what the register-resident select holds (with few pairs and
+  // long contexts the select, one CTA per pair, would otherwise cost more than the scan saves)
   int chunk = 8192;
-  while (chunk > 2048 && (long long)pairs * ((max_seq_len + chunk - 1) / chunk) < 6LL * num_sms())
+  while (chunk > 2048 &&
+         (long long)pairs * ((max_seq_len + chunk - 1) / chunk) < 6LL * num_sms() &&
+         (long long)((max_seq_len + chunk / 2 - 1) / (chunk / 2)) * kRegionsPerChunk <=
+             kSelWarps * kSelRegsPerWarp)
     chunk >>= 1;
   while (chunk % page_size) chunk <<= 1;
   while ((long long)((max_seq_len + chunk - 1) / chunk) * kRegionsPerChunk > kMaxRegions) chunk <<= 1;

@@ -82,6 +82,7 @@ __global__ void __launch_bounds__(kStoreThreads)
     if (D != 128 && D != 256) {  // any even D: 32-bit words, lane-strided
       static_assert(D % 2 == 0, "head dim");
       const uint32_t* k32 = reinterpret_cast<const uint32_t*>(krow);
+#pragma unroll
       for (int w = lane; w < D / 2; w += 32) {
         const uint32_t v = k32[w];
         kw[2 * w] = bf16_lo(v);
@@ -90,6 +91,7 @@ __global__ void __launch_bounds__(kStoreThreads)
       if (DECODE) {
         const int64_t base = page * page_stride + off * slot_stride + (int64_t)h * head_stride;
         const uint32_t* v32 = reinterpret_cast<const uint32_t*>(v_new + (int64_t)t * k_stride_t + (int64_t)h * D);
+#pragma unroll
         for (int w = lane; w < D / 2; w += 32) {
           reinterpret_cast<uint32_t*>(k_cache + base)[w] = k32[w];
           reinterpret_cast<uint32_t*>(v_cache + base)[w] = v32[w];
@@ -210,7 +212,9 @@ cudaError_t dispatch_store(int d, int r, int t, int h_kv, int tpb, cudaStream_t 
 cudaError_t launch_store(const uint16_t* k, int64_t k_stride_t, const int64_t* slot_mapping,
                          int t, int h_kv, int d, int r, const float* basis, uint8_t* score_cache,
                          int64_t num_pages, int page_size, cudaStream_t s, bool bf16_codes) {
-  const int tpb = t >= 4096 ? 256 : store_detail::kStoreWarps;
+  // tokens per CTA: many for bulk stores; for a few tokens (a decode step's) two per CTA, so
+  // that more CTAs share the per-token products over the staged basis slices
+  const int tpb = t >= 4096 ? 256 : (t >= 256 ? store_detail::kStoreWarps : 2);
   if (bf16_codes)
     return store_detail::dispatch_store<false, true>(d, r, t, h_kv, tpb, s, k, k_stride_t,
                                slot_mapping, basis, score_cache, num_pages, page_size, nullptr,
