@@ -1,7 +1,8 @@
 """Parity of the multi-head latent attention path with the CPU oracle, through the C ABI:
 the latent scoring store (576-dim rows, basis [M_lat 0; 0 I] of 128 rows), score + top-B with one
 latent head (d 576, r 128, 64-token pages; one context past the sampling point, one ragged) and
-the absorbed latent attention over the selected rows (32 query heads = two 16-head blocks).
+the absorbed latent attention over the selected rows (32 query heads padded into one 128-head
+tensor-core tile; 128 and 144 heads).
 Criteria are in ``parity.py``.
 """
 
@@ -90,6 +91,25 @@ def test_mla_attend(case, budget):
     out = J.mla_attend(case.q.cuda(), kv, case.bt.cuda(), torch.from_numpy(ref_idx).cuda(),
                        torch.from_numpy(ref_count).cuda(), scale)
     ref = O.indexed_attend_step(f64(case.q), case.np_kv, case.np_kv[..., :512], case.np_bt, ref_idx,
+                                ref_count, scale)
+    check_output(f64(out), ref)
+
+
+@pytest.mark.parametrize("h_q", [128, 144])
+def test_mla_attend_head_counts(case, h_q):
+    # 128 heads fill one M = 128 tensor-core tile; 144 heads take two head blocks, the second
+    # padded with zero queries (16 real heads); both split the index set several ways
+    J = jssa()
+    f = layer_factors(1500, 0, 1, D)
+    q = sample_decode_queries(f, len(case.lens), h_q, 1501)
+    budget = 2048
+    ref_idx, ref_count, _ = O.select_step(f64(q), case.m_big.astype(np.float64), case.codes,
+                                          case.np_bt, case.lens, budget)
+    scale = 1.0 / math.sqrt(D)
+    kv = case.kv.cuda().view(case.kv.shape[0], PS, D)
+    out = J.mla_attend(q.cuda(), kv, case.bt.cuda(), torch.from_numpy(ref_idx).cuda(),
+                       torch.from_numpy(ref_count).cuda(), scale)
+    ref = O.indexed_attend_step(f64(q), case.np_kv, case.np_kv[..., :512], case.np_bt, ref_idx,
                                 ref_count, scale)
     check_output(f64(out), ref)
 

@@ -22,12 +22,12 @@
 // as 9 column blocks of 64 dimensions (128 bytes per token, 128-byte swizzle), the layout that
 // serves both as the K-major B operand of S (N = 64 tokens) and as the MN-major B operand of P V
 // (N = 128 value dimensions, K = 64 tokens), so each row is read from L2 once per CTA. One
-// thread issues the MMAs; the 4 warps read S (one head per thread: the softmax needs no
-// shuffles), keep the online softmax with a lazy rescale (O is rescaled through tensor memory
-// only when a row's maximum grows by more than 2^8), and write P back. Every wait on the tensor
-// cores is bounded (a timeout raises JSSA_DEVERR_TIMEOUT and the CTA still releases its tensor
-// memory). Splits of one (sequence, head block, quarter) merge through fp32 partials and a
-// ticket.
+// thread issues the MMAs; 8 warps, two per 32 tensor-memory lanes (heads), each taking half of a
+// tile's tokens, read S, keep the online softmax with a lazy rescale (O is rescaled through
+// tensor memory only when a row's maximum grows by more than 2^8; the two halves exchange the
+// row maximum through shared memory) and write P back. Every wait on the tensor cores is bounded
+// (a timeout raises JSSA_DEVERR_TIMEOUT and the CTA still releases its tensor memory). Splits of
+// one (sequence, head block, quarter) merge through fp32 partials and a ticket.
 #include "common.cuh"
 #include "tcgen05.cuh"
 
