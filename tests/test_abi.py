@@ -73,6 +73,25 @@ def test_workspace_sizes_are_host_only(lib):
         api.workspace_size(_lib.FN_DECODE, 1, 30, 8, 128, 64, 16, 64)  # h_q not a multiple of h_kv
 
 
+def test_mla_workspace_and_budget_limit(lib):
+    from token_level_sparse_fp8_b200 import api, _lib
+    # one sequence, 128 heads: a single split needs no partials; many splits need
+    # (tickets +) 128 rows x 132 floats per (head block, value quarter, split)
+    assert api.workspace_size(_lib.FN_MLA_ATTEND, 64, 128, 1, 576, 2048, 64, 1024) == 0
+    n = api.workspace_size(_lib.FN_MLA_ATTEND, 1, 128, 1, 576, 2048, 64, 2048)
+    assert n >= 4 * 2 * 128 * 132 * 4
+    big = api.workspace_size(_lib.FN_MLA_ATTEND, 1, 128, 1, 576, 8192, 64, 256 * 1024)
+    assert big > n
+    with pytest.raises(_lib.JSSAError):
+        api.workspace_size(_lib.FN_MLA_ATTEND, 1, 128, 1, 576, 8192, 64, 256 * 1024 + 1)
+    with pytest.raises(_lib.JSSAError):
+        api.workspace_size(_lib.FN_MLA_ATTEND, 1, 100, 1, 576, 2048, 64, 2048)  # h_q % 16
+    # the entry refuses the same budget before touching any pointer
+    st = lib.jssa_mla_attend(None, None, 64 * 576, 576, None, 16, None, None, 1, 128,
+                             256 * 1024 + 1, 10, 64, ctypes.c_float(0.1), None, None, 0, None)
+    assert st == -3
+
+
 def test_argument_checks_reject_before_launch(lib):
     from token_level_sparse_fp8_b200 import _lib
     # NULL inputs, unsupported shapes and bad alignment are refused on the host

@@ -55,6 +55,7 @@ using jssa::AttendArgs;
 
 constexpr int kVersion = 100;  // 0.1.0
 constexpr int64_t kMaxContext = jssa::kScoreMaxContext;
+constexpr int kMlaMaxBudget = 256 * 1024;  // selected positions per sequence, latent attention
 
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? JSSA_OK : (int)e; }
 inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
@@ -164,7 +165,8 @@ int jssa_workspace_size(int fn, int batch, int h_q, int h_kv, int d, int max_pag
       return JSSA_OK;
     case JSSA_FN_MLA_ATTEND:
       if (budget <= 0 || h_kv != 1 || d != 576 || h_q % 16) return JSSA_ERR_SHAPE;
-      if (jssa::plan_mla(batch, h_q, budget).splits == 0) return JSSA_ERR_UNSUPPORTED;
+      if (budget > kMlaMaxBudget || jssa::plan_mla(batch, h_q, budget).splits == 0)
+        return JSSA_ERR_UNSUPPORTED;
       *bytes = jssa::plan_mla(batch, h_q, budget).ws_bytes;
       return JSSA_OK;
     case JSSA_FN_DENSE_DECODE: {
@@ -374,7 +376,7 @@ int jssa_mla_attend(const jssa_bf16* q, const jssa_bf16* kv_cache, int64_t kv_pa
                     int64_t num_pages, int page_size, float softmax_scale, jssa_bf16* out,
                     void* ws, size_t ws_bytes, jssa_stream_t stream) {
   if (batch < 0 || h_q <= 0 || budget <= 0) return JSSA_ERR_SHAPE;
-  if (h_q % 16 || budget > 256 * 1024) return JSSA_ERR_UNSUPPORTED;
+  if (h_q % 16 || budget > kMlaMaxBudget) return JSSA_ERR_UNSUPPORTED;
   int st = check_paging(max_pages, num_pages, page_size);
   if (st) return st;
   if (batch == 0) return JSSA_OK;
