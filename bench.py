@@ -289,6 +289,17 @@ def peaks():
         return 6650.0, "fallback"
 
 
+def bf16_peak():
+    """Dense bf16 tensor throughput (TFLOP/s) for a kernel timed alone: the measured burst
+    figure, else the pool's earlier measurement."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            return float(json.load(fh)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
 # ------------------------------------------------------------------------------------------------
 # CPU oracle baseline
 # ------------------------------------------------------------------------------------------------
@@ -988,6 +999,16 @@ def run_mla(args):
         "mla_attend": {"ms": t_att * 1e3, "tflops_algorithmic": flops_att / t_att / 1e12,
                        "hbm_gbs": batch * min(B, L) * 1152 / t_att / 1e9},
         "score_topk": {"ms": t_sc * 1e3, "hbm_gbs": batch * (L * 128 + 4 * (-(-L // ps))) / t_sc / 1e9},
+        # the two calls of the step, each against its own bound: score + top-B streams the
+        # scoring cache (HBM), the latent attention is a bf16 contraction on tcgen05
+        "roofline": {"bound": "hbm", "kernel": "score_topk",
+                     "achieved": batch * (L * 128 + 4 * (-(-L // ps))) / t_sc / 1e9, "peak": peak,
+                     "unit": "GB/s", "frac": batch * (L * 128 + 4 * (-(-L // ps))) / t_sc / 1e9 / peak,
+                     "traffic": None, "peak_kind": peak_kind},
+        "roofline_attend": {"bound": "tensor", "kernel": "mla_attend",
+                            "achieved": flops_att / t_att / 1e12, "peak": bf16_peak()[0],
+                            "unit": "TFLOP/s", "frac": flops_att / t_att / 1e12 / bf16_peak()[0],
+                            "traffic": None, "peak_kind": bf16_peak()[1]},
         "clocks": clocks,
         "gpu_launches": 5 * n_steps,  # store, prep, scan, select, latent attention
         "timing": "CUDA events around replays of a CUDA graph holding 8 consecutive steps",
