@@ -90,6 +90,11 @@ def test_mla_workspace_and_budget_limit(lib):
     st = lib.jssa_mla_attend(None, None, 64 * 576, 576, None, 16, None, None, 1, 128,
                              256 * 1024 + 1, 10, 64, ctypes.c_float(0.1), None, None, 0, None)
     assert st == -3
+    # an output 8- but not 16-byte aligned (the kernel writes 16-byte pieces of each row)
+    st = lib.jssa_mla_attend(0x10000, 0x20000, 64 * 576, 576, 0x30000, 16, 0x40000, 0x50000, 1,
+                             128, 2048, 10, 64, ctypes.c_float(0.1), 0x60008, 0x70000, 1 << 30,
+                             None)
+    assert st == -4
 
 
 def test_argument_checks_reject_before_launch(lib):
