@@ -146,6 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int
   // copies of a tile: 8 threads per row, thread q of a row takes the q-th 16-byte chunk of each
   // 128-byte column block (a warp instruction covers 128 contiguous bytes of each of its 4 rows)
   const int n_tiles = (n_mine + kTT - 1) / kTT;
+  static_assert(kThreads / 8 == 32 && kTT % 32 == 0, "32 rows per copy pass");
   const int cp_row = tid >> 3, cp_q = tid & 7;
   auto issue = [&](int tl, int st) {
     const uint32_t stage = ring + st * kTileBytes;
