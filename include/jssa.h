@@ -302,8 +302,9 @@ JSSA_API int jssa_decode(const jssa_bf16* q, const jssa_bf16* k_new, const jssa_
  * library holds that array until the process exits. Sizes whose scratch would exceed it return
  * JSSA_ERR_SCRATCH_LIMIT without launching (jssa_workspace_size(JSSA_FN_INDEXED_ATTEND, ...)
  * gives the requirement). The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current) and caches it; make that first call before
- * any stream capture. The call itself allocates nothing (it clears the ticket counters with
+ * (cudaGetSymbolAddress, with that device current) and caches it with the id of the device's
+ * CUDA context; the first call after a cudaDeviceReset (a new context) looks it up again. Make
+ * those first calls before any stream capture. The call itself allocates nothing (it clears the ticket counters with
  * cudaMemsetAsync on `stream`, then launches). All calls on a device share the array and it
  * keeps the last call's contents: calls that overlap on the GPU (different streams or threads
  * of the same process) race and must be serialised by the caller.

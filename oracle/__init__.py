@@ -7,7 +7,9 @@ nothing of theirs; the two sides share only the seeded input generator in ``synt
 Precision: float64 throughout. Every function cites the page section or equation it follows.
 
 Parity pins (tests marked ``not gpu``): E4M3 encoder exhaustively against torch's CPU cast and
-the format's closed forms; ``M M^T = I_r``; the Ky Fan closed form of the marginal objective at
+the format's closed forms; the second moments and the calibration Grams against the pair sum of
+squared score errors that eqs. (2)-(3) define (with planted per-head, centred and mis-indexed
+moments caught); ``M M^T = I_r``; the Ky Fan closed form of the marginal objective at
 the optimum; brute-force projector search for tiny ``d``; the bound of eq. (4) on random
 projectors; LAPACK against an independent Jacobi solver; selection against brute-force sorting
 with ties; ``r = d`` without FP8 reproducing the exact group-mean logits ranking; ``r = d`` with

@@ -9,8 +9,9 @@
 // array of fixed size instead of a caller-provided workspace.
 //
 // The array lives in every GPU that loads the library until the process exits. In host code its
-// name only stands for the symbol; the device address is looked up once per device with
-// cudaGetSymbolAddress (on the first call made with that device current) and cached. Calls share
+// name only stands for the symbol; the device address is looked up with cudaGetSymbolAddress
+// (on the first call made with that device current, and again after the device's context was
+// reset) and cached. Calls share
 // the array: it keeps the previous call's contents, the ticket counters are cleared on the
 // stream before every launch, and calls that overlap on the GPU (other streams, other threads)
 // race on it.
@@ -27,22 +28,68 @@ namespace noalloc_detail {
 static __device__ __align__(256) unsigned char g_attend_scratch[JSSA_NOALLOC_SCRATCH_BYTES];
 
 std::mutex g_mu;
-void* g_scratch_addr[64] = {nullptr};
 
-// Device address of g_attend_scratch on the current device (looked up once per device).
+// The cached address of g_attend_scratch per device, with the unique id of the CUDA context it
+// was looked up in: cudaDeviceReset (or any teardown of the device's primary context) makes a
+// new context, whose module copy of the array may sit elsewhere, so a changed id repeats the
+// lookup.
+struct ScratchSlot {
+  void* addr;
+  unsigned long long ctx_id;
+};
+ScratchSlot g_slot[64] = {};
+
+// Driver entry points for the current context and its process-unique id, fetched once through
+// the runtime (no link against the driver library is needed).
+typedef int (*CtxGetCurrentFn)(void** ctx);
+typedef int (*CtxGetIdFn)(void* ctx, unsigned long long* id);
+CtxGetCurrentFn g_ctx_current = nullptr;
+CtxGetIdFn g_ctx_id = nullptr;
+std::once_flag g_entry_once;
+
+// Unique id of the calling thread's current context, or 0 when there is none yet or the driver
+// does not provide the query.
+unsigned long long current_context_id() {
+  std::call_once(g_entry_once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_current = reinterpret_cast<CtxGetCurrentFn>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_id = reinterpret_cast<CtxGetIdFn>(f);
+  });
+  if (!g_ctx_current || !g_ctx_id) return 0ull;
+  void* ctx = nullptr;
+  unsigned long long id = 0ull;
+  if (g_ctx_current(&ctx) != 0 || ctx == nullptr) return 0ull;
+  if (g_ctx_id(ctx, &id) != 0) return 0ull;
+  return id;
+}
+
+// Device address of g_attend_scratch on the current device. The set-up (cudaGetSymbolAddress
+// with the device current) runs on the first call for a device and again whenever the device's
+// context changed since; other calls return the cached address. Without a context id from the
+// driver the lookup runs on every call.
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_attend_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
+  const unsigned long long id = current_context_id();
+  if (id != 0ull && g_slot[dev].addr != nullptr && g_slot[dev].ctx_id == id) {
+    *out = g_slot[dev].addr;
+    return cudaSuccess;
   }
-  *out = g_scratch_addr[dev];
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_attend_scratch);
+  if (e != cudaSuccess) return e;
+  g_slot[dev].addr = p;
+  g_slot[dev].ctx_id = current_context_id();  // the lookup made the context current if needed
+  *out = p;
   return cudaSuccess;
 }
 

@@ -3,28 +3,33 @@
 // programmatic dependent launch:
 //
 // prep   one CTA per (sequence, KV head). p = M_h qbar (qbar = mean of the G query heads of KV
-//        head h), fp32, written as a sum of 8 FP8 "digit" vectors with power-of-two column
-//        scales, p = sum_c 2^e_c D_c with D_c in E4M3 (digit c rounds what the earlier digits
-//        left), which represents p to ~2^-32 of its largest component. Then a candidate
-//        threshold: the scores of a stratified random sample of 2048 positions give a key that
-//        about twice the budget (plus a margin of several standard deviations) of all tokens
-//        reach. The threshold only decides how many keys travel to the select kernel -- the
-//        selection itself is exact (see select). At decode the same kernel first stores the new
-//        token: its K and V rows and its scoring code e4m3(M_h k) (float64 sum, one rounding).
-// scan   CTAs over (chunk of positions, sequence x KV head), no cluster and no shared key array:
-//        a pure stream of the FP8 scoring rows (page-table indexed, 8-byte non-allocating loads,
-//        register double buffering). The codes are consumed as they are by the tensor cores: one
-//        mma.sync m16n8k32 E4M3 x E4M3 -> fp32 per 16 tokens and 32 code bytes multiplies the 16
-//        rows by the 8 digit columns, and s = sum_c 2^e_c C[:, c]. (Widening the codes on the
-//        CUDA cores costs ~3 instructions per byte and leaves this HBM-bound loop issue-bound.)
-//        Every warp walks a contiguous run of tiles and appends the keys at or above the
-//        threshold, with their positions, to its own workspace region in position order.
+//        head h) in fp32, written as a sum of two f16 "digit" vectors with power-of-two weights,
+//        p ~ 2^-e0 D0 + 2^-e1 D1 (D1 rounds what D0 left; about 22 significant bits of every
+//        component relative to the largest one). BF16 codes use four bf16 digits instead. Then a
+//        candidate threshold: a stratified sample of 2048 positions (512 strata, a run of 4
+//        consecutive positions in each) is scored exactly as the scan scores, and the k-th
+//        largest sampled key, k = ceil(E + 4 sqrt(E) + 8) with E = B * 2048 / L, is found by
+//        histograms spaced evenly in score over the sample's range, refined until the bin that
+//        holds it has at most 256 keys, which are ranked against each other. The threshold only
+//        decides which keys travel to the select kernel; the selection itself is exact. At decode
+//        the same kernel first stores the new token: its K and V rows and its scoring code
+//        e4m3(M_h k) (float64 sum, one rounding).
+// scan   CTAs over (chunk of positions, sequence x KV head): a stream of the FP8 scoring rows,
+//        page-table indexed. Each of the 8 warps walks a contiguous run of 16-token tiles through
+//        its own ring of shared-memory stages filled by 16-byte cp.async copies (3 stages at
+//        32-byte rows, 4 at 64-byte rows, 2 at 128-byte rows), all but one stage in flight ahead
+//        of the tile being scored. The codes are widened exactly to f16 (cvt e4m3x2 -> f16x2) and
+//        multiplied by the two digit vectors on the tensor cores (mma.sync m16n8k16, fp32
+//        accumulation); every lane ends up with one complete score. Keys at or above the
+//        threshold are appended with their positions, in position order, to the warp's region.
 // select one CTA per (sequence, KV head): the exact budget-th largest key among the candidates
-//        (radix digits of 11, 11 and 10 bits over order-preserving 32-bit keys), every key above
-//        it and the equal keys in position order up to the budget (ties go to the lower
-//        position), written as the index set in ascending order. If the candidates are fewer
-//        than the budget (the sampled threshold was too high -- not expected in practice), the
-//        CTA first rescans the sequence with no threshold, so the result is exact in every case.
+//        and the ordered emission of the index set (keys above it, then equal keys in position
+//        order up to the budget: ties go to the lower position), ascending. Three tiers: the
+//        candidates of up to 128 regions held in registers, up to 6144 candidates flattened into
+//        registers, or candidates staged in shared memory (or read in place) with a general
+//        histogram / radix selection. If the candidates are fewer than the budget (the sampled
+//        threshold was too high -- not expected in practice), the CTA first rescans the sequence
+//        with no threshold, so the result is exact in every case.
 // seq_len <= budget selects every position without scoring.
 #include <cuda_fp16.h>
 
