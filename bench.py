@@ -34,7 +34,7 @@ METRIC = "JSSA decode-attn steps/s & HBM GB/s at 128K ctx vs dense full-KV, 1×B
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=800)
+    ap.add_argument("--steps", type=int, default=64)
     ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", choices=["jssa", "reference"], default="jssa")
     ap.add_argument("--workload", choices=["llama128k", "hybrid", "mla"], default="llama128k",
@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--no-check", action="store_true", help="skip the oracle agreement in the CPU baseline leg")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--mla-batch", type=int, default=16, help="sequences of the mla workload")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="llama128k: skip the hybrid and mla sub-measurements of the default line")
     return ap.parse_args()
 
 
@@ -172,6 +174,19 @@ def workload(args, rank):
     return w.replace(seed=w.seed + 7919 * rank)
 
 
+def config_of(w, world):
+    """The workload description both arms print (identical for the same arguments)."""
+    return {
+        "workload": f"llama3-8b-layer-128k: h_q {w.h_q}, h_kv {w.h_kv}, d {w.d}, L {w.seq_len}, "
+                    f"page {w.page_size} (permuted), r {w.rank}, B {w.budget}, batch {w.batch} per GPU",
+        "global_batch": w.batch * world,
+        "seq_len": w.seq_len,
+        "budget": w.budget,
+        "parallelism": f"dp{world} (independent sequences per GPU)",
+        "l2": "inputs larger than L2: the 512 MiB scoring cache is streamed every step; 8 query sets rotate",
+    }
+
+
 def setup_gpu(w, dev):
     import torch
     import token_level_sparse_fp8_b200 as J
@@ -217,33 +232,95 @@ def timed(fn, steps, warmup, stream, barrier):
 
 
 class GraphSteps:
-    """`per` consecutive calls fn(0..per-1) captured once in a CUDA graph; stepping replays it.
-    Removes the host launch cost from device timings (the kernels themselves are unchanged)."""
+    """`per` consecutive calls fn(first..first+per-1) captured once in a CUDA graph; calling it
+    replays the graph. Removes the host launch cost from device timings (the kernels themselves
+    are unchanged)."""
 
-    def __init__(self, fn, per, warmup=2):
+    def __init__(self, fn, per, warmup=2, first=0):
         import torch
         for i in range(warmup):
-            fn(i)
+            fn(first + i)
         torch.cuda.synchronize()
         self.per = per
         self.graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.graph):
             for i in range(per):
-                fn(i)
+                fn(first + i)
         torch.cuda.synchronize()
 
-    def __call__(self, i):
+    def __call__(self, i=0):
         self.graph.replay()
 
 
 def timed_graph(fn, steps, warmup, stream, barrier, per=8):
-    """Device time of `steps` calls (rounded up to whole graphs of `per` calls) and the count."""
+    """Device time of `steps` calls (rounded up to whole graphs of `per` calls) and the count
+    (used for the per-kernel figures, not for the headline steps)."""
     g = GraphSteps(fn, per)
     reps = max(1, -(-steps // per))
     wreps = max(1, -(-warmup // per))
     t = timed(g, reps, wreps, stream, barrier)
     del g
     return t, reps * per
+
+
+class ExactSteps:
+    """Exactly `steps` consecutive calls fn(0..steps-1) per run: a CUDA graph of `per` calls
+    replayed steps // per times, then a graph of the steps % per remaining calls (query sets
+    rotate with i, so the remainder continues the rotation)."""
+
+    def __init__(self, fn, steps, per=8):
+        self.steps = steps
+        self.n_main = steps // per
+        self.main = GraphSteps(fn, per) if self.n_main else None
+        rem = steps % per
+        self.rem = GraphSteps(fn, rem, warmup=0, first=self.n_main * per) if rem else None
+
+    def __call__(self):
+        for _ in range(self.n_main):
+            self.main()
+        if self.rem is not None:
+            self.rem()
+
+
+def repeated_runs(run, steps, warmup_fn, warmup, stream, group, sampler=None, min_region_s=0.2,
+                  max_repeats=400):
+    """Runs of exactly `steps` steps (`run()` issues them), each bracketed by a barrier and a
+    device synchronisation on both sides and timed with CUDA events on `stream`, repeated until
+    about `min_region_s` of device time so that the clock sampler sees the region; `warmup`
+    untimed steps first. Returns the per-run seconds (max over ranks), one entry per run."""
+    import torch
+    for i in range(warmup):
+        warmup_fn(i)
+    torch.cuda.synchronize()
+
+    def one():
+        group.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        group.barrier()
+        return group.max_over_ranks(e0.elapsed_time(e1) / 1e3)
+
+    first = one()
+    repeats = int(group.max_over_ranks(min(max_repeats, max(1, math.ceil(min_region_s / max(first, 1e-9))))))
+    if sampler is not None:
+        sampler.start()
+    times = [one() for _ in range(repeats)]
+    clocks = sampler.stop() if sampler is not None else None
+    return times, clocks
+
+
+def step_stats(times, steps):
+    """Per-step milliseconds over the runs: median, p10, p90 (and the run count)."""
+    import numpy as np
+    per = np.asarray(times) / steps * 1e3
+    return {"median": float(np.median(per)), "p10": float(np.percentile(per, 10)),
+            "p90": float(np.percentile(per, 90)), "runs": len(times),
+            "timed_region_s": float(np.sum(times))}
 
 
 def algorithmic_bytes(w, dense=False):
@@ -310,12 +387,15 @@ def oracle_pair_inputs(state, w, b, h):
     the caches (one head) with an identity page table."""
     import numpy as np
     import torch
+    from oracle import jssa as O
     layer = state["layer"]
     bt = state["kv"]["block_table"][b].long()
     k = layer.k_cache[bt][:, :, h : h + 1].to(torch.float64).cpu().numpy()
     v = layer.v_cache[bt][:, :, h : h + 1].to(torch.float64).cpu().numpy()
-    sc = layer.score_cache[bt][:, h : h + 1].cpu().numpy()
     m = layer.basis[h : h + 1].double().cpu().numpy()
+    # the oracle's own store of every position (not the library's scoring cache)
+    n_pages, ps = k.shape[0], k.shape[1]
+    sc = O.store_codes(k[:, :, 0].reshape(-1, k.shape[-1]), m[0]).reshape(n_pages, 1, ps, -1)
     return k, v, sc, m, np.arange(bt.numel(), dtype=np.int64)[None]
 
 
@@ -371,11 +451,14 @@ def cpu_baseline(state, w, seconds, check=True):
             agreement.append(dict(pair=[b, h], **pair_agreement(s[(0, 0)], sym, w.budget, go, rout[0])))
         done += 1
     per_pair = t_total / done
-    steps_per_s = 1.0 / (per_pair * w.batch * w.h_kv)
+    pairs_per_step = w.batch * w.h_kv
+    steps_per_s = 1.0 / (per_pair * pairs_per_step)
     res = {"value": steps_per_s, "unit": "steps/s", "cores": cores, "kind": "oracle",
+           "measured_s_per_pair": per_pair, "extrapolated_pairs_per_step": pairs_per_step,
            "sample": f"{done} oracle calls on 2 (sequence, KV head) pairs of the timed workload "
-                     f"(score+top-B+attend over {w.seq_len} tokens, float64 NumPy), {t_total:.1f} s; "
-                     f"steps/s = 1 / (time per pair x {w.batch * w.h_kv} pairs per step)"}
+                     f"(score+top-B+attend over {w.seq_len} tokens, float64 NumPy), {t_total:.1f} s "
+                     f"measured; steps/s extrapolated = 1 / (measured time per pair x "
+                     f"{pairs_per_step} pairs per step)"}
     if check:
         res["agreement"] = {"ok": all(a["ok"] for a in agreement), "pairs": agreement}
     return res
@@ -425,7 +508,7 @@ def cpu_baseline_hybrid(state, w, seconds, local_kv, q0, scale, check=True):
     return res
 
 
-def cpu_baseline_mla(q, latent, bt, lens, m_big, sc, idx, count, out, budget, scale, step,
+def cpu_baseline_mla(q, latent, bt, lens, m_lat, sc, idx, count, out, budget, scale, step,
                      seconds, check=True):
     """The oracle on host cores for the MLA step on one sequence (select over the latent scoring
     cache + latent attention over the selected rows), repeated for about `seconds`; the first
@@ -442,10 +525,13 @@ def cpu_baseline_mla(q, latent, bt, lens, m_big, sc, idx, count, out, budget, sc
     L = int(lens[b])
     pages = bt[b].long()
     kv = latent[pages].double().cpu().numpy()[:, :, None]          # [pages, ps, 1, 576]
-    codes = sc[pages].cpu().numpy()
     ident = np.arange(pages.numel(), dtype=np.int64)[None]
     qn = q[b:b + 1].double().cpu().numpy()
-    mn = m_big.double().cpu().numpy()
+    mn = O.mla_scoring_basis(m_lat[0].double().cpu().numpy())  # the oracle's block basis [128, 576]
+    # the oracle's own store of every position (not the library's scoring cache)
+    n_pages, ps = kv.shape[0], kv.shape[1]
+    codes = O.store_codes(kv.reshape(-1, 576), mn).reshape(n_pages, 1, ps, -1)
+    mn = mn[None]
     done, t_total = 0, 0.0
     while t_total < seconds or done < 1:
         t0 = time.perf_counter()
@@ -474,12 +560,13 @@ def cpu_baseline_mla(q, latent, bt, lens, m_big, sc, idx, count, out, budget, sc
 
 
 def run_reference(args):
-    """CPU oracle arm: rank 0 only, bounded sample of the same workload."""
+    """CPU oracle arm: rank 0 only. Each step is a bounded sample of the workload, the oracle's
+    score + top-B + attend for one (sequence, KV head) pair of it; `ms_per_step` is the measured
+    time of that sample, and `value` extrapolates it to whole steps (pairs per step stated)."""
     rank, world, _ = dist_env()
     if rank != 0:
         return
     import numpy as np
-    import torch
     from oracle import jssa as O
     from synth import build_paged_kv, layer_factors, sample_decode_queries
     w = workload(args, 0)
@@ -505,21 +592,25 @@ def run_reference(args):
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             times.append(dt)
-    per_pair = statistics.mean(times)
+    per_pair = statistics.median(times)
     value = 1.0 / (per_pair * pairs_per_step)
+    sample = (f"each step: the oracle's score+top-B+attend (float64 NumPy) for one (sequence, KV "
+              f"head) pair of the workload, {w.seq_len} tokens, timed; value extrapolates the "
+              f"median measured time per pair to {pairs_per_step} pairs per step")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": per_pair * pairs_per_step * 1e3, "higher_is_better": True,
+        "ms_per_step": per_pair * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"llama3-8b-layer-128k (h_q {w.h_q}, h_kv {w.h_kv}, d {w.d}, L {w.seq_len}, "
-                               f"ps {w.page_size}, r {w.rank}, B {w.budget}, batch {w.batch})",
-                   "global_batch": w.batch, "seq_len": w.seq_len, "parallelism": "host cores"},
+        "config": config_of(w, world),
+        "step_is": "one (sequence, KV head) pair per timed step (a bounded sample of one step)",
+        "measured_ms_per_pair": {"median": per_pair * 1e3, "p10": float(np.percentile(times, 10)) * 1e3,
+                                 "p90": float(np.percentile(times, 90)) * 1e3},
+        "extrapolated_pairs_per_step": pairs_per_step,
         "cpu_baseline": {"value": value, "unit": "steps/s", "cores": cores, "kind": "oracle",
-                         "sample": f"each step: one (sequence, KV head) pair of the workload "
-                                   f"(score+top-B+attend in float64 NumPy), scaled by "
-                                   f"{pairs_per_step} pairs per step"},
+                         "sample": sample},
         "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "impl_detail": f"float64 NumPy oracle on {cores} host cores",
     }
     print(json.dumps(line), flush=True)
 
@@ -548,26 +639,14 @@ def run_jssa(args):
     def step(i):
         layer.step(qs[i % nq], k_new, v_new, out)
 
-    sampler = ClockSampler(local)
-    # the whole step sequence is replayed from a CUDA graph (as in the pages' decode protocol)
-    g_step = GraphSteps(step, nq)
-    reps = max(1, -(-args.steps // nq))
-    for _ in range(max(1, -(-args.warmup // nq))):
-        g_step(0)
-    barrier()
-    torch.cuda.synchronize()
-    sampler.start()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(reps):
-        g_step(0)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    clocks = sampler.stop()
-    barrier()
-    n_steps = reps * nq
-    t_step = max_over_ranks(e0.elapsed_time(e1) / 1e3)
-    del g_step
+    # exactly args.steps steps per run, replayed from CUDA graphs (as in the pages' decode
+    # protocol); runs repeat until the timed region spans about 0.2 s
+    step(0)  # sizes the workspace before capture
+    runs = ExactSteps(step, args.steps, nq)
+    times, clocks = repeated_runs(runs, args.steps, step, args.warmup, stream, group,
+                                  ClockSampler(local))
+    del runs
+    st = step_stats(times, args.steps)
     launches_per_step = 4  # prep, scan, select, attention
 
     # per-kernel device times (same configuration, each kernel launched alone)
@@ -652,7 +731,12 @@ def run_jssa(args):
         layer.step(q_dev, kn_dev, vn_dev, out)
         out_host.copy_(out, non_blocking=True)
 
-    t_e2e = max_over_ranks(timed(e2e_step, args.steps, args.warmup, stream, barrier))
+    def e2e_run():
+        for i in range(args.steps):
+            e2e_step(i)
+
+    e2e_times, _ = repeated_runs(e2e_run, args.steps, e2e_step, args.warmup, stream, group)
+    t_e2e = statistics.median(e2e_times)
     h2d = qs[0].numel() * 2 + k_new.numel() * 2 + v_new.numel() * 2
     d2h = out.numel() * 2
 
@@ -660,13 +744,9 @@ def run_jssa(args):
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline(state, w, args.cpu_seconds, check=not args.no_check)
 
-    group.close()
-    if rank != 0:
-        return
-
     peak, peak_kind = peaks()
-    ms_step = t_step / n_steps * 1e3
-    steps_per_s = whole_job_rate(world, n_steps, t_step)
+    ms_step = st["median"]
+    steps_per_s = world / (ms_step / 1e3)
     bytes_step = algorithmic_bytes(w)
     score_launch_s = t_score
     achieved = score_bytes(w) / score_launch_s / 1e9
@@ -675,23 +755,16 @@ def run_jssa(args):
         "value": steps_per_s,
         "unit": "steps/s",
         "n_gpus": world,
-        "steps": n_steps,
+        "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": ms_step,
+        "ms_per_step_stats": st,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16 K/V, e4m3 scoring cache, fp32 math",
         "data": "synthetic",
-        "config": {
-            "workload": f"llama3-8b-layer-128k: h_q {w.h_q}, h_kv {w.h_kv}, d {w.d}, L {w.seq_len}, "
-                        f"page {w.page_size} (permuted), r {w.rank}, B {w.budget}, batch {w.batch} per GPU",
-            "global_batch": w.batch * world,
-            "seq_len": w.seq_len,
-            "budget": w.budget,
-            "parallelism": f"dp{world} (independent sequences per GPU)",
-            "l2": "inputs larger than L2: the 512 MiB scoring cache is streamed every step; 8 query sets rotate",
-        },
+        "config": config_of(w, world),
         "hbm_gbs": bytes_step / (ms_step / 1e3) / 1e9,
         "roofline_step": {"bound": "hbm", "achieved": bytes_step / (ms_step / 1e3) / 1e9, "peak": peak,
                           "unit": "GB/s", "frac": bytes_step / (ms_step / 1e3) / 1e9 / peak,
@@ -705,9 +778,14 @@ def run_jssa(args):
                        "attend_gbs": attend_bytes(w) / t_attend / 1e9},
         "clocks": clocks,
         "e2e": {"value": whole_job_rate(world, args.steps, t_e2e), "unit": "steps/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches_per_step * n_steps,
-        "timing": "CUDA events around replays of a CUDA graph holding 8 consecutive steps",
+                "d2h_bytes_per_step": d2h,
+                "timing": f"median of {len(e2e_times)} runs of exactly {args.steps} steps through the "
+                          f"Python API (pinned-host H2D of q, k_new, v_new; D2H of the output)"},
+        "gpu_launches": launches_per_step * args.steps,
+        "timing": (f"each run: exactly {args.steps} steps replayed from CUDA graphs (8 consecutive "
+                   f"steps per graph, then the remainder), CUDA events on the launching stream, "
+                   f"barrier + synchronise on both sides; {st['runs']} runs, median per step "
+                   f"(p10 / p90 in ms_per_step_stats)"),
     }
     if t_dense is not None:
         dense_bytes = algorithmic_bytes(w, dense=True)
@@ -732,7 +810,21 @@ def run_jssa(args):
             "gather_free": t_dense / t_attend, "gather_then_attend": t_dense / t_gta}
     if cpu is not None:
         line["cpu_baseline"] = cpu
-    print(json.dumps(line), flush=True)
+    # the other two workloads of the method (hybrid local/global stack, MLA layer), measured in the
+    # same run as sub-objects; the headline keys above describe the 128K layer only
+    del state, layer, qs, k_new, v_new, out, sets, bufs, ws_score, ws_attend, ws_gta
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    if not args.headline_only:
+        for name, fn in (("hybrid", measure_hybrid), ("mla", measure_mla)):
+            sub = fn(args, group, dev, local, rank, world, with_cpu=False)
+            line[name] = {k: v for k, v in sub.items()
+                          if k not in ("n_gpus", "higher_is_better", "vs_baseline", "data", "warmup")}
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+    group.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
 
 
 def hybrid_bytes(w, dense=False):
@@ -748,7 +840,21 @@ def hybrid_bytes(w, dense=False):
     return glob + local
 
 
-def run_hybrid(args):
+def run_workload(args, measure):
+    """One workload alone (``--workload hybrid`` / ``mla``): its own JSON line."""
+    import torch
+    rank, world, local = dist_env()
+    assert torch.cuda.is_available(), "bench needs a CUDA device"
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    group = RankGroup("nccl", dev)
+    line = measure(args, group, dev, local, rank, world, with_cpu=True)
+    group.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def measure_hybrid(args, group, dev, local, rank, world, with_cpu=True):
     """One stack step of a hybrid model: (layers - 1) sliding-window layers, each dense paged
     decode over the last `window` positions of its own KV cache, and one global layer, a full JSSA
     decode step (store + score + top-B + indexed attend) over the whole context."""
@@ -756,11 +862,6 @@ def run_hybrid(args):
     import token_level_sparse_fp8_b200 as J
     from synth import WORKLOADS, build_paged_kv, layer_factors
 
-    rank, world, local = dist_env()
-    assert torch.cuda.is_available(), "bench needs a CUDA device"
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    group = RankGroup("nccl", dev)
     barrier, max_over_ranks = group.barrier, group.max_over_ranks
     w = WORKLOADS["hybrid"]
     w = w.replace(seed=w.seed + 7919 * rank)
@@ -793,38 +894,35 @@ def run_hybrid(args):
         local_layers(i)
         layer.dense(qs[i % nq], out)
 
-    sampler = ClockSampler(local)
     step(0)
     dense_step(0)  # sizes the workspaces before capture
     torch.cuda.synchronize()
-    barrier()
-    sampler.start()
-    t_step, n_steps = timed_graph(step, args.steps, args.warmup, stream, barrier, nq)
-    clocks = sampler.stop()
-    t_step = max_over_ranks(t_step)
+    runs = ExactSteps(step, args.steps, nq)
+    times, clocks = repeated_runs(runs, args.steps, step, args.warmup, stream, group,
+                                  ClockSampler(local))
+    del runs
+    st = step_stats(times, args.steps)
     t_dense = None
     if not args.no_dense:
         t_dense, n_dense = timed_graph(dense_step, max(8, args.steps // 4), 8, stream, barrier, nq)
         t_dense = max_over_ranks(t_dense) / n_dense
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu:
+    if with_cpu and rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline_hybrid(state, w, args.cpu_seconds, locals_[0], qs[0], scale,
                                   check=not args.no_check)
-    group.close()
-    if rank != 0:
-        return
     peak, peak_kind = peaks()
-    ms_step = t_step / n_steps * 1e3
+    ms_step = st["median"]
     bytes_step = hybrid_bytes(w)
     achieved = bytes_step / (ms_step / 1e3) / 1e9
     line = {
         "metric": "hybrid local/global stack decode steps/s (5 sliding-window + 1 global JSSA layer), 1xB200",
-        "value": whole_job_rate(world, n_steps, t_step),
+        "value": world / (ms_step / 1e3),
         "unit": "steps/s",
         "n_gpus": world,
-        "steps": n_steps,
+        "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": ms_step,
+        "ms_per_step_stats": st,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -846,8 +944,9 @@ def run_hybrid(args):
                           "frac": achieved / peak, "traffic": None, "bytes_per_step": bytes_step,
                           "peak_kind": peak_kind},
         "clocks": clocks,
-        "gpu_launches": (w.layers - 1 + 4) * n_steps,  # a dense kernel per local layer + 4
-        "timing": "CUDA events around replays of a CUDA graph holding 8 consecutive stack steps",
+        "gpu_launches": (w.layers - 1 + 4) * args.steps,  # a dense kernel per local layer + 4
+        "timing": (f"each run: exactly {args.steps} stack steps replayed from CUDA graphs, CUDA "
+                   f"events; {st['runs']} runs, median per step"),
     }
     if t_dense is not None:
         dense_bytes = hybrid_bytes(w, dense=True)
@@ -856,7 +955,7 @@ def run_hybrid(args):
         line["speedup_vs_dense"] = t_dense / (ms_step / 1e3)
     if cpu is not None:
         line["cpu_baseline"] = cpu
-    print(json.dumps(line), flush=True)
+    return line
 
 
 def mla_bytes(batch, seq_len, budget, page_size, dense=False):
@@ -868,7 +967,7 @@ def mla_bytes(batch, seq_len, budget, page_size, dense=False):
     return batch * (seq_len * 128 + min(budget, seq_len) * 1152 + 4 * pages)
 
 
-def run_mla(args):
+def measure_mla(args, group, dev, local, rank, world, with_cpu=True):
     """One decode step of a multi-head latent attention layer (128 query heads, one latent head of
     512 + 64 dims, 64-token pages): store of the new token's scoring row, score + top-B on the
     latent scoring cache, absorbed latent attention over the selected rows."""
@@ -876,26 +975,18 @@ def run_mla(args):
     import token_level_sparse_fp8_b200 as J
     from synth import build_paged_kv, layer_factors, sample_calibration, sample_decode_queries
 
-    rank, world, local = dist_env()
-    assert torch.cuda.is_available(), "bench needs a CUDA device"
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    group = RankGroup("nccl", dev)
     barrier, max_over_ranks = group.barrier, group.max_over_ranks
     batch, h_q, L, ps, B, r_lat = args.mla_batch, 128, args.seq_len, 64, args.budget, 64
     seed = 1004 + 7919 * rank
     J._lib.load()
     f = layer_factors(seed, 0, 1, 576)
-    # latent basis: second moments of the head-mean latent queries and of the latent rows, then
-    # the top-64 eigenvectors (the library's Jacobi solver)
+    # latent basis [1, 64, 512]: the library's second moments of the head-mean latent queries and
+    # of the latent rows, then its Jacobi solver at d 512
     qc, kc = sample_calibration(f, 4096, h_q, seed, device=dev)
-    qbar = qc[..., :512].double().mean(dim=1)
-    lat = kc[:, 0, :512].double()
-    gram_q = (qbar.T @ qbar)[None].contiguous()
-    gram_k = (lat.T @ lat)[None].contiguous()
-    del qc, kc, qbar, lat
-    m_lat, _ = J.compute_basis(gram_q, gram_k, r_lat)
-    m_big = J.mla_scoring_basis(m_lat)
+    cal = J.Calibration(1, 512, dev)
+    cal.add_latent(qc, kc[:, 0])
+    m_lat, _ = cal.basis(r_lat)
+    del qc, kc, cal
     kv = build_paged_kv(f, [L] * batch, ps, seed, device=dev)
     latent = kv["k_cache"].view(kv["k_cache"].shape[0], ps, 576)
     del kv["v_cache"]
@@ -906,7 +997,7 @@ def run_mla(args):
     for p0 in range(0, num_pages, 4096):
         p1 = min(num_pages, p0 + 4096)
         slots = torch.arange(p0 * ps, p1 * ps, dtype=torch.int64, device=dev)
-        J.store(flat[p0 * ps:p1 * ps], slots, m_big, sc)
+        J.store(flat[p0 * ps:p1 * ps], slots, m_lat, sc)
     nq = 8
     qs = [sample_decode_queries(f, batch, h_q, seed, step=i, device=dev) for i in range(nq)]
     # the new token of each step is the last cached position (rewriting its code is idempotent)
@@ -921,18 +1012,17 @@ def run_mla(args):
     stream = torch.cuda.current_stream(dev)
 
     def step(i):
-        J.store(k_new, new_slots, m_big, sc)
-        J.score_topk(qs[i % nq], m_big, sc, bt, lens, B, idx, count, ws_s)
+        J.store(k_new, new_slots, m_lat, sc)
+        J.score_topk(qs[i % nq], m_lat, sc, bt, lens, B, idx, count, ws_s)
         J.mla_attend(qs[i % nq], latent, bt, idx, count, scale, out, ws_a)
 
-    sampler = ClockSampler(local)
-    step(0)
+    step(0)  # sizes the workspaces before capture
     torch.cuda.synchronize()
-    barrier()
-    sampler.start()
-    t_step, n_steps = timed_graph(step, args.steps, args.warmup, stream, barrier, nq)
-    clocks = sampler.stop()
-    t_step = max_over_ranks(t_step)
+    runs = ExactSteps(step, args.steps, nq)
+    times, clocks = repeated_runs(runs, args.steps, step, args.warmup, stream, group,
+                                  ClockSampler(local))
+    del runs
+    st = step_stats(times, args.steps)
 
     def attend_only(i):
         J.mla_attend(qs[i % nq], latent, bt, idx, count, scale, out, ws_a)
@@ -941,7 +1031,7 @@ def run_mla(args):
     t_att = max_over_ranks(t_att) / n_att
 
     def score_only(i):
-        J.score_topk(qs[i % nq], m_big, sc, bt, lens, B, idx, count, ws_s)
+        J.score_topk(qs[i % nq], m_lat, sc, bt, lens, B, idx, count, ws_s)
 
     t_sc, n_sc = timed_graph(score_only, args.steps, args.warmup, stream, barrier, nq)
     t_sc = max_over_ranks(t_sc) / n_sc
@@ -958,25 +1048,23 @@ def run_mla(args):
         t_dense, n_dense = timed_graph(dense, max(8, args.steps // 8), 8, stream, barrier, nq)
         t_dense = max_over_ranks(t_dense) / n_dense
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu:
-        cpu = cpu_baseline_mla(qs[0], latent, bt, lens, m_big, sc, idx, count, out, B, scale, step,
+    if with_cpu and rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline_mla(qs[0], latent, bt, lens, m_lat, sc, idx, count, out, B, scale, step,
                                args.cpu_seconds, check=not args.no_check)
-    group.close()
-    if rank != 0:
-        return
     peak, peak_kind = peaks()
-    ms_step = t_step / n_steps * 1e3
+    ms_step = st["median"]
     bytes_step = mla_bytes(batch, L, B, ps)
     achieved = bytes_step / (ms_step / 1e3) / 1e9
     flops_att = 2.0 * batch * h_q * min(B, L) * (576 + 512)
     line = {
         "metric": "MLA decode steps/s (128 heads, 576-dim latent rows) at 128K ctx, 1xB200",
-        "value": whole_job_rate(world, n_steps, t_step),
+        "value": world / (ms_step / 1e3),
         "unit": "steps/s",
         "n_gpus": world,
-        "steps": n_steps,
+        "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": ms_step,
+        "ms_per_step_stats": st,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -1010,8 +1098,9 @@ def run_mla(args):
                             "unit": "TFLOP/s", "frac": flops_att / t_att / 1e12 / bf16_peak()[0],
                             "traffic": None, "peak_kind": bf16_peak()[1]},
         "clocks": clocks,
-        "gpu_launches": 5 * n_steps,  # store, prep, scan, select, latent attention
-        "timing": "CUDA events around replays of a CUDA graph holding 8 consecutive steps",
+        "gpu_launches": 5 * args.steps,  # store, prep, scan, select, latent attention
+        "timing": (f"each run: exactly {args.steps} steps replayed from CUDA graphs, CUDA events; "
+                   f"{st['runs']} runs, median per step"),
     }
     if t_dense is not None:
         dense_bytes = mla_bytes(batch, L, B, ps, dense=True)
@@ -1021,7 +1110,7 @@ def run_mla(args):
         line["speedup_vs_dense"] = t_dense / (ms_step / 1e3)
     if cpu is not None:
         line["cpu_baseline"] = cpu
-    print(json.dumps(line), flush=True)
+    return line
 
 
 def main():
@@ -1029,9 +1118,9 @@ def main():
     if args.impl == "reference":
         run_reference(args)
     elif args.workload == "hybrid":
-        run_hybrid(args)
+        run_workload(args, measure_hybrid)
     elif args.workload == "mla":
-        run_mla(args)
+        run_workload(args, measure_mla)
     else:
         run_jssa(args)
 

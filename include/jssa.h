@@ -35,9 +35,16 @@
  * - Device-side checks: a page number outside [0, num_pages), a position outside the block
  *   table, or a seq_len above max_pages*page_size is never dereferenced: the row is skipped and
  *   a flag is raised in the library's device error word (jssa_device_error). Kernels never trap.
- * - Supported template shapes: d = 128 with r in {32, 64}, and d = 256 with r = 64 (the
- *   global layer of a hybrid sliding-window / global stack); G <= 8 for attention; calibration
- *   needs G * d <= 2048.
+ * - Supported template shapes: d = 128 with r in {16, 32, 64}, and d = 256 with r = 64 (the
+ *   global layer of a hybrid sliding-window / global stack); G <= 8 for attention. A basis of
+ *   rank below 16 runs through the r = 16 instance with zero rows appended: their codes are
+ *   zero and the scores, hence the selections, are those of the smaller rank.
+ * - Multi-head latent attention (one latent "KV head" of 576 dimensions per token: 512 latent +
+ *   64 rotary): the store and score entry points take d = 576 and r = 64, the rank of the latent
+ *   basis, float32 [1, r, 512], which projects the 512 latent dimensions; the 64 rotary
+ *   dimensions pass through unprojected, so a scoring row holds r + 64 = 128 codes (JSSA README,
+ *   section 4 notes: the MLA basis is [1, r, kv_lora_rank]; JSSA summary, section 3.4: 64 latent
+ *   + 64 RoPE scoring dimensions). The scoring cache is then uint8 [num_pages, 1, page_size, 128].
  */
 #ifndef JSSA_H_
 #define JSSA_H_
@@ -97,6 +104,18 @@ JSSA_API const char* jssa_status_string(int status);
 JSSA_API int jssa_version(void);
 
 /*
+ * Debug control (the pages have no counterpart): the clock-cycle limit of each wait on the tensor
+ * cores inside the tile loop of jssa_mla_attend (default 2e9 cycles, about one second at the
+ * boost clock). A wait that runs out raises JSSA_DEVERR_TIMEOUT in the device error word; the
+ * CTA then waits, with the default limit, for every tensor-core operation it issued, frees its
+ * tensor memory and returns, so the context stays usable and the next call runs normally (its
+ * output is invalid only for the call that timed out). cycles <= 0 restores the default. The limit
+ * is read when a call is enqueued (a kernel argument): a CUDA graph keeps the limit it was captured
+ * with. Returns the previous limit. Process-wide; not synchronised with calls in flight.
+ */
+JSSA_API long long jssa_set_wait_limit(long long cycles);
+
+/*
  * Bytes of device workspace the entry point `fn` needs for these sizes (written to *bytes; 0
  * means none). max_pages and page_size are the block-table width and page size the call will
  * get (every seq_len is at most max_pages*page_size); budget is the token budget B, except for
@@ -124,12 +143,32 @@ JSSA_API int jssa_workspace_init(void* ws, size_t ws_bytes, jssa_stream_t stream
  * q: bf16 [n, h_q, d], row n at q + n*q_stride_n (elements, >= h_q*d, multiple of 8).
  * k: bf16 [n, h_kv, d], row n at k + n*k_stride_n (elements, >= h_kv*d, multiple of 8).
  * gram_q, gram_k: float64 [h_kv, d, d], accumulated in place (zero them before the first call).
- * Products of the exact bf16 inputs are summed in fp32 on tensor cores within a tile of samples
- * and added to the float64 totals. n may be 0 (no-op).
+ * d in {128, 256, 512}; n <= 16776960 per call (JSSA_ERR_SHAPE beyond), any G.
+ * Products of exact bf16 inputs are summed in fp32 on tensor cores within a tile of samples and
+ * added to the float64 totals: for G * d <= 2048 the G^2 products of each sample's query heads
+ * (exact), otherwise the group mean formed in fp32 and split exactly into three bf16 planes (the
+ * six largest plane products; the rest are below 2^-24 of the result). n may be 0 (no-op).
  */
 JSSA_API int jssa_calibrate_accumulate(const jssa_bf16* q, int64_t q_stride_n, const jssa_bf16* k,
                               int64_t k_stride_n, int n, int h_q, int h_kv, int d,
                               double* gram_q, double* gram_k, jssa_stream_t stream);
+
+/*
+ * Calibration, step 1, for a multi-head latent layer: the second moments of the head mean of the
+ * latent part of the absorbed queries and of the latent part of the cached rows, from which
+ * jssa_compute_basis (d = 512) gives the latent basis [1, r, 512]. JSSA README, section 2 (the MLA
+ * basis [1, r, kv_lora_rank]; the Gram collection of large latent models) and section 4 notes.
+ *   gram_q += sum_n qbar_n qbar_n^T, qbar_n = (1/h_q) sum_i q[n, i, 0:512]
+ *   gram_k += sum_n c_n c_n^T,       c_n = kv[n, 0:512]
+ * q: bf16 absorbed queries, head i of sample n at q + n*q_stride_n + i*q_stride_head (576 per
+ * head, q_stride_head >= 512; strides multiples of 8 elements). kv: bf16 latent rows, row n at
+ * kv + n*kv_stride_n (>= 512). gram_q, gram_k: float64 [1, 512, 512], accumulated in place.
+ * Same arithmetic and limits as jssa_calibrate_accumulate (the mean-plane form).
+ */
+JSSA_API int jssa_mla_calibrate_accumulate(const jssa_bf16* q, int64_t q_stride_n,
+                                           int64_t q_stride_head, const jssa_bf16* kv,
+                                           int64_t kv_stride_n, int n, int h_q, double* gram_q,
+                                           double* gram_k, jssa_stream_t stream);
 
 /*
  * Calibration, step 2: M = TopEig_r(gram_q/tr(gram_q) + gram_k/tr(gram_k))^T per KV head.
@@ -150,7 +189,9 @@ JSSA_API int jssa_compute_basis(const double* gram_q, const double* gram_k, int 
  * section 4 notes (r bytes per token and KV head). The projection is summed in float64 and
  * rounded once to E4M3 (round to nearest even, saturating to +-448, no scale).
  * k: bf16 [t, h_kv, d] with row stride k_stride_t elements. slot_mapping: int64 [t], flat slot
- * page*page_size + offset, negative = skip. score_cache: see conventions.
+ * page*page_size + offset, negative = skip. score_cache: see conventions. A latent layer (d 576,
+ * r 64) writes e4m3(M_lat k[0:512]) and then e4m3(k[512:576]) (the rotary dimensions, one
+ * rounding each).
  */
 JSSA_API int jssa_store(const jssa_bf16* k, int64_t k_stride_t, const int64_t* slot_mapping, int t,
                int h_kv, int d, int r, const float* basis, uint8_t* score_cache,
@@ -230,8 +271,8 @@ JSSA_API int jssa_score_topk_bf16(const jssa_bf16* q, const float* basis,
  * rotary dimensions, attended in place):
  *   out[b, i, :] = sum_j softmax_j(softmax_scale * q[b, i] . kv[j]) kv[j, 0:512]
  * over j in the index set of sequence b, i.e. jssa_score_topk run with h_kv = 1, d = 576 and
- * r = 128 on the latent scoring cache (basis rows: the projected 512 latent dimensions, then the
- * 64 rotary dimensions passed through).
+ * r = 64 on the latent scoring cache (the latent basis [1, 64, 512]; the 64 rotary dimensions
+ * pass through).
  * q: bf16 [batch, h_q, 576] absorbed queries (h_q a multiple of 16; budget <= 262144,
  * JSSA_ERR_UNSUPPORTED otherwise). kv_cache: bf16 latent cache,
  * row (page p, slot s) at p*kv_page_stride + s*kv_slot_stride elements (576 contiguous, 16-byte

@@ -124,7 +124,8 @@ def test_mla_decode_step_full_size():
     # the basis only has to be some calibrated basis of this generator: 32 query heads suffice
     qc, kc = sample_calibration(f, 2048, 32, seed)
     cal = O.calibrate(f64(qc)[..., :512], f64(kc)[..., :512], r_lat)
-    m_big = O.mla_scoring_basis(cal["M"][0]).astype(np.float32)[None]   # [1, 128, 576]
+    m_lat = cal["M"].astype(np.float32)                                  # [1, 64, 512]
+    m_big = O.mla_scoring_basis(m_lat[0]).astype(np.float32)[None]       # the oracle's [1, 128, 576]
     del qc, kc
     kv = build_paged_kv(f, [L] * batch, ps, seed, device=dev)
     latent = kv["k_cache"].view(kv["k_cache"].shape[0], ps, D)
@@ -134,7 +135,7 @@ def test_mla_decode_step_full_size():
     checked = (0, batch - 1)
     host = {b: f64(latent[btl[b]].reshape(-1, D).cpu()) for b in checked}  # before the path runs
     num_pages = latent.shape[0]
-    basis = torch.from_numpy(m_big).to(dev)
+    basis = torch.from_numpy(m_lat).to(dev)
     sc = torch.zeros((num_pages, 1, ps, 128), dtype=torch.uint8, device=dev)
     flat = latent.view(num_pages * ps, 1, D)
     for p0 in range(0, num_pages, 4096):

@@ -1,8 +1,10 @@
 """Parity of the multi-head latent attention path with the CPU oracle, through the C ABI:
-the latent scoring store (576-dim rows, basis [M_lat 0; 0 I] of 128 rows), score + top-B with one
-latent head (d 576, r 128, 64-token pages; one context past the sampling point, one ragged) and
-the absorbed latent attention over the selected rows (32 query heads padded into one 128-head
-tensor-core tile; 128 and 144 heads).
+the latent calibration (second moments of the head-mean latent queries and of the latent rows,
+then the latent basis), the latent scoring store (576-dim rows: the library takes the latent basis
+[1, 64, 512] and passes the 64 rotary dimensions through; the oracle builds the block basis
+[M_lat 0; 0 I] of 128 rows), score + top-B with one latent head (d 576, r 64, 64-token pages; one
+context past the sampling point, one ragged) and the absorbed latent attention over the selected
+rows (32 query heads padded into one 128-head tensor-core tile; 128 and 144 heads).
 Criteria are in ``parity.py``.
 """
 
@@ -37,7 +39,9 @@ class MlaCase:
         f = layer_factors(seed, 0, 1, D)
         qc, kc = sample_calibration(f, 2048, H_Q, seed)
         cal = O.calibrate(f64(qc)[..., :512], f64(kc)[..., :512], R_LAT)
-        self.m_big = O.mla_scoring_basis(cal["M"][0]).astype(np.float32)[None]  # [1, 128, 576]
+        self.m_lat = cal["M"].astype(np.float32)                                  # [1, 64, 512]
+        # the oracle's block basis of the same float32 values
+        self.m_big = O.mla_scoring_basis(self.m_lat[0]).astype(np.float32)[None]  # [1, 128, 576]
         kv = build_paged_kv(f, list(seq_lens), PS, seed, extra_pages=2)
         self.kv = kv["k_cache"]                      # [pages, 64, 1, 576]
         self.bt = kv["block_table"]
@@ -64,14 +68,14 @@ def test_mla_store_codes(case):
     sc = torch.zeros((num_pages, 1, PS, 128), dtype=torch.uint8, device="cuda")
     flat = case.kv.cuda().view(num_pages * PS, 1, D)
     slots = torch.arange(num_pages * PS, dtype=torch.int64, device="cuda")
-    J.store(flat, slots, torch.from_numpy(case.m_big).cuda(), sc)
+    J.store(flat, slots, torch.from_numpy(case.m_lat).cuda(), sc)
     assert check_codes(sc.cpu().numpy(), case.ys) <= 8
 
 
 @pytest.mark.parametrize("budget", [2048, 700])
 def test_mla_score_topk(case, budget):
     J = jssa()
-    idx, count = J.score_topk(case.q.cuda(), torch.from_numpy(case.m_big).cuda(),
+    idx, count = J.score_topk(case.q.cuda(), torch.from_numpy(case.m_lat).cuda(),
                               torch.from_numpy(case.codes).cuda(), case.bt.cuda(), case.lens_t.cuda(),
                               budget)
     ref_idx, ref_count, s = O.select_step(f64(case.q), case.m_big.astype(np.float64), case.codes,
@@ -119,7 +123,7 @@ def test_mla_short_empty_and_exact_budget():
     J = jssa()
     c = MlaCase([0, 100, 512], seed=1510)
     budget = 512
-    idx, count = J.score_topk(c.q.cuda(), torch.from_numpy(c.m_big).cuda(),
+    idx, count = J.score_topk(c.q.cuda(), torch.from_numpy(c.m_lat).cuda(),
                               torch.from_numpy(c.codes).cuda(), c.bt.cuda(), c.lens_t.cuda(), budget)
     assert count.cpu().numpy().ravel().tolist() == [0, 100, 512]
     gi = idx.cpu().numpy()
@@ -133,3 +137,58 @@ def test_mla_short_empty_and_exact_budget():
                                 count.cpu().numpy(), scale)
     check_output(f64(out), ref)
     assert torch.count_nonzero(out[0]).item() == 0
+
+
+@pytest.mark.parametrize("h_q", [128, 32])
+def test_mla_calibration(h_q):
+    # the latent second moments through the library (128 heads: the mean-plane form of the Gram
+    # kernel; 32 heads: also the mean-plane form, G d = 16384) and the latent basis solved at d 512
+    J = jssa()
+    f = layer_factors(1520, 0, 1, D)
+    # (generated on the device: 128 heads of 576 dimensions are slow to mix on the host)
+    qc, kc = sample_calibration(f, 700, h_q, 1520, device="cuda")
+    res = O.calibrate(f64(qc)[..., :512], f64(kc)[..., :512], R_LAT)
+    acc = J.Calibration(1, 512)
+    acc.add_latent(qc, kc[:, 0])
+    m, lam = acc.basis(R_LAT)
+    torch.cuda.synchronize()
+    for g, rg in ((f64(acc.gram_q), res["gram_q"]), (f64(acc.gram_k), res["gram_k"])):
+        assert np.max(np.abs(g - rg)) <= 1e-5 * np.max(np.abs(rg))
+    m, lam = f64(m)[0], f64(lam)[0]
+    assert np.max(np.abs(m @ m.T - np.eye(R_LAT))) <= 1e-6
+    a_q, a_k = O.unit_trace(res["gram_q"][0]), O.unit_trace(res["gram_k"][0])
+    # the subspace of the float32 rows, as an exact projector (rounding the rows to float32 moves
+    # L_marg by up to ~1e-7 either way at d 512, which says nothing about the subspace)
+    basis64, _ = np.linalg.qr(m.T)
+    p_gpu, p_ref = basis64 @ basis64.T, O.projector(res["M"][0])
+    opt = O.l_marg(p_ref, a_q, a_k)
+    assert -1e-12 <= O.l_marg(p_gpu, a_q, a_k) - opt <= 1e-7
+    assert np.max(np.abs(lam - res["eigvals"][0])) <= 1e-5 * lam[0]
+
+
+def test_mla_wait_timeout_then_recovery(case):
+    # a wait limit of one clock cycle makes the first wait on the tensor cores run out on a correct
+    # launch: the call raises the timeout flag, waits (with the default limit) for what it issued
+    # and frees its tensor memory; with the default restored, the next call is correct and clean
+    J = jssa()
+    budget = 2048
+    ref_idx, ref_count, _ = O.select_step(f64(case.q), case.m_big.astype(np.float64), case.codes,
+                                          case.np_bt, case.lens, budget)
+    scale = 1.0 / math.sqrt(D)
+    kv = case.kv.cuda().view(case.kv.shape[0], PS, D)
+    args = (case.q.cuda(), kv, case.bt.cuda(), torch.from_numpy(ref_idx).cuda(),
+            torch.from_numpy(ref_count).cuda(), scale)
+    J.device_error(clear=True)
+    prev = J.set_wait_limit(1)
+    try:
+        J.mla_attend(*args)
+        torch.cuda.synchronize()
+    finally:
+        J.set_wait_limit(0)
+    assert prev == 2000000000
+    assert J.device_error(clear=True) & 32  # JSSA_DEVERR_TIMEOUT
+    out = J.mla_attend(*args)
+    ref = O.indexed_attend_step(f64(case.q), case.np_kv, case.np_kv[..., :512], case.np_bt, ref_idx,
+                                ref_count, scale)
+    check_output(f64(out), ref)
+    assert J.device_error(clear=True) == 0

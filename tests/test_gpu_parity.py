@@ -53,7 +53,7 @@ def _select_oracle(case, budget):
 # ------------------------------------------------------------------------------------------------
 
 
-@pytest.mark.parametrize("r", [32, 64])
+@pytest.mark.parametrize("r", [16, 32, 64])
 def test_store_codes(r):
     case = Case([2048, 300], r=r, seed=1020 + r)
     J = jssa()
@@ -125,6 +125,21 @@ def test_score_topk_rank64_and_page32():
     ref_idx, ref_count, s = _select_oracle(case, budget)
     gi, gc = idx.cpu().numpy(), count.cpu().numpy()
     for b in range(2):
+        for h in range(case.h_kv):
+            check_selection(gi[b, h], gc[b, h], ref_idx[b, h], ref_count[b, h], s[(b, h)], budget)
+
+
+@pytest.mark.parametrize("page_size,lens,budget", [(16, [20000, 3000, 511], 512), (8, [17000, 900], 256)])
+def test_score_topk_rank16(page_size, lens, budget):
+    # 16-byte scoring rows: two 16-token tiles per warp copy instruction, a sampled threshold past
+    # 16384 positions, a context under the budget; 8-token pages split a tile over two pages
+    case = Case(lens, r=16, page_size=page_size, seed=1042 + page_size, calib=2048)
+    J = jssa()
+    idx, count = J.score_topk(case.gpu(case.q), case.gpu_np(case.m32), case.gpu_np(case.codes),
+                              case.gpu(case.block_table), case.gpu(case.seq_lens_t), budget)
+    ref_idx, ref_count, s = _select_oracle(case, budget)
+    gi, gc = idx.cpu().numpy(), count.cpu().numpy()
+    for b in range(len(lens)):
         for h in range(case.h_kv):
             check_selection(gi[b, h], gc[b, h], ref_idx[b, h], ref_count[b, h], s[(b, h)], budget)
 
@@ -365,6 +380,33 @@ def test_decode_step_long_contexts():
     check_output(f64(out), ref["out"])
 
 
+def test_decode_step_rank16():
+    # the fused decode store and the whole step at r = 16
+    case = Case([20000, 5000, 96], r=16, seed=1075, calib=2048)
+    J = jssa()
+    budget = 512
+    lens = np.asarray(case.seq_lens)
+    rng = np.random.default_rng(9)
+    k_new = torch.from_numpy(rng.standard_normal((len(lens), case.h_kv, case.d))).to(torch.bfloat16)
+    v_new = torch.from_numpy(rng.standard_normal((len(lens), case.h_kv, case.d))).to(torch.bfloat16)
+    k_cache, v_cache = case.gpu(case.k_cache).clone(), case.gpu(case.v_cache).clone()
+    sc = case.gpu_np(case.codes).clone()
+    scale = 1.0 / math.sqrt(case.d)
+    out, idx, count = J.decode(case.gpu(case.q), k_new.cuda(), v_new.cuda(), k_cache, v_cache, sc,
+                               case.gpu_np(case.m32), case.gpu(case.block_table),
+                               case.gpu(case.seq_lens_t), budget, scale)
+    ref = O.decode_step(case.np_q, f64(k_new), f64(v_new), case.np_k, case.np_v, case.codes,
+                        case.np_bt, lens, case.m32.astype(np.float64), budget, scale)
+    assert np.array_equal(sc.cpu().numpy(), ref["score_cache"])
+    gi, gc = idx.cpu().numpy(), count.cpu().numpy()
+    assert np.array_equal(gc, ref["count"])
+    for b in range(len(lens)):
+        for h in range(case.h_kv):
+            check_selection(gi[b, h], gc[b, h], ref["idx"][b, h], ref["count"][b, h],
+                            ref["scores"][(b, h)], budget)
+    check_output(f64(out), ref["out"])
+
+
 def test_page_permutation_invariance_on_gpu(tiny):
     # the same logical cache under another physical page order gives identical results
     J = jssa()
@@ -426,6 +468,26 @@ def test_calibration(tiny, n):
         assert np.max(np.abs(lam[h] - res["eigvals"][h])) <= 1e-5 * lam[h, 0]
         # rows agree with the oracle's rows up to the shared sign rule
         assert np.max(np.abs(m[h] - res["M"][h])) <= 5e-3
+
+
+def test_calibration_many_heads_per_group():
+    # 32 query heads per KV head (G d = 4096): the Gram kernel forms the group mean and sums its
+    # bf16 planes instead of the G^2 head products
+    from synth import layer_factors, sample_calibration
+    J = jssa()
+    h_kv, d, g, r = 2, 128, 32, 32
+    f = layer_factors(1530, 0, h_kv, d)
+    q, k = sample_calibration(f, 1000, g, 1530)
+    res = O.calibrate(f64(q), f64(k), r)
+    got = J.calibrate(q.cuda(), k.cuda(), r, batch=700)
+    for gg, rg in ((f64(got["gram_q"]), res["gram_q"]), (f64(got["gram_k"]), res["gram_k"])):
+        assert np.max(np.abs(gg - rg)) <= 1e-5 * np.max(np.abs(rg))
+    m = f64(got["M"])
+    for h in range(h_kv):
+        a_q, a_k = O.unit_trace(res["gram_q"][h]), O.unit_trace(res["gram_k"][h])
+        opt = O.l_marg(O.projector(res["M"][h]), a_q, a_k)
+        basis64, _ = np.linalg.qr(m[h].T)  # the float32 rows' subspace as an exact projector
+        assert -1e-12 <= O.l_marg(basis64 @ basis64.T, a_q, a_k) - opt <= 1e-7
 
 
 # ------------------------------------------------------------------------------------------------

@@ -33,9 +33,11 @@ DEVERR_PAGE, DEVERR_INDEX, DEVERR_SEQLEN = 1, 2, 4
 SIGNATURES = {
     "jssa_status_string": (ctypes.c_char_p, [c_int]),
     "jssa_version": (c_int, []),
+    "jssa_set_wait_limit": (ctypes.c_longlong, [ctypes.c_longlong]),
     "jssa_workspace_size": (c_int, [c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_size_t_p]),
     "jssa_workspace_init": (c_int, [P, c_size_t, P]),
     "jssa_calibrate_accumulate": (c_int, [P, c_int64, P, c_int64, c_int, c_int, c_int, c_int, P, P, P]),
+    "jssa_mla_calibrate_accumulate": (c_int, [P, c_int64, c_int64, P, c_int64, c_int, c_int, P, P, P]),
     "jssa_compute_basis": (c_int, [P, P, c_int, c_int, c_int, P, P, P, c_size_t, P]),
     "jssa_store": (c_int, [P, c_int64, P, c_int, c_int, c_int, c_int, P, P, c_int64, c_int, P]),
     "jssa_score_topk": (c_int, [P, P, P, P, c_int, P, c_int, c_int, c_int, c_int, c_int, c_int64,

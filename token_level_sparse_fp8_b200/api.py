@@ -19,10 +19,11 @@ from ._lib import (FN_COMPUTE_BASIS, FN_DECODE, FN_DENSE_DECODE, FN_INDEXED_ATTE
                    FN_SCORE_TOPK, JSSAError, call)
 
 __all__ = [
-    "gather_kv", "staged_pages", "gather_then_attend", "mla_scoring_basis", "mla_attend",
+    "gather_kv", "staged_pages", "gather_then_attend", "mla_calibrate_accumulate", "mla_attend",
     "JSSAError", "workspace_size", "Workspace", "calibrate_accumulate", "compute_basis",
     "calibrate", "store", "score_topk", "indexed_attend", "dense_decode", "decode",
-    "device_error", "kv_strides", "default_rank", "PagedLayer",
+    "device_error", "kv_strides", "default_rank", "PagedLayer", "Calibration", "save_basis",
+    "load_basis", "set_wait_limit",
 ]
 
 
@@ -116,6 +117,23 @@ def calibrate_accumulate(q: torch.Tensor, k: torch.Tensor, gram_q: torch.Tensor,
          h_kv, d, gram_q.data_ptr(), gram_k.data_ptr(), _stream(q.device))
 
 
+def mla_calibrate_accumulate(q: torch.Tensor, kv: torch.Tensor, gram_q: torch.Tensor,
+                             gram_k: torch.Tensor) -> None:
+    """Add the latent second moments of a batch of multi-head latent attention samples into
+    ``gram_q``/``gram_k`` (float64 ``[1, 512, 512]``): the head mean of the absorbed queries'
+    latent part (``q`` bf16 ``[n, h_q, 576]``) and the latent rows' latent part (``kv`` bf16
+    ``[n, 576]`` or ``[n, 1, 576]``)."""
+    _need(q, "q", torch.bfloat16, contiguous=False)
+    _need(kv, "kv", torch.bfloat16, contiguous=False)
+    _need(gram_q, "gram_q", torch.float64)
+    _need(gram_k, "gram_k", torch.float64)
+    n, h_q, dq = q.shape
+    if dq < 512 or q.stride(2) != 1 or kv.stride(-1) != 1 or kv.shape[-1] < 512 or kv.shape[0] != n:
+        raise ValueError("q must be [n, h_q, >= 512] and kv [n, (1,) >= 512] with contiguous rows")
+    call("jssa_mla_calibrate_accumulate", q.data_ptr(), q.stride(0), q.stride(1), kv.data_ptr(),
+         kv.stride(0), n, h_q, gram_q.data_ptr(), gram_k.data_ptr(), _stream(q.device))
+
+
 def compute_basis(gram_q: torch.Tensor, gram_k: torch.Tensor, rank: int,
                   with_eigvals: bool = True):
     """``M = TopEig_r(G_Q/tr + G_K/tr)^T`` per KV head: float32 ``[h_kv, r, d]`` (and float64
@@ -135,14 +153,101 @@ def compute_basis(gram_q: torch.Tensor, gram_k: torch.Tensor, rank: int,
 
 def calibrate(q: torch.Tensor, k: torch.Tensor, rank: int, batch: int = 8192):
     """Whole calibration over ``n`` samples, in batches of ``batch`` samples."""
-    n, h_q, d = q.shape
-    h_kv = k.shape[1]
-    gq = torch.zeros((h_kv, d, d), dtype=torch.float64, device=q.device)
-    gk = torch.zeros_like(gq)
-    for s in range(0, n, batch):
-        calibrate_accumulate(q[s:s + batch], k[s:s + batch], gq, gk)
-    basis, eig = compute_basis(gq, gk, rank)
-    return {"M": basis, "eigvals": eig, "gram_q": gq, "gram_k": gk}
+    acc = Calibration(k.shape[1], q.shape[2], q.device)
+    for s in range(0, q.shape[0], batch):
+        acc.add(q[s:s + batch], k[s:s + batch])
+    basis, eig = acc.basis(rank)
+    return {"M": basis, "eigvals": eig, "gram_q": acc.gram_q, "gram_k": acc.gram_k}
+
+
+class Calibration:
+    """Running second moments of one layer (float64 ``[h_kv, d, d]`` on the device) and the
+    number of samples they hold; ``add`` accumulates a batch, ``basis`` solves for ``M``, and
+    ``state``/``from_state`` carry the moments across processes so that a calibration can stop
+    and resume (JSSA README, section 2: second moments from calibration sequences, optionally
+    saved with the basis)."""
+
+    def __init__(self, h_kv: int, d: int, device=None, gram_q=None, gram_k=None, samples: int = 0):
+        dev = torch.device(device or "cuda")
+        self.gram_q = (torch.zeros((h_kv, d, d), dtype=torch.float64, device=dev) if gram_q is None
+                       else gram_q.to(dev, torch.float64).contiguous())
+        self.gram_k = (torch.zeros_like(self.gram_q) if gram_k is None
+                       else gram_k.to(dev, torch.float64).contiguous())
+        if self.gram_q.shape != (h_kv, d, d) or self.gram_k.shape != (h_kv, d, d):
+            raise ValueError("second moments must be [h_kv, d, d]")
+        self.samples = int(samples)
+
+    def add(self, q: torch.Tensor, k: torch.Tensor) -> None:
+        calibrate_accumulate(q, k, self.gram_q, self.gram_k)
+        self.samples += int(q.shape[0])
+
+    def add_latent(self, q: torch.Tensor, kv: torch.Tensor) -> None:
+        """A multi-head latent layer's samples (``Calibration(1, 512)``): absorbed queries
+        ``[n, h_q, 576]`` and latent rows ``[n, 576]``."""
+        mla_calibrate_accumulate(q, kv, self.gram_q, self.gram_k)
+        self.samples += int(q.shape[0])
+
+    def basis(self, rank: int, with_eigvals: bool = True):
+        return compute_basis(self.gram_q, self.gram_k, rank, with_eigvals)
+
+    def state(self) -> dict:
+        """Host copies of the moments and the sample count."""
+        return {"gram_q": self.gram_q.cpu(), "gram_k": self.gram_k.cpu(), "samples": self.samples}
+
+    @classmethod
+    def from_state(cls, state: dict, device=None) -> "Calibration":
+        gq = state["gram_q"]
+        return cls(gq.shape[0], gq.shape[1], device, gq, state["gram_k"], state.get("samples", 0))
+
+
+def save_basis(path: str, bases: dict, calibrations: Optional[dict] = None,
+               eigvals: Optional[dict] = None, rank: Optional[int] = None) -> None:
+    """Write a basis file: ``{'M': {layer: Tensor[h_kv, r, d]}}`` (the layout the pages' runtime
+    reads; a latent layer's basis is ``[1, r, kv_lora_rank]``), plus, when given, each layer's
+    second moments under ``'grams'`` (``{layer: {'gram_q', 'gram_k', 'samples'}}``, so that the
+    calibration can resume) and eigenvalues under ``'eigvals'``. JSSA README, section 2 (the
+    output file; ``--save_grams``)."""
+    out = {"M": {int(layer): m.detach().to("cpu", torch.float32).contiguous()
+                 for layer, m in bases.items()}}
+    for layer, m in out["M"].items():
+        if m.dim() != 3:
+            raise ValueError(f"basis of layer {layer} must be [h_kv, r, d]")
+        if rank is not None and m.shape[1] != rank:
+            raise ValueError(f"basis of layer {layer} has rank {m.shape[1]}, not {rank}")
+    if calibrations:
+        out["grams"] = {int(layer): (c.state() if isinstance(c, Calibration) else
+                                     {"gram_q": c["gram_q"].detach().cpu(),
+                                      "gram_k": c["gram_k"].detach().cpu(),
+                                      "samples": int(c.get("samples", 0))})
+                        for layer, c in calibrations.items()}
+    if eigvals:
+        out["eigvals"] = {int(layer): e.detach().to("cpu", torch.float64) for layer, e in eigvals.items()}
+    torch.save(out, path)
+
+
+def load_basis(path: str, device=None, rank: Optional[int] = None) -> dict:
+    """Read a basis file written by :func:`save_basis` (or any file with the same ``'M'``
+    layout). Returns ``{'M': {layer: float32 Tensor}}`` on ``device`` and, when the file has
+    them, ``'grams'`` as :class:`Calibration` objects (resume with ``add``) and ``'eigvals'``.
+    A ``rank`` that differs from a stored basis's raises (the runtime's rank must match the
+    basis: JSSA README, section 4, ``jssa_rank``)."""
+    raw = torch.load(path, map_location="cpu", weights_only=True)
+    if "M" not in raw:
+        raise ValueError(f"{path}: not a basis file (no 'M')")
+    dev = torch.device(device) if device is not None else None
+    res = {"M": {}}
+    for layer, m in raw["M"].items():
+        if m.dim() != 3:
+            raise ValueError(f"{path}: basis of layer {layer} is not [h_kv, r, d]")
+        if rank is not None and m.shape[1] != rank:
+            raise ValueError(f"{path}: basis of layer {layer} has rank {m.shape[1]}, not {rank}")
+        m = m.to(torch.float32).contiguous()
+        res["M"][int(layer)] = m.to(dev) if dev is not None else m
+    if "grams" in raw:
+        res["grams"] = {int(layer): Calibration.from_state(st, dev or "cpu") for layer, st in raw["grams"].items()}
+    if "eigvals" in raw:
+        res["eigvals"] = {int(layer): (e.to(dev) if dev is not None else e) for layer, e in raw["eigvals"].items()}
+    return res
 
 
 # ------------------------------------------------------------------------------------------------
@@ -155,14 +260,19 @@ def store(k: torch.Tensor, slot_mapping: torch.Tensor, basis: torch.Tensor,
     """Write ``e4m3(M_h k)`` of each token ``k[t]`` (bf16 ``[t, h_kv, d]``) at flat slot
     ``slot_mapping[t]`` (int64; negative = skip) of the scoring cache
     (uint8 ``[num_pages, h_kv, page_size, r]``; a bfloat16 cache of that shape holds
-    ``bf16(M_h k)`` instead, the scoring-cache ablation)."""
+    ``bf16(M_h k)`` instead, the scoring-cache ablation). A latent layer (``d`` 576, basis
+    ``[1, r, 512]``) has ``r + 64`` code columns (the rotary dimensions pass through)."""
     _need(k, "k", torch.bfloat16, contiguous=False)
     _need(slot_mapping, "slot_mapping", torch.int64)
     _need(basis, "basis", torch.float32)
     bf16 = score_cache.dtype == torch.bfloat16
     _need(score_cache, "score_cache", torch.bfloat16 if bf16 else torch.uint8)
     t, h_kv, d = k.shape
-    num_pages, _, page_size, r = score_cache.shape
+    num_pages, _, page_size, cols = score_cache.shape
+    r = basis.shape[1]
+    if cols != (r + 64 if d == 576 else r):
+        raise ValueError(f"scoring cache has {cols} code columns; rank {r} at d {d} needs "
+                         f"{r + 64 if d == 576 else r}")
     if k.stride(2) != 1 or k.stride(1) != d:
         raise ValueError("k rows must be [h_kv, d] contiguous")
     call("jssa_store_bf16" if bf16 else "jssa_store", k.data_ptr(), k.stride(0),
@@ -223,17 +333,6 @@ def indexed_attend(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
     call("jssa_indexed_attend", q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), *strides,
          block_table.data_ptr(), block_table.shape[1], idx.data_ptr(), count.data_ptr(), batch, h_q,
          h_kv, d, budget, num_pages, page_size, scale, out.data_ptr(), p, n, _stream(q.device))
-    return out
-
-
-def mla_scoring_basis(m_lat: torch.Tensor, rope_dims: int = 64) -> torch.Tensor:
-    """Rows of the latent scoring projection of multi-head latent attention: the rank-r basis of
-    the latent dimensions, then the rotary dimensions passed through (float32
-    ``[1, r + rope_dims, latent + rope_dims]`` from ``m_lat`` ``[1, r, latent]``)."""
-    _, r, lat = m_lat.shape
-    out = torch.zeros((1, r + rope_dims, lat + rope_dims), dtype=torch.float32, device=m_lat.device)
-    out[0, :r, :lat] = m_lat[0]
-    out[0, r:, lat:] = torch.eye(rope_dims, dtype=torch.float32, device=m_lat.device)
     return out
 
 
@@ -382,6 +481,12 @@ def decode(q: torch.Tensor, k_new: Optional[torch.Tensor], v_new: Optional[torch
          num_pages, page_size, budget, scale, idx.data_ptr(), count.data_ptr(), out.data_ptr(), p, n,
          _stream(q.device))
     return out, idx, count
+
+
+def set_wait_limit(cycles: int) -> int:
+    """Clock-cycle limit of the tensor-core waits in the latent attention's tile loop (a debug
+    control; <= 0 restores the default). Returns the previous limit."""
+    return int(_lib.load().jssa_set_wait_limit(int(cycles)))
 
 
 def device_error(clear: bool = True, device=None) -> int:

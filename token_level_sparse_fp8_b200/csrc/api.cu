@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -20,6 +21,16 @@ std::mutex g_cfg_mu;
 std::map<std::pair<const void*, int>, int> g_cfg_smem;  // (kernel, device) -> configured bytes
 int g_sms[64] = {0};
 }  // namespace
+
+namespace {
+constexpr long long kDefaultWaitLimit = 2000000000ll;  // ~1 s at the boost clock
+std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
+}  // namespace
+
+long long tc_wait_limit() { return g_wait_limit.load(std::memory_order_relaxed); }
+void set_tc_wait_limit(long long cycles) {
+  g_wait_limit.store(cycles > 0 ? cycles : kDefaultWaitLimit, std::memory_order_relaxed);
+}
 
 int num_sms() {
   int dev = 0;
@@ -56,13 +67,15 @@ using jssa::AttendArgs;
 constexpr int kVersion = 100;  // 0.1.0
 constexpr int64_t kMaxContext = jssa::kScoreMaxContext;
 constexpr int kMlaMaxBudget = 256 * 1024;  // selected positions per sequence, latent attention
+constexpr int kMaxCalibSamples = 256 * 65535;  // calibration samples per call (grid z of chunks)
 
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? JSSA_OK : (int)e; }
 inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 inline cudaStream_t as_stream(jssa_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
 bool supported_dr(int d, int r) {
-  return (d == 128 && (r == 32 || r == 64)) || (d == 256 && r == 64) || (d == 576 && r == 128);
+  // d 576: a multi-head latent layer, r the rank of its latent basis (r + 64 code columns)
+  return (d == 128 && (r == 16 || r == 32 || r == 64)) || (d == 256 && r == 64) || (d == 576 && r == 64);
 }
 bool supported_d(int d) { return d == 128 || d == 256; }
 
@@ -135,6 +148,12 @@ const char* jssa_status_string(int status) {
 
 int jssa_version(void) { return kVersion; }
 
+long long jssa_set_wait_limit(long long cycles) {
+  const long long prev = jssa::tc_wait_limit();
+  jssa::set_tc_wait_limit(cycles);
+  return prev;
+}
+
 int jssa_workspace_size(int fn, int batch, int h_q, int h_kv, int d, int max_pages,
                         int page_size, int budget, size_t* bytes) {
   if (!bytes) return JSSA_ERR_NULL;
@@ -185,20 +204,37 @@ int jssa_workspace_init(void* ws, size_t ws_bytes, jssa_stream_t stream) {
   return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, as_stream(stream)));
 }
 
+static int calibrate_common(const jssa_bf16* q, int64_t q_stride_n, int64_t q_stride_head,
+                            const jssa_bf16* k, int64_t k_stride_n, int n, int h_q, int h_kv,
+                            int d, double* gram_q, double* gram_k, jssa_stream_t stream) {
+  if (n < 0 || n > kMaxCalibSamples) return JSSA_ERR_SHAPE;
+  int st = check_heads(h_q, h_kv);
+  if (st) return st;
+  if (!supported_d(d) && d != 512) return JSSA_ERR_UNSUPPORTED;
+  if (n == 0) return JSSA_OK;
+  if (!q || !k || !gram_q || !gram_k) return JSSA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || (q_stride_n & 7) || (q_stride_head & 7) || (k_stride_n & 7))
+    return JSSA_ERR_ALIGN;
+  if (q_stride_head < d || q_stride_n < (int64_t)(h_q - 1) * q_stride_head + d ||
+      k_stride_n < (int64_t)h_kv * d)
+    return JSSA_ERR_SHAPE;
+  return cuda_status(jssa::launch_gram(q, q_stride_n, q_stride_head, k, k_stride_n, n, h_q, h_kv,
+                                       d, gram_q, gram_k, as_stream(stream)));
+}
+
 int jssa_calibrate_accumulate(const jssa_bf16* q, int64_t q_stride_n, const jssa_bf16* k,
                               int64_t k_stride_n, int n, int h_q, int h_kv, int d,
                               double* gram_q, double* gram_k, jssa_stream_t stream) {
-  if (n < 0) return JSSA_ERR_SHAPE;
-  int st = check_heads(h_q, h_kv);
-  if (st) return st;
-  if (!supported_d(d)) return JSSA_ERR_UNSUPPORTED;
-  if (h_q / h_kv > 16 || (h_q / h_kv) * d > 2048) return JSSA_ERR_UNSUPPORTED;
-  if (n == 0) return JSSA_OK;
-  if (!q || !k || !gram_q || !gram_k) return JSSA_ERR_NULL;
-  if (!aligned16(q) || !aligned16(k) || (q_stride_n & 7) || (k_stride_n & 7)) return JSSA_ERR_ALIGN;
-  if (q_stride_n < (int64_t)h_q * d || k_stride_n < (int64_t)h_kv * d) return JSSA_ERR_SHAPE;
-  return cuda_status(jssa::launch_gram(q, q_stride_n, k, k_stride_n, n, h_q, h_kv, d, gram_q,
-                                       gram_k, as_stream(stream)));
+  return calibrate_common(q, q_stride_n, d, k, k_stride_n, n, h_q, h_kv, d, gram_q, gram_k,
+                          stream);
+}
+
+int jssa_mla_calibrate_accumulate(const jssa_bf16* q, int64_t q_stride_n, int64_t q_stride_head,
+                                  const jssa_bf16* kv, int64_t kv_stride_n, int n, int h_q,
+                                  double* gram_q, double* gram_k, jssa_stream_t stream) {
+  // the latent part (first 512 dimensions) of each head's absorbed query and of each latent row
+  return calibrate_common(q, q_stride_n, q_stride_head, kv, kv_stride_n, n, h_q, 1, 512, gram_q,
+                          gram_k, stream);
 }
 
 int jssa_compute_basis(const double* gram_q, const double* gram_k, int h_kv, int d, int r,

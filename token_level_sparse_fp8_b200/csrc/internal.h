@@ -101,15 +101,19 @@ struct MlaPlan {
   size_t ws_bytes;
 };
 MlaPlan plan_mla(int batch, int h_q, int budget);
+// Clock-cycle limit of the tensor-core waits in a tile loop (default about one second).
+long long tc_wait_limit();
+void set_tc_wait_limit(long long cycles);  // <= 0: the default
 cudaError_t launch_mla(const uint16_t* q, const uint16_t* kv, int64_t page_stride,
                        int64_t slot_stride, const int32_t* block_table, int max_pages,
                        const int32_t* idx, const int32_t* count, int batch, int h_q, int budget,
                        int64_t num_pages, int page_size, float scale, uint16_t* out, void* ws,
                        const MlaPlan& plan, bool pdl, cudaStream_t s);
 
-cudaError_t launch_gram(const uint16_t* q, int64_t q_stride, const uint16_t* k, int64_t k_stride,
-                        int n, int h_q, int h_kv, int d, double* gram_q, double* gram_k,
-                        cudaStream_t s);
+// Second moments; q_hstride: elements between the head rows of one query sample.
+cudaError_t launch_gram(const uint16_t* q, int64_t q_stride, int64_t q_hstride, const uint16_t* k,
+                        int64_t k_stride, int n, int h_q, int h_kv, int d, double* gram_q,
+                        double* gram_k, cudaStream_t s);
 
 cudaError_t launch_basis(const double* gram_q, const double* gram_k, int h_kv, int d, int r,
                          float* basis, double* eigvals, double* ws, cudaStream_t s);

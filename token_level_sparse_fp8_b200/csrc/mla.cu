@@ -71,6 +71,7 @@ struct Args {
   float scale;
   uint16_t* out;
   void* ws;
+  long long wait_limit;  // clock cycles a wait in the tile loop may take (the drain waits longer)
 };
 
 __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int splits) {
@@ -210,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int
   bool ok = true;
   for (int i = 0; i < n_tiles; ++i) {
     if (i > 0) {  // P V of the previous tile done: its stage, S / P and O are free
-      const bool w = tc::mbar_wait(bar_o, (i - 1) & 1);
+      const bool w = tc::mbar_wait(bar_o, (i - 1) & 1, a.wait_limit);
       if (__syncthreads_or(!w)) {
         ok = false;
         break;
@@ -235,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int
       tc::mma_commit(bar_s);
     }
     {
-      const bool w = tc::mbar_wait(bar_s, i & 1);
+      const bool w = tc::mbar_wait(bar_s, i & 1, a.wait_limit);
       if (__syncthreads_or(!w)) {
         ok = false;
         break;
@@ -313,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int
     }
   }
   if (ok && n_tiles > 0) {
-    const bool w = tc::mbar_wait(bar_o, (n_tiles - 1) & 1);
+    const bool w = tc::mbar_wait(bar_o, (n_tiles - 1) & 1, a.wait_limit);
     if (__syncthreads_or(!w)) ok = false;
     tc::fence_after_sync();
   }
@@ -504,7 +505,7 @@ cudaError_t launch_mla(const uint16_t* q, const uint16_t* kv, int64_t page_strid
   cudaError_t e = configure_kernel((const void*)mla_kernel, kSmem, false);
   if (e != cudaSuccess) return e;
   Args a = {q, kv, page_stride, slot_stride, block_table, max_pages, idx, count, batch, h_q,
-            budget, num_pages, page_size, scale, out, ws};
+            budget, num_pages, page_size, scale, out, ws, tc_wait_limit()};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(((h_q + kM - 1) / kM) * kQuarters, plan.splits, batch);
   cfg.blockDim = dim3(kThreads, 1, 1);

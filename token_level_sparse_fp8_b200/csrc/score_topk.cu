@@ -481,7 +481,9 @@ struct DigitFrags {
 // memory by shared-window address, and from global memory (streamed, no L1 allocation).
 template <int LB>
 __device__ __forceinline__ void load_srow(uint32_t* dst, const uint8_t* src) {
-  if (LB == 8) {
+  if (LB == 4) {
+    dst[0] = *reinterpret_cast<const uint32_t*>(src);
+  } else if (LB == 8) {
     const uint2 v = *reinterpret_cast<const uint2*>(src);
     dst[0] = v.x;
     dst[1] = v.y;
@@ -499,7 +501,9 @@ __device__ __forceinline__ void load_srow(uint32_t* dst, const uint8_t* src) {
 
 template <int LB>
 __device__ __forceinline__ void lds_row(uint32_t* dst, uint32_t saddr) {
-  if (LB == 8) {
+  if (LB == 4) {
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(dst[0]) : "r"(saddr) : "memory");
+  } else if (LB == 8) {
     asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
                  : "=r"(dst[0]), "=r"(dst[1])
                  : "r"(saddr)
@@ -517,7 +521,9 @@ __device__ __forceinline__ void lds_row(uint32_t* dst, uint32_t saddr) {
 
 template <int LB>
 __device__ __forceinline__ void load_row(uint32_t* dst, const uint8_t* src) {
-  if (LB == 8) {
+  if (LB == 4) {
+    dst[0] = __ldcs(reinterpret_cast<const unsigned int*>(src));
+  } else if (LB == 8) {
     const uint2 v = ld_stream_v2(src);
     dst[0] = v.x;
     dst[1] = v.y;
@@ -715,14 +721,15 @@ __device__ __forceinline__ uint32_t scan_warp(const ChunkGeom& cg, const int32_t
 // The scan kernel's warps stream their tiles through a ring of scan_stages<C>() shared-memory
 // stages (kUnroll tiles each) filled by asynchronous 16-byte copies, all but one stage ahead of
 // the one being scored: deeper than a register double buffer without holding the rows in
-// registers. 32-byte rows: three stages and four CTAs per SM; 64-byte rows: four stages and
-// three; 128-byte rows (the latent scoring of multi-head latent attention): two stages and three.
+// registers. 16- and 32-byte rows: three stages and four CTAs per SM; 64-byte rows: four stages
+// and three; 128-byte rows (the latent scoring of multi-head latent attention): two stages and
+// three.
 template <class C>
 constexpr int scan_stage_bytes() { return ScanBuf<C>::kUnroll * 16 * C::kBytes; }
 template <class C>
-constexpr int scan_stages() { return C::kBytes == 32 ? 3 : C::kBytes == 64 ? 4 : 2; }
+constexpr int scan_stages() { return C::kBytes <= 32 ? 3 : C::kBytes == 64 ? 4 : 2; }
 template <class C>
-constexpr int scan_ctas_per_sm() { return C::kBytes == 32 ? 4 : 3; }
+constexpr int scan_ctas_per_sm() { return C::kBytes <= 32 ? 4 : 3; }
 template <class C>
 constexpr int scan_ring_bytes() { return kWarps * scan_stages<C>() * scan_stage_bytes<C>(); }
 
@@ -739,6 +746,33 @@ __device__ __forceinline__ uint32_t scan_issue(uint32_t dst, const ChunkGeom& cg
   static_assert(kU * kTileBytes == scan_stage_bytes<C>(), "stage size");
   const int pmask = (1 << cg.page_shift) - 1;
   uint32_t ok = BIG ? 0u : ~0u;
+  if constexpr (kPieces == 0) {
+    // tiles under 512 bytes (16-byte rows): a warp instruction copies 512 / kTileBytes whole
+    // tiles, piece (32 i + lane) of the stage being tile piece / (kTileBytes / 16)
+    constexpr int kPerTile = kTileBytes / 16;
+    static_assert(kPerTile > 0 && 32 % kPerTile == 0 && (kU * kPerTile) % 32 == 0, "tile pieces");
+#pragma unroll
+    for (int i = 0; i < kU * kPerTile / 32; ++i) {
+      const int piece = 32 * i + lane;
+      const int u = piece / kPerTile, o = (piece % kPerTile) * 16;
+      const int tok0 = (t0 + u) * 16;
+      const bool live = t0 + u < t_end && tok0 < cg.n_local;
+      const int tok = tok0 + o / RB;
+      const int pg = live && (BIG || tok < cg.n_local) ? s_page[(BIG ? tok0 : tok) >> cg.page_shift] : -1;
+      const uint8_t* src = cg.head_base + (size_t)(uint32_t)max(pg, 0) * cg.page_bytes +
+                           (BIG ? (tok0 & pmask) * RB + o : (tok & pmask) * RB + o % RB);
+      cp_async16(dst + u * kTileBytes + o, src, pg >= 0 ? 16 : 0);
+    }
+    if (BIG) {
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int tok0 = (t0 + u) * 16;
+        const bool live = t0 + u < t_end && tok0 < cg.n_local;
+        ok |= (uint32_t)(live && s_page[tok0 >> cg.page_shift] >= 0) << u;
+      }
+    }
+    return ok;
+  }
 #pragma unroll
   for (int u = 0; u < kU; ++u) {
     const int tok0 = (t0 + u) * 16;
@@ -960,10 +994,22 @@ template <int D>
 constexpr int q_groups() { return kThreads / (D / 8); }
 constexpr int kSampleBins = 256;          // histogram bins of the sampled scores
 
-// M_h is staged in shared memory when it takes at most 64 KB; otherwise (d 576, r 128: the
-// latent scoring of multi-head latent attention) the projection reads it from global memory.
+// Multi-head latent attention (d 576 = 512 latent + 64 rotary dimensions): the basis projects the
+// 512 latent dimensions only, [R - 64, 512], and the 64 rotary dimensions pass through as the last
+// 64 code columns (JSSA README, section 4 notes: the MLA basis is [1, r, kv_lora_rank]; section
+// 3.4 of the JSSA summary: 64 latent + 64 RoPE scoring dimensions).
+template <int D>
+constexpr bool latent_layer() { return D == 576; }
+constexpr int kRopeDims = 64;
+template <int D>
+constexpr int proj_dims() { return latent_layer<D>() ? D - kRopeDims : D; }  // dims the basis reads
 template <int D, class C>
-constexpr bool prep_m_in_smem() { return C::R * D * 4 <= 64 * 1024; }
+constexpr int proj_rows() { return latent_layer<D>() ? C::R - kRopeDims : C::R; }  // basis rows
+
+// M_h is staged in shared memory when it takes at most 64 KB; otherwise (the latent basis of
+// multi-head latent attention, 64 x 512) the projection reads it from global memory.
+template <int D, class C>
+constexpr bool prep_m_in_smem() { return proj_rows<D, C>() * proj_dims<D>() * 4 <= 64 * 1024; }
 
 // Dynamic shared memory of the prep kernel.
 template <int D, class C>
@@ -1000,7 +1046,8 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
   const int G = a.h_q / a.h_kv;
   const int page_size = 1 << a.page_shift;
   const int32_t* bt = a.block_table + (int64_t)b * a.max_pages;
-  const float* m_h = a.basis + (int64_t)h * R * D;
+  constexpr int kPD = proj_dims<D>(), kPR = proj_rows<D, C>();
+  const float* m_h = a.basis + (int64_t)h * kPR * kPD;
 
   // launched as a programmatic dependent of whatever precedes it on the stream: nothing is read
   // before that kernel has completed. The scan may be scheduled at once (it waits for this grid
@@ -1018,7 +1065,7 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
     // into L2 in 4 KB pieces first, so that those rounds wait on L2 and not on HBM
     constexpr int kPiece = 4096;
     const int q_bytes = G > kQGroups ? G * D * 2 : 0;
-    const int m_bytes = kMSmem ? 0 : R * D * 4;
+    const int m_bytes = kMSmem ? 0 : kPR * kPD * 4;
     const int q_pieces = (q_bytes + kPiece - 1) / kPiece, m_pieces = (m_bytes + kPiece - 1) / kPiece;
     const uint8_t* q_src = reinterpret_cast<const uint8_t*>(a.q + ((int64_t)b * a.h_q + (int64_t)h * G) * D);
     const uint8_t* m_src = reinterpret_cast<const uint8_t*>(m_h);
@@ -1162,11 +1209,24 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
 
   // ---- p = M_h qbar and, at decode, the new token's code e4m3(M_h k) (or bf16(M_h k)) ----------
   if (!kMSmem) {
-    // M_h from global memory: each warp owns R / kWarps output rows and reads them together,
-    // lanes striding over the dimensions (coalesced 128-byte reads, R / kWarps independent loads
-    // per step), then one warp reduction per row
-    constexpr int kRW = R / kWarps;
-    static_assert(D % 32 == 0 && R % kWarps == 0, "projection split");
+    // M_h from global memory: each warp owns kPR / kWarps output rows and reads them together,
+    // lanes striding over the projected dimensions (coalesced 128-byte reads, kPR / kWarps
+    // independent loads per step), then one warp reduction per row. A latent layer's last 64
+    // code columns are its rotary dimensions, passed through (p_j = qbar of that dimension; at
+    // decode the code is that dimension of k, rounded once).
+    constexpr int kRW = kPR / kWarps;
+    static_assert(kPD % 32 == 0 && kPR % kWarps == 0, "projection split");
+    if (latent_layer<D>() && tid < R - kPR) {
+      const int j = kPR + tid;
+      s_p[j] = s_qbar[kPD + tid];
+      if (store && st_page >= 0) {
+        const int pos = L - 1;
+        uint8_t* row = a.store.score_cache +
+            (((int64_t)st_page * a.h_kv + h) * page_size + (pos & (page_size - 1))) * RB;
+        if (C::kBF16) reinterpret_cast<uint16_t*>(row)[j] = f64_to_bf16((double)s_k[kPD + tid]);
+        else row[j] = f64_to_e4m3((double)s_k[kPD + tid]);
+      }
+    }
     float acc[kRW];
     double acc_k[kRW];
 #pragma unroll
@@ -1174,14 +1234,14 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
       acc[jj] = 0.f;
       acc_k[jj] = 0.0;
     }
-    const float* mbase = m_h + (int64_t)(warp * kRW) * D;
+    const float* mbase = m_h + (int64_t)(warp * kRW) * kPD;
 #pragma unroll 3
-    for (int e = lane; e < D; e += 32) {
+    for (int e = lane; e < kPD; e += 32) {
       const float qv = s_qbar[e];
       const double kv = store ? (double)s_k[e] : 0.0;
 #pragma unroll
       for (int jj = 0; jj < kRW; ++jj) {
-        const float mv = __ldg(mbase + jj * D + e);
+        const float mv = __ldg(mbase + jj * kPD + e);
         acc[jj] = fmaf(mv, qv, acc[jj]);
         if (store) acc_k[jj] = fma((double)mv, kv, acc_k[jj]);
       }
@@ -1246,14 +1306,15 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
     // f16(r 2^e1) for the remainder r = p 2^e0 - D0 (exact in fp32), scaled the same way; about
     // 22 significant bits of every component relative to the largest one. BF16 codes multiply
     // bf16 digits (8 significant bits each), four of them for about 24 bits.
-    float rem[R / 32];
+    constexpr int kPL = (R + 31) / 32;  // components per lane
+    float rem[kPL];
 #pragma unroll
-    for (int i = 0; i < R / 32; ++i) rem[i] = s_p[lane + 32 * i];
+    for (int i = 0; i < kPL; ++i) rem[i] = lane + 32 * i < R ? s_p[lane + 32 * i] : 0.f;
     float weight = 1.f;  // 2^-(e0 + ... + e_c): the value of one unit of the current remainder
     for (int c = 0; c < kDigits; ++c) {
       float mx = 0.f;
 #pragma unroll
-      for (int i = 0; i < R / 32; ++i) mx = fmaxf(mx, fabsf(rem[i]));
+      for (int i = 0; i < kPL; ++i) mx = fmaxf(mx, fabsf(rem[i]));
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       int ex = 0;
@@ -1261,15 +1322,16 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
       const float up = ldexpf(1.0f, ex);
       weight = ldexpf(weight, -ex);
 #pragma unroll
-      for (int i = 0; i < R / 32; ++i) {
+      for (int i = 0; i < kPL; ++i) {
         const float v = rem[i] * up;
+        const bool in = lane + 32 * i < R;
         if (C::kBF16) {
           const uint16_t db = f_to_bf16(v);
-          s_dig[c * R + lane + 32 * i] = db;
+          if (in) s_dig[c * R + lane + 32 * i] = db;
           rem[i] = v - bf16_to_f(db);
         } else {
           const __half dh = __float2half_rn(v);
-          s_dig[c * R + lane + 32 * i] = __half_as_ushort(dh);
+          if (in) s_dig[c * R + lane + 32 * i] = __half_as_ushort(dh);
           rem[i] = v - __half2float(dh);
         }
       }
@@ -1952,10 +2014,12 @@ cudaError_t launch_score_topk(const uint16_t* q, const float* basis, const uint8
       return launch_t<128, Codes<32, true>>(plan, pairs, pa, sa, sel, st, pdl, s);
     return cudaErrorInvalidValue;
   }
+  if (d == 128 && r == 16) return launch_t<128, Codes<16, false>>(plan, pairs, pa, sa, sel, st, pdl, s);
   if (d == 128 && r == 32) return launch_t<128, Codes<32, false>>(plan, pairs, pa, sa, sel, st, pdl, s);
   if (d == 128 && r == 64) return launch_t<128, Codes<64, false>>(plan, pairs, pa, sa, sel, st, pdl, s);
   if (d == 256 && r == 64) return launch_t<256, Codes<64, false>>(plan, pairs, pa, sa, sel, st, pdl, s);
-  if (d == 576 && r == 128) return launch_t<576, Codes<128, false>>(plan, pairs, pa, sa, sel, st, pdl, s);
+  // multi-head latent attention: basis rank r over the 512 latent dimensions, r + 64 code columns
+  if (d == 576 && r == 64) return launch_t<576, Codes<128, false>>(plan, pairs, pa, sa, sel, st, pdl, s);
   return cudaErrorInvalidValue;
 }
 

@@ -3,12 +3,17 @@
 //
 // BF16 = true stores bf16(M_h k) instead (two bytes per dimension: the scoring-cache ablation).
 //
-// One CTA per (KV head, slice of basis rows, range of tokens). The slice of the head's basis rows
-// (all r rows up to r = 64; 32 rows at r = 128, where the whole basis would not fit) is staged
-// in shared memory once, widened to float64; each warp takes one token at a time, lane j
-// computes output j (and j+32, ...) of the slice as a float64 dot product over the d dimensions
-// and rounds it once. At decode the same kernel also writes the new token's K and V rows into
-// the paged cache.
+// One CTA per (KV head, slice of code columns, range of tokens). The slice of the head's basis
+// rows (all r rows up to r = 64; 32 rows for the 128 code columns of a latent row, where the
+// whole basis would not fit) is staged in shared memory once, widened to float64; each warp takes
+// one token at a time, lane j computes output j (and j+32, ...) of the slice as a float64 dot
+// product over the projected dimensions and rounds it once. At decode the same kernel also writes
+// the new token's K and V rows into the paged cache.
+//
+// Multi-head latent attention (d 576): the basis [r, 512] projects the 512 latent dimensions and
+// the 64 rotary dimensions pass through as the last 64 code columns (JSSA README, section 4
+// notes: the MLA basis is [1, r, kv_lora_rank]; JSSA summary, section 3.4: 64 latent + 64 RoPE
+// scoring dimensions); their slices stage no basis and round the key's own values.
 #include "common.cuh"
 
 namespace jssa {
@@ -31,26 +36,33 @@ __global__ void __launch_bounds__(kStoreThreads)
                  int64_t head_stride, const int32_t* __restrict__ block_table, int max_pages,
                  const int32_t* __restrict__ seq_lens) {
   constexpr int RS = store_rows_per_cta(R);
+  constexpr bool kLatent = D == 576;
+  constexpr int PD = kLatent ? D - 64 : D;  // dimensions the basis projects
+  constexpr int PR = kLatent ? R - 64 : R;  // basis rows (the projected code columns)
+  static_assert(PR % RS == 0, "slices of projected columns");
   // both operands of the float64 products are widened once, when staged: the slice of basis
   // rows per CTA and each warp's key row per token
   extern __shared__ double store_smem[];
-  double* s_m = store_smem;                        // [RS][D+1]
-  double* s_k = store_smem + RS * (D + 1);         // [warps][D]
+  double* s_m = store_smem;                        // [RS][PD+1]
+  double* s_k = store_smem + RS * (PD + 1);        // [warps][D]
   const int h = blockIdx.x / (R / RS), r0 = (blockIdx.x % (R / RS)) * RS;
+  const bool rope_slice = kLatent && r0 >= PR;     // code columns that copy rotary dimensions
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   // the slice of basis rows, 16-byte loads (several in flight per thread) into the padded layout
-  static_assert(D % 4 == 0, "basis rows in 16-byte pieces");
-  const float4* m_h = reinterpret_cast<const float4*>(basis + ((int64_t)h * R + r0) * D);
+  static_assert(PD % 4 == 0, "basis rows in 16-byte pieces");
+  if (!rope_slice) {
+    const float4* m_h = reinterpret_cast<const float4*>(basis + ((int64_t)h * PR + r0) * PD);
 #pragma unroll 6
-  for (int i = threadIdx.x; i < RS * D / 4; i += kStoreThreads) {
-    const float4 v = m_h[i];
-    double* dst = s_m + (4 * i / D) * (D + 1) + (4 * i) % D;
-    dst[0] = v.x;
-    dst[1] = v.y;
-    dst[2] = v.z;
-    dst[3] = v.w;
+    for (int i = threadIdx.x; i < RS * PD / 4; i += kStoreThreads) {
+      const float4 v = m_h[i];
+      double* dst = s_m + (4 * i / PD) * (PD + 1) + (4 * i) % PD;
+      dst[0] = v.x;
+      dst[1] = v.y;
+      dst[2] = v.z;
+      dst[3] = v.w;
+    }
   }
   __syncthreads();
 
@@ -136,12 +148,19 @@ __global__ void __launch_bounds__(kStoreThreads)
 #pragma unroll
     for (int j0 = 0; j0 < RS; j0 += 32) {
       const int j = j0 + lane;
-      const double* mrow = s_m + j * (D + 1);
+      if (RS % 32 != 0 && j >= RS) continue;  // a slice narrower than the warp (r = 16)
+      if (rope_slice) {  // a rotary dimension of the latent row, rounded once
+        const double y = kw[PD + (r0 - PR) + j];
+        if (BF16) reinterpret_cast<uint16_t*>(dst)[j] = f64_to_bf16(y);
+        else dst[j] = f64_to_e4m3(y);
+        continue;
+      }
+      const double* mrow = s_m + j * (PD + 1);
       // float64 dot product in four interleaved partial sums (short dependency chains), one
       // rounding at the end
       double acc0 = 0.0, acc1 = 0.0, acc2 = 0.0, acc3 = 0.0;
 #pragma unroll 4
-      for (int i = 0; i < D; i += 4) {
+      for (int i = 0; i < PD; i += 4) {
         acc0 = fma(mrow[i], kw[i], acc0);
         acc1 = fma(mrow[i + 1], kw[i + 1], acc1);
         acc2 = fma(mrow[i + 2], kw[i + 2], acc2);
@@ -183,11 +202,14 @@ cudaError_t dispatch_store(int d, int r, int t, int h_kv, int tpb, cudaStream_t 
                            int64_t head_stride, const int32_t* block_table, int max_pages,
                            const int32_t* seq_lens) {
   if (t <= 0) return cudaSuccess;
-  const int rs = store_rows_per_cta(r);
-  dim3 grid(h_kv * (r / rs), (t + tpb - 1) / tpb);
-  const size_t smem = (size_t)(rs * (d + 1) + kStoreWarps * d) * sizeof(double);
+  // a latent layer (d 576, basis rank r over the 512 latent dimensions) has r + 64 code columns
+  const int cols = d == 576 ? r + 64 : r;
+  const int pd = d == 576 ? d - 64 : d;
+  const int rs = store_rows_per_cta(cols);
+  dim3 grid(h_kv * (cols / rs), (t + tpb - 1) / tpb);
+  const size_t smem = (size_t)(rs * (pd + 1) + kStoreWarps * d) * sizeof(double);
 #define JSSA_STORE_CASE(DD, RR)                                                                  \
-  if (d == DD && r == RR)                                                                        \
+  if (d == DD && cols == RR)                                                                     \
     return launch_store_t<DD, RR, DECODE, BF16>(grid, smem, s, k, k_stride_t, slot_mapping, t,   \
                                           h_kv,                                                  \
                                           basis, score_cache, num_pages, page_size, tpb, v_new,  \
@@ -197,11 +219,12 @@ cudaError_t dispatch_store(int d, int r, int t, int h_kv, int tpb, cudaStream_t 
     JSSA_STORE_CASE(128, 32)
     return cudaErrorInvalidValue;
   }
+  JSSA_STORE_CASE(128, 16)
   JSSA_STORE_CASE(128, 32)
   JSSA_STORE_CASE(128, 64)
   JSSA_STORE_CASE(256, 64)
   if (!DECODE) {
-    JSSA_STORE_CASE(576, 128)
+    JSSA_STORE_CASE(576, 128)  // latent rows: rank-64 basis + 64 rotary columns
   }
 #undef JSSA_STORE_CASE
   return cudaErrorInvalidValue;

@@ -28,13 +28,39 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Wait for the phase with the given parity to complete; false after about `limit` cycles.
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// try_wait that suspends the thread for at most about `ns` nanoseconds.
+__device__ __forceinline__ bool mbar_try_wait_ns(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+// Wait for the phase with the given parity to complete; false once more than `limit` clock cycles
+// have passed. The clock is checked between a non-blocking test and a short suspension (200 ns at
+// most), so the limit holds to within one suspension whatever the hardware's own wait window.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           long long limit = 2000000000ll) {
   const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity))
+  for (;;) {
+    if (mbar_test(bar, parity)) return true;
     if (clock64() - t0 > limit) return false;
-  return true;
+    if (mbar_try_wait_ns(bar, parity, 200u)) return true;
+  }
 }
 
 // Make this thread's generic-proxy writes to shared memory (st.shared, cp.async) visible to the
