@@ -50,6 +50,7 @@ def parse():
     ap.add_argument("--no-check", action="store_true", help="skip the oracle agreement in the CPU baseline leg")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--mla-batch", type=int, default=16, help="sequences of the mla workload")
+    ap.add_argument("--hybrid-batch", type=int, default=8, help="sequences of the hybrid workload")
     ap.add_argument("--headline-only", action="store_true",
                     help="llama128k: skip the hybrid and mla sub-measurements of the default line")
     return ap.parse_args()
@@ -863,7 +864,7 @@ def measure_hybrid(args, group, dev, local, rank, world, with_cpu=True):
     from synth import WORKLOADS, build_paged_kv, layer_factors
 
     barrier, max_over_ranks = group.barrier, group.max_over_ranks
-    w = WORKLOADS["hybrid"]
+    w = WORKLOADS["hybrid"].replace(batch=args.hybrid_batch)
     w = w.replace(seed=w.seed + 7919 * rank)
     J._lib.load()
     state = setup_gpu(w, dev)
@@ -1011,10 +1012,13 @@ def measure_mla(args, group, dev, local, rank, world, with_cpu=True):
     scale = 1.0 / math.sqrt(576.0)
     stream = torch.cuda.current_stream(dev)
 
+    kv_new = k_new.view(batch, 576)
+    ws_d = J.Workspace(dev)
+
     def step(i):
-        J.store(k_new, new_slots, m_lat, sc)
-        J.score_topk(qs[i % nq], m_lat, sc, bt, lens, B, idx, count, ws_s)
-        J.mla_attend(qs[i % nq], latent, bt, idx, count, scale, out, ws_a)
+        # one call: the new latent row and its scoring code, score + top-B, latent attention
+        J.mla_decode(qs[i % nq], kv_new, latent, sc, m_lat, bt, lens, B, scale, out, idx, count,
+                     ws_d)
 
     step(0)  # sizes the workspaces before capture
     torch.cuda.synchronize()
@@ -1039,10 +1043,10 @@ def measure_mla(args, group, dev, local, rank, world, with_cpu=True):
     if not args.no_dense:
         idx_full = torch.arange(L, dtype=torch.int32, device=dev).repeat(batch, 1).view(batch, 1, L)
         count_full = torch.full((batch, 1), L, dtype=torch.int32, device=dev)
-        ws_d = J.Workspace(dev)
+        ws_full = J.Workspace(dev)
 
         def dense(i):
-            J.mla_attend(qs[i % nq], latent, bt, idx_full, count_full, scale, out, ws_d)
+            J.mla_attend(qs[i % nq], latent, bt, idx_full, count_full, scale, out, ws_full)
 
         dense(0)
         t_dense, n_dense = timed_graph(dense, max(8, args.steps // 8), 8, stream, barrier, nq)
@@ -1098,7 +1102,7 @@ def measure_mla(args, group, dev, local, rank, world, with_cpu=True):
                             "unit": "TFLOP/s", "frac": flops_att / t_att / 1e12 / bf16_peak()[0],
                             "traffic": None, "peak_kind": bf16_peak()[1]},
         "clocks": clocks,
-        "gpu_launches": 5 * args.steps,  # store, prep, scan, select, latent attention
+        "gpu_launches": 4 * args.steps,  # prep (with the store), scan, select, latent attention
         "timing": (f"each run: exactly {args.steps} steps replayed from CUDA graphs, CUDA events; "
                    f"{st['runs']} runs, median per step"),
     }

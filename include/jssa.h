@@ -94,7 +94,8 @@ enum jssa_fn {
   JSSA_FN_DENSE_DECODE = 3,
   JSSA_FN_DECODE = 4,
   JSSA_FN_COMPUTE_BASIS = 5,
-  JSSA_FN_MLA_ATTEND = 6
+  JSSA_FN_MLA_ATTEND = 6,
+  JSSA_FN_MLA_DECODE = 7
 };
 
 /* Text for a status code (static storage). */
@@ -288,6 +289,29 @@ JSSA_API int jssa_mla_attend(const jssa_bf16* q, const jssa_bf16* kv_cache, int6
                              const int32_t* idx, const int32_t* count, int batch, int h_q,
                              int budget, int64_t num_pages, int page_size, float softmax_scale,
                              jssa_bf16* out, void* ws, size_t ws_bytes, jssa_stream_t stream);
+
+/*
+ * One whole decode step of a multi-head latent attention layer: (1) when kv_new is non-NULL,
+ * write the new token's latent row (position seq_len-1 of each sequence) into the latent cache
+ * and its scoring code (e4m3 of the latent basis applied to the 512 latent dimensions, then the 64
+ * rotary dimensions) into the scoring cache; (2) score + top-B over the latent scoring cache
+ * (jssa_score_topk with h_kv = 1, d = 576); (3) the latent attention over the selected rows
+ * (jssa_mla_attend). The kernels are chained on `stream` with programmatic dependent launch and
+ * no host synchronisation. JSSA README, paper-to-code map (JSSA on MLA) and section 4 notes; JSSA
+ * summary, sections 3.1 and 3.4.
+ * q: bf16 [batch, h_q, 576] absorbed queries (h_q a multiple of 16). kv_new: bf16 [batch, 576]
+ * or NULL. kv_cache, strides, idx, count, out: as in jssa_mla_attend. basis: float32 [1, r, 512],
+ * r = 64. score_cache: uint8 [num_pages, 1, page_size, r + 64]. ws: >=
+ * jssa_workspace_size(JSSA_FN_MLA_DECODE, batch, h_q, 1, 576, max_pages, page_size, budget); no
+ * clearing needed (the selection clears the attention's split counters).
+ */
+JSSA_API int jssa_mla_decode(const jssa_bf16* q, const jssa_bf16* kv_new, jssa_bf16* kv_cache,
+                             int64_t kv_page_stride, int64_t kv_slot_stride, uint8_t* score_cache,
+                             const float* basis, const int32_t* block_table, int max_pages,
+                             const int32_t* seq_lens, int batch, int h_q, int r, int64_t num_pages,
+                             int page_size, int budget, float softmax_scale, int32_t* idx,
+                             int32_t* count, jssa_bf16* out, void* ws, size_t ws_bytes,
+                             jssa_stream_t stream);
 
 /*
  * Gather-then-attend ablation, step 1: copy the selected K and V rows of every (sequence, KV

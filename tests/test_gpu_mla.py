@@ -192,3 +192,51 @@ def test_mla_wait_timeout_then_recovery(case):
                                 ref_count, scale)
     check_output(f64(out), ref)
     assert J.device_error(clear=True) == 0
+
+
+@pytest.mark.parametrize("budget", [2048, 512])
+def test_mla_decode_step(budget):
+    # one whole latent decode step through jssa_mla_decode: the new latent row and its scoring code
+    # are stored by the first kernel, then score + top-B and the latent attention (contexts past
+    # the sampling point, ragged, below the budget, empty)
+    J = jssa()
+    c = MlaCase([20000, 3001, 300, 0], seed=1530)
+    lens = c.lens
+    rng = np.random.default_rng(11)
+    kv_new = torch.from_numpy(rng.standard_normal((len(lens), D))).to(torch.bfloat16)
+    # the oracle's copies: the new row at position L - 1, its code from the oracle's store
+    np_kv = c.np_kv.copy()
+    codes = c.codes.copy()
+    for b, L in enumerate(lens):
+        if L == 0:
+            continue
+        page, slot = c.np_bt[b, (L - 1) // PS], (L - 1) % PS
+        np_kv[page, slot, 0] = f64(kv_new[b])
+        codes[page, 0, slot] = O.store_codes(f64(kv_new[b])[None], c.m_big[0])[0]
+    kv = c.kv.cuda().view(c.kv.shape[0], PS, D).clone()
+    sc = torch.from_numpy(c.codes).cuda().clone()
+    scale = 1.0 / math.sqrt(D)
+    out, idx, count = J.mla_decode(c.q.cuda(), kv_new.cuda(), kv, sc,
+                                   torch.from_numpy(c.m_lat).cuda(), c.bt.cuda(), c.lens_t.cuda(),
+                                   budget, scale)
+    torch.cuda.synchronize()
+    assert J.device_error() == 0
+    assert np.array_equal(f64(kv).reshape(np_kv.shape), np_kv)
+    y = np.zeros((len(lens), 128))
+    gsc = sc.cpu().numpy()
+    for b, L in enumerate(lens):
+        if L == 0:
+            continue
+        page, slot = c.np_bt[b, (L - 1) // PS], (L - 1) % PS
+        check_codes(gsc[page, 0, slot][None], (f64(kv_new[b]) @ c.m_big[0].astype(np.float64).T)[None])
+    ref_idx, ref_count, s = O.select_step(f64(c.q), c.m_big.astype(np.float64), codes, c.np_bt,
+                                          lens, budget)
+    gi, gc = idx.cpu().numpy(), count.cpu().numpy()
+    for b in range(len(lens)):
+        check_selection(gi[b, 0], gc[b, 0], ref_idx[b, 0], ref_count[b, 0], s[(b, 0)], budget)
+    ref = O.indexed_attend_step(f64(c.q), np_kv, np_kv[..., :512], c.np_bt, ref_idx, ref_count, scale)
+    check_output(f64(out), ref)
+    # a second step reuses the workspace: the selection clears the attention's split counters
+    out2, _, _ = J.mla_decode(c.q.cuda(), None, kv, sc, torch.from_numpy(c.m_lat).cuda(),
+                              c.bt.cuda(), c.lens_t.cuda(), budget, scale)
+    check_output(f64(out2), ref)

@@ -26,7 +26,7 @@ STATUS_NAMES = {
     -7: "JSSA_ERR_SCRATCH_LIMIT",
 }
 FN_SCORE_TOPK, FN_INDEXED_ATTEND, FN_DENSE_DECODE, FN_DECODE, FN_COMPUTE_BASIS = 1, 2, 3, 4, 5
-FN_MLA_ATTEND = 6
+FN_MLA_ATTEND, FN_MLA_DECODE = 6, 7
 DEVERR_PAGE, DEVERR_INDEX, DEVERR_SEQLEN = 1, 2, 4
 
 # name -> (restype, argtypes), in header order
@@ -51,6 +51,8 @@ SIGNATURES = {
                                      c_int64, c_int, c_int, P, P, P, c_size_t, P]),
     "jssa_mla_attend": (c_int, [P, P, c_int64, c_int64, P, c_int, P, P, c_int, c_int, c_int, c_int64,
                                 c_int, c_float, P, P, c_size_t, P]),
+    "jssa_mla_decode": (c_int, [P, P, P, c_int64, c_int64, P, P, P, c_int, P, c_int, c_int, c_int,
+                                c_int64, c_int, c_int, c_float, P, P, P, P, c_size_t, P]),
     "jssa_gather_kv": (c_int, [P, P, c_int64, c_int64, c_int64, P, c_int, P, P, c_int, c_int, c_int,
                                c_int, c_int64, c_int, P, P, P, P]),
     "jssa_decode": (c_int, [P, P, P, P, P, c_int64, c_int64, c_int64, P, P, P, c_int, P, c_int, c_int,

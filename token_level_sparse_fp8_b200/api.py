@@ -16,10 +16,11 @@ import torch
 
 from . import _lib
 from ._lib import (FN_COMPUTE_BASIS, FN_DECODE, FN_DENSE_DECODE, FN_INDEXED_ATTEND, FN_MLA_ATTEND,
-                   FN_SCORE_TOPK, JSSAError, call)
+                   FN_MLA_DECODE, FN_SCORE_TOPK, JSSAError, call)
 
 __all__ = [
     "gather_kv", "staged_pages", "gather_then_attend", "mla_calibrate_accumulate", "mla_attend",
+    "mla_decode",
     "JSSAError", "workspace_size", "Workspace", "calibrate_accumulate", "compute_basis",
     "calibrate", "store", "score_topk", "indexed_attend", "dense_decode", "decode",
     "device_error", "kv_strides", "default_rank", "PagedLayer", "Calibration", "save_basis",
@@ -360,6 +361,41 @@ def mla_attend(q: torch.Tensor, kv_cache: torch.Tensor, block_table: torch.Tenso
          block_table.data_ptr(), block_table.shape[1], idx.data_ptr(), count.data_ptr(), batch, h_q,
          budget, num_pages, page_size, scale, out.data_ptr(), p, n, _stream(q.device))
     return out
+
+
+def mla_decode(q: torch.Tensor, kv_new: Optional[torch.Tensor], kv_cache: torch.Tensor,
+               score_cache: torch.Tensor, basis: torch.Tensor, block_table: torch.Tensor,
+               seq_lens: torch.Tensor, budget: int, scale: float,
+               out: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
+               count: Optional[torch.Tensor] = None, ws: Optional[Workspace] = None):
+    """One decode step of a multi-head latent attention layer: store the new latent row and its
+    scoring code (when ``kv_new`` bf16 ``[batch, 576]`` is given), score + top-B over the latent
+    scoring cache, latent attention over the selected rows. Returns ``(out, idx, count)``."""
+    _need(q, "q", torch.bfloat16)
+    if kv_new is not None:
+        _need(kv_new, "kv_new", torch.bfloat16)
+    _need(kv_cache, "kv_cache", torch.bfloat16, contiguous=False)
+    for t, n, dt in ((basis, "basis", torch.float32), (score_cache, "score_cache", torch.uint8),
+                     (block_table, "block_table", torch.int32), (seq_lens, "seq_lens", torch.int32)):
+        _need(t, n, dt)
+    batch, h_q, dk = q.shape
+    num_pages, page_size, dkc = kv_cache.shape
+    if dk != 576 or dkc != 576 or kv_cache.stride(2) != 1:
+        raise ValueError("latent rows must be 576 contiguous bf16")
+    r = basis.shape[1]
+    max_pages = block_table.shape[1]
+    out = torch.empty((batch, h_q, 512), dtype=torch.bfloat16, device=q.device) if out is None else out
+    if idx is None:
+        idx = torch.empty((batch, 1, budget), dtype=torch.int32, device=q.device)
+    if count is None:
+        count = torch.empty((batch, 1), dtype=torch.int32, device=q.device)
+    w = _ws(q.device, ws, FN_MLA_DECODE)
+    p, n = w.get(workspace_size(FN_MLA_DECODE, batch, h_q, 1, 576, max_pages, page_size, budget))
+    call("jssa_mla_decode", q.data_ptr(), _ptr(kv_new), kv_cache.data_ptr(), kv_cache.stride(0),
+         kv_cache.stride(1), score_cache.data_ptr(), basis.data_ptr(), block_table.data_ptr(),
+         max_pages, seq_lens.data_ptr(), batch, h_q, r, num_pages, page_size, budget, scale,
+         idx.data_ptr(), count.data_ptr(), out.data_ptr(), p, n, _stream(q.device))
+    return out, idx, count
 
 
 def gather_kv(k_cache: torch.Tensor, v_cache: torch.Tensor, block_table: torch.Tensor,

@@ -183,10 +183,13 @@ int jssa_workspace_size(int fn, int batch, int h_q, int h_kv, int d, int max_pag
                score_ws_bytes(batch, h_kv, max_seq_len, page_size);
       return JSSA_OK;
     case JSSA_FN_MLA_ATTEND:
+    case JSSA_FN_MLA_DECODE:
       if (budget <= 0 || h_kv != 1 || d != 576 || h_q % 16) return JSSA_ERR_SHAPE;
       if (budget > kMlaMaxBudget || jssa::plan_mla(batch, h_q, budget).splits == 0)
         return JSSA_ERR_UNSUPPORTED;
       *bytes = jssa::plan_mla(batch, h_q, budget).ws_bytes;
+      if (fn == JSSA_FN_MLA_DECODE)
+        *bytes = align256(*bytes) + score_ws_bytes(batch, 1, max_seq_len, page_size);
       return JSSA_OK;
     case JSSA_FN_DENSE_DECODE: {
       const int span = (budget > 0 && budget < max_seq_len) ? budget : max_seq_len;
@@ -404,6 +407,57 @@ int jssa_dense_decode(const jssa_bf16* q, const jssa_bf16* k_cache, const jssa_b
   a.num_pages = num_pages; a.page_size = page_size; a.scale = softmax_scale; a.out = out;
   a.ws = ws;
   return cuda_status(jssa::launch_attend(a, false, plan, false, as_stream(stream)));
+}
+
+static int check_mla_kv(const jssa_bf16* q, const void* kv_cache, int64_t kv_page_stride,
+                        int64_t kv_slot_stride, const jssa_bf16* out) {
+  if (!q || !kv_cache || !out) return JSSA_ERR_NULL;
+  if (kv_page_stride <= 0 || kv_slot_stride < 576) return JSSA_ERR_SHAPE;
+  if (!aligned16(kv_cache) || !aligned16(q) || ((kv_page_stride | kv_slot_stride) & 7) ||
+      !aligned16(out))
+    return JSSA_ERR_ALIGN;
+  return JSSA_OK;
+}
+
+int jssa_mla_decode(const jssa_bf16* q, const jssa_bf16* kv_new, jssa_bf16* kv_cache,
+                    int64_t kv_page_stride, int64_t kv_slot_stride, uint8_t* score_cache,
+                    const float* basis, const int32_t* block_table, int max_pages,
+                    const int32_t* seq_lens, int batch, int h_q, int r, int64_t num_pages,
+                    int page_size, int budget, float softmax_scale, int32_t* idx, int32_t* count,
+                    jssa_bf16* out, void* ws, size_t ws_bytes, jssa_stream_t stream) {
+  int st = check_score_args(q, basis, score_cache, block_table, max_pages, seq_lens, batch, h_q, 1,
+                            576, r, num_pages, page_size, budget, idx, count);
+  if (st || batch == 0) return st;
+  if (h_q % 16 || budget > kMlaMaxBudget) return JSSA_ERR_UNSUPPORTED;
+  if ((st = check_mla_kv(q, kv_cache, kv_page_stride, kv_slot_stride, out))) return st;
+  if (kv_new && !aligned16(kv_new)) return JSSA_ERR_ALIGN;
+  const jssa::MlaPlan plan = jssa::plan_mla(batch, h_q, budget);
+  if (plan.splits == 0) return JSSA_ERR_UNSUPPORTED;
+  // workspace: [latent attention tickets + partials | score candidates]; the select kernel clears
+  // each sequence's tickets before the attention runs, so no prior clearing is needed
+  const size_t score_ws = score_ws_bytes(batch, 1, max_pages * page_size, page_size);
+  const size_t attend_bytes = align256(plan.ws_bytes);
+  if (!ws || ws_bytes < attend_bytes + score_ws) return JSSA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return JSSA_ERR_ALIGN;
+  void* attend_ws = ws;
+  void* cand_ws = static_cast<uint8_t*>(ws) + attend_bytes;
+  cudaStream_t s = as_stream(stream);
+  jssa::StoreNew sn = {};
+  if (kv_new) {
+    sn.k_new = kv_new; sn.v_new = nullptr; sn.k_cache = kv_cache; sn.v_cache = nullptr;
+    sn.page_stride = kv_page_stride; sn.slot_stride = kv_slot_stride; sn.head_stride = 0;
+    sn.score_cache = score_cache;
+  }
+  cudaError_t e = jssa::launch_score_topk(
+      q, basis, score_cache, block_table, max_pages, seq_lens, batch, h_q, 1, 576, r, num_pages,
+      page_size, budget, idx, count, cand_ws,
+      plan.ws_bytes ? static_cast<int*>(attend_ws) : nullptr, kv_new ? &sn : nullptr, true, s,
+      false, jssa::mla_tickets_per_sequence(h_q));
+  if (e != cudaSuccess) return (int)e;
+  return cuda_status(jssa::launch_mla(q, kv_cache, kv_page_stride, kv_slot_stride, block_table,
+                                      max_pages, idx, count, batch, h_q, budget, num_pages,
+                                      page_size, softmax_scale, out,
+                                      plan.ws_bytes ? attend_ws : nullptr, plan, true, s));
 }
 
 int jssa_mla_attend(const jssa_bf16* q, const jssa_bf16* kv_cache, int64_t kv_page_stride,

@@ -21,9 +21,9 @@ struct ScorePlan {
 // The new token of a decode step, stored by the score kernels' prep stage.
 struct StoreNew {
   const uint16_t* k_new;  // bf16 [batch, h_kv, d]
-  const uint16_t* v_new;  // bf16 [batch, h_kv, d]
+  const uint16_t* v_new;  // bf16 [batch, h_kv, d], or null (a latent row is its own value)
   uint16_t* k_cache;
-  uint16_t* v_cache;
+  uint16_t* v_cache;      // or null with v_new
   int64_t page_stride, slot_stride, head_stride;
   uint8_t* score_cache;
 };
@@ -61,7 +61,7 @@ cudaError_t launch_score_topk(const uint16_t* q, const float* basis, const uint8
                               int batch, int h_q, int h_kv, int d, int r, int64_t num_pages,
                               int page_size, int budget, int32_t* idx, int32_t* count,
                               void* ws, int* attend_tickets, const StoreNew* store, bool pdl,
-                              cudaStream_t s, bool bf16_codes = false);
+                              cudaStream_t s, bool bf16_codes = false, int tickets_per_pair = 1);
 
 struct AttendArgs {
   const uint16_t* q;
@@ -101,6 +101,8 @@ struct MlaPlan {
   size_t ws_bytes;
 };
 MlaPlan plan_mla(int batch, int h_q, int budget);
+// Split counters of the latent attention per sequence (head blocks x value quarters).
+int mla_tickets_per_sequence(int h_q);
 // Clock-cycle limit of the tensor-core waits in a tile loop (default about one second).
 long long tc_wait_limit();
 void set_tc_wait_limit(long long cycles);  // <= 0: the default

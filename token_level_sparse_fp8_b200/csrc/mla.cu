@@ -471,6 +471,11 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int
 
 }  // namespace mla_detail
 
+int mla_tickets_per_sequence(int h_q) {
+  using namespace mla_detail;
+  return ((h_q + kM - 1) / kM) * kQuarters;
+}
+
 MlaPlan plan_mla(int batch, int h_q, int budget) {
   using namespace mla_detail;
   MlaPlan p;

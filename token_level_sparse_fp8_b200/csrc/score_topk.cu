@@ -431,8 +431,17 @@ struct Cands {
   uint32_t* key;       // [pairs][n_chunks][kRegionsPerChunk][chunk / kRegionsPerChunk]
   int32_t* pos;        // same layout
   uint32_t* cnt;       // [pairs][n_chunks][kRegionsPerChunk]
-  int* attend_tickets; // [pairs] split-K tickets of the attention that follows, or null
+  int* attend_tickets; // [pairs][tickets_per_pair] split-K tickets of the attention that follows,
+                       // or null
+  int tickets_per_pair;
 };
+
+// The select of a pair clears the split-K tickets the attention that follows uses for it.
+__device__ __forceinline__ void clear_attend_tickets(const Cands& c, int pair) {
+  if (!c.attend_tickets) return;
+  for (int i = threadIdx.x; i < c.tickets_per_pair; i += blockDim.x)
+    c.attend_tickets[(int64_t)pair * c.tickets_per_pair + i] = 0;
+}
 
 __device__ __forceinline__ uint32_t mix32(uint32_t x) {
   x ^= x >> 16;
@@ -1093,7 +1102,7 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
     k_el[u] = v_el[u] = 0;
     if (STORE && i < D) {
       k_el[u] = a.store.k_new[((int64_t)b * a.h_kv + h) * D + i];
-      v_el[u] = a.store.v_new[((int64_t)b * a.h_kv + h) * D + i];
+      if (a.store.v_new) v_el[u] = a.store.v_new[((int64_t)b * a.h_kv + h) * D + i];
     }
   }
   for (int i = tid; i < kSampleBins; i += kThreads) sm.hist[i] = 0u;
@@ -1193,7 +1202,7 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
                              (int64_t)(pos & (page_size - 1)) * st.slot_stride +
                              (int64_t)h * st.head_stride;
         st.k_cache[base + i] = k_el[u];
-        st.v_cache[base + i] = v_el[u];
+        if (st.v_cache) st.v_cache[base + i] = v_el[u];
       }
     }
   }
@@ -1501,9 +1510,9 @@ __device__ __forceinline__ void select_finish(const SelectArgs& s, int pair, uin
   if (tid == 0) {
     if (written != want) raise_flag(8u);
     s.count[pair] = (int)want;
-    // the attention launched next merges its splits through these counters
-    if (s.scan.cands.attend_tickets) s.scan.cands.attend_tickets[pair] = 0;
   }
+  // the attention launched next merges its splits through these counters
+  clear_attend_tickets(s.scan.cands, pair);
 }
 
 // Region-major register path (at most kSelWarps * kSelRegsPerWarp regions): warp w holds
@@ -1680,10 +1689,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
   pdl_trigger();  // the attention may be scheduled; it waits for this grid to complete
   if (mode == kModeAll) {
     for (int j = tid; j < budget; j += kSelThreads) out_idx[j] = j < L ? j : -1;
-    if (tid == 0) {
-      s.count[pair] = L;
-      if (a.cands.attend_tickets) a.cands.attend_tickets[pair] = 0;
-    }
+    if (tid == 0) s.count[pair] = L;
+    clear_attend_tickets(a.cands, pair);
     return;
   }
   const int n_reg = a.n_chunks * kRegionsPerChunk;
@@ -1892,9 +1899,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs s) {
   if (tid == 0) {
     if (written != want) raise_flag(8u);
     s.count[pair] = (int)want;
-    // the attention launched next merges its splits through these counters
-    if (a.cands.attend_tickets) a.cands.attend_tickets[pair] = 0;
   }
+  // the attention launched next merges its splits through these counters
+  clear_attend_tickets(a.cands, pair);
 }
 
 template <typename Kern, typename... Args>
@@ -1921,8 +1928,9 @@ cudaError_t launch_t(const ScorePlan& plan, int pairs, const PrepArgs& pa, const
   cudaError_t e;
   const size_t prep_smem = sizeof(PrepSmem<D, C>);
   if (store) {
-    // (the fused decode store exists for the head dimensions that have decode attention)
-    if constexpr (D == 128 || D == 256) {
+    // (the fused decode store exists for the head dimensions that have decode attention: the GQA
+    // layers and the latent rows of multi-head latent attention)
+    if constexpr (D == 128 || D == 256 || D == 576) {
       e = configure_kernel((const void*)prep_kernel<D, C, true>, (int)prep_smem, false);
       if (e == cudaSuccess)
         e = launch_k(prep_kernel<D, C, true>, dim3(pairs), kThreads, prep_smem, pdl, s, pa);
@@ -1979,7 +1987,7 @@ cudaError_t launch_score_topk(const uint16_t* q, const float* basis, const uint8
                               int batch, int h_q, int h_kv, int d, int r, int64_t num_pages,
                               int page_size, int budget, int32_t* idx, int32_t* count, void* ws,
                               int* attend_tickets, const StoreNew* store, bool pdl,
-                              cudaStream_t s, bool bf16_codes) {
+                              cudaStream_t s, bool bf16_codes, int tickets_per_pair) {
   using namespace score_detail;
   const int pairs = batch * h_kv;
   if (pairs == 0) return cudaSuccess;
@@ -1995,6 +2003,7 @@ cudaError_t launch_score_topk(const uint16_t* q, const float* basis, const uint8
   cands.key = reinterpret_cast<uint32_t*>(w + (size_t)pairs * kPrepBytes + counts);
   cands.pos = reinterpret_cast<int32_t*>(w + (size_t)pairs * kPrepBytes + counts + entries * 4);
   cands.attend_tickets = attend_tickets;
+  cands.tickets_per_pair = tickets_per_pair;
 
   PrepArgs pa = {};
   pa.q = q; pa.basis = basis; pa.score_cache = score_cache;

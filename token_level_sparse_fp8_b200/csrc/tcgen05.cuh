@@ -1,5 +1,6 @@
 // 5th-generation tensor-core primitives (sm_100a): tensor-memory allocation, tcgen05.mma with
-// the A operand in tensor memory and B described in shared memory, commits to mbarriers,
+// the A operand in tensor memory or shared memory and B described in shared memory, commits to
+// mbarriers,
 // tensor-memory loads and stores, and the fences that order them with thread barriers.
 //
 // Tensor-memory addresses are (lane << 16) | column. A warp touches lanes 32 (w % 4) .. +31.
@@ -115,6 +116,17 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
       : "memory");
 }
+// D[tmem] (+)= A[smem] . B[smem]^T (both operands described in shared memory), issued by one
+// thread.
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, bool accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+      : "memory");
+}
+
 // Arrive once on the mbarrier when every MMA this thread issued before has completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
