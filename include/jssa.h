@@ -237,7 +237,9 @@ JSSA_API int jssa_indexed_attend(const jssa_bf16* q, const jssa_bf16* k_cache, c
  * Dense paged decode attention (the full-KV baseline): out[b, i] = attention of q_i over every
  * position [lo, seq_len) with lo = max(0, seq_len - window) when window > 0, else 0.
  * JSSA README, section 3 (attention microbenchmark against full-KV decode) and section 4 notes
- * (sliding-window layers keep dense attention). Same kernel body as jssa_indexed_attend.
+ * (sliding-window layers keep dense attention). Same kernel body as jssa_indexed_attend. Launched
+ * with programmatic dependent launch: it may be scheduled while the preceding kernel on `stream`
+ * finishes, and reads nothing before that kernel has completed.
  */
 JSSA_API int jssa_dense_decode(const jssa_bf16* q, const jssa_bf16* k_cache, const jssa_bf16* v_cache,
                       int64_t kv_page_stride, int64_t kv_slot_stride, int64_t kv_head_stride,

@@ -15,7 +15,11 @@ projectors; LAPACK against an independent Jacobi solver; selection against brute
 with ties; ``r = d`` without FP8 reproducing the exact group-mean logits ranking; ``r = d`` with
 ``B = L`` reproducing dense attention; dense attention against torch's CPU scaled-dot-product
 attention with grouped heads; paged against unpaged addressing; the printed 6.25% scoring-cache
-size. End-to-end output values are "parity unpinned" by the pages, which print no worked example.
+size; the sign rule of the basis rows; bf16 scores through a coordinate basis against plain dot
+products. Every function here has a pin. The pages print no worked example, so no end-to-end value
+is compared with a printed number: the whole decode step is pinned through its special cases
+(``r = d`` without FP8 gives the exact group-mean logits; ``r = d`` with ``B = L`` gives dense
+attention, itself pinned to torch's CPU SDPA) and through the pins of each step it composes.
 """
 
 from . import fp8, jssa, jacobi  # noqa: F401

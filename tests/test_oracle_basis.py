@@ -165,3 +165,20 @@ def test_planted_mistakes_are_caught(tiny_calib):
     wv2, u2 = np.linalg.eigh(g_q + g_k)
     m_raw = u2[:, ::-1][:, : w.rank].T
     assert np.max(np.abs(O.projector(m_raw) - O.projector(res["M"][h]))) > 1e-3
+
+
+def test_sign_rule_of_basis_rows():
+    # each row keeps its direction and is signed so that its largest-magnitude entry is positive,
+    # the lowest column winning a tie in magnitude
+    rng = np.random.default_rng(15)
+    m = rng.standard_normal((6, 9))
+    s = O.sign_rows(m)
+    for a, b in zip(m, s):
+        assert np.allclose(np.abs(a), np.abs(b)) and (np.allclose(a, b) or np.allclose(a, -b))
+        assert b[np.argmax(np.abs(b))] > 0
+    tie = np.array([[-2.0, 2.0, 1.0], [2.0, -2.0, 0.5], [0.0, 0.0, 0.0]])
+    out = O.sign_rows(tie)
+    assert np.array_equal(out[0], [2.0, -2.0, -1.0])   # column 0 wins the tie, was negative
+    assert np.array_equal(out[1], [2.0, -2.0, 0.5])    # column 0 wins, already positive
+    assert np.array_equal(out[2], [0.0, 0.0, 0.0])     # a zero row stays as it is
+    assert np.array_equal(O.sign_rows(out), out)        # idempotent

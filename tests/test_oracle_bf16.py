@@ -45,3 +45,20 @@ def test_float64_just_off_a_midpoint():
     assert bf16_round(up) == 1.0 + 2.0 ** -7
     assert bf16_round(down) == 1.0
     assert bf16_encode(np.array([up]))[0] == 0x3F81
+
+
+def test_bf16_scores_with_a_coordinate_basis():
+    # a basis that selects coordinates leaves bf16 keys exactly representable, so the bf16
+    # scoring cache holds the keys' own coordinates and the scores are plain dot products
+    from oracle import jssa as O
+    rng = np.random.default_rng(16)
+    d, r = 32, 8
+    k = torch.from_numpy(rng.standard_normal((50, d))).to(torch.bfloat16).double().numpy()
+    dims = rng.choice(d, size=r, replace=False)
+    m = np.zeros((r, d))
+    m[np.arange(r), dims] = 1.0
+    codes = O.store_codes_bf16(k, m)
+    assert np.array_equal(bf16_decode(codes), k[:, dims])  # the cache holds the coordinates
+    p = rng.standard_normal(r)
+    want = np.array([sum(float(k[t, dims[j]]) * p[j] for j in range(r)) for t in range(k.shape[0])])
+    assert np.allclose(O.scores_bf16(codes, p), want, rtol=1e-12, atol=1e-12)

@@ -406,7 +406,8 @@ int jssa_dense_decode(const jssa_bf16* q, const jssa_bf16* k_cache, const jssa_b
   a.window = window; a.batch = batch; a.h_q = h_q; a.h_kv = h_kv; a.d = d; a.budget = 0;
   a.num_pages = num_pages; a.page_size = page_size; a.scale = softmax_scale; a.out = out;
   a.ws = ws;
-  return cuda_status(jssa::launch_attend(a, false, plan, false, as_stream(stream)));
+  // programmatic dependent launch: the kernel waits for the preceding kernel before any read
+  return cuda_status(jssa::launch_attend(a, false, plan, true, as_stream(stream)));
 }
 
 static int check_mla_kv(const jssa_bf16* q, const void* kv_cache, int64_t kv_page_stride,

@@ -70,6 +70,10 @@ __global__ void __launch_bounds__(kThreads, Ring<D>::kCtasPerSm)
   const int G = a.h_q / a.h_kv;
   const int max_len = a.max_pages * a.page_size;
 
+  // dense mode: launched as a programmatic dependent of whatever precedes it on the stream, so
+  // nothing (queries, lengths, caches) is read before that kernel has completed; the launch itself
+  // overlaps the previous kernel's tail
+  if (!INDEXED) pdl_wait();
   // Q^T fragments (B operand of S^T = K Q^T): column n = head g of this KV head (zero for g >= G);
   // k-block kb: dims 16kb + 2t, +1 (b0) and 16kb + 8 + 2t, +1 (b1)
   uint32_t qb0[KB], qb1[KB];
