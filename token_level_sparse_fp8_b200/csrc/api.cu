@@ -458,7 +458,8 @@ int jssa_mla_decode(const jssa_bf16* q, const jssa_bf16* kv_new, jssa_bf16* kv_c
   return cuda_status(jssa::launch_mla(q, kv_cache, kv_page_stride, kv_slot_stride, block_table,
                                       max_pages, idx, count, batch, h_q, budget, num_pages,
                                       page_size, softmax_scale, out,
-                                      plan.ws_bytes ? attend_ws : nullptr, plan, true, s));
+                                      plan.ws_bytes ? attend_ws : nullptr, plan, true, s,
+                                      /*q_early=*/true));
 }
 
 int jssa_mla_attend(const jssa_bf16* q, const jssa_bf16* kv_cache, int64_t kv_page_stride,

@@ -110,7 +110,7 @@ cudaError_t launch_mla(const uint16_t* q, const uint16_t* kv, int64_t page_strid
                        int64_t slot_stride, const int32_t* block_table, int max_pages,
                        const int32_t* idx, const int32_t* count, int batch, int h_q, int budget,
                        int64_t num_pages, int page_size, float scale, uint16_t* out, void* ws,
-                       const MlaPlan& plan, bool pdl, cudaStream_t s);
+                       const MlaPlan& plan, bool pdl, cudaStream_t s, bool q_early = false);
 
 // Second moments; q_hstride: elements between the head rows of one query sample.
 cudaError_t launch_gram(const uint16_t* q, int64_t q_stride, int64_t q_hstride, const uint16_t* k,

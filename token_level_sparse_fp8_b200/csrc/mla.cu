@@ -18,7 +18,8 @@
 //   columns 288-351  S (64 tokens, fp32), then in place P = softmax weights as two bf16 parts
 //                    (high 288-319, low 320-351: P V is two MMAs and the weights keep ~16 bits)
 //   columns 384-511  O, this CTA's 128 value dimensions (fp32 accumulator)
-// Latent rows arrive by 16-byte cp.async, 64 tokens per tile, in a 2-stage ring. A tile is kept
+// Latent rows arrive by 16-byte cp.async, 64 tokens per tile, in a 3-stage ring (tile i + 1 is
+// copied into the stage of tile i - 2 while P V of tile i - 1 runs). A tile is kept
 // as 9 column blocks of 64 dimensions (128 bytes per token, 128-byte swizzle), the layout that
 // serves both as the K-major B operand of S (N = 64 tokens) and as the MN-major B operand of P V
 // (N = 128 value dimensions, K = 64 tokens), so each row is read from L2 once per CTA. One
@@ -42,7 +43,7 @@ constexpr int kQuarters = 4;         // value-dimension quarters (one per CTA)
 constexpr int kDQ = kDV / kQuarters; // 128 value dimensions per CTA
 constexpr int kThreads = 256;        // thread t <-> head t % 128 (tensor-memory lane), half t / 128
 constexpr int kTT = 64;              // tokens per tile
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kBlocks = kDK / 64;                // 9 column blocks of 64 dimensions
 constexpr int kBlockBytes = kTT * 128;           // 8 KB
 constexpr int kTileBytes = kBlocks * kBlockBytes;  // 72 KB
@@ -50,7 +51,7 @@ constexpr int kSmem = 1024 + kStages * kTileBytes;  // (+ the 1024-byte alignmen
 constexpr int kMaxChunk = 1024;                  // positions per CTA
 constexpr uint32_t kCols = 512;
 constexpr uint32_t kQCol = 0, kSCol = 288, kOCol = 384;
-constexpr int kMaxMergeSplits = kStages * kTileBytes / (kM * 4);  // 288 (merge weights)
+constexpr int kMaxMergeSplits = kStages * kTileBytes / (kM * 4);  // 432 (merge weights)
 constexpr float kRescaleSlack = 8.f;             // log2 units
 constexpr int kPRow = kDQ + 4;                   // partial row: m, l, 2 pad, o[128] (16-byte aligned)
 
@@ -72,6 +73,9 @@ struct Args {
   uint16_t* out;
   void* ws;
   long long wait_limit;  // clock cycles a wait in the tile loop may take (the drain waits longer)
+  // the queries are complete before the preceding kernel starts (the decode step's own score
+  // kernels precede this one): they are loaded while that kernel still runs
+  int q_early;
 };
 
 __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int splits) {
@@ -103,6 +107,43 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int
   if (warp == 0) {
     tc::tmem_alloc(smem_u32(&s_tmem), kCols);
     tc::tmem_relinquish();
+  }
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+  // the query row of head `row` -> its tensor-memory lane, columns [0, 288): half 0 writes the
+  // column groups 0-4, half 1 the groups 5-8 (24 independent 16-byte loads per round)
+  auto load_q = [&](uint32_t tm) {
+    const int head = hb * kM + row;
+    const bool hv = head < a.h_q;
+    const uint4* qrow = reinterpret_cast<const uint4*>(a.q + ((int64_t)b * a.h_q + (hv ? head : 0)) * kDK);
+    const int g_begin = half ? 5 : 0, g_end = half ? kDK / 64 : 5;
+#pragma unroll 1
+    for (int g0 = g_begin; g0 < g_end; g0 += 3) {
+      const int n = min(3, g_end - g0);  // (uniform over a warp)
+      uint4 x[24];
+#pragma unroll
+      for (int u = 0; u < 24; ++u)
+        x[u] = (hv && u < 8 * n) ? __ldg(qrow + g0 * 8 + u) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int g3 = 0; g3 < 3; ++g3) {
+        if (g3 >= n) break;
+        uint32_t v[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          v[4 * u] = x[8 * g3 + u].x;
+          v[4 * u + 1] = x[8 * g3 + u].y;
+          v[4 * u + 2] = x[8 * g3 + u].z;
+          v[4 * u + 3] = x[8 * g3 + u].w;
+        }
+        tc::tmem_st32(tm + lane_base + kQCol + 32 * (g0 + g3), v);
+      }
+    }
+    tc::tmem_wait_st();
+  };
+  if (a.q_early) {
+    tc::fence_before_sync();
+    __syncthreads();  // the tensor-memory base address
+    tc::fence_after_sync();
+    load_q(s_tmem);
   }
 
   pdl_wait();  // index sets come from the preceding score + top-B kernel
@@ -142,7 +183,6 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = s_tmem;
-  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
 
   // copies of a tile: 8 threads per row, thread q of a row takes the q-th 16-byte chunk of each
   // 128-byte column block (a warp instruction covers 128 contiguous bytes of each of its 4 rows)
@@ -163,42 +203,10 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int
         cp_async16(dst + blk * kBlockBytes, src + blk * 64, off >= 0 ? 16 : 0);
     }
   };
-#pragma unroll
-  for (int i = 0; i < kStages - 1; ++i) {
-    if (i < n_tiles) issue(i, i);
-    cp_async_commit();
-  }
+  if (n_tiles > 0) issue(0, 0);
+  cp_async_commit();
 
-  // the query row of head `row` -> its tensor-memory lane, columns [0, 288): half 0 writes the
-  // column groups 0-4, half 1 the groups 5-8 (24 independent 16-byte loads per round)
-  {
-    const int head = hb * kM + row;
-    const bool hv = head < a.h_q;
-    const uint4* qrow = reinterpret_cast<const uint4*>(a.q + ((int64_t)b * a.h_q + (hv ? head : 0)) * kDK);
-    const int g_begin = half ? 5 : 0, g_end = half ? kDK / 64 : 5;
-#pragma unroll 1
-    for (int g0 = g_begin; g0 < g_end; g0 += 3) {
-      const int n = min(3, g_end - g0);  // (uniform over a warp)
-      uint4 x[24];
-#pragma unroll
-      for (int u = 0; u < 24; ++u)
-        x[u] = (hv && u < 8 * n) ? __ldg(qrow + g0 * 8 + u) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-      for (int g3 = 0; g3 < 3; ++g3) {
-        if (g3 >= n) break;
-        uint32_t v[32];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          v[4 * u] = x[8 * g3 + u].x;
-          v[4 * u + 1] = x[8 * g3 + u].y;
-          v[4 * u + 2] = x[8 * g3 + u].z;
-          v[4 * u + 3] = x[8 * g3 + u].w;
-        }
-        tc::tmem_st32(tmem + lane_base + kQCol + 32 * (g0 + g3), v);
-      }
-    }
-    tc::tmem_wait_st();
-  }
+  if (!a.q_early) load_q(tmem);
   pdl_trigger();
   tc::fence_before_sync();
   __syncthreads();  // Q in tensor memory before the first MMA
@@ -210,29 +218,32 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(Args a, int chunk, int
   float m_ref = -INFINITY, l_run = 0.f;
   bool ok = true;
   for (int i = 0; i < n_tiles; ++i) {
-    if (i > 0) {  // P V of the previous tile done: its stage, S / P and O are free
-      const bool w = tc::mbar_wait(bar_o, (i - 1) & 1, a.wait_limit);
-      if (__syncthreads_or(!w)) {
-        ok = false;
-        break;
-      }
-      tc::fence_after_sync();
-    }
-    if (i + kStages - 1 < n_tiles) issue(i + kStages - 1, (i + kStages - 1) % kStages);
+    // tile i + 1 goes to the stage of tile i - 2, whose P V completed before the previous
+    // iteration's S: the copies are issued while P V of tile i - 1 still runs
+    if (i + 1 < n_tiles) issue(i + 1, (i + 1) % kStages);
     cp_async_commit();
-    cp_async_wait<kStages - 1>();
+    cp_async_wait<1>();  // tile i (all but the newest group)
     tc::fence_proxy_async_smem();
-    __syncthreads();
+    // P V of the previous tile done: S / P and O are free (and every thread's copies of tile i
+    // are in once the barrier below passes)
+    const bool w = i == 0 || tc::mbar_wait(bar_o, (i - 1) & 1, a.wait_limit);
+    if (__syncthreads_or(!w)) {
+      ok = false;
+      break;
+    }
     const uint32_t stage = ring + (i % kStages) * kTileBytes;
     if (tid == 0) {
       tc::fence_after_sync();
       // S = Q K^T: 36 steps of 16 dimensions; step kk reads 32 bytes at (kk % 4) * 32 of the
-      // 128-byte rows of column block kk / 4
-#pragma unroll 4
-      for (int kk = 0; kk < kDK / 16; ++kk) {
-        const uint64_t bd = tc::sw128_desc(stage + (kk >> 2) * kBlockBytes + (kk & 3) * 32, 16, 1024);
-        tc::mma_ts(tmem + kSCol, tmem + kQCol + kk * 8, bd, kIdescS, kk > 0);
-      }
+      // 128-byte rows of column block kk / 4. Fully unrolled, each descriptor the stage's plus a
+      // constant (the address field holds the shared-memory address / 16 and cannot carry): the
+      // issuing thread keeps up with the tensor cores
+      const uint64_t b0 = tc::sw128_desc(stage, 16, 1024);
+#pragma unroll
+      for (int kk = 0; kk < kDK / 16; ++kk)
+        tc::mma_ts(tmem + kSCol, tmem + kQCol + kk * 8,
+                   b0 + (uint64_t)(((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4), kIdescS,
+                   kk > 0);
       tc::mma_commit(bar_s);
     }
     {
@@ -503,14 +514,14 @@ cudaError_t launch_mla(const uint16_t* q, const uint16_t* kv, int64_t page_strid
                        int64_t slot_stride, const int32_t* block_table, int max_pages,
                        const int32_t* idx, const int32_t* count, int batch, int h_q, int budget,
                        int64_t num_pages, int page_size, float scale, uint16_t* out, void* ws,
-                       const MlaPlan& plan, bool pdl, cudaStream_t s) {
+                       const MlaPlan& plan, bool pdl, cudaStream_t s, bool q_early) {
   using namespace mla_detail;
   if (batch == 0) return cudaSuccess;
   static_assert(kSmem - 1024 >= kMaxMergeSplits * kM * 4, "merge buffer");
   cudaError_t e = configure_kernel((const void*)mla_kernel, kSmem, false);
   if (e != cudaSuccess) return e;
   Args a = {q, kv, page_stride, slot_stride, block_table, max_pages, idx, count, batch, h_q,
-            budget, num_pages, page_size, scale, out, ws, tc_wait_limit()};
+            budget, num_pages, page_size, scale, out, ws, tc_wait_limit(), q_early ? 1 : 0};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(((h_q + kM - 1) / kM) * kQuarters, plan.splits, batch);
   cfg.blockDim = dim3(kThreads, 1, 1);
