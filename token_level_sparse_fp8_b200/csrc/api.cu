@@ -111,9 +111,9 @@ size_t basis_ws_bytes(int h_kv, int d) {
   return n * sizeof(double);
 }
 
-size_t score_ws_bytes(int batch, int h_kv, int max_seq_len, int page_size) {
+size_t score_ws_bytes(int batch, int h_kv, int max_seq_len, int page_size, int d) {
   if (batch * h_kv == 0) return 0;
-  return jssa::plan_score(batch * h_kv, max_seq_len, page_size).ws_bytes;
+  return jssa::plan_score(batch * h_kv, max_seq_len, page_size, d).ws_bytes;
 }
 
 inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
@@ -171,7 +171,7 @@ int jssa_workspace_size(int fn, int batch, int h_q, int h_kv, int d, int max_pag
   if (st) return st;
   switch (fn) {
     case JSSA_FN_SCORE_TOPK:
-      *bytes = score_ws_bytes(batch, h_kv, max_seq_len, page_size);
+      *bytes = score_ws_bytes(batch, h_kv, max_seq_len, page_size, d);
       return JSSA_OK;
     case JSSA_FN_INDEXED_ATTEND:
       if (budget <= 0) return JSSA_ERR_SHAPE;
@@ -180,7 +180,7 @@ int jssa_workspace_size(int fn, int batch, int h_q, int h_kv, int d, int max_pag
     case JSSA_FN_DECODE:
       if (budget <= 0) return JSSA_ERR_SHAPE;
       *bytes = align256(attend_plan_indexed(batch, h_q, h_kv, d, budget).ws_bytes) +
-               score_ws_bytes(batch, h_kv, max_seq_len, page_size);
+               score_ws_bytes(batch, h_kv, max_seq_len, page_size, d);
       return JSSA_OK;
     case JSSA_FN_MLA_ATTEND:
     case JSSA_FN_MLA_DECODE:
@@ -189,7 +189,7 @@ int jssa_workspace_size(int fn, int batch, int h_q, int h_kv, int d, int max_pag
         return JSSA_ERR_UNSUPPORTED;
       *bytes = jssa::plan_mla(batch, h_q, budget).ws_bytes;
       if (fn == JSSA_FN_MLA_DECODE)
-        *bytes = align256(*bytes) + score_ws_bytes(batch, 1, max_seq_len, page_size);
+        *bytes = align256(*bytes) + score_ws_bytes(batch, 1, max_seq_len, page_size, 576);
       return JSSA_OK;
     case JSSA_FN_DENSE_DECODE: {
       const int span = (budget > 0 && budget < max_seq_len) ? budget : max_seq_len;
@@ -312,7 +312,7 @@ int jssa_score_topk(const jssa_bf16* q, const float* basis, const uint8_t* score
   int st = check_score_args(q, basis, score_cache, block_table, max_pages, seq_lens, batch, h_q,
                             h_kv, d, r, num_pages, page_size, budget, idx, count);
   if (st || batch == 0) return st;
-  const size_t need = score_ws_bytes(batch, h_kv, max_pages * page_size, page_size);
+  const size_t need = score_ws_bytes(batch, h_kv, max_pages * page_size, page_size, d);
   if (!ws || ws_bytes < need) return JSSA_ERR_WORKSPACE;
   if (!aligned16(ws)) return JSSA_ERR_ALIGN;
   return cuda_status(jssa::launch_score_topk(q, basis, score_cache, block_table, max_pages,
@@ -331,7 +331,7 @@ int jssa_score_topk_bf16(const jssa_bf16* q, const float* basis, const jssa_bf16
                             r, num_pages, page_size, budget, idx, count);
   if (st || batch == 0) return st;
   if (!(d == 128 && r == 32)) return JSSA_ERR_UNSUPPORTED;
-  const size_t need = score_ws_bytes(batch, h_kv, max_pages * page_size, page_size);
+  const size_t need = score_ws_bytes(batch, h_kv, max_pages * page_size, page_size, d);
   if (!ws || ws_bytes < need) return JSSA_ERR_WORKSPACE;
   if (!aligned16(ws)) return JSSA_ERR_ALIGN;
   return cuda_status(jssa::launch_score_topk(q, basis, sc, block_table, max_pages, seq_lens,
@@ -436,7 +436,7 @@ int jssa_mla_decode(const jssa_bf16* q, const jssa_bf16* kv_new, jssa_bf16* kv_c
   if (plan.splits == 0) return JSSA_ERR_UNSUPPORTED;
   // workspace: [latent attention tickets + partials | score candidates]; the select kernel clears
   // each sequence's tickets before the attention runs, so no prior clearing is needed
-  const size_t score_ws = score_ws_bytes(batch, 1, max_pages * page_size, page_size);
+  const size_t score_ws = score_ws_bytes(batch, 1, max_pages * page_size, page_size, 576);
   const size_t attend_bytes = align256(plan.ws_bytes);
   if (!ws || ws_bytes < attend_bytes + score_ws) return JSSA_ERR_WORKSPACE;
   if (!aligned16(ws)) return JSSA_ERR_ALIGN;
@@ -527,7 +527,7 @@ int jssa_decode(const jssa_bf16* q, const jssa_bf16* k_new, const jssa_bf16* v_n
   const jssa::AttendPlan plan = attend_plan_indexed(batch, h_q, h_kv, d, budget);
   // workspace: [attention tickets + partials | score candidates]; the score kernel clears the
   // tickets of every (sequence, KV head) before the attention runs, so no prior clearing is needed
-  const size_t score_ws = score_ws_bytes(batch, h_kv, max_pages * page_size, page_size);
+  const size_t score_ws = score_ws_bytes(batch, h_kv, max_pages * page_size, page_size, d);
   const size_t attend_bytes = align256(plan.ws_bytes);
   if (!ws || ws_bytes < attend_bytes + score_ws) return JSSA_ERR_WORKSPACE;
   if (!aligned16(ws)) return JSSA_ERR_ALIGN;

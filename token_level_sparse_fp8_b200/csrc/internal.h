@@ -40,7 +40,7 @@ int num_sms();
 // later calls are lock-protected lookups, so launches stay cheap and safe under stream capture.
 cudaError_t configure_kernel(const void* fn, int smem_bytes, bool nonportable_cluster);
 
-ScorePlan plan_score(int pairs, int max_seq_len, int page_size);
+ScorePlan plan_score(int pairs, int max_seq_len, int page_size, int d);
 AttendPlan plan_attend(int pairs, int positions, int group, int d);
 
 cudaError_t launch_store(const uint16_t* k, int64_t k_stride_t, const int64_t* slot_mapping,

@@ -1957,18 +1957,21 @@ cudaError_t launch_t(const ScorePlan& plan, int pairs, const PrepArgs& pa, const
 
 }  // namespace score_detail
 
-ScorePlan plan_score(int pairs, int max_seq_len, int page_size) {
+ScorePlan plan_score(int pairs, int max_seq_len, int page_size, int d) {
   using namespace score_detail;
   ScorePlan p;
   // positions per scan CTA: a power of two in [2048, 8192] and a multiple of the page size,
   // smaller while the grid would not cover every SM several times over, as long as a pair's
-  // candidate regions stay within what the register-resident select holds (with few pairs and
-  // long contexts the select, one CTA per pair, would otherwise cost more than the scan saves)
+  // candidate regions stay within what the select handles cheaply: the region-major register
+  // tier, or twice that for d = 128 (16- to 64-byte scoring rows, where a scan CTA is short and
+  // the flattened register tier costs less than the SMs the scan would leave idle; measured at
+  // 128K context, 1 and 4 sequences). With few pairs and long contexts the select, one CTA per
+  // pair, would otherwise cost more than the scan saves.
+  const long long region_cap = (d == 128 ? 2LL : 1LL) * kSelWarps * kSelRegsPerWarp;
   int chunk = 8192;
   while (chunk > 2048 &&
          (long long)pairs * ((max_seq_len + chunk - 1) / chunk) < 6LL * num_sms() &&
-         (long long)((max_seq_len + chunk / 2 - 1) / (chunk / 2)) * kRegionsPerChunk <=
-             kSelWarps * kSelRegsPerWarp)
+         (long long)((max_seq_len + chunk / 2 - 1) / (chunk / 2)) * kRegionsPerChunk <= region_cap)
     chunk >>= 1;
   while (chunk % page_size) chunk <<= 1;
   while ((long long)((max_seq_len + chunk - 1) / chunk) * kRegionsPerChunk > kMaxRegions) chunk <<= 1;
@@ -1991,7 +1994,7 @@ cudaError_t launch_score_topk(const uint16_t* q, const float* basis, const uint8
   using namespace score_detail;
   const int pairs = batch * h_kv;
   if (pairs == 0) return cudaSuccess;
-  const ScorePlan plan = plan_score(pairs, max_pages * page_size, page_size);
+  const ScorePlan plan = plan_score(pairs, max_pages * page_size, page_size, d);
   int shift = 0;
   while ((1 << shift) < page_size) ++shift;
   uint8_t* w = static_cast<uint8_t*>(ws);
