@@ -7,6 +7,10 @@ contexts in 16-token pages with a random page permutation, r 32, B 2048, batch 1
 low-rank keys/queries from the seeded generator; the basis is calibrated on the GPU from 32768
 seeded samples per KV head.
 
+The ``e2e`` key times the same steps fed from pinned host buffers through the C ABI
+(``jssa_decode_host``: per step the uploads of q, k_new, v_new and the download of the output,
+overlapped with the neighbouring steps' kernels).
+
 Prints one JSON line (rank 0). ``--impl reference`` times the float64 CPU oracle instead (the
 only reference that exists for this method) on a bounded sample of the same workload.
 Multi-GPU (``torchrun``): every rank runs its own batch of sequences (weak scaling, no
@@ -723,18 +727,17 @@ def run_jssa(args):
     q_host = [q.cpu().pin_memory() for q in qs]
     kn_host, vn_host = k_new.cpu().pin_memory(), v_new.cpu().pin_memory()
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    q_dev, kn_dev, vn_dev = torch.empty_like(qs[0]), torch.empty_like(k_new), torch.empty_like(v_new)
+    # the library's host-buffer decode (jssa_decode_host): a step's uploads run under the previous
+    # step's kernels and its download under the next step's; the run ends after the last download
+    pipe = J.HostPipeline(layer, qs[0].shape, k_new.shape)
 
     def e2e_step(i):
-        q_dev.copy_(q_host[i % nq], non_blocking=True)
-        kn_dev.copy_(kn_host, non_blocking=True)
-        vn_dev.copy_(vn_host, non_blocking=True)
-        layer.step(q_dev, kn_dev, vn_dev, out)
-        out_host.copy_(out, non_blocking=True)
+        pipe.step(q_host[i % nq], kn_host, vn_host, out_host)
 
     def e2e_run():
         for i in range(args.steps):
             e2e_step(i)
+        pipe.join()
 
     e2e_times, _ = repeated_runs(e2e_run, args.steps, e2e_step, args.warmup, stream, group)
     t_e2e = statistics.median(e2e_times)
@@ -781,7 +784,9 @@ def run_jssa(args):
         "e2e": {"value": whole_job_rate(world, args.steps, t_e2e), "unit": "steps/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "timing": f"median of {len(e2e_times)} runs of exactly {args.steps} steps through the "
-                          f"Python API (pinned-host H2D of q, k_new, v_new; D2H of the output)"},
+                          f"C ABI's host-buffer decode (HostPipeline -> jssa_decode_host; per step: pinned-host "
+                          f"H2D of q, k_new, v_new and D2H of the output, overlapped with the "
+                          f"neighbouring steps' kernels)"},
         "gpu_launches": launches_per_step * args.steps,
         "timing": (f"each run: exactly {args.steps} steps replayed from CUDA graphs (8 consecutive "
                    f"steps per graph, then the remainder), CUDA events on the launching stream, "

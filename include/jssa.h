@@ -95,7 +95,8 @@ enum jssa_fn {
   JSSA_FN_DECODE = 4,
   JSSA_FN_COMPUTE_BASIS = 5,
   JSSA_FN_MLA_ATTEND = 6,
-  JSSA_FN_MLA_DECODE = 7
+  JSSA_FN_MLA_DECODE = 7,
+  JSSA_FN_DECODE_HOST = 8
 };
 
 /* Text for a status code (static storage). */
@@ -353,6 +354,41 @@ JSSA_API int jssa_decode(const jssa_bf16* q, const jssa_bf16* k_new, const jssa_
                 int64_t num_pages, int page_size, int budget, float softmax_scale,
                 int32_t* idx, int32_t* count, jssa_bf16* out, void* ws, size_t ws_bytes,
                 jssa_stream_t stream);
+
+/*
+ * jssa_decode fed from host memory: copies this step's q (bf16 [batch, h_q, d]) and, when
+ * non-NULL, k_new and v_new (bf16 [batch, h_kv, d]) from host memory into device staging inside
+ * `ws`, runs jssa_decode on `stream` and copies the output back to out_host (bf16
+ * [batch, h_q, d]); the caches, basis, page table, lengths and idx / count are device memory as
+ * for jssa_decode. The library has no counterpart of this in the pages: it is the host
+ * plumbing of a serving loop. Consecutive calls on the same workspace alternate between two
+ * staging sets: the uploads of a call run on an internal stream while the previous call's
+ * kernels run, and its download on a second internal stream while the next call's kernels run
+ * (events order the three streams; use pinned host memory, or the copies are synchronous).
+ * Every call returns before its copies complete: out_host holds the step's output, and the host
+ * inputs may be rewritten, once the device has been synchronised, or once `stream` has been
+ * synchronised after jssa_decode_host_join. The first call on a workspace (per device) creates
+ * the two streams and the events, which live until the process exits; make it outside stream
+ * capture. Calls sharing one workspace must come from one thread at a time.
+ * ws: >= jssa_workspace_size(JSSA_FN_DECODE_HOST, batch, h_q, h_kv, d, max_pages, page_size,
+ * budget). Errors as jssa_decode (host pointers are not checked for alignment).
+ */
+JSSA_API int jssa_decode_host(const jssa_bf16* q_host, const jssa_bf16* k_new_host,
+                              const jssa_bf16* v_new_host, jssa_bf16* k_cache,
+                              jssa_bf16* v_cache, int64_t kv_page_stride, int64_t kv_slot_stride,
+                              int64_t kv_head_stride, uint8_t* score_cache, const float* basis,
+                              const int32_t* block_table, int max_pages, const int32_t* seq_lens,
+                              int batch, int h_q, int h_kv, int d, int r, int64_t num_pages,
+                              int page_size, int budget, float softmax_scale, int32_t* idx,
+                              int32_t* count, jssa_bf16* out_host, void* ws, size_t ws_bytes,
+                              jssa_stream_t stream);
+
+/*
+ * Make `stream` wait for every copy that jssa_decode_host has issued with this workspace (the
+ * last output included); the next jssa_decode_host call on it orders its copies after the work
+ * then on its `stream`. No-op for a workspace that has not been used by jssa_decode_host.
+ */
+JSSA_API int jssa_decode_host_join(const void* ws, jssa_stream_t stream);
 
 /* Size of the device scratch array used by jssa_indexed_attend_noalloc (per GPU, bytes). */
 #define JSSA_NOALLOC_SCRATCH_BYTES (4u << 20)

@@ -121,6 +121,19 @@ def test_argument_checks_reject_before_launch(lib):
     assert st == 0  # batch 0 is a no-op
     st = lib.jssa_compute_basis(16, 16, 2, 128, 32, 16, None, 16, 100, None)
     assert st == -5  # workspace too small
+    # host-buffer decode: NULL host buffers, a lone new K row, and a workspace without room for
+    # the two staging sets are refused before any copy or stream is created
+    args = (0x1000, 0x2000, 16 * 2 * 128, 2 * 128, 128, 0x4000, 0x5000, 0x6000, 16, 0x7000, 2, 8,
+            2, 128, 32, 10, 16, 128, ctypes.c_float(0.1), 0x8000, 0x9000)
+    st = lib.jssa_decode_host(None, None, None, *args, 0xA000, 0xB000, 1 << 30, None)
+    assert st == -1
+    st = lib.jssa_decode_host(0xC000, 0xD000, None, *args, 0xA000, 0xB000, 1 << 30, None)
+    assert st == -1
+    need = _lib_ws(lib, 8, 2, 8, 2, 128, 16, 16, 128)
+    st = lib.jssa_decode_host(0xC000, None, None, *args, 0xA000, 0xB000, need - 1, None)
+    assert st == -5
+    assert need >= _lib_ws(lib, 4, 2, 8, 2, 128, 16, 16, 128) + 2 * 2 * (2 * 8 * 128 * 2)
+    assert lib.jssa_decode_host_join(None, None) == -1
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(lib):
@@ -139,3 +152,10 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(lib):
     # a size that fits is not refused by that check (it fails later only for want of a GPU)
     small = api.workspace_size(_lib.FN_INDEXED_ATTEND, 1, 8, 2, 128, 16, 16, 256)
     assert small <= limit
+
+
+def _lib_ws(lib, fn, batch, h_q, h_kv, d, max_pages, page_size, budget):
+    n = ctypes.c_size_t(0)
+    assert lib.jssa_workspace_size(fn, batch, h_q, h_kv, d, max_pages, page_size, budget,
+                                   ctypes.byref(n)) == 0
+    return n.value

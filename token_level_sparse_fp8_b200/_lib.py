@@ -26,7 +26,7 @@ STATUS_NAMES = {
     -7: "JSSA_ERR_SCRATCH_LIMIT",
 }
 FN_SCORE_TOPK, FN_INDEXED_ATTEND, FN_DENSE_DECODE, FN_DECODE, FN_COMPUTE_BASIS = 1, 2, 3, 4, 5
-FN_MLA_ATTEND, FN_MLA_DECODE = 6, 7
+FN_MLA_ATTEND, FN_MLA_DECODE, FN_DECODE_HOST = 6, 7, 8
 DEVERR_PAGE, DEVERR_INDEX, DEVERR_SEQLEN = 1, 2, 4
 
 # name -> (restype, argtypes), in header order
@@ -58,6 +58,10 @@ SIGNATURES = {
     "jssa_decode": (c_int, [P, P, P, P, P, c_int64, c_int64, c_int64, P, P, P, c_int, P, c_int, c_int,
                             c_int, c_int, c_int, c_int64, c_int, c_int, c_float, P, P, P, P, c_size_t,
                             P]),
+    "jssa_decode_host": (c_int, [P, P, P, P, P, c_int64, c_int64, c_int64, P, P, P, c_int, P, c_int,
+                                 c_int, c_int, c_int, c_int, c_int64, c_int, c_int, c_float, P, P, P,
+                                 P, c_size_t, P]),
+    "jssa_decode_host_join": (c_int, [P, P]),
     "jssa_indexed_attend_noalloc": (c_int, [P, P, P, c_int64, c_int64, c_int64, P, c_int, P, P, c_int,
                                             c_int, c_int, c_int, c_int, c_int64, c_int, c_float, P, P]),
     "jssa_device_error": (c_int, [c_uint32_p, c_int, P]),

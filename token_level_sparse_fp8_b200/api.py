@@ -15,15 +15,16 @@ from typing import Optional, Tuple
 import torch
 
 from . import _lib
-from ._lib import (FN_COMPUTE_BASIS, FN_DECODE, FN_DENSE_DECODE, FN_INDEXED_ATTEND, FN_MLA_ATTEND,
-                   FN_MLA_DECODE, FN_SCORE_TOPK, JSSAError, call)
+from ._lib import (FN_COMPUTE_BASIS, FN_DECODE, FN_DECODE_HOST, FN_DENSE_DECODE,
+                   FN_INDEXED_ATTEND, FN_MLA_ATTEND, FN_MLA_DECODE, FN_SCORE_TOPK, JSSAError, call,
+                   check, load)
 
 __all__ = [
     "gather_kv", "staged_pages", "gather_then_attend", "mla_calibrate_accumulate", "mla_attend",
     "mla_decode",
     "JSSAError", "workspace_size", "Workspace", "calibrate_accumulate", "compute_basis",
     "calibrate", "store", "score_topk", "indexed_attend", "dense_decode", "decode",
-    "device_error", "kv_strides", "default_rank", "PagedLayer", "Calibration", "save_basis",
+    "device_error", "kv_strides", "default_rank", "PagedLayer", "HostPipeline", "Calibration", "save_basis",
     "load_basis", "set_wait_limit",
 ]
 
@@ -572,3 +573,62 @@ class PagedLayer:
     def dense(self, q, out=None, window=-1):
         return dense_decode(q, self.k_cache, self.v_cache, self.block_table, self.seq_lens,
                             self.scale, window, out, self.ws_dense)
+
+
+class HostPipeline:
+    """Decode steps of a ``PagedLayer`` fed from host memory through ``jssa_decode_host``: each
+    ``step`` copies that step's query and new K / V rows (host, pinned for overlap) to device
+    staging, runs the decode step and copies the output back to host, with the uploads of a step
+    running while the previous step computes and its download while the next one does (two
+    staging sets and two copy streams inside the library, ordered by events). Steps run on the
+    CUDA stream that is current when the pipeline is built. Calls are asynchronous: a step's
+    output is in its host buffer, and its host inputs may be rewritten, after ``synchronize``."""
+
+    def __init__(self, layer: "PagedLayer", q_shape, kv_new_shape):
+        dev = layer.k_cache.device
+        batch, h_q, d = q_shape
+        num_pages, page_size, h_kv, _ = layer.k_cache.shape
+        r = layer.basis.shape[1]
+        self.device = dev
+        self.layer = layer
+        self.ws = Workspace(dev)
+        ws_p, ws_n = self.ws.get(workspace_size(FN_DECODE_HOST, batch, h_q, h_kv, d,
+                                                layer.block_table.shape[1], page_size,
+                                                layer.budget))
+        self._stream = _stream(dev)
+        self._mid = (layer.k_cache.data_ptr(), layer.v_cache.data_ptr(), *kv_strides(layer.k_cache),
+                     layer.score_cache.data_ptr(), layer.basis.data_ptr(),
+                     layer.block_table.data_ptr(), layer.block_table.shape[1],
+                     layer.seq_lens.data_ptr(), batch, h_q, h_kv, d, r, num_pages, page_size,
+                     layer.budget, layer.scale, layer.idx.data_ptr(), layer.count.data_ptr())
+        self._tail = (ws_p, ws_n, self._stream)
+        self._ws_p = ws_p
+        self._q_shape, self._kv_shape = tuple(q_shape), tuple(kv_new_shape)
+        self._fn = load().jssa_decode_host
+
+    def _host(self, t, name, shape):
+        if not isinstance(t, torch.Tensor) or t.device.type != "cpu" or t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be a bf16 tensor in host memory")
+        if tuple(t.shape) != shape or not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous with shape {shape}")
+
+    def step(self, q_host, k_new_host, v_new_host, out_host):
+        self._host(q_host, "q_host", self._q_shape)
+        self._host(out_host, "out_host", self._q_shape)
+        if (k_new_host is None) != (v_new_host is None):
+            raise ValueError("k_new_host and v_new_host go together")
+        if k_new_host is not None:
+            self._host(k_new_host, "k_new_host", self._kv_shape)
+            self._host(v_new_host, "v_new_host", self._kv_shape)
+        check("jssa_decode_host",
+              self._fn(q_host.data_ptr(), _ptr(k_new_host), _ptr(v_new_host), *self._mid,
+                       out_host.data_ptr(), *self._tail))
+
+    def join(self):
+        """Make the pipeline's stream wait for every copy issued so far (the last output
+        included)."""
+        call("jssa_decode_host_join", self._ws_p, self._stream)
+
+    def synchronize(self):
+        self.join()
+        torch.cuda.synchronize(self.device)

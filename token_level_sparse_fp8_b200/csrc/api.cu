@@ -126,6 +126,54 @@ jssa::AttendPlan attend_plan_dense(int batch, int h_q, int h_kv, int d, int max_
   return jssa::plan_attend(batch * h_kv, max_seq_len, h_q / h_kv, d);
 }
 
+
+size_t decode_ws_bytes(int batch, int h_q, int h_kv, int d, int max_seq_len, int page_size,
+                       int budget) {
+  return align256(attend_plan_indexed(batch, h_q, h_kv, d, budget).ws_bytes) +
+         score_ws_bytes(batch, h_kv, max_seq_len, page_size, d);
+}
+
+// Device staging of one step of jssa_decode_host: q, k_new, v_new, out (each 256-byte aligned).
+size_t host_set_bytes(int batch, int h_q, int h_kv, int d) {
+  const size_t q = (size_t)batch * h_q * d * 2, kv = (size_t)batch * h_kv * d * 2;
+  return 2 * align256(q) + 2 * align256(kv);
+}
+
+// Per-workspace state of jssa_decode_host: two copy streams, the events that order the two
+// staging sets between them and the caller's stream, and which set the next call takes.
+struct HostPipe {
+  cudaStream_t up = nullptr, down = nullptr;
+  cudaEvent_t uploaded[2] = {}, decoded[2] = {}, downloaded[2] = {}, start = nullptr;
+  cudaEvent_t mark_up = nullptr, mark_down = nullptr;
+  bool used[2] = {false, false};
+  bool fresh = true;  // the next call orders the copy streams after the caller's stream
+  int next = 0;
+};
+std::mutex g_pipe_mu;
+std::map<std::pair<int, const void*>, HostPipe> g_pipes;
+
+cudaError_t host_pipe(const void* ws, bool create, HostPipe** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  auto it = g_pipes.find({dev, ws});
+  if (it != g_pipes.end()) {
+    *out = &it->second;
+    return cudaSuccess;
+  }
+  *out = nullptr;
+  if (!create) return cudaSuccess;
+  HostPipe p;
+  if ((e = cudaStreamCreateWithFlags(&p.up, cudaStreamNonBlocking)) != cudaSuccess) return e;
+  if ((e = cudaStreamCreateWithFlags(&p.down, cudaStreamNonBlocking)) != cudaSuccess) return e;
+  cudaEvent_t* evs[] = {&p.uploaded[0], &p.uploaded[1], &p.decoded[0], &p.decoded[1],
+                        &p.downloaded[0], &p.downloaded[1], &p.start, &p.mark_up, &p.mark_down};
+  for (cudaEvent_t* ev : evs)
+    if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+  *out = &(g_pipes[{dev, ws}] = p);
+  return cudaSuccess;
+}
 }  // namespace
 
 extern "C" {
@@ -179,8 +227,12 @@ int jssa_workspace_size(int fn, int batch, int h_q, int h_kv, int d, int max_pag
       return JSSA_OK;
     case JSSA_FN_DECODE:
       if (budget <= 0) return JSSA_ERR_SHAPE;
-      *bytes = align256(attend_plan_indexed(batch, h_q, h_kv, d, budget).ws_bytes) +
-               score_ws_bytes(batch, h_kv, max_seq_len, page_size, d);
+      *bytes = decode_ws_bytes(batch, h_q, h_kv, d, max_seq_len, page_size, budget);
+      return JSSA_OK;
+    case JSSA_FN_DECODE_HOST:
+      if (budget <= 0) return JSSA_ERR_SHAPE;
+      *bytes = align256(decode_ws_bytes(batch, h_q, h_kv, d, max_seq_len, page_size, budget)) +
+               2 * host_set_bytes(batch, h_q, h_kv, d);
       return JSSA_OK;
     case JSSA_FN_MLA_ATTEND:
     case JSSA_FN_MLA_DECODE:
@@ -554,6 +606,88 @@ int jssa_decode(const jssa_bf16* q, const jssa_bf16* k_new, const jssa_bf16* v_n
   a.num_pages = num_pages; a.page_size = page_size; a.scale = softmax_scale; a.out = out;
   a.ws = plan.ws_bytes ? attend_ws : nullptr;
   return cuda_status(jssa::launch_attend(a, true, plan, true, s));
+}
+
+int jssa_decode_host(const jssa_bf16* q_host, const jssa_bf16* k_new_host,
+                     const jssa_bf16* v_new_host, jssa_bf16* k_cache, jssa_bf16* v_cache,
+                     int64_t kv_page_stride, int64_t kv_slot_stride, int64_t kv_head_stride,
+                     uint8_t* score_cache, const float* basis, const int32_t* block_table,
+                     int max_pages, const int32_t* seq_lens, int batch, int h_q, int h_kv, int d,
+                     int r, int64_t num_pages, int page_size, int budget, float softmax_scale,
+                     int32_t* idx, int32_t* count, jssa_bf16* out_host, void* ws,
+                     size_t ws_bytes, jssa_stream_t stream) {
+  if (!q_host || !out_host) return JSSA_ERR_NULL;
+  if ((k_new_host == nullptr) != (v_new_host == nullptr)) return JSSA_ERR_NULL;
+  if (batch < 0 || h_q <= 0 || h_kv <= 0 || d <= 0 || max_pages < 0 || page_size <= 0 ||
+      budget <= 0)
+    return JSSA_ERR_SHAPE;
+  if (batch == 0) return JSSA_OK;
+  const int max_seq_len = max_pages * page_size;
+  const size_t dec = align256(decode_ws_bytes(batch, h_q, h_kv, d, max_seq_len, page_size, budget));
+  const size_t set = host_set_bytes(batch, h_q, h_kv, d);
+  if (!ws || ws_bytes < dec + 2 * set) return JSSA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return JSSA_ERR_ALIGN;
+  HostPipe* p = nullptr;
+  cudaError_t e = host_pipe(ws, true, &p);
+  if (e != cudaSuccess) return (int)e;
+  cudaStream_t s = as_stream(stream);
+  const size_t q_bytes = (size_t)batch * h_q * d * 2, kv_bytes = (size_t)batch * h_kv * d * 2;
+  const int k = p->next;
+  uint8_t* base = static_cast<uint8_t*>(ws) + dec + k * set;
+  jssa_bf16* q_dev = reinterpret_cast<jssa_bf16*>(base);
+  jssa_bf16* out_dev = reinterpret_cast<jssa_bf16*>(base + align256(q_bytes));
+  jssa_bf16* kn_dev = reinterpret_cast<jssa_bf16*>(base + 2 * align256(q_bytes));
+  jssa_bf16* vn_dev = reinterpret_cast<jssa_bf16*>(base + 2 * align256(q_bytes) + align256(kv_bytes));
+  if (p->fresh) {  // copies after everything already enqueued on the caller's stream
+    if ((e = cudaEventRecord(p->start, s)) != cudaSuccess) return (int)e;
+    if ((e = cudaStreamWaitEvent(p->up, p->start, 0)) != cudaSuccess) return (int)e;
+    if ((e = cudaStreamWaitEvent(p->down, p->start, 0)) != cudaSuccess) return (int)e;
+    p->fresh = false;
+  }
+  // uploads: once the step two back has read this staging set
+  if (p->used[k] && (e = cudaStreamWaitEvent(p->up, p->decoded[k], 0)) != cudaSuccess) return (int)e;
+  if ((e = cudaMemcpyAsync(q_dev, q_host, q_bytes, cudaMemcpyHostToDevice, p->up)) != cudaSuccess)
+    return (int)e;
+  if (k_new_host) {
+    if ((e = cudaMemcpyAsync(kn_dev, k_new_host, kv_bytes, cudaMemcpyHostToDevice, p->up)) != cudaSuccess)
+      return (int)e;
+    if ((e = cudaMemcpyAsync(vn_dev, v_new_host, kv_bytes, cudaMemcpyHostToDevice, p->up)) != cudaSuccess)
+      return (int)e;
+  }
+  if ((e = cudaEventRecord(p->uploaded[k], p->up)) != cudaSuccess) return (int)e;
+  // the step: after its uploads and after the download of the step two back (same output buffer)
+  if ((e = cudaStreamWaitEvent(s, p->uploaded[k], 0)) != cudaSuccess) return (int)e;
+  if (p->used[k] && (e = cudaStreamWaitEvent(s, p->downloaded[k], 0)) != cudaSuccess) return (int)e;
+  const int st = jssa_decode(q_dev, k_new_host ? kn_dev : nullptr, k_new_host ? vn_dev : nullptr,
+                             k_cache, v_cache, kv_page_stride, kv_slot_stride, kv_head_stride,
+                             score_cache, basis, block_table, max_pages, seq_lens, batch, h_q, h_kv,
+                             d, r, num_pages, page_size, budget, softmax_scale, idx, count, out_dev,
+                             ws, dec, stream);
+  if (st != JSSA_OK) return st;
+  if ((e = cudaEventRecord(p->decoded[k], s)) != cudaSuccess) return (int)e;
+  // download, overlapping the next step
+  if ((e = cudaStreamWaitEvent(p->down, p->decoded[k], 0)) != cudaSuccess) return (int)e;
+  if ((e = cudaMemcpyAsync(out_host, out_dev, q_bytes, cudaMemcpyDeviceToHost, p->down)) != cudaSuccess)
+    return (int)e;
+  if ((e = cudaEventRecord(p->downloaded[k], p->down)) != cudaSuccess) return (int)e;
+  p->used[k] = true;
+  p->next = k ^ 1;
+  return JSSA_OK;
+}
+
+int jssa_decode_host_join(const void* ws, jssa_stream_t stream) {
+  if (!ws) return JSSA_ERR_NULL;
+  HostPipe* p = nullptr;
+  cudaError_t e = host_pipe(ws, false, &p);
+  if (e != cudaSuccess) return (int)e;
+  if (!p) return JSSA_OK;  // no step issued with this workspace
+  cudaStream_t s = as_stream(stream);
+  if ((e = cudaEventRecord(p->mark_up, p->up)) != cudaSuccess) return (int)e;
+  if ((e = cudaEventRecord(p->mark_down, p->down)) != cudaSuccess) return (int)e;
+  if ((e = cudaStreamWaitEvent(s, p->mark_up, 0)) != cudaSuccess) return (int)e;
+  if ((e = cudaStreamWaitEvent(s, p->mark_down, 0)) != cudaSuccess) return (int)e;
+  p->fresh = true;
+  return JSSA_OK;
 }
 
 int jssa_device_error(uint32_t* flags, int clear, jssa_stream_t stream) {
