@@ -822,7 +822,7 @@ def run_jssa(args):
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
     if not args.headline_only:
-        for name, fn in (("hybrid", measure_hybrid), ("mla", measure_mla)):
+        for name, fn in (("hybrid", measure_hybrid), ("mla", measure_mla), ("sweep", measure_sweep)):
             sub = fn(args, group, dev, local, rank, world, with_cpu=False)
             line[name] = {k: v for k, v in sub.items()
                           if k not in ("n_gpus", "higher_is_better", "vs_baseline", "data", "warmup")}
@@ -831,6 +831,56 @@ def run_jssa(args):
     group.close()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def measure_sweep(args, group, dev, local, rank, world, with_cpu=False):
+    """The decode step at the other sizes of the metric's configurations: the 128K layer at
+    batch 1, 4, 8 and 32 (B 2048) and at batch 16 with B 1024 and 4096, and the 32K layer (batch
+    8, B 2048). Each row: runs of exactly 32 steps from CUDA graphs repeated over about 0.1 s
+    (median), the dense kernel over the same caches, the roofline fraction of the measured copy
+    bandwidth."""
+    import torch
+    import token_level_sparse_fp8_b200 as J
+    from synth import WORKLOADS
+
+    peak, peak_kind = peaks()
+    rows = []
+    cases = [("llama128k", 1, 2048), ("llama128k", 4, 2048), ("llama128k", 8, 2048),
+             ("llama128k", 32, 2048), ("llama128k", 16, 1024), ("llama128k", 16, 4096),
+             ("llama32k", 8, 2048)]
+    stream = torch.cuda.current_stream(dev)
+    for name, batch, budget in cases:
+        w = WORKLOADS[name].replace(batch=batch, budget=budget)
+        w = w.replace(seed=w.seed + 7919 * rank)
+        state = setup_gpu(w, dev)
+        layer, qs, k_new, v_new = state["layer"], state["qs"], state["k_new"], state["v_new"]
+        out = torch.empty_like(qs[0])
+        nq = len(qs)
+
+        def step(i):
+            layer.step(qs[i % nq], k_new, v_new, out)
+
+        step(0)
+        runs = ExactSteps(step, 32, nq)
+        times, _ = repeated_runs(runs, 32, step, 4, stream, group, min_region_s=0.1)
+        del runs
+        ms = step_stats(times, 32)["median"]
+        t_dense, n_dense = timed_graph(lambda i: layer.dense(qs[i % nq], out), 8, 3, stream,
+                                       group.barrier, nq)
+        t_dense = group.max_over_ranks(t_dense) / n_dense
+        gbs = algorithmic_bytes(w) / (ms / 1e3) / 1e9
+        rows.append({"workload": name, "seq_len": w.seq_len, "batch": batch, "budget": budget,
+                     "ms_per_step": ms, "steps_per_s": world / (ms / 1e3), "hbm_gbs": gbs,
+                     "frac": gbs / peak, "dense_ms_per_step": t_dense * 1e3,
+                     "speedup_vs_dense": t_dense / (ms / 1e3)})
+        del state, layer, qs, k_new, v_new, out
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return {"rows": rows, "peak": peak, "peak_kind": peak_kind,
+            "timing": "per row: runs of exactly 32 steps replayed from CUDA graphs, CUDA events, "
+                      "repeated over about 0.1 s, median per step; dense: 8-step graphs",
+            "config": {"workload": "llama3-8b layer (32/8 heads, d 128, 16-token permuted pages, "
+                                   "r 32) at 128K and 32K context, the listed batch and budget"}}
 
 
 def hybrid_bytes(w, dense=False):
