@@ -7,7 +7,9 @@
   K/V rows written in place); sampled pairs, two per KV head, are checked element by element
   against the oracle: every scoring code of the pair, the index set (tie tolerance) and the
   attention output of the pair's four query heads. At this size a pair's scan spans 16 chunks of
-  8192 positions, 128 candidate regions: the edge of the select kernel's register tier.
+  8192 positions, 128 candidate regions: the edge of the select kernel's register tier. The same
+  step at batch 1 (8 pairs, all of them sampled) takes 4096-position chunks, 256 candidate
+  regions per pair: the flattened register tier.
 * MLA: the 128-head latent layer (576-dim latent rows, 64-token pages, scoring in 64 latent +
   64 rotary dimensions, B 2048) at 128K context and batch 16: the store of every scoring row,
   score + top-B, and the absorbed latent attention; two sampled sequences against the oracle,
@@ -54,9 +56,10 @@ def _pair_rows(cache, bt_row, h, L):
     return cache[pages][:, :, h].reshape(-1, cache.shape[-1])[:L].cpu()
 
 
-def test_gqa_decode_step_full_size():
+@pytest.mark.parametrize("batch", [16, 1])
+def test_gqa_decode_step_full_size(batch):
     import token_level_sparse_fp8_b200 as J
-    w = WORKLOADS["llama128k"]              # batch 16, L 131072, B 2048: the bench's workload
+    w = WORKLOADS["llama128k"].replace(batch=batch)  # L 131072, B 2048: the bench's workload
     dev = torch.device("cuda")
     L, B, G, d, r, ps = w.seq_len, w.budget, w.group, w.d, w.rank, w.page_size
     f = layer_factors(w.seed, 0, w.h_kv, w.d)
@@ -74,7 +77,11 @@ def test_gqa_decode_step_full_size():
     # runs, with the new token placed at position L - 1 on the host
     bt = kv["block_table"].long()
     rng = np.random.default_rng(5)
-    sampled = [(int(b), h) for h in range(w.h_kv) for b in rng.choice(w.batch, size=2, replace=False)]
+    if w.batch >= 2:
+        sampled = [(int(b), h) for h in range(w.h_kv)
+                   for b in rng.choice(w.batch, size=2, replace=False)]
+    else:
+        sampled = [(0, h) for h in range(w.h_kv)]
     host = {}
     for b, h in sampled:
         k_rows, v_rows = _pair_rows(kv["k_cache"], bt[b], h, L), _pair_rows(kv["v_cache"], bt[b], h, L)
