@@ -1039,8 +1039,8 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
   constexpr int kTilesPerWarp = kS / 16 / kWarps;  // 16 (8 for 128-byte rows)
   extern __shared__ __align__(16) uint8_t prep_dyn[];
   PrepSmem<D, C>& sm = *reinterpret_cast<PrepSmem<D, C>*>(prep_dyn);
-  __shared__ float s_qbar[D];
-  __shared__ float s_k[D];
+  __shared__ __align__(16) float s_qbar[D];
+  __shared__ __align__(16) float s_k[D];
   __shared__ float s_p[R];
   __shared__ __align__(16) uint16_t s_dig[kDigits * R];  // f16 (E4M3 codes) or bf16 digits
   __shared__ float s_scale[kDigits];
@@ -1244,15 +1244,32 @@ __global__ void __launch_bounds__(kThreads, 2) prep_kernel(PrepArgs a) {
       acc_k[jj] = 0.0;
     }
     const float* mbase = m_h + (int64_t)(warp * kRW) * kPD;
-#pragma unroll 3
-    for (int e = lane; e < kPD; e += 32) {
-      const float qv = s_qbar[e];
-      const double kv = store ? (double)s_k[e] : 0.0;
+    static_assert(kPD % 128 == 0, "float4 projection");
+    // lane l takes dims 4 l .. 4 l + 3 of every 128-dim span (16-byte loads: the basis is 16-byte
+    // aligned, every row starts at a multiple of 512 bytes); two spans' loads in flight together
+#pragma unroll 1
+    for (int e = 4 * lane; e < kPD; e += 128) {
+      const float4 qv = *reinterpret_cast<const float4*>(s_qbar + e);
+      double kv[4] = {0.0, 0.0, 0.0, 0.0};
+      if (store) {
+        const float4 k4 = *reinterpret_cast<const float4*>(s_k + e);
+        kv[0] = k4.x; kv[1] = k4.y; kv[2] = k4.z; kv[3] = k4.w;
+      }
+      float4 mv[kRW];
+#pragma unroll
+      for (int jj = 0; jj < kRW; ++jj) mv[jj] = __ldg(reinterpret_cast<const float4*>(mbase + jj * kPD + e));
 #pragma unroll
       for (int jj = 0; jj < kRW; ++jj) {
-        const float mv = __ldg(mbase + jj * kPD + e);
-        acc[jj] = fmaf(mv, qv, acc[jj]);
-        if (store) acc_k[jj] = fma((double)mv, kv, acc_k[jj]);
+        acc[jj] = fmaf(mv[jj].x, qv.x, acc[jj]);
+        acc[jj] = fmaf(mv[jj].y, qv.y, acc[jj]);
+        acc[jj] = fmaf(mv[jj].z, qv.z, acc[jj]);
+        acc[jj] = fmaf(mv[jj].w, qv.w, acc[jj]);
+        if (store) {
+          acc_k[jj] = fma((double)mv[jj].x, kv[0], acc_k[jj]);
+          acc_k[jj] = fma((double)mv[jj].y, kv[1], acc_k[jj]);
+          acc_k[jj] = fma((double)mv[jj].z, kv[2], acc_k[jj]);
+          acc_k[jj] = fma((double)mv[jj].w, kv[3], acc_k[jj]);
+        }
       }
     }
 #pragma unroll
