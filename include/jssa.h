@@ -14,7 +14,8 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  * - Pointers are DEVICE pointers owned by the caller, except where stated. The library never
- *   allocates or frees memory and never synchronises a stream (jssa_device_error excepted).
+ *   allocates or frees memory and never synchronises a stream (jssa_device_error excepted);
+ *   jssa_decode_host creates two streams and a few events per workspace on its first call.
  *   Every call is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy default).
  * - bf16 tensors are passed as `const jssa_bf16*` (raw 16-bit storage).
  * - Return value: JSSA_OK (0); a negative JSSA_ERR_* code when the host-side argument check
