@@ -370,7 +370,10 @@ JSSA_API int jssa_decode(const jssa_bf16* q, const jssa_bf16* k_new, const jssa_
  * inputs may be rewritten, once the device has been synchronised, or once `stream` has been
  * synchronised after jssa_decode_host_join. The first call on a workspace (per device) creates
  * the two streams and the events, which live until the process exits; make it outside stream
- * capture. Calls sharing one workspace must come from one thread at a time.
+ * capture. Calls sharing one workspace must come from one thread at a time. The state is keyed
+ * by the workspace address: before a sequence of calls on memory that an earlier sequence used
+ * as its workspace (for instance freed and allocated again), call jssa_decode_host_join on it,
+ * which makes the next call order its copies after the work already on its stream.
  * ws: >= jssa_workspace_size(JSSA_FN_DECODE_HOST, batch, h_q, h_kv, d, max_pages, page_size,
  * budget). Errors as jssa_decode (host pointers are not checked for alignment).
  */

@@ -605,6 +605,9 @@ class HostPipeline:
         self._ws_p = ws_p
         self._q_shape, self._kv_shape = tuple(q_shape), tuple(kv_new_shape)
         self._fn = load().jssa_decode_host
+        # the library keys its copy streams by workspace address: if an earlier pipeline used this
+        # address, its next step orders its copies after the work already on the stream again
+        call("jssa_decode_host_join", ws_p, self._stream)
 
     def _host(self, t, name, shape):
         if not isinstance(t, torch.Tensor) or t.device.type != "cpu" or t.dtype != torch.bfloat16:
