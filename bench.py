@@ -55,9 +55,48 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--mla-batch", type=int, default=16, help="sequences of the mla workload")
     ap.add_argument("--hybrid-batch", type=int, default=8, help="sequences of the hybrid workload")
+    ap.add_argument("--jsonl", default=None,
+                    help="also append one JSON record per measured configuration (the headline, each "
+                         "sweep row, the hybrid stack, the MLA layer) to this file")
     ap.add_argument("--headline-only", action="store_true",
                     help="llama128k: skip the hybrid and mla sub-measurements of the default line")
     return ap.parse_args()
+
+
+def append_records(path, line):
+    """One record per measured configuration of a bench line (time, rate, algorithmic GB/s,
+    roofline fraction, the oracle agreement where the line has one), appended to `path`."""
+    if not path:
+        return
+    recs = []
+    base = {"impl": line.get("impl", "jssa"), "n_gpus": line.get("n_gpus", 1),
+            "metric": line.get("metric"), "time": time.strftime("%Y-%m-%dT%H:%M:%SZ", time.gmtime())}
+
+    def rec(name, d):
+        r = dict(base)
+        r.update({"configuration": name, "config": d.get("config"), "steps_per_s": d.get("value"),
+                  "ms_per_step": d.get("ms_per_step"), "hbm_gbs": d.get("hbm_gbs"),
+                  "roofline_frac": (d.get("roofline_step") or {}).get("frac"),
+                  "speedup_vs_dense": d.get("speedup_vs_dense")})
+        agree = (d.get("cpu_baseline") or {}).get("agreement")
+        if agree is not None:
+            r["oracle_agreement"] = agree
+        return r
+
+    recs.append(rec(line.get("config", {}).get("workload", "headline"), line))
+    for name in ("hybrid", "mla"):
+        if isinstance(line.get(name), dict):
+            recs.append(rec(name, line[name]))
+    for row in (line.get("sweep") or {}).get("rows", []):
+        r = dict(base)
+        r.update({"configuration": f"{row['workload']} batch {row['batch']} B {row['budget']}",
+                  "steps_per_s": row["steps_per_s"], "ms_per_step": row["ms_per_step"],
+                  "hbm_gbs": row["hbm_gbs"], "roofline_frac": row["frac"],
+                  "speedup_vs_dense": row["speedup_vs_dense"]})
+        recs.append(r)
+    with open(path, "a") as f:
+        for r in recs:
+            f.write(json.dumps(r) + "\n")
 
 
 def dist_env():
@@ -618,6 +657,7 @@ def run_reference(args):
         "impl_detail": f"float64 NumPy oracle on {cores} host cores",
     }
     print(json.dumps(line), flush=True)
+    append_records(args.jsonl, line)
 
 
 def run_jssa(args):
@@ -831,6 +871,7 @@ def run_jssa(args):
     group.close()
     if rank == 0:
         print(json.dumps(line), flush=True)
+        append_records(args.jsonl, line)
 
 
 def measure_sweep(args, group, dev, local, rank, world, with_cpu=False):
@@ -908,6 +949,7 @@ def run_workload(args, measure):
     group.close()
     if rank == 0:
         print(json.dumps(line), flush=True)
+        append_records(args.jsonl, line)
 
 
 def measure_hybrid(args, group, dev, local, rank, world, with_cpu=True):

@@ -3,6 +3,7 @@ the gloo backend and two ranks: the barrier, the max over ranks of a time, disti
 workload seeds, the weak-scaling aggregate, and a clean shutdown."""
 
 import multiprocessing as mp
+import json
 import os
 import socket
 import sys
@@ -61,3 +62,28 @@ def test_single_rank_has_no_process_group(monkeypatch):
     assert g.world == 1 and g.max_over_ranks(3.0) == 3.0
     g.barrier()
     g.close()
+
+
+def test_jsonl_records_one_per_configuration(tmp_path):
+    # --jsonl: the headline, each sweep row and each sub-workload become one record each
+    import bench
+    line = {"metric": "m", "value": 6900.0, "ms_per_step": 0.145, "hbm_gbs": 4630.0,
+            "roofline_step": {"frac": 0.71}, "speedup_vs_dense": 9.2,
+            "config": {"workload": "llama3-8b-layer-128k"},
+            "cpu_baseline": {"agreement": {"pairs": 2, "selections_equal": True}},
+            "mla": {"value": 7100.0, "ms_per_step": 0.14, "roofline_step": {"frac": 0.33},
+                    "config": {"workload": "MLA layer"}},
+            "sweep": {"rows": [{"workload": "llama128k", "batch": b, "budget": 2048,
+                                "steps_per_s": 1.0, "ms_per_step": 1.0, "hbm_gbs": 1.0,
+                                "frac": 0.1, "speedup_vs_dense": 2.0} for b in (1, 4)]}}
+    path = tmp_path / "runs.jsonl"
+    bench.append_records(str(path), line)
+    bench.append_records(str(path), line)  # appended, not overwritten
+    recs = [json.loads(x) for x in path.read_text().splitlines()]
+    assert len(recs) == 8
+    names = [r["configuration"] for r in recs[:4]]
+    assert names == ["llama3-8b-layer-128k", "mla", "llama128k batch 1 B 2048",
+                     "llama128k batch 4 B 2048"]
+    assert recs[0]["roofline_frac"] == 0.71 and recs[0]["oracle_agreement"]["selections_equal"]
+    assert recs[2]["steps_per_s"] == 1.0 and recs[2]["impl"] == "jssa"
+    bench.append_records(None, line)  # no path: nothing written
