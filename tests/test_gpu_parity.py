@@ -144,9 +144,11 @@ def test_score_topk_rank16(page_size, lens, budget):
             check_selection(gi[b, h], gc[b, h], ref_idx[b, h], ref_count[b, h], s[(b, h)], budget)
 
 
-@pytest.mark.parametrize("page_size,lens,budget", [(4, [3000, 777], 200), (8, [20000], 512)])
+@pytest.mark.parametrize("page_size,lens,budget", [(4, [3000, 777], 200), (8, [20000], 512),
+                                                     (8, [131072], 2048)])
 def test_score_topk_small_pages(page_size, lens, budget):
-    # pages shorter than a 16-token scan tile (rows of one tile come from several pages)
+    # pages shorter than a 16-token scan tile (rows of one tile come from several pages); the
+    # 128K case takes 4096-position chunks, 256 candidate regions per pair (the flattened tier)
     case = Case(lens, page_size=page_size, seed=1045 + page_size, calib=2048)
     J = jssa()
     idx, count = J.score_topk(case.gpu(case.q), case.gpu_np(case.m32), case.gpu_np(case.codes),
