@@ -9,7 +9,8 @@
   attention output of the pair's four query heads. At this size a pair's scan spans 16 chunks of
   8192 positions, 128 candidate regions: the edge of the select kernel's register tier. The same
   step at batch 1 (8 pairs, all of them sampled) takes 4096-position chunks, 256 candidate
-  regions per pair: the flattened register tier.
+  regions per pair: the flattened register tier. The global layer of the hybrid stack (16 query
+  / 8 KV heads, d 256, r 64, 64K context, batch 8, B 2048) runs through the same checks.
 * MLA: the 128-head latent layer (576-dim latent rows, 64-token pages, scoring in 64 latent +
   64 rotary dimensions, B 2048) at 128K context and batch 16: the store of every scoring row,
   score + top-B, and the absorbed latent attention; two sampled sequences against the oracle,
@@ -56,10 +57,10 @@ def _pair_rows(cache, bt_row, h, L):
     return cache[pages][:, :, h].reshape(-1, cache.shape[-1])[:L].cpu()
 
 
-@pytest.mark.parametrize("batch", [16, 1])
-def test_gqa_decode_step_full_size(batch):
+@pytest.mark.parametrize("name,batch", [("llama128k", 16), ("llama128k", 1), ("hybrid", 8)])
+def test_gqa_decode_step_full_size(name, batch):
     import token_level_sparse_fp8_b200 as J
-    w = WORKLOADS["llama128k"].replace(batch=batch)  # L 131072, B 2048: the bench's workload
+    w = WORKLOADS[name].replace(batch=batch)  # the bench's workloads at their full sizes
     dev = torch.device("cuda")
     L, B, G, d, r, ps = w.seq_len, w.budget, w.group, w.d, w.rank, w.page_size
     f = layer_factors(w.seed, 0, w.h_kv, w.d)
