@@ -5,8 +5,9 @@
   ``jssa_decode`` with a new token. Every (sequence, KV head) pair is checked for the properties
   that hold at any size (count, ascending unique in-range positions, -1 padding, the new token's
   K/V rows written in place); sampled pairs, two per KV head, are checked element by element
-  against the oracle: every scoring code of the pair, the index set (tie tolerance) and the
-  attention output of the pair's four query heads. At this size a pair's scan spans 16 chunks of
+  against the oracle: every scoring code of the pair, the index set (tie tolerance), the
+  attention output of the pair's query heads, and the dense baseline's output over every
+  position. At this size a pair's scan spans 16 chunks of
   8192 positions, 128 candidate regions: the edge of the select kernel's register tier. The same
   step at batch 1 (8 pairs, all of them sampled) takes 4096-position chunks, 256 candidate
   regions per pair: the flattened register tier. The global layer of the hybrid stack (16 query
@@ -89,6 +90,8 @@ def test_gqa_decode_step_full_size(name, batch):
         k_rows[L - 1], v_rows[L - 1] = k_new[b, h], v_new[b, h]
         host[(b, h)] = (k_rows, v_rows)  # bf16 until used
     out, idx, count = layer.step(q, k_new.to(dev), v_new.to(dev))
+    # the dense baseline over the same caches (the new token included), as the bench times it
+    dense = layer.dense(q)
     torch.cuda.synchronize()
     assert J.device_error() == 0
 
@@ -102,6 +105,7 @@ def test_gqa_decode_step_full_size(name, batch):
 
     qn = f64(q)
     out_np = f64(out)
+    dense_np = f64(dense)
     scale = 1.0 / math.sqrt(d)
     for b, h in sampled:
         k_rows, v_rows = (f64(t) for t in host.pop((b, h)))
@@ -116,11 +120,14 @@ def test_gqa_decode_step_full_size(name, batch):
         s = O.scores(codes, O.projected_query(qbar, m32[h].astype(np.float64)))
         ref = O.select_top_b(s, B)
         check_selection(gi[b, h], gc[b, h], ref, ref.shape[0], s, B)
-        # attention of the four query heads over the oracle's own index set
+        # attention of the pair's query heads over the oracle's own index set, and the dense
+        # baseline over every position
         for g in range(G):
             i = h * G + g
             o = O.attend(qn[b, i], k_rows[ref], v_rows[ref], scale)
             check_output(out_np[b, i][None], o[None])
+            o_all = O.attend(qn[b, i], k_rows, v_rows, scale)
+            check_output(dense_np[b, i][None], o_all[None])
 
 
 def test_mla_decode_step_full_size():
