@@ -15,7 +15,8 @@
 * MLA: the 128-head latent layer (576-dim latent rows, 64-token pages, scoring in 64 latent +
   64 rotary dimensions, B 2048) at 128K context and batch 16: the store of every scoring row,
   score + top-B, and the absorbed latent attention; two sampled sequences against the oracle,
-  properties on all.
+  properties on all; and the same latent attention over every position (the layer's dense
+  baseline), eight heads of the two sequences against the oracle.
 
 Inputs come from the seeded generator (built on the GPU, copied to the host for the oracle);
 the basis is the oracle's calibration. Criteria are in ``parity.py``.
@@ -161,6 +162,10 @@ def test_mla_decode_step_full_size():
     idx, count = J.score_topk(q, basis, sc, bt, kv["seq_lens"], B)
     scale = 1.0 / math.sqrt(D)
     out = J.mla_attend(q, latent, bt, idx, count, scale)
+    # the dense baseline of the latent layer: the same kernel over every position
+    idx_full = torch.arange(L, dtype=torch.int32, device=dev).repeat(batch, 1).view(batch, 1, L)
+    count_full = torch.full((batch, 1), L, dtype=torch.int32, device=dev)
+    out_full = J.mla_attend(q, latent, bt, idx_full, count_full, scale)
     torch.cuda.synchronize()
     assert J.device_error() == 0
     gi, gc = idx.cpu().numpy(), count.cpu().numpy()
@@ -179,3 +184,7 @@ def test_mla_decode_step_full_size():
         ref_out = np.stack([O.attend(qn[b, i], rows[ref], rows[ref][:, :512], scale)
                             for i in range(h_q)])
         check_output(out_np[b], ref_out)
+        # dense over all 131072 rows, for eight of the heads (each one a pass over 600 MB)
+        heads = (0, 1, 31, 63, 64, 95, 126, 127)
+        ref_full = np.stack([O.attend(qn[b, i], rows, rows[:, :512], scale) for i in heads])
+        check_output(f64(out_full[b])[list(heads)], ref_full)
