@@ -354,6 +354,34 @@ def test_decode_step(ragged, budget):
     check_output(f64(out), ref["out"])
 
 
+@pytest.mark.parametrize("h_q,h_kv,lens,budget", [(8, 1, [20000, 3000], 512),  # MQA, G = 8
+                                                   (4, 4, [5000, 700], 256)])     # G = 1
+def test_decode_step_group_sizes(h_q, h_kv, lens, budget):
+    # the largest group the attention's m16 tile holds (8 query heads on one KV head) and one query
+    # head per KV head, through the whole decode step with a new token
+    J = jssa()
+    case = Case(lens, h_q=h_q, h_kv=h_kv, seed=1090 + h_q * 10 + h_kv, calib=2048)
+    rng = np.random.default_rng(9)
+    k_new = torch.from_numpy(rng.standard_normal((len(lens), h_kv, case.d))).to(torch.bfloat16)
+    v_new = torch.from_numpy(rng.standard_normal((len(lens), h_kv, case.d))).to(torch.bfloat16)
+    k_cache, v_cache = case.gpu(case.k_cache).clone(), case.gpu(case.v_cache).clone()
+    sc = case.gpu_np(case.codes).clone()
+    scale = 1.0 / math.sqrt(case.d)
+    out, idx, count = J.decode(case.gpu(case.q), k_new.cuda(), v_new.cuda(), k_cache, v_cache, sc,
+                               case.gpu_np(case.m32), case.gpu(case.block_table),
+                               case.gpu(case.seq_lens_t), budget, scale)
+    ref = O.decode_step(case.np_q, f64(k_new), f64(v_new), case.np_k, case.np_v, case.codes,
+                        case.np_bt, np.asarray(lens), case.m32.astype(np.float64), budget, scale)
+    assert np.array_equal(sc.cpu().numpy(), ref["score_cache"])
+    gi, gc = idx.cpu().numpy(), count.cpu().numpy()
+    assert np.array_equal(gc, ref["count"])
+    for b in range(len(lens)):
+        for h in range(h_kv):
+            check_selection(gi[b, h], gc[b, h], ref["idx"][b, h], ref["count"][b, h],
+                            ref["scores"][(b, h)], budget)
+    check_output(f64(out), ref["out"])
+
+
 def test_decode_step_long_contexts():
     # contexts past the all-candidates limit: the new token is stored by the same kernel that
     # draws the threshold sample, and the scan reads its code afterwards
