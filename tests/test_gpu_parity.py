@@ -382,6 +382,34 @@ def test_decode_step_group_sizes(h_q, h_kv, lens, budget):
     check_output(f64(out), ref["out"])
 
 
+@pytest.mark.parametrize("page_size,lens,budget", [(64, [20000, 1000], 512), (128, [17001, 300], 256)])
+def test_decode_step_large_pages(page_size, lens, budget):
+    # pages larger than a scan chunk's 16-token tiles and than an attention tile: several tiles and
+    # several selected rows per page, the new token in the middle of its page
+    J = jssa()
+    case = Case(lens, page_size=page_size, seed=1100 + page_size, calib=2048)
+    rng = np.random.default_rng(11)
+    k_new = torch.from_numpy(rng.standard_normal((len(lens), case.h_kv, case.d))).to(torch.bfloat16)
+    v_new = torch.from_numpy(rng.standard_normal((len(lens), case.h_kv, case.d))).to(torch.bfloat16)
+    k_cache, v_cache = case.gpu(case.k_cache).clone(), case.gpu(case.v_cache).clone()
+    sc = case.gpu_np(case.codes).clone()
+    scale = 1.0 / math.sqrt(case.d)
+    out, idx, count = J.decode(case.gpu(case.q), k_new.cuda(), v_new.cuda(), k_cache, v_cache, sc,
+                               case.gpu_np(case.m32), case.gpu(case.block_table),
+                               case.gpu(case.seq_lens_t), budget, scale)
+    ref = O.decode_step(case.np_q, f64(k_new), f64(v_new), case.np_k, case.np_v, case.codes,
+                        case.np_bt, np.asarray(lens), case.m32.astype(np.float64), budget, scale)
+    assert np.array_equal(f64(k_cache), ref["k_cache"])
+    assert np.array_equal(sc.cpu().numpy(), ref["score_cache"])
+    gi, gc = idx.cpu().numpy(), count.cpu().numpy()
+    assert np.array_equal(gc, ref["count"])
+    for b in range(len(lens)):
+        for h in range(case.h_kv):
+            check_selection(gi[b, h], gc[b, h], ref["idx"][b, h], ref["count"][b, h],
+                            ref["scores"][(b, h)], budget)
+    check_output(f64(out), ref["out"])
+
+
 def test_decode_step_long_contexts():
     # contexts past the all-candidates limit: the new token is stored by the same kernel that
     # draws the threshold sample, and the scan reads its code afterwards
