@@ -236,7 +236,9 @@ def test_mla_decode_step(budget):
         check_selection(gi[b, 0], gc[b, 0], ref_idx[b, 0], ref_count[b, 0], s[(b, 0)], budget)
     ref = O.indexed_attend_step(f64(c.q), np_kv, np_kv[..., :512], c.np_bt, ref_idx, ref_count, scale)
     check_output(f64(out), ref)
-    # a second step reuses the workspace: the selection clears the attention's split counters
-    out2, _, _ = J.mla_decode(c.q.cuda(), None, kv, sc, torch.from_numpy(c.m_lat).cuda(),
-                              c.bt.cuda(), c.lens_t.cuda(), budget, scale)
+    # a second step reuses the workspace: the selection clears the attention's split counters;
+    # on the same caches (the new row already stored) it is bit-identical to the first
+    out2, idx2, _ = J.mla_decode(c.q.cuda(), None, kv, sc, torch.from_numpy(c.m_lat).cuda(),
+                                 c.bt.cuda(), c.lens_t.cuda(), budget, scale)
     check_output(f64(out2), ref)
+    assert torch.equal(idx2, idx) and torch.equal(out2, out)

@@ -410,6 +410,26 @@ def test_decode_step_large_pages(page_size, lens, budget):
     check_output(f64(out), ref["out"])
 
 
+def test_decode_step_is_deterministic(ragged):
+    # the same step on the same inputs gives bit-identical outputs, index sets and caches (the
+    # split-K merge combines the splits in a fixed order whichever CTA finishes last)
+    J = jssa()
+    case = ragged
+    rng = np.random.default_rng(13)
+    k_new = torch.from_numpy(rng.standard_normal((len(case.seq_lens), case.h_kv, case.d))).to(torch.bfloat16).cuda()
+    v_new = torch.from_numpy(rng.standard_normal((len(case.seq_lens), case.h_kv, case.d))).to(torch.bfloat16).cuda()
+    results = []
+    for _ in range(2):
+        k_cache, v_cache = case.gpu(case.k_cache).clone(), case.gpu(case.v_cache).clone()
+        sc = case.gpu_np(case.codes).clone()
+        out, idx, count = J.decode(case.gpu(case.q), k_new, v_new, k_cache, v_cache, sc,
+                                   case.gpu_np(case.m32), case.gpu(case.block_table),
+                                   case.gpu(case.seq_lens_t), 700, 1.0 / math.sqrt(case.d))
+        results.append((out.cpu(), idx.cpu(), count.cpu(), sc.cpu(), k_cache.cpu()))
+    for a, b in zip(*results):
+        assert torch.equal(a, b)
+
+
 def test_decode_step_long_contexts():
     # contexts past the all-candidates limit: the new token is stored by the same kernel that
     # draws the threshold sample, and the scan reads its code afterwards
