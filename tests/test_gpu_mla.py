@@ -35,9 +35,9 @@ def jssa():
 
 
 class MlaCase:
-    def __init__(self, seq_lens, seed=1500):
+    def __init__(self, seq_lens, seed=1500, h_q=H_Q):
         f = layer_factors(seed, 0, 1, D)
-        qc, kc = sample_calibration(f, 2048, H_Q, seed)
+        qc, kc = sample_calibration(f, 2048, h_q, seed)
         cal = O.calibrate(f64(qc)[..., :512], f64(kc)[..., :512], R_LAT)
         self.m_lat = cal["M"].astype(np.float32)                                  # [1, 64, 512]
         # the oracle's block basis of the same float32 values
@@ -47,7 +47,7 @@ class MlaCase:
         self.bt = kv["block_table"]
         self.lens_t = kv["seq_lens"]
         self.lens = np.asarray(seq_lens)
-        self.q = sample_decode_queries(f, len(seq_lens), H_Q, seed)  # [batch, 32, 576]
+        self.q = sample_decode_queries(f, len(seq_lens), h_q, seed)  # [batch, h_q, 576]
         self.np_kv = f64(self.kv)
         self.np_bt = self.bt.numpy()
         num_pages = self.np_kv.shape[0]
@@ -199,8 +199,20 @@ def test_mla_decode_step(budget):
     # one whole latent decode step through jssa_mla_decode: the new latent row and its scoring code
     # are stored by the first kernel, then score + top-B and the latent attention (contexts past
     # the sampling point, ragged, below the budget, empty)
+    check_decode_step(MlaCase([20000, 3001, 300, 0], seed=1530), budget)
+
+
+@pytest.mark.parametrize("batch", [20, 40, 80])
+def test_mla_decode_step_larger_batches(batch):
+    # larger latent batches (up to more sequences than SMs for the prep and the select): 128 query
+    # heads, one context past the sampling point, the rest ragged, below the budget and empty
+    rng = np.random.default_rng(batch)
+    lens = [17000, 0, 700] + [int(x) for x in rng.integers(1100, 2600, batch - 3)]
+    check_decode_step(MlaCase(lens, seed=1540 + batch, h_q=128), 1024)
+
+
+def check_decode_step(c, budget):
     J = jssa()
-    c = MlaCase([20000, 3001, 300, 0], seed=1530)
     lens = c.lens
     rng = np.random.default_rng(11)
     kv_new = torch.from_numpy(rng.standard_normal((len(lens), D))).to(torch.bfloat16)
