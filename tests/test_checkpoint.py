@@ -4,7 +4,9 @@ The file layout follows the pages' basis file (JSSA README, section 2: ``{'M': {
 Tensor[H_kv, r, d]}}``, a latent layer ``[1, r, kv_lora_rank]``; ``--save_grams`` adds the second
 moments). The CPU tests round-trip a file; the GPU test shows that a calibration stopped after
 half of its samples, saved, loaded and resumed gives the same second moments and basis as one
-that ran in one go.
+that ran in one go. A data-parallel calibration sums its ranks' moments with
+``Calibration.all_reduce``: two gloo ranks on CPU, each with its own samples, end with identical
+moments equal to the oracle's over all samples, and the same basis.
 """
 
 import numpy as np
@@ -84,3 +86,60 @@ def test_resumed_calibration_matches_one_shot(tmp_path):
         p0 = O.projector(one["M"][h].double().cpu().numpy())
         assert np.max(np.abs(p1 - p0)) <= 1e-6
     assert np.max(np.abs(e2.cpu().numpy() - one["eigvals"].cpu().numpy())) <= 1e-10
+
+
+def _reduce_rank(rank, world, port, out):
+    # one rank of a data-parallel calibration: the moments of this rank's own samples, summed
+    # over the ranks by Calibration.all_reduce on a gloo group
+    import os
+    import sys
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    sys.path.insert(0, os.path.join(root, "tests"))
+    import torch.distributed as dist
+    import token_level_sparse_fp8_b200 as J
+    from oracle import jssa as O
+    from synth import layer_factors, sample_calibration
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    f = layer_factors(1700, 0, 2, 64)
+    q, k = sample_calibration(f, 300, 4, 1700 + rank)  # this rank's samples
+    g_q, g_k = O.second_moments(O.group_mean_query(q.double().numpy(), 2), k.double().numpy())
+    cal = J.Calibration(2, 64, "cpu", torch.from_numpy(g_q), torch.from_numpy(g_k), samples=300)
+    cal.all_reduce()
+    dist.destroy_process_group()
+    out.put((rank, cal.gram_q.numpy(), cal.gram_k.numpy(), cal.samples))
+
+
+def test_calibration_all_reduce_two_gloo_ranks():
+    import multiprocessing as mp
+    import socket
+    from oracle import jssa as O
+    from synth import layer_factors, sample_calibration
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    procs = [ctx.Process(target=_reduce_rank, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted((out.get(timeout=120) for _ in procs), key=lambda x: x[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (_, q0, k0, n0), (_, q1, k1, n1) = res
+    # every rank holds the same moments: those of both ranks' samples together
+    assert np.array_equal(q0, q1) and np.array_equal(k0, k1) and n0 == n1 == 600
+    f = layer_factors(1700, 0, 2, 64)
+    qs, ks = zip(*(sample_calibration(f, 300, 4, 1700 + r) for r in range(2)))
+    q, k = torch.cat(qs).double().numpy(), torch.cat(ks).double().numpy()
+    g_q, g_k = O.second_moments(O.group_mean_query(q, 2), k)
+    np.testing.assert_allclose(q0, g_q, rtol=1e-12, atol=1e-9)
+    np.testing.assert_allclose(k0, g_k, rtol=1e-12, atol=1e-9)
+    # and the basis solved from the reduced moments is the one-shot calibration's
+    m_red, _ = O.joint_basis(q0, k0, 16)
+    m_one, _ = O.joint_basis(g_q, g_k, 16)
+    p_red = np.einsum("hri,hrj->hij", m_red, m_red)
+    p_one = np.einsum("hri,hrj->hij", m_one, m_one)
+    np.testing.assert_allclose(p_red, p_one, atol=1e-9)

@@ -192,6 +192,25 @@ class Calibration:
     def basis(self, rank: int, with_eigvals: bool = True):
         return compute_basis(self.gram_q, self.gram_k, rank, with_eigvals)
 
+    def all_reduce(self, group=None) -> None:
+        """Sum the moments and the sample counts over the ranks of ``group`` (the default process
+        group when None): one all-reduce of ``2 h_kv d^2 + 1`` float64 values (NCCL over NVLink
+        between GPUs). The moments are sums over samples, so ranks that each calibrate on their
+        own sequences then all hold the moments of every rank's samples, bit-identical, and
+        ``basis`` solves for the same M on every rank (JSSA README, section 2: the latent
+        calibration runs across the GPUs of a tensor-parallel group; JSSA summary, section 3.2:
+        calibration is second-moment accumulation)."""
+        import torch.distributed as dist
+        n = self.gram_q.numel()
+        flat = torch.empty(2 * n + 1, dtype=torch.float64, device=self.gram_q.device)
+        flat[:n] = self.gram_q.reshape(-1)
+        flat[n:2 * n] = self.gram_k.reshape(-1)
+        flat[2 * n] = float(self.samples)
+        dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)
+        self.gram_q.copy_(flat[:n].view_as(self.gram_q))
+        self.gram_k.copy_(flat[n:2 * n].view_as(self.gram_k))
+        self.samples = int(round(float(flat[2 * n].item())))
+
     def state(self) -> dict:
         """Host copies of the moments and the sample count."""
         return {"gram_q": self.gram_q.cpu(), "gram_k": self.gram_k.cpu(), "samples": self.samples}
