@@ -6,7 +6,8 @@ moments). The CPU tests round-trip a file; the GPU test shows that a calibration
 half of its samples, saved, loaded and resumed gives the same second moments and basis as one
 that ran in one go. A data-parallel calibration sums its ranks' moments with
 ``Calibration.all_reduce``: two gloo ranks on CPU, each with its own samples, end with identical
-moments equal to the oracle's over all samples, and the same basis.
+moments equal to the oracle's over all samples, and the same basis; on the GPU the same call
+runs through an NCCL group of one rank.
 """
 
 import numpy as np
@@ -143,3 +144,40 @@ def test_calibration_all_reduce_two_gloo_ranks():
     p_red = np.einsum("hri,hrj->hij", m_red, m_red)
     p_one = np.einsum("hri,hrj->hij", m_one, m_one)
     np.testing.assert_allclose(p_red, p_one, atol=1e-9)
+
+
+def _nccl_single_rank(port, out):
+    # Calibration.all_reduce on the GPU's own moments through an NCCL group of one rank
+    import os
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import torch.distributed as dist
+    import token_level_sparse_fp8_b200 as J
+    torch.cuda.set_device(0)
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1)
+    g = torch.Generator(device="cuda").manual_seed(5)
+    gq = torch.randn(8, 128, 128, generator=g, dtype=torch.float64, device="cuda")
+    gk = torch.randn(8, 128, 128, generator=g, dtype=torch.float64, device="cuda")
+    cal = J.Calibration(8, 128, "cuda", gq.clone(), gk.clone(), samples=1234)
+    cal.all_reduce()
+    ok = (torch.equal(cal.gram_q, gq) and torch.equal(cal.gram_k, gk) and cal.samples == 1234
+          and cal.gram_q.is_cuda)
+    dist.destroy_process_group()
+    out.put(ok)
+
+
+@pytest.mark.gpu
+def test_calibration_all_reduce_nccl_single_rank():
+    import multiprocessing as mp
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    p = ctx.Process(target=_nccl_single_rank, args=(port, out))
+    p.start()
+    ok = out.get(timeout=300)
+    p.join(timeout=60)
+    assert p.exitcode == 0 and ok
