@@ -1,6 +1,7 @@
 """The multi-rank plumbing of bench.py (one process per GPU under torchrun), exercised on CPU with
 the gloo backend and two ranks: the barrier, the max over ranks of a time, distinct per-rank
-workload seeds, the weak-scaling aggregate, and a clean shutdown."""
+workload seeds, the weak-scaling aggregate, and a clean shutdown. Also the JSON-lines record and
+the line of the reference arm (the float64 oracle on host cores), which runs without a GPU."""
 
 import multiprocessing as mp
 import json
@@ -87,3 +88,33 @@ def test_jsonl_records_one_per_configuration(tmp_path):
     assert recs[0]["roofline_frac"] == 0.71 and recs[0]["oracle_agreement"]["selections_equal"]
     assert recs[2]["steps_per_s"] == 1.0 and recs[2]["impl"] == "jssa"
     bench.append_records(None, line)  # no path: nothing written
+
+
+def test_reference_arm_line():
+    # `bench.py --impl reference` (the float64 oracle on host cores) prints one JSON line with the
+    # GPU arm's metric, unit and config, exactly the requested steps, and its own CPU baseline and
+    # end-to-end keys (no host-device copies)
+    import subprocess
+    sys.path.insert(0, ROOT)
+    import bench
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--steps", "2", "--warmup", "1"],
+                         cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [l for l in res.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "steps/s"
+    assert d["steps"] == 2 and d["warmup"] == 1 and d["n_gpus"] == 1 and d["higher_is_better"]
+
+    class Args:
+        batch, budget, seq_len = 16, 2048, 131072
+
+    assert d["config"] == bench.config_of(bench.workload(Args, 0), 1)
+    assert d["value"] > 0 and abs(d["ms_per_step"] - d["measured_ms_per_pair"]["median"]) < 1e-9
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    e2e = d["e2e"]
+    assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
