@@ -39,4 +39,5 @@ def bf16_encode(y) -> np.ndarray:
 def bf16_decode(bits) -> np.ndarray:
     """Value (float64) of each bf16 bit pattern."""
     b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
-    return b.view(np.float32).astype(np.float64)
+    with np.errstate(invalid="ignore"):  # NaN patterns widen to NaN (numpy flags the cast)
+        return b.view(np.float32).astype(np.float64)
